@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark: KDA prefill tokens/s (B=1, H=32, T=65536, d=128, bf16, split
+fast/slow decay, nonzero fp32 state) and decode GB/s (256 sequences x 32
+heads, d=128, fp32 state), each as a fraction of its roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one full prefill pass over the T=65536 workload (all prefill
+kernels).  The decode step is timed in the same run on its own workload and
+reported under "decode".  For N > 1 (launched with torchrun) every rank runs
+an independent replica on its own GPU (the path has no exchange step), the
+elapsed time is the max over ranks, and `value` counts the tokens of all
+ranks.  Inputs are seeded synthetic data generated on the device.
+
+`--impl reference` times the fp64 CPU oracle on the host cores (rank 0 only)
+on a bounded sample of the same workload, with the same metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "KDA prefill tokens/s (H32,d128,T64k) + decode GB/s; % of roofline"
+PREFILL_WORKLOAD = "prefill_h32_t65536_d128_split"
+DECODE_WORKLOAD = "decode_n256_h32_d128"
+L2_BYTES = 126 * 2**20
+
+# algorithmic bytes (the minimum the path must move), per (token, head)
+PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 + 128 * 2      # q,k,v,g,beta in; o out (bf16)
+STATE_BYTES = 128 * 128 * 4                                   # one fp32 state, one direction
+DECODE_BYTES_PER_UNIT = 2 * STATE_BYTES + 4 * 128 * 2 + 2 + 128 * 2
+SLOT_BYTES = 66560                                            # per (chunk, head) workspace slot
+FLOPS_PER_TOKEN_HEAD = 139264                                 # algorithmic MMA flops (causal halves once)
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() in ("active", "1", "0x1"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- ours
+
+def time_prefill(binding, d, o, s_out, ws, steps, warmup, profile=False):
+    st = torch.cuda.current_stream()
+    call = lambda: binding.kda_chunk_prefill(d.q, d.k, d.v, d.g, d.beta, d.state_in, None,
+                                             o=o, state_out=s_out, workspace=ws)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    if profile:
+        binding.kda_profile_enable(True)
+        per = []
+        for _ in range(steps):
+            call()
+            per.append(binding.kda_profile_last())
+        binding.kda_profile_enable(False)
+        return per
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for _ in range(steps):
+        call()
+    ev1.record(st)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1)
+
+
+def run_ours(args, rank, world, dev):
+    from kda_delta_rule_chunkwise_b200 import binding
+    from kda_delta_rule_chunkwise_b200 import build as kbuild
+    from kda_delta_rule_chunkwise_b200 import inputs as kin
+
+    if rank == 0:
+        kbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+    binding.load()
+    peaks = measured_peaks()
+
+    # ---------------- prefill workload (inputs resident in HBM)
+    w = kin.WORKLOADS[PREFILL_WORKLOAD]
+    d = kin.workload_inputs(PREFILL_WORKLOAD, seed=args.seed + rank, device=dev)
+    B, T, H = d.B, d.T, d.H
+    tokens = B * T
+    o = torch.empty_like(d.v)
+    s_out = torch.empty((d.N, H, 128, 128), dtype=torch.float32, device=dev)
+    ws = torch.empty(binding.kda_chunk_prefill_workspace_bytes(tokens, d.N, H, 128, 128,
+                                                                torch.bfloat16),
+                     dtype=torch.uint8, device=dev)
+    in_bytes = sum(x.numel() * x.element_size() for x in (d.q, d.k, d.v, d.g, d.beta, d.state_in))
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        ms = time_prefill(binding, d, o, s_out, ws, args.steps, args.warmup)
+    torch.cuda.synchronize()
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    value = tokens * world * args.steps / (ms_max / 1e3)
+
+    # per-kernel device time (separate profiled pass, same inputs)
+    per = time_prefill(binding, d, o, s_out, ws, max(2, args.steps), 1, profile=True)
+    n_k = len(per[0])
+    k_avg = [sum(p[i] for p in per) / len(per) for i in range(n_k)]
+    names = ["chunk_table_kernel", "intra_chunk_kernel", "state_pass_kernel"][:n_k]
+    head_chunks = H * B * ((T + 63) // 64)
+    k_bytes = {
+        "chunk_table_kernel": 8 * (d.N + 1),
+        "intra_chunk_kernel": head_chunks * (64 * (3 * 128 * 2 + 2) + SLOT_BYTES),
+        "state_pass_kernel": head_chunks * (SLOT_BYTES + 2 * 64 * 128 * 2)
+        + d.N * H * 2 * STATE_BYTES,
+    }
+    dom = max(range(n_k), key=lambda i: k_avg[i])
+    dom_name = names[dom]
+    achieved = k_bytes[dom_name] / (k_avg[dom] / 1e3) / 1e9
+    roofline = {
+        "kernel": dom_name, "bound": "hbm", "achieved": round(achieved, 1),
+        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+        "traffic": None, "peak_source": peaks["source"],
+        "kernel_ms": {n: round(x, 4) for n, x in zip(names, k_avg)},
+        "kernel_share": {n: round(x / sum(k_avg), 4) for n, x in zip(names, k_avg)},
+    }
+    path_bytes = tokens * H * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * d.N * H * STATE_BYTES
+    path_gbs = path_bytes / (ms_step / 1e3) / 1e9
+    path_tflops = tokens * H * FLOPS_PER_TOKEN_HEAD / (ms_step / 1e3) / 1e12
+    roofline_path = {
+        "bound": "hbm", "algorithmic_bytes": path_bytes, "achieved": round(path_gbs, 1),
+        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(path_gbs / peaks["hbm_gbs"], 4),
+        "tensor_tflops": round(path_tflops, 1),
+        "tensor_frac": round(path_tflops / peaks["bf16_tflops_sustained"], 4),
+    }
+
+    # ---------------- end to end through the public API, host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = lambda x: x.cpu().pin_memory()
+        hq, hk, hv, hg, hb, hs = (pin(x) for x in (d.q, d.k, d.v, d.g, d.beta, d.state_in))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hso = torch.empty(s_out.shape, dtype=s_out.dtype, pin_memory=True)
+        dq, dk_, dv_, dg, db, ds = (torch.empty_like(x) for x in (d.q, d.k, d.v, d.g, d.beta,
+                                                                  d.state_in))
+
+        def e2e_step():
+            for dst, src in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (ds, hs)):
+                dst.copy_(src, non_blocking=True)
+            binding.kda_chunk_prefill(dq, dk_, dv_, dg, db, ds, None, o=o, state_out=s_out,
+                                      workspace=ws)
+            ho.copy_(o, non_blocking=True)
+            hso.copy_(s_out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        st = torch.cuda.current_stream()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(st)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        ev1.record(st)
+        torch.cuda.synchronize()
+        e_ms = ev0.elapsed_time(ev1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": tokens * world * args.e2e_steps / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": in_bytes,
+               "d2h_bytes_per_step": o.numel() * o.element_size()
+               + s_out.numel() * s_out.element_size(),
+               "steps": args.e2e_steps}
+        del hq, hk, hv, hg, hb, hs, ho, hso, dq, dk_, dv_, dg, db, ds
+
+    del d, o, s_out, ws
+    torch.cuda.empty_cache()
+
+    # ---------------- decode workload
+    dw = kin.WORKLOADS[DECODE_WORKLOAD]
+    Nd, Hd = dw["N"], dw["H"]
+    dec = kin.decode_inputs(args.decode_steps, Nd, Hd, 128, 128, "bf16",
+                            seed=args.seed + 1000 + rank, device=dev)
+    pristine = dec.state.clone()
+    S = dec.state
+    od = torch.empty((Nd, Hd, 128), dtype=torch.bfloat16, device=dev)
+
+    def dec_step(t):
+        binding.kda_decode_step(dec.q[t], dec.k[t], dec.v[t], dec.g[t], dec.beta[t], S, o=od)
+
+    for t in range(min(args.warmup, args.decode_steps)):
+        dec_step(t)
+    S.copy_(pristine)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    st = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for t in range(args.decode_steps):
+        dec_step(t)
+    ev1.record(st)
+    torch.cuda.synchronize()
+    d_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t_ = torch.tensor([d_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+        d_ms = float(t_.item())
+    d_bytes = Nd * Hd * DECODE_BYTES_PER_UNIT
+    d_gbs = d_bytes * args.decode_steps / (d_ms / 1e3) / 1e9
+    decode = {
+        "workload": DECODE_WORKLOAD, "steps": args.decode_steps,
+        "steps_per_s": round(world * args.decode_steps / (d_ms / 1e3), 1),
+        "gbs": round(world * d_gbs, 1), "gbs_per_gpu": round(d_gbs, 1),
+        "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(d_gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(d_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "bytes_per_launch": d_bytes},
+        "state_bytes": S.numel() * 4,
+    }
+    del dec, pristine, S, od
+    torch.cuda.empty_cache()
+
+    launches = args.steps * 3 + args.decode_steps
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": PREFILL_WORKLOAD, "B": B, "T": T, "H": H, "dk": 128, "dv": 128,
+                   "decay": w["decay"], "state": w["state"], "global_batch": B * world,
+                   "seq_len": T, "parallelism": f"replicas{world}",
+                   "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
+        "roofline": roofline, "roofline_path": roofline_path, "decode": decode,
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
+    }
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle
+
+def oracle_sample(seed, n_tokens, heads, threads):
+    """Time the fp64 oracle on the first n_tokens of the prefill workload, given heads."""
+    import numpy as np
+    import oracle
+    from kda_delta_rule_chunkwise_b200 import inputs as kin
+    w = kin.WORKLOADS[PREFILL_WORKLOAD]
+    inp = kin.prefill_inputs(1, n_tokens, w["H"], w["dk"], w["dv"], w["dtype"], seed,
+                             w["decay"], w["state"], device="cpu")
+    hs = list(range(heads))
+    pick = lambda x: x[:, :, hs].contiguous()
+    args = [pick(x) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta)]
+    s_in = inp.state_in[:, hs].contiguous()
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.recurrence(*args, state_in=s_in, n_threads=threads)
+    dt = time.perf_counter() - t0
+    # tokens/s with all H heads = head-tokens processed / H / seconds
+    return n_tokens * heads / w["H"] / dt, dt
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def sized_oracle_sample(seed, target_s, threads, cap_tokens=65536):
+    """Calibrate on a short sample, then time one sample sized to ~target_s seconds."""
+    heads = min(32, max(1, threads))
+    v0, dt0 = oracle_sample(seed, 256, heads, threads)
+    n = int(256 * target_s / max(dt0, 1e-3))
+    n = max(256, min(cap_tokens, n))
+    v, dt = oracle_sample(seed, n, heads, threads)
+    sample = f"first {n} tokens x {heads} of 32 heads of {PREFILL_WORKLOAD}, fp64, {dt:.1f} s"
+    return v, dt, sample
+
+
+def run_reference(args):
+    threads = cpu_threads()
+    vals = []
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        target = 2.0 if i < args.warmup else args.ref_seconds
+        v, dt, smp = sized_oracle_sample(args.seed, target, threads)
+        if i >= args.warmup:
+            vals.append((v, dt))
+            sample = smp
+    value = statistics.median(v for v, _ in vals)
+    ms = statistics.median(dt for _, dt in vals) * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": PREFILL_WORKLOAD, "B": 1, "T": 65536, "H": 32, "dk": 128,
+                   "dv": 128, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--ref-seconds", type=float, default=15.0,
+                    help="target CPU seconds of one oracle sample (reference arm, cpu_baseline)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warmup raised to 3 (minimum)")
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}), flush=True)
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        res = run_ours(args, rank, world, dev)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            threads = cpu_threads()
+            v, dt, smp = sized_oracle_sample(args.seed, args.ref_seconds, threads)
+            res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": threads,
+                                   "kind": "oracle", "sample": smp}
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

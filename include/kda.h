@@ -1,0 +1,170 @@
+/*
+ * libkda: Kimi Delta Attention (KDA) prefill and decode on NVIDIA B200 (sm_100a).
+ *
+ * The operation (per sequence n and head h, tokens t in order):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t,          log-decay g bounded below at -5
+ *
+ * i.e. linear attention with a fixed-size per-head state S (dk x dv) updated
+ * by the delta rule with per-channel retention.  The pages that describe it:
+ *   - neurohive.io, "Kimi K3 ... overview", section "Sequence length: hybrid
+ *     KDA and Gated MLA attention": delta rule (forget old content, write new
+ *     content), fixed-size recurrent state, log-decay bounded from below at
+ *     -5 so that every tile can run as a dense tensor-core product.
+ *   - best.xiaohu.ai, "Kimi K3 tech report", section "Sequence length:
+ *     replacing most attention layers with fixed-size memory": the state
+ *     decays gradually across channels; memory stays constant in length.
+ *   - neurohive.io, same article, section "Training and inference
+ *     infrastructure": the KDA recurrent state is fixed in size with a single
+ *     copy per request (the decode step updates it in place).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller, dense and
+ *    row-major in the shapes given; the library never frees or keeps them.
+ *  - q, k, g share the shape [rows, H, dk]; v and o are [rows, H, dv];
+ *    beta is [rows, H].  Element type is `dtype` for q, k, v, g, beta and o.
+ *  - The state is always fp32 [N, H, dk, dv]: row c = key channel, column j
+ *    = value channel, so o_t[j] = sum_c S_t[c][j] q_t[c].
+ *  - g is the per-step log-decay; the contract is g in [-5, 0].  Values
+ *    below -5 are treated as -5 (max(g, -5)); values above 0 are used as
+ *    given.  q and k are expected L2-normalised by the caller; the library
+ *    does not normalise and applies no 1/sqrt(dk) scale.
+ *  - Supported sizes: dk == dv, both 64 or 128.  Anything else returns
+ *    KDA_ERR_UNSUPPORTED with nothing launched.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Argument errors are returned synchronously, before
+ *    anything is launched.  Launch failures return KDA_ERR_CUDA.
+ *  - Device-side waits are bounded: a kernel that gives up waiting records
+ *    it in a per-library error word and exits; kda_check_device_error()
+ *    reports it as KDA_ERR_TIMEOUT.  Kernels never trap.
+ *  - Thread safety: calls on different streams may run concurrently, except
+ *    that the error word is shared by every call in the process.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, bad cu_seqlens shape, short workspace */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. dk != dv, d not 64/128) */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 4        /* a device-side bounded wait gave up (see kda_check_device_error) */
+} kda_status;
+
+typedef enum {
+    KDA_F32 = 0,   /* fp32 q, k, v, g, beta, o; fp32 arithmetic throughout (reference precision) */
+    KDA_BF16 = 1   /* bf16 q, k, v, g, beta, o; tensor-core products with fp32 accumulation, fp32 state */
+} kda_dtype;
+
+/*
+ * Bytes of device workspace kda_chunk_prefill needs for a call with
+ * `rows` = B*T packed tokens, N sequences and H heads.  The value is an
+ * upper bound valid for every cu_seqlens with that many rows and sequences.
+ * Returns 0 when the call needs no workspace (the fp32 path).
+ */
+KDA_API size_t kda_chunk_prefill_workspace_bytes(int64_t rows, int N, int H, int dk, int dv,
+                                         kda_dtype dtype);
+
+/*
+ * Chunked prefill: runs the recurrence above over whole sequences.
+ *
+ * Chunked form (chunk C = 64 tokens; exact arithmetic does not depend on C):
+ * chunk-local log-space cumulative decay G, decay-rescaled intra-chunk
+ * products Akk/Aqk, the unit-lower-triangular (UT/WY) solve that turns the
+ * sequential delta rule into matrix products, then the inter-chunk pass of
+ * the fp32 state with the outputs.
+ *
+ *  q, k, g     [B, T, H, dk]  (B == 1 when cu_seqlens is given)
+ *  v           [B, T, H, dv]
+ *  beta        [B, T, H]
+ *  state_in    [N, H, dk, dv] fp32, or NULL for a zero initial state
+ *  cu_seqlens  device int32 [N+1], offsets of the N packed sequences into the
+ *              T rows (cu_seqlens[0] == 0, non-decreasing, cu_seqlens[N] <= T),
+ *              or NULL: then N must equal B and sequence b owns batch row b.
+ *              Values are read on the device.  Offsets that break these rules
+ *              never make the library read or write outside the buffers
+ *              (offsets are clamped to [0, T] and raised to the previous
+ *              offset), but the results for such sequences are unspecified.
+ *  o           [B, T, H, dv], written for every token that belongs to a sequence
+ *  state_out   [N, H, dk, dv] fp32, final state per sequence, or NULL (not
+ *              written).  May alias state_in exactly (in-place update).
+ *              A zero-length sequence gets state_out = state_in (or zeros).
+ *  workspace   device scratch of at least kda_chunk_prefill_workspace_bytes()
+ *              bytes, 256-byte aligned, or NULL when that size is 0.  Its
+ *              contents on return are the per-chunk intermediates of the
+ *              bf16 path (laid out for the state pass); callers may ignore them.
+ */
+KDA_API kda_status kda_chunk_prefill(const void *q, const void *k, const void *v,
+                             const void *g, const void *beta,
+                             const float *state_in, const int32_t *cu_seqlens,
+                             int B, int64_t T, int N, int H, int dk, int dv,
+                             kda_dtype dtype, void *o, float *state_out,
+                             void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/*
+ * Single-token decode step, state updated in place (one read and one write
+ * of each (n, h) state):
+ *     S' = Diag(exp g) S;  delta = beta (v - S'^T k);  S = S' + k delta^T;
+ *     o = S^T q
+ *  q, k, g [N, H, dk];  v [N, H, dv];  beta [N, H];  o [N, H, dv]
+ *  state   [N, H, dk, dv] fp32, read and overwritten.
+ */
+KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *state,
+                           int N, int H, int dk, int dv, kda_dtype dtype,
+                           void *o, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word.
+ * Returns KDA_ERR_TIMEOUT if any kernel since the last call gave up a bounded
+ * wait, KDA_ERR_CUDA if the stream reported an error, KDA_OK otherwise.
+ */
+KDA_API kda_status kda_check_device_error(void *stream);
+
+/*
+ * Diagnostic: launches one tiny kernel that waits on an mbarrier no one will
+ * ever complete, with the same bounded wait the production kernels use,
+ * giving up after `timeout_us` microseconds.  It records the timeout in the
+ * error word exactly as a production kernel would, so a following
+ * kda_check_device_error() returns KDA_ERR_TIMEOUT and the context stays
+ * usable.  timeout_us must be in [1, 10^7]; otherwise KDA_ERR_INVALID_ARG.
+ */
+KDA_API kda_status kda_selftest_bounded_wait(int64_t timeout_us, void *stream);
+
+/*
+ * Kernel timing.  kda_profile_enable(1) makes every following prefill/decode
+ * call on this device record CUDA events on its stream around each kernel it
+ * launches; kda_profile_enable(0) stops it (and is the default).  Each call
+ * replaces the previous record.  kda_profile_last() waits for the last
+ * recorded event and writes the device time of each kernel of the most
+ * recent call, in launch order, to ms[0 .. *count-1] (at most `capacity`).
+ * Prefill (bf16) launches three kernels: chunk table, intra-chunk products,
+ * state pass; prefill (fp32) and decode launch one.
+ */
+KDA_API kda_status kda_profile_enable(int enable);
+KDA_API kda_status kda_profile_last(float *ms, int capacity, int *count);
+
+/* Static, human-readable name of a status code. */
+KDA_API const char *kda_status_string(kda_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,194 @@
+"""ctypes binding of libkda (include/kda.h), same names as the C ABI.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels inside libkda.so.  Tensors are torch CUDA tensors (device memory and
+streams come from PyTorch); their data pointers are passed straight through.
+If libkda.so is missing or cannot be loaded, every call raises: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_F32, KDA_BF16 = 0, 1
+_DTYPE = {torch.float32: KDA_F32, torch.bfloat16: KDA_BF16}
+
+# Every symbol the public header declares.
+EXPORTED = (
+    "kda_chunk_prefill_workspace_bytes",
+    "kda_chunk_prefill",
+    "kda_decode_step",
+    "kda_check_device_error",
+    "kda_selftest_bounded_wait",
+    "kda_profile_enable",
+    "kda_profile_last",
+    "kda_status_string",
+)
+
+
+class KDAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libkda.so (raises if it is missing: build it first)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libkda.so not found at {path}; build it with "
+            "`python -m kda_delta_rule_chunkwise_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.kda_chunk_prefill_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i32]
+    lib.kda_chunk_prefill_workspace_bytes.restype = sz
+    lib.kda_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                      i32, vp, vp, vp, sz, vp]
+    lib.kda_chunk_prefill.restype = i32
+    lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+    lib.kda_decode_step.restype = i32
+    lib.kda_check_device_error.argtypes = [vp]
+    lib.kda_check_device_error.restype = i32
+    lib.kda_selftest_bounded_wait.argtypes = [i64, vp]
+    lib.kda_selftest_bounded_wait.restype = i32
+    lib.kda_profile_enable.argtypes = [i32]
+    lib.kda_profile_enable.restype = i32
+    lib.kda_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32)]
+    lib.kda_profile_last.restype = i32
+    lib.kda_status_string.argtypes = [i32]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().kda_status_string(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != KDA_OK:
+        raise KDAError(code, where)
+
+
+def kda_chunk_prefill_workspace_bytes(rows: int, N: int, H: int, dk: int, dv: int,
+                                      dtype: torch.dtype) -> int:
+    return int(load().kda_chunk_prefill_workspace_bytes(rows, N, H, dk, dv, _DTYPE[dtype]))
+
+
+def _contig(name, t):
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def kda_chunk_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=None,
+                      state_out=None, workspace=None, want_state=True, stream=None):
+    """Chunked prefill.  Shapes follow include/kda.h; returns (o, state_out).
+
+    q, k, g: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H] (all one dtype,
+    bf16 or fp32); state_in: [N, H, dk, dv] fp32 or None; cu_seqlens: int32
+    [N+1] on the device or None.  Output buffers are allocated if not given.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta),
+                    ("state_in", state_in), ("cu_seqlens", cu_seqlens)):
+        _contig(name, t)
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if state_out is None and want_state:
+        state_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = kda_chunk_prefill_workspace_bytes(B * T, N, H, dk, dv, q.dtype)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = load().kda_chunk_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens),
+        B, T, N, H, dk, dv, _DTYPE[q.dtype], _ptr(o), _ptr(state_out),
+        _ptr(workspace) if need else None, ws_bytes if need else 0, _stream(stream))
+    _check(code, "kda_chunk_prefill")
+    return o, state_out
+
+
+def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
+    """One decode step; `state` [N, H, dk, dv] fp32 is updated in place.  Returns o."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("state", state)):
+        _contig(name, t)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    code = load().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                  N, H, dk, dv, _DTYPE[q.dtype], _ptr(o), _stream(stream))
+    _check(code, "kda_decode_step")
+    return o
+
+
+def kda_check_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status code."""
+    return int(load().kda_check_device_error(_stream(stream)))
+
+
+def kda_selftest_bounded_wait(timeout_us: int, stream=None):
+    _check(load().kda_selftest_bounded_wait(int(timeout_us), _stream(stream)),
+           "kda_selftest_bounded_wait")
+
+
+def kda_profile_enable(enable: bool = True):
+    _check(load().kda_profile_enable(1 if enable else 0), "kda_profile_enable")
+
+
+def kda_profile_last(capacity: int = 8):
+    """Device milliseconds of each kernel of the most recent call (launch order)."""
+    buf = (ctypes.c_float * capacity)()
+    cnt = ctypes.c_int(0)
+    _check(load().kda_profile_last(buf, capacity, ctypes.byref(cnt)), "kda_profile_last")
+    return [float(buf[i]) for i in range(cnt.value)]
+
+
+# ---------------------------------------------------------------- raw C-ABI access
+
+def raw_prefill(args: dict) -> int:
+    """Call kda_chunk_prefill with raw integers/pointers (for ABI-level tests)."""
+    lib = load()
+    return int(lib.kda_chunk_prefill(
+        args.get("q"), args.get("k"), args.get("v"), args.get("g"), args.get("beta"),
+        args.get("state_in"), args.get("cu_seqlens"), args["B"], args["T"], args["N"],
+        args["H"], args["dk"], args["dv"], args["dtype"], args.get("o"), args.get("state_out"),
+        args.get("workspace"), args.get("workspace_bytes", 0), args.get("stream")))
+
+
+def raw_decode(args: dict) -> int:
+    lib = load()
+    return int(lib.kda_decode_step(
+        args.get("q"), args.get("k"), args.get("v"), args.get("g"), args.get("beta"),
+        args.get("state"), args["N"], args["H"], args["dk"], args["dv"], args["dtype"],
+        args.get("o"), args.get("stream")))

@@ -1,0 +1,211 @@
+// C ABI of libkda (declared in include/kda.h): argument validation, the
+// device error word, and dispatch to the kernels.  All argument errors are
+// reported before anything is launched.
+#include "kda.h"
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+#include <mutex>
+
+namespace {
+
+// One error word per device context, in this library's own device memory.
+// Kernels receive its device address as an argument.
+__device__ uint32_t g_kda_error_word;
+
+constexpr int kMaxDevices = 64;
+uint32_t *g_err_ptr[kMaxDevices];
+std::mutex g_err_mu;
+
+uint32_t *error_word_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kda_error_word) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<uint32_t *>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+bool supported_dim(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// ---- kernel timing (kda_profile_enable / kda_profile_last)
+constexpr int kMaxMarks = 8;
+struct ProfState {
+    bool enabled = false;
+    int device = -1;
+    cudaEvent_t ev[kMaxMarks] = {};
+    int n = 0;   // events recorded in the current record
+};
+ProfState g_prof;
+std::mutex g_prof_mu;
+
+}  // namespace
+
+namespace kda {
+
+void Profiler::begin(cudaStream_t st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.n = 0;
+    if (!g_prof.enabled) return;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != g_prof.device) return;
+    if (cudaEventRecord(g_prof.ev[0], st) == cudaSuccess) g_prof.n = 1;
+}
+
+void Profiler::mark(cudaStream_t st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof.enabled || g_prof.n == 0 || g_prof.n >= kMaxMarks) return;
+    if (cudaEventRecord(g_prof.ev[g_prof.n], st) == cudaSuccess) ++g_prof.n;
+}
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns, uint32_t *err) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    // Nothing ever arrives on `bar`: phase 0 never completes, the bounded
+    // wait gives up after `limit_ns` and records the timeout.
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, err, limit_ns)) atomicOr(err, ERR_SELFTEST);
+}
+
+cudaError_t launch_selftest_wait(uint64_t timeout_us, uint32_t *err, cudaStream_t st) {
+    selftest_wait_kernel<<<1, 32, 0, st>>>(timeout_us * 1000ull, err);
+    return cudaGetLastError();
+}
+
+}  // namespace kda
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+size_t kda_chunk_prefill_workspace_bytes(int64_t rows, int N, int H, int dk, int dv,
+                                         kda_dtype dtype) {
+    if (rows < 0 || N < 0 || H <= 0 || !supported_dim(dk, dv)) return 0;
+    if (dtype != KDA_BF16) return 0;
+    return kda::prefill_tc_workspace_bytes(rows, N, H, dk);
+}
+
+kda_status kda_chunk_prefill(const void *q, const void *k, const void *v, const void *g,
+                             const void *beta, const float *state_in,
+                             const int32_t *cu_seqlens, int B, int64_t T, int N, int H,
+                             int dk, int dv, kda_dtype dtype, void *o, float *state_out,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    if (B < 0 || T < 0 || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens ? B != 1 : N != B) return KDA_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * T;
+    if (rows > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)N * H > (int64_t)INT32_MAX / 2) return KDA_ERR_UNSUPPORTED;
+    const size_t need = kda_chunk_prefill_workspace_bytes(rows, N, H, dk, dv, dtype);
+    if (need > 0 && (!workspace || workspace_bytes < need ||
+                     (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+        return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+
+    uint32_t *err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    kda::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv,
+                       o, state_out, workspace, workspace_bytes, err};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kda::Profiler::begin(st);
+    if (dtype == KDA_F32) return from_cuda(kda::launch_prefill_simt(a, false, st));
+    return from_cuda(kda::launch_prefill_tc(a, st));
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *g,
+                           const void *beta, float *state, int N, int H, int dk, int dv,
+                           kda_dtype dtype, void *o, void *stream) {
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (N > 0 && (!q || !k || !v || !g || !beta || !state || !o)) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)N * H > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    if ((reinterpret_cast<uintptr_t>(state) & 15u) != 0) return KDA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kda::Profiler::begin(st);
+    return from_cuda(kda::launch_decode(q, k, v, g, beta, state, N, H, dk, dtype == KDA_BF16, o,
+                                        st));
+}
+
+kda_status kda_check_device_error(void *stream) {
+    uint32_t *err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_kda_error_word, sizeof(word)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (word != 0) {
+        const uint32_t zero = 0;
+        if (cudaMemcpyToSymbol(g_kda_error_word, &zero, sizeof(zero)) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        return KDA_ERR_TIMEOUT;
+    }
+    return KDA_OK;
+}
+
+kda_status kda_profile_enable(int enable) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.n = 0;
+    if (!enable) {
+        g_prof.enabled = false;
+        return KDA_OK;
+    }
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    if (g_prof.device != dev) {
+        for (int i = 0; i < kMaxMarks; ++i)
+            if (g_prof.ev[i]) {
+                cudaEventDestroy(g_prof.ev[i]);
+                g_prof.ev[i] = nullptr;
+            }
+        for (int i = 0; i < kMaxMarks; ++i)
+            if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return KDA_ERR_CUDA;
+        g_prof.device = dev;
+    }
+    g_prof.enabled = true;
+    return KDA_OK;
+}
+
+kda_status kda_profile_last(float *ms, int capacity, int *count) {
+    if (!ms || !count || capacity < 0) return KDA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    *count = 0;
+    if (g_prof.n < 2) return KDA_OK;
+    if (cudaEventSynchronize(g_prof.ev[g_prof.n - 1]) != cudaSuccess) return KDA_ERR_CUDA;
+    int c = 0;
+    for (int i = 1; i < g_prof.n && c < capacity; ++i, ++c)
+        if (cudaEventElapsedTime(&ms[c], g_prof.ev[i - 1], g_prof.ev[i]) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    *count = c;
+    return KDA_OK;
+}
+
+kda_status kda_selftest_bounded_wait(int64_t timeout_us, void *stream) {
+    if (timeout_us < 1 || timeout_us > 10000000) return KDA_ERR_INVALID_ARG;
+    uint32_t *err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    return from_cuda(kda::launch_selftest_wait((uint64_t)timeout_us, err,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,121 @@
+// Shared device helpers for the KDA kernels: element conversion, bounded
+// waits and the device error word protocol.  sm_100a only.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+// Bits recorded in the device error word (one 32-bit word per library
+// instance and device, cleared by kda_check_device_error).
+enum : uint32_t {
+    ERR_WAIT_TIMEOUT = 1u,     // a bounded mbarrier/flag wait gave up
+    ERR_SELFTEST = 2u,         // set by the bounded-wait self test
+};
+
+// Upper bound on the wall time of one device-side wait.  Legitimate waits in
+// these kernels last microseconds; anything past this bound means a missing
+// arrival, and the waiting thread gives up instead of hanging the GPU.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+        "r"(bytes)
+        : "memory");
+}
+
+// One poll of the phase with the given parity; true once that phase completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on the phase with the given parity.  Gives up after
+// `limit_ns` nanoseconds of wall time (measured with %globaltimer): it then
+// sets ERR_WAIT_TIMEOUT in the error word and returns false; the caller must
+// stop issuing work and leave through its normal exit path.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) break;
+    }
+    if (err) atomicOr(err, ERR_WAIT_TIMEOUT);
+    return false;
+}
+
+// As mbar_wait, and also gives up as soon as another thread of the CTA has
+// raised the shared abort flag (set here on a timeout), or any CTA has set the
+// device error word, so that one missing arrival ends every waiting role of
+// every CTA within microseconds instead of one time limit per CTA.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t parity,
+                                                    uint32_t *err, volatile uint32_t *abort,
+                                                    uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    const volatile uint32_t *gerr = err;
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (gerr && *gerr) {   // some CTA already gave up: do not wait out the limit too
+            *abort = 1u;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > limit_ns) break;
+    }
+    if (err) atomicOr(err, ERR_WAIT_TIMEOUT);
+    *abort = 1u;
+    return false;
+}
+
+}  // namespace kda

@@ -1,0 +1,40 @@
+// Internal launch interface between the C ABI (kda_abi.cu) and the kernel
+// translation units.  Not part of the public header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+struct PrefillArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *state_in;
+    const int32_t *cu_seqlens;   // device, N+1 entries, or nullptr
+    int B;
+    int64_t T;                   // rows per batch entry (packed rows when cu_seqlens)
+    int N, H, dk, dv;
+    void *o;
+    float *state_out;
+    void *workspace;
+    size_t workspace_bytes;
+    uint32_t *err;               // device error word
+};
+
+// Optional per-kernel event recording (see kda_profile_enable).  Launchers
+// call mark() before their first kernel and after each kernel.
+struct Profiler {
+    static void begin(cudaStream_t st);   // start a new record
+    static void mark(cudaStream_t st);    // event after a kernel
+};
+
+cudaError_t launch_prefill_simt(const PrefillArgs &a, bool bf16, cudaStream_t st);
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st);
+size_t prefill_tc_workspace_bytes(int64_t rows, int N, int H, int d);
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *g,
+                          const void *beta, float *state, int N, int H, int d, bool bf16,
+                          void *o, cudaStream_t st);
+cudaError_t launch_selftest_wait(uint64_t timeout_us, uint32_t *err, cudaStream_t st);
+
+}  // namespace kda

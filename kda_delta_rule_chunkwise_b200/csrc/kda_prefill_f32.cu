@@ -1,0 +1,234 @@
+// KDA chunked prefill, fp32 reference-precision path (SIMT, fp32 FMA).
+//
+// One CTA per (sequence, head).  The state S (dk x dv, fp32) stays in shared
+// memory for the whole sequence; the sequence is walked in chunks of C
+// tokens, and each chunk is done in the chunk-parallel (WY) form:
+//
+//   G_r    = sum_{s<=r} max(g_s, -5)                  chunk-local cumsum
+//   Akk    = strictly-lower  beta_r sum_c k_r k_s exp(G_r - G_s)
+//   Aqk    = lower (incl. diagonal)  sum_c q_r k_s exp(G_r - G_s)
+//   X      = (I + Akk)^-1 (forward substitution),  T = X Diag(beta)
+//   U      = T (V - (K * exp(G)) S)
+//   O      = (Q * exp(G)) S + Aqk U
+//   S     <- Diag(exp(G_L)) S + (K * exp(G_L - G))^T U
+//
+// This is the recurrence S_t = (I - beta k k^T) Diag(exp g) S_{t-1} +
+// beta k v^T, o_t = S_t^T q_t (the delta rule with per-channel retention of
+// neurohive.io "Kimi K3 ... overview", section "Sequence length: hybrid KDA
+// and Gated MLA attention") unrolled over one chunk.  Each pairwise decay
+// exp(G_r - G_s) <= 1 is evaluated directly in fp32, so no rescaling is
+// needed on this path; it exists for fp32 inputs with a 1e-4 error budget.
+#include "kda_common.cuh"
+
+namespace kda {
+
+template <int DK, int DV, int C>
+struct F32Smem {
+    static constexpr int kS = DK * DV;
+    static constexpr int kFloats = kS + 3 * C * DK + 2 * C * DV + 2 * C * C + C + 2 * DK;
+    static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+template <int DK, int DV, int C, typename Tin>
+__global__ void __launch_bounds__(256)
+prefill_f32_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                   const Tin *__restrict__ v, const Tin *__restrict__ g,
+                   const Tin *__restrict__ beta, const float *state_in,
+                   const int32_t *__restrict__ cu_seqlens, int64_t T, int N, int H,
+                   Tin *__restrict__ o, float *state_out) {
+    constexpr int NT = 256;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = blockIdx.x / H, h = blockIdx.x % H;
+    if (n >= N) return;
+
+    int64_t r0, r1;
+    if (cu_seqlens) {
+        int64_t a = cu_seqlens[n], b = cu_seqlens[n + 1];
+        a = a < 0 ? 0 : (a > T ? T : a);
+        b = b < 0 ? 0 : (b > T ? T : b);
+        r0 = a;
+        r1 = b < a ? a : b;
+    } else {
+        r0 = (int64_t)n * T;
+        r1 = r0 + T;
+    }
+
+    extern __shared__ float sm[];
+    float *S = sm;                 // [DK][DV]
+    float *Qs = S + DK * DV;       // [C][DK]  q, then q*exp(G)
+    float *Ks = Qs + C * DK;       // [C][DK]  k, then k*exp(G)
+    float *Gs = Ks + C * DK;       // [C][DK]  G, then k*exp(G_L - G)
+    float *Vs = Gs + C * DK;       // [C][DV]  v, then v - Ktilde S
+    float *Us = Vs + C * DV;       // [C][DV]
+    float *Akk = Us + C * DV;      // [C][C]   Akk, then T
+    float *Aqk = Akk + C * C;      // [C][C]
+    float *bs = Aqk + C * C;       // [C]
+    float *GL = bs + C;            // [DK] G at the last valid row
+    float *GLe = GL + DK;          // [DK] exp(G_L)
+
+    const size_t sbase = ((size_t)n * H + h) * (size_t)DK * DV;
+    for (int i = tid; i < DK * DV; i += NT) S[i] = state_in ? state_in[sbase + i] : 0.f;
+
+    for (int64_t t0 = r0; t0 < r1; t0 += C) {
+        const int L = (int)((r1 - t0) < C ? (r1 - t0) : C);
+        __syncthreads();
+        // 1. load the chunk (rows >= L are zero; g clamped at -5)
+        for (int i = tid; i < C * DK; i += NT) {
+            const int r = i / DK, c = i % DK;
+            float qv = 0.f, kv = 0.f, gv = 0.f;
+            if (r < L) {
+                const size_t off = ((size_t)(t0 + r) * H + h) * DK + c;
+                qv = to_f32(q[off]);
+                kv = to_f32(k[off]);
+                gv = fmaxf(to_f32(g[off]), -5.f);
+            }
+            Qs[i] = qv;
+            Ks[i] = kv;
+            Gs[i] = gv;
+        }
+        for (int i = tid; i < C * DV; i += NT) {
+            const int r = i / DV, j = i % DV;
+            Vs[i] = r < L ? to_f32(v[((size_t)(t0 + r) * H + h) * DV + j]) : 0.f;
+        }
+        for (int r = tid; r < C; r += NT)
+            bs[r] = r < L ? to_f32(beta[(size_t)(t0 + r) * H + h]) : 0.f;
+        __syncthreads();
+        // 2. chunk-local inclusive cumsum of the log-decay, per channel
+        for (int c = tid; c < DK; c += NT) {
+            float acc = 0.f, last = 0.f;
+            for (int r = 0; r < C; ++r) {
+                acc += Gs[r * DK + c];
+                Gs[r * DK + c] = acc;
+                if (r == L - 1) last = acc;
+            }
+            GL[c] = last;
+            GLe[c] = expf(last);
+        }
+        __syncthreads();
+        // 3. Akk / Aqk, one warp per (r, s) pair with s <= r
+        for (int p = warp; p < C * (C + 1) / 2; p += NT / 32) {
+            int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+            while ((r + 1) * (r + 2) / 2 <= p) ++r;
+            while (r * (r + 1) / 2 > p) --r;
+            const int s = p - r * (r + 1) / 2;
+            float kk = 0.f, qk = 0.f;
+            for (int c = lane; c < DK; c += 32) {
+                const float e = expf(Gs[r * DK + c] - Gs[s * DK + c]);
+                const float ks = Ks[s * DK + c] * e;
+                kk = fmaf(Ks[r * DK + c], ks, kk);
+                qk = fmaf(Qs[r * DK + c], ks, qk);
+            }
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) {
+                kk += __shfl_xor_sync(0xffffffffu, kk, m);
+                qk += __shfl_xor_sync(0xffffffffu, qk, m);
+            }
+            if (lane == 0) {
+                Akk[r * C + s] = s < r ? bs[r] * kk : 0.f;
+                Aqk[r * C + s] = qk;
+                if (s < r) {
+                    Akk[s * C + r] = 0.f;
+                    Aqk[s * C + r] = 0.f;
+                }
+            }
+        }
+        __syncthreads();
+        // 4. X = (I + Akk)^-1 by forward substitution (row r needs rows < r)
+        //    X[r][j] = -A[r][j] - sum_{j<s<r} A[r][s] X[s][j]   (X[j][j] = 1 implicit)
+        for (int r = 1; r < C; ++r) {
+            float x = 0.f;
+            const int j = tid;
+            if (j < r) {
+                x = -Akk[r * C + j];
+                for (int s = j + 1; s < r; ++s) x = fmaf(-Akk[r * C + s], Akk[s * C + j], x);
+            }
+            __syncthreads();
+            if (j < r) Akk[r * C + j] = x;
+            __syncthreads();
+        }
+        // X has an implicit unit diagonal; T = X Diag(beta) (T[r][r] = beta_r)
+        for (int i = tid; i < C * C; i += NT) {
+            const int r = i / C, s = i % C;
+            const float x = r == s ? 1.f : (s < r ? Akk[i] : 0.f);
+            Akk[i] = x * bs[s];
+        }
+        __syncthreads();
+        // 5. q*exp(G), k*exp(G), k*exp(G_L - G)
+        for (int i = tid; i < C * DK; i += NT) {
+            const int c = i % DK;
+            const float gg = Gs[i], kv = Ks[i];
+            const float eg = expf(gg);
+            Qs[i] *= eg;
+            Ks[i] = kv * eg;
+            Gs[i] = kv * expf(GL[c] - gg);
+        }
+        __syncthreads();
+        // 6. Vs <- V - Ktilde S, then U = T Vs
+        for (int i = tid; i < C * DV; i += NT) {
+            const int r = i / DV, j = i % DV;
+            float acc = Vs[i];
+            for (int c = 0; c < DK; ++c) acc = fmaf(-Ks[r * DK + c], S[c * DV + j], acc);
+            Vs[i] = acc;
+        }
+        __syncthreads();
+        for (int i = tid; i < C * DV; i += NT) {
+            const int r = i / DV, j = i % DV;
+            float acc = 0.f;
+            for (int s = 0; s <= r; ++s) acc = fmaf(Akk[r * C + s], Vs[s * DV + j], acc);
+            Us[i] = acc;
+        }
+        __syncthreads();
+        // 7. O = Qtilde S + Aqk U
+        for (int i = tid; i < C * DV; i += NT) {
+            const int r = i / DV, j = i % DV;
+            if (r >= L) continue;
+            float acc = 0.f;
+            for (int c = 0; c < DK; ++c) acc = fmaf(Qs[r * DK + c], S[c * DV + j], acc);
+            for (int s = 0; s <= r; ++s) acc = fmaf(Aqk[r * C + s], Us[s * DV + j], acc);
+            o[((size_t)(t0 + r) * H + h) * DV + j] = from_f32<Tin>(acc);
+        }
+        __syncthreads();
+        // 8. S <- Diag(exp G_L) S + Khat^T U
+        for (int i = tid; i < DK * DV; i += NT) {
+            const int c = i / DV, j = i % DV;
+            float acc = GLe[c] * S[i];
+            for (int r = 0; r < L; ++r) acc = fmaf(Gs[r * DK + c], Us[r * DV + j], acc);
+            S[i] = acc;
+        }
+    }
+    __syncthreads();
+    if (state_out)
+        for (int i = tid; i < DK * DV; i += NT) state_out[sbase + i] = S[i];
+}
+
+}  // namespace kda
+
+#include "kda_launch.h"
+
+namespace kda {
+
+template <int D, int C, typename Tin>
+static cudaError_t launch_f32_t(const PrefillArgs &a, cudaStream_t st) {
+    constexpr size_t smem = F32Smem<D, D, C>::kBytes;
+    auto kern = prefill_f32_kernel<D, D, C, Tin>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = a.N * a.H;
+    if (grid == 0) return cudaSuccess;
+    kern<<<grid, 256, smem, st>>>((const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v,
+                                  (const Tin *)a.g, (const Tin *)a.beta, a.state_in,
+                                  a.cu_seqlens, a.T, a.N, a.H, (Tin *)a.o, a.state_out);
+    e = cudaGetLastError();
+    Profiler::mark(st);
+    return e;
+}
+
+// fp32 (and, for cross-checks, bf16-input) SIMT chunked prefill.
+cudaError_t launch_prefill_simt(const PrefillArgs &a, bool bf16, cudaStream_t st) {
+    if (a.dk == 64)
+        return bf16 ? launch_f32_t<64, 64, __nv_bfloat16>(a, st) : launch_f32_t<64, 64, float>(a, st);
+    return bf16 ? launch_f32_t<128, 32, __nv_bfloat16>(a, st) : launch_f32_t<128, 32, float>(a, st);
+}
+
+}  // namespace kda

@@ -1,0 +1,122 @@
+"""The C ABI: library loads, exports every declared symbol, rejects bad
+arguments synchronously (no device needed for any of these)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kda_delta_rule_chunkwise_b200 import binding
+from kda_delta_rule_chunkwise_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return binding.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(binding.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED",
+                                 "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]):
+        assert binding.status_string(code) == name
+
+
+def test_workspace_bytes(lib):
+    f = lib.kda_chunk_prefill_workspace_bytes
+    assert f(1000, 1, 4, 64, 64, binding.KDA_F32) == 0          # fp32 path: no workspace
+    assert f(1000, 1, 4, 96, 96, binding.KDA_BF16) == 0         # unsupported size
+    w1 = f(64 * 10, 1, 4, 128, 128, binding.KDA_BF16)
+    w2 = f(64 * 10, 3, 4, 128, 128, binding.KDA_BF16)
+    assert w1 > 0 and w2 > w1                                    # bound grows with N
+    assert w1 % 256 == 0
+    # upper bound holds for any split of the rows into N sequences
+    assert f(0, 0, 1, 128, 128, binding.KDA_BF16) >= 0
+
+
+def _args(**kw):
+    base = dict(q=1, k=2, v=3, g=4, beta=5, o=6, B=1, T=16, N=1, H=2, dk=64, dv=64,
+                dtype=binding.KDA_F32)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("bad", [
+    dict(B=-1), dict(T=-5), dict(H=0), dict(N=2),                   # N must equal B
+    dict(q=None), dict(o=None), dict(dtype=7),
+    dict(cu_seqlens=9, B=2),                                         # packed needs B == 1
+])
+def test_prefill_rejects_invalid_arguments(lib, bad):
+    assert binding.raw_prefill(_args(**bad)) == binding.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [dict(dk=96, dv=96), dict(dk=64, dv=128), dict(dk=32, dv=32)])
+def test_prefill_rejects_unsupported_sizes(lib, bad):
+    assert binding.raw_prefill(_args(**bad)) == binding.KDA_ERR_UNSUPPORTED
+
+
+def test_prefill_bf16_requires_workspace(lib):
+    a = _args(dtype=binding.KDA_BF16, dk=128, dv=128)
+    assert binding.raw_prefill(a) == binding.KDA_ERR_INVALID_ARG
+    need = lib.kda_chunk_prefill_workspace_bytes(16, 1, 2, 128, 128, binding.KDA_BF16)
+    a.update(workspace=4096, workspace_bytes=need - 1)
+    assert binding.raw_prefill(a) == binding.KDA_ERR_INVALID_ARG
+    a.update(workspace=4096 + 16, workspace_bytes=need)           # not 256-byte aligned
+    assert binding.raw_prefill(a) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_prefill_zero_sequences_is_a_no_op(lib):
+    # N = B = 0: nothing to do, nothing launched
+    assert binding.raw_prefill(_args(B=0, N=0, q=None, k=None, v=None, g=None, beta=None,
+                                     o=None)) == binding.KDA_OK
+
+
+def _dargs(**kw):
+    base = dict(q=1, k=2, v=3, g=4, beta=5, state=16, o=6, N=4, H=2, dk=128, dv=128,
+                dtype=binding.KDA_BF16)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("bad", [dict(N=-1), dict(H=0), dict(state=None), dict(o=None),
+                                 dict(dtype=3), dict(state=18)])   # state must be 16B aligned
+def test_decode_rejects_invalid_arguments(lib, bad):
+    assert binding.raw_decode(_dargs(**bad)) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_unsupported_sizes(lib):
+    assert binding.raw_decode(_dargs(dk=128, dv=64)) == binding.KDA_ERR_UNSUPPORTED
+
+
+def test_decode_zero_sequences_is_a_no_op(lib):
+    assert binding.raw_decode(_dargs(N=0)) == binding.KDA_OK
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.kda_selftest_bounded_wait(0, None) == binding.KDA_ERR_INVALID_ARG
+    assert lib.kda_selftest_bounded_wait(10**7 + 1, None) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(RuntimeError, match="libkda.so not found"):
+        binding.load(str(tmp_path / "nope.so"))

@@ -38,9 +38,9 @@ DECODE_WORKLOAD = "decode_n256_h32_d128"
 L2_BYTES = 126 * 2**20
 
 # algorithmic bytes (the minimum the path must move), per (token, head)
-PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 + 128 * 2      # q,k,v,g,beta in; o out (bf16)
+PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 + 128 * 4      # q,k,v,g,beta in (bf16); o out (fp32)
 STATE_BYTES = 128 * 128 * 4                                   # one fp32 state, one direction
-DECODE_BYTES_PER_UNIT = 2 * STATE_BYTES + 4 * 128 * 2 + 2 + 128 * 2
+DECODE_BYTES_PER_UNIT = 2 * STATE_BYTES + 4 * 128 * 2 + 2 + 128 * 4
 SLOT_BYTES = 66560                                            # per (chunk, head) workspace slot
 FLOPS_PER_TOKEN_HEAD = 139264                                 # algorithmic MMA flops (causal halves once)
 
@@ -165,7 +165,7 @@ def run_ours(args, rank, world, dev):
     d = kin.workload_inputs(PREFILL_WORKLOAD, seed=args.seed + rank, device=dev)
     B, T, H = d.B, d.T, d.H
     tokens = B * T
-    o = torch.empty_like(d.v)
+    o = torch.empty(d.v.shape, dtype=torch.float32, device=dev)
     s_out = torch.empty((d.N, H, 128, 128), dtype=torch.float32, device=dev)
     ws = torch.empty(binding.kda_chunk_prefill_workspace_bytes(tokens, d.N, H, 128, 128,
                                                                 torch.bfloat16),
@@ -195,7 +195,7 @@ def run_ours(args, rank, world, dev):
     k_bytes = {
         "chunk_table_kernel": 8 * (d.N + 1),
         "intra_chunk_kernel": head_chunks * (64 * (3 * 128 * 2 + 2) + SLOT_BYTES),
-        "state_pass_kernel": head_chunks * (SLOT_BYTES + 2 * 64 * 128 * 2)
+        "state_pass_kernel": head_chunks * (SLOT_BYTES + 64 * 128 * 2 + 64 * 128 * 4)
         + d.N * H * 2 * STATE_BYTES,
     }
     dom = max(range(n_k), key=lambda i: k_avg[i])
@@ -269,7 +269,7 @@ def run_ours(args, rank, world, dev):
                             seed=args.seed + 1000 + rank, device=dev)
     pristine = dec.state.clone()
     S = dec.state
-    od = torch.empty((Nd, Hd, 128), dtype=torch.bfloat16, device=dev)
+    od = torch.empty((Nd, Hd, 128), dtype=torch.float32, device=dev)
 
     def dec_step(t):
         binding.kda_decode_step(dec.q[t], dec.k[t], dec.v[t], dec.g[t], dec.beta[t], S, o=od)

@@ -24,9 +24,11 @@
  *  - All tensor arguments are DEVICE pointers owned by the caller, dense and
  *    row-major in the shapes given; the library never frees or keeps them.
  *  - q, k, g share the shape [rows, H, dk]; v and o are [rows, H, dv];
- *    beta is [rows, H].  Element type is `dtype` for q, k, v, g, beta and o.
- *  - The state is always fp32 [N, H, dk, dv]: row c = key channel, column j
- *    = value channel, so o_t[j] = sum_c S_t[c][j] q_t[c].
+ *    beta is [rows, H].  Element type is `dtype` for q, k, v, g and beta.
+ *  - o is always fp32, and so is the state [N, H, dk, dv]: row c = key
+ *    channel, column j = value channel, so o_t[j] = sum_c S_t[c][j] q_t[c].
+ *    (Both accumulate in fp32; rounding o to bf16 alone would cost up to
+ *    ~4e-2 of max|error|/rms(o) on heavy-tailed outputs.)
  *  - g is the per-step log-decay; the contract is g in [-5, 0].  Values
  *    below -5 are treated as -5 (max(g, -5)); values above 0 are used as
  *    given.  q and k are expected L2-normalised by the caller; the library
@@ -67,8 +69,10 @@ typedef enum {
 } kda_status;
 
 typedef enum {
-    KDA_F32 = 0,   /* fp32 q, k, v, g, beta, o; fp32 arithmetic throughout (reference precision) */
-    KDA_BF16 = 1   /* bf16 q, k, v, g, beta, o; tensor-core products with fp32 accumulation, fp32 state */
+    KDA_F32 = 0,   /* fp32 q, k, v, g, beta; fp32 arithmetic throughout (reference precision) */
+    KDA_BF16 = 1   /* bf16 q, k, v, g, beta; tensor-core products (tf32 for the decay-rescaled
+                      intra-chunk products, fp16 elsewhere) with fp32 accumulation; fp32 state
+                      and o.  |v| and |state| must stay below 65504 (fp16 operand range). */
 } kda_dtype;
 
 /*
@@ -100,7 +104,7 @@ KDA_API size_t kda_chunk_prefill_workspace_bytes(int64_t rows, int N, int H, int
  *              never make the library read or write outside the buffers
  *              (offsets are clamped to [0, T] and raised to the previous
  *              offset), but the results for such sequences are unspecified.
- *  o           [B, T, H, dv], written for every token that belongs to a sequence
+ *  o           [B, T, H, dv] fp32, written for every token that belongs to a sequence
  *  state_out   [N, H, dk, dv] fp32, final state per sequence, or NULL (not
  *              written).  May alias state_in exactly (in-place update).
  *              A zero-length sequence gets state_out = state_in (or zeros).
@@ -122,7 +126,7 @@ KDA_API kda_status kda_chunk_prefill(const void *q, const void *k, const void *v
  * of each (n, h) state):
  *     S' = Diag(exp g) S;  delta = beta (v - S'^T k);  S = S' + k delta^T;
  *     o = S^T q
- *  q, k, g [N, H, dk];  v [N, H, dv];  beta [N, H];  o [N, H, dv]
+ *  q, k, g [N, H, dk];  v [N, H, dv];  beta [N, H];  o [N, H, dv] fp32
  *  state   [N, H, dk, dv] fp32, read and overwritten.
  */
 KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,

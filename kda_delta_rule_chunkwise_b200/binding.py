@@ -112,7 +112,8 @@ def kda_chunk_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=Non
 
     q, k, g: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H] (all one dtype,
     bf16 or fp32); state_in: [N, H, dk, dv] fp32 or None; cu_seqlens: int32
-    [N+1] on the device or None.  Output buffers are allocated if not given.
+    [N+1] on the device or None.  o [B, T, H, dv] and the state are fp32.
+    Output buffers are allocated if not given.
     """
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -123,7 +124,7 @@ def kda_chunk_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=Non
     if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
         raise ValueError("cu_seqlens must be int32")
     if o is None:
-        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
     if state_out is None and want_state:
         state_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
     need = kda_chunk_prefill_workspace_bytes(B * T, N, H, dk, dv, q.dtype)
@@ -139,13 +140,13 @@ def kda_chunk_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=Non
 
 
 def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
-    """One decode step; `state` [N, H, dk, dv] fp32 is updated in place.  Returns o."""
+    """One decode step; `state` [N, H, dk, dv] fp32 is updated in place.  Returns o (fp32)."""
     N, H, dk = q.shape
     dv = v.shape[-1]
     for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("state", state)):
         _contig(name, t)
     if o is None:
-        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+        o = torch.empty((N, H, dv), dtype=torch.float32, device=q.device)
     code = load().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
                                   N, H, dk, dv, _DTYPE[q.dtype], _ptr(o), _stream(stream))
     _check(code, "kda_decode_step")

@@ -8,6 +8,7 @@
 // neurohive.io "Kimi K3 ... overview", section "Training and inference
 // infrastructure", advanced by one token.
 //
+// o is written in fp32 for either input dtype (the step accumulates in fp32).
 // The step is bound by HBM: each (n, h) state (dk*dv fp32, 64 KiB at d=128)
 // is read once and written once; everything else is ~1 KiB.  One CTA of 256
 // threads per (n, h).  Each thread keeps a (DK/RG) x 4 block of S in
@@ -24,7 +25,7 @@ template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256, 2)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const Tin *__restrict__ g, const Tin *__restrict__ beta, float *__restrict__ state,
-              Tin *__restrict__ o, int units) {
+              float *__restrict__ o, int units) {
     constexpr int NT = 256;
     constexpr int CG = DV / 4;        // 16-byte column groups per row
     constexpr int RG = NT / CG;       // row groups
@@ -87,7 +88,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         }
         const float d = b_sh * (vs[tid] - pj);
         dl[tid] = d;
-        o[(size_t)unit * DV + tid] = from_f32<Tin>(fmaf(kq_sh, d, yj));
+        o[(size_t)unit * DV + tid] = fmaf(kq_sh, d, yj);
     }
     __syncthreads();
     const float4 d4 = reinterpret_cast<const float4 *>(dl)[cg];
@@ -113,7 +114,7 @@ static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, 
                                    cudaStream_t st) {
     decode_kernel<D, D, Tin><<<units, 256, 0, st>>>(
         (const Tin *)q, (const Tin *)k, (const Tin *)v, (const Tin *)g, (const Tin *)beta,
-        state, (Tin *)o, units);
+        state, (float *)o, units);
     cudaError_t e = cudaGetLastError();
     Profiler::mark(st);
     return e;

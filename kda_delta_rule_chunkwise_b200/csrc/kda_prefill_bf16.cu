@@ -30,10 +30,21 @@
 // With U = T V - W S this is the WY form: U are the chunk's pseudo-values and
 // O = Q*exp(G) S + Aqk U, the chunk's outputs.
 //
-// Roles in phase B: warp 0 = producer (1-D bulk copy of the slot + cp.async
-// of the V slice), warp 1 = MMA issuer and TMEM owner, warps 4-7 = U/O
+// Roles in phase B: warp 0 = producer (1-D bulk copy of the slot, V slice
+// converted to fp16), warp 1 = MMA issuer and TMEM owner, warps 4-7 = U/O
 // epilogue (TMEM -> registers), warps 8-11 = state epilogue (Gamma scaling
-// of the TMEM state, bf16 copy of S for the next chunk's MMA).
+// of the TMEM state, fp16 copy of S for the next chunk's MMA).
+//
+// Precision.  Inputs are bf16; every product accumulates in fp32 (TMEM); the
+// state and the outputs o are fp32.  The decay-rescaled operands of Akk/Aqk
+// need the fp32 exponent range (factors down to e^-80 and up to e^75), so
+// those MMAs run in tf32.  Every other stored operand is O(1) in magnitude
+// and is kept in fp16, whose 11-bit significand is what the error bound
+// max|do|/rms(o) <= 2e-2 needs on heavy-tailed outputs (8-bit bf16
+// intermediates alone cost about 3e-2 there).  The fp16 operands assume
+// |v| and |state| stay below 65504.
+#include <cuda_fp16.h>
+
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "sm100.cuh"
@@ -140,14 +151,20 @@ __device__ __forceinline__ void seq_rows(const int32_t *hdr, bool packed, int64_
     }
 }
 
+// eight fp32 values -> eight fp16 (round to nearest) in one 16-byte word
 __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
     uint4 u;
-    __nv_bfloat162 t;
-    t = __floats2bfloat162_rn(x[0], x[1]); u.x = *reinterpret_cast<uint32_t *>(&t);
-    t = __floats2bfloat162_rn(x[2], x[3]); u.y = *reinterpret_cast<uint32_t *>(&t);
-    t = __floats2bfloat162_rn(x[4], x[5]); u.z = *reinterpret_cast<uint32_t *>(&t);
-    t = __floats2bfloat162_rn(x[6], x[7]); u.w = *reinterpret_cast<uint32_t *>(&t);
+    __half2 t;
+    t = __floats2half2_rn(x[0], x[1]); u.x = *reinterpret_cast<uint32_t *>(&t);
+    t = __floats2half2_rn(x[2], x[3]); u.y = *reinterpret_cast<uint32_t *>(&t);
+    t = __floats2half2_rn(x[4], x[5]); u.z = *reinterpret_cast<uint32_t *>(&t);
+    t = __floats2half2_rn(x[6], x[7]); u.w = *reinterpret_cast<uint32_t *>(&t);
     return u;
+}
+
+// four fp32 values rounded to tf32, as one 16-byte word
+__device__ __forceinline__ float4 pack4_tf32(float a, float b, float c, float d) {
+    return make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
 
 __device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
@@ -263,71 +280,79 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     __syncthreads();
 
-    // ---- A1: MMA operands for Akk / Aqk (bf16, K-major, 128B swizzle)
+    // ---- A1: Akk / Aqk on tensor cores, tf32 operands (K-major, 128B swizzle),
+    // accumulated over two 64-channel halves that reuse one operand buffer.
     // B tiles: row 32a + i      = q_r * exp(G_r - R_a),  r = 16a + i
     //          row 32a + 16 + i = k_r * exp(G_r - R_a)
-    for (int task = tid; task < 128 * 16; task += 256) {
-        const int row = task >> 4, ch = task & 15;
-        const int a = row >> 5, isk = (row >> 4) & 1, r = 16 * a + (row & 15);
-        float x[8];
-        if (r < L) {
-            const __nv_bfloat16 *src = (isk ? k : q) + ((size_t)(t0 + r) * H + h) * D + ch * 8;
-            unpack8(*reinterpret_cast<const uint4 *>(src), x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int c = ch * 8 + e;
-                x[e] *= __expf(Gs[r * D + c] - Rref[a * 128 + c]);
+    // A tiles: K^(a) row s (s <= 16a+15) = k_s * exp(R_a - G_s), packed from
+    //          row-group at_group(a)
+    // D^(a) (M=64 rows s, N=32: the 16 q-rows and 16 k-rows of block a) goes to
+    // TMEM columns 32a.
+    const uint32_t tmem_hold = 0;  // (TMEM base read after the first barrier below)
+    (void)tmem_hold;
+    bool ok = true;
+    for (int hf = 0; hf < 2; ++hf) {
+        const int c0 = 64 * hf;
+        if (ok) {
+            for (int task = tid; task < 128 * 16; task += 256) {
+                const int row = task >> 4, ch = task & 15;   // ch: 4-channel chunk of this half
+                const int a = row >> 5, isk = (row >> 4) & 1, r = 16 * a + (row & 15);
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (r < L) {
+                    const __nv_bfloat16 *src =
+                        (isk ? k : q) + ((size_t)(t0 + r) * H + h) * D + c0 + ch * 4;
+                    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+                    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+                    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+                    const int c = c0 + ch * 4;
+                    const float *gr = Gs + r * D + c, *ra = Rref + a * 128 + c;
+                    x = pack4_tf32(f0.x * __expf(gr[0] - ra[0]), f0.y * __expf(gr[1] - ra[1]),
+                                   f1.x * __expf(gr[2] - ra[2]), f1.y * __expf(gr[3] - ra[3]));
+                }
+                *reinterpret_cast<float4 *>(sm + A_BT + sw128_kmajor_off32(row, ch * 4, 16384)) = x;
             }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = 0.f;
-        }
-        *reinterpret_cast<uint4 *>(sm + A_BT + sw128_kmajor_off(row, ch * 8, 16384)) = pack8(x);
-    }
-    // A tiles: K^(a) row s (s <= 16a+15) = k_s * exp(R_a - G_s), packed from row-group at_group(a)
-    for (int task = tid; task < 160 * 16; task += 256) {
-        const int prow = task >> 4, ch = task & 15;
-        int a = 3;
-        if (prow < 16) a = 0; else if (prow < 48) a = 1; else if (prow < 96) a = 2;
-        const int s = prow - at_group(a) * 8;
-        float x[8];
-        if (s < L) {
-            const __nv_bfloat16 *src = k + ((size_t)(t0 + s) * H + h) * D + ch * 8;
-            unpack8(*reinterpret_cast<const uint4 *>(src), x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int c = ch * 8 + e;
-                x[e] *= __expf(Rref[a * 128 + c] - Gs[s * D + c]);
+            for (int task = tid; task < 160 * 16; task += 256) {
+                const int prow = task >> 4, ch = task & 15;
+                int a = 3;
+                if (prow < 16) a = 0; else if (prow < 48) a = 1; else if (prow < 96) a = 2;
+                const int s = prow - at_group(a) * 8;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s < L) {
+                    const __nv_bfloat16 *src = k + ((size_t)(t0 + s) * H + h) * D + c0 + ch * 4;
+                    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+                    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+                    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+                    const int c = c0 + ch * 4;
+                    const float *gs = Gs + s * D + c, *ra = Rref + a * 128 + c;
+                    x = pack4_tf32(f0.x * __expf(ra[0] - gs[0]), f0.y * __expf(ra[1] - gs[1]),
+                                   f1.x * __expf(ra[2] - gs[2]), f1.y * __expf(ra[3] - gs[3]));
+                }
+                *reinterpret_cast<float4 *>(sm + A_AT + sw128_kmajor_off32(prow, ch * 4, A_ATKB)) = x;
             }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = 0.f;
         }
-        *reinterpret_cast<uint4 *>(sm + A_AT + sw128_kmajor_off(prow, ch * 8, A_ATKB)) = pack8(x);
+        fence_async_smem();
+        __syncthreads();
+        tc_fence_after();
+        if (ok && tid == 0) {
+            const uint32_t tm = *tmem_ptr;
+            const uint32_t id = idesc(FMT_TF32, 64, 32, 0, 0);
+            for (int a = 0; a < 4; ++a)
+                for (int kk = 0; kk < 8; ++kk) {          // 8 steps of K=8 over 64 channels
+                    const uint32_t koff = kk >> 2, kin = (kk & 3) * 32;
+                    const uint64_t ad = smem_desc(
+                        sbase + A_AT + at_group(a) * 1024 + koff * A_ATKB + kin, 16, 1024, SW_128B);
+                    const uint64_t bd = smem_desc(sbase + A_BT + (4 * a) * 1024 + koff * 16384 + kin,
+                                                  16, 1024, SW_128B);
+                    mma_tf32(tm + 32 * a, ad, bd, id, (hf > 0 || kk > 0) ? 1u : 0u);
+                }
+            mma_commit(&bars[hf]);
+        }
+        if (ok) ok = mbar_wait_abortable(&bars[hf], 0, err, abort_flag);
+        tc_fence_after();
     }
-    fence_async_smem();
-    __syncthreads();
-    tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
 
-    // D^(a) (M=64 rows s, N=32: 16 q-rows and 16 k-rows of block a) at TMEM column 32a
-    if (tid == 0) {
-        const uint32_t id = idesc_bf16(64, 32, 0, 0);
-        for (int a = 0; a < 4; ++a)
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2), kin = (kk & 3) * 32;
-                const uint64_t ad = smem_desc(sbase + A_AT + at_group(a) * 1024 + koff * A_ATKB + kin,
-                                              16, 1024, SW_128B);
-                const uint64_t bd = smem_desc(sbase + A_BT + (4 * a) * 1024 + koff * 16384 + kin,
-                                              16, 1024, SW_128B);
-                mma_bf16(tmem + 32 * a, ad, bd, id, kk > 0);
-            }
-        mma_commit(&bars[0]);
-    }
-    bool ok = mbar_wait_abortable(&bars[0], 0, err, abort_flag);
-    tc_fence_after();
-
-    // ---- A2: Akk (fp32, beta applied, strictly lower) and Aqk (bf16, lower incl. diagonal)
+    // ---- A2: Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal)
     if (ok && warp < 4) {
         const int s = 16 * warp + (lane & 15);
         for (int a = 0; a < 4; ++a) {
@@ -341,8 +366,8 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                     const int r = 16 * a + j;
                     AK[r * 64 + s] = (s < r && r < L) ? bs[r] * vk[j] : 0.f;
                     const float aq = (s <= r && r < L) ? vq[j] : 0.f;
-                    reinterpret_cast<__nv_bfloat16 *>(sm + A_AQ + sw128_kmajor_off(r, s, 0))[0] =
-                        __float2bfloat16_rn(aq);
+                    reinterpret_cast<__half *>(sm + A_AQ + sw128_kmajor_off(r, s, 0))[0] =
+                        __float2half_rn(aq);
                 }
             }
         }
@@ -436,15 +461,15 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 
     // ---- A4: R = Aqk T  (M=64, N=64, K=64) into TMEM columns 128..191
     if (ok && tid == 0) {
-        const uint32_t id = idesc_bf16(64, 64, 0, 1);
+        const uint32_t id = idesc(FMT_F16, 64, 64, 0, 1);
         for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = smem_desc(sbase + A_AQ + kk * 32, 16, 1024, SW_128B);
             const uint64_t bd = smem_desc(sbase + A_TR + kk * 2048, 8192, 1024, SW_128B);
-            mma_bf16(tmem + 128, ad, bd, id, kk > 0);
+            mma_f16(tmem + 128, ad, bd, id, kk > 0);
         }
-        mma_commit(&bars[1]);
+        mma_commit(&bars[2]);
     }
-    if (ok) ok = mbar_wait_abortable(&bars[1], 0, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[2], 0, err, abort_flag);
     tc_fence_after();
     if (ok && warp < 4) {
         const int r = 16 * warp + (lane & 15);
@@ -472,13 +497,13 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 
     // ---- A5: D1 = [T; R] (K*exp(G))  (M=128, N=128, K=64) into TMEM columns 0..127
     if (ok && tid == 0) {
-        const uint32_t id = idesc_bf16(128, 128, 0, 1);
+        const uint32_t id = idesc(FMT_F16, 128, 128, 0, 1);
         for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = smem_desc(sbase + A_TR + kk * 32, 16, 1024, SW_128B);
             const uint64_t bd = smem_desc(sbase + A_KT + kk * 2048, kKhMNBlock, 1024, SW_128B);
-            mma_bf16(tmem, ad, bd, id, kk > 0);
+            mma_f16(tmem, ad, bd, id, kk > 0);
         }
-        mma_commit(&bars[2]);
+        mma_commit(&bars[3]);
     }
     // [T; R] is final: copy it to the slot while the MMA runs (reads only)
     if (ok) {
@@ -506,7 +531,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         if (tid < 128) reinterpret_cast<float *>(slot + kSlotGam)[tid] = __expf(GL[tid]);
     }
-    if (ok) ok = mbar_wait_abortable(&bars[2], 0, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[3], 0, err, abort_flag);
     tc_fence_after();
 
     // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = Q*exp(G) - R (K*exp(G))
@@ -588,7 +613,7 @@ template <int DVS>
 __global__ void __launch_bounds__(384, 1)
 state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                   const int32_t *__restrict__ cu, int64_t T, int N, int H,
-                  const uint8_t *__restrict__ ws, __nv_bfloat16 *__restrict__ o,
+                  const uint8_t *__restrict__ ws, float *__restrict__ o,
                   float *state_out, uint32_t *err) {
     using Lay = BLayout<DVS>;
     constexpr int NSL = D / DVS;
@@ -656,16 +681,26 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             }
             const int64_t t0 = ra + (int64_t)j * C;
             const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+            // V slice -> fp16 MMA operand (MN-major, interleaved core matrices);
+            // rows past the end of the sequence are zero
             uint8_t *vt = stg + kSlotBytes;
             constexpr int CPR = DVS / 8;   // 16-byte chunks per row
             for (int task = lane; task < 64 * CPR; task += 32) {
                 const int r = task / CPR, ch = task % CPR;
-                const int rr = r < L ? r : 0;
-                const __nv_bfloat16 *vs = v + ((size_t)(t0 + rr) * H + h) * D + j0 + ch * 8;
-                cp_async16(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup), vs,
-                           r < L ? 16u : 0u);
+                float x[8];
+                if (r < L) {
+                    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                        v + ((size_t)(t0 + r) * H + h) * D + j0 + ch * 8));
+                    unpack8(u, x);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = 0.f;
+                }
+                *reinterpret_cast<uint4 *>(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup)) =
+                    pack8(x);
             }
-            cp_async_arrive(&bars[FULL0 + st]);
+            fence_async_smem();
+            mbar_arrive(&bars[FULL0 + st]);
             issued_last = j;
         }
         // drain: never leave the CTA with bulk copies still landing in its shared memory
@@ -674,8 +709,8 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t id_nn = idesc_bf16(128, DVS, 0, 1);   // A K-major, B MN-major
-            const uint32_t id_mm = idesc_bf16(128, DVS, 1, 1);   // A MN-major, B MN-major
+            const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
+            const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
             for (int j = 0; j < nch; ++j) {
                 const int st = j & 1, b = j & 1;
                 const uint32_t stg = sbase + (st ? Lay::oStage1 : Lay::oStage0);
@@ -690,7 +725,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                     const uint64_t ad = smem_desc(stg + kSlotTR + kk * 32, 16, 1024, SW_128B);
                     const uint64_t bd = smem_desc(stg + kSlotBytes + kk * 2 * Lay::kKGroup,
                                                   Lay::kKGroup, 128, SW_NONE);
-                    mma_bf16(tTD, ad, bd, id_nn, kk > 0);
+                    mma_f16(tTD, ad, bd, id_nn, kk > 0);
                 }
                 if (!mbar_wait_abortable(&bars[SBREADY], j & 1, err, abort_flag)) break;
                 tc_fence_after();
@@ -700,7 +735,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         stg + kSlotWP + (kk >> 2) * kWPKBlock + (kk & 3) * 32, 16, 1024, SW_128B);
                     const uint64_t bd = smem_desc(sbase + Lay::oSB + kk * 2 * Lay::kKGroup,
                                                   Lay::kKGroup, 128, SW_NONE);
-                    mma_bf16(tTD, ad, bd, id_nn, 1);
+                    mma_f16(tTD, ad, bd, id_nn, 1);
                 }
                 mma_commit(&bars[TDFULL0 + b]);
                 if (!mbar_wait_abortable(&bars[UBREADY], j & 1, err, abort_flag)) break;
@@ -712,7 +747,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                                                   SW_128B);
                     const uint64_t bd = smem_desc(sbase + Lay::oUB + kk * 2 * Lay::kKGroup,
                                                   Lay::kKGroup, 128, SW_NONE);
-                    mma_bf16(tTS, ad, bd, id_mm, 1);
+                    mma_f16(tTS, ad, bd, id_mm, 1);
                 }
                 mma_commit(&bars[TSFULL]);
                 mma_commit(&bars[EMPTY0 + st]);
@@ -753,10 +788,11 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         sm + Lay::oUB + interleave_mnmajor_off(16 * p + 8, row, Lay::kKGroup)) =
                         pack8(y1);
                 } else if (r < L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(t0 + r) * H + h) * D + j0 +
-                                                           16 * p);
-                    dst[0] = pack8(y0);
-                    dst[1] = pack8(y1);
+                    float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * D + j0 +
+                                                             16 * p);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
                 }
             }
             if (quad < 2) {
@@ -910,7 +946,7 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
     const int grid = a.N * a.H * (tc::D / DVS);
     kern<<<grid, 384, Lay::kBytes, st>>>((const __nv_bfloat16 *)a.v, a.state_in, a.cu_seqlens,
                                          a.T, a.N, a.H, (const uint8_t *)a.workspace,
-                                         (__nv_bfloat16 *)a.o, a.state_out, a.err);
+                                         (float *)a.o, a.state_out, a.err);
     e = cudaGetLastError();
     Profiler::mark(st);
     return e;

@@ -35,7 +35,7 @@ prefill_f32_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                    const Tin *__restrict__ v, const Tin *__restrict__ g,
                    const Tin *__restrict__ beta, const float *state_in,
                    const int32_t *__restrict__ cu_seqlens, int64_t T, int N, int H,
-                   Tin *__restrict__ o, float *state_out) {
+                   float *__restrict__ o, float *state_out) {
     constexpr int NT = 256;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = blockIdx.x / H, h = blockIdx.x % H;
@@ -185,7 +185,7 @@ prefill_f32_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             float acc = 0.f;
             for (int c = 0; c < DK; ++c) acc = fmaf(Qs[r * DK + c], S[c * DV + j], acc);
             for (int s = 0; s <= r; ++s) acc = fmaf(Aqk[r * C + s], Us[s * DV + j], acc);
-            o[((size_t)(t0 + r) * H + h) * DV + j] = from_f32<Tin>(acc);
+            o[((size_t)(t0 + r) * H + h) * DV + j] = acc;
         }
         __syncthreads();
         // 8. S <- Diag(exp G_L) S + Khat^T U
@@ -218,7 +218,7 @@ static cudaError_t launch_f32_t(const PrefillArgs &a, cudaStream_t st) {
     if (grid == 0) return cudaSuccess;
     kern<<<grid, 256, smem, st>>>((const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v,
                                   (const Tin *)a.g, (const Tin *)a.beta, a.state_in,
-                                  a.cu_seqlens, a.T, a.N, a.H, (Tin *)a.o, a.state_out);
+                                  a.cu_seqlens, a.T, a.N, a.H, (float *)a.o, a.state_out);
     e = cudaGetLastError();
     Profiler::mark(st);
     return e;

@@ -30,12 +30,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
     return d;
 }
 
-// kind::f16 instruction descriptor: bf16 x bf16 -> fp32, dense.
-// a_mn / b_mn: 0 = K-major, 1 = MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+// Instruction descriptor, fp32 accumulate, dense.  `fmt` is the A/B element
+// format (A and B always share it): kind::f16 -> 0 = fp16, 1 = bf16;
+// kind::tf32 -> 2 = tf32.  a_mn / b_mn: 0 = K-major, 1 = MN-major.
+enum : uint32_t { FMT_F16 = 0, FMT_BF16 = 1, FMT_TF32 = 2 };
+__host__ __device__ constexpr uint32_t idesc(uint32_t fmt, int M, int N, int a_mn, int b_mn) {
     return (1u << 4)                        // D format: f32
-           | (1u << 7)                      // A format: bf16
-           | (1u << 10)                     // B format: bf16
+           | (fmt << 7)                     // A format
+           | (fmt << 10)                    // B format (same type as A)
            | ((uint32_t)a_mn << 15)         // A major
            | ((uint32_t)b_mn << 16)         // B major
            | ((uint32_t)(N >> 3) << 17)     // N / 8
@@ -71,15 +73,35 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]; single thread issues.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[smem] * B[smem], 16-bit inputs (K = 16 per instruction);
+// single thread issues.  The idesc must name the same 16-bit type for A and B.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t id, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate)
         : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], tf32 inputs stored as 32-bit words
+// (K = 8 per instruction).
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t id, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate)
+        : "memory");
+}
+
+// Round an fp32 value to tf32 (nearest, ties away), low 13 mantissa bits zero.
+__device__ __forceinline__ float to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
 }
 
 // Arrive (once) on an mbarrier when all prior tcgen05 ops of this thread complete.
@@ -158,7 +180,18 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
 
 // ------------------------------------------------------------ smem layouts
 
-// Byte offset of element (row, col) in a K-major, 128-byte-swizzled bf16
+// Byte offset of element (row, col) in a K-major, 128-byte-swizzled 32-bit
+// (tf32) tile whose rows hold 32 elements (one 128-byte line) per K-block;
+// same swizzle rule as below.
+__host__ __device__ __forceinline__ uint32_t sw128_kmajor_off32(uint32_t row, uint32_t col,
+                                                                uint32_t kblock_bytes) {
+    const uint32_t kb = col >> 5, c = col & 31u;
+    const uint32_t chunk = (c >> 2) ^ (row & 7u);
+    return kb * kblock_bytes + (row >> 3) * 1024u + (row & 7u) * 128u + chunk * 16u +
+           (c & 3u) * 4u;
+}
+
+// Byte offset of element (row, col) in a K-major, 128-byte-swizzled 16-bit
 // tile whose rows hold 64 elements (one 128-byte line) per K-block:
 // 8-row groups are 1024 bytes apart, K-blocks `kblock_bytes` apart.
 // The 16-byte chunk index is XOR-ed with (row % 8); the tile base must be
@@ -171,7 +204,7 @@ __host__ __device__ __forceinline__ uint32_t sw128_kmajor_off(uint32_t row, uint
            (c & 7u) * 2u;
 }
 
-// Byte offset of element (mn, k) in an MN-major, 128-byte-swizzled bf16 tile:
+// Byte offset of element (mn, k) in an MN-major, 128-byte-swizzled 16-bit tile:
 // 64 MN-contiguous elements per 128-byte line, k rows 128 bytes apart,
 // 8-row k groups 1024 bytes apart, 64-wide MN blocks `mnblock_bytes` apart.
 __host__ __device__ __forceinline__ uint32_t sw128_mnmajor_off(uint32_t mn, uint32_t k,
@@ -182,7 +215,7 @@ __host__ __device__ __forceinline__ uint32_t sw128_mnmajor_off(uint32_t mn, uint
            (m & 7u) * 2u;
 }
 
-// Byte offset of element (mn, k) in an MN-major tile without swizzle:
+// Byte offset of element (mn, k) in an MN-major 16-bit tile without swizzle:
 // 8x8 core matrices (8 MN elements x 8 k rows, 128 contiguous bytes),
 // MN-adjacent core matrices 128 bytes apart, k-adjacent ones `kgroup_bytes` apart.
 __host__ __device__ __forceinline__ uint32_t interleave_mnmajor_off(uint32_t mn, uint32_t k,

@@ -164,6 +164,39 @@ KDA_API kda_status kda_selftest_bounded_wait(int64_t timeout_us, void *stream);
 KDA_API kda_status kda_profile_enable(int enable);
 KDA_API kda_status kda_profile_last(float *ms, int capacity, int *count);
 
+/*
+ * Prefill without any device allocation, for callers that cannot allocate:
+ * code running in a serving step whose device memory is fully reserved up
+ * front (a cudaMalloc there can fail under memory pressure and synchronises
+ * the device, stalling every stream), or a plugin hosted by a runtime that
+ * owns all allocation and gives it no allocator.  The paper has no
+ * counterpart to this call; it is a property of this library.
+ *
+ * Same arguments and results as kda_chunk_prefill, without the workspace:
+ * the bf16 path's scratch is a fixed array of KDA_STATIC_SCRATCH_BYTES in the
+ * library's own device memory (every GPU that loads libkda holds it until the
+ * process exits).  The caller still passes every input and output.
+ *  - A call whose scratch need, kda_chunk_prefill_workspace_bytes(B*T, N, H,
+ *    dk, dv, dtype), exceeds KDA_STATIC_SCRATCH_BYTES returns
+ *    KDA_ERR_UNSUPPORTED with nothing launched (with H = 32 and d = 128 that
+ *    is about 3.9k packed tokens per call for one sequence).
+ *  - The first call on a device looks up the array's device address (no
+ *    allocation); make that first call before any stream capture.
+ *  - Every call on a device shares the one array, and the array keeps the
+ *    last call's contents (nothing in it needs to start at zero: each call
+ *    writes all the scratch it reads).  Calls whose kernels overlap on the
+ *    GPU (other streams, other threads) race on it: serialise them.
+ *  - The fp32 path needs no scratch and behaves exactly as kda_chunk_prefill.
+ */
+#define KDA_STATIC_SCRATCH_BYTES ((size_t)128 << 20)
+KDA_API kda_status kda_chunk_prefill_static_scratch(const void *q, const void *k, const void *v,
+                                                    const void *g, const void *beta,
+                                                    const float *state_in,
+                                                    const int32_t *cu_seqlens, int B, int64_t T,
+                                                    int N, int H, int dk, int dv,
+                                                    kda_dtype dtype, void *o, float *state_out,
+                                                    void *stream);
+
 /* Static, human-readable name of a status code. */
 KDA_API const char *kda_status_string(kda_status s);
 

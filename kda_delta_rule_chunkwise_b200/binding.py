@@ -30,6 +30,7 @@ EXPORTED = (
     "kda_selftest_bounded_wait",
     "kda_profile_enable",
     "kda_profile_last",
+    "kda_chunk_prefill_static_scratch",
     "kda_status_string",
 )
 
@@ -69,6 +70,9 @@ def load(path: str = LIB_PATH):
     lib.kda_profile_enable.restype = i32
     lib.kda_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32)]
     lib.kda_profile_last.restype = i32
+    lib.kda_chunk_prefill_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
+                                                     i32, i32, i32, i32, vp, vp, vp]
+    lib.kda_chunk_prefill_static_scratch.restype = i32
     lib.kda_status_string.argtypes = [i32]
     lib.kda_status_string.restype = ctypes.c_char_p
     _lib = lib

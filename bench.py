@@ -161,8 +161,8 @@ def run_ours(args, rank, world, dev):
     peaks = measured_peaks()
 
     # ---------------- prefill workload (inputs resident in HBM)
-    w = kin.WORKLOADS[PREFILL_WORKLOAD]
-    d = kin.workload_inputs(PREFILL_WORKLOAD, seed=args.seed + rank, device=dev)
+    w = kin.WORKLOADS[args.workload]
+    d = kin.workload_inputs(args.workload, seed=args.seed + rank, device=dev)
     B, T, H = d.B, d.T, d.H
     tokens = B * T
     o = torch.empty(d.v.shape, dtype=torch.float32, device=dev)
@@ -170,12 +170,24 @@ def run_ours(args, rank, world, dev):
     ws = torch.empty(binding.kda_chunk_prefill_workspace_bytes(tokens, d.N, H, 128, 128,
                                                                 torch.bfloat16),
                      dtype=torch.uint8, device=dev)
-    in_bytes = sum(x.numel() * x.element_size() for x in (d.q, d.k, d.v, d.g, d.beta, d.state_in))
+    in_bytes = sum(x.numel() * x.element_size() for x in (d.q, d.k, d.v, d.g, d.beta, d.state_in)
+                   if x is not None)
 
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+    # clocks are sampled from the timed prefill region through the end of the decode timing
+    clk = ClockSampler(dev.index if dev.index is not None else 0).__enter__()
+    try:
+        return _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, tokens,
+                               o, s_out, ws, in_bytes, clk)
+    finally:
+        clk.__exit__(None, None, None)
+
+
+def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, tokens, o, s_out,
+                    ws, in_bytes, clk):
+    if True:
         ms = time_prefill(binding, d, o, s_out, ws, args.steps, args.warmup)
     torch.cuda.synchronize()
     ms_max = ms
@@ -221,16 +233,17 @@ def run_ours(args, rank, world, dev):
     # ---------------- end to end through the public API, host buffers
     e2e = None
     if args.e2e_steps > 0:
-        pin = lambda x: x.cpu().pin_memory()
+        pin = lambda x: None if x is None else x.cpu().pin_memory()
         hq, hk, hv, hg, hb, hs = (pin(x) for x in (d.q, d.k, d.v, d.g, d.beta, d.state_in))
         ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         hso = torch.empty(s_out.shape, dtype=s_out.dtype, pin_memory=True)
-        dq, dk_, dv_, dg, db, ds = (torch.empty_like(x) for x in (d.q, d.k, d.v, d.g, d.beta,
-                                                                  d.state_in))
+        dq, dk_, dv_, dg, db, ds = (None if x is None else torch.empty_like(x)
+                                    for x in (d.q, d.k, d.v, d.g, d.beta, d.state_in))
 
         def e2e_step():
             for dst, src in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (ds, hs)):
-                dst.copy_(src, non_blocking=True)
+                if dst is not None:
+                    dst.copy_(src, non_blocking=True)
             binding.kda_chunk_prefill(dq, dk_, dv_, dg, db, ds, None, o=o, state_out=s_out,
                                       workspace=ws)
             ho.copy_(o, non_blocking=True)
@@ -263,6 +276,10 @@ def run_ours(args, rank, world, dev):
     torch.cuda.empty_cache()
 
     # ---------------- decode workload
+    decode = None
+    if args.decode_steps <= 0:
+        return finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path,
+                      decode, e2e, clk)
     dw = kin.WORKLOADS[DECODE_WORKLOAD]
     Nd, Hd = dw["N"], dw["H"]
     dec = kin.decode_inputs(args.decode_steps, Nd, Hd, 128, 128, "bf16",
@@ -307,20 +324,25 @@ def run_ours(args, rank, world, dev):
     del dec, pristine, S, od
     torch.cuda.empty_cache()
 
-    launches = args.steps * 3 + args.decode_steps
-    res = {
+    return finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path,
+                  decode, e2e, clk)
+
+
+def finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path, decode,
+           e2e, clk):
+    launches = args.steps * 3 + max(0, args.decode_steps)
+    return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": PREFILL_WORKLOAD, "B": B, "T": T, "H": H, "dk": 128, "dv": 128,
+        "config": {"workload": args.workload, "B": B, "T": T, "H": H, "dk": 128, "dv": 128,
                    "decay": w["decay"], "state": w["state"], "global_batch": B * world,
                    "seq_len": T, "parallelism": f"replicas{world}",
                    "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
         "roofline": roofline, "roofline_path": roofline_path, "decode": decode,
         "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
     }
-    return res
 
 
 # ----------------------------------------------------------------------------- oracle
@@ -397,6 +419,10 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=PREFILL_WORKLOAD,
+                    choices=["prefill_h32_t65536_d128_split", "prefill_h32_t8192_d128",
+                             "varlen_64seq_128to16384_h32_d128"],
+                    help="prefill workload of a step (default: the headline T=65536 one)")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--ref-seconds", type=float, default=15.0,

@@ -180,21 +180,48 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
 // ======================================================================
 // Phase A
 // ======================================================================
+// Decay factors.  With G the chunk-local cumsum and R_a = G at the end of the
+// 16-row block before block a (R_0 = 0), every decay term is built from
+//   E1[r] = exp(G_r - R_a(r))        in [e^-80, 1]   (one exp per element)
+// and per-channel block tables (one exp per channel and block):
+//   ER[a]    = exp(R_a)               Gamma_r          = E1[r] ER[a(r)]
+//   EL[a]    = exp(G_L - R_a)         exp(G_L - G_s)   = EL[a(s)] / E1[s]
+//   PF[a][b] = exp(R_a - R_b), b < a  exp(R_a - G_s)   = PF[a][b(s)] / E1[s]
+// Every product above is of two factors that are each <= 1 or each within
+// [e^-80, e^80], so none of them overflows, and a factor underflows only where
+// the exact value is itself negligible.
+//
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t A_G = 0;            // fp32 [64][128] G (cumsum)              32 KiB
-constexpr uint32_t A_BT = 32768;       // bf16 B tiles [Q'_a; K'_a], 128 rows    32 KiB
-constexpr uint32_t A_AT = 65536;       // bf16 A tiles K^(a), 20 row-groups      40 KiB
-constexpr uint32_t A_ATKB = 20480;     //   bytes between its two K-blocks
-// reused after the Akk/Aqk MMAs have completed:
-constexpr uint32_t A_AK = 32768;       // fp32 [64][64] Akk                      16 KiB
-constexpr uint32_t A_AQ = 49152;       // bf16 Aqk, K-major SW128 64x64            8 KiB
-constexpr uint32_t A_TR = 57344;       // bf16 [T; R], K-major SW128 128x64       16 KiB
-constexpr uint32_t A_KT = 73728;       // bf16 K*exp(G), MN-major SW128           16 KiB
-constexpr uint32_t A_XS = 90112;       // fp32 [64][64] X = (I+Akk)^-1 (+ scratch) 16 KiB
-constexpr uint32_t A_MISC = 106496;    // beta[64], Rref[4][128], GL[128], barriers
-constexpr uint32_t A_SMEM = A_MISC + 4096 + 1024;   // + alignment slack
+constexpr uint32_t A_E1 = 0;          // fp32 [64][128]: G, then E1 in place          32 KiB
+constexpr uint32_t A_MISC = 32768;    // beta, GL, Rref, ER, EL, PF, barriers         10 KiB
+constexpr uint32_t A_OPS = 43008;     // operand region (two uses, below)
+// before the Akk/Aqk MMAs (one 32-channel round at a time, tf32, K-major SW128):
+constexpr uint32_t A_BT = A_OPS;              // [Q'_a; K'_a], 128 rows x 128 B   16 KiB
+constexpr uint32_t A_AT = A_OPS + 16384;      // packed K^(a), 160 rows x 128 B   20 KiB
+// after them:
+constexpr uint32_t A_AK = A_OPS;              // fp32 [64][64] Akk, then X in place 16 KiB
+constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64      8 KiB
+constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64  16 KiB
+constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128       16 KiB
+constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 [16][16] solve scratch          1 KiB
+constexpr uint32_t A_SMEM = A_OPS + 58368 + 1024;   // + alignment slack (= 102400)
 // first row-group of the packed K^(a) tile: 0, 2, 6, 12
 __device__ __forceinline__ int at_group(int a) { return a * (a + 1); }
+// index of the block pair (a, b), b < a, in PF
+__device__ __forceinline__ int pf_index(int a, int b) { return a * (a - 1) / 2 + b; }
+
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
+    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+}
+__device__ __forceinline__ float4 bf4(uint2 u) {   // four bf16 -> fp32
+    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(f0.x, f0.y, f1.x, f1.y);
+}
+__device__ __forceinline__ float4 tf4(float4 a) {
+    return make_float4(to_tf32(a.x), to_tf32(a.y), to_tf32(a.z), to_tf32(a.w));
+}
 
 __global__ void __launch_bounds__(256, 2)
 intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -205,15 +232,18 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(sm);
-    float *Gs = reinterpret_cast<float *>(sm + A_G);
-    float *AK = reinterpret_cast<float *>(sm + A_AK);
-    float *XS = reinterpret_cast<float *>(sm + A_XS);
-    float *bs = reinterpret_cast<float *>(sm + A_MISC);          // [64]
-    float *Rref = bs + 64;                                        // [4][128]
-    float *GL = Rref + 4 * 128;                                   // [128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(GL + 128);      // [4]
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 4);
+    float *E1 = reinterpret_cast<float *>(sm + A_E1);
+    float *bs = reinterpret_cast<float *>(sm + A_MISC);   // [64]
+    float *GL = bs + 64;                                   // [128]
+    float *Rref = GL + 128;                                // [4][128]
+    float *ER = Rref + 4 * 128;                            // [4][128]
+    float *EL = ER + 4 * 128;                              // [4][128]
+    float *PF = EL + 4 * 128;                              // [6][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(PF + 6 * 128);   // [8]
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 8);
     volatile uint32_t *abort_flag = tmem_ptr + 1;
+    float *AK = reinterpret_cast<float *>(sm + A_AK);
+    float *Yb = reinterpret_cast<float *>(sm + A_Y);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y;
@@ -233,6 +263,9 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     const int64_t t0 = ra + (int64_t)(cidx - chunk_off[n]) * C;
     const int L = (int)((rb - t0) < C ? (rb - t0) : C);
     uint8_t *slot = ws + header_bytes(N) + ((size_t)cidx * H + h) * kSlotBytes;
+    auto row_ptr = [&](const __nv_bfloat16 *base, int r) {
+        return base + ((size_t)(t0 + r) * H + h) * D;
+    };
 
     if (warp == 0) {
         tmem_alloc(tmem_ptr, 256);
@@ -240,12 +273,12 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         tc_fence_before();
     }
     if (tid == 32) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
         *abort_flag = 0u;
     }
 
-    // ---- A0: beta and the chunk-local cumsum of the clamped log-decay
+    // ---- A0: beta and the chunk-local cumsum G of the clamped log-decay (fp32)
     if (tid < 64) bs[tid] = tid < L ? __bfloat162float(beta[(size_t)(t0 + tid) * H + h]) : 0.f;
     {
         const int c = tid & 127, half = tid >> 7;
@@ -253,81 +286,96 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int r = half * 32 + i;
-            gv[i] = r < L ? fmaxf(__bfloat162float(g[((size_t)(t0 + r) * H + h) * D + c]), -5.f)
-                          : 0.f;
+            gv[i] = r < L ? fmaxf(__bfloat162float(row_ptr(g, r)[c]), -5.f) : 0.f;
         }
         float acc = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             acc += gv[i];
-            Gs[(half * 32 + i) * D + c] = acc;
+            E1[(half * 32 + i) * D + c] = acc;
         }
     }
     __syncthreads();
     if (tid >= 128) {
         const int c = tid & 127;
-        const float base = Gs[31 * D + c];
-        for (int i = 32; i < 64; ++i) Gs[i * D + c] += base;
+        const float base = E1[31 * D + c];
+        for (int i = 32; i < 64; ++i) E1[i * D + c] += base;
     }
     __syncthreads();
     if (tid < 128) {
         const int c = tid;
-        GL[c] = L > 0 ? Gs[(L - 1) * D + c] : 0.f;
-        Rref[c] = 0.f;
-        Rref[128 + c] = Gs[15 * D + c];
-        Rref[256 + c] = Gs[31 * D + c];
-        Rref[384 + c] = Gs[47 * D + c];
+        const float gl = L > 0 ? E1[(L - 1) * D + c] : 0.f;
+        float rr[4] = {0.f, E1[15 * D + c], E1[31 * D + c], E1[47 * D + c]};
+        GL[c] = gl;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            Rref[a * 128 + c] = rr[a];
+            ER[a * 128 + c] = __expf(rr[a]);
+            EL[a * 128 + c] = __expf(gl - rr[a]);
+        }
+#pragma unroll
+        for (int a = 1; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < a; ++b) PF[pf_index(a, b) * 128 + c] = __expf(rr[a] - rr[b]);
+    }
+    __syncthreads();
+    // E1 in place: exp(G_r - R_a(r)), one row per warp-iteration, float4 per lane
+    for (int r = warp; r < 64; r += 8) {
+        float4 gr = ld4(E1 + r * D + 4 * lane);
+        const float4 rf = ld4(Rref + (r >> 4) * 128 + 4 * lane);
+        gr = make_float4(__expf(gr.x - rf.x), __expf(gr.y - rf.y), __expf(gr.z - rf.z),
+                         __expf(gr.w - rf.w));
+        *reinterpret_cast<float4 *>(E1 + r * D + 4 * lane) = gr;
     }
     __syncthreads();
 
-    // ---- A1: Akk / Aqk on tensor cores, tf32 operands (K-major, 128B swizzle),
-    // accumulated over two 64-channel halves that reuse one operand buffer.
-    // B tiles: row 32a + i      = q_r * exp(G_r - R_a),  r = 16a + i
-    //          row 32a + 16 + i = k_r * exp(G_r - R_a)
-    // A tiles: K^(a) row s (s <= 16a+15) = k_s * exp(R_a - G_s), packed from
-    //          row-group at_group(a)
-    // D^(a) (M=64 rows s, N=32: the 16 q-rows and 16 k-rows of block a) goes to
-    // TMEM columns 32a.
-    const uint32_t tmem_hold = 0;  // (TMEM base read after the first barrier below)
-    (void)tmem_hold;
+    // ---- A1: Akk / Aqk on tensor cores (tf32), four rounds of 32 channels.
+    // B tile row 32a + i      = q_r E1[r]      (r = 16a + i)
+    //        row 32a + 16 + i = k_r E1[r]
+    // A tile (packed from row-group at_group(a)) row s, s <= 16a+15:
+    //        k_s exp(R_a - G_s) = k_s / E1[s]             (s in block a)
+    //                           = k_s PF[a][b(s)] / E1[s]  (s in an earlier block)
+    // D^(a) = K^(a) [Q'_a; K'_a]^T (M=64 rows s, N=32) accumulates in TMEM columns 32a.
+    // Task: (token row r, 4-channel piece p of the round); lane -> (row group, piece).
     bool ok = true;
-    for (int hf = 0; hf < 2; ++hf) {
-        const int c0 = 64 * hf;
+    const int p_l = lane & 7, rsub = lane >> 3;   // 8 pieces x 4 rows per warp
+    for (int rd = 0; rd < 4; ++rd) {
+        const int c0 = 32 * rd + 4 * p_l;
         if (ok) {
-            for (int task = tid; task < 128 * 16; task += 256) {
-                const int row = task >> 4, ch = task & 15;   // ch: 4-channel chunk of this half
-                const int a = row >> 5, isk = (row >> 4) & 1, r = 16 * a + (row & 15);
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            uint2 qv[2], kv[2];
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int r = 32 * it + 4 * warp + rsub;
                 if (r < L) {
-                    const __nv_bfloat16 *src =
-                        (isk ? k : q) + ((size_t)(t0 + r) * H + h) * D + c0 + ch * 4;
-                    const uint2 u = *reinterpret_cast<const uint2 *>(src);
-                    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-                    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-                    const int c = c0 + ch * 4;
-                    const float *gr = Gs + r * D + c, *ra = Rref + a * 128 + c;
-                    x = pack4_tf32(f0.x * __expf(gr[0] - ra[0]), f0.y * __expf(gr[1] - ra[1]),
-                                   f1.x * __expf(gr[2] - ra[2]), f1.y * __expf(gr[3] - ra[3]));
+                    qv[it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(q, r) + c0));
+                    kv[it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(k, r) + c0));
+                } else {
+                    qv[it] = make_uint2(0u, 0u);
+                    kv[it] = make_uint2(0u, 0u);
                 }
-                *reinterpret_cast<float4 *>(sm + A_BT + sw128_kmajor_off32(row, ch * 4, 16384)) = x;
             }
-            for (int task = tid; task < 160 * 16; task += 256) {
-                const int prow = task >> 4, ch = task & 15;
-                int a = 3;
-                if (prow < 16) a = 0; else if (prow < 48) a = 1; else if (prow < 96) a = 2;
-                const int s = prow - at_group(a) * 8;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (s < L) {
-                    const __nv_bfloat16 *src = k + ((size_t)(t0 + s) * H + h) * D + c0 + ch * 4;
-                    const uint2 u = *reinterpret_cast<const uint2 *>(src);
-                    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-                    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-                    const int c = c0 + ch * 4;
-                    const float *gs = Gs + s * D + c, *ra = Rref + a * 128 + c;
-                    x = pack4_tf32(f0.x * __expf(ra[0] - gs[0]), f0.y * __expf(ra[1] - gs[1]),
-                                   f1.x * __expf(ra[2] - gs[2]), f1.y * __expf(ra[3] - gs[3]));
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int r = 32 * it + 4 * warp + rsub;
+                const int a = r >> 4, i = r & 15;
+                const float4 e = ld4(E1 + r * D + c0);
+                const float4 qf = bf4(qv[it]), kf = bf4(kv[it]);
+                const float4 inv = make_float4(__frcp_rn(e.x), __frcp_rn(e.y), __frcp_rn(e.z),
+                                               __frcp_rn(e.w));
+                *reinterpret_cast<float4 *>(sm + A_BT + sw128_kmajor_off32(32 * a + i, 4 * p_l, 0)) =
+                    tf4(mul4(qf, e));
+                *reinterpret_cast<float4 *>(sm + A_BT +
+                                            sw128_kmajor_off32(32 * a + 16 + i, 4 * p_l, 0)) =
+                    tf4(mul4(kf, e));
+                const float4 ki = mul4(kf, inv);
+                *reinterpret_cast<float4 *>(sm + A_AT + sw128_kmajor_off32(8 * at_group(a) + r, 4 * p_l, 0)) =
+                    tf4(ki);
+                for (int a2 = a + 1; a2 < 4; ++a2) {
+                    const float4 pf = ld4(PF + pf_index(a2, a) * 128 + c0);
+                    *reinterpret_cast<float4 *>(
+                        sm + A_AT + sw128_kmajor_off32(8 * at_group(a2) + r, 4 * p_l, 0)) =
+                        tf4(mul4(ki, pf));
                 }
-                *reinterpret_cast<float4 *>(sm + A_AT + sw128_kmajor_off32(prow, ch * 4, A_ATKB)) = x;
             }
         }
         fence_async_smem();
@@ -337,22 +385,23 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             const uint32_t tm = *tmem_ptr;
             const uint32_t id = idesc(FMT_TF32, 64, 32, 0, 0);
             for (int a = 0; a < 4; ++a)
-                for (int kk = 0; kk < 8; ++kk) {          // 8 steps of K=8 over 64 channels
-                    const uint32_t koff = kk >> 2, kin = (kk & 3) * 32;
-                    const uint64_t ad = smem_desc(
-                        sbase + A_AT + at_group(a) * 1024 + koff * A_ATKB + kin, 16, 1024, SW_128B);
-                    const uint64_t bd = smem_desc(sbase + A_BT + (4 * a) * 1024 + koff * 16384 + kin,
-                                                  16, 1024, SW_128B);
-                    mma_tf32(tm + 32 * a, ad, bd, id, (hf > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk) {          // 4 steps of K=8 over 32 channels
+                    const uint64_t ad = smem_desc(sbase + A_AT + at_group(a) * 1024 + kk * 32, 16,
+                                                  1024, SW_128B);
+                    const uint64_t bd = smem_desc(sbase + A_BT + (4 * a) * 1024 + kk * 32, 16,
+                                                  1024, SW_128B);
+                    mma_tf32(tm + 32 * a, ad, bd, id, (rd > 0 || kk > 0) ? 1u : 0u);
                 }
-            mma_commit(&bars[hf]);
+            mma_commit(&bars[rd]);
         }
-        if (ok) ok = mbar_wait_abortable(&bars[hf], 0, err, abort_flag);
+        if (ok) ok = mbar_wait_abortable(&bars[rd], 0, err, abort_flag);
         tc_fence_after();
     }
     const uint32_t tmem = *tmem_ptr;
 
-    // ---- A2: Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal)
+    // ---- A2: Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal,
+    // MN-major: element (r, s) at (s, r) of a 64-wide MN block, so a thread's 16 rows are
+    // 32 contiguous bytes)
     if (ok && warp < 4) {
         const int s = 16 * warp + (lane & 15);
         for (int a = 0; a < 4; ++a) {
@@ -361,87 +410,88 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             tmem_ld16(taddr(tmem, 32 * warp, 32 * a + 16), vk);
             tmem_wait_ld();
             if (lane < 16) {
+                float y0[8], y1[8];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int r = 16 * a + j;
                     AK[r * 64 + s] = (s < r && r < L) ? bs[r] * vk[j] : 0.f;
                     const float aq = (s <= r && r < L) ? vq[j] : 0.f;
-                    reinterpret_cast<__half *>(sm + A_AQ + sw128_kmajor_off(r, s, 0))[0] =
-                        __float2half_rn(aq);
+                    if (j < 8) y0[j] = aq; else y1[j - 8] = aq;
                 }
+                *reinterpret_cast<uint4 *>(sm + A_AQ + sw128_mnmajor_off(16 * a, s, 0)) = pack8(y0);
+                *reinterpret_cast<uint4 *>(sm + A_AQ + sw128_mnmajor_off(16 * a + 8, s, 0)) =
+                    pack8(y1);
             }
         }
     }
-    // K*exp(G) as the MN-major B operand of W = T (K*exp(G)) (region freed by the MMA above)
+    // K*Gamma = k E1 ER as the MN-major B operand of W = T (K*Gamma)
     if (ok && warp >= 4) {
         for (int task = tid - 128; task < 64 * 16; task += 128) {
-            const int s = task >> 4, ch = task & 15;
+            const int s = task >> 4, ch = task & 15, c = ch * 8;
             float x[8];
             if (s < L) {
-                const __nv_bfloat16 *src = k + ((size_t)(t0 + s) * H + h) * D + ch * 8;
-                unpack8(*reinterpret_cast<const uint4 *>(src), x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= __expf(Gs[s * D + ch * 8 + e]);
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + c)), x);
+                const float4 e0 = ld4(E1 + s * D + c), e1 = ld4(E1 + s * D + c + 4);
+                const float4 r0 = ld4(ER + (s >> 4) * 128 + c), r1 = ld4(ER + (s >> 4) * 128 + c + 4);
+                x[0] *= e0.x * r0.x; x[1] *= e0.y * r0.y; x[2] *= e0.z * r0.z; x[3] *= e0.w * r0.w;
+                x[4] *= e1.x * r1.x; x[5] *= e1.y * r1.y; x[6] *= e1.z * r1.z; x[7] *= e1.w * r1.w;
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = 0.f;
             }
-            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(ch * 8, s, kKhMNBlock)) =
-                pack8(x);
+            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(c, s, kKhMNBlock)) = pack8(x);
         }
     }
     tc_fence_before();
     __syncthreads();
 
-    // ---- A3: X = (I + Akk)^-1, blocked over 16x16 blocks, fp32
+    // ---- A3: X = (I + Akk)^-1 in place over AK, blocked over 16x16 blocks, fp32.
     // (every __syncthreads below is reached by all threads, whatever `ok` is)
-    // diagonal blocks by forward substitution: thread (a, j) owns column j of block a
-    if (ok && tid < 64) {
-        const int a = tid >> 4, j = tid & 15, o = 16 * a;
+    // diagonal blocks by forward substitution, thread (a, j) owns column j of block a
+    {
         float x[16];
+        const int a = tid >> 4, j = tid & 15, o = 16 * a;
+        if (ok && tid < 64) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float acc = (i == j) ? 1.f : 0.f;
+            for (int i = 0; i < 16; ++i) {
+                float acc = (i == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int m = 0; m < i; ++m) acc = fmaf(-AK[(o + i) * 64 + o + m], x[m], acc);
-            x[i] = acc;
+                for (int m = 0; m < i; ++m) acc = fmaf(-AK[(o + i) * 64 + o + m], x[m], acc);
+                x[i] = acc;
+            }
         }
+        __syncthreads();
+        if (ok && tid < 64) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) XS[(o + i) * 64 + o + j] = x[i];
+            for (int i = 0; i < 16; ++i) AK[(o + i) * 64 + o + j] = x[i];
+        }
     }
     __syncthreads();
-    // off-diagonal blocks, by distance d = a - b:
-    //   Y_ab = sum_{m=b}^{a-1} A_am X_mb ;  X_ab = -X_aa Y_ab
-    // Y_ab is parked in the (unused) upper-triangular block (b, a) of XS.
-    for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;   // blocks at this distance
-        if (ok) {
-            for (int e = tid; e < nb * 256; e += 256) {
-                const int b = e >> 8, a = b + d, i = (e >> 4) & 15, j = e & 15;
+    // off-diagonal blocks, row by row, b increasing (so A_am, m >= b, is still unmodified):
+    //   Y = sum_{m=b}^{a-1} A_am X_mb ;   X_ab = -X_aa Y  (written over A_ab)
+    for (int a = 1; a < 4; ++a)
+        for (int b = 0; b < a; ++b) {
+            const int i = tid >> 4, j = tid & 15;
+            if (ok) {
                 float acc = 0.f;
                 for (int m = b; m < a; ++m)
 #pragma unroll
                     for (int t = 0; t < 16; ++t)
-                        acc = fmaf(AK[(16 * a + i) * 64 + 16 * m + t],
-                                   XS[(16 * m + t) * 64 + 16 * b + j], acc);
-                XS[(16 * b + i) * 64 + 16 * a + j] = acc;
+                        acc = fmaf(AK[(16 * a + i) * 64 + 16 * m + t], AK[(16 * m + t) * 64 + 16 * b + j],
+                                   acc);
+                Yb[i * 16 + j] = acc;
             }
-        }
-        __syncthreads();
-        if (ok) {
-            for (int e = tid; e < nb * 256; e += 256) {
-                const int b = e >> 8, a = b + d, i = (e >> 4) & 15, j = e & 15;
+            __syncthreads();
+            if (ok) {
                 float acc = 0.f;
 #pragma unroll
                 for (int t = 0; t < 16; ++t)
-                    acc = fmaf(XS[(16 * a + i) * 64 + 16 * a + t],
-                               XS[(16 * b + t) * 64 + 16 * a + j], acc);
-                XS[(16 * a + i) * 64 + 16 * b + j] = -acc;
+                    acc = fmaf(AK[(16 * a + i) * 64 + 16 * a + t], Yb[t * 16 + j], acc);
+                AK[(16 * a + i) * 64 + 16 * b + j] = -acc;
             }
+            __syncthreads();
         }
-        __syncthreads();
-    }
-    // T = X Diag(beta) into rows 0..63 of [T; R] (bf16, K-major SW128)
+    // T = X Diag(beta) into rows 0..63 of [T; R] (fp16, K-major SW128)
     if (ok) {
         for (int task = tid; task < 64 * 8; task += 256) {
             const int r = task >> 3, ch = task & 7;
@@ -449,8 +499,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int s = ch * 8 + e;
-                const float xv = (s == r) ? 1.f : (s < r ? XS[r * 64 + s] : 0.f);
-                x[e] = xv * bs[s];
+                x[e] = (s <= r) ? AK[r * 64 + s] * bs[s] : 0.f;
             }
             *reinterpret_cast<uint4 *>(sm + A_TR + sw128_kmajor_off(r, ch * 8, 0)) = pack8(x);
         }
@@ -459,17 +508,17 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
     tc_fence_after();
 
-    // ---- A4: R = Aqk T  (M=64, N=64, K=64) into TMEM columns 128..191
+    // ---- A4: R = Aqk T  (M=64, N=64, K=64; A MN-major, B MN-major) into TMEM columns 128..191
     if (ok && tid == 0) {
-        const uint32_t id = idesc(FMT_F16, 64, 64, 0, 1);
+        const uint32_t id = idesc(FMT_F16, 64, 64, 1, 1);
         for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc(sbase + A_AQ + kk * 32, 16, 1024, SW_128B);
+            const uint64_t ad = smem_desc(sbase + A_AQ + kk * 2048, 8192, 1024, SW_128B);
             const uint64_t bd = smem_desc(sbase + A_TR + kk * 2048, 8192, 1024, SW_128B);
             mma_f16(tmem + 128, ad, bd, id, kk > 0);
         }
-        mma_commit(&bars[2]);
+        mma_commit(&bars[4]);
     }
-    if (ok) ok = mbar_wait_abortable(&bars[2], 0, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[4], 0, err, abort_flag);
     tc_fence_after();
     if (ok && warp < 4) {
         const int r = 16 * warp + (lane & 15);
@@ -495,7 +544,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
     tc_fence_after();
 
-    // ---- A5: D1 = [T; R] (K*exp(G))  (M=128, N=128, K=64) into TMEM columns 0..127
+    // ---- A5: D1 = [T; R] (K*Gamma)  (M=128, N=128, K=64) into TMEM columns 0..127
     if (ok && tid == 0) {
         const uint32_t id = idesc(FMT_F16, 128, 128, 0, 1);
         for (int kk = 0; kk < 4; ++kk) {
@@ -503,69 +552,61 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             const uint64_t bd = smem_desc(sbase + A_KT + kk * 2048, kKhMNBlock, 1024, SW_128B);
             mma_f16(tmem, ad, bd, id, kk > 0);
         }
-        mma_commit(&bars[3]);
+        mma_commit(&bars[5]);
     }
-    // [T; R] is final: copy it to the slot while the MMA runs (reads only)
+    // [T; R] is final: copy it to the slot while the MMA runs (reads only);
+    // Khat = k EL / E1 and Gamma_L straight to the slot
     if (ok) {
         const uint4 *src = reinterpret_cast<const uint4 *>(sm + A_TR);
         uint4 *dst = reinterpret_cast<uint4 *>(slot + kSlotTR);
         for (int i = tid; i < 16384 / 16; i += 256) dst[i] = src[i];
-        // Khat and Gamma_L straight to the slot
         for (int task = tid; task < 64 * 16; task += 256) {
-            const int s = task >> 4, ch = task & 15;
+            const int s = task >> 4, ch = task & 15, c = ch * 8;
             float x[8];
             if (s < L) {
-                const __nv_bfloat16 *srck = k + ((size_t)(t0 + s) * H + h) * D + ch * 8;
-                unpack8(*reinterpret_cast<const uint4 *>(srck), x);
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + c)), x);
+                const float *e1 = E1 + s * D + c, *el = EL + (s >> 4) * 128 + c;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int c = ch * 8 + e;
-                    x[e] *= __expf(GL[c] - Gs[s * D + c]);
-                }
+                for (int e = 0; e < 8; ++e) x[e] *= el[e] * __frcp_rn(e1[e]);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = 0.f;
             }
-            *reinterpret_cast<uint4 *>(slot + kSlotKh + sw128_mnmajor_off(ch * 8, s, kKhMNBlock)) =
+            *reinterpret_cast<uint4 *>(slot + kSlotKh + sw128_mnmajor_off(c, s, kKhMNBlock)) =
                 pack8(x);
         }
         if (tid < 128) reinterpret_cast<float *>(slot + kSlotGam)[tid] = __expf(GL[tid]);
     }
-    if (ok) ok = mbar_wait_abortable(&bars[3], 0, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[5], 0, err, abort_flag);
     tc_fence_after();
 
-    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = Q*exp(G) - R (K*exp(G))
+    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = q E1 ER - R (K*Gamma)
     if (ok) {
         const int quad = warp & 3, chalf = warp >> 2;
         const int row = 32 * quad + lane;
+        const int r = row & 63;
         float x[64];
 #pragma unroll
         for (int p = 0; p < 4; ++p)
             tmem_ld16(taddr(tmem, 32 * quad, 64 * chalf + 16 * p),
                       *reinterpret_cast<float(*)[16]>(x + 16 * p));
         tmem_wait_ld();
-        const int r = row & 63;
         if (row < 64) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) x[i] = -x[i];
-        } else {
-            if (r < L) {
+        } else if (r < L) {
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float qv[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(
-                                q + ((size_t)(t0 + r) * H + h) * D + 64 * chalf + ch * 8),
-                            qv);
+            for (int ch = 0; ch < 8; ++ch) {
+                const int c = 64 * chalf + ch * 8;
+                float qv[8];
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(row_ptr(q, r) + c)), qv);
+                const float *e1 = E1 + r * D + c, *er = ER + (r >> 4) * 128 + c;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int c = 64 * chalf + ch * 8 + e;
-                        x[ch * 8 + e] = qv[e] * __expf(Gs[r * D + c]) - x[ch * 8 + e];
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = 0.f;
+                for (int e = 0; e < 8; ++e) x[ch * 8 + e] = qv[e] * e1[e] * er[e] - x[ch * 8 + e];
             }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) x[i] = 0.f;
         }
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -681,23 +722,25 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             }
             const int64_t t0 = ra + (int64_t)j * C;
             const int L = (int)((rb - t0) < C ? (rb - t0) : C);
-            // V slice -> fp16 MMA operand (MN-major, interleaved core matrices);
-            // rows past the end of the sequence are zero
+            // V slice -> fp16 MMA operand (MN-major, interleaved core matrices).
+            // All 16-byte pieces are fetched asynchronously straight into their
+            // operand positions (rows past the end of the sequence zero-filled),
+            // then each lane converts the pieces it fetched from bf16 to fp16 in place.
             uint8_t *vt = stg + kSlotBytes;
-            constexpr int CPR = DVS / 8;   // 16-byte chunks per row
+            constexpr int CPR = DVS / 8;   // 16-byte pieces per row
             for (int task = lane; task < 64 * CPR; task += 32) {
                 const int r = task / CPR, ch = task % CPR;
+                const int rr = r < L ? r : 0;
+                cp_async16(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup),
+                           v + ((size_t)(t0 + rr) * H + h) * D + j0 + ch * 8, r < L ? 16u : 0u);
+            }
+            cp_async_wait_all();
+            for (int task = lane; task < 64 * CPR; task += 32) {
+                const int r = task / CPR, ch = task % CPR;
+                uint4 *pc = reinterpret_cast<uint4 *>(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup));
                 float x[8];
-                if (r < L) {
-                    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
-                        v + ((size_t)(t0 + r) * H + h) * D + j0 + ch * 8));
-                    unpack8(u, x);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = 0.f;
-                }
-                *reinterpret_cast<uint4 *>(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup)) =
-                    pack8(x);
+                unpack8(*pc, x);
+                *pc = pack8(x);
             }
             fence_async_smem();
             mbar_arrive(&bars[FULL0 + st]);

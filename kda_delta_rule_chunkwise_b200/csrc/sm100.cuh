@@ -172,6 +172,11 @@ __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src, uint
                  : "memory");
 }
 
+// Wait until all of this thread's prior cp.async copies have landed.
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // The mbarrier receives one arrival when all prior cp.async of this thread land.
 __device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))

@@ -31,9 +31,11 @@
 // O = Q*exp(G) S + Aqk U, the chunk's outputs.
 //
 // Roles in phase B: warp 0 = producer (1-D bulk copy of the slot, V slice
-// converted to fp16), warp 1 = MMA issuer and TMEM owner, warps 4-7 = U/O
-// epilogue (TMEM -> registers), warps 8-11 = state epilogue (Gamma scaling
-// of the TMEM state, fp16 copy of S for the next chunk's MMA).
+// converted to fp16), warp 1 = TMEM owner, warps 4-7 = U/O epilogue (TMEM ->
+// registers; its elected thread issues the state update), warps 8-11 = state
+// epilogue (Gamma scaling of the TMEM state, fp16 copy of S; its elected
+// thread issues the chunk products).  Each chunk costs two hand-offs: state
+// copy -> chunk products -> U copy -> state update -> state copy.
 //
 // Precision.  Inputs are bf16; every product accumulates in fp32 (TMEM); the
 // state and the outputs o are fp32.  The decay-rescaled operands of Akk/Aqk
@@ -182,33 +184,48 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
 // ======================================================================
 // Decay factors.  With G the chunk-local cumsum and R_a = G at the end of the
 // 16-row block before block a (R_0 = 0), every decay term is built from
-//   E1[r] = exp(G_r - R_a(r))        in [e^-80, 1]   (one exp per element)
-// and per-channel block tables (one exp per channel and block):
-//   ER[a]    = exp(R_a)               Gamma_r          = E1[r] ER[a(r)]
-//   EL[a]    = exp(G_L - R_a)         exp(G_L - G_s)   = EL[a(s)] / E1[s]
-//   PF[a][b] = exp(R_a - R_b), b < a  exp(R_a - G_s)   = PF[a][b(s)] / E1[s]
-// Every product above is of two factors that are each <= 1 or each within
-// [e^-80, e^80], so none of them overflows, and a factor underflows only where
-// the exact value is itself negligible.
+//   E1[r] = exp(G_r - R_a(r))    in [e^-80, 1]   (one exp per element)
+// and per-channel block factors
+//   F_m   = exp(R_{m+1} - R_m)   (the decay of block m, <= 1), m = 0, 1, 2
+//   EL[a] = exp(G_L - R_a)       (<= 1 for every block holding a valid row)
+// as
+//   Gamma_r         = E1[r] * prod_{m < a(r)} F_m
+//   exp(G_L - G_s)  = EL[a(s)] / E1[s]
+//   exp(R_a - G_s)  = (prod_{m = b(s)}^{a-1} F_m) / E1[s]       (a >= b(s))
+// Each product is of factors that are all <= 1, or of one factor <= 1 and
+// 1/E1 <= e^80 whose product is <= 1, so nothing overflows, and a factor
+// underflows only where the exact value is itself negligible.
 //
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t A_E1 = 0;          // fp32 [64][128]: G, then E1 in place          32 KiB
-constexpr uint32_t A_MISC = 32768;    // beta, GL, Rref, ER, EL, PF, barriers         10 KiB
-constexpr uint32_t A_OPS = 43008;     // operand region (two uses, below)
-// before the Akk/Aqk MMAs (one 32-channel round at a time, tf32, K-major SW128):
-constexpr uint32_t A_BT = A_OPS;              // [Q'_a; K'_a], 128 rows x 128 B   16 KiB
-constexpr uint32_t A_AT = A_OPS + 16384;      // packed K^(a), 160 rows x 128 B   20 KiB
+constexpr uint32_t A_E1 = 0;          // fp32 [64][128] E1                           32 KiB
+constexpr uint32_t A_MISC = 32768;    // beta, F, EL, Gamma_L, barriers, TMEM address  5 KiB
+constexpr uint32_t A_M_BETA = 0;      //   fp32 [64]
+constexpr uint32_t A_M_F = 256;       //   fp32 [3][128]
+constexpr uint32_t A_M_EL = 1792;     //   fp32 [4][128]
+constexpr uint32_t A_M_GAML = 3840;   //   fp32 [128]
+constexpr uint32_t A_M_BARS = 4352;   //   8 mbarriers
+constexpr uint32_t A_M_TMEM = 4416;   //   TMEM base address + abort flag
+constexpr uint32_t A_M_END = 4424;
+constexpr uint32_t A_OPS = 37888;     // operand region (two uses, below)
+static_assert(A_MISC + A_M_END <= A_OPS, "phase A misc region overflows into the operands");
+static_assert(A_M_BARS % 8 == 0 && A_M_F % 16 == 0 && A_M_EL % 16 == 0, "misc alignment");
+// before the Akk/Aqk MMAs: two buffers of one 32-channel round (tf32, K-major SW128)
+constexpr uint32_t A_RBUF = 36864;            // bytes per round buffer
+constexpr uint32_t A_BT = 0;                  //   + [Q'_a; K'_a], 128 rows x 128 B    16 KiB
+constexpr uint32_t A_AT = 16384;              //   + packed K^(a), 160 rows x 128 B    20 KiB
 // after them:
-constexpr uint32_t A_AK = A_OPS;              // fp32 [64][64] Akk, then X in place 16 KiB
-constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64      8 KiB
-constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64  16 KiB
-constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128       16 KiB
-constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 [16][16] solve scratch          1 KiB
-constexpr uint32_t A_SMEM = A_OPS + 58368 + 1024;   // + alignment slack (= 102400)
+constexpr uint32_t A_AK = A_OPS;              // fp32 [64][64] Akk, then X in place    16 KiB
+constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64         8 KiB
+constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64     16 KiB
+constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128          16 KiB
+constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 solve scratch (32 x 32)               4 KiB
+constexpr uint32_t A_SMEM = A_OPS + 2 * A_RBUF + 1024;   // + alignment slack (= 112640)
+static_assert(A_Y + 4096 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
+static_assert(A_OPS + 4096 + 16384 <= A_OPS + A_RBUF, "g staging must fit in round buffer 0");
+static_assert(A_OPS % 1024 == 0 && A_RBUF % 1024 == 0 && A_AQ % 1024 == 0 && A_TR % 1024 == 0 &&
+              A_KT % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // first row-group of the packed K^(a) tile: 0, 2, 6, 12
 __device__ __forceinline__ int at_group(int a) { return a * (a + 1); }
-// index of the block pair (a, b), b < a, in PF
-__device__ __forceinline__ int pf_index(int a, int b) { return a * (a - 1) / 2 + b; }
 
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) {
@@ -219,8 +236,22 @@ __device__ __forceinline__ float4 bf4(uint2 u) {   // four bf16 -> fp32
     const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
     return make_float4(f0.x, f0.y, f1.x, f1.y);
 }
+// round to tf32 (nearest, ties away from zero) with integer ops: add half an ulp
+// of the 10-bit significand, clear the 13 low bits (finite inputs only)
+__device__ __forceinline__ float tf32r(float x) {
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
 __device__ __forceinline__ float4 tf4(float4 a) {
-    return make_float4(to_tf32(a.x), to_tf32(a.y), to_tf32(a.z), to_tf32(a.w));
+    return make_float4(tf32r(a.x), tf32r(a.y), tf32r(a.z), tf32r(a.w));
+}
+// approximate reciprocal (about 1 ulp): enough for operands rounded to tf32/fp16 next
+__device__ __forceinline__ float rcpa(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float4 rcp4(float4 a) {
+    return make_float4(rcpa(a.x), rcpa(a.y), rcpa(a.z), rcpa(a.w));
 }
 
 __global__ void __launch_bounds__(256, 2)
@@ -233,15 +264,16 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(sm);
     float *E1 = reinterpret_cast<float *>(sm + A_E1);
-    float *bs = reinterpret_cast<float *>(sm + A_MISC);   // [64]
-    float *GL = bs + 64;                                   // [128]
-    float *Rref = GL + 128;                                // [4][128]
-    float *ER = Rref + 4 * 128;                            // [4][128]
-    float *EL = ER + 4 * 128;                              // [4][128]
-    float *PF = EL + 4 * 128;                              // [6][128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(PF + 6 * 128);   // [8]
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 8);
+    float *bs = reinterpret_cast<float *>(sm + A_MISC + A_M_BETA);    // [64]
+    float *Fb = reinterpret_cast<float *>(sm + A_MISC + A_M_F);       // [3][128] block decays F_m
+    float *EL = reinterpret_cast<float *>(sm + A_MISC + A_M_EL);      // [4][128]
+    float *GamL = reinterpret_cast<float *>(sm + A_MISC + A_M_GAML);  // [128] exp(G_L)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + A_MISC + A_M_BARS);   // [8]
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + A_MISC + A_M_TMEM);
     volatile uint32_t *abort_flag = tmem_ptr + 1;
+    // used only inside A0, before any operand round: parked in the operand region
+    float *tot = reinterpret_cast<float *>(sm + A_OPS);              // [3][128] half sums
+    float *GLv = tot + 3 * 128;                                       // [128] G_L
     float *AK = reinterpret_cast<float *>(sm + A_AK);
     float *Yb = reinterpret_cast<float *>(sm + A_Y);
 
@@ -249,23 +281,73 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     const int h = blockIdx.y;
     const int32_t *chunk_off = reinterpret_cast<const int32_t *>(ws);
     const int cidx = blockIdx.x;
-    const int total = chunk_off[N];
-    if (cidx >= total) return;
-    // sequence owning this chunk: last n with chunk_off[n] <= cidx
-    int lo = 0, hi = N - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (chunk_off[mid] <= cidx) lo = mid; else hi = mid - 1;
+    int64_t t0;
+    int L;
+    if (cu == nullptr) {
+        // equal-length batch: chunk -> (sequence, start) by arithmetic, no table read
+        const int64_t cps = (T + C - 1) / C;
+        const int64_t n = cidx / cps, j = cidx - n * cps;
+        if (n >= N) return;
+        t0 = n * T + j * C;
+        L = (int)((T - j * C) < C ? (T - j * C) : C);
+    } else {
+        const int total = chunk_off[N];
+        if (cidx >= total) return;
+        // sequence owning this chunk: last n with chunk_off[n] <= cidx
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (chunk_off[mid] <= cidx) lo = mid; else hi = mid - 1;
+        }
+        int64_t ra, rb;
+        seq_rows(chunk_off, true, T, N, lo, ra, rb);
+        t0 = ra + (int64_t)(cidx - chunk_off[lo]) * C;
+        L = (int)((rb - t0) < C ? (rb - t0) : C);
     }
-    const int n = lo;
-    int64_t ra, rb;
-    seq_rows(chunk_off, cu != nullptr, T, N, n, ra, rb);
-    const int64_t t0 = ra + (int64_t)(cidx - chunk_off[n]) * C;
-    const int L = (int)((rb - t0) < C ? (rb - t0) : C);
     uint8_t *slot = ws + header_bytes(N) + ((size_t)cidx * H + h) * kSlotBytes;
     auto row_ptr = [&](const __nv_bfloat16 *base, int r) {
         return base + ((size_t)(t0 + r) * H + h) * D;
     };
+
+    // ---- issue every global load of the operand rounds up front (one round trip)
+    // round task: lane -> 4-channel piece p_l of the round, token rows 32*it + 4*warp + rsub
+    const int p_l = lane & 7, rsub = lane >> 3;
+    uint2 qv[4][2], kv[4][2];
+#pragma unroll
+    for (int rd = 0; rd < 4; ++rd)
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const int r = 32 * it + 4 * warp + rsub;
+            const int c0 = 32 * rd + 4 * p_l;
+            if (r < L) {
+                qv[rd][it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(q, r) + c0));
+                kv[rd][it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(k, r) + c0));
+            } else {
+                qv[rd][it] = make_uint2(0u, 0u);
+                kv[rd][it] = make_uint2(0u, 0u);
+            }
+        }
+    // g: coalesced 16-byte loads, staged as bf16 [64][128] in the (still idle) operand region
+    uint4 gv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int task = tid + 256 * i, r = task >> 4, cc = (task & 15) * 8;
+        gv[i] = r < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(g, r) + cc))
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const float bval = (tid < L) ? __bfloat162float(beta[(size_t)(t0 + (tid < 64 ? tid : 0)) * H + h]) : 0.f;
+    __nv_bfloat16 *gst = reinterpret_cast<__nv_bfloat16 *>(sm + A_OPS + 4096);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int task = tid + 256 * i;
+        reinterpret_cast<uint4 *>(gst)[task] = gv[i];
+    }
+    if (tid < 64) bs[tid] = bval;
+    __syncthreads();
+    const int c = tid & 127, half = tid >> 7;
+    float p[32];   // clamped log-decay of rows 32*half + i, then its prefix sums
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = fmaxf(__bfloat162float(gst[(half * 32 + i) * D + c]), -5.f);
 
     if (warp == 0) {
         tmem_alloc(tmem_ptr, 256);
@@ -278,103 +360,80 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         *abort_flag = 0u;
     }
 
-    // ---- A0: beta and the chunk-local cumsum G of the clamped log-decay (fp32)
-    if (tid < 64) bs[tid] = tid < L ? __bfloat162float(beta[(size_t)(t0 + tid) * H + h]) : 0.f;
-    {
-        const int c = tid & 127, half = tid >> 7;
-        float gv[32];
+    // ---- A0: chunk-local cumsum (fp32) and E1 = exp(G - R_a), per channel c and half
+    // G_r - R_a(r) = p_i for the first 16 rows of a half and p_i - p_15 for the
+    // last 16 (R of the half's first block is the base the half starts from).
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = half * 32 + i;
-            gv[i] = r < L ? fmaxf(__bfloat162float(row_ptr(g, r)[c]), -5.f) : 0.f;
-        }
-        float acc = 0.f;
+    for (int i = 1; i < 32; ++i) p[i] += p[i - 1];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            acc += gv[i];
-            E1[(half * 32 + i) * D + c] = acc;
-        }
+    for (int i = 0; i < 32; ++i) {
+        const float x = i < 16 ? p[i] : p[i] - p[15];
+        E1[(half * 32 + i) * D + c] = __expf(x);
+    }
+    if (half == 0) {
+        tot[c] = p[31];
+        tot[128 + c] = p[15];
+        Fb[c] = __expf(p[15]);                 // F_0
+        Fb[128 + c] = __expf(p[31] - p[15]);   // F_1
+    } else {
+        tot[256 + c] = p[15];
+        Fb[256 + c] = __expf(p[15]);           // F_2
     }
     __syncthreads();
-    if (tid >= 128) {
-        const int c = tid & 127;
-        const float base = E1[31 * D + c];
-        for (int i = 32; i < 64; ++i) E1[i * D + c] += base;
+    {
+        // G_L: the owner half of row L-1 writes it
+        const int lr = L - 1;
+        if (lr >= 0 && (lr >> 5) == half) {
+            const float base = half ? tot[c] : 0.f;
+            float v = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (i == (lr & 31)) v = p[i];
+            GLv[c] = base + v;
+        }
+        if (L <= 0 && half == 0) GLv[c] = 0.f;
     }
     __syncthreads();
     if (tid < 128) {
-        const int c = tid;
-        const float gl = L > 0 ? E1[(L - 1) * D + c] : 0.f;
-        float rr[4] = {0.f, E1[15 * D + c], E1[31 * D + c], E1[47 * D + c]};
-        GL[c] = gl;
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            Rref[a * 128 + c] = rr[a];
-            ER[a * 128 + c] = __expf(rr[a]);
-            EL[a * 128 + c] = __expf(gl - rr[a]);
-        }
-#pragma unroll
-        for (int a = 1; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < a; ++b) PF[pf_index(a, b) * 128 + c] = __expf(rr[a] - rr[b]);
-    }
-    __syncthreads();
-    // E1 in place: exp(G_r - R_a(r)), one row per warp-iteration, float4 per lane
-    for (int r = warp; r < 64; r += 8) {
-        float4 gr = ld4(E1 + r * D + 4 * lane);
-        const float4 rf = ld4(Rref + (r >> 4) * 128 + 4 * lane);
-        gr = make_float4(__expf(gr.x - rf.x), __expf(gr.y - rf.y), __expf(gr.z - rf.z),
-                         __expf(gr.w - rf.w));
-        *reinterpret_cast<float4 *>(E1 + r * D + 4 * lane) = gr;
+        const float gl = GLv[c];
+        const float r1 = tot[128 + c], r2 = tot[c], r3 = tot[c] + tot[256 + c];
+        EL[c] = __expf(gl);
+        EL[128 + c] = __expf(gl - r1);
+        EL[256 + c] = __expf(gl - r2);
+        EL[384 + c] = __expf(gl - r3);
+        GamL[c] = __expf(gl);
     }
     __syncthreads();
 
-    // ---- A1: Akk / Aqk on tensor cores (tf32), four rounds of 32 channels.
+    // ---- A1: Akk / Aqk on tensor cores (tf32), four double-buffered rounds of 32 channels.
     // B tile row 32a + i      = q_r E1[r]      (r = 16a + i)
     //        row 32a + 16 + i = k_r E1[r]
     // A tile (packed from row-group at_group(a)) row s, s <= 16a+15:
-    //        k_s exp(R_a - G_s) = k_s / E1[s]             (s in block a)
-    //                           = k_s PF[a][b(s)] / E1[s]  (s in an earlier block)
+    //        k_s exp(R_a - G_s) = k_s (prod_{m=b(s)}^{a-1} F_m) / E1[s]
     // D^(a) = K^(a) [Q'_a; K'_a]^T (M=64 rows s, N=32) accumulates in TMEM columns 32a.
-    // Task: (token row r, 4-channel piece p of the round); lane -> (row group, piece).
     bool ok = true;
-    const int p_l = lane & 7, rsub = lane >> 3;   // 8 pieces x 4 rows per warp
-    for (int rd = 0; rd < 4; ++rd) {
-        const int c0 = 32 * rd + 4 * p_l;
-        if (ok) {
-            uint2 qv[2], kv[2];
 #pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int r = 32 * it + 4 * warp + rsub;
-                if (r < L) {
-                    qv[it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(q, r) + c0));
-                    kv[it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(k, r) + c0));
-                } else {
-                    qv[it] = make_uint2(0u, 0u);
-                    kv[it] = make_uint2(0u, 0u);
-                }
-            }
+    for (int rd = 0; rd < 4; ++rd) {
+        const uint32_t buf = A_OPS + (rd & 1) * A_RBUF;
+        if (rd >= 2 && ok) ok = mbar_wait_abortable(&bars[rd - 2], 0, err, abort_flag);
+        if (ok) {
+            const int c0 = 32 * rd + 4 * p_l;
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const int r = 32 * it + 4 * warp + rsub;
                 const int a = r >> 4, i = r & 15;
+                // every row this task writes is congruent to r mod 8: one swizzled chunk offset
+                const uint32_t co = (r & 7) * 128 + ((p_l ^ (r & 7)) << 4);
+                uint8_t *bt = sm + buf + A_BT + co, *at = sm + buf + A_AT + co;
                 const float4 e = ld4(E1 + r * D + c0);
-                const float4 qf = bf4(qv[it]), kf = bf4(kv[it]);
-                const float4 inv = make_float4(__frcp_rn(e.x), __frcp_rn(e.y), __frcp_rn(e.z),
-                                               __frcp_rn(e.w));
-                *reinterpret_cast<float4 *>(sm + A_BT + sw128_kmajor_off32(32 * a + i, 4 * p_l, 0)) =
-                    tf4(mul4(qf, e));
-                *reinterpret_cast<float4 *>(sm + A_BT +
-                                            sw128_kmajor_off32(32 * a + 16 + i, 4 * p_l, 0)) =
-                    tf4(mul4(kf, e));
-                const float4 ki = mul4(kf, inv);
-                *reinterpret_cast<float4 *>(sm + A_AT + sw128_kmajor_off32(8 * at_group(a) + r, 4 * p_l, 0)) =
-                    tf4(ki);
+                const float4 qf = bf4(qv[rd][it]), kf = bf4(kv[rd][it]);
+                *reinterpret_cast<float4 *>(bt + ((32 * a + i) >> 3) * 1024) = tf4(mul4(qf, e));
+                *reinterpret_cast<float4 *>(bt + ((32 * a + 16 + i) >> 3) * 1024) = tf4(mul4(kf, e));
+                float4 ki = mul4(kf, rcp4(e));
+                *reinterpret_cast<float4 *>(at + ((8 * at_group(a) + r) >> 3) * 1024) = tf4(ki);
                 for (int a2 = a + 1; a2 < 4; ++a2) {
-                    const float4 pf = ld4(PF + pf_index(a2, a) * 128 + c0);
-                    *reinterpret_cast<float4 *>(
-                        sm + A_AT + sw128_kmajor_off32(8 * at_group(a2) + r, 4 * p_l, 0)) =
-                        tf4(mul4(ki, pf));
+                    ki = mul4(ki, ld4(Fb + (a2 - 1) * 128 + c0));
+                    *reinterpret_cast<float4 *>(at + ((8 * at_group(a2) + r) >> 3) * 1024) = tf4(ki);
                 }
             }
         }
@@ -386,22 +445,31 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             const uint32_t id = idesc(FMT_TF32, 64, 32, 0, 0);
             for (int a = 0; a < 4; ++a)
                 for (int kk = 0; kk < 4; ++kk) {          // 4 steps of K=8 over 32 channels
-                    const uint64_t ad = smem_desc(sbase + A_AT + at_group(a) * 1024 + kk * 32, 16,
-                                                  1024, SW_128B);
-                    const uint64_t bd = smem_desc(sbase + A_BT + (4 * a) * 1024 + kk * 32, 16,
+                    const uint64_t ad = smem_desc(sbase + buf + A_AT + at_group(a) * 1024 + kk * 32,
+                                                  16, 1024, SW_128B);
+                    const uint64_t bd = smem_desc(sbase + buf + A_BT + (4 * a) * 1024 + kk * 32, 16,
                                                   1024, SW_128B);
                     mma_tf32(tm + 32 * a, ad, bd, id, (rd > 0 || kk > 0) ? 1u : 0u);
                 }
             mma_commit(&bars[rd]);
         }
-        if (ok) ok = mbar_wait_abortable(&bars[rd], 0, err, abort_flag);
-        tc_fence_after();
     }
+    // next loads (K*Gamma operand, warps 4-7) go out before the last MMA wait
+    uint4 kt_pref[8];
+    if (warp >= 4) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int task = (tid - 128) + 128 * i, s = task >> 4, cc = (task & 15) * 8;
+            kt_pref[i] = s < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
+                               : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    if (ok) ok = mbar_wait_abortable(&bars[3], 0, err, abort_flag);
+    tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
 
     // ---- A2: Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal,
-    // MN-major: element (r, s) at (s, r) of a 64-wide MN block, so a thread's 16 rows are
-    // 32 contiguous bytes)
+    // MN-major: element (r, s) at (mn = r, k = s), so a thread's 16 rows are 32 contiguous bytes)
     if (ok && warp < 4) {
         const int s = 16 * warp + (lane & 15);
         for (int a = 0; a < 4; ++a) {
@@ -424,30 +492,40 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
         }
     }
-    // K*Gamma = k E1 ER as the MN-major B operand of W = T (K*Gamma)
+    // K*Gamma = k E1 prod_{m<a} F_m as the MN-major B operand of W = T (K*Gamma)
     if (ok && warp >= 4) {
-        for (int task = tid - 128; task < 64 * 16; task += 128) {
-            const int s = task >> 4, ch = task & 15, c = ch * 8;
-            float x[8];
-            if (s < L) {
-                unpack8(__ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + c)), x);
-                const float4 e0 = ld4(E1 + s * D + c), e1 = ld4(E1 + s * D + c + 4);
-                const float4 r0 = ld4(ER + (s >> 4) * 128 + c), r1 = ld4(ER + (s >> 4) * 128 + c + 4);
-                x[0] *= e0.x * r0.x; x[1] *= e0.y * r0.y; x[2] *= e0.z * r0.z; x[3] *= e0.w * r0.w;
-                x[4] *= e1.x * r1.x; x[5] *= e1.y * r1.y; x[6] *= e1.z * r1.z; x[7] *= e1.w * r1.w;
-            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        for (int i = 0; i < 8; ++i) {
+            const int task = (tid - 128) + 128 * i, s = task >> 4, cc = (task & 15) * 8;
+            float x[8];
+            unpack8(kt_pref[i], x);
+            const int a = s >> 4;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+                float4 e = ld4(E1 + s * D + cc + 4 * hv);
+                for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
+                x[4 * hv] *= e.x; x[4 * hv + 1] *= e.y; x[4 * hv + 2] *= e.z; x[4 * hv + 3] *= e.w;
             }
-            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(c, s, kKhMNBlock)) = pack8(x);
+            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(cc, s, kKhMNBlock)) = pack8(x);
         }
     }
     tc_fence_before();
     __syncthreads();
 
-    // ---- A3: X = (I + Akk)^-1 in place over AK, blocked over 16x16 blocks, fp32.
-    // (every __syncthreads below is reached by all threads, whatever `ok` is)
-    // diagonal blocks by forward substitution, thread (a, j) owns column j of block a
+    // Khat loads for A5 go out now; the solve below hides their latency
+    uint4 kh_pref[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
+        kh_pref[i] = s < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
+                           : make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    // ---- A3: X = (I + Akk)^-1 in place over AK (fp32), by 2x2 block merges:
+    //   inv([[L11, 0], [L21, L22]]) = [[X11, 0], [-X22 (L21 X11), X22]]
+    // 16x16 diagonal blocks by forward substitution, then two merges 16 -> 32
+    // (in parallel), then one merge 32 -> 64.  The strictly upper part of AK is
+    // zero throughout.  (Every __syncthreads below is reached by all threads.)
     {
         float x[16];
         const int a = tid >> 4, j = tid & 15, o = 16 * a;
@@ -467,30 +545,77 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
     }
     __syncthreads();
-    // off-diagonal blocks, row by row, b increasing (so A_am, m >= b, is still unmodified):
-    //   Y = sum_{m=b}^{a-1} A_am X_mb ;   X_ab = -X_aa Y  (written over A_ab)
-    for (int a = 1; a < 4; ++a)
-        for (int b = 0; b < a; ++b) {
-            const int i = tid >> 4, j = tid & 15;
-            if (ok) {
-                float acc = 0.f;
-                for (int m = b; m < a; ++m)
+    // merge 16 -> 32 for diagonal pairs p = 0, 1 (rows/cols 32p .. 32p+31):
+    //   Y = A_{2p+1,2p} X_{2p,2p};  X_{2p+1,2p} = -X_{2p+1,2p+1} Y
+    {
+        const int pr = tid >> 7, e0 = tid & 127;   // pair, then 2 elements per thread
+        const int o = 32 * pr;
+        if (ok) {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t)
-                        acc = fmaf(AK[(16 * a + i) * 64 + 16 * m + t], AK[(16 * m + t) * 64 + 16 * b + j],
-                                   acc);
-                Yb[i * 16 + j] = acc;
-            }
-            __syncthreads();
-            if (ok) {
+            for (int qq = 0; qq < 2; ++qq) {
+                const int e = e0 + 128 * qq, i = e >> 4, j = e & 15;
                 float acc = 0.f;
 #pragma unroll
                 for (int t = 0; t < 16; ++t)
-                    acc = fmaf(AK[(16 * a + i) * 64 + 16 * a + t], Yb[t * 16 + j], acc);
-                AK[(16 * a + i) * 64 + 16 * b + j] = -acc;
+                    acc = fmaf(AK[(o + 16 + i) * 64 + o + t], AK[(o + t) * 64 + o + j], acc);
+                Yb[pr * 256 + e] = acc;
             }
-            __syncthreads();
         }
+        __syncthreads();
+        if (ok) {
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const int e = e0 + 128 * qq, i = e >> 4, j = e & 15;
+                float acc = 0.f;
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    acc = fmaf(AK[(o + 16 + i) * 64 + o + 16 + t], Yb[pr * 256 + t * 16 + j], acc);
+                AK[(o + 16 + i) * 64 + o + j] = -acc;
+            }
+        }
+        __syncthreads();
+    }
+    // merge 32 -> 64:  Z = A21 X11 (32x32);  X21 = -X22 Z
+    // thread (i0 = warp, j = lane) computes rows i0 + 8q, q = 0..3, of column j;
+    // the row operands are warp-uniform (broadcast float4 loads), the zero upper
+    // triangles make the fixed trip counts exact
+    {
+        const int j = lane, i0 = warp;
+        if (ok) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4) {
+                float xv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) xv[u] = AK[(4 * t4 + u) * 64 + j];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const float4 av = ld4(AK + (32 + i0 + 8 * qq) * 64 + 4 * t4);
+                    acc[qq] = fmaf(av.x, xv[0], fmaf(av.y, xv[1], fmaf(av.z, xv[2], fmaf(av.w, xv[3], acc[qq]))));
+                }
+            }
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) Yb[(i0 + 8 * qq) * 32 + j] = acc[qq];
+        }
+        __syncthreads();
+        if (ok) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4) {
+                float zv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) zv[u] = Yb[(4 * t4 + u) * 32 + j];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const float4 av = ld4(AK + (32 + i0 + 8 * qq) * 64 + 32 + 4 * t4);
+                    acc[qq] = fmaf(av.x, zv[0], fmaf(av.y, zv[1], fmaf(av.z, zv[2], fmaf(av.w, zv[3], acc[qq]))));
+                }
+            }
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) AK[(32 + i0 + 8 * qq) * 64 + j] = -acc[qq];
+        }
+        __syncthreads();
+    }
     // T = X Diag(beta) into rows 0..63 of [T; R] (fp16, K-major SW128)
     if (ok) {
         for (int task = tid; task < 64 * 8; task += 256) {
@@ -498,8 +623,8 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             float x[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int s = ch * 8 + e;
-                x[e] = (s <= r) ? AK[r * 64 + s] * bs[s] : 0.f;
+                const int s_ = ch * 8 + e;
+                x[e] = (s_ <= r) ? AK[r * 64 + s_] * bs[s_] : 0.f;
             }
             *reinterpret_cast<uint4 *>(sm + A_TR + sw128_kmajor_off(r, ch * 8, 0)) = pack8(x);
         }
@@ -517,6 +642,21 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             mma_f16(tmem + 128, ad, bd, id, kk > 0);
         }
         mma_commit(&bars[4]);
+    }
+    // Khat = k EL / E1 and Gamma_L straight to the slot while the MMA runs
+    if (ok) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
+            float x[8];
+            unpack8(kh_pref[i], x);
+            const float *e1 = E1 + s * D + cc, *el = EL + (s >> 4) * 128 + cc;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= el[e] * rcpa(e1[e]);
+            *reinterpret_cast<uint4 *>(slot + kSlotKh + sw128_mnmajor_off(cc, s, kKhMNBlock)) =
+                pack8(x);
+        }
+        if (tid < 128) reinterpret_cast<float *>(slot + kSlotGam)[tid] = GamL[tid];
     }
     if (ok) ok = mbar_wait_abortable(&bars[4], 0, err, abort_flag);
     tc_fence_after();
@@ -554,59 +694,53 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         mma_commit(&bars[5]);
     }
-    // [T; R] is final: copy it to the slot while the MMA runs (reads only);
-    // Khat = k EL / E1 and Gamma_L straight to the slot
+    const int quad = warp & 3, chalf = warp >> 2;
+    const int row6 = 32 * quad + lane, r6 = row6 & 63;
+    // q loads for P go out before the wait
+    uint4 qp[8];
+    if (row6 >= 64) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+            qp[ch] = r6 < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(q, r6) + 64 * chalf + ch * 8))
+                            : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // [T; R] is final: copy it to the slot while the MMA runs (reads only)
     if (ok) {
         const uint4 *src = reinterpret_cast<const uint4 *>(sm + A_TR);
         uint4 *dst = reinterpret_cast<uint4 *>(slot + kSlotTR);
         for (int i = tid; i < 16384 / 16; i += 256) dst[i] = src[i];
-        for (int task = tid; task < 64 * 16; task += 256) {
-            const int s = task >> 4, ch = task & 15, c = ch * 8;
-            float x[8];
-            if (s < L) {
-                unpack8(__ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + c)), x);
-                const float *e1 = E1 + s * D + c, *el = EL + (s >> 4) * 128 + c;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= el[e] * __frcp_rn(e1[e]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = 0.f;
-            }
-            *reinterpret_cast<uint4 *>(slot + kSlotKh + sw128_mnmajor_off(c, s, kKhMNBlock)) =
-                pack8(x);
-        }
-        if (tid < 128) reinterpret_cast<float *>(slot + kSlotGam)[tid] = __expf(GL[tid]);
     }
     if (ok) ok = mbar_wait_abortable(&bars[5], 0, err, abort_flag);
     tc_fence_after();
 
-    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = q E1 ER - R (K*Gamma)
+    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = q Gamma - R (K*Gamma)
     if (ok) {
-        const int quad = warp & 3, chalf = warp >> 2;
-        const int row = 32 * quad + lane;
-        const int r = row & 63;
         float x[64];
 #pragma unroll
-        for (int p = 0; p < 4; ++p)
-            tmem_ld16(taddr(tmem, 32 * quad, 64 * chalf + 16 * p),
-                      *reinterpret_cast<float(*)[16]>(x + 16 * p));
+        for (int pp = 0; pp < 4; ++pp)
+            tmem_ld16(taddr(tmem, 32 * quad, 64 * chalf + 16 * pp),
+                      *reinterpret_cast<float(*)[16]>(x + 16 * pp));
         tmem_wait_ld();
-        if (row < 64) {
+        if (row6 < 64) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) x[i] = -x[i];
-        } else if (r < L) {
+        } else {
+            const int a = r6 >> 4;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                const int c = 64 * chalf + ch * 8;
-                float qv[8];
-                unpack8(__ldg(reinterpret_cast<const uint4 *>(row_ptr(q, r) + c)), qv);
-                const float *e1 = E1 + r * D + c, *er = ER + (r >> 4) * 128 + c;
+                const int cc = 64 * chalf + ch * 8;
+                float qv8[8];
+                unpack8(qp[ch], qv8);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[ch * 8 + e] = qv[e] * e1[e] * er[e] - x[ch * 8 + e];
+                for (int hv = 0; hv < 2; ++hv) {
+                    float4 e = ld4(E1 + r6 * D + cc + 4 * hv);
+                    for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
+                    x[ch * 8 + 4 * hv] = qv8[4 * hv] * e.x - x[ch * 8 + 4 * hv];
+                    x[ch * 8 + 4 * hv + 1] = qv8[4 * hv + 1] * e.y - x[ch * 8 + 4 * hv + 1];
+                    x[ch * 8 + 4 * hv + 2] = qv8[4 * hv + 2] * e.z - x[ch * 8 + 4 * hv + 2];
+                    x[ch * 8 + 4 * hv + 3] = qv8[4 * hv + 3] * e.w - x[ch * 8 + 4 * hv + 3];
+                }
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) x[i] = 0.f;
         }
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -614,7 +748,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
             for (int e = 0; e < 8; ++e) y[e] = x[ch * 8 + e];
             *reinterpret_cast<uint4 *>(slot + kSlotWP +
-                                       sw128_kmajor_off(row, 64 * chalf + ch * 8, kWPKBlock)) =
+                                       sw128_kmajor_off(row6, 64 * chalf + ch * 8, kWPKBlock)) =
                 pack8(y);
         }
     }
@@ -631,25 +765,36 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 // ======================================================================
 template <int DVS>
 struct BLayout {
+    static constexpr int NST = DVS == 32 ? 3 : 2;              // slot ring depth (smem bound)
     static constexpr uint32_t kVBytes = 64 * DVS * 2;          // V slice tile
     static constexpr uint32_t kStage = kSlotBytes + kVBytes;   // slot image + V
-    static constexpr uint32_t kSB = 128 * DVS * 2;             // bf16 S  (K=128 x N=DVS)
-    static constexpr uint32_t kUB = 64 * DVS * 2;              // bf16 U  (K=64 x N=DVS)
+    static constexpr uint32_t kStageR = (kStage + 1023) & ~1023u;
+    static constexpr uint32_t kSB = 128 * DVS * 2;             // fp16 S  (K=128 x N=DVS)
+    static constexpr uint32_t kUB = 64 * DVS * 2;              // fp16 U  (K=64 x N=DVS)
     static constexpr uint32_t kKGroup = (DVS / 8) * 128;       // k-group stride, interleaved MN-major
-    static constexpr uint32_t oStage0 = 0;
-    static constexpr uint32_t oStage1 = (kStage + 1023) & ~1023u;
-    static constexpr uint32_t oSB = oStage1 + ((kStage + 1023) & ~1023u);
+    static constexpr uint32_t oSB = NST * kStageR;
     static constexpr uint32_t oUB = oSB + kSB;
     static constexpr uint32_t oBar = oUB + kUB;
     static constexpr uint32_t kBytes = oBar + 256 + 1024;      // + barriers + alignment slack
     static constexpr uint32_t kTmemCols = DVS == 32 ? 128 : (DVS == 64 ? 256 : 512);
+    static_assert(kBytes <= 227 * 1024, "state pass shared memory");
 };
 
 enum BBar {
-    FULL0 = 0, FULL1, EMPTY0, EMPTY1, TDFULL0, TDFULL1, TDEMPTY0, TDEMPTY1,
-    SBREADY, TSSCALED, UBREADY, TSFULL, DRAIN, NBARS
+    FULL0 = 0, EMPTY0 = 3, TDFULL0 = 6, TDFULL1, TDEMPTY0, TDEMPTY1,
+    TSSCALED, TSFULL, DRAIN_S, DRAIN_U, NBARS
 };
 
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Roles (384 threads): warp 0 producer; warp 1 owns the TMEM allocation;
+// warps 4-7 U/O epilogue, whose elected thread (warp 4, lane 0) issues the
+// state update S += Khat^T U; warps 8-11 state epilogue, whose elected thread
+// (warp 8, lane 0) issues [U; O] = [T; R] V + [-W; P] S.  Every bar.sync below
+// is executed by all threads of its group in every iteration (a failed bounded
+// wait only skips work), so a timeout can never leave a barrier half-joined.
 template <int DVS>
 __global__ void __launch_bounds__(384, 1)
 state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
@@ -665,6 +810,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::oBar);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + NBARS);
     volatile uint32_t *abort_flag = tmem_ptr + 1;
+    volatile uint32_t *s_grp_ok = tmem_ptr + 2;   // S issuer -> state warps
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int slice = blockIdx.x % NSL;
@@ -684,57 +830,42 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&bars[FULL0], 33);
-        mbar_init(&bars[FULL1], 33);
-        mbar_init(&bars[EMPTY0], 1);
-        mbar_init(&bars[EMPTY1], 1);
+        for (int i = 0; i < Lay::NST; ++i) {
+            mbar_init(&bars[FULL0 + i], 33);
+            mbar_init(&bars[EMPTY0 + i], 1);
+        }
         mbar_init(&bars[TDFULL0], 1);
         mbar_init(&bars[TDFULL1], 1);
         mbar_init(&bars[TDEMPTY0], 4);
         mbar_init(&bars[TDEMPTY1], 4);
-        mbar_init(&bars[SBREADY], 4);
-        mbar_init(&bars[TSSCALED], 4);
-        mbar_init(&bars[UBREADY], 2);
+        mbar_init(&bars[TSSCALED], 1);
         mbar_init(&bars[TSFULL], 1);
-        mbar_init(&bars[DRAIN], 1);
+        mbar_init(&bars[DRAIN_S], 1);
+        mbar_init(&bars[DRAIN_U], 1);
         mbar_fence_init();
         *abort_flag = 0u;
+        *s_grp_ok = 1u;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
     const uint32_t tTD0 = tmem, tTD1 = tmem + DVS, tTS = tmem + 2 * DVS;
+    constexpr int NST = Lay::NST;
+    auto stage_addr = [&](int st) { return sbase + st * Lay::kStageR; };
+    auto full_par = [&](int j) { return (uint32_t)((j / NST) & 1); };          // FULL[j % NST]
+    auto empty_par = [&](int j) { return (uint32_t)(((j / NST) + 1) & 1); };   // EMPTY before reuse
 
     if (warp == 0) {
         // ------------------------------------------------ producer
-        int issued_last = -1;
-        for (int j = 0; j < nch; ++j) {
-            const int st = j & 1;
-            if (j >= 2 && !mbar_wait_abortable(&bars[EMPTY0 + st], ((j >> 1) + 1) & 1, err,
-                                               abort_flag))
-                break;
-            uint8_t *stg = sm + (st ? Lay::oStage1 : Lay::oStage0);
-            const uint8_t *src = slots + ((size_t)(c0 + j) * H + h) * kSlotBytes;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[FULL0 + st], kSlotBytes);
-                bulk_g2s(stg, src, kSlotBytes, &bars[FULL0 + st]);
-            }
-            const int64_t t0 = ra + (int64_t)j * C;
-            const int L = (int)((rb - t0) < C ? (rb - t0) : C);
-            // V slice -> fp16 MMA operand (MN-major, interleaved core matrices).
-            // All 16-byte pieces are fetched asynchronously straight into their
-            // operand positions (rows past the end of the sequence zero-filled),
-            // then each lane converts the pieces it fetched from bf16 to fp16 in place.
-            uint8_t *vt = stg + kSlotBytes;
-            constexpr int CPR = DVS / 8;   // 16-byte pieces per row
-            for (int task = lane; task < 64 * CPR; task += 32) {
-                const int r = task / CPR, ch = task % CPR;
-                const int rr = r < L ? r : 0;
-                cp_async16(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup),
-                           v + ((size_t)(t0 + rr) * H + h) * D + j0 + ch * 8, r < L ? 16u : 0u);
-            }
-            cp_async_wait_all();
+        // Chunk j's slot image goes in with one bulk copy; its V slice with
+        // cp.async straight into the fp16 operand positions (rows past the end
+        // of the sequence zero-filled), converted from bf16 in place by the lane
+        // that fetched it.  The conversion of chunk j - 1 waits on its own
+        // cp.async group only, so chunk j's loads are already in flight.
+        constexpr int CPR = DVS / 8;   // 16-byte pieces per row
+        auto convert_v = [&](int j) {
+            uint8_t *vt = sm + (j % NST) * Lay::kStageR + kSlotBytes;
             for (int task = lane; task < 64 * CPR; task += 32) {
                 const int r = task / CPR, ch = task % CPR;
                 uint4 *pc = reinterpret_cast<uint4 *>(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup));
@@ -743,118 +874,129 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 *pc = pack8(x);
             }
             fence_async_smem();
-            mbar_arrive(&bars[FULL0 + st]);
-            issued_last = j;
-        }
-        // drain: never leave the CTA with bulk copies still landing in its shared memory
-        for (int j = issued_last - 1; j <= issued_last; ++j)
-            if (j >= 0) mbar_wait(&bars[FULL0 + (j & 1)], (j >> 1) & 1, err, 1u << 22);
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
-            const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
-            for (int j = 0; j < nch; ++j) {
-                const int st = j & 1, b = j & 1;
-                const uint32_t stg = sbase + (st ? Lay::oStage1 : Lay::oStage0);
-                const uint32_t tTD = b ? tTD1 : tTD0;
-                if (!mbar_wait_abortable(&bars[FULL0 + st], (j >> 1) & 1, err, abort_flag)) break;
-                if (j >= 2 && !mbar_wait_abortable(&bars[TDEMPTY0 + b], ((j >> 1) + 1) & 1, err,
-                                                   abort_flag))
-                    break;
-                tc_fence_after();
-                // [U; O] = [T; R] V
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = smem_desc(stg + kSlotTR + kk * 32, 16, 1024, SW_128B);
-                    const uint64_t bd = smem_desc(stg + kSlotBytes + kk * 2 * Lay::kKGroup,
-                                                  Lay::kKGroup, 128, SW_NONE);
-                    mma_f16(tTD, ad, bd, id_nn, kk > 0);
-                }
-                if (!mbar_wait_abortable(&bars[SBREADY], j & 1, err, abort_flag)) break;
-                tc_fence_after();
-                // [U; O] += [-W; P] S
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = smem_desc(
-                        stg + kSlotWP + (kk >> 2) * kWPKBlock + (kk & 3) * 32, 16, 1024, SW_128B);
-                    const uint64_t bd = smem_desc(sbase + Lay::oSB + kk * 2 * Lay::kKGroup,
-                                                  Lay::kKGroup, 128, SW_NONE);
-                    mma_f16(tTD, ad, bd, id_nn, 1);
-                }
-                mma_commit(&bars[TDFULL0 + b]);
-                if (!mbar_wait_abortable(&bars[UBREADY], j & 1, err, abort_flag)) break;
-                if (!mbar_wait_abortable(&bars[TSSCALED], j & 1, err, abort_flag)) break;
-                tc_fence_after();
-                // S += Khat^T U
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = smem_desc(stg + kSlotKh + kk * 2048, kKhMNBlock, 1024,
-                                                  SW_128B);
-                    const uint64_t bd = smem_desc(sbase + Lay::oUB + kk * 2 * Lay::kKGroup,
-                                                  Lay::kKGroup, 128, SW_NONE);
-                    mma_f16(tTS, ad, bd, id_mm, 1);
-                }
-                mma_commit(&bars[TSFULL]);
-                mma_commit(&bars[EMPTY0 + st]);
+            mbar_arrive(&bars[FULL0 + j % NST]);
+        };
+        int issued = 0;
+        bool okp = true;
+        for (int j = 0; j < nch; ++j) {
+            const int st = j % NST;
+            if (j >= NST && !mbar_wait_abortable(&bars[EMPTY0 + st], empty_par(j), err, abort_flag)) {
+                okp = false;
+                break;
             }
-            // drain: every MMA issued above has completed before TMEM is released
-            mma_commit(&bars[DRAIN]);
-            mbar_wait(&bars[DRAIN], 0, err, 1u << 22);
+            uint8_t *stg = sm + st * Lay::kStageR;
+            const uint8_t *src = slots + ((size_t)(c0 + j) * H + h) * kSlotBytes;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars[FULL0 + st], kSlotBytes);
+                bulk_g2s(stg, src, kSlotBytes, &bars[FULL0 + st]);
+            }
+            const int64_t t0 = ra + (int64_t)j * C;
+            const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+            uint8_t *vt = stg + kSlotBytes;
+            for (int task = lane; task < 64 * CPR; task += 32) {
+                const int r = task / CPR, ch = task % CPR;
+                const int rr = r < L ? r : 0;
+                cp_async16(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup),
+                           v + ((size_t)(t0 + rr) * H + h) * D + j0 + ch * 8, r < L ? 16u : 0u);
+            }
+            cp_async_commit();
+            issued = j + 1;
+            if (j >= 1) {
+                cp_async_wait_group1();   // chunk j - 1's pieces have landed
+                convert_v(j - 1);
+            }
         }
-        __syncwarp();
+        cp_async_wait_all();
+        if (issued >= 1) convert_v(issued - 1);
+        (void)okp;
+        // drain: never leave the CTA with bulk copies still landing in its shared memory
+        for (int j = issued - NST; j < issued; ++j)
+            if (j >= 0) mbar_wait(&bars[FULL0 + j % NST], full_par(j), err, 1ull << 28);
     } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------------ U / O epilogue
+        // ------------------------------------------------ U / O epilogue (+ state-update issue)
         const int quad = warp - 4;
         const int row = 32 * quad + lane;
+        const bool issuer = (warp == 4 && lane == 0);
+        const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
+        bool ok = true;
         for (int j = 0; j < nch; ++j) {
-            const int b = j & 1;
+            const int b = j & 1, st = j % NST;
             const uint32_t tTD = b ? tTD1 : tTD0;
-            if (!mbar_wait_abortable(&bars[TDFULL0 + b], (j >> 1) & 1, err, abort_flag)) break;
+            if (ok) ok = mbar_wait_abortable(&bars[TDFULL0 + b], (j >> 1) & 1, err, abort_flag);
             tc_fence_after();
             const int64_t t0 = ra + (int64_t)j * C;
             const int L = (int)((rb - t0) < C ? (rb - t0) : C);
             const int r = row - 64;
+            if (ok) {
+                float xa[DVS];
 #pragma unroll
-            for (int p = 0; p < DVS / 16; ++p) {
-                float x[16];
-                tmem_ld16(taddr(tTD, 32 * quad, 16 * p), x);
+                for (int p = 0; p < DVS / 16; ++p)
+                    tmem_ld16(taddr(tTD, 32 * quad, 16 * p), *reinterpret_cast<float(*)[16]>(xa + 16 * p));
                 tmem_wait_ld();
-                float y0[8], y1[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    y0[e] = x[e];
-                    y1[e] = x[8 + e];
-                }
-                if (quad < 2) {
-                    // U rows -> bf16 B operand (MN-major, interleaved core matrices)
-                    *reinterpret_cast<uint4 *>(
-                        sm + Lay::oUB + interleave_mnmajor_off(16 * p, row, Lay::kKGroup)) = pack8(y0);
-                    *reinterpret_cast<uint4 *>(
-                        sm + Lay::oUB + interleave_mnmajor_off(16 * p + 8, row, Lay::kKGroup)) =
-                        pack8(y1);
-                } else if (r < L) {
-                    float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * D + j0 +
-                                                             16 * p);
+                for (int p = 0; p < DVS / 16; ++p) {
+                    const float *x = xa + 16 * p;
+                    float y0[8], y1[8];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+                    for (int e = 0; e < 8; ++e) {
+                        y0[e] = x[e];
+                        y1[e] = x[8 + e];
+                    }
+                    if (quad < 2) {
+                        // U rows -> fp16 B operand (MN-major, interleaved core matrices)
+                        *reinterpret_cast<uint4 *>(
+                            sm + Lay::oUB + interleave_mnmajor_off(16 * p, row, Lay::kKGroup)) = pack8(y0);
+                        *reinterpret_cast<uint4 *>(
+                            sm + Lay::oUB + interleave_mnmajor_off(16 * p + 8, row, Lay::kKGroup)) =
+                            pack8(y1);
+                    } else if (r < L) {
+                        float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * D +
+                                                                 j0 + 16 * p);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+                    }
                 }
             }
             if (quad < 2) {
                 fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[UBREADY]);
+                named_bar(1, 64);   // both U warps (4 and 5) have written their rows
+                if (issuer && ok) {
+                    // and the state is scaled by Gamma_j
+                    ok = mbar_wait_abortable(&bars[TSSCALED], j & 1, err, abort_flag);
+                    if (ok) {
+                        tc_fence_after();
+                        // S += Khat^T U   (descriptors advance by their start-address field)
+                        const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotKh, kKhMNBlock, 1024, SW_128B);
+                        const uint64_t bd0 = smem_desc(sbase + Lay::oUB, Lay::kKGroup, 128, SW_NONE);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f16(tTS, ad0 + (uint64_t)(kk * 2048 / 16),
+                                    bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_mm, 1);
+                        mma_commit(&bars[TSFULL]);
+                        mma_commit(&bars[EMPTY0 + st]);
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[TDEMPTY0 + b]);
         }
+        if (issuer) {
+            // every MMA this thread issued has completed before TMEM is released
+            mma_commit(&bars[DRAIN_U]);
+            mbar_wait(&bars[DRAIN_U], 0, err, 1ull << 28);
+        }
     } else if (warp >= 8) {
-        // ------------------------------------------------ state epilogue
+        // ------------------------------------------------ state epilogue (+ chunk-product issue)
         const int quad = warp - 8;
         const int c = 32 * quad + lane;   // key channel = TMEM lane
+        const bool issuer = (warp == 8 && lane == 0);
         const uint32_t tS = taddr(tTS, 32 * quad, 0);
         const size_t srow = (((size_t)n * H + h) * D + c) * D + j0;
+        const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
         uint8_t *sbp = sm + Lay::oSB;
-        auto put_sb = [&](int p, const float (&x)[16]) {
+        auto put_sb = [&](int p, const float *x) {
             float y0[8], y1[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -866,17 +1008,62 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p + 8, c, Lay::kKGroup)) =
                 pack8(y1);
         };
-        auto signal = [&](int which) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[which]);
+        // [T; R]_j V_j into TD[j % 2] (the V term; independent of the state)
+        int v_issued = -1;   // highest chunk whose V term has been issued (issuer only)
+        auto issue_vterm = [&](int j) {
+            const int st = j % NST;
+            const uint32_t tTD = (j & 1) ? tTD1 : tTD0;
+            const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotTR, 16, 1024, SW_128B);
+            const uint64_t bd0 = smem_desc(stage_addr(st) + kSlotBytes, Lay::kKGroup, 128, SW_NONE);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(tTD, ad0 + (uint64_t)(kk * 32 / 16),
+                        bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, kk > 0);
+            v_issued = j;
         };
-        auto stage_gamma = [&](int j, float &gam) -> bool {
-            const int st = j & 1;
-            if (!mbar_wait_abortable(&bars[FULL0 + st], (j >> 1) & 1, err, abort_flag))
-                return false;
-            gam = reinterpret_cast<const float *>(sm + (st ? Lay::oStage1 : Lay::oStage0) +
-                                                  kSlotGam)[c];
-            return true;
+        // After the fp16 copy of S_j is in place: the elected thread issues
+        // [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j into TD[j % 2] and tells the
+        // group whether it succeeded.  When the next chunk's slot and
+        // accumulator are already free it also issues that chunk's V term, so
+        // that only the state term remains on the chunk-to-chunk path.
+        auto issue_chunk = [&](int j) {
+            fence_async_smem();
+            named_bar(2, 128);
+            if (issuer) {
+                const int st = j % NST, b = j & 1;
+                bool okk = *s_grp_ok != 0u;
+                if (v_issued < j) {
+                    if (okk) okk = mbar_wait_abortable(&bars[FULL0 + st], full_par(j), err, abort_flag);
+                    if (okk && j >= 2)
+                        okk = mbar_wait_abortable(&bars[TDEMPTY0 + b], ((j >> 1) + 1) & 1, err,
+                                                  abort_flag);
+                    if (okk) {
+                        tc_fence_after();
+                        issue_vterm(j);
+                    }
+                }
+                if (okk) {
+                    tc_fence_after();
+                    const uint32_t tTD = b ? tTD1 : tTD0;
+                    const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotWP, 16, 1024, SW_128B);
+                    const uint64_t bd0 = smem_desc(sbase + Lay::oSB, Lay::kKGroup, 128, SW_NONE);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_f16(tTD, ad0 + (uint64_t)(((kk >> 2) * kWPKBlock + (kk & 3) * 32) / 16),
+                                bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, 1);
+                    mma_commit(&bars[TDFULL0 + b]);
+                    // early V term of chunk j + 1, only if nothing has to be waited for
+                    const int jn = j + 1;
+                    if (jn < nch && mbar_try_wait(&bars[FULL0 + jn % NST], full_par(jn)) &&
+                        (jn < 2 || mbar_try_wait(&bars[TDEMPTY0 + (jn & 1)], ((jn >> 1) + 1) & 1))) {
+                        tc_fence_after();
+                        issue_vterm(jn);
+                    }
+                }
+                *s_grp_ok = okk ? 1u : 0u;
+            }
+            named_bar(2, 128);
+            return *s_grp_ok != 0u;
         };
         if (nch == 0) {
             // empty sequence: the state passes through unchanged
@@ -886,9 +1073,8 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         state_in ? reinterpret_cast<const float4 *>(state_in + srow)[i]
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
-            // S_0: bf16 copy for the first MMA, fp32 copy (already scaled by Gamma_0) into TMEM
-            float gam = 0.f;
             bool ok = true;
+            // S_0: fp16 copy for the first chunk's products
             for (int p = 0; p < DVS / 16; ++p) {
                 float x[16];
 #pragma unroll
@@ -900,63 +1086,64 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 }
                 put_sb(p, x);
             }
-            fence_async_smem();
-            signal(SBREADY);
-            ok = stage_gamma(0, gam);
-            if (ok) {
-                for (int p = 0; p < DVS / 16; ++p) {
-                    float x[16];
+            ok = issue_chunk(0);
+            // x = S_j in registers (fp32); TS <- Gamma_j S_j; then wait for the
+            // update S_{j+1} = TS + Khat_j^T U_j, copy it to fp16 for the next
+            // chunk's products, and keep it in registers for the next scaling.
+            float xa[DVS];
+            for (int p = 0; p < DVS / 16; ++p)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float4 f = state_in
-                            ? reinterpret_cast<const float4 *>(state_in + srow)[4 * p + i]
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                        x[4 * i] = f.x * gam; x[4 * i + 1] = f.y * gam;
-                        x[4 * i + 2] = f.z * gam; x[4 * i + 3] = f.w * gam;
+                for (int i = 0; i < 4; ++i) {
+                    const float4 f = state_in
+                        ? reinterpret_cast<const float4 *>(state_in + srow)[4 * p + i]
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    xa[16 * p + 4 * i] = f.x; xa[16 * p + 4 * i + 1] = f.y;
+                    xa[16 * p + 4 * i + 2] = f.z; xa[16 * p + 4 * i + 3] = f.w;
+                }
+            for (int j = 0; j < nch; ++j) {
+                float gam = 0.f;
+                if (ok) ok = mbar_wait_abortable(&bars[FULL0 + j % NST], full_par(j), err, abort_flag);
+                if (ok) gam = reinterpret_cast<const float *>(sm + (j % NST) * Lay::kStageR + kSlotGam)[c];
+                if (ok) {
+#pragma unroll
+                    for (int p = 0; p < DVS / 16; ++p) {
+                        float x[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) x[e] = xa[16 * p + e] * gam;
+                        tmem_st16(tS + 16 * p, x);
                     }
-                    tmem_st16(tS + 16 * p, x);
+                    tmem_wait_st();
                 }
-                tmem_wait_st();
                 tc_fence_before();
-                signal(TSSCALED);
-            }
-            for (int j = 0; ok && j < nch; ++j) {
-                if (!mbar_wait_abortable(&bars[TSFULL], j & 1, err, abort_flag)) { ok = false; break; }
+                named_bar(2, 128);
+                if (issuer) mbar_arrive(&bars[TSSCALED]);
+                // S_{j+1} = TS after the state update of chunk j
+                if (ok) ok = mbar_wait_abortable(&bars[TSFULL], j & 1, err, abort_flag);
                 tc_fence_after();
-                if (j + 1 == nch) break;
-                // S_{j+1}: bf16 copy for the next chunk's MMA (critical path) ...
-                for (int p = 0; p < DVS / 16; ++p) {
-                    float x[16];
-                    tmem_ld16(tS + 16 * p, x);
-                    tmem_wait_ld();
-                    put_sb(p, x);
-                }
-                fence_async_smem();
-                signal(SBREADY);
-                // ... then the fp32 copy scaled by Gamma_{j+1} for the next state update
-                if (!stage_gamma(j + 1, gam)) { ok = false; break; }
-                for (int p = 0; p < DVS / 16; ++p) {
-                    float x[16];
-                    tmem_ld16(tS + 16 * p, x);
-                    tmem_wait_ld();
+                if (ok) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) x[e] *= gam;
-                    tmem_st16(tS + 16 * p, x);
+                    for (int p = 0; p < DVS / 16; ++p)
+                        tmem_ld16(tS + 16 * p, *reinterpret_cast<float(*)[16]>(xa + 16 * p));
+                    tmem_wait_ld();
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                signal(TSSCALED);
+                if (j + 1 == nch) break;
+                if (ok) {
+#pragma unroll
+                    for (int p = 0; p < DVS / 16; ++p) put_sb(p, xa + 16 * p);
+                }
+                if (issuer) *s_grp_ok = ok ? 1u : 0u;
+                const bool ok2 = issue_chunk(j + 1);
+                ok = ok && ok2;
             }
             if (ok && state_out && !*abort_flag) {
-                for (int p = 0; p < DVS / 16; ++p) {
-                    float x[16];
-                    tmem_ld16(tS + 16 * p, x);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        reinterpret_cast<float4 *>(state_out + srow)[4 * p + i] =
-                            make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
-                }
+                for (int i = 0; i < DVS / 4; ++i)
+                    reinterpret_cast<float4 *>(state_out + srow)[i] =
+                        make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
+            }
+            if (issuer) {
+                mma_commit(&bars[DRAIN_S]);
+                mbar_wait(&bars[DRAIN_S], 0, err, 1ull << 28);
             }
         }
     }

@@ -172,6 +172,16 @@ __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src, uint
                  : "memory");
 }
 
+// Close the current group of this thread's cp.async copies.
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Wait until at most one of this thread's committed cp.async groups is pending.
+__device__ __forceinline__ void cp_async_wait_group1() {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
 // Wait until all of this thread's prior cp.async copies have landed.
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");

@@ -44,6 +44,30 @@ DECODE_BYTES_PER_UNIT = 2 * STATE_BYTES + 4 * 128 * 2 + 2 + 128 * 4
 SLOT_BYTES = 66560                                            # per (chunk, head) workspace slot
 FLOPS_PER_TOKEN_HEAD = 139264                                 # algorithmic MMA flops (causal halves once)
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per (chunk, head) or per
+# launch from one ncu capture (profiles/), valid only for the kernel source it was taken
+# on: the sha256 prefix of that .cu file.  A changed source reports null.
+NCU_TRAFFIC = {
+    "intra_chunk_kernel": ("kda_prefill_bf16.cu", "73141276c9cba024", 457123840 / 4096),
+    "state_pass_kernel": ("kda_prefill_bf16.cu", "73141276c9cba024", 448756480 / 4096),
+    "decode_kernel": ("kda_decode.cu", "c088165a18adb1b1", 1027868672),
+}
+
+
+def ncu_traffic(kernel: str, units: float):
+    """Measured bytes for one launch covering `units` (head-chunks; 1 for decode), or None."""
+    import hashlib
+    ent = NCU_TRAFFIC.get(kernel)
+    if ent is None:
+        return None
+    fname, digest, per_unit = ent
+    path = os.path.join(ROOT, "kda_delta_rule_chunkwise_b200", "csrc", fname)
+    try:
+        cur = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return round(per_unit * units) if cur == digest else None
+
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
@@ -122,6 +146,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar (elapsed ms) over all ranks; identity for one rank."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank_step: float, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (ms_max / 1e3)
+
+
 # ----------------------------------------------------------------------------- ours
 
 def time_prefill(binding, d, o, s_out, ws, steps, warmup, profile=False):
@@ -190,13 +230,9 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
     if True:
         ms = time_prefill(binding, d, o, s_out, ws, args.steps, args.warmup)
     torch.cuda.synchronize()
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     ms_step = ms_max / args.steps
-    value = tokens * world * args.steps / (ms_max / 1e3)
+    value = aggregate_throughput(tokens, world, args.steps, ms_max)
 
     # per-kernel device time (separate profiled pass, same inputs)
     per = time_prefill(binding, d, o, s_out, ws, max(2, args.steps), 1, profile=True)
@@ -216,7 +252,8 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
     roofline = {
         "kernel": dom_name, "bound": "hbm", "achieved": round(achieved, 1),
         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-        "traffic": None, "peak_source": peaks["source"],
+        "traffic": ncu_traffic(dom_name, head_chunks), "peak_source": peaks["source"],
+        "algorithmic_bytes": k_bytes[dom_name],
         "kernel_ms": {n: round(x, 4) for n, x in zip(names, k_avg)},
         "kernel_share": {n: round(x / sum(k_avg), 4) for n, x in zip(names, k_avg)},
     }
@@ -260,12 +297,8 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
             e2e_step()
         ev1.record(st)
         torch.cuda.synchronize()
-        e_ms = ev0.elapsed_time(ev1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": tokens * world * args.e2e_steps / (e_ms / 1e3), "unit": "tokens/s",
+        e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        e2e = {"value": aggregate_throughput(tokens, world, args.e2e_steps, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": in_bytes,
                "d2h_bytes_per_step": o.numel() * o.element_size()
                + s_out.numel() * s_out.element_size(),
@@ -304,11 +337,7 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
         dec_step(t)
     ev1.record(st)
     torch.cuda.synchronize()
-    d_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t_ = torch.tensor([d_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
-        d_ms = float(t_.item())
+    d_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     d_bytes = Nd * Hd * DECODE_BYTES_PER_UNIT
     d_gbs = d_bytes * args.decode_steps / (d_ms / 1e3) / 1e9
     decode = {
@@ -317,7 +346,8 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
         "gbs": round(world * d_gbs, 1), "gbs_per_gpu": round(d_gbs, 1),
         "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(d_gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(d_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "frac": round(d_gbs / peaks["hbm_gbs"], 4),
+                     "traffic": ncu_traffic("decode_kernel", 1),
                      "bytes_per_launch": d_bytes},
         "state_bytes": S.numel() * 4,
     }

@@ -219,11 +219,18 @@ constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64 
 constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64     16 KiB
 constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128          16 KiB
 constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 solve scratch (32 x 32)               4 KiB
+constexpr uint32_t A_QP = A_AK;               // bf16 q rows [64][128] for P, once T is out  16 KiB
 constexpr uint32_t A_SMEM = A_OPS + 2 * A_RBUF + 1024;   // + alignment slack (= 112640)
 static_assert(A_Y + 4096 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
 static_assert(A_OPS + 4096 + 16384 <= A_OPS + A_RBUF, "g staging must fit in round buffer 0");
 static_assert(A_OPS % 1024 == 0 && A_RBUF % 1024 == 0 && A_AQ % 1024 == 0 && A_TR % 1024 == 0 &&
               A_KT % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+// E1 is stored [64][128] fp32 with its 16-byte pieces (4 channels) permuted per
+// row: piece p of row r sits at p ^ (r % 32).  Reads of the same channels in
+// consecutive rows (one row per lane) then spread over all banks.
+__device__ __forceinline__ int e1_at(int row, int col4) {   // col4: multiple of 4
+    return row * 128 + (((col4 >> 2) ^ (row & 31)) << 2);
+}
 // first row-group of the packed K^(a) tile: 0, 2, 6, 12
 __device__ __forceinline__ int at_group(int a) { return a * (a + 1); }
 
@@ -310,14 +317,18 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     };
 
     // ---- issue every global load of the operand rounds up front (one round trip)
-    // round task: lane -> 4-channel piece p_l of the round, token rows 32*it + 4*warp + rsub
+    // round task: lane -> 4-channel piece p_l of the round and two token rows, one
+    // in the first and one in the second half of the chunk, paired so that every
+    // warp writes the same number of packed K^(a) copies (rows of block b have
+    // 4 - b of them): warps 0-3 take blocks 0 and 3, warps 4-7 blocks 1 and 2
     const int p_l = lane & 7, rsub = lane >> 3;
+    auto a1_row = [&](int it) { return it == 0 ? 4 * warp + rsub : 32 + 4 * (warp ^ 4) + rsub; };
     uint2 qv[4][2], kv[4][2];
 #pragma unroll
     for (int rd = 0; rd < 4; ++rd)
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
-            const int r = 32 * it + 4 * warp + rsub;
+            const int r = a1_row(it);
             const int c0 = 32 * rd + 4 * p_l;
             if (r < L) {
                 qv[rd][it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(q, r) + c0));
@@ -368,7 +379,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const float x = i < 16 ? p[i] : p[i] - p[15];
-        E1[(half * 32 + i) * D + c] = __expf(x);
+        E1[e1_at(half * 32 + i, c & ~3) + (c & 3)] = __expf(x);
     }
     if (half == 0) {
         tot[c] = p[31];
@@ -385,10 +396,11 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const int lr = L - 1;
         if (lr >= 0 && (lr >> 5) == half) {
             const float base = half ? tot[c] : 0.f;
+            // multiply-add selection keeps p[] in registers (no indexed access)
+            const int li = lr & 31;
             float v = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (i == (lr & 31)) v = p[i];
+            for (int i = 0; i < 32; ++i) v = fmaf(i == li ? 1.f : 0.f, p[i], v);
             GLv[c] = base + v;
         }
         if (L <= 0 && half == 0) GLv[c] = 0.f;
@@ -420,12 +432,12 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             const int c0 = 32 * rd + 4 * p_l;
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
-                const int r = 32 * it + 4 * warp + rsub;
+                const int r = a1_row(it);
                 const int a = r >> 4, i = r & 15;
                 // every row this task writes is congruent to r mod 8: one swizzled chunk offset
                 const uint32_t co = (r & 7) * 128 + ((p_l ^ (r & 7)) << 4);
                 uint8_t *bt = sm + buf + A_BT + co, *at = sm + buf + A_AT + co;
-                const float4 e = ld4(E1 + r * D + c0);
+                const float4 e = ld4(E1 + e1_at(r, c0));
                 const float4 qf = bf4(qv[rd][it]), kf = bf4(kv[rd][it]);
                 *reinterpret_cast<float4 *>(bt + ((32 * a + i) >> 3) * 1024) = tf4(mul4(qf, e));
                 *reinterpret_cast<float4 *>(bt + ((32 * a + 16 + i) >> 3) * 1024) = tf4(mul4(kf, e));
@@ -502,7 +514,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             const int a = s >> 4;
 #pragma unroll
             for (int hv = 0; hv < 2; ++hv) {
-                float4 e = ld4(E1 + s * D + cc + 4 * hv);
+                float4 e = ld4(E1 + e1_at(s, cc + 4 * hv));
                 for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
                 x[4 * hv] *= e.x; x[4 * hv + 1] *= e.y; x[4 * hv + 2] *= e.z; x[4 * hv + 3] *= e.w;
             }
@@ -512,13 +524,18 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     tc_fence_before();
     __syncthreads();
 
-    // Khat loads for A5 go out now; the solve below hides their latency
-    uint4 kh_pref[4];
+    // Khat = k EL / E1 for the slot, by warps 2-7 while warps 0-1 run the
+    // diagonal blocks of the solve below; its loads go out now
+    constexpr int KH_TASKS = 6;   // 1024 8-channel pieces over 192 threads
+    uint4 kh_pref[KH_TASKS];
+    if (warp >= 2) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
-        kh_pref[i] = s < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
-                           : make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < KH_TASKS; ++i) {
+            const int task = (tid - 64) + 192 * i, s = task >> 4, cc = (task & 15) * 8;
+            kh_pref[i] = (task < 1024 && s < L)
+                ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
+                : make_uint4(0u, 0u, 0u, 0u);
+        }
     }
 
     // ---- A3: X = (I + Akk)^-1 in place over AK (fp32), by 2x2 block merges:
@@ -537,6 +554,24 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 for (int m = 0; m < i; ++m) acc = fmaf(-AK[(o + i) * 64 + o + m], x[m], acc);
                 x[i] = acc;
             }
+        }
+        if (ok && warp >= 2) {
+#pragma unroll
+            for (int i = 0; i < KH_TASKS; ++i) {
+                const int task = (tid - 64) + 192 * i, s = task >> 4, cc = (task & 15) * 8;
+                if (task < 1024) {
+                    float xk[8];
+                    unpack8(kh_pref[i], xk);
+                    const float *el = EL + (s >> 4) * 128 + cc;
+                    const float4 ea = ld4(E1 + e1_at(s, cc)), eb = ld4(E1 + e1_at(s, cc + 4));
+                    const float e1[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xk[e] *= el[e] * rcpa(e1[e]);
+                    *reinterpret_cast<uint4 *>(slot + kSlotKh +
+                                               sw128_mnmajor_off(cc, s, kKhMNBlock)) = pack8(xk);
+                }
+            }
+            if (tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = GamL[tid - 128];
         }
         __syncthreads();
         if (ok && tid < 64) {
@@ -620,18 +655,30 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     if (ok) {
         for (int task = tid; task < 64 * 8; task += 256) {
             const int r = task >> 3, ch = task & 7;
+            const float4 xa = ld4(AK + r * 64 + ch * 8), xb = ld4(AK + r * 64 + ch * 8 + 4);
+            const float4 ba = ld4(bs + ch * 8), bb = ld4(bs + ch * 8 + 4);
+            const float xv[8] = {xa.x * ba.x, xa.y * ba.y, xa.z * ba.z, xa.w * ba.w,
+                                 xb.x * bb.x, xb.y * bb.y, xb.z * bb.z, xb.w * bb.w};
             float x[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int s_ = ch * 8 + e;
-                x[e] = (s_ <= r) ? AK[r * 64 + s_] * bs[s_] : 0.f;
-            }
+            for (int e = 0; e < 8; ++e) x[e] = (ch * 8 + e <= r) ? xv[e] : 0.f;
             *reinterpret_cast<uint4 *>(sm + A_TR + sw128_kmajor_off(r, ch * 8, 0)) = pack8(x);
         }
     }
     fence_async_smem();
     __syncthreads();
     tc_fence_after();
+
+    // q rows for P (A6) go to the Akk region, dead since T was written: cp.async,
+    // landed by the barrier before A5 (rows past L zero-filled).  Row r's 16-byte
+    // piece p sits at slot p ^ (r % 16), so that A6's row-per-lane reads are
+    // free of bank conflicts.
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int task = tid + 256 * i, r = task >> 4, cc = (task & 15) * 8;
+        cp_async16(sm + A_QP + (r * 16 + ((task & 15) ^ (r & 15))) * 16, row_ptr(q, r < L ? r : 0) + cc,
+                   r < L ? 16u : 0u);
+    }
 
     // ---- A4: R = Aqk T  (M=64, N=64, K=64; A MN-major, B MN-major) into TMEM columns 128..191
     if (ok && tid == 0) {
@@ -642,21 +689,6 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             mma_f16(tmem + 128, ad, bd, id, kk > 0);
         }
         mma_commit(&bars[4]);
-    }
-    // Khat = k EL / E1 and Gamma_L straight to the slot while the MMA runs
-    if (ok) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
-            float x[8];
-            unpack8(kh_pref[i], x);
-            const float *e1 = E1 + s * D + cc, *el = EL + (s >> 4) * 128 + cc;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] *= el[e] * rcpa(e1[e]);
-            *reinterpret_cast<uint4 *>(slot + kSlotKh + sw128_mnmajor_off(cc, s, kKhMNBlock)) =
-                pack8(x);
-        }
-        if (tid < 128) reinterpret_cast<float *>(slot + kSlotGam)[tid] = GamL[tid];
     }
     if (ok) ok = mbar_wait_abortable(&bars[4], 0, err, abort_flag);
     tc_fence_after();
@@ -679,6 +711,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
         }
     }
+    cp_async_wait_all();   // this thread's q rows for A6
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -696,14 +729,6 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     const int quad = warp & 3, chalf = warp >> 2;
     const int row6 = 32 * quad + lane, r6 = row6 & 63;
-    // q loads for P go out before the wait
-    uint4 qp[8];
-    if (row6 >= 64) {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-            qp[ch] = r6 < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(q, r6) + 64 * chalf + ch * 8))
-                            : make_uint4(0u, 0u, 0u, 0u);
-    }
     // [T; R] is final: copy it to the slot while the MMA runs (reads only)
     if (ok) {
         const uint4 *src = reinterpret_cast<const uint4 *>(sm + A_TR);
@@ -730,10 +755,11 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             for (int ch = 0; ch < 8; ++ch) {
                 const int cc = 64 * chalf + ch * 8;
                 float qv8[8];
-                unpack8(qp[ch], qv8);
+                unpack8(reinterpret_cast<const uint4 *>(sm + A_QP)[r6 * 16 + ((8 * chalf + ch) ^ (r6 & 15))],
+                        qv8);
 #pragma unroll
                 for (int hv = 0; hv < 2; ++hv) {
-                    float4 e = ld4(E1 + r6 * D + cc + 4 * hv);
+                    float4 e = ld4(E1 + e1_at(r6, cc + 4 * hv));
                     for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
                     x[ch * 8 + 4 * hv] = qv8[4 * hv] * e.x - x[ch * 8 + 4 * hv];
                     x[ch * 8 + 4 * hv + 1] = qv8[4 * hv + 1] * e.y - x[ch * 8 + 4 * hv + 1];
@@ -781,19 +807,25 @@ struct BLayout {
 };
 
 enum BBar {
-    FULL0 = 0, EMPTY0 = 3, TDFULL0 = 6, TDFULL1, TDEMPTY0, TDEMPTY1,
+    FULL0 = 0,       // [NST] slot image landed (bulk copy tx)
+    EMPTY0 = 3,      // [NST] every MMA reading the stage has completed
+    VRAW0 = 6,       // [NST] the producer lanes' cp.async of the V slice have landed
+    VREADY0 = 9,     // [NST] V slice converted to fp16 in place
+    TDFULL0 = 12, TDFULL1, TDEMPTY0, TDEMPTY1,
     TSSCALED, TSFULL, DRAIN_S, DRAIN_U, NBARS
 };
+static_assert(NBARS * 8 + 16 <= 256, "phase B barrier area");
 
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Roles (384 threads): warp 0 producer; warp 1 owns the TMEM allocation;
-// warps 4-7 U/O epilogue, whose elected thread (warp 4, lane 0) issues the
-// state update S += Khat^T U; warps 8-11 state epilogue, whose elected thread
-// (warp 8, lane 0) issues [U; O] = [T; R] V + [-W; P] S.  Every bar.sync below
-// is executed by all threads of its group in every iteration (a failed bounded
+// warps 2-3 convert each V slice from bf16 to fp16 in place; warps 4-7 U/O
+// epilogue, whose elected thread (warp 4, lane 0) issues the state update
+// S += Khat^T U; warps 8-11 state epilogue, whose elected thread (warp 8,
+// lane 0) issues [U; O] = [T; R] V + [-W; P] S.  Every bar.sync below is
+// executed by all threads of its group in every iteration (a failed bounded
 // wait only skips work), so a timeout can never leave a barrier half-joined.
 template <int DVS>
 __global__ void __launch_bounds__(384, 1)
@@ -803,6 +835,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                   float *state_out, uint32_t *err) {
     using Lay = BLayout<DVS>;
     constexpr int NSL = D / DVS;
+    constexpr int CPR = DVS / 8;   // 16-byte pieces per V row
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -831,8 +864,10 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     }
     if (tid == 0) {
         for (int i = 0; i < Lay::NST; ++i) {
-            mbar_init(&bars[FULL0 + i], 33);
+            mbar_init(&bars[FULL0 + i], 1);
             mbar_init(&bars[EMPTY0 + i], 1);
+            mbar_init(&bars[VRAW0 + i], 32);
+            mbar_init(&bars[VREADY0 + i], 1);
         }
         mbar_init(&bars[TDFULL0], 1);
         mbar_init(&bars[TDFULL1], 1);
@@ -855,35 +890,22 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     auto stage_addr = [&](int st) { return sbase + st * Lay::kStageR; };
     auto full_par = [&](int j) { return (uint32_t)((j / NST) & 1); };          // FULL[j % NST]
     auto empty_par = [&](int j) { return (uint32_t)(((j / NST) + 1) & 1); };   // EMPTY before reuse
+    auto chunk_len = [&](int j) {
+        const int64_t t0 = ra + (int64_t)j * C;
+        return (int)((rb - t0) < C ? (rb - t0) : C);
+    };
 
     if (warp == 0) {
         // ------------------------------------------------ producer
         // Chunk j's slot image goes in with one bulk copy; its V slice with
-        // cp.async straight into the fp16 operand positions (rows past the end
-        // of the sequence zero-filled), converted from bf16 in place by the lane
-        // that fetched it.  The conversion of chunk j - 1 waits on its own
-        // cp.async group only, so chunk j's loads are already in flight.
-        constexpr int CPR = DVS / 8;   // 16-byte pieces per row
-        auto convert_v = [&](int j) {
-            uint8_t *vt = sm + (j % NST) * Lay::kStageR + kSlotBytes;
-            for (int task = lane; task < 64 * CPR; task += 32) {
-                const int r = task / CPR, ch = task % CPR;
-                uint4 *pc = reinterpret_cast<uint4 *>(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup));
-                float x[8];
-                unpack8(*pc, x);
-                *pc = pack8(x);
-            }
-            fence_async_smem();
-            mbar_arrive(&bars[FULL0 + j % NST]);
-        };
+        // cp.async straight into the operand positions (rows past the end of
+        // the sequence zero-filled), whose landing the lanes report on VRAW.
+        // Nothing here waits for a copy, so loads run NST chunks ahead.
         int issued = 0;
-        bool okp = true;
         for (int j = 0; j < nch; ++j) {
             const int st = j % NST;
-            if (j >= NST && !mbar_wait_abortable(&bars[EMPTY0 + st], empty_par(j), err, abort_flag)) {
-                okp = false;
+            if (j >= NST && !mbar_wait_abortable(&bars[EMPTY0 + st], empty_par(j), err, abort_flag))
                 break;
-            }
             uint8_t *stg = sm + st * Lay::kStageR;
             const uint8_t *src = slots + ((size_t)(c0 + j) * H + h) * kSlotBytes;
             if (lane == 0) {
@@ -891,7 +913,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 bulk_g2s(stg, src, kSlotBytes, &bars[FULL0 + st]);
             }
             const int64_t t0 = ra + (int64_t)j * C;
-            const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+            const int L = chunk_len(j);
             uint8_t *vt = stg + kSlotBytes;
             for (int task = lane; task < 64 * CPR; task += 32) {
                 const int r = task / CPR, ch = task % CPR;
@@ -899,19 +921,35 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 cp_async16(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup),
                            v + ((size_t)(t0 + rr) * H + h) * D + j0 + ch * 8, r < L ? 16u : 0u);
             }
-            cp_async_commit();
+            cp_async_arrive(&bars[VRAW0 + st]);
             issued = j + 1;
-            if (j >= 1) {
-                cp_async_wait_group1();   // chunk j - 1's pieces have landed
-                convert_v(j - 1);
-            }
         }
+        // drain: never leave the CTA with copies still landing in its shared memory
         cp_async_wait_all();
-        if (issued >= 1) convert_v(issued - 1);
-        (void)okp;
-        // drain: never leave the CTA with bulk copies still landing in its shared memory
         for (int j = issued - NST; j < issued; ++j)
             if (j >= 0) mbar_wait(&bars[FULL0 + j % NST], full_par(j), err, 1ull << 28);
+    } else if (warp == 2 || warp == 3) {
+        // ------------------------------------------------ V converters (64 threads)
+        // bf16 -> fp16 in place; each 16-byte piece holds 8 values of one row.
+        const int ct = tid - 64;
+        bool ok = true;
+        for (int j = 0; j < nch; ++j) {
+            const int st = j % NST;
+            if (ok) ok = mbar_wait_abortable(&bars[VRAW0 + st], full_par(j), err, abort_flag);
+            if (ok) {
+                uint8_t *vt = sm + st * Lay::kStageR + kSlotBytes;
+#pragma unroll
+                for (int i = 0; i < CPR; ++i) {
+                    uint4 *pc = reinterpret_cast<uint4 *>(vt) + ct + 64 * i;
+                    float x[8];
+                    unpack8(*pc, x);
+                    *pc = pack8(x);
+                }
+            }
+            fence_async_smem();
+            named_bar(3, 64);
+            if (ct == 0 && ok) mbar_arrive(&bars[VREADY0 + st]);
+        }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------ U / O epilogue (+ state-update issue)
         const int quad = warp - 4;
@@ -925,7 +963,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             if (ok) ok = mbar_wait_abortable(&bars[TDFULL0 + b], (j >> 1) & 1, err, abort_flag);
             tc_fence_after();
             const int64_t t0 = ra + (int64_t)j * C;
-            const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+            const int L = chunk_len(j);
             const int r = row - 64;
             if (ok) {
                 float xa[DVS];
@@ -962,7 +1000,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 fence_async_smem();
                 named_bar(1, 64);   // both U warps (4 and 5) have written their rows
                 if (issuer && ok) {
-                    // and the state is scaled by Gamma_j
+                    // and the state is scaled by Gamma_j (normally long since)
                     ok = mbar_wait_abortable(&bars[TSSCALED], j & 1, err, abort_flag);
                     if (ok) {
                         tc_fence_after();
@@ -996,17 +1034,27 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         const size_t srow = (((size_t)n * H + h) * D + c) * D + j0;
         const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
         uint8_t *sbp = sm + Lay::oSB;
-        auto put_sb = [&](int p, const float *x) {
-            float y0[8], y1[8];
+        // fp16 copy of S (B operand of the state term) and TS <- Gamma * S (the
+        // base the state update accumulates onto), from the fp32 S in xa
+        auto put_state = [&](const float *xa, float gam) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                y0[e] = x[e];
-                y1[e] = x[8 + e];
+            for (int p = 0; p < DVS / 16; ++p) {
+                const float *x = xa + 16 * p;
+                float y0[8], y1[8], z[16];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    y0[e] = x[e];
+                    y1[e] = x[8 + e];
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) z[e] = x[e] * gam;
+                tmem_st16(tS + 16 * p, z);
+                *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p, c, Lay::kKGroup)) =
+                    pack8(y0);
+                *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p + 8, c, Lay::kKGroup)) =
+                    pack8(y1);
             }
-            *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p, c, Lay::kKGroup)) =
-                pack8(y0);
-            *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p + 8, c, Lay::kKGroup)) =
-                pack8(y1);
+            tmem_wait_st();
         };
         // [T; R]_j V_j into TD[j % 2] (the V term; independent of the state)
         int v_issued = -1;   // highest chunk whose V term has been issued (issuer only)
@@ -1021,19 +1069,29 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, kk > 0);
             v_issued = j;
         };
-        // After the fp16 copy of S_j is in place: the elected thread issues
+        auto vterm_ready = [&](int j) {   // one poll: slot, V slice and accumulator free
+            return mbar_try_wait(&bars[FULL0 + j % NST], full_par(j)) &&
+                   mbar_try_wait(&bars[VREADY0 + j % NST], full_par(j)) &&
+                   (j < 2 || mbar_try_wait(&bars[TDEMPTY0 + (j & 1)], ((j >> 1) + 1) & 1));
+        };
+        // After the fp16 copy of S_j and the scaled TS are in place: the elected
+        // thread releases the state update of chunk j (TSSCALED), issues
         // [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j into TD[j % 2] and tells the
-        // group whether it succeeded.  When the next chunk's slot and
-        // accumulator are already free it also issues that chunk's V term, so
-        // that only the state term remains on the chunk-to-chunk path.
+        // group whether it succeeded.  When the next chunk's slot, V slice and
+        // accumulator are already free it also issues that chunk's V term: the
+        // pipe then runs it while the U warps copy U out, and only the state
+        // term remains on the chunk-to-chunk path.
         auto issue_chunk = [&](int j) {
             fence_async_smem();
+            tc_fence_before();
             named_bar(2, 128);
             if (issuer) {
                 const int st = j % NST, b = j & 1;
                 bool okk = *s_grp_ok != 0u;
-                if (v_issued < j) {
-                    if (okk) okk = mbar_wait_abortable(&bars[FULL0 + st], full_par(j), err, abort_flag);
+                if (okk) mbar_arrive(&bars[TSSCALED]);
+                if (okk && v_issued < j) {
+                    okk = mbar_wait_abortable(&bars[FULL0 + st], full_par(j), err, abort_flag);
+                    if (okk) okk = mbar_wait_abortable(&bars[VREADY0 + st], full_par(j), err, abort_flag);
                     if (okk && j >= 2)
                         okk = mbar_wait_abortable(&bars[TDEMPTY0 + b], ((j >> 1) + 1) & 1, err,
                                                   abort_flag);
@@ -1054,8 +1112,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                     mma_commit(&bars[TDFULL0 + b]);
                     // early V term of chunk j + 1, only if nothing has to be waited for
                     const int jn = j + 1;
-                    if (jn < nch && mbar_try_wait(&bars[FULL0 + jn % NST], full_par(jn)) &&
-                        (jn < 2 || mbar_try_wait(&bars[TDEMPTY0 + (jn & 1)], ((jn >> 1) + 1) & 1))) {
+                    if (jn < nch && vterm_ready(jn)) {
                         tc_fence_after();
                         issue_vterm(jn);
                     }
@@ -1064,6 +1121,11 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             }
             named_bar(2, 128);
             return *s_grp_ok != 0u;
+        };
+        auto gamma_of = [&](int j, bool &ok) {
+            if (ok) ok = mbar_wait_abortable(&bars[FULL0 + j % NST], full_par(j), err, abort_flag);
+            return ok ? reinterpret_cast<const float *>(sm + (j % NST) * Lay::kStageR + kSlotGam)[c]
+                      : 0.f;
         };
         if (nch == 0) {
             // empty sequence: the state passes through unchanged
@@ -1074,22 +1136,9 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
             bool ok = true;
-            // S_0: fp16 copy for the first chunk's products
-            for (int p = 0; p < DVS / 16; ++p) {
-                float x[16];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 f = state_in
-                        ? reinterpret_cast<const float4 *>(state_in + srow)[4 * p + i]
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                    x[4 * i] = f.x; x[4 * i + 1] = f.y; x[4 * i + 2] = f.z; x[4 * i + 3] = f.w;
-                }
-                put_sb(p, x);
-            }
-            ok = issue_chunk(0);
-            // x = S_j in registers (fp32); TS <- Gamma_j S_j; then wait for the
-            // update S_{j+1} = TS + Khat_j^T U_j, copy it to fp16 for the next
-            // chunk's products, and keep it in registers for the next scaling.
+            // xa = S_j in registers (fp32).  Per chunk: S_j -> fp16 copy and
+            // TS = Gamma_j S_j, the chunk products are issued, and the state
+            // update S_{j+1} = TS + Khat_j^T U_j lands in TS.
             float xa[DVS];
             for (int p = 0; p < DVS / 16; ++p)
 #pragma unroll
@@ -1100,23 +1149,13 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                     xa[16 * p + 4 * i] = f.x; xa[16 * p + 4 * i + 1] = f.y;
                     xa[16 * p + 4 * i + 2] = f.z; xa[16 * p + 4 * i + 3] = f.w;
                 }
+            {
+                const float gam = gamma_of(0, ok);
+                if (ok) put_state(xa, gam);
+                if (issuer) *s_grp_ok = ok ? 1u : 0u;
+                ok = issue_chunk(0) && ok;
+            }
             for (int j = 0; j < nch; ++j) {
-                float gam = 0.f;
-                if (ok) ok = mbar_wait_abortable(&bars[FULL0 + j % NST], full_par(j), err, abort_flag);
-                if (ok) gam = reinterpret_cast<const float *>(sm + (j % NST) * Lay::kStageR + kSlotGam)[c];
-                if (ok) {
-#pragma unroll
-                    for (int p = 0; p < DVS / 16; ++p) {
-                        float x[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) x[e] = xa[16 * p + e] * gam;
-                        tmem_st16(tS + 16 * p, x);
-                    }
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                named_bar(2, 128);
-                if (issuer) mbar_arrive(&bars[TSSCALED]);
                 // S_{j+1} = TS after the state update of chunk j
                 if (ok) ok = mbar_wait_abortable(&bars[TSFULL], j & 1, err, abort_flag);
                 tc_fence_after();
@@ -1127,10 +1166,8 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                     tmem_wait_ld();
                 }
                 if (j + 1 == nch) break;
-                if (ok) {
-#pragma unroll
-                    for (int p = 0; p < DVS / 16; ++p) put_sb(p, xa + 16 * p);
-                }
+                const float gam = gamma_of(j + 1, ok);
+                if (ok) put_state(xa, gam);
                 if (issuer) *s_grp_ok = ok ? 1u : 0u;
                 const bool ok2 = issue_chunk(j + 1);
                 ok = ok && ok2;

@@ -220,9 +220,14 @@ constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x
 constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128          16 KiB
 constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 solve scratch (32 x 32)               4 KiB
 constexpr uint32_t A_QP = A_AK;               // bf16 q rows [64][128] for P, once T is out  16 KiB
+// next item's rows, prefetched once D1 has completed (all of the above but A_QP is dead)
+constexpr uint32_t A_QST = A_OPS + 16384;     // bf16 q [64][128], pieces permuted per row   16 KiB
+constexpr uint32_t A_KST = A_OPS + 32768;     // bf16 k, same layout                         16 KiB
+constexpr uint32_t A_GST = A_OPS + 49152;     // bf16 g [64][128]                            16 KiB
 constexpr uint32_t A_SMEM = A_OPS + 2 * A_RBUF + 1024;   // + alignment slack (= 112640)
 static_assert(A_Y + 4096 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
-static_assert(A_OPS + 4096 + 16384 <= A_OPS + A_RBUF, "g staging must fit in round buffer 0");
+static_assert(A_QST >= A_QP + 16384 && A_GST + 16384 <= A_OPS + 2 * A_RBUF, "staging area");
+static_assert(3 * 128 * 4 + 128 * 4 <= 16384, "A0 scratch (tot, G_L) must not reach the staging area");
 static_assert(A_OPS % 1024 == 0 && A_RBUF % 1024 == 0 && A_AQ % 1024 == 0 && A_TR % 1024 == 0 &&
               A_KT % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // E1 is stored [64][128] fp32 with its 16-byte pieces (4 channels) permuted per
@@ -285,91 +290,100 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     float *Yb = reinterpret_cast<float *>(sm + A_Y);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int h = blockIdx.y;
     const int32_t *chunk_off = reinterpret_cast<const int32_t *>(ws);
-    const int cidx = blockIdx.x;
-    int64_t t0;
-    int L;
-    if (cu == nullptr) {
-        // equal-length batch: chunk -> (sequence, start) by arithmetic, no table read
-        const int64_t cps = (T + C - 1) / C;
-        const int64_t n = cidx / cps, j = cidx - n * cps;
-        if (n >= N) return;
-        t0 = n * T + j * C;
-        L = (int)((T - j * C) < C ? (T - j * C) : C);
-    } else {
-        const int total = chunk_off[N];
-        if (cidx >= total) return;
-        // sequence owning this chunk: last n with chunk_off[n] <= cidx
-        int lo = 0, hi = N - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (chunk_off[mid] <= cidx) lo = mid; else hi = mid - 1;
+    // items are (chunk, head) pairs, item = chunk * H + head, which is also the
+    // index of the item's workspace slot
+    const int64_t cps = (T + C - 1) / C;
+    const int64_t n_items = (cu == nullptr ? (int64_t)N * cps : (int64_t)chunk_off[N]) * H;
+    // first row and length of an item's chunk
+    auto locate = [&](int64_t item, int64_t &t0_, int &L_) {
+        const int64_t cidx = item / H;
+        if (cu == nullptr) {
+            // equal-length batch: chunk -> (sequence, start) by arithmetic, no table read
+            const int64_t n = cidx / cps, j = cidx - n * cps;
+            t0_ = n * T + j * C;
+            L_ = (int)((T - j * C) < C ? (T - j * C) : C);
+        } else {
+            // sequence owning this chunk: last n with chunk_off[n] <= cidx
+            int lo = 0, hi = N - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (chunk_off[mid] <= cidx) lo = mid; else hi = mid - 1;
+            }
+            int64_t ra, rb;
+            seq_rows(chunk_off, true, T, N, lo, ra, rb);
+            t0_ = ra + (cidx - chunk_off[lo]) * C;
+            L_ = (int)((rb - t0_) < C ? (rb - t0_) : C);
         }
-        int64_t ra, rb;
-        seq_rows(chunk_off, true, T, N, lo, ra, rb);
-        t0 = ra + (int64_t)(cidx - chunk_off[lo]) * C;
-        L = (int)((rb - t0) < C ? (rb - t0) : C);
-    }
-    uint8_t *slot = ws + header_bytes(N) + ((size_t)cidx * H + h) * kSlotBytes;
-    auto row_ptr = [&](const __nv_bfloat16 *base, int r) {
-        return base + ((size_t)(t0 + r) * H + h) * D;
     };
 
-    // ---- issue every global load of the operand rounds up front (one round trip)
     // round task: lane -> 4-channel piece p_l of the round and two token rows, one
     // in the first and one in the second half of the chunk, paired so that every
     // warp writes the same number of packed K^(a) copies (rows of block b have
     // 4 - b of them): warps 0-3 take blocks 0 and 3, warps 4-7 blocks 1 and 2
     const int p_l = lane & 7, rsub = lane >> 3;
     auto a1_row = [&](int it) { return it == 0 ? 4 * warp + rsub : 32 + 4 * (warp ^ 4) + rsub; };
-    uint2 qv[4][2], kv[4][2];
+
+    // Next item's q, k, g rows go to the staging area with cp.async (rows past
+    // the chunk zero-filled) while the current item finishes; beta into a
+    // register.  q and k rows have their 16-byte piece p at p ^ 4 (r % 4) so the
+    // operand-round reads below are free of bank conflicts; g is row-major.
+    float bnext = 0.f;
+    auto prefetch = [&](int64_t item) {
+        int64_t t0n;
+        int Ln;
+        locate(item, t0n, Ln);
+        const int hn = (int)(item % H);
 #pragma unroll
-    for (int rd = 0; rd < 4; ++rd)
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const int r = a1_row(it);
-            const int c0 = 32 * rd + 4 * p_l;
-            if (r < L) {
-                qv[rd][it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(q, r) + c0));
-                kv[rd][it] = __ldg(reinterpret_cast<const uint2 *>(row_ptr(k, r) + c0));
-            } else {
-                qv[rd][it] = make_uint2(0u, 0u);
-                kv[rd][it] = make_uint2(0u, 0u);
-            }
+        for (int i = 0; i < 4; ++i) {
+            const int task = tid + 256 * i, r = task >> 4, pc = task & 15;
+            const size_t off = ((size_t)(t0n + (r < Ln ? r : 0)) * H + hn) * D + pc * 8;
+            const uint32_t src_bytes = r < Ln ? 16u : 0u;
+            const uint32_t sw = (uint32_t)(r * 256 + ((pc ^ ((r & 3) << 2)) << 4));
+            cp_async16(sm + A_QST + sw, q + off, src_bytes);
+            cp_async16(sm + A_KST + sw, k + off, src_bytes);
+            cp_async16(sm + A_GST + task * 16, g + off, src_bytes);
         }
-    // g: coalesced 16-byte loads, staged as bf16 [64][128] in the (still idle) operand region
-    uint4 gv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int task = tid + 256 * i, r = task >> 4, cc = (task & 15) * 8;
-        gv[i] = r < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(g, r) + cc))
-                      : make_uint4(0u, 0u, 0u, 0u);
-    }
-    const float bval = (tid < L) ? __bfloat162float(beta[(size_t)(t0 + (tid < 64 ? tid : 0)) * H + h]) : 0.f;
-    __nv_bfloat16 *gst = reinterpret_cast<__nv_bfloat16 *>(sm + A_OPS + 4096);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int task = tid + 256 * i;
-        reinterpret_cast<uint4 *>(gst)[task] = gv[i];
-    }
-    if (tid < 64) bs[tid] = bval;
-    __syncthreads();
-    const int c = tid & 127, half = tid >> 7;
-    float p[32];   // clamped log-decay of rows 32*half + i, then its prefix sums
-#pragma unroll
-    for (int i = 0; i < 32; ++i) p[i] = fmaxf(__bfloat162float(gst[(half * 32 + i) * D + c]), -5.f);
+        bnext = (tid < Ln) ? __bfloat162float(beta[(size_t)(t0n + (tid < 64 ? tid : 0)) * H + hn]) : 0.f;
+    };
 
     if (warp == 0) {
         tmem_alloc(tmem_ptr, 256);
         tmem_relinquish();
-        tc_fence_before();
     }
     if (tid == 32) {
         for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
         *abort_flag = 0u;
     }
+    if ((int64_t)blockIdx.x < n_items) prefetch(blockIdx.x);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+
+    uint32_t ph = 0;   // mbarrier phase parity: each barrier completes once per item
+    // (items fit in int32: the host checks max_chunks * H against INT32_MAX)
+    for (int item = blockIdx.x; item < (int)n_items; item += gridDim.x, ph ^= 1u) {
+    const int h = (int)(item % H);
+    int64_t t0;
+    int L;
+    locate(item, t0, L);
+    uint8_t *slot = ws + header_bytes(N) + (size_t)item * kSlotBytes;
+    auto row_ptr = [&](const __nv_bfloat16 *base, int r) {
+        return base + ((size_t)(t0 + r) * H + h) * D;
+    };
+
+    // ---- this item's rows have landed (each thread waits for its own copies)
+    cp_async_wait_all();
+    if (__syncthreads_or(*abort_flag != 0u)) break;
+    const __nv_bfloat16 *gst = reinterpret_cast<const __nv_bfloat16 *>(sm + A_GST);
+    const int c = tid & 127, half = tid >> 7;
+    float p[32];   // clamped log-decay of rows 32*half + i, then its prefix sums
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = fmaxf(__bfloat162float(gst[(half * 32 + i) * D + c]), -5.f);
+    if (tid < 64) bs[tid] = bnext;
+    __syncthreads();
 
     // ---- A0: chunk-local cumsum (fp32) and E1 = exp(G - R_a), per channel c and half
     // G_r - R_a(r) = p_i for the first 16 rows of a half and p_i - p_15 for the
@@ -415,6 +429,19 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         EL[384 + c] = __expf(gl - r3);
         GamL[c] = __expf(gl);
     }
+    // q, k of the operand rounds into registers; the staging area is free after the barrier
+    uint2 qv[4][2], kv[4][2];
+#pragma unroll
+    for (int rd = 0; rd < 4; ++rd)
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const int r = a1_row(it);
+            const int c0 = 32 * rd + 4 * p_l;   // 16-byte piece c0 / 8, 8-byte half (c0 / 4) & 1
+            const uint32_t sw =
+                (uint32_t)(r * 256 + (((c0 >> 3) ^ ((r & 3) << 2)) << 4) + ((c0 >> 2) & 1) * 8);
+            qv[rd][it] = *reinterpret_cast<const uint2 *>(sm + A_QST + sw);
+            kv[rd][it] = *reinterpret_cast<const uint2 *>(sm + A_KST + sw);
+        }
     __syncthreads();
 
     // ---- A1: Akk / Aqk on tensor cores (tf32), four double-buffered rounds of 32 channels.
@@ -427,7 +454,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
     for (int rd = 0; rd < 4; ++rd) {
         const uint32_t buf = A_OPS + (rd & 1) * A_RBUF;
-        if (rd >= 2 && ok) ok = mbar_wait_abortable(&bars[rd - 2], 0, err, abort_flag);
+        if (rd >= 2 && ok) ok = mbar_wait_abortable(&bars[rd - 2], ph, err, abort_flag);
         if (ok) {
             const int c0 = 32 * rd + 4 * p_l;
 #pragma unroll
@@ -453,7 +480,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         __syncthreads();
         tc_fence_after();
         if (ok && tid == 0) {
-            const uint32_t tm = *tmem_ptr;
+            const uint32_t tm = tmem;
             const uint32_t id = idesc(FMT_TF32, 64, 32, 0, 0);
             for (int a = 0; a < 4; ++a)
                 for (int kk = 0; kk < 4; ++kk) {          // 4 steps of K=8 over 32 channels
@@ -476,11 +503,29 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                                : make_uint4(0u, 0u, 0u, 0u);
         }
     }
-    if (ok) ok = mbar_wait_abortable(&bars[3], 0, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[3], ph, err, abort_flag);
     tc_fence_after();
-    const uint32_t tmem = *tmem_ptr;
 
-    // ---- A2: Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal,
+    // ---- A2 (warps 4-7): K*Gamma = k E1 prod_{m<a} F_m as the MN-major B operand of
+    // W = T (K*Gamma).  (This branch comes first in program order so that its
+    // prefetched rows are dead before the other branch: fewer live registers.)
+    if (ok && warp >= 4) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int task = (tid - 128) + 128 * i, s = task >> 4, cc = (task & 15) * 8;
+            float x[8];
+            unpack8(kt_pref[i], x);
+            const int a = s >> 4;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+                float4 e = ld4(E1 + e1_at(s, cc + 4 * hv));
+                for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
+                x[4 * hv] *= e.x; x[4 * hv + 1] *= e.y; x[4 * hv + 2] *= e.z; x[4 * hv + 3] *= e.w;
+            }
+            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(cc, s, kKhMNBlock)) = pack8(x);
+        }
+    }
+    // ---- A2 (warps 0-3): Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal,
     // MN-major: element (r, s) at (mn = r, k = s), so a thread's 16 rows are 32 contiguous bytes)
     if (ok && warp < 4) {
         const int s = 16 * warp + (lane & 15);
@@ -504,39 +549,10 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
         }
     }
-    // K*Gamma = k E1 prod_{m<a} F_m as the MN-major B operand of W = T (K*Gamma)
-    if (ok && warp >= 4) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int task = (tid - 128) + 128 * i, s = task >> 4, cc = (task & 15) * 8;
-            float x[8];
-            unpack8(kt_pref[i], x);
-            const int a = s >> 4;
-#pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-                float4 e = ld4(E1 + e1_at(s, cc + 4 * hv));
-                for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
-                x[4 * hv] *= e.x; x[4 * hv + 1] *= e.y; x[4 * hv + 2] *= e.z; x[4 * hv + 3] *= e.w;
-            }
-            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(cc, s, kKhMNBlock)) = pack8(x);
-        }
-    }
     tc_fence_before();
     __syncthreads();
 
-    // Khat = k EL / E1 for the slot, by warps 2-7 while warps 0-1 run the
-    // diagonal blocks of the solve below; its loads go out now
-    constexpr int KH_TASKS = 6;   // 1024 8-channel pieces over 192 threads
-    uint4 kh_pref[KH_TASKS];
-    if (warp >= 2) {
-#pragma unroll
-        for (int i = 0; i < KH_TASKS; ++i) {
-            const int task = (tid - 64) + 192 * i, s = task >> 4, cc = (task & 15) * 8;
-            kh_pref[i] = (task < 1024 && s < L)
-                ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
-                : make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
+    constexpr int KH_TASKS = 6;   // Khat: 1024 8-channel pieces over the 192 threads of warps 2-7
 
     // ---- A3: X = (I + Akk)^-1 in place over AK (fp32), by 2x2 block merges:
     //   inv([[L11, 0], [L21, L22]]) = [[X11, 0], [-X22 (L21 X11), X22]]
@@ -546,16 +562,17 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     {
         float x[16];
         const int a = tid >> 4, j = tid & 15, o = 16 * a;
-        if (ok && tid < 64) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float acc = (i == j) ? 1.f : 0.f;
-#pragma unroll
-                for (int m = 0; m < i; ++m) acc = fmaf(-AK[(o + i) * 64 + o + m], x[m], acc);
-                x[i] = acc;
-            }
-        }
+        // Khat = k EL / E1 for the slot, by warps 2-7 while warps 0-1 run the
+        // diagonal blocks of the solve (whose latency also covers these loads)
         if (ok && warp >= 2) {
+            uint4 kh_pref[KH_TASKS];
+#pragma unroll
+            for (int i = 0; i < KH_TASKS; ++i) {
+                const int task = (tid - 64) + 192 * i, s = task >> 4, cc = (task & 15) * 8;
+                kh_pref[i] = (task < 1024 && s < L)
+                    ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
+                    : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
             for (int i = 0; i < KH_TASKS; ++i) {
                 const int task = (tid - 64) + 192 * i, s = task >> 4, cc = (task & 15) * 8;
@@ -572,6 +589,15 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 }
             }
             if (tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = GamL[tid - 128];
+        }
+        if (ok && tid < 64) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float acc = (i == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int m = 0; m < i; ++m) acc = fmaf(-AK[(o + i) * 64 + o + m], x[m], acc);
+                x[i] = acc;
+            }
         }
         __syncthreads();
         if (ok && tid < 64) {
@@ -690,24 +716,25 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         mma_commit(&bars[4]);
     }
-    if (ok) ok = mbar_wait_abortable(&bars[4], 0, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[4], ph, err, abort_flag);
     tc_fence_after();
     if (ok && warp < 4) {
         const int r = 16 * warp + (lane & 15);
-        float x[64];
-        tmem_ld16(taddr(tmem, 32 * warp, 128), *reinterpret_cast<float(*)[16]>(x));
-        tmem_ld16(taddr(tmem, 32 * warp, 144), *reinterpret_cast<float(*)[16]>(x + 16));
-        tmem_ld16(taddr(tmem, 32 * warp, 160), *reinterpret_cast<float(*)[16]>(x + 32));
-        tmem_ld16(taddr(tmem, 32 * warp, 176), *reinterpret_cast<float(*)[16]>(x + 48));
-        tmem_wait_ld();
-        if (lane < 16) {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                float y[8];
+        for (int hh = 0; hh < 2; ++hh) {
+            float x[32];
+            tmem_ld16(taddr(tmem, 32 * warp, 128 + 32 * hh), *reinterpret_cast<float(*)[16]>(x));
+            tmem_ld16(taddr(tmem, 32 * warp, 144 + 32 * hh), *reinterpret_cast<float(*)[16]>(x + 16));
+            tmem_wait_ld();
+            if (lane < 16) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = x[ch * 8 + e];
-                *reinterpret_cast<uint4 *>(sm + A_TR + sw128_kmajor_off(64 + r, ch * 8, 0)) =
-                    pack8(y);
+                for (int ch = 0; ch < 4; ++ch) {
+                    float y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = x[ch * 8 + e];
+                    *reinterpret_cast<uint4 *>(sm + A_TR + sw128_kmajor_off(64 + r, 32 * hh + ch * 8, 0)) =
+                        pack8(y);
+                }
             }
         }
     }
@@ -729,55 +756,68 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     const int quad = warp & 3, chalf = warp >> 2;
     const int row6 = 32 * quad + lane, r6 = row6 & 63;
-    // [T; R] is final: copy it to the slot while the MMA runs (reads only)
-    if (ok) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(sm + A_TR);
-        uint4 *dst = reinterpret_cast<uint4 *>(slot + kSlotTR);
-        for (int i = tid; i < 16384 / 16; i += 256) dst[i] = src[i];
+    // [T; R] is final: one bulk store to the slot while the MMA runs
+    if (ok && tid == 0) {
+        bulk_s2g(slot + kSlotTR, sm + A_TR, 16384);
+        bulk_commit();
     }
-    if (ok) ok = mbar_wait_abortable(&bars[5], 0, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[5], ph, err, abort_flag);
     tc_fence_after();
+    // the operand tiles are free once D1 has completed and the bulk store has
+    // read [T; R]: the next item's rows go out now
+    if (tid == 0) bulk_wait_read();
+    __syncthreads();
+    if (ok && (int64_t)item + gridDim.x < n_items) prefetch(item + gridDim.x);
 
-    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = q Gamma - R (K*Gamma)
+    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = q Gamma - R (K*Gamma), in two
+    // halves of 32 columns (fewer live registers)
     if (ok) {
-        float x[64];
+        const int a = r6 >> 4;
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp)
-            tmem_ld16(taddr(tmem, 32 * quad, 64 * chalf + 16 * pp),
-                      *reinterpret_cast<float(*)[16]>(x + 16 * pp));
-        tmem_wait_ld();
-        if (row6 < 64) {
+        for (int hh = 0; hh < 2; ++hh) {
+            float x[32];
+            tmem_ld16(taddr(tmem, 32 * quad, 64 * chalf + 32 * hh), *reinterpret_cast<float(*)[16]>(x));
+            tmem_ld16(taddr(tmem, 32 * quad, 64 * chalf + 32 * hh + 16),
+                      *reinterpret_cast<float(*)[16]>(x + 16));
+            tmem_wait_ld();
+            if (row6 < 64) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) x[i] = -x[i];
-        } else {
-            const int a = r6 >> 4;
+                for (int i = 0; i < 32; ++i) x[i] = -x[i];
+            } else {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const int cc = 64 * chalf + ch * 8;
-                float qv8[8];
-                unpack8(reinterpret_cast<const uint4 *>(sm + A_QP)[r6 * 16 + ((8 * chalf + ch) ^ (r6 & 15))],
-                        qv8);
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int pc = 8 * chalf + 4 * hh + ch, cc = 8 * pc;
+                    float qv8[8];
+                    unpack8(reinterpret_cast<const uint4 *>(sm + A_QP)[r6 * 16 + (pc ^ (r6 & 15))], qv8);
 #pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    float4 e = ld4(E1 + e1_at(r6, cc + 4 * hv));
-                    for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
-                    x[ch * 8 + 4 * hv] = qv8[4 * hv] * e.x - x[ch * 8 + 4 * hv];
-                    x[ch * 8 + 4 * hv + 1] = qv8[4 * hv + 1] * e.y - x[ch * 8 + 4 * hv + 1];
-                    x[ch * 8 + 4 * hv + 2] = qv8[4 * hv + 2] * e.z - x[ch * 8 + 4 * hv + 2];
-                    x[ch * 8 + 4 * hv + 3] = qv8[4 * hv + 3] * e.w - x[ch * 8 + 4 * hv + 3];
+                    for (int hv = 0; hv < 2; ++hv) {
+                        float4 e = ld4(E1 + e1_at(r6, cc + 4 * hv));
+                        for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
+                        float *xx = x + ch * 8 + 4 * hv;
+                        xx[0] = qv8[4 * hv] * e.x - xx[0];
+                        xx[1] = qv8[4 * hv + 1] * e.y - xx[1];
+                        xx[2] = qv8[4 * hv + 2] * e.z - xx[2];
+                        xx[3] = qv8[4 * hv + 3] * e.w - xx[3];
+                    }
                 }
             }
-        }
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-            float y[8];
+            for (int ch = 0; ch < 4; ++ch) {
+                float y[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = x[ch * 8 + e];
-            *reinterpret_cast<uint4 *>(slot + kSlotWP +
-                                       sw128_kmajor_off(row6, 64 * chalf + ch * 8, kWPKBlock)) =
-                pack8(y);
+                for (int e = 0; e < 8; ++e) y[e] = x[ch * 8 + e];
+                *reinterpret_cast<uint4 *>(
+                    slot + kSlotWP + sw128_kmajor_off(row6, 64 * chalf + 32 * hh + ch * 8, kWPKBlock)) =
+                    pack8(y);
+            }
         }
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    }   // item loop
+    cp_async_wait_all();
+    if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -1234,9 +1274,14 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
         e = cudaFuncSetAttribute(tc::intra_chunk_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::A_SMEM);
         if (e != cudaSuccess) return e;
-        if (max_chunks > INT32_MAX || a.H > 65535) return cudaErrorInvalidValue;
-        dim3 grid((unsigned)max_chunks, (unsigned)a.H);
-        tc::intra_chunk_kernel<<<grid, 256, tc::A_SMEM, st>>>(
+        // persistent: two CTAs per SM walk the (chunk, head) items
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t items = max_chunks * a.H;
+        if (items > INT32_MAX - 65536) return cudaErrorInvalidValue;
+        const int64_t ctas = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
+        tc::intra_chunk_kernel<<<(unsigned)ctas, 256, tc::A_SMEM, st>>>(
             (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
             (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, ws, a.err);
         e = cudaGetLastError();

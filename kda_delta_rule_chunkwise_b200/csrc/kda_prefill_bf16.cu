@@ -5,16 +5,17 @@
 // "Kimi K3 ... overview", section "Sequence length: hybrid KDA and Gated MLA
 // attention") is evaluated in chunks of C = 64 tokens in two kernels:
 //
-// Phase A, intra_chunk_kernel (one CTA per (chunk, head), all in parallel):
+// Phase A, intra_chunk_kernel (persistent: two CTAs per SM walk the
+// (chunk, head) items; the next item's rows are prefetched while one finishes):
 //   G     chunk-local inclusive cumsum of max(g, -5)                     (fp32)
 //   Akk, Aqk  decay-rescaled intra-chunk products on tensor cores.  The
 //         pairwise decay exp(G_r - G_s) is split as
 //         exp(G_r - R_a) * exp(R_a - G_s), R_a = G at the end of the
-//         previous 16-row block a.  Both factors stay inside the bf16
-//         exponent range because g >= -5: the first is in [e^-80, 1], the
-//         second <= e^75.  That bound is what lets every tile (diagonal ones
-//         included) run as a dense bf16 MMA; it is the point of the lower
-//         bound on the log-decay in the section cited above.
+//         previous 16-row block a.  Because g >= -5 the first factor is in
+//         [e^-80, 1] and the second at most e^80, inside the fp32 exponent
+//         range of tf32 operands.  That bound is what lets every tile
+//         (diagonal ones included) run as a dense MMA; it is the point of the
+//         lower bound on the log-decay in the section cited above.
 //   T     = (I + Akk)^-1 Diag(beta): blocked unit-lower-triangular inverse,
 //         fp32 (the UT/WY step that turns the sequential delta rule into
 //         matrix products)
@@ -30,12 +31,12 @@
 // With U = T V - W S this is the WY form: U are the chunk's pseudo-values and
 // O = Q*exp(G) S + Aqk U, the chunk's outputs.
 //
-// Roles in phase B: warp 0 = producer (1-D bulk copy of the slot, V slice
-// converted to fp16), warp 1 = TMEM owner, warps 4-7 = U/O epilogue (TMEM ->
-// registers; its elected thread issues the state update), warps 8-11 = state
-// epilogue (Gamma scaling of the TMEM state, fp16 copy of S; its elected
-// thread issues the chunk products).  Each chunk costs two hand-offs: state
-// copy -> chunk products -> U copy -> state update -> state copy.
+// Roles in phase B: warp 0 = producer (1-D bulk copy of the slot, cp.async of
+// the V slice), warp 1 = TMEM owner, warps 2-3 convert V to fp16 in place,
+// warps 4-7 = U/O epilogue (TMEM -> registers; its elected thread issues the
+// state update), warps 8-11 = state epilogue (fp16 copy of S, Gamma scaling of
+// the TMEM state; its elected thread issues the chunk products).  Each chunk
+// costs two hand-offs: state copy -> chunk products -> U copy -> state update.
 //
 // Precision.  Inputs are bf16; every product accumulates in fp32 (TMEM); the
 // state and the outputs o are fp32.  The decay-rescaled operands of Akk/Aqk
@@ -167,6 +168,17 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
 // four fp32 values rounded to tf32, as one 16-byte word
 __device__ __forceinline__ float4 pack4_tf32(float a, float b, float c, float d) {
     return make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
+}
+
+// eight fp16 -> fp32
+__device__ __forceinline__ void unpack8h(uint4 u, float (&x)[8]) {
+    const __half2 *p = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(p[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
 }
 
 __device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
@@ -480,39 +492,36 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         __syncthreads();
         tc_fence_after();
         if (ok && tid == 0) {
-            const uint32_t tm = tmem;
+            // descriptors advance by their start-address field (address / 16)
+            const uint64_t ad0 = smem_desc(sbase + buf + A_AT, 16, 1024, SW_128B);
+            const uint64_t bd0 = smem_desc(sbase + buf + A_BT, 16, 1024, SW_128B);
             const uint32_t id = idesc(FMT_TF32, 64, 32, 0, 0);
+#pragma unroll
             for (int a = 0; a < 4; ++a)
-                for (int kk = 0; kk < 4; ++kk) {          // 4 steps of K=8 over 32 channels
-                    const uint64_t ad = smem_desc(sbase + buf + A_AT + at_group(a) * 1024 + kk * 32,
-                                                  16, 1024, SW_128B);
-                    const uint64_t bd = smem_desc(sbase + buf + A_BT + (4 * a) * 1024 + kk * 32, 16,
-                                                  1024, SW_128B);
-                    mma_tf32(tm + 32 * a, ad, bd, id, (rd > 0 || kk > 0) ? 1u : 0u);
-                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)            // 4 steps of K=8 over 32 channels
+                    mma_tf32(tmem + 32 * a, ad0 + (uint64_t)((at_group(a) * 1024 + kk * 32) >> 4),
+                             bd0 + (uint64_t)((4 * a * 1024 + kk * 32) >> 4), id,
+                             (rd > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&bars[rd]);
         }
     }
-    // next loads (K*Gamma operand, warps 4-7) go out before the last MMA wait
-    uint4 kt_pref[8];
-    if (warp >= 4) {
+    // next loads (the K*Gamma operand, 4 pieces per thread) go out before the last MMA wait
+    uint4 kt_pref[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int task = (tid - 128) + 128 * i, s = task >> 4, cc = (task & 15) * 8;
-            kt_pref[i] = s < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
-                               : make_uint4(0u, 0u, 0u, 0u);
-        }
+    for (int i = 0; i < 4; ++i) {
+        const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
+        kt_pref[i] = s < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
+                           : make_uint4(0u, 0u, 0u, 0u);
     }
     if (ok) ok = mbar_wait_abortable(&bars[3], ph, err, abort_flag);
     tc_fence_after();
 
-    // ---- A2 (warps 4-7): K*Gamma = k E1 prod_{m<a} F_m as the MN-major B operand of
-    // W = T (K*Gamma).  (This branch comes first in program order so that its
-    // prefetched rows are dead before the other branch: fewer live registers.)
-    if (ok && warp >= 4) {
+    // ---- A2: K*Gamma = k E1 prod_{m<a} F_m as the MN-major B operand of W = T (K*Gamma)
+    if (ok) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int task = (tid - 128) + 128 * i, s = task >> 4, cc = (task & 15) * 8;
+        for (int i = 0; i < 4; ++i) {
+            const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
             float x[8];
             unpack8(kt_pref[i], x);
             const int a = s >> 4;
@@ -525,14 +534,17 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(cc, s, kKhMNBlock)) = pack8(x);
         }
     }
-    // ---- A2 (warps 0-3): Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal,
-    // MN-major: element (r, s) at (mn = r, k = s), so a thread's 16 rows are 32 contiguous bytes)
-    if (ok && warp < 4) {
-        const int s = 16 * warp + (lane & 15);
-        for (int a = 0; a < 4; ++a) {
+    // and Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal,
+    // MN-major: element (r, s) at (mn = r, k = s), so a thread's 16 rows are 32 contiguous
+    // bytes) out of TMEM.  Warps w and w + 4 share TMEM lanes 32 (w % 4) ...; the first
+    // takes row blocks a = 0, 1 and the second a = 2, 3.
+    if (ok) {
+        const int quad = warp & 3, s = 16 * quad + (lane & 15);
+        const int a0 = 2 * (warp >> 2);
+        for (int a = a0; a < a0 + 2; ++a) {
             float vq[16], vk[16];
-            tmem_ld16(taddr(tmem, 32 * warp, 32 * a), vq);
-            tmem_ld16(taddr(tmem, 32 * warp, 32 * a + 16), vk);
+            tmem_ld16(taddr(tmem, 32 * quad, 32 * a), vq);
+            tmem_ld16(taddr(tmem, 32 * quad, 32 * a + 16), vk);
             tmem_wait_ld();
             if (lane < 16) {
                 float y0[8], y1[8];
@@ -761,6 +773,25 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         bulk_s2g(slot + kSlotTR, sm + A_TR, 16384);
         bulk_commit();
     }
+    // meanwhile every thread turns its staged q pieces into Q*Gamma = q E1 prod_{m<a} F_m
+    // (fp16, in place), so that A6's P rows only subtract
+    if (ok) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int task = tid + 256 * i, r = task >> 4, pc = task & 15, cc = 8 * pc;
+            uint4 *qp = reinterpret_cast<uint4 *>(sm + A_QP) + r * 16 + (pc ^ (r & 15));
+            float x[8];
+            unpack8(*qp, x);
+            const int a = r >> 4;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+                float4 e = ld4(E1 + e1_at(r, cc + 4 * hv));
+                for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
+                x[4 * hv] *= e.x; x[4 * hv + 1] *= e.y; x[4 * hv + 2] *= e.z; x[4 * hv + 3] *= e.w;
+            }
+            *qp = pack8(x);
+        }
+    }
     if (ok) ok = mbar_wait_abortable(&bars[5], ph, err, abort_flag);
     tc_fence_after();
     // the operand tiles are free once D1 has completed and the bulk store has
@@ -769,10 +800,9 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
     if (ok && (int64_t)item + gridDim.x < n_items) prefetch(item + gridDim.x);
 
-    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = q Gamma - R (K*Gamma), in two
+    // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = Q*Gamma - R (K*Gamma), in two
     // halves of 32 columns (fewer live registers)
     if (ok) {
-        const int a = r6 >> 4;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             float x[32];
@@ -780,35 +810,26 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             tmem_ld16(taddr(tmem, 32 * quad, 64 * chalf + 32 * hh + 16),
                       *reinterpret_cast<float(*)[16]>(x + 16));
             tmem_wait_ld();
-            if (row6 < 64) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = -x[i];
-            } else {
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int pc = 8 * chalf + 4 * hh + ch, cc = 8 * pc;
-                    float qv8[8];
-                    unpack8(reinterpret_cast<const uint4 *>(sm + A_QP)[r6 * 16 + (pc ^ (r6 & 15))], qv8);
-#pragma unroll
-                    for (int hv = 0; hv < 2; ++hv) {
-                        float4 e = ld4(E1 + e1_at(r6, cc + 4 * hv));
-                        for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
-                        float *xx = x + ch * 8 + 4 * hv;
-                        xx[0] = qv8[4 * hv] * e.x - xx[0];
-                        xx[1] = qv8[4 * hv + 1] * e.y - xx[1];
-                        xx[2] = qv8[4 * hv + 2] * e.z - xx[2];
-                        xx[3] = qv8[4 * hv + 3] * e.w - xx[3];
-                    }
-                }
-            }
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float y[8];
+                uint4 u;
+                if (row6 < 64) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = x[ch * 8 + e];
+                    for (int e = 0; e < 8; ++e) y[e] = x[ch * 8 + e];
+                    u = pack8(y);
+                    u.x ^= 0x80008000u; u.y ^= 0x80008000u;   // -W: flip the fp16 signs
+                    u.z ^= 0x80008000u; u.w ^= 0x80008000u;
+                } else {
+                    const int pc = 8 * chalf + 4 * hh + ch;
+                    float qg[8];
+                    unpack8h(reinterpret_cast<const uint4 *>(sm + A_QP)[r6 * 16 + (pc ^ (r6 & 15))], qg);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = qg[e] - x[ch * 8 + e];
+                    u = pack8(y);
+                }
                 *reinterpret_cast<uint4 *>(
-                    slot + kSlotWP + sw128_kmajor_off(row6, 64 * chalf + 32 * hh + ch * 8, kWPKBlock)) =
-                    pack8(y);
+                    slot + kSlotWP + sw128_kmajor_off(row6, 64 * chalf + 32 * hh + ch * 8, kWPKBlock)) = u;
             }
         }
     }

@@ -252,18 +252,22 @@ __device__ __forceinline__ int e1_at(int row, int col4) {   // col4: multiple of
 __device__ __forceinline__ int at_group(int a) { return a * (a + 1); }
 
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
-    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) {   // two packed f32x2 multiplies
+    const float2 lo = __fmul2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
+    const float2 hi = __fmul2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 __device__ __forceinline__ float4 bf4(uint2 u) {   // four bf16 -> fp32
     const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
     const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
     return make_float4(f0.x, f0.y, f1.x, f1.y);
 }
-// round to tf32 (nearest, ties away from zero) with integer ops: add half an ulp
-// of the 10-bit significand, clear the 13 low bits (finite inputs only)
+// round to tf32 (nearest, ties away from zero) for a tf32 MMA operand: add half an
+// ulp of the 10-bit significand to the magnitude; the tensor core reads only the
+// 19 high bits of each 32-bit operand, which completes the rounding (finite
+// inputs far from the fp32 maximum only)
 __device__ __forceinline__ float tf32r(float x) {
-    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+    return __uint_as_float(__float_as_uint(x) + 0x1000u);
 }
 __device__ __forceinline__ float4 tf4(float4 a) {
     return make_float4(tf32r(a.x), tf32r(a.y), tf32r(a.z), tf32r(a.w));
@@ -364,7 +368,8 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         tmem_relinquish();
     }
     if (tid == 32) {
-        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 4);   // operand rounds: four issuers
+        for (int i = 4; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
         *abort_flag = 0u;
     }
@@ -482,6 +487,12 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 *reinterpret_cast<float4 *>(bt + ((32 * a + 16 + i) >> 3) * 1024) = tf4(mul4(kf, e));
                 float4 ki = mul4(kf, rcp4(e));
                 *reinterpret_cast<float4 *>(at + ((8 * at_group(a) + r) >> 3) * 1024) = tf4(ki);
+                {   // Khat = k EL / E1 straight to the slot (fp16, MN-major, 4 channels)
+                    const float4 kh = mul4(ki, ld4(EL + a * 128 + c0));
+                    __half2 h0 = __floats2half2_rn(kh.x, kh.y), h1 = __floats2half2_rn(kh.z, kh.w);
+                    *reinterpret_cast<uint2 *>(slot + kSlotKh + sw128_mnmajor_off(c0, r, kKhMNBlock)) =
+                        make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
+                }
                 for (int a2 = a + 1; a2 < 4; ++a2) {
                     ki = mul4(ki, ld4(Fb + (a2 - 1) * 128 + c0));
                     *reinterpret_cast<float4 *>(at + ((8 * at_group(a2) + r) >> 3) * 1024) = tf4(ki);
@@ -491,18 +502,19 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         fence_async_smem();
         __syncthreads();
         tc_fence_after();
-        if (ok && tid == 0) {
+        // row block a's chain is issued by lane 0 of warp 2a: a tcgen05.mma costs
+        // its issuing thread tens of cycles, so four issuers keep that off any
+        // one warp's path (each commits; the round's barrier counts four)
+        if (ok && lane == 0 && (warp & 1) == 0) {
+            const int a = warp >> 1;
             // descriptors advance by their start-address field (address / 16)
-            const uint64_t ad0 = smem_desc(sbase + buf + A_AT, 16, 1024, SW_128B);
-            const uint64_t bd0 = smem_desc(sbase + buf + A_BT, 16, 1024, SW_128B);
+            const uint64_t ad0 = smem_desc(sbase + buf + A_AT + at_group(a) * 1024, 16, 1024, SW_128B);
+            const uint64_t bd0 = smem_desc(sbase + buf + A_BT + 4 * a * 1024, 16, 1024, SW_128B);
             const uint32_t id = idesc(FMT_TF32, 64, 32, 0, 0);
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)            // 4 steps of K=8 over 32 channels
-                    mma_tf32(tmem + 32 * a, ad0 + (uint64_t)((at_group(a) * 1024 + kk * 32) >> 4),
-                             bd0 + (uint64_t)((4 * a * 1024 + kk * 32) >> 4), id,
-                             (rd > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)            // 4 steps of K=8 over 32 channels
+                mma_tf32(tmem + 32 * a, ad0 + (uint64_t)((kk * 32) >> 4), bd0 + (uint64_t)((kk * 32) >> 4),
+                         id, (rd > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&bars[rd]);
         }
     }
@@ -564,7 +576,6 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     tc_fence_before();
     __syncthreads();
 
-    constexpr int KH_TASKS = 6;   // Khat: 1024 8-channel pieces over the 192 threads of warps 2-7
 
     // ---- A3: X = (I + Akk)^-1 in place over AK (fp32), by 2x2 block merges:
     //   inv([[L11, 0], [L21, L22]]) = [[X11, 0], [-X22 (L21 X11), X22]]
@@ -574,34 +585,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     {
         float x[16];
         const int a = tid >> 4, j = tid & 15, o = 16 * a;
-        // Khat = k EL / E1 for the slot, by warps 2-7 while warps 0-1 run the
-        // diagonal blocks of the solve (whose latency also covers these loads)
-        if (ok && warp >= 2) {
-            uint4 kh_pref[KH_TASKS];
-#pragma unroll
-            for (int i = 0; i < KH_TASKS; ++i) {
-                const int task = (tid - 64) + 192 * i, s = task >> 4, cc = (task & 15) * 8;
-                kh_pref[i] = (task < 1024 && s < L)
-                    ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
-                    : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int i = 0; i < KH_TASKS; ++i) {
-                const int task = (tid - 64) + 192 * i, s = task >> 4, cc = (task & 15) * 8;
-                if (task < 1024) {
-                    float xk[8];
-                    unpack8(kh_pref[i], xk);
-                    const float *el = EL + (s >> 4) * 128 + cc;
-                    const float4 ea = ld4(E1 + e1_at(s, cc)), eb = ld4(E1 + e1_at(s, cc + 4));
-                    const float e1[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) xk[e] *= el[e] * rcpa(e1[e]);
-                    *reinterpret_cast<uint4 *>(slot + kSlotKh +
-                                               sw128_mnmajor_off(cc, s, kKhMNBlock)) = pack8(xk);
-                }
-            }
-            if (tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = GamL[tid - 128];
-        }
+        if (ok && tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = GamL[tid - 128];
         if (ok && tid < 64) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -904,7 +888,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::oBar);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + NBARS);
     volatile uint32_t *abort_flag = tmem_ptr + 1;
-    volatile uint32_t *s_grp_ok = tmem_ptr + 2;   // S issuer -> state warps
+    volatile uint32_t *s_grp_ok = tmem_ptr + 2;   // elected state thread -> state warps
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int slice = blockIdx.x % NSL;
@@ -926,18 +910,18 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     if (tid == 0) {
         for (int i = 0; i < Lay::NST; ++i) {
             mbar_init(&bars[FULL0 + i], 1);
-            mbar_init(&bars[EMPTY0 + i], 1);
+            mbar_init(&bars[EMPTY0 + i], 2);   // both state-update issuers commit
             mbar_init(&bars[VRAW0 + i], 32);
             mbar_init(&bars[VREADY0 + i], 1);
         }
-        mbar_init(&bars[TDFULL0], 1);
-        mbar_init(&bars[TDFULL1], 1);
+        mbar_init(&bars[TDFULL0], 4);   // four state-term issuers commit
+        mbar_init(&bars[TDFULL1], 4);
         mbar_init(&bars[TDEMPTY0], 4);
         mbar_init(&bars[TDEMPTY1], 4);
         mbar_init(&bars[TSSCALED], 1);
-        mbar_init(&bars[TSFULL], 1);
-        mbar_init(&bars[DRAIN_S], 1);
-        mbar_init(&bars[DRAIN_U], 1);
+        mbar_init(&bars[TSFULL], 2);
+        mbar_init(&bars[DRAIN_S], 4);
+        mbar_init(&bars[DRAIN_U], 2);
         mbar_fence_init();
         *abort_flag = 0u;
         *s_grp_ok = 1u;
@@ -1015,7 +999,9 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         // ------------------------------------------------ U / O epilogue (+ state-update issue)
         const int quad = warp - 4;
         const int row = 32 * quad + lane;
-        const bool issuer = (warp == 4 && lane == 0);
+        // lane 0 of warps 4 and 5 each issue half of the state update (a tcgen05.mma
+        // costs its issuing thread tens of cycles; two issuers halve that path)
+        const bool issuer = (quad < 2 && lane == 0);
         const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
         bool ok = true;
         for (int j = 0; j < nch; ++j) {
@@ -1069,7 +1055,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotKh, kKhMNBlock, 1024, SW_128B);
                         const uint64_t bd0 = smem_desc(sbase + Lay::oUB, Lay::kKGroup, 128, SW_NONE);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
+                        for (int kk = 2 * quad; kk < 2 * quad + 2; ++kk)
                             mma_f16(tTS, ad0 + (uint64_t)(kk * 2048 / 16),
                                     bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_mm, 1);
                         mma_commit(&bars[TSFULL]);
@@ -1090,7 +1076,8 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         // ------------------------------------------------ state epilogue (+ chunk-product issue)
         const int quad = warp - 8;
         const int c = 32 * quad + lane;   // key channel = TMEM lane
-        const bool issuer = (warp == 8 && lane == 0);
+        const bool issuer = (warp == 8 && lane == 0);   // V terms, TSSCALED, group status
+        const bool sissuer = (lane == 0);                 // a quarter of the state term each
         const uint32_t tS = taddr(tTS, 32 * quad, 0);
         const size_t srow = (((size_t)n * H + h) * D + c) * D + j0;
         const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
@@ -1136,19 +1123,22 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                    (j < 2 || mbar_try_wait(&bars[TDEMPTY0 + (j & 1)], ((j >> 1) + 1) & 1));
         };
         // After the fp16 copy of S_j and the scaled TS are in place: the elected
-        // thread releases the state update of chunk j (TSSCALED), issues
-        // [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j into TD[j % 2] and tells the
-        // group whether it succeeded.  When the next chunk's slot, V slice and
-        // accumulator are already free it also issues that chunk's V term: the
-        // pipe then runs it while the U warps copy U out, and only the state
-        // term remains on the chunk-to-chunk path.
-        auto issue_chunk = [&](int j) {
+        // thread releases the state update of chunk j (TSSCALED) and makes sure
+        // the V term of chunk j has been issued; then lane 0 of each state warp
+        // adds a quarter of [-W; P]_j S_j onto it in TD[j % 2].  When the next
+        // chunk's slot, V slice and accumulator are already free, the elected
+        // thread also issues that chunk's V term: the pipe then runs it while
+        // the U warps copy U out, and only the state term remains on the
+        // chunk-to-chunk path.
+        // (ok_in: the elected thread's own status; the group status travels in
+        // s_grp_ok, written only between the two barriers below)
+        auto issue_chunk = [&](int j, bool ok_in) {
+            const int st = j % NST, b = j & 1;
             fence_async_smem();
             tc_fence_before();
             named_bar(2, 128);
             if (issuer) {
-                const int st = j % NST, b = j & 1;
-                bool okk = *s_grp_ok != 0u;
+                bool okk = ok_in;
                 if (okk) mbar_arrive(&bars[TSSCALED]);
                 if (okk && v_issued < j) {
                     okk = mbar_wait_abortable(&bars[FULL0 + st], full_par(j), err, abort_flag);
@@ -1161,27 +1151,31 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         issue_vterm(j);
                     }
                 }
-                if (okk) {
-                    tc_fence_after();
-                    const uint32_t tTD = b ? tTD1 : tTD0;
-                    const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotWP, 16, 1024, SW_128B);
-                    const uint64_t bd0 = smem_desc(sbase + Lay::oSB, Lay::kKGroup, 128, SW_NONE);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_f16(tTD, ad0 + (uint64_t)(((kk >> 2) * kWPKBlock + (kk & 3) * 32) / 16),
-                                bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, 1);
-                    mma_commit(&bars[TDFULL0 + b]);
-                    // early V term of chunk j + 1, only if nothing has to be waited for
-                    const int jn = j + 1;
-                    if (jn < nch && vterm_ready(jn)) {
-                        tc_fence_after();
-                        issue_vterm(jn);
-                    }
-                }
                 *s_grp_ok = okk ? 1u : 0u;
+                tc_fence_before();
             }
-            named_bar(2, 128);
-            return *s_grp_ok != 0u;
+            named_bar(2, 128);   // the V term of chunk j is issued before any state term
+            const bool okk = *s_grp_ok != 0u;
+            if (sissuer && okk) {
+                tc_fence_after();
+                const uint32_t tTD = b ? tTD1 : tTD0;
+                const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotWP, 16, 1024, SW_128B);
+                const uint64_t bd0 = smem_desc(sbase + Lay::oSB, Lay::kKGroup, 128, SW_NONE);
+#pragma unroll
+                for (int kk = 2 * quad; kk < 2 * quad + 2; ++kk)
+                    mma_f16(tTD, ad0 + (uint64_t)(((kk >> 2) * kWPKBlock + (kk & 3) * 32) / 16),
+                            bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, 1);
+                mma_commit(&bars[TDFULL0 + b]);
+            }
+            if (issuer && okk) {
+                // early V term of chunk j + 1, only if nothing has to be waited for
+                const int jn = j + 1;
+                if (jn < nch && vterm_ready(jn)) {
+                    tc_fence_after();
+                    issue_vterm(jn);
+                }
+            }
+            return okk;
         };
         auto gamma_of = [&](int j, bool &ok) {
             if (ok) ok = mbar_wait_abortable(&bars[FULL0 + j % NST], full_par(j), err, abort_flag);
@@ -1213,8 +1207,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             {
                 const float gam = gamma_of(0, ok);
                 if (ok) put_state(xa, gam);
-                if (issuer) *s_grp_ok = ok ? 1u : 0u;
-                ok = issue_chunk(0) && ok;
+                ok = issue_chunk(0, ok) && ok;
             }
             for (int j = 0; j < nch; ++j) {
                 // S_{j+1} = TS after the state update of chunk j
@@ -1229,8 +1222,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 if (j + 1 == nch) break;
                 const float gam = gamma_of(j + 1, ok);
                 if (ok) put_state(xa, gam);
-                if (issuer) *s_grp_ok = ok ? 1u : 0u;
-                const bool ok2 = issue_chunk(j + 1);
+                const bool ok2 = issue_chunk(j + 1, ok);
                 ok = ok && ok2;
             }
             if (ok && state_out && !*abort_flag) {
@@ -1239,7 +1231,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                     reinterpret_cast<float4 *>(state_out + srow)[i] =
                         make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
             }
-            if (issuer) {
+            if (sissuer) {
                 mma_commit(&bars[DRAIN_S]);
                 mbar_wait(&bars[DRAIN_S], 0, err, 1ull << 28);
             }

@@ -80,6 +80,7 @@ def compare_units(ref, got, tol, what=""):
     s_ref = np.concatenate([ref[u][1].reshape(-1) for u in ref])
     s_got = np.concatenate([got[u][1].reshape(-1) for u in ref])
     eo, es = rel_err(o_got, o_ref), rel_err(s_got, s_ref)
+    print(f"{what}: output error {eo:.3e}, final-state error {es:.3e} (bar {tol})")
     assert np.all(np.isfinite(o_got)) and np.all(np.isfinite(s_got)), f"{what}: non-finite output"
     assert eo <= tol, f"{what}: output error {eo:.3e} > {tol}"
     assert es <= tol, f"{what}: final-state error {es:.3e} > {tol}"

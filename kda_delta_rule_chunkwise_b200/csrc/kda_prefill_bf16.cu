@@ -214,13 +214,14 @@ constexpr uint32_t A_MISC = 32768;    // beta, F, EL, Gamma_L, barriers, TMEM ad
 constexpr uint32_t A_M_BETA = 0;      //   fp32 [64]
 constexpr uint32_t A_M_F = 256;       //   fp32 [3][128]
 constexpr uint32_t A_M_EL = 1792;     //   fp32 [4][128]
-constexpr uint32_t A_M_GAML = 3840;   //   fp32 [128]
-constexpr uint32_t A_M_BARS = 4352;   //   8 mbarriers
-constexpr uint32_t A_M_TMEM = 4416;   //   TMEM base address + abort flag
-constexpr uint32_t A_M_END = 4424;
+constexpr uint32_t A_M_PF = 3840;     //   fp32 [2][128]: F_0 F_1 and F_0 F_1 F_2
+constexpr uint32_t A_M_BARS = 4864;   //   8 mbarriers
+constexpr uint32_t A_M_TMEM = 4928;   //   TMEM base address + abort flag
+constexpr uint32_t A_M_END = 4936;
 constexpr uint32_t A_OPS = 37888;     // operand region (two uses, below)
 static_assert(A_MISC + A_M_END <= A_OPS, "phase A misc region overflows into the operands");
-static_assert(A_M_BARS % 8 == 0 && A_M_F % 16 == 0 && A_M_EL % 16 == 0, "misc alignment");
+static_assert(A_M_BARS % 8 == 0 && A_M_F % 16 == 0 && A_M_EL % 16 == 0 && A_M_PF % 16 == 0,
+              "misc alignment");
 // before the Akk/Aqk MMAs: two buffers of one 32-channel round (tf32, K-major SW128)
 constexpr uint32_t A_RBUF = 36864;            // bytes per round buffer
 constexpr uint32_t A_BT = 0;                  //   + [Q'_a; K'_a], 128 rows x 128 B    16 KiB
@@ -231,14 +232,13 @@ constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64 
 constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64     16 KiB
 constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128          16 KiB
 constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 solve scratch (32 x 32)               4 KiB
-constexpr uint32_t A_QP = A_AK;               // bf16 q rows [64][128] for P, once T is out  16 KiB
-// next item's rows, prefetched once D1 has completed (all of the above but A_QP is dead)
+// next item's rows, prefetched once D1 has completed (all of the above is dead by then)
 constexpr uint32_t A_QST = A_OPS + 16384;     // bf16 q [64][128], pieces permuted per row   16 KiB
 constexpr uint32_t A_KST = A_OPS + 32768;     // bf16 k, same layout                         16 KiB
 constexpr uint32_t A_GST = A_OPS + 49152;     // bf16 g [64][128]                            16 KiB
 constexpr uint32_t A_SMEM = A_OPS + 2 * A_RBUF + 1024;   // + alignment slack (= 112640)
 static_assert(A_Y + 4096 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
-static_assert(A_QST >= A_QP + 16384 && A_GST + 16384 <= A_OPS + 2 * A_RBUF, "staging area");
+static_assert(A_QST >= A_AK + 16384 && A_GST + 16384 <= A_OPS + 2 * A_RBUF, "staging area");
 static_assert(3 * 128 * 4 + 128 * 4 <= 16384, "A0 scratch (tot, G_L) must not reach the staging area");
 static_assert(A_OPS % 1024 == 0 && A_RBUF % 1024 == 0 && A_AQ % 1024 == 0 && A_TR % 1024 == 0 &&
               A_KT % 1024 == 0, "swizzled tiles need 1024-byte alignment");
@@ -295,7 +295,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     float *bs = reinterpret_cast<float *>(sm + A_MISC + A_M_BETA);    // [64]
     float *Fb = reinterpret_cast<float *>(sm + A_MISC + A_M_F);       // [3][128] block decays F_m
     float *EL = reinterpret_cast<float *>(sm + A_MISC + A_M_EL);      // [4][128]
-    float *GamL = reinterpret_cast<float *>(sm + A_MISC + A_M_GAML);  // [128] exp(G_L)
+    float *PF = reinterpret_cast<float *>(sm + A_MISC + A_M_PF);      // [2][128] F_0 F_1 (F_2)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + A_MISC + A_M_BARS);   // [8]
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + A_MISC + A_M_TMEM);
     volatile uint32_t *abort_flag = tmem_ptr + 1;
@@ -382,14 +382,10 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint32_t ph = 0;   // mbarrier phase parity: each barrier completes once per item
     // (items fit in int32: the host checks max_chunks * H against INT32_MAX)
     for (int item = blockIdx.x; item < (int)n_items; item += gridDim.x, ph ^= 1u) {
-    const int h = (int)(item % H);
     int64_t t0;
     int L;
     locate(item, t0, L);
     uint8_t *slot = ws + header_bytes(N) + (size_t)item * kSlotBytes;
-    auto row_ptr = [&](const __nv_bfloat16 *base, int r) {
-        return base + ((size_t)(t0 + r) * H + h) * D;
-    };
 
     // ---- this item's rows have landed (each thread waits for its own copies)
     cp_async_wait_all();
@@ -444,7 +440,8 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         EL[128 + c] = __expf(gl - r1);
         EL[256 + c] = __expf(gl - r2);
         EL[384 + c] = __expf(gl - r3);
-        GamL[c] = __expf(gl);
+        PF[c] = Fb[c] * Fb[128 + c];
+        PF[128 + c] = PF[c] * Fb[256 + c];
     }
     // q, k of the operand rounds into registers; the staging area is free after the barrier
     uint2 qv[4][2], kv[4][2];
@@ -481,10 +478,23 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 // every row this task writes is congruent to r mod 8: one swizzled chunk offset
                 const uint32_t co = (r & 7) * 128 + ((p_l ^ (r & 7)) << 4);
                 uint8_t *bt = sm + buf + A_BT + co, *at = sm + buf + A_AT + co;
-                const float4 e = ld4(E1 + e1_at(r, c0));
+                float *e1p = E1 + e1_at(r, c0);
+                const float4 e = ld4(e1p);
                 const float4 qf = bf4(qv[rd][it]), kf = bf4(kv[rd][it]);
-                *reinterpret_cast<float4 *>(bt + ((32 * a + i) >> 3) * 1024) = tf4(mul4(qf, e));
-                *reinterpret_cast<float4 *>(bt + ((32 * a + 16 + i) >> 3) * 1024) = tf4(mul4(kf, e));
+                const float4 qe = mul4(qf, e), ke = mul4(kf, e);
+                *reinterpret_cast<float4 *>(bt + ((32 * a + i) >> 3) * 1024) = tf4(qe);
+                *reinterpret_cast<float4 *>(bt + ((32 * a + 16 + i) >> 3) * 1024) = tf4(ke);
+                {   // Q*Gamma and K*Gamma = (q, k) E1 prod_{m<a} F_m as fp16 pairs (low: Q*Gamma,
+                    // high: K*Gamma), in place of this task's E1 values, read by nobody else
+                    const float4 pf = a == 0 ? make_float4(1.f, 1.f, 1.f, 1.f)
+                                             : ld4((a == 1 ? Fb : PF + (a - 2) * 128) + c0);
+                    const float4 qg = mul4(qe, pf), kg = mul4(ke, pf);
+                    __half2 p0 = __floats2half2_rn(qg.x, kg.x), p1 = __floats2half2_rn(qg.y, kg.y);
+                    __half2 p2 = __floats2half2_rn(qg.z, kg.z), p3 = __floats2half2_rn(qg.w, kg.w);
+                    *reinterpret_cast<uint4 *>(e1p) =
+                        make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
+                                   *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
+                }
                 float4 ki = mul4(kf, rcp4(e));
                 *reinterpret_cast<float4 *>(at + ((8 * at_group(a) + r) >> 3) * 1024) = tf4(ki);
                 {   // Khat = k EL / E1 straight to the slot (fp16, MN-major, 4 channels)
@@ -518,32 +528,20 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             mma_commit(&bars[rd]);
         }
     }
-    // next loads (the K*Gamma operand, 4 pieces per thread) go out before the last MMA wait
-    uint4 kt_pref[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
-        kt_pref[i] = s < L ? __ldg(reinterpret_cast<const uint4 *>(row_ptr(k, s) + cc))
-                           : make_uint4(0u, 0u, 0u, 0u);
-    }
     if (ok) ok = mbar_wait_abortable(&bars[3], ph, err, abort_flag);
     tc_fence_after();
 
-    // ---- A2: K*Gamma = k E1 prod_{m<a} F_m as the MN-major B operand of W = T (K*Gamma)
+    // ---- A2: K*Gamma (the high halves of the packed pairs) into the MN-major B operand of
+    // W = T (K*Gamma)
     if (ok) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int task = tid + 256 * i, s = task >> 4, cc = (task & 15) * 8;
-            float x[8];
-            unpack8(kt_pref[i], x);
-            const int a = s >> 4;
-#pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-                float4 e = ld4(E1 + e1_at(s, cc + 4 * hv));
-                for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
-                x[4 * hv] *= e.x; x[4 * hv + 1] *= e.y; x[4 * hv + 2] *= e.z; x[4 * hv + 3] *= e.w;
-            }
-            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(cc, s, kKhMNBlock)) = pack8(x);
+            const uint4 u0 = *reinterpret_cast<const uint4 *>(E1 + e1_at(s, cc));
+            const uint4 u1 = *reinterpret_cast<const uint4 *>(E1 + e1_at(s, cc + 4));
+            const uint4 kg = make_uint4(__byte_perm(u0.x, u0.y, 0x7632), __byte_perm(u0.z, u0.w, 0x7632),
+                                        __byte_perm(u1.x, u1.y, 0x7632), __byte_perm(u1.z, u1.w, 0x7632));
+            *reinterpret_cast<uint4 *>(sm + A_KT + sw128_mnmajor_off(cc, s, kKhMNBlock)) = kg;
         }
     }
     // and Akk (fp32, beta applied, strictly lower) and Aqk (fp16, lower incl. diagonal,
@@ -585,7 +583,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     {
         float x[16];
         const int a = tid >> 4, j = tid & 15, o = 16 * a;
-        if (ok && tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = GamL[tid - 128];
+        if (ok && tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = EL[tid - 128];
         if (ok && tid < 64) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -691,17 +689,6 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
     tc_fence_after();
 
-    // q rows for P (A6) go to the Akk region, dead since T was written: cp.async,
-    // landed by the barrier before A5 (rows past L zero-filled).  Row r's 16-byte
-    // piece p sits at slot p ^ (r % 16), so that A6's row-per-lane reads are
-    // free of bank conflicts.
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int task = tid + 256 * i, r = task >> 4, cc = (task & 15) * 8;
-        cp_async16(sm + A_QP + (r * 16 + ((task & 15) ^ (r & 15))) * 16, row_ptr(q, r < L ? r : 0) + cc,
-                   r < L ? 16u : 0u);
-    }
-
     // ---- A4: R = Aqk T  (M=64, N=64, K=64; A MN-major, B MN-major) into TMEM columns 128..191
     if (ok && tid == 0) {
         const uint32_t id = idesc(FMT_F16, 64, 64, 1, 1);
@@ -734,7 +721,6 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
         }
     }
-    cp_async_wait_all();   // this thread's q rows for A6
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -756,25 +742,6 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     if (ok && tid == 0) {
         bulk_s2g(slot + kSlotTR, sm + A_TR, 16384);
         bulk_commit();
-    }
-    // meanwhile every thread turns its staged q pieces into Q*Gamma = q E1 prod_{m<a} F_m
-    // (fp16, in place), so that A6's P rows only subtract
-    if (ok) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int task = tid + 256 * i, r = task >> 4, pc = task & 15, cc = 8 * pc;
-            uint4 *qp = reinterpret_cast<uint4 *>(sm + A_QP) + r * 16 + (pc ^ (r & 15));
-            float x[8];
-            unpack8(*qp, x);
-            const int a = r >> 4;
-#pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-                float4 e = ld4(E1 + e1_at(r, cc + 4 * hv));
-                for (int m = 0; m < a; ++m) e = mul4(e, ld4(Fb + m * 128 + cc + 4 * hv));
-                x[4 * hv] *= e.x; x[4 * hv + 1] *= e.y; x[4 * hv + 2] *= e.z; x[4 * hv + 3] *= e.w;
-            }
-            *qp = pack8(x);
-        }
     }
     if (ok) ok = mbar_wait_abortable(&bars[5], ph, err, abort_flag);
     tc_fence_after();
@@ -805,9 +772,14 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                     u.x ^= 0x80008000u; u.y ^= 0x80008000u;   // -W: flip the fp16 signs
                     u.z ^= 0x80008000u; u.w ^= 0x80008000u;
                 } else {
-                    const int pc = 8 * chalf + 4 * hh + ch;
+                    const int cc = 8 * (8 * chalf + 4 * hh + ch);
+                    // Q*Gamma: the low halves of the packed pairs
+                    const uint4 u0 = *reinterpret_cast<const uint4 *>(E1 + e1_at(r6, cc));
+                    const uint4 u1 = *reinterpret_cast<const uint4 *>(E1 + e1_at(r6, cc + 4));
                     float qg[8];
-                    unpack8h(reinterpret_cast<const uint4 *>(sm + A_QP)[r6 * 16 + (pc ^ (r6 & 15))], qg);
+                    unpack8h(make_uint4(__byte_perm(u0.x, u0.y, 0x5410), __byte_perm(u0.z, u0.w, 0x5410),
+                                        __byte_perm(u1.x, u1.y, 0x5410), __byte_perm(u1.z, u1.w, 0x5410)),
+                             qg);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y[e] = qg[e] - x[ch * 8 + e];
                     u = pack8(y);

@@ -560,9 +560,10 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 float y0[8], y1[8];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
+                    // (rows r >= L are zero already: their q, k and beta are zero)
                     const int r = 16 * a + j;
-                    AK[r * 64 + s] = (s < r && r < L) ? bs[r] * vk[j] : 0.f;
-                    const float aq = (s <= r && r < L) ? vq[j] : 0.f;
+                    AK[r * 64 + s] = s < r ? bs[r] * vk[j] : 0.f;
+                    const float aq = s <= r ? vq[j] : 0.f;
                     if (j < 8) y0[j] = aq; else y1[j - 8] = aq;
                 }
                 *reinterpret_cast<uint4 *>(sm + A_AQ + sw128_mnmajor_off(16 * a, s, 0)) = pack8(y0);
@@ -602,31 +603,38 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
     // merge 16 -> 32 for diagonal pairs p = 0, 1 (rows/cols 32p .. 32p+31):
     //   Y = A_{2p+1,2p} X_{2p,2p};  X_{2p+1,2p} = -X_{2p+1,2p+1} Y
+    // thread: pair pr, column j, rows i and i + 8 (row operands as float4, the
+    // column operand shared by both rows)
     {
-        const int pr = tid >> 7, e0 = tid & 127;   // pair, then 2 elements per thread
+        const int pr = tid >> 7, j = tid & 15, i = (tid >> 4) & 7;
         const int o = 32 * pr;
+        const float *r0 = AK + (o + 16 + i) * 64 + o, *r1 = r0 + 8 * 64;
         if (ok) {
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const int e = e0 + 128 * qq, i = e >> 4, j = e & 15;
-                float acc = 0.f;
-#pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    acc = fmaf(AK[(o + 16 + i) * 64 + o + t], AK[(o + t) * 64 + o + j], acc);
-                Yb[pr * 256 + e] = acc;
+            for (int t4 = 0; t4 < 4; ++t4) {
+                const float4 a0 = ld4(r0 + 4 * t4), a1 = ld4(r1 + 4 * t4);
+                const float x0 = AK[(o + 4 * t4) * 64 + o + j], x1 = AK[(o + 4 * t4 + 1) * 64 + o + j];
+                const float x2 = AK[(o + 4 * t4 + 2) * 64 + o + j], x3 = AK[(o + 4 * t4 + 3) * 64 + o + j];
+                acc0 = fmaf(a0.x, x0, fmaf(a0.y, x1, fmaf(a0.z, x2, fmaf(a0.w, x3, acc0))));
+                acc1 = fmaf(a1.x, x0, fmaf(a1.y, x1, fmaf(a1.z, x2, fmaf(a1.w, x3, acc1))));
             }
+            Yb[pr * 256 + i * 16 + j] = acc0;
+            Yb[pr * 256 + (i + 8) * 16 + j] = acc1;
         }
         __syncthreads();
         if (ok) {
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const int e = e0 + 128 * qq, i = e >> 4, j = e & 15;
-                float acc = 0.f;
-#pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    acc = fmaf(AK[(o + 16 + i) * 64 + o + 16 + t], Yb[pr * 256 + t * 16 + j], acc);
-                AK[(o + 16 + i) * 64 + o + j] = -acc;
+            for (int t4 = 0; t4 < 4; ++t4) {
+                const float4 a0 = ld4(r0 + 16 + 4 * t4), a1 = ld4(r1 + 16 + 4 * t4);
+                const float *yc = Yb + pr * 256 + 64 * t4 + j;
+                const float y0 = yc[0], y1 = yc[16], y2 = yc[32], y3 = yc[48];
+                acc0 = fmaf(a0.x, y0, fmaf(a0.y, y1, fmaf(a0.z, y2, fmaf(a0.w, y3, acc0))));
+                acc1 = fmaf(a1.x, y0, fmaf(a1.y, y1, fmaf(a1.z, y2, fmaf(a1.w, y3, acc1))));
             }
+            AK[(o + 16 + i) * 64 + o + j] = -acc0;
+            AK[(o + 24 + i) * 64 + o + j] = -acc1;
         }
         __syncthreads();
     }

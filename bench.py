@@ -405,14 +405,23 @@ def cpu_threads():
 
 
 def sized_oracle_sample(seed, target_s, threads, cap_tokens=65536):
-    """Calibrate on a short sample, then time one sample sized to ~target_s seconds."""
-    heads = min(32, max(1, threads))
+    """Calibrate on a short sample, then time one sample sized to ~target_s seconds.
+
+    All 32 heads (the oracle threads over (sequence, head) units, so at most 32
+    threads work); the token count grows up to the whole workload.
+    """
+    heads = 32
     v0, dt0 = oracle_sample(seed, 256, heads, threads)
     n = int(256 * target_s / max(dt0, 1e-3))
     n = max(256, min(cap_tokens, n))
     v, dt = oracle_sample(seed, n, heads, threads)
     sample = f"first {n} tokens x {heads} of 32 heads of {PREFILL_WORKLOAD}, fp64, {dt:.1f} s"
     return v, dt, sample
+
+
+def oracle_cores(threads):
+    """Threads the oracle actually runs on: one per (sequence, head) unit at most."""
+    return min(threads, 32)
 
 
 def run_reference(args):
@@ -434,7 +443,7 @@ def run_reference(args):
         "data": "synthetic",
         "config": {"workload": PREFILL_WORKLOAD, "B": 1, "T": 65536, "H": 32, "dk": 128,
                    "dv": 128, "parallelism": "host cores"},
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": oracle_cores(threads),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -493,7 +502,7 @@ def main():
         if not args.no_cpu_baseline:
             threads = cpu_threads()
             v, dt, smp = sized_oracle_sample(args.seed, args.ref_seconds, threads)
-            res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": threads,
+            res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": oracle_cores(threads),
                                    "kind": "oracle", "sample": smp}
         print(json.dumps(res), flush=True)
     return 0

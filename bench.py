@@ -305,6 +305,40 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
                "steps": args.e2e_steps}
         del hq, hk, hv, hg, hb, hs, ho, hso, dq, dk_, dv_, dg, db, ds
 
+    # ---------------- the same step with intermediate states every CKPT_INTERVAL tokens
+    ckpt_res = None
+    if args.ckpt_interval > 0 and d.cu_seqlens is None:
+        iv = args.ckpt_interval
+        cnt = binding.kda_prefill_checkpoint_count(None, B, T, iv)
+        ck = torch.empty((max(cnt, 1), H, 128, 128), dtype=torch.float32, device=dev)
+
+        def ck_step():
+            binding.kda_chunk_prefill_checkpointed(d.q, d.k, d.v, d.g, d.beta, d.state_in, None,
+                                                   interval=iv, ckpt=ck[:cnt], o=o,
+                                                   state_out=s_out, workspace=ws)
+
+        for _ in range(args.warmup):
+            ck_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        st = torch.cuda.current_stream()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(st)
+        for _ in range(args.steps):
+            ck_step()
+        ev1.record(st)
+        torch.cuda.synchronize()
+        c_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        ckpt_res = {"interval": iv, "snapshots_per_step": cnt * H,
+                    "snapshot_bytes_per_step": cnt * H * STATE_BYTES,
+                    "ms_per_step": round(c_ms / args.steps, 4),
+                    "value": aggregate_throughput(tokens, world, args.steps, c_ms),
+                    "unit": "tokens/s",
+                    "overhead_vs_plain": round(c_ms / args.steps / ms_step - 1.0, 4)}
+        del ck
+    extra = {"prefill_checkpointed": ckpt_res}
+
     del d, o, s_out, ws
     torch.cuda.empty_cache()
 
@@ -312,7 +346,7 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
     decode = None
     if args.decode_steps <= 0:
         return finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path,
-                      decode, e2e, clk)
+                      decode, e2e, clk, extra)
     dw = kin.WORKLOADS[DECODE_WORKLOAD]
     Nd, Hd = dw["N"], dw["H"]
     dec = kin.decode_inputs(args.decode_steps, Nd, Hd, 128, 128, "bf16",
@@ -351,16 +385,49 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
                      "bytes_per_launch": d_bytes},
         "state_bytes": S.numel() * 4,
     }
-    del dec, pristine, S, od
+    del pristine, S
+    torch.cuda.empty_cache()
+
+    # ---------------- the same decode on a pooled state (continuous batching): the N
+    # requests own random distinct entries of a pool of 2N
+    P = 2 * Nd
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed + 2000 + rank)
+    pool = torch.randn((P, Hd, 128, 128), generator=gen, device=dev) * 0.1
+    slots = torch.randperm(P, generator=gen, device=dev)[:Nd].to(torch.int32).contiguous()
+
+    def idx_step(t):
+        binding.kda_decode_step_indexed(dec.q[t], dec.k[t], dec.v[t], dec.g[t], dec.beta[t],
+                                        pool, slots, o=od)
+
+    for t in range(min(args.warmup, args.decode_steps)):
+        idx_step(t)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ev0.record(st)
+    for t in range(args.decode_steps):
+        idx_step(t)
+    ev1.record(st)
+    torch.cuda.synchronize()
+    i_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    i_gbs = d_bytes * args.decode_steps / (i_ms / 1e3) / 1e9
+    decode["indexed"] = {
+        "pool_entries": P, "requests": Nd, "steps_per_s": round(world * args.decode_steps / (i_ms / 1e3), 1),
+        "gbs": round(world * i_gbs, 1),
+        "roofline": {"kernel": "decode_kernel (indexed)", "bound": "hbm", "achieved": round(i_gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(i_gbs / peaks["hbm_gbs"], 4)},
+    }
+    del dec, pool, slots, od
     torch.cuda.empty_cache()
 
     return finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path,
-                  decode, e2e, clk)
+                  decode, e2e, clk, extra)
 
 
 def finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path, decode,
-           e2e, clk):
-    launches = args.steps * 3 + max(0, args.decode_steps)
+           e2e, clk, extra):
+    launches = args.steps * 3 + 2 * max(0, args.decode_steps)   # prefill, decode, indexed decode
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -371,7 +438,7 @@ def finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline
                    "seq_len": T, "parallelism": f"replicas{world}",
                    "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
         "roofline": roofline, "roofline_path": roofline_path, "decode": decode,
-        "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(), **extra,
     }
 
 
@@ -458,6 +525,9 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ckpt-interval", type=int, default=512,
+                    help="also time the prefill step with intermediate states every this many "
+                         "tokens (a multiple of 64; 0 skips it)")
     ap.add_argument("--workload", default=PREFILL_WORKLOAD,
                     choices=["prefill_h32_t65536_d128_split", "prefill_h32_t8192_d128",
                              "varlen_64seq_128to16384_h32_d128"],

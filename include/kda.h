@@ -122,6 +122,40 @@ KDA_API kda_status kda_chunk_prefill(const void *q, const void *k, const void *v
                              void *stream);
 
 /*
+ * Prefill that also stores intermediate states, for prefix caching: for each
+ * sequence, the state after its first m * interval tokens for every m >= 1
+ * with m * interval < its length (the state after all of its tokens is
+ * state_out).  Serving layers keep such snapshots so that a later request
+ * sharing a prefix resumes from one instead of recomputing it; the pages give
+ * no interface for it.  Everything else is exactly kda_chunk_prefill.
+ *  interval       tokens between snapshots: a positive multiple of 64 (the
+ *                 chunk length), else KDA_ERR_UNSUPPORTED (also for KDA_F32)
+ *  ckpt           fp32 [ckpt_capacity, H, dk, dv], 16-byte aligned.  Entry
+ *                 e = (number of snapshots of sequences 0..n-1) + m - 1 holds
+ *                 sequence n's m-th snapshot; kda_prefill_checkpoint_count()
+ *                 gives the total.  Snapshots past ckpt_capacity are not
+ *                 written and the next kda_check_device_error() returns
+ *                 KDA_ERR_INVALID_ARG.
+ */
+KDA_API kda_status kda_chunk_prefill_checkpointed(const void *q, const void *k, const void *v,
+                                          const void *g, const void *beta,
+                                          const float *state_in, const int32_t *cu_seqlens,
+                                          int B, int64_t T, int N, int H, int dk, int dv,
+                                          kda_dtype dtype, void *o, float *state_out,
+                                          int64_t interval, float *ckpt, int64_t ckpt_capacity,
+                                          void *workspace, size_t workspace_bytes,
+                                          void *stream);
+
+/*
+ * Number of snapshots kda_chunk_prefill_checkpointed() writes, from the
+ * host's copy of cu_seqlens (same clamping as the device) or, with
+ * cu_seqlens_host NULL, for N = B sequences of T tokens.  -1 for invalid
+ * arguments.
+ */
+KDA_API int64_t kda_prefill_checkpoint_count(const int32_t *cu_seqlens_host, int B, int64_t T,
+                                             int N, int64_t interval);
+
+/*
  * Single-token decode step, state updated in place (one read and one write
  * of each (n, h) state):
  *     S' = Diag(exp g) S;  delta = beta (v - S'^T k);  S = S' + k delta^T;
@@ -135,9 +169,31 @@ KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            void *o, void *stream);
 
 /*
+ * The same decode step on a pooled state (continuous batching): request n's
+ * state is entry slots[n] of a pool of P, and only those entries are read and
+ * overwritten.  This keeps the per-request state a single copy wherever the
+ * serving layer keeps it (the "fixed-size state, single copy per request" of
+ * neurohive.io "Kimi K3 ... overview", section "Training and inference
+ * infrastructure"); the pages give no interface for it.
+ *  q, k, g [N, H, dk];  v [N, H, dv];  beta [N, H];  o [N, H, dv] fp32
+ *  state_pool  [P, H, dk, dv] fp32, 16-byte aligned, entries slots[n] updated in place
+ *  slots       device int32 [N].  Must be distinct (two requests on one entry
+ *              race).  Values are read on the device: an entry outside [0, P)
+ *              is skipped (its o is not written, no memory outside the pool is
+ *              touched) and the next kda_check_device_error() returns
+ *              KDA_ERR_INVALID_ARG.
+ */
+KDA_API kda_status kda_decode_step_indexed(const void *q, const void *k, const void *v,
+                                   const void *g, const void *beta, float *state_pool,
+                                   const int32_t *slots, int N, int P, int H, int dk, int dv,
+                                   kda_dtype dtype, void *o, void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.
- * Returns KDA_ERR_TIMEOUT if any kernel since the last call gave up a bounded
- * wait, KDA_ERR_CUDA if the stream reported an error, KDA_OK otherwise.
+ * Returns KDA_ERR_INVALID_ARG if a kernel since the last call skipped work
+ * because of an out-of-range index read on the device (kda_decode_step_indexed
+ * slots), else KDA_ERR_TIMEOUT if one gave up a bounded wait, KDA_ERR_CUDA if
+ * the stream reported an error, KDA_OK otherwise.
  */
 KDA_API kda_status kda_check_device_error(void *stream);
 

@@ -25,7 +25,10 @@ _DTYPE = {torch.float32: KDA_F32, torch.bfloat16: KDA_BF16}
 EXPORTED = (
     "kda_chunk_prefill_workspace_bytes",
     "kda_chunk_prefill",
+    "kda_chunk_prefill_checkpointed",
+    "kda_prefill_checkpoint_count",
     "kda_decode_step",
+    "kda_decode_step_indexed",
     "kda_check_device_error",
     "kda_selftest_bounded_wait",
     "kda_profile_enable",
@@ -60,8 +63,17 @@ def load(path: str = LIB_PATH):
     lib.kda_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
                                       i32, vp, vp, vp, sz, vp]
     lib.kda_chunk_prefill.restype = i32
+    lib.kda_chunk_prefill_checkpointed.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                                   i32, i32, i32, vp, vp, i64, vp, i64, vp, sz,
+                                                   vp]
+    lib.kda_chunk_prefill_checkpointed.restype = i32
+    lib.kda_prefill_checkpoint_count.argtypes = [vp, i32, i64, i32, i64]
+    lib.kda_prefill_checkpoint_count.restype = i64
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     lib.kda_decode_step.restype = i32
+    lib.kda_decode_step_indexed.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                            i32, vp, vp]
+    lib.kda_decode_step_indexed.restype = i32
     lib.kda_check_device_error.argtypes = [vp]
     lib.kda_check_device_error.restype = i32
     lib.kda_selftest_bounded_wait.argtypes = [i64, vp]
@@ -143,6 +155,52 @@ def kda_chunk_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=Non
     return o, state_out
 
 
+def kda_prefill_checkpoint_count(cu_seqlens, B: int, T: int, interval: int) -> int:
+    """Snapshots kda_chunk_prefill_checkpointed writes (cu_seqlens: int32 tensor or None;
+    a device tensor is copied to the host)."""
+    if cu_seqlens is None:
+        n = load().kda_prefill_checkpoint_count(None, B, T, B, int(interval))
+    else:
+        host = cu_seqlens.to("cpu", torch.int32).contiguous()
+        n = load().kda_prefill_checkpoint_count(_ptr(host), 1, T, host.numel() - 1, int(interval))
+    if n < 0:
+        raise KDAError(KDA_ERR_INVALID_ARG, "kda_prefill_checkpoint_count")
+    return int(n)
+
+
+def kda_chunk_prefill_checkpointed(q, k, v, g, beta, state_in=None, cu_seqlens=None, *,
+                                   interval: int, ckpt=None, o=None, state_out=None,
+                                   workspace=None, stream=None):
+    """kda_chunk_prefill plus the state every `interval` tokens inside each sequence.
+
+    Returns (o, state_out, ckpt) with ckpt [count, H, dk, dv] fp32 (allocated if not
+    given), entries in sequence order (see include/kda.h)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta),
+                    ("state_in", state_in), ("cu_seqlens", cu_seqlens), ("ckpt", ckpt)):
+        _contig(name, t)
+    if ckpt is None:
+        cnt = kda_prefill_checkpoint_count(cu_seqlens, B, T, interval)
+        ckpt = torch.empty((cnt, H, dk, dv), dtype=torch.float32, device=q.device)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if state_out is None:
+        state_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = kda_chunk_prefill_workspace_bytes(B * T, N, H, dk, dv, q.dtype)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = load().kda_chunk_prefill_checkpointed(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens),
+        B, T, N, H, dk, dv, _DTYPE[q.dtype], _ptr(o), _ptr(state_out), int(interval),
+        _ptr(ckpt) if ckpt.numel() else None, ckpt.shape[0],
+        _ptr(workspace) if need else None, ws_bytes if need else 0, _stream(stream))
+    _check(code, "kda_chunk_prefill_checkpointed")
+    return o, state_out, ckpt
+
+
 def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
     """One decode step; `state` [N, H, dk, dv] fp32 is updated in place.  Returns o (fp32)."""
     N, H, dk = q.shape
@@ -154,6 +212,25 @@ def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
     code = load().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
                                   N, H, dk, dv, _DTYPE[q.dtype], _ptr(o), _stream(stream))
     _check(code, "kda_decode_step")
+    return o
+
+
+def kda_decode_step_indexed(q, k, v, g, beta, state_pool, slots, *, o=None, stream=None):
+    """One decode step on pool entries `slots` (int32 [N], distinct) of `state_pool`
+    [P, H, dk, dv] fp32, updated in place.  Returns o (fp32)."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta),
+                    ("state_pool", state_pool), ("slots", slots)):
+        _contig(name, t)
+    if slots.dtype != torch.int32 or slots.numel() != N:
+        raise ValueError("slots must be an int32 tensor with one entry per request")
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=torch.float32, device=q.device)
+    code = load().kda_decode_step_indexed(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool), _ptr(slots), N,
+        state_pool.shape[0], H, dk, dv, _DTYPE[q.dtype], _ptr(o), _stream(stream))
+    _check(code, "kda_decode_step_indexed")
     return o
 
 
@@ -189,6 +266,24 @@ def raw_prefill(args: dict) -> int:
         args.get("state_in"), args.get("cu_seqlens"), args["B"], args["T"], args["N"],
         args["H"], args["dk"], args["dv"], args["dtype"], args.get("o"), args.get("state_out"),
         args.get("workspace"), args.get("workspace_bytes", 0), args.get("stream")))
+
+
+def raw_prefill_checkpointed(args: dict) -> int:
+    lib = load()
+    return int(lib.kda_chunk_prefill_checkpointed(
+        args.get("q"), args.get("k"), args.get("v"), args.get("g"), args.get("beta"),
+        args.get("state_in"), args.get("cu_seqlens"), args["B"], args["T"], args["N"],
+        args["H"], args["dk"], args["dv"], args["dtype"], args.get("o"), args.get("state_out"),
+        args["interval"], args.get("ckpt"), args.get("ckpt_capacity", 0),
+        args.get("workspace"), args.get("workspace_bytes", 0), args.get("stream")))
+
+
+def raw_decode_indexed(args: dict) -> int:
+    lib = load()
+    return int(lib.kda_decode_step_indexed(
+        args.get("q"), args.get("k"), args.get("v"), args.get("g"), args.get("beta"),
+        args.get("state"), args.get("slots"), args["N"], args["P"], args["H"], args["dk"],
+        args["dv"], args["dtype"], args.get("o"), args.get("stream")))
 
 
 def raw_decode(args: dict) -> int:

@@ -102,11 +102,14 @@ size_t kda_chunk_prefill_workspace_bytes(int64_t rows, int N, int H, int dk, int
     return kda::prefill_tc_workspace_bytes(rows, N, H, dk);
 }
 
-kda_status kda_chunk_prefill(const void *q, const void *k, const void *v, const void *g,
-                             const void *beta, const float *state_in,
-                             const int32_t *cu_seqlens, int B, int64_t T, int N, int H,
-                             int dk, int dv, kda_dtype dtype, void *o, float *state_out,
-                             void *workspace, size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+kda_status prefill_impl(const void *q, const void *k, const void *v, const void *g,
+                        const void *beta, const float *state_in, const int32_t *cu_seqlens,
+                        int B, int64_t T, int N, int H, int dk, int dv, kda_dtype dtype, void *o,
+                        float *state_out, void *workspace, size_t workspace_bytes, void *stream,
+                        int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity) {
     if (B < 0 || T < 0 || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (cu_seqlens ? B != 1 : N != B) return KDA_ERR_INVALID_ARG;
@@ -123,11 +126,58 @@ kda_status kda_chunk_prefill(const void *q, const void *k, const void *v, const 
     uint32_t *err = error_word_ptr();
     if (!err) return KDA_ERR_CUDA;
     kda::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv,
-                       o, state_out, workspace, workspace_bytes, err};
+                       o, state_out, workspace, workspace_bytes, err,
+                       ckpt_interval, ckpt, ckpt_capacity};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     kda::Profiler::begin(st);
     if (dtype == KDA_F32) return from_cuda(kda::launch_prefill_simt(a, false, st));
     return from_cuda(kda::launch_prefill_tc(a, st));
+}
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_prefill(const void *q, const void *k, const void *v, const void *g,
+                             const void *beta, const float *state_in,
+                             const int32_t *cu_seqlens, int B, int64_t T, int N, int H,
+                             int dk, int dv, kda_dtype dtype, void *o, float *state_out,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv, dtype, o,
+                        state_out, workspace, workspace_bytes, stream, 0, nullptr, 0);
+}
+
+int64_t kda_prefill_checkpoint_count(const int32_t *cu_seqlens_host, int B, int64_t T, int N,
+                                     int64_t interval) {
+    if (B < 0 || T < 0 || N < 0 || interval <= 0) return -1;
+    if (cu_seqlens_host ? B != 1 : N != B) return -1;
+    if (!cu_seqlens_host) return T > 0 ? (int64_t)N * ((T - 1) / interval) : 0;
+    // the same clamping as the device: offsets into [0, T], made non-decreasing
+    int64_t total = 0, prev = 0;
+    for (int i = 0; i <= N; ++i) {
+        int64_t x = cu_seqlens_host[i];
+        x = x < 0 ? 0 : (x > T ? T : x);
+        if (x < prev) x = prev;
+        if (i > 0 && x > prev) total += (x - prev - 1) / interval;
+        prev = x;
+    }
+    return total;
+}
+
+kda_status kda_chunk_prefill_checkpointed(const void *q, const void *k, const void *v,
+                                          const void *g, const void *beta,
+                                          const float *state_in, const int32_t *cu_seqlens,
+                                          int B, int64_t T, int N, int H, int dk, int dv,
+                                          kda_dtype dtype, void *o, float *state_out,
+                                          int64_t interval, float *ckpt, int64_t ckpt_capacity,
+                                          void *workspace, size_t workspace_bytes,
+                                          void *stream) {
+    if (interval <= 0 || ckpt_capacity < 0 || (ckpt_capacity > 0 && !ckpt))
+        return KDA_ERR_INVALID_ARG;
+    if (interval % 64 != 0 || dtype != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(ckpt) & 15u) != 0) return KDA_ERR_INVALID_ARG;
+    return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv, dtype, o,
+                        state_out, workspace, workspace_bytes, stream, interval, ckpt,
+                        ckpt_capacity);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *g,
@@ -143,7 +193,28 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     kda::Profiler::begin(st);
     return from_cuda(kda::launch_decode(q, k, v, g, beta, state, N, H, dk, dtype == KDA_BF16, o,
-                                        st));
+                                        nullptr, N, nullptr, st));
+}
+
+kda_status kda_decode_step_indexed(const void *q, const void *k, const void *v, const void *g,
+                                   const void *beta, float *state_pool, const int32_t *slots,
+                                   int N, int P, int H, int dk, int dv, kda_dtype dtype, void *o,
+                                   void *stream) {
+    if (N < 0 || P < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (N > 0 && (!q || !k || !v || !g || !beta || !state_pool || !slots || !o))
+        return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)N * H > (int64_t)INT32_MAX || (int64_t)P * H > (int64_t)INT32_MAX)
+        return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    if ((reinterpret_cast<uintptr_t>(state_pool) & 15u) != 0) return KDA_ERR_INVALID_ARG;
+    uint32_t *err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kda::Profiler::begin(st);
+    return from_cuda(kda::launch_decode(q, k, v, g, beta, state_pool, N, H, dk,
+                                        dtype == KDA_BF16, o, slots, P, err, st));
 }
 
 kda_status kda_check_device_error(void *stream) {
@@ -158,7 +229,7 @@ kda_status kda_check_device_error(void *stream) {
         const uint32_t zero = 0;
         if (cudaMemcpyToSymbol(g_kda_error_word, &zero, sizeof(zero)) != cudaSuccess)
             return KDA_ERR_CUDA;
-        return KDA_ERR_TIMEOUT;
+        return (word & kda::ERR_BAD_INDEX) ? KDA_ERR_INVALID_ARG : KDA_ERR_TIMEOUT;
     }
     return KDA_OK;
 }

@@ -13,6 +13,7 @@ namespace kda {
 enum : uint32_t {
     ERR_WAIT_TIMEOUT = 1u,     // a bounded mbarrier/flag wait gave up
     ERR_SELFTEST = 2u,         // set by the bounded-wait self test
+    ERR_BAD_INDEX = 4u,        // an index argument read on the device was out of range
 };
 
 // Upper bound on the wall time of one device-side wait.  Legitimate waits in

@@ -10,7 +10,13 @@
 //
 // o is written in fp32 for either input dtype (the step accumulates in fp32).
 // The step is bound by HBM: each (n, h) state (dk*dv fp32, 64 KiB at d=128)
-// is read once and written once; everything else is ~1 KiB.  One CTA of 256
+// is read once and written once; everything else is ~1 KiB.
+//
+// Indexed form (continuous batching over a state pool): request n's state is
+// pool entry slots[n] of P, so the per-request state stays a single copy that
+// the step updates in place wherever the serving layer keeps it.  A slot
+// outside [0, P) is not touched: the unit is skipped and ERR_BAD_INDEX is
+// recorded in the device error word.  One CTA of 256
 // threads per (n, h).  Each thread keeps a (DK/RG) x 4 block of S in
 // registers (loaded as coalesced 16-byte vectors, a warp covering whole rows),
 // reduces p and y over its rows, the CTA reduces across row groups through
@@ -25,7 +31,8 @@ template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256, 2)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const Tin *__restrict__ g, const Tin *__restrict__ beta, float *__restrict__ state,
-              float *__restrict__ o, int units) {
+              float *__restrict__ o, int units, int H, const int32_t *__restrict__ slots, int P,
+              uint32_t *err) {
     constexpr int NT = 256;
     constexpr int CG = DV / 4;        // 16-byte column groups per row
     constexpr int RG = NT / CG;       // row groups
@@ -40,7 +47,16 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     __shared__ float dl[DV];
     __shared__ float kq_sh, b_sh;
 
-    float4 *S4 = reinterpret_cast<float4 *>(state + (size_t)unit * DK * DV);
+    size_t sunit = (size_t)unit;   // state entry of this (request, head)
+    if (slots != nullptr) {
+        const int n = unit / H, slot = slots[n];
+        if (slot < 0 || slot >= P) {
+            if (tid == 0 && err) atomicOr(err, ERR_BAD_INDEX);
+            return;
+        }
+        sunit = (size_t)slot * H + (unit - n * H);
+    }
+    float4 *S4 = reinterpret_cast<float4 *>(state + sunit * DK * DV);
 
     // issue the state loads first: they are the long pole
     float4 s[RPT];
@@ -110,11 +126,11 @@ namespace kda {
 
 template <int D, typename Tin>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const void *g,
-                                   const void *beta, float *state, void *o, int units,
-                                   cudaStream_t st) {
+                                   const void *beta, float *state, void *o, int units, int H,
+                                   const int32_t *slots, int P, uint32_t *err, cudaStream_t st) {
     decode_kernel<D, D, Tin><<<units, 256, 0, st>>>(
         (const Tin *)q, (const Tin *)k, (const Tin *)v, (const Tin *)g, (const Tin *)beta,
-        state, (float *)o, units);
+        state, (float *)o, units, H, slots, P, err);
     cudaError_t e = cudaGetLastError();
     Profiler::mark(st);
     return e;
@@ -122,14 +138,18 @@ static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, 
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *g,
                           const void *beta, float *state, int N, int H, int d, bool bf16,
-                          void *o, cudaStream_t st) {
+                          void *o, const int32_t *slots, int P, uint32_t *err, cudaStream_t st) {
     const int units = N * H;
     if (units == 0) return cudaSuccess;
     if (d == 64)
-        return bf16 ? launch_decode_t<64, __nv_bfloat16>(q, k, v, g, beta, state, o, units, st)
-                    : launch_decode_t<64, float>(q, k, v, g, beta, state, o, units, st);
-    return bf16 ? launch_decode_t<128, __nv_bfloat16>(q, k, v, g, beta, state, o, units, st)
-                : launch_decode_t<128, float>(q, k, v, g, beta, state, o, units, st);
+        return bf16 ? launch_decode_t<64, __nv_bfloat16>(q, k, v, g, beta, state, o, units, H,
+                                                         slots, P, err, st)
+                    : launch_decode_t<64, float>(q, k, v, g, beta, state, o, units, H, slots, P,
+                                                 err, st);
+    return bf16 ? launch_decode_t<128, __nv_bfloat16>(q, k, v, g, beta, state, o, units, H, slots,
+                                                      P, err, st)
+                : launch_decode_t<128, float>(q, k, v, g, beta, state, o, units, H, slots, P,
+                                              err, st);
 }
 
 }  // namespace kda

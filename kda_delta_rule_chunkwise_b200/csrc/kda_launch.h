@@ -20,6 +20,11 @@ struct PrefillArgs {
     void *workspace;
     size_t workspace_bytes;
     uint32_t *err;               // device error word
+    // intermediate states: every ckpt_interval tokens (a multiple of the chunk
+    // length; 0 = none) inside each sequence, into ckpt [ckpt_capacity, H, dk, dv]
+    int64_t ckpt_interval = 0;
+    float *ckpt = nullptr;
+    int64_t ckpt_capacity = 0;
 };
 
 // Optional per-kernel event recording (see kda_profile_enable).  Launchers
@@ -32,9 +37,10 @@ struct Profiler {
 cudaError_t launch_prefill_simt(const PrefillArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st);
 size_t prefill_tc_workspace_bytes(int64_t rows, int N, int H, int d);
+// slots == nullptr: request n owns state entry n; otherwise entry slots[n] of P.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *g,
                           const void *beta, float *state, int N, int H, int d, bool bf16,
-                          void *o, cudaStream_t st);
+                          void *o, const int32_t *slots, int P, uint32_t *err, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t timeout_us, uint32_t *err, cudaStream_t st);
 
 }  // namespace kda

@@ -70,22 +70,25 @@ constexpr uint32_t kWPKBlock = 16384;    // bytes between the two 64-column K-bl
 constexpr uint32_t kKhMNBlock = 8192;    // bytes between the two 64-channel MN-blocks of Khat
 
 // Workspace header: int32 chunk_off[N+1] (first chunk of each sequence, total
-// in chunk_off[N]) followed by int32 bound[N+1] (the row offsets actually used:
+// in chunk_off[N]), int32 bound[N+1] (the row offsets actually used:
 // cu_seqlens clamped to [0, T] and made non-decreasing by a running maximum,
 // so that sequences never overlap and the chunk total never exceeds the
-// workspace bound).  Then the slots, 1024-aligned.
+// workspace bound) and int32 ckpt_off[N+1] (first intermediate-state entry of
+// each sequence, total in ckpt_off[N]).  Then the slots, 1024-aligned.
 __host__ __device__ inline uint32_t header_bytes(int N) {
-    return (uint32_t)(((size_t)(N + 1) * 8 + 1023) & ~(size_t)1023);
+    return (uint32_t)(((size_t)(N + 1) * 12 + 1023) & ~(size_t)1023);
 }
 
 // ======================================================================
 // chunk table (one block of 1024 threads)
 // ======================================================================
 __global__ void __launch_bounds__(1024)
-chunk_table_kernel(const int32_t *__restrict__ cu, int64_t T, int N, int32_t *__restrict__ hdr) {
+chunk_table_kernel(const int32_t *__restrict__ cu, int64_t T, int N, int64_t ckpt_interval,
+                   int32_t *__restrict__ hdr) {
     __shared__ int64_t part[1024];
     int32_t *chunk_off = hdr;
     int32_t *bound = hdr + (N + 1);
+    int32_t *ckpt_off = hdr + 2 * (N + 1);
     const int tid = threadIdx.x, nt = blockDim.x;
     const int per = (N + 1 + nt - 1) / nt;             // offsets 0..N, contiguous per thread
     const int i0 = tid * per, i1 = min(N + 1, i0 + per);
@@ -113,32 +116,39 @@ chunk_table_kernel(const int32_t *__restrict__ cu, int64_t T, int N, int32_t *__
         __syncthreads();
     }
     __threadfence_block();
-    // chunks per sequence, exclusive sum
-    auto nchunks = [&](int n) -> int64_t {
-        const int64_t len = cu ? (int64_t)bound[n + 1] - bound[n] : T;
-        return (len + C - 1) / C;
+    // chunks and intermediate states per sequence, exclusive sums
+    auto seqlen = [&](int n) -> int64_t { return cu ? (int64_t)bound[n + 1] - bound[n] : T; };
+    auto nchunks = [&](int n) -> int64_t { return (seqlen(n) + C - 1) / C; };
+    auto nckpt = [&](int n) -> int64_t {   // states after m * interval tokens, m >= 1, inside
+        const int64_t len = seqlen(n);
+        return (ckpt_interval > 0 && len > 0) ? (len - 1) / ckpt_interval : 0;
     };
     const int pn = (N + nt - 1) / nt;
     const int n0 = tid * pn, n1 = min(N, n0 + pn);
-    int64_t sum = 0;
-    for (int n = n0; n < n1; ++n) sum += nchunks(n);
-    part[tid] = sum;
-    __syncthreads();
-    if (tid == 0) {
-        int64_t acc = 0;
-        for (int i = 0; i < nt; ++i) {
-            const int64_t v = part[i];
-            part[i] = acc;
-            acc += v;
+    auto exclusive_sum = [&](auto count, int32_t *out) {
+        int64_t sum = 0;
+        for (int n = n0; n < n1; ++n) sum += count(n);
+        part[tid] = sum;
+        __syncthreads();
+        if (tid == 0) {
+            int64_t acc = 0;
+            for (int i = 0; i < nt; ++i) {
+                const int64_t v = part[i];
+                part[i] = acc;
+                acc += v;
+            }
+            out[N] = (int32_t)acc;
         }
-        chunk_off[N] = (int32_t)acc;
-    }
-    __syncthreads();
-    int64_t acc = part[tid];
-    for (int n = n0; n < n1; ++n) {
-        chunk_off[n] = (int32_t)acc;
-        acc += nchunks(n);
-    }
+        __syncthreads();
+        int64_t acc = part[tid];
+        for (int n = n0; n < n1; ++n) {
+            out[n] = (int32_t)acc;
+            acc += count(n);
+        }
+        __syncthreads();
+    };
+    exclusive_sum(nchunks, chunk_off);
+    exclusive_sum(nckpt, ckpt_off);
 }
 
 // Rows [a, b) of sequence n (bound[] from the header when packed).
@@ -857,7 +867,8 @@ __global__ void __launch_bounds__(384, 1)
 state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                   const int32_t *__restrict__ cu, int64_t T, int N, int H,
                   const uint8_t *__restrict__ ws, float *__restrict__ o,
-                  float *state_out, uint32_t *err) {
+                  float *state_out, int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity,
+                  uint32_t *err) {
     using Lay = BLayout<DVS>;
     constexpr int NSL = D / DVS;
     constexpr int CPR = DVS / 8;   // 16-byte pieces per V row
@@ -890,18 +901,18 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     if (tid == 0) {
         for (int i = 0; i < Lay::NST; ++i) {
             mbar_init(&bars[FULL0 + i], 1);
-            mbar_init(&bars[EMPTY0 + i], 2);   // both state-update issuers commit
+            mbar_init(&bars[EMPTY0 + i], 1);
             mbar_init(&bars[VRAW0 + i], 32);
             mbar_init(&bars[VREADY0 + i], 1);
         }
-        mbar_init(&bars[TDFULL0], 4);   // four state-term issuers commit
-        mbar_init(&bars[TDFULL1], 4);
+        mbar_init(&bars[TDFULL0], 1);
+        mbar_init(&bars[TDFULL1], 1);
         mbar_init(&bars[TDEMPTY0], 4);
         mbar_init(&bars[TDEMPTY1], 4);
         mbar_init(&bars[TSSCALED], 1);
-        mbar_init(&bars[TSFULL], 2);
-        mbar_init(&bars[DRAIN_S], 4);
-        mbar_init(&bars[DRAIN_U], 2);
+        mbar_init(&bars[TSFULL], 1);
+        mbar_init(&bars[DRAIN_S], 1);
+        mbar_init(&bars[DRAIN_U], 1);
         mbar_fence_init();
         *abort_flag = 0u;
         *s_grp_ok = 1u;
@@ -979,9 +990,9 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         // ------------------------------------------------ U / O epilogue (+ state-update issue)
         const int quad = warp - 4;
         const int row = 32 * quad + lane;
-        // lane 0 of warps 4 and 5 each issue half of the state update (a tcgen05.mma
-        // costs its issuing thread tens of cycles; two issuers halve that path)
-        const bool issuer = (quad < 2 && lane == 0);
+        // one thread issues the whole state update: its K steps then accumulate in
+        // a fixed order and the result is the same on every run
+        const bool issuer = (warp == 4 && lane == 0);
         const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
         bool ok = true;
         for (int j = 0; j < nch; ++j) {
@@ -1035,7 +1046,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotKh, kKhMNBlock, 1024, SW_128B);
                         const uint64_t bd0 = smem_desc(sbase + Lay::oUB, Lay::kKGroup, 128, SW_NONE);
 #pragma unroll
-                        for (int kk = 2 * quad; kk < 2 * quad + 2; ++kk)
+                        for (int kk = 0; kk < 4; ++kk)
                             mma_f16(tTS, ad0 + (uint64_t)(kk * 2048 / 16),
                                     bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_mm, 1);
                         mma_commit(&bars[TSFULL]);
@@ -1056,8 +1067,9 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         // ------------------------------------------------ state epilogue (+ chunk-product issue)
         const int quad = warp - 8;
         const int c = 32 * quad + lane;   // key channel = TMEM lane
-        const bool issuer = (warp == 8 && lane == 0);   // V terms, TSSCALED, group status
-        const bool sissuer = (lane == 0);                 // a quarter of the state term each
+        // one thread issues the V and state terms: their K steps then accumulate in a
+        // fixed order and the result is the same on every run
+        const bool issuer = (warp == 8 && lane == 0);
         const uint32_t tS = taddr(tTS, 32 * quad, 0);
         const size_t srow = (((size_t)n * H + h) * D + c) * D + j0;
         const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
@@ -1103,13 +1115,12 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                    (j < 2 || mbar_try_wait(&bars[TDEMPTY0 + (j & 1)], ((j >> 1) + 1) & 1));
         };
         // After the fp16 copy of S_j and the scaled TS are in place: the elected
-        // thread releases the state update of chunk j (TSSCALED) and makes sure
-        // the V term of chunk j has been issued; then lane 0 of each state warp
-        // adds a quarter of [-W; P]_j S_j onto it in TD[j % 2].  When the next
-        // chunk's slot, V slice and accumulator are already free, the elected
-        // thread also issues that chunk's V term: the pipe then runs it while
-        // the U warps copy U out, and only the state term remains on the
-        // chunk-to-chunk path.
+        // thread releases the state update of chunk j (TSSCALED), issues
+        // [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j into TD[j % 2] and tells the
+        // group whether it succeeded.  When the next chunk's slot, V slice and
+        // accumulator are already free it also issues that chunk's V term: the
+        // pipe then runs it while the U warps copy U out, and only the state
+        // term remains on the chunk-to-chunk path.
         // (ok_in: the elected thread's own status; the group status travels in
         // s_grp_ok, written only between the two barriers below)
         auto issue_chunk = [&](int j, bool ok_in) {
@@ -1131,31 +1142,27 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         issue_vterm(j);
                     }
                 }
-                *s_grp_ok = okk ? 1u : 0u;
-                tc_fence_before();
-            }
-            named_bar(2, 128);   // the V term of chunk j is issued before any state term
-            const bool okk = *s_grp_ok != 0u;
-            if (sissuer && okk) {
-                tc_fence_after();
-                const uint32_t tTD = b ? tTD1 : tTD0;
-                const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotWP, 16, 1024, SW_128B);
-                const uint64_t bd0 = smem_desc(sbase + Lay::oSB, Lay::kKGroup, 128, SW_NONE);
-#pragma unroll
-                for (int kk = 2 * quad; kk < 2 * quad + 2; ++kk)
-                    mma_f16(tTD, ad0 + (uint64_t)(((kk >> 2) * kWPKBlock + (kk & 3) * 32) / 16),
-                            bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, 1);
-                mma_commit(&bars[TDFULL0 + b]);
-            }
-            if (issuer && okk) {
-                // early V term of chunk j + 1, only if nothing has to be waited for
-                const int jn = j + 1;
-                if (jn < nch && vterm_ready(jn)) {
+                if (okk) {
                     tc_fence_after();
-                    issue_vterm(jn);
+                    const uint32_t tTD = b ? tTD1 : tTD0;
+                    const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotWP, 16, 1024, SW_128B);
+                    const uint64_t bd0 = smem_desc(sbase + Lay::oSB, Lay::kKGroup, 128, SW_NONE);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_f16(tTD, ad0 + (uint64_t)(((kk >> 2) * kWPKBlock + (kk & 3) * 32) / 16),
+                                bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, 1);
+                    mma_commit(&bars[TDFULL0 + b]);
+                    // early V term of chunk j + 1, only if nothing has to be waited for
+                    const int jn = j + 1;
+                    if (jn < nch && vterm_ready(jn)) {
+                        tc_fence_after();
+                        issue_vterm(jn);
+                    }
                 }
+                *s_grp_ok = okk ? 1u : 0u;
             }
-            return okk;
+            named_bar(2, 128);
+            return *s_grp_ok != 0u;
         };
         auto gamma_of = [&](int j, bool &ok) {
             if (ok) ok = mbar_wait_abortable(&bars[FULL0 + j % NST], full_par(j), err, abort_flag);
@@ -1199,6 +1206,23 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         tmem_ld16(tS + 16 * p, *reinterpret_cast<float(*)[16]>(xa + 16 * p));
                     tmem_wait_ld();
                 }
+                // intermediate state: S after (j + 1) C tokens, when that is a multiple of
+                // the interval strictly inside the sequence
+                if (ckpt_interval > 0 && ok) {
+                    const int64_t done = (int64_t)(j + 1) * C;
+                    if (done % ckpt_interval == 0 && done < rb - ra) {
+                        const int64_t e = (int64_t)chunk_off[2 * (N + 1) + n] + done / ckpt_interval - 1;
+                        if (e < ckpt_capacity) {
+                            float4 *dst = reinterpret_cast<float4 *>(
+                                ckpt + (((size_t)e * H + h) * D + c) * D + j0);
+#pragma unroll
+                            for (int i = 0; i < DVS / 4; ++i)
+                                dst[i] = make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
+                        } else if (lane == 0) {
+                            atomicOr(err, ERR_BAD_INDEX);   // the caller's array is too small
+                        }
+                    }
+                }
                 if (j + 1 == nch) break;
                 const float gam = gamma_of(j + 1, ok);
                 if (ok) put_state(xa, gam);
@@ -1211,7 +1235,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                     reinterpret_cast<float4 *>(state_out + srow)[i] =
                         make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
             }
-            if (sissuer) {
+            if (issuer) {
                 mma_commit(&bars[DRAIN_S]);
                 mbar_wait(&bars[DRAIN_S], 0, err, 1ull << 28);
             }
@@ -1246,7 +1270,8 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
     const int grid = a.N * a.H * (tc::D / DVS);
     kern<<<grid, 384, Lay::kBytes, st>>>((const __nv_bfloat16 *)a.v, a.state_in, a.cu_seqlens,
                                          a.T, a.N, a.H, (const uint8_t *)a.workspace,
-                                         (float *)a.o, a.state_out, a.err);
+                                         (float *)a.o, a.state_out, a.ckpt_interval, a.ckpt,
+                                         a.ckpt_capacity, a.err);
     e = cudaGetLastError();
     Profiler::mark(st);
     return e;
@@ -1256,6 +1281,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
     if (a.dk != tc::D || a.dv != tc::D) return cudaErrorInvalidValue;
     uint8_t *ws = (uint8_t *)a.workspace;
     tc::chunk_table_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.T, a.N,
+                                               a.ckpt_interval,
                                                reinterpret_cast<int32_t *>(ws));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

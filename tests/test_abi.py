@@ -111,6 +111,55 @@ def test_decode_zero_sequences_is_a_no_op(lib):
     assert binding.raw_decode(_dargs(N=0)) == binding.KDA_OK
 
 
+# ---------------------------------------------------------------- intermediate states
+
+def test_checkpoint_count_dense_and_packed(lib):
+    count = lambda cu, B, T, N, iv: lib.kda_prefill_checkpoint_count(cu, B, T, N, iv)
+    assert count(None, 3, 1000, 3, 128) == 3 * 7          # 128 .. 896 inside 1000 tokens
+    assert count(None, 2, 1024, 2, 512) == 2 * 1          # 512 only; 1024 is state_out
+    assert count(None, 1, 0, 1, 64) == 0
+    cu = (ctypes.c_int32 * 5)(0, 64, 64, 700, 1000)     # lengths 64, 0, 636, 300
+    assert count(cu, 1, 1000, 4, 64) == 0 + 0 + 9 + 4
+    bad = (ctypes.c_int32 * 4)(0, 900, 500, 5000)        # clamped to 0, 900, 900, 1000
+    assert count(bad, 1, 1000, 3, 256) == 3 + 0 + 0
+    assert count(None, 2, 10, 2, 0) == -1 and count(None, 2, 10, 3, 64) == -1
+
+
+def _cargs(**kw):
+    base = _args(interval=128, ckpt=64, ckpt_capacity=4, dtype=binding.KDA_BF16)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(interval=0), "KDA_ERR_INVALID_ARG"), (dict(interval=-64), "KDA_ERR_INVALID_ARG"),
+    (dict(ckpt=None), "KDA_ERR_INVALID_ARG"), (dict(ckpt=72), "KDA_ERR_INVALID_ARG"),
+    (dict(ckpt_capacity=-1), "KDA_ERR_INVALID_ARG"),
+    (dict(interval=100), "KDA_ERR_UNSUPPORTED"), (dict(dtype=binding.KDA_F32), "KDA_ERR_UNSUPPORTED")])
+def test_checkpointed_prefill_rejects(lib, bad, code):
+    assert binding.raw_prefill_checkpointed(_cargs(**bad)) == getattr(binding, code)
+
+
+def _iargs(**kw):
+    base = _dargs(slots=64, P=4)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("bad", [dict(N=-1), dict(P=-1), dict(H=0), dict(state=None),
+                                 dict(slots=None), dict(o=None), dict(dtype=3), dict(state=18)])
+def test_decode_indexed_rejects_invalid_arguments(lib, bad):
+    assert binding.raw_decode_indexed(_iargs(**bad)) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_decode_indexed_rejects_unsupported_sizes(lib):
+    assert binding.raw_decode_indexed(_iargs(dk=128, dv=64)) == binding.KDA_ERR_UNSUPPORTED
+
+
+def test_decode_indexed_zero_requests_is_a_no_op(lib):
+    assert binding.raw_decode_indexed(_iargs(N=0)) == binding.KDA_OK
+
+
 def test_selftest_rejects_bad_limits(lib):
     assert lib.kda_selftest_bounded_wait(0, None) == binding.KDA_ERR_INVALID_ARG
     assert lib.kda_selftest_bounded_wait(10**7 + 1, None) == binding.KDA_ERR_INVALID_ARG

@@ -61,3 +61,69 @@ def test_decode_full_n256_h32_sampled():
     go, wo, gs, ws = run_steps(inp, 20, n_sel=sel)
     assert rel_err(go, wo) <= TOL_BF16
     assert rel_err(gs, ws) <= TOL_BF16
+
+
+# ---------------------------------------------------------------- pooled (indexed) state
+
+def _pool_case(P, N, H, d, dtype, seed):
+    gen = np.random.default_rng(seed)
+    inp = kin.decode_inputs(3, N, H, d, d, dtype, seed=seed)
+    pool = torch.randn((P, H, d, d), generator=torch.Generator().manual_seed(seed)) * 0.1
+    slots = torch.as_tensor(gen.permutation(P)[:N].astype(np.int32))
+    return inp, pool, slots
+
+
+@pytest.mark.parametrize("dtype,d,tol", [("bf16", 128, TOL_BF16), ("f32", 64, TOL_F32)])
+def test_decode_indexed_matches_oracle_and_leaves_other_entries(dtype, d, tol):
+    P, N, H = 24, 10, 3
+    inp, pool, slots = _pool_case(P, N, H, d, dtype, seed=5)
+    pool_g = pool.clone().cuda()
+    slots_g = slots.cuda()
+    S_ref = pool.double().numpy()[slots.numpy()]
+    for t in range(3):
+        cu = lambda x: x[t].contiguous().cuda()
+        o = binding.kda_decode_step_indexed(cu(inp.q), cu(inp.k), cu(inp.v), cu(inp.g),
+                                            cu(inp.beta), pool_g, slots_g)
+        o_ref, S_ref = oracle.decode_step(inp.q[t], inp.k[t], inp.v[t], inp.g[t], inp.beta[t],
+                                          S_ref)
+        assert rel_err(to_np(o), o_ref) <= tol, f"step {t}: output"
+    assert binding.kda_check_device_error() == binding.KDA_OK
+    got = to_np(pool_g)
+    assert rel_err(got[slots.numpy()], S_ref) <= tol, "touched entries"
+    untouched = np.setdiff1d(np.arange(P), slots.numpy())
+    np.testing.assert_array_equal(got[untouched], pool.double().numpy()[untouched])
+
+
+def test_decode_indexed_identity_slots_equal_the_dense_step():
+    """slots = 0..N-1 over a pool of exactly N entries is the dense step, bit for bit."""
+    inp = kin.decode_inputs(1, 6, 4, 128, 128, "bf16", seed=9)
+    dense = inp.state.clone().cuda()
+    pooled = inp.state.clone().cuda()
+    cu = lambda x: x[0].contiguous().cuda()
+    o1 = binding.kda_decode_step(cu(inp.q), cu(inp.k), cu(inp.v), cu(inp.g), cu(inp.beta), dense)
+    o2 = binding.kda_decode_step_indexed(cu(inp.q), cu(inp.k), cu(inp.v), cu(inp.g), cu(inp.beta),
+                                         pooled, torch.arange(6, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(dense, pooled)
+
+
+def test_decode_indexed_out_of_range_slot_is_skipped_and_reported():
+    P, N, H = 8, 4, 2
+    inp, pool, slots = _pool_case(P, N, H, 128, "bf16", seed=6)
+    slots[2] = P          # outside the pool: this request is skipped on the device
+    pool_g = pool.clone().cuda()
+    o = torch.full((N, H, 128), float("nan"), device="cuda")
+    cu = lambda x: x[0].contiguous().cuda()
+    binding.kda_decode_step_indexed(cu(inp.q), cu(inp.k), cu(inp.v), cu(inp.g), cu(inp.beta),
+                                    pool_g, slots.cuda(), o=o)
+    assert binding.kda_check_device_error() == binding.KDA_ERR_INVALID_ARG
+    assert binding.kda_check_device_error() == binding.KDA_OK      # cleared
+    ok = [0, 1, 3]
+    o_ref, S_ref = oracle.decode_step(inp.q[0][ok], inp.k[0][ok], inp.v[0][ok], inp.g[0][ok],
+                                      inp.beta[0][ok], pool.double().numpy()[slots.numpy()[ok]])
+    assert rel_err(to_np(o)[ok], o_ref) <= TOL_BF16
+    assert torch.isnan(o[2]).all()                                  # not written
+    got = to_np(pool_g)
+    assert rel_err(got[slots.numpy()[ok]], S_ref) <= TOL_BF16
+    untouched = np.setdiff1d(np.arange(P), slots.numpy()[ok])
+    np.testing.assert_array_equal(got[untouched], pool.double().numpy()[untouched])

@@ -162,3 +162,15 @@ def test_bf16_full_varlen_64_sequences():
     lens = np.diff(inp.cu_seqlens.cpu().numpy())
     seqs = [int(np.argmin(lens)), int(np.argmax(lens)), 17]
     check(inp, TOL_BF16, heads=[3], seqs=seqs, what="varlen 64 seqs")
+
+
+def test_bf16_prefill_is_deterministic():
+    """Two identical calls give the same bits (one issuing thread per accumulator)."""
+    inp = kin.prefill_inputs(1, 1065, 8, 128, 128, "bf16", seed=33, decay="split", state="normal",
+                             lengths=[300, 0, 700, 65])
+    d = inp.to("cuda")
+    o1, s1 = binding.kda_chunk_prefill(d.q, d.k, d.v, d.g, d.beta, d.state_in, d.cu_seqlens)
+    o2, s2 = binding.kda_chunk_prefill(d.q, d.k, d.v, d.g, d.beta, d.state_in, d.cu_seqlens)
+    torch.cuda.synchronize()
+    rows = torch.cat([torch.arange(0, 300), torch.arange(300, 1000), torch.arange(1000, 1065)])
+    assert torch.equal(o1[0, rows], o2[0, rows]) and torch.equal(s1, s2)

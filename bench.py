@@ -337,7 +337,36 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
                     "unit": "tokens/s",
                     "overhead_vs_plain": round(c_ms / args.steps / ms_step - 1.0, 4)}
         del ck
-    extra = {"prefill_checkpointed": ckpt_res}
+    # ---------------- the same step from raw projections: gates from logits and q, k
+    # normalised inside the prefill (same shapes; fresh inputs of that form)
+    prep_res = None
+    if args.prep and d.cu_seqlens is None:
+        raw = kin.prefill_raw_inputs(B, T, H, 128, 128, "bf16", seed=args.seed + 3000 + rank,
+                                     state=w["state"], device=dev)
+        flags = binding.KDA_PREP_GATE_LOGIT | binding.KDA_PREP_L2NORM_QK
+
+        def prep_step():
+            binding.kda_chunk_prefill_ex(raw.q, raw.k, raw.v, raw.g, raw.beta, raw.state_in, None,
+                                         flags=flags, o=o, state_out=s_out, workspace=ws)
+
+        for _ in range(args.warmup):
+            prep_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        st = torch.cuda.current_stream()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(st)
+        for _ in range(args.steps):
+            prep_step()
+        ev1.record(st)
+        torch.cuda.synchronize()
+        p_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        prep_res = {"flags": "gate_logit|l2norm_qk", "ms_per_step": round(p_ms / args.steps, 4),
+                    "value": aggregate_throughput(tokens, world, args.steps, p_ms),
+                    "unit": "tokens/s", "overhead_vs_plain": round(p_ms / args.steps / ms_step - 1.0, 4)}
+        del raw
+    extra = {"prefill_checkpointed": ckpt_res, "prefill_preprocessed": prep_res}
 
     del d, o, s_out, ws
     torch.cuda.empty_cache()
@@ -525,6 +554,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-prep", dest="prep", action="store_false",
+                    help="skip timing the step with gate/normalisation preprocessing")
     ap.add_argument("--ckpt-interval", type=int, default=512,
                     help="also time the prefill step with intermediate states every this many "
                          "tokens (a multiple of 64; 0 skips it)")

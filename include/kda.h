@@ -129,7 +129,8 @@ KDA_API kda_status kda_chunk_prefill(const void *q, const void *k, const void *v
  * sharing a prefix resumes from one instead of recomputing it; the pages give
  * no interface for it.  Everything else is exactly kda_chunk_prefill.
  *  interval       tokens between snapshots: a positive multiple of 64 (the
- *                 chunk length), else KDA_ERR_UNSUPPORTED (also for KDA_F32)
+ *                 chunk length), else KDA_ERR_UNSUPPORTED (also for KDA_F32
+ *                 and for d = 64: snapshots come from the d = 128 bf16 path)
  *  ckpt           fp32 [ckpt_capacity, H, dk, dv], 16-byte aligned.  Entry
  *                 e = (number of snapshots of sequences 0..n-1) + m - 1 holds
  *                 sequence n's m-th snapshot; kda_prefill_checkpoint_count()
@@ -145,6 +146,36 @@ KDA_API kda_status kda_chunk_prefill_checkpointed(const void *q, const void *k, 
                                           int64_t interval, float *ckpt, int64_t ckpt_capacity,
                                           void *workspace, size_t workspace_bytes,
                                           void *stream);
+
+/*
+ * Input preprocessing done inside the prefill (flags of kda_chunk_prefill_ex):
+ *  KDA_PREP_GATE_LOGIT   g holds gate logits x; the log-decay used is
+ *                        g = -5 sigmoid(x), which lies in (-5, 0) by
+ *                        construction (the lower bound of neurohive.io "Kimi
+ *                        K3 ... overview", section "Sequence length: hybrid KDA
+ *                        and Gated MLA attention", written as a parametrisation)
+ *  KDA_PREP_L2NORM_QK    q and k are normalised to unit L2 norm over dk per
+ *                        (token, head) before use; an all-zero vector stays zero
+ * The pages do not give the layer's gate form; this is the parametrisation the
+ * synthetic inputs use, moved into the kernel so that callers pass raw
+ * projections.
+ */
+enum { KDA_PREP_GATE_LOGIT = 1u, KDA_PREP_L2NORM_QK = 2u };
+
+/*
+ * The general prefill: kda_chunk_prefill with input preprocessing `flags`
+ * (KDA_PREP_*; 0 = none) and, when ckpt_interval > 0, the intermediate states
+ * of kda_chunk_prefill_checkpointed.  flags != 0 needs KDA_BF16 and d = 128
+ * (else KDA_ERR_UNSUPPORTED); unknown flag bits are KDA_ERR_INVALID_ARG.  With
+ * flags = 0 and ckpt_interval = 0 it is exactly kda_chunk_prefill.
+ */
+KDA_API kda_status kda_chunk_prefill_ex(const void *q, const void *k, const void *v,
+                                const void *g, const void *beta,
+                                const float *state_in, const int32_t *cu_seqlens,
+                                int B, int64_t T, int N, int H, int dk, int dv,
+                                kda_dtype dtype, uint32_t flags, void *o, float *state_out,
+                                int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Number of snapshots kda_chunk_prefill_checkpointed() writes, from the

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_F32, KDA_BF16 = 0, 1
+KDA_PREP_GATE_LOGIT, KDA_PREP_L2NORM_QK = 1, 2
 _DTYPE = {torch.float32: KDA_F32, torch.bfloat16: KDA_BF16}
 
 # Every symbol the public header declares.
@@ -26,6 +27,7 @@ EXPORTED = (
     "kda_chunk_prefill_workspace_bytes",
     "kda_chunk_prefill",
     "kda_chunk_prefill_checkpointed",
+    "kda_chunk_prefill_ex",
     "kda_prefill_checkpoint_count",
     "kda_decode_step",
     "kda_decode_step_indexed",
@@ -67,6 +69,9 @@ def load(path: str = LIB_PATH):
                                                    i32, i32, i32, vp, vp, i64, vp, i64, vp, sz,
                                                    vp]
     lib.kda_chunk_prefill_checkpointed.restype = i32
+    lib.kda_chunk_prefill_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                         i32, ctypes.c_uint32, vp, vp, i64, vp, i64, vp, sz, vp]
+    lib.kda_chunk_prefill_ex.restype = i32
     lib.kda_prefill_checkpoint_count.argtypes = [vp, i32, i64, i32, i64]
     lib.kda_prefill_checkpoint_count.restype = i64
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
@@ -198,6 +203,38 @@ def kda_chunk_prefill_checkpointed(q, k, v, g, beta, state_in=None, cu_seqlens=N
         _ptr(ckpt) if ckpt.numel() else None, ckpt.shape[0],
         _ptr(workspace) if need else None, ws_bytes if need else 0, _stream(stream))
     _check(code, "kda_chunk_prefill_checkpointed")
+    return o, state_out, ckpt
+
+
+def kda_chunk_prefill_ex(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, flags=0,
+                         ckpt_interval=0, ckpt=None, o=None, state_out=None, workspace=None,
+                         stream=None):
+    """The general prefill: preprocessing `flags` (KDA_PREP_*) and, with ckpt_interval > 0,
+    intermediate states.  Returns (o, state_out, ckpt or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta),
+                    ("state_in", state_in), ("cu_seqlens", cu_seqlens), ("ckpt", ckpt)):
+        _contig(name, t)
+    if ckpt_interval and ckpt is None:
+        cnt = kda_prefill_checkpoint_count(cu_seqlens, B, T, ckpt_interval)
+        ckpt = torch.empty((cnt, H, dk, dv), dtype=torch.float32, device=q.device)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if state_out is None:
+        state_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = kda_chunk_prefill_workspace_bytes(B * T, N, H, dk, dv, q.dtype)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    has_ck = ckpt is not None and ckpt.numel() > 0
+    code = load().kda_chunk_prefill_ex(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens),
+        B, T, N, H, dk, dv, _DTYPE[q.dtype], int(flags), _ptr(o), _ptr(state_out),
+        int(ckpt_interval), _ptr(ckpt) if has_ck else None, ckpt.shape[0] if has_ck else 0,
+        _ptr(workspace) if need else None, ws_bytes if need else 0, _stream(stream))
+    _check(code, "kda_chunk_prefill_ex")
     return o, state_out, ckpt
 
 

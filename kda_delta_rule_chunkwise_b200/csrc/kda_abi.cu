@@ -109,7 +109,8 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
                         const void *beta, const float *state_in, const int32_t *cu_seqlens,
                         int B, int64_t T, int N, int H, int dk, int dv, kda_dtype dtype, void *o,
                         float *state_out, void *workspace, size_t workspace_bytes, void *stream,
-                        int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity) {
+                        int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity,
+                        uint32_t flags) {
     if (B < 0 || T < 0 || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (cu_seqlens ? B != 1 : N != B) return KDA_ERR_INVALID_ARG;
@@ -127,10 +128,13 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
     if (!err) return KDA_ERR_CUDA;
     kda::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv,
                        o, state_out, workspace, workspace_bytes, err,
-                       ckpt_interval, ckpt, ckpt_capacity};
+                       ckpt_interval, ckpt, ckpt_capacity, flags};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     kda::Profiler::begin(st);
-    if (dtype == KDA_F32) return from_cuda(kda::launch_prefill_simt(a, false, st));
+    // the tensor-core path is for bf16 at d = 128; fp32, and bf16 at d = 64, take the
+    // fp32 SIMT kernel (which reads either input type)
+    if (dtype == KDA_F32 || dk != 128)
+        return from_cuda(kda::launch_prefill_simt(a, dtype == KDA_BF16, st));
     return from_cuda(kda::launch_prefill_tc(a, st));
 }
 }  // namespace
@@ -143,7 +147,27 @@ kda_status kda_chunk_prefill(const void *q, const void *k, const void *v, const 
                              int dk, int dv, kda_dtype dtype, void *o, float *state_out,
                              void *workspace, size_t workspace_bytes, void *stream) {
     return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv, dtype, o,
-                        state_out, workspace, workspace_bytes, stream, 0, nullptr, 0);
+                        state_out, workspace, workspace_bytes, stream, 0, nullptr, 0, 0u);
+}
+
+kda_status kda_chunk_prefill_ex(const void *q, const void *k, const void *v, const void *g,
+                                const void *beta, const float *state_in,
+                                const int32_t *cu_seqlens, int B, int64_t T, int N, int H,
+                                int dk, int dv, kda_dtype dtype, uint32_t flags, void *o,
+                                float *state_out, int64_t ckpt_interval, float *ckpt,
+                                int64_t ckpt_capacity, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    if ((flags & ~(uint32_t)(KDA_PREP_GATE_LOGIT | KDA_PREP_L2NORM_QK)) != 0)
+        return KDA_ERR_INVALID_ARG;
+    if (ckpt_interval < 0 || ckpt_capacity < 0 || (ckpt_capacity > 0 && !ckpt))
+        return KDA_ERR_INVALID_ARG;
+    if ((flags != 0 || ckpt_interval > 0) && (dtype != KDA_BF16 || dk != 128))
+        return KDA_ERR_UNSUPPORTED;
+    if (ckpt_interval > 0 && ckpt_interval % 64 != 0) return KDA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(ckpt) & 15u) != 0) return KDA_ERR_INVALID_ARG;
+    return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv, dtype, o,
+                        state_out, workspace, workspace_bytes, stream, ckpt_interval,
+                        ckpt_interval > 0 ? ckpt : nullptr, ckpt_capacity, flags);
 }
 
 int64_t kda_prefill_checkpoint_count(const int32_t *cu_seqlens_host, int B, int64_t T, int N,
@@ -173,11 +197,11 @@ kda_status kda_chunk_prefill_checkpointed(const void *q, const void *k, const vo
                                           void *stream) {
     if (interval <= 0 || ckpt_capacity < 0 || (ckpt_capacity > 0 && !ckpt))
         return KDA_ERR_INVALID_ARG;
-    if (interval % 64 != 0 || dtype != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+    if (interval % 64 != 0 || dtype != KDA_BF16 || dk != 128) return KDA_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(ckpt) & 15u) != 0) return KDA_ERR_INVALID_ARG;
     return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv, dtype, o,
                         state_out, workspace, workspace_bytes, stream, interval, ckpt,
-                        ckpt_capacity);
+                        ckpt_capacity, 0u);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *g,

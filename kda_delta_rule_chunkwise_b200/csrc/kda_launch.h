@@ -3,6 +3,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include "kda.h"
 #include <stddef.h>
 #include <stdint.h>
 
@@ -25,6 +27,7 @@ struct PrefillArgs {
     int64_t ckpt_interval = 0;
     float *ckpt = nullptr;
     int64_t ckpt_capacity = 0;
+    uint32_t flags = 0;          // KDA_PREP_* input preprocessing (kda.h)
 };
 
 // Optional per-kernel event recording (see kda_profile_enable).  Launchers

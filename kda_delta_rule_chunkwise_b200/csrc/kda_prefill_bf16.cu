@@ -292,10 +292,13 @@ __device__ __forceinline__ float4 rcp4(float4 a) {
     return make_float4(rcpa(a.x), rcpa(a.y), rcpa(a.z), rcpa(a.w));
 }
 
+// PREP: the input-preprocessing variant (flags at run time); the plain variant
+// compiles without any of it.
+template <bool PREP>
 __global__ void __launch_bounds__(256, 2)
 intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ g, const __nv_bfloat16 *__restrict__ beta,
-                   const int32_t *__restrict__ cu, int64_t T, int N, int H,
+                   const int32_t *__restrict__ cu, int64_t T, int N, int H, uint32_t flags,
                    uint8_t *__restrict__ ws, uint32_t *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -404,9 +407,37 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     const int c = tid & 127, half = tid >> 7;
     float p[32];   // clamped log-decay of rows 32*half + i, then its prefix sums
 #pragma unroll
-    for (int i = 0; i < 32; ++i) p[i] = fmaxf(__bfloat162float(gst[(half * 32 + i) * D + c]), -5.f);
+    for (int i = 0; i < 32; ++i) {
+        const float x = __bfloat162float(gst[(half * 32 + i) * D + c]);
+        // gate from a logit: g = -5 sigmoid(x), inside (-5, 0) by construction.  Rows
+        // past the chunk's end decay by nothing (their staged x is 0, which the
+        // gate would map to -2.5): the block factors and EL then stay <= 1.
+        if (PREP) {
+            const float gv = (flags & KDA_PREP_GATE_LOGIT) ? -5.f / (1.f + __expf(-x)) : fmaxf(x, -5.f);
+            p[i] = (half * 32 + i < L) ? gv : 0.f;
+        } else {
+            p[i] = fmaxf(x, -5.f);   // rows past the end are staged as zero
+        }
+    }
     if (tid < 64) bs[tid] = bnext;
     __syncthreads();
+    // the g staging is free now: it holds 1 / |q_r| and 1 / |k_r| when q, k are to be
+    // normalised here (two threads per row; a zero row stays zero)
+    float *inv_norm = reinterpret_cast<float *>(sm + A_GST);   // [2][64]: q rows, then k rows
+    if (PREP && (flags & KDA_PREP_L2NORM_QK)) {
+        const int which = tid >> 7, row = (tid >> 1) & 63, hf = tid & 1;
+        const uint8_t *src = sm + (which ? A_KST : A_QST) + row * 256;
+        float ss = 0.f;
+#pragma unroll
+        for (int pc = 8 * hf; pc < 8 * hf + 8; ++pc) {
+            float x[8];
+            unpack8(*reinterpret_cast<const uint4 *>(src + ((pc ^ ((row & 3) << 2)) << 4)), x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (hf == 0) inv_norm[which * 64 + row] = ss > 0.f ? rsqrtf(ss) : 0.f;
+    }
 
     // ---- A0: chunk-local cumsum (fp32) and E1 = exp(G - R_a), per channel c and half
     // G_r - R_a(r) = p_i for the first 16 rows of a half and p_i - p_15 for the
@@ -454,6 +485,14 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         PF[128 + c] = PF[c] * Fb[256 + c];
     }
     // q, k of the operand rounds into registers; the staging area is free after the barrier
+    float qn[2] = {1.f, 1.f}, kn[2] = {1.f, 1.f};   // row scales (normalisation)
+    if (PREP && (flags & KDA_PREP_L2NORM_QK)) {
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            qn[it] = inv_norm[a1_row(it)];
+            kn[it] = inv_norm[64 + a1_row(it)];
+        }
+    }
     uint2 qv[4][2], kv[4][2];
 #pragma unroll
     for (int rd = 0; rd < 4; ++rd)
@@ -490,7 +529,11 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 uint8_t *bt = sm + buf + A_BT + co, *at = sm + buf + A_AT + co;
                 float *e1p = E1 + e1_at(r, c0);
                 const float4 e = ld4(e1p);
-                const float4 qf = bf4(qv[rd][it]), kf = bf4(kv[rd][it]);
+                float4 qf = bf4(qv[rd][it]), kf = bf4(kv[rd][it]);
+                if (PREP && (flags & KDA_PREP_L2NORM_QK)) {
+                    qf = make_float4(qf.x * qn[it], qf.y * qn[it], qf.z * qn[it], qf.w * qn[it]);
+                    kf = make_float4(kf.x * kn[it], kf.y * kn[it], kf.z * kn[it], kf.w * kn[it]);
+                }
                 const float4 qe = mul4(qf, e), ke = mul4(kf, e);
                 *reinterpret_cast<float4 *>(bt + ((32 * a + i) >> 3) * 1024) = tf4(qe);
                 *reinterpret_cast<float4 *>(bt + ((32 * a + 16 + i) >> 3) * 1024) = tf4(ke);
@@ -1290,8 +1333,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
     const int64_t max_chunks =
         a.cu_seqlens ? (rows + tc::C - 1) / tc::C + a.N : (int64_t)a.N * ((a.T + tc::C - 1) / tc::C);
     if (max_chunks > 0) {
-        e = cudaFuncSetAttribute(tc::intra_chunk_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::A_SMEM);
+        auto kern = a.flags ? tc::intra_chunk_kernel<true> : tc::intra_chunk_kernel<false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::A_SMEM);
         if (e != cudaSuccess) return e;
         // persistent: two CTAs per SM walk the (chunk, head) items
         int dev = 0, sms = 148;
@@ -1300,9 +1343,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
         const int64_t items = max_chunks * a.H;
         if (items > INT32_MAX - 65536) return cudaErrorInvalidValue;
         const int64_t ctas = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
-        tc::intra_chunk_kernel<<<(unsigned)ctas, 256, tc::A_SMEM, st>>>(
+        kern<<<(unsigned)ctas, 256, tc::A_SMEM, st>>>(
             (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
-            (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, ws, a.err);
+            (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, a.flags, ws, a.err);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -145,6 +145,37 @@ def prefill_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16"
                          dict(seed=seed, decay=decay, state=state))
 
 
+def prefill_raw_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16",
+                       seed: int = 0, state: str = "normal", lengths=None,
+                       device="cpu") -> PrefillInputs:
+    """Like prefill_inputs, but q and k are raw projections (N(0, 1) scaled by a random
+    per-(token, head) norm in [0.5, 4], not normalised) and g holds gate logits
+    ~ N(0, 1), for a prefill that normalises q, k and forms the gate itself."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    tdt = DTYPES[dtype]
+    scale = lambda: 0.5 + 3.5 * torch.rand((B, T, H, 1), generator=gen, device=device)
+    q = _normal((B, T, H, dk), gen, device) * scale()
+    k = _normal((B, T, H, dk), gen, device) * scale()
+    v = _normal((B, T, H, dv), gen, device)
+    g = _normal((B, T, H, dk), gen, device)
+    beta = torch.sigmoid(_normal((B, T, H), gen, device))
+    if lengths is not None:
+        if B != 1 or sum(lengths) != T:
+            raise ValueError("packed inputs need B == 1 and T == sum(lengths)")
+        cu = torch.zeros(len(lengths) + 1, dtype=torch.int64)
+        cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0)
+        cu_seqlens = cu.to(torch.int32).to(device)
+        N = len(lengths)
+    else:
+        cu_seqlens = None
+        N = B
+    s0 = _normal((N, H, dk, dv), gen, device, std=0.1) if state == "normal" else None
+    cast = lambda x: x.to(tdt).contiguous()
+    return PrefillInputs(cast(q), cast(k), cast(v), cast(g), cast(beta), s0, cu_seqlens, dtype,
+                         dict(seed=seed, decay="logits", state=state))
+
+
 def varlen_lengths(n_seqs: int, lo: int, hi: int, seed: int = 0) -> list:
     """Integer-uniform sequence lengths in [lo, hi], inclusive, seeded (CPU)."""
     gen = torch.Generator(device="cpu")

@@ -140,6 +140,30 @@ def recurrence(q, k, v, g, beta, state_in=None, cu_seqlens=None,
     return o, s_out
 
 
+GATE_LOGIT = 1     # g holds logits x; the log-decay is -5 sigmoid(x)
+L2NORM_QK = 2      # q and k are scaled to unit L2 norm over dk per (token, head)
+
+
+def preprocess(q, k, g, flags: int):
+    """The input preprocessing a fused prefill applies, in fp64, before the recurrence.
+
+    GATE_LOGIT: g <- -5 / (1 + exp(-x)), the lower bound -5 on the log-decay of
+    neurohive.io "Kimi K3 ... overview", section "Sequence length: hybrid KDA and
+    Gated MLA attention", written as a parametrisation (the form the synthetic
+    inputs use).  L2NORM_QK: x <- x / ||x||_2 over the last axis; a zero vector
+    stays zero.  Returns fp64 (q, k, g).
+    """
+    q, k, g = _f64(q), _f64(k), _f64(g)
+    if flags & GATE_LOGIT:
+        g = -5.0 / (1.0 + np.exp(-g))
+    if flags & L2NORM_QK:
+        def unit(x):
+            n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+            return np.divide(x, n, out=np.zeros_like(x), where=n > 0)
+        q, k = unit(q), unit(k)
+    return q, k, g
+
+
 def decode_step(q, k, v, g, beta, state, n_threads: int | None = None, lib=None):
     """One decode step: the same recurrence with a single token per sequence.
 

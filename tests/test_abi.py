@@ -126,7 +126,7 @@ def test_checkpoint_count_dense_and_packed(lib):
 
 
 def _cargs(**kw):
-    base = _args(interval=128, ckpt=64, ckpt_capacity=4, dtype=binding.KDA_BF16)
+    base = _args(interval=128, ckpt=64, ckpt_capacity=4, dtype=binding.KDA_BF16, dk=128, dv=128)
     base.update(kw)
     return base
 
@@ -138,6 +138,32 @@ def _cargs(**kw):
     (dict(interval=100), "KDA_ERR_UNSUPPORTED"), (dict(dtype=binding.KDA_F32), "KDA_ERR_UNSUPPORTED")])
 def test_checkpointed_prefill_rejects(lib, bad, code):
     assert binding.raw_prefill_checkpointed(_cargs(**bad)) == getattr(binding, code)
+
+
+def _xargs(**kw):
+    base = dict(_args(dtype=binding.KDA_BF16), flags=0, ckpt_interval=0, ckpt=None,
+                ckpt_capacity=0)
+    base.update(kw)
+    return base
+
+
+def raw_ex(a):
+    return int(binding.load().kda_chunk_prefill_ex(
+        a.get("q"), a.get("k"), a.get("v"), a.get("g"), a.get("beta"), a.get("state_in"),
+        a.get("cu_seqlens"), a["B"], a["T"], a["N"], a["H"], a["dk"], a["dv"], a["dtype"],
+        a["flags"], a.get("o"), a.get("state_out"), a["ckpt_interval"], a.get("ckpt"),
+        a["ckpt_capacity"], a.get("workspace"), a.get("workspace_bytes", 0), a.get("stream")))
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(flags=4), "KDA_ERR_INVALID_ARG"), (dict(ckpt_interval=-64), "KDA_ERR_INVALID_ARG"),
+    (dict(ckpt_capacity=2), "KDA_ERR_INVALID_ARG"),                       # capacity without array
+    (dict(flags=1, dtype=binding.KDA_F32), "KDA_ERR_UNSUPPORTED"),
+    (dict(ckpt_interval=100, ckpt=64, ckpt_capacity=1), "KDA_ERR_UNSUPPORTED"),
+    (dict(flags=3), "KDA_ERR_UNSUPPORTED"),      # preprocessing needs the d = 128 bf16 path
+    (dict(flags=3, dk=128, dv=128), "KDA_ERR_INVALID_ARG")])   # no workspace given
+def test_prefill_ex_rejects(lib, bad, code):
+    assert raw_ex(_xargs(**bad)) == getattr(binding, code)
 
 
 def _iargs(**kw):

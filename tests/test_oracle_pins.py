@@ -228,3 +228,43 @@ def test_thread_count_does_not_change_bits():
     r8 = oracle.recurrence(q, k, v, g, b, s0, n_threads=8)
     np.testing.assert_array_equal(r1[0], r8[0])
     np.testing.assert_array_equal(r1[1], r8[1])
+
+
+# ---------------------------------------------------------------- input preprocessing
+
+def test_preprocess_gate_is_minus_five_sigmoid():
+    x = np.array([[-40.0, -3.0, 0.0, 3.0, 40.0]])
+    _, _, g = oracle.preprocess(np.ones((1, 2)), np.ones((1, 2)), x, oracle.GATE_LOGIT)
+    assert g[0, 2] == -2.5                                   # sigmoid(0) = 1/2
+    assert np.all(g <= 0) and np.all(g >= -5)                 # inside the bound
+    assert np.all(np.diff(g[0]) < 0)                          # more decay for larger logits
+    np.testing.assert_allclose(g + g[:, ::-1], -5.0, rtol=0, atol=1e-15)   # s(x) + s(-x) = 1
+    np.testing.assert_allclose(g[0, 3], -5.0 / (1.0 + np.exp(-3.0)), rtol=1e-15)
+
+
+def test_preprocess_l2norm_gives_unit_rows_and_keeps_zero_rows():
+    rng = np.random.default_rng(0)
+    q = rng.normal(size=(4, 3, 128)) * 7.0
+    k = rng.normal(size=(4, 3, 128))
+    k[1, 2] = 0.0
+    qn, kn, g = oracle.preprocess(q, k, np.zeros((4, 3, 128)), oracle.L2NORM_QK)
+    np.testing.assert_allclose(np.linalg.norm(qn, axis=-1), 1.0, rtol=1e-14)
+    assert not kn[1, 2].any()
+    np.testing.assert_allclose(qn * np.linalg.norm(q, axis=-1, keepdims=True), q, rtol=1e-13)
+    assert not g.any()                                        # gate untouched without the flag
+
+
+def test_preprocess_then_recurrence_equals_recurrence_on_preprocessed_inputs():
+    """Scale invariance: scaling q by c > 0 changes nothing once q is normalised."""
+    rng = np.random.default_rng(1)
+    T, H, d = 37, 2, 8
+    q, k, v = (rng.normal(size=(1, T, H, d)) for _ in range(3))
+    x = rng.normal(size=(1, T, H, d))
+    b = 1 / (1 + np.exp(-rng.normal(size=(1, T, H))))
+    flags = oracle.GATE_LOGIT | oracle.L2NORM_QK
+    out1 = oracle.recurrence(*oracle.preprocess(q, k, x, flags)[:2], v,
+                             oracle.preprocess(q, k, x, flags)[2], b)
+    out2 = oracle.recurrence(*oracle.preprocess(3.0 * q, 0.5 * k, x, flags)[:2], v,
+                             oracle.preprocess(3.0 * q, 0.5 * k, x, flags)[2], b)
+    np.testing.assert_allclose(out1[0], out2[0], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(out1[1], out2[1], rtol=1e-12, atol=1e-13)

@@ -174,3 +174,9 @@ def test_bf16_prefill_is_deterministic():
     torch.cuda.synchronize()
     rows = torch.cat([torch.arange(0, 300), torch.arange(300, 1000), torch.arange(1000, 1065)])
     assert torch.equal(o1[0, rows], o2[0, rows]) and torch.equal(s1, s2)
+
+
+def test_bf16_d64_prefill_uses_the_simt_kernel():
+    """bf16 inputs at d = 64 (no tensor-core path at that size) through the fp32 SIMT kernel."""
+    inp = kin.prefill_inputs(2, 333, 3, 64, 64, "bf16", seed=34, state="normal")
+    check(inp, TOL_BF16, what="bf16 d64")

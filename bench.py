@@ -48,9 +48,9 @@ FLOPS_PER_TOKEN_HEAD = 139264                                 # algorithmic MMA 
 # launch from one ncu capture (profiles/), valid only for the kernel source it was taken
 # on: the sha256 prefix of that .cu file.  A changed source reports null.
 NCU_TRAFFIC = {
-    "intra_chunk_kernel": ("kda_prefill_bf16.cu", "7d9b9c213bb0dabc", (202233344 + 218482944) / 4096),
-    "state_pass_kernel": ("kda_prefill_bf16.cu", "7d9b9c213bb0dabc", (339801600 + 110648832) / 4096),
-    "decode_kernel": ("kda_decode.cu", "c088165a18adb1b1", 545289984 + 483119872),
+    "intra_chunk_kernel": ("kda_prefill_bf16.cu", "1698401d6e201f53", (202423040 + 216636672) / 4096),
+    "state_pass_kernel": ("kda_prefill_bf16.cu", "1698401d6e201f53", (339787264 + 110925824) / 4096),
+    "decode_kernel": ("kda_decode.cu", "4f1c8c21d6ac8934", 545290752 + 482616576),
 }
 
 

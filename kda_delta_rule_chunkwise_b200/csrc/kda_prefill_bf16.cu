@@ -723,8 +723,12 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 for (int u = 0; u < 4; ++u) zv[u] = Yb[(4 * t4 + u) * 32 + j];
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
-                    const float4 av = ld4(AK + (32 + i0 + 8 * qq) * 64 + 32 + 4 * t4);
-                    acc[qq] = fmaf(av.x, zv[0], fmaf(av.y, zv[1], fmaf(av.z, zv[2], fmaf(av.w, zv[3], acc[qq]))));
+                    // X22 is lower triangular: row i0 + 8 qq has no terms past column
+                    // i0 + 8 qq (a warp-uniform bound, so whole blocks are skipped)
+                    if (t4 <= (i0 >> 2) + 2 * qq) {
+                        const float4 av = ld4(AK + (32 + i0 + 8 * qq) * 64 + 32 + 4 * t4);
+                        acc[qq] = fmaf(av.x, zv[0], fmaf(av.y, zv[1], fmaf(av.z, zv[2], fmaf(av.w, zv[3], acc[qq]))));
+                    }
                 }
             }
 #pragma unroll
@@ -1249,8 +1253,15 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         tmem_ld16(tS + 16 * p, *reinterpret_cast<float(*)[16]>(xa + 16 * p));
                     tmem_wait_ld();
                 }
+                if (j + 1 == nch) break;
+                const float gam = gamma_of(j + 1, ok);
+                if (ok) put_state(xa, gam);
+                const bool ok2 = issue_chunk(j + 1, ok);
+                ok = ok && ok2;
                 // intermediate state: S after (j + 1) C tokens, when that is a multiple of
-                // the interval strictly inside the sequence
+                // the interval strictly inside the sequence.  Written here, after the next
+                // chunk's products are issued, so the stores overlap the wait for the next
+                // state update instead of delaying it (xa still holds that state).
                 if (ckpt_interval > 0 && ok) {
                     const int64_t done = (int64_t)(j + 1) * C;
                     if (done % ckpt_interval == 0 && done < rb - ra) {
@@ -1266,11 +1277,6 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                         }
                     }
                 }
-                if (j + 1 == nch) break;
-                const float gam = gamma_of(j + 1, ok);
-                if (ok) put_state(xa, gam);
-                const bool ok2 = issue_chunk(j + 1, ok);
-                ok = ok && ok2;
             }
             if (ok && state_out && !*abort_flag) {
 #pragma unroll

@@ -220,6 +220,28 @@ KDA_API kda_status kda_decode_step_indexed(const void *q, const void *k, const v
                                    kda_dtype dtype, void *o, void *stream);
 
 /*
+ * Backward of the recurrence (training): given do = dL/do [B, T, H, dv] fp32
+ * and dL/dS_final (dstate_out [N, H, dk, dv] fp32, or NULL for zero), writes
+ * dq, dk, dg [B, T, H, dk], dv [B, T, H, dv], dbeta [B, T, H] (all fp32, for
+ * every token that belongs to a sequence) and dL/dS_0 (dstate_in, or NULL).
+ * The inputs are those of the forward call (q, k, v, g, beta in `dtype`,
+ * state_in fp32 or NULL, the same cu_seqlens convention).  g's clamp at -5
+ * passes no gradient below the bound.  The pages give no formulas for the
+ * backward; it is the exact derivative of the recurrence (one CTA per
+ * (sequence, head), fp32, recomputing states from stored chunk starts).
+ *  workspace  at least kda_backward_workspace_bytes() bytes, 16-byte aligned
+ * Supported sizes as for the prefill (dk == dv in {64, 128}).
+ */
+KDA_API size_t kda_backward_workspace_bytes(int64_t rows, int N, int H, int dk, int dv);
+KDA_API kda_status kda_backward(const void *q, const void *k, const void *v, const void *g,
+                                const void *beta, const float *state_in,
+                                const int32_t *cu_seqlens, int B, int64_t T, int N, int H,
+                                int dk, int dv, kda_dtype dtype, const float *dout,
+                                const float *dstate_out, float *dq, float *dk_out, float *dv_out,
+                                float *dg, float *dbeta, float *dstate_in, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.
  * Returns KDA_ERR_INVALID_ARG if a kernel since the last call skipped work
  * because of an out-of-range index read on the device (kda_decode_step_indexed

@@ -31,6 +31,8 @@ EXPORTED = (
     "kda_prefill_checkpoint_count",
     "kda_decode_step",
     "kda_decode_step_indexed",
+    "kda_backward_workspace_bytes",
+    "kda_backward",
     "kda_check_device_error",
     "kda_selftest_bounded_wait",
     "kda_profile_enable",
@@ -74,6 +76,11 @@ def load(path: str = LIB_PATH):
     lib.kda_chunk_prefill_ex.restype = i32
     lib.kda_prefill_checkpoint_count.argtypes = [vp, i32, i64, i32, i64]
     lib.kda_prefill_checkpoint_count.restype = i64
+    lib.kda_backward_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+    lib.kda_backward_workspace_bytes.restype = sz
+    lib.kda_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32,
+                                 vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.kda_backward.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step_indexed.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
@@ -236,6 +243,32 @@ def kda_chunk_prefill_ex(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, fl
         _ptr(workspace) if need else None, ws_bytes if need else 0, _stream(stream))
     _check(code, "kda_chunk_prefill_ex")
     return o, state_out, ckpt
+
+
+def kda_backward(q, k, v, g, beta, state_in, cu_seqlens, dout, dstate_out=None, *,
+                 want_dstate_in=True, workspace=None, stream=None):
+    """Gradients of the recurrence: returns (dq, dk, dv, dg, dbeta, dstate_in), all fp32
+    (dstate_in None unless want_dstate_in).  Inputs as for kda_chunk_prefill; dout like o."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("state_in", state_in),
+                    ("cu_seqlens", cu_seqlens), ("dout", dout), ("dstate_out", dstate_out)):
+        _contig(name, t)
+    f32 = lambda shape: torch.zeros(shape, dtype=torch.float32, device=q.device)
+    dq, dk_, dg = f32(q.shape), f32(k.shape), f32(g.shape)
+    dv_, db = f32(v.shape), f32(beta.shape)
+    ds0 = f32((N, H, dk, dv)) if want_dstate_in else None
+    need = int(load().kda_backward_workspace_bytes(B * T, N, H, dk, dv))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    code = load().kda_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), B, T, N,
+        H, dk, dv, _DTYPE[q.dtype], _ptr(dout), _ptr(dstate_out), _ptr(dq), _ptr(dk_), _ptr(dv_),
+        _ptr(dg), _ptr(db), _ptr(ds0), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(code, "kda_backward")
+    return dq, dk_, dv_, dg, db, ds0
 
 
 def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):

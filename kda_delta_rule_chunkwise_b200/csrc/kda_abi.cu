@@ -241,6 +241,40 @@ kda_status kda_decode_step_indexed(const void *q, const void *k, const void *v, 
                                         dtype == KDA_BF16, o, slots, P, err, st));
 }
 
+size_t kda_backward_workspace_bytes(int64_t rows, int N, int H, int dk, int dv) {
+    if (rows < 0 || N < 0 || H <= 0 || !supported_dim(dk, dv)) return 0;
+    return kda::backward_workspace_bytes(rows, N, H, dk);
+}
+
+kda_status kda_backward(const void *q, const void *k, const void *v, const void *g,
+                        const void *beta, const float *state_in, const int32_t *cu_seqlens,
+                        int B, int64_t T, int N, int H, int dk, int dv, kda_dtype dtype,
+                        const float *dout, const float *dstate_out, float *dq, float *dk_out,
+                        float *dv_out, float *dg, float *dbeta, float *dstate_in,
+                        void *workspace, size_t workspace_bytes, void *stream) {
+    if (B < 0 || T < 0 || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens ? B != 1 : N != B) return KDA_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * T;
+    if (rows > 0 && (!q || !k || !v || !g || !beta || !dout || !dq || !dk_out || !dv_out || !dg ||
+                     !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)N * H > (int64_t)INT32_MAX / 2) return KDA_ERR_UNSUPPORTED;
+    for (const void *p : {(const void *)state_in, (const void *)dstate_out, (const void *)dstate_in})
+        if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_backward_workspace_bytes(rows, N, H, dk, dv);
+    if (N > 0 && (!workspace || workspace_bytes < need ||
+                  (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0))
+        return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    kda::BackwardArgs a{q, k, v, g, beta, state_in, cu_seqlens, rows, T, N, H, dk, dout,
+                        dstate_out, dq, dk_out, dv_out, dg, dbeta, dstate_in, workspace};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kda::Profiler::begin(st);
+    return from_cuda(kda::launch_backward(a, dtype == KDA_BF16, st));
+}
+
 kda_status kda_check_device_error(void *stream) {
     uint32_t *err = error_word_ptr();
     if (!err) return KDA_ERR_CUDA;

@@ -1,0 +1,307 @@
+// KDA backward: gradients of the recurrence
+//     S_t = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1} + beta_t k_t v_t^T,
+//     o_t = S_t^T q_t,   a_t = exp(max(g_t, -5))
+// with respect to q, k, v, g, beta and the initial state, given dL/do and
+// dL/dS_T (the training use of the delta rule with per-channel retention of
+// neurohive.io "Kimi K3 ... overview", section "Sequence length: hybrid KDA
+// and Gated MLA attention"; the pages give no formulas for it).
+//
+// Per token, with S' = Diag(a) S_{t-1}, p = S'^T k, delta = beta (v - p),
+// S_t = S' + k delta^T, and dS the gradient flowing into S_t:
+//     dS  += q do^T;            dq = S_t do
+//     dd   = dS^T k;            dbeta = dd . (v - p);   dv = beta dd
+//     dp   = -beta dd;          dk = dS delta + S' dp
+//     dS'  = dS + k dp^T;       da = rowsum(dS' * S_{t-1})
+//     dg   = da * a  (0 where g < -5);   dS_{t-1} = Diag(a) dS'
+//
+// One CTA of 256 threads per (sequence, head), fp32 throughout (bf16 inputs
+// are read exactly).  Each thread keeps a (D / RG) x 4 block of S and of dS in
+// registers; column sums over rows and row sums over columns go through
+// shared memory.  Pass 1 runs the recurrence forward and stores the state at
+// every chunk start (C = 64 tokens) in the workspace.  Pass 2 walks the chunks
+// backwards: it reruns the chunk forward from its stored start state, storing
+// the state before each token, then applies the token steps above in reverse.
+// Reads and writes are sequential per (sequence, head); the work is the
+// recurrence's ~12 dk dv flops per token three times over.  This is the
+// straightforward form of the backward, not a tensor-core chunked one.
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+namespace bwd {
+
+constexpr int C = 64;     // tokens per stored chunk state
+constexpr int NT = 256;   // threads per CTA
+
+template <int D>
+struct Lay {
+    static constexpr int CG = D / 4;         // column groups of 4
+    static constexpr int RG = NT / CG;       // row groups
+    static constexpr int RPT = D / RG;       // rows per thread
+    static_assert(D % RG == 0, "rows must split evenly");
+};
+
+// rows [a, b) of sequence n: equal-length batch, or the packed offsets clamped
+// to [0, T] and made non-decreasing (the prefill's rule)
+__device__ __forceinline__ void rows_of(const int32_t *cu, int64_t T, int n, int64_t &a, int64_t &b) {
+    if (!cu) {
+        a = (int64_t)n * T;
+        b = a + T;
+        return;
+    }
+    auto cl = [&](int64_t x) { return x < 0 ? 0 : (x > T ? T : x); };
+    int64_t run = 0;
+    for (int i = 0; i <= n; ++i) run = max(run, cl(cu[i]));
+    a = run;
+    b = max(run, cl(cu[n + 1]));
+}
+
+// index of sequence n's first stored chunk state: chunks of sequences 0..n-1
+__device__ __forceinline__ int64_t chunk_base(const int32_t *cu, int64_t T, int n) {
+    if (!cu) return (int64_t)n * ((T + C - 1) / C);
+    int64_t acc = 0, a, b;
+    for (int i = 0; i < n; ++i) {
+        rows_of(cu, T, i, a, b);
+        acc += (b - a + C - 1) / C;
+    }
+    return acc;
+}
+
+template <int D, typename Tin>
+__global__ void __launch_bounds__(NT, 1)
+backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                const Tin *__restrict__ g, const Tin *__restrict__ beta, const float *state_in,
+                const int32_t *__restrict__ cu, int64_t T, int N, int H,
+                const float *__restrict__ dout, const float *dstate_out,
+                float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv,
+                float *__restrict__ dg, float *__restrict__ dbeta, float *dstate_in,
+                float *__restrict__ ws_chunks, float *__restrict__ ws_tokens) {
+    using L = Lay<D>;
+    constexpr int CG = L::CG, RG = L::RG, RPT = L::RPT;
+    const int unit = blockIdx.x;
+    const int n = unit / H, h = unit % H;
+    if (n >= N) return;
+    const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+
+    extern __shared__ float shm[];
+    float *qs = shm, *ks = qs + D, *vs = ks + D, *as = vs + D, *ms = as + D, *dos = ms + D;
+    float *pv = dos + D, *dl = pv + D, *vp = dl + D, *ddv = vp + D, *dpv = ddv + D;
+    float *aks = dpv + D;                // a * k (the column weights of p = (Diag(a) S)^T k)
+    float *red_c = aks + D;              // [RG][D] column partials (sums over a thread's rows)
+    float *red_r = red_c + RG * D;       // [2][CG][D] row partials (sums over a thread's columns)
+    __shared__ float bsh;
+
+    int64_t ra, rb;
+    rows_of(cu, T, n, ra, rb);
+    const int64_t len = rb - ra;
+    const int nch = (int)((len + C - 1) / C);
+    float *chunks = ws_chunks + (size_t)(chunk_base(cu, T, n) * H + (int64_t)h * nch) * D * D;
+    float *toks = ws_tokens + (size_t)unit * C * D * D;
+    const size_t sbase = ((size_t)n * H + h) * D * D;
+
+    // this thread's block: rows rg + RG i, columns 4 cg .. 4 cg + 3
+    auto ld_block = [&](const float *src, float4 (&x)[RPT]) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i)
+            x[i] = src ? reinterpret_cast<const float4 *>(src + (size_t)(rg + RG * i) * D)[cg]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    auto st_block = [&](float *dst, const float4 (&x)[RPT]) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) reinterpret_cast<float4 *>(dst + (size_t)(rg + RG * i) * D)[cg] = x[i];
+    };
+    auto tok_off = [&](int64_t t, int d) { return ((size_t)(ra + t) * H + h) * d; };
+    // token t's k, v, g (-> a and the clamp mask), beta into shared memory
+    auto load_kvgb = [&](int64_t t) {
+        for (int c = tid; c < D; c += NT) {
+            ks[c] = to_f32(k[tok_off(t, D) + c]);
+            vs[c] = to_f32(v[tok_off(t, D) + c]);
+            const float gv = to_f32(g[tok_off(t, D) + c]);
+            as[c] = expf(fmaxf(gv, -5.f));
+            ms[c] = gv >= -5.f ? 1.f : 0.f;
+            aks[c] = as[c] * ks[c];
+        }
+        if (tid == 0) bsh = to_f32(beta[(size_t)(ra + t) * H + h]);
+    };
+    // column sums over rows of x[r][j] * w[r], result into out[j]
+    auto col_sum = [&](const float4 (&x)[RPT], const float *w, float *out) {
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const float wr = w[rg + RG * i];
+            s.x = fmaf(x[i].x, wr, s.x); s.y = fmaf(x[i].y, wr, s.y);
+            s.z = fmaf(x[i].z, wr, s.z); s.w = fmaf(x[i].w, wr, s.w);
+        }
+        reinterpret_cast<float4 *>(red_c + rg * D)[cg] = s;
+        __syncthreads();
+        if (tid < D) {
+            float acc = 0.f;
+#pragma unroll 8
+            for (int r = 0; r < RG; ++r) acc += red_c[r * D + tid];
+            out[tid] = acc;
+        }
+        __syncthreads();
+    };
+    // one forward token step on the block S: S <- Diag(a) S + k delta^T
+    auto fwd_step = [&](float4 (&S)[RPT]) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const float a = as[rg + RG * i];
+            S[i].x *= a; S[i].y *= a; S[i].z *= a; S[i].w *= a;
+        }
+        col_sum(S, ks, pv);                           // p = S'^T k
+        if (tid < D) dl[tid] = bsh * (vs[tid] - pv[tid]);
+        __syncthreads();
+        const float4 d4 = reinterpret_cast<const float4 *>(dl)[cg];
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const float kr = ks[rg + RG * i];
+            S[i].x = fmaf(kr, d4.x, S[i].x); S[i].y = fmaf(kr, d4.y, S[i].y);
+            S[i].z = fmaf(kr, d4.z, S[i].z); S[i].w = fmaf(kr, d4.w, S[i].w);
+        }
+    };
+
+    // ---- pass 1: forward, storing the state at every chunk start
+    float4 S[RPT];
+    ld_block(state_in ? state_in + sbase : nullptr, S);
+    for (int64_t t = 0; t < len; ++t) {
+        if ((t % C) == 0) st_block(chunks + (size_t)(t / C) * D * D, S);
+        __syncthreads();
+        load_kvgb(t);
+        __syncthreads();
+        fwd_step(S);
+    }
+
+    // ---- pass 2: chunks in reverse
+    float4 dS[RPT];
+    ld_block(dstate_out ? dstate_out + sbase : nullptr, dS);
+    for (int ci = nch - 1; ci >= 0; --ci) {
+        const int64_t t0 = (int64_t)ci * C;
+        const int cl = (int)((len - t0) < C ? (len - t0) : C);
+        ld_block(chunks + (size_t)ci * D * D, S);
+        for (int u = 0; u < cl; ++u) {   // rerun the chunk, keeping S before each token
+            st_block(toks + (size_t)u * D * D, S);
+            __syncthreads();
+            load_kvgb(t0 + u);
+            __syncthreads();
+            fwd_step(S);
+        }
+        for (int u = cl - 1; u >= 0; --u) {
+            const int64_t t = t0 + u;
+            __syncthreads();
+            load_kvgb(t);
+            for (int c = tid; c < D; c += NT) {
+                qs[c] = to_f32(q[tok_off(t, D) + c]);
+                dos[c] = dout[tok_off(t, D) + c];
+            }
+            __syncthreads();
+            float4 Sp[RPT];                       // S_{t-1}; S' = Diag(a) S_{t-1} is formed inline
+            ld_block(toks + (size_t)u * D * D, Sp);
+            col_sum(Sp, aks, pv);                 // p = S'^T k
+            if (tid < D) {
+                vp[tid] = vs[tid] - pv[tid];
+                dl[tid] = bsh * vp[tid];          // delta
+            }
+            __syncthreads();
+            const float4 d4 = reinterpret_cast<const float4 *>(dl)[cg];
+            const float4 do4 = reinterpret_cast<const float4 *>(dos)[cg];
+            // dS += q do^T; row partials of dq = S_t do; column partials of dd = dS^T k
+            float4 cs = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = rg + RG * i;
+                const float qr = qs[r], kr = ks[r], a = as[r];
+                dS[i].x = fmaf(qr, do4.x, dS[i].x); dS[i].y = fmaf(qr, do4.y, dS[i].y);
+                dS[i].z = fmaf(qr, do4.z, dS[i].z); dS[i].w = fmaf(qr, do4.w, dS[i].w);
+                const float4 St = make_float4(fmaf(kr, d4.x, a * Sp[i].x), fmaf(kr, d4.y, a * Sp[i].y),
+                                              fmaf(kr, d4.z, a * Sp[i].z), fmaf(kr, d4.w, a * Sp[i].w));
+                red_r[cg * D + r] = St.x * do4.x + St.y * do4.y + St.z * do4.z + St.w * do4.w;
+                cs.x = fmaf(dS[i].x, kr, cs.x); cs.y = fmaf(dS[i].y, kr, cs.y);
+                cs.z = fmaf(dS[i].z, kr, cs.z); cs.w = fmaf(dS[i].w, kr, cs.w);
+            }
+            reinterpret_cast<float4 *>(red_c + rg * D)[cg] = cs;
+            __syncthreads();
+            if (tid < D) {
+                float aq = 0.f, ad = 0.f;
+                for (int x = 0; x < CG; ++x) aq += red_r[x * D + tid];
+#pragma unroll 8
+                for (int x = 0; x < RG; ++x) ad += red_c[x * D + tid];
+                dq[tok_off(t, D) + tid] = aq;
+                ddv[tid] = ad;                                   // dd
+                dv[tok_off(t, D) + tid] = bsh * ad;
+                dpv[tid] = -bsh * ad;                            // dp
+            }
+            __syncthreads();
+            if (tid < 32) {                                      // dbeta = dd . (v - p)
+                float s = 0.f;
+                for (int c = tid; c < D; c += 32) s = fmaf(ddv[c], vp[c], s);
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+                if (tid == 0) dbeta[(size_t)(ra + t) * H + h] = s;
+            }
+            const float4 dp4 = reinterpret_cast<const float4 *>(dpv)[cg];
+            // row partials of dk = dS delta + S' dp and of da = rowsum(dS' * S_{t-1}),
+            // with dS' = dS + k dp^T; then dS <- Diag(a) dS'
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = rg + RG * i;
+                const float kr = ks[r], a = as[r];
+                red_r[cg * D + r] = dS[i].x * d4.x + dS[i].y * d4.y + dS[i].z * d4.z + dS[i].w * d4.w +
+                                    a * (Sp[i].x * dp4.x + Sp[i].y * dp4.y + Sp[i].z * dp4.z +
+                                         Sp[i].w * dp4.w);
+                dS[i].x = fmaf(kr, dp4.x, dS[i].x); dS[i].y = fmaf(kr, dp4.y, dS[i].y);
+                dS[i].z = fmaf(kr, dp4.z, dS[i].z); dS[i].w = fmaf(kr, dp4.w, dS[i].w);
+                red_r[CG * D + cg * D + r] = dS[i].x * Sp[i].x + dS[i].y * Sp[i].y +
+                                             dS[i].z * Sp[i].z + dS[i].w * Sp[i].w;
+                dS[i].x *= a; dS[i].y *= a; dS[i].z *= a; dS[i].w *= a;
+            }
+            __syncthreads();
+            if (tid < D) {
+                float akk = 0.f, aa = 0.f;
+                for (int x = 0; x < CG; ++x) {
+                    akk += red_r[x * D + tid];
+                    aa += red_r[CG * D + x * D + tid];
+                }
+                dk[tok_off(t, D) + tid] = akk;
+                dg[tok_off(t, D) + tid] = aa * as[tid] * ms[tid];
+            }
+        }
+    }
+    __syncthreads();
+    if (dstate_in) st_block(dstate_in + sbase, dS);
+}
+
+}  // namespace bwd
+
+size_t backward_workspace_bytes(int64_t rows, int N, int H, int d) {
+    const int64_t chunk_states = ((rows + bwd::C - 1) / bwd::C + N) * (int64_t)H;
+    const int64_t token_states = (int64_t)N * H * bwd::C;
+    return (size_t)(chunk_states + token_states) * d * d * sizeof(float);
+}
+
+template <int D, typename Tin>
+static cudaError_t launch_bwd_t(const BackwardArgs &a, cudaStream_t st) {
+    using L = bwd::Lay<D>;
+    const size_t smem = (size_t)(12 * D + L::RG * D + 2 * L::CG * D) * sizeof(float);
+    auto kern = bwd::backward_kernel<D, Tin>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t chunk_states = ((a.rows + bwd::C - 1) / bwd::C + a.N) * (int64_t)a.H;
+    float *ws = (float *)a.workspace;
+    kern<<<a.N * a.H, bwd::NT, smem, st>>>(
+        (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, (const Tin *)a.g, (const Tin *)a.beta,
+        a.state_in, a.cu_seqlens, a.T, a.N, a.H, a.dout, a.dstate_out, a.dq, a.dk, a.dv, a.dg,
+        a.dbeta, a.dstate_in, ws, ws + (size_t)chunk_states * D * D);
+    e = cudaGetLastError();
+    Profiler::mark(st);
+    return e;
+}
+
+cudaError_t launch_backward(const BackwardArgs &a, bool bf16, cudaStream_t st) {
+    if (a.N * (int64_t)a.H == 0) return cudaSuccess;
+    if (a.d == 64)
+        return bf16 ? launch_bwd_t<64, __nv_bfloat16>(a, st) : launch_bwd_t<64, float>(a, st);
+    return bf16 ? launch_bwd_t<128, __nv_bfloat16>(a, st) : launch_bwd_t<128, float>(a, st);
+}
+
+}  // namespace kda

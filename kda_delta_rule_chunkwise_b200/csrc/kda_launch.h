@@ -46,4 +46,18 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const voi
                           void *o, const int32_t *slots, int P, uint32_t *err, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t timeout_us, uint32_t *err, cudaStream_t st);
 
+// Backward (kda_backward.cu).  Gradients are fp32; inputs fp32 or bf16.
+struct BackwardArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *state_in;
+    const int32_t *cu_seqlens;
+    int64_t rows, T;
+    int N, H, d;
+    const float *dout, *dstate_out;
+    float *dq, *dk, *dv, *dg, *dbeta, *dstate_in;
+    void *workspace;
+};
+size_t backward_workspace_bytes(int64_t rows, int N, int H, int d);
+cudaError_t launch_backward(const BackwardArgs &a, bool bf16, cudaStream_t st);
+
 }  // namespace kda

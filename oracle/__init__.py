@@ -4,9 +4,12 @@ TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this module; the library's
 product path never does, and this module imports nothing from it.
 
-The arithmetic lives in ``kda_oracle.c`` (plain C, fp64, one token at a
-time).  This wrapper only compiles that file with gcc, converts the caller's
-arrays to contiguous fp64 (an exact conversion from bf16/fp32), and calls it.
+The forward arithmetic lives in ``kda_oracle.c`` (plain C, fp64, one token
+at a time); this wrapper compiles it with gcc, converts the caller's arrays to
+contiguous fp64 (an exact conversion from bf16/fp32), and calls it.  Two
+helpers are written here: ``preprocess`` (the gate-from-logit and q/k
+normalisation a fused prefill applies, fp64 numpy) and ``backward`` (the
+gradients, by PyTorch autograd in fp64 over the token recurrence written out).
 
 Recurrence (the delta rule with per-channel retention described in words in
 neurohive.io "Kimi K3 ... overview", section "Sequence length: hybrid KDA and
@@ -162,6 +165,46 @@ def preprocess(q, k, g, flags: int):
             return np.divide(x, n, out=np.zeros_like(x), where=n > 0)
         q, k = unit(q), unit(k)
     return q, k, g
+
+
+def backward(q, k, v, g, beta, state_in, dout, dstate_out=None, cu_seqlens=None):
+    """Gradients of L = sum(o * dout) + sum(S_final * dstate_out) with respect to
+    q, k, v, g, beta and the initial state, by reverse-mode differentiation
+    (PyTorch autograd on CPU, fp64) of the recurrence written out token by token:
+        a = exp(clamp(g, min=-5)),  S' = Diag(a) S,  p = S'^T k,
+        S = S' + beta k (v - p)^T,  o = S^T q
+    the same recurrence as kda_oracle.c (the clamp passes no gradient below -5).
+    Shapes as in recurrence(); dout like o, dstate_out like the final state (or
+    None).  Returns fp64 numpy arrays (dq, dk, dv, dg, dbeta, dstate_in).
+    """
+    import torch
+    t64 = lambda x: torch.from_numpy(_f64(x))
+    q, k, v, g, beta = (t64(x).requires_grad_(True) for x in (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        spans = [(b, 0, T) for b in range(B)]
+    else:
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        spans = [(0, int(cu[n]), int(cu[n + 1])) for n in range(len(cu) - 1)]
+    N = len(spans)
+    S0 = (t64(state_in) if state_in is not None else torch.zeros((N, H, dk, dv), dtype=torch.float64))
+    S0.requires_grad_(True)
+    dout_t = t64(dout)
+    loss = torch.zeros((), dtype=torch.float64)
+    for n, (b, t0, t1) in enumerate(spans):
+        S = S0[n]
+        for t in range(t0, t1):
+            a = torch.exp(torch.clamp(g[b, t], min=-5.0))                      # [H, dk]
+            Sp = a[:, :, None] * S
+            p = torch.einsum("hcj,hc->hj", Sp, k[b, t])
+            S = Sp + beta[b, t][:, None, None] * k[b, t][:, :, None] * (v[b, t] - p)[:, None, :]
+            o = torch.einsum("hcj,hc->hj", S, q[b, t])
+            loss = loss + (o * dout_t[b, t]).sum()
+        if dstate_out is not None:
+            loss = loss + (S * t64(dstate_out)[n]).sum()
+    loss.backward()
+    return tuple(x.grad.numpy() for x in (q, k, v, g, beta, S0))
 
 
 def decode_step(q, k, v, g, beta, state, n_threads: int | None = None, lib=None):

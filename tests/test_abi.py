@@ -166,6 +166,41 @@ def test_prefill_ex_rejects(lib, bad, code):
     assert raw_ex(_xargs(**bad)) == getattr(binding, code)
 
 
+def test_backward_workspace_bytes(lib):
+    assert lib.kda_backward_workspace_bytes(1000, 1, 2, 128, 128) == \
+        ((1000 + 63) // 64 + 1) * 2 * 128 * 128 * 4 + 1 * 2 * 64 * 128 * 128 * 4
+    assert lib.kda_backward_workspace_bytes(10, 1, 2, 96, 96) == 0
+
+
+def _bargs(**kw):
+    base = dict(q=16, k=32, v=48, g=64, beta=80, state_in=None, cu=None, B=1, T=16, N=1, H=2,
+                dk=64, dv=64, dtype=binding.KDA_F32, do=96, ds=None, dq=112, dkk=128, dvv=144,
+                dg=160, db=176, ds0=None, ws=None, wsb=0)
+    base.update(kw)
+    return base
+
+
+def raw_bwd(a):
+    return int(binding.load().kda_backward(
+        a["q"], a["k"], a["v"], a["g"], a["beta"], a["state_in"], a["cu"], a["B"], a["T"], a["N"],
+        a["H"], a["dk"], a["dv"], a["dtype"], a["do"], a["ds"], a["dq"], a["dkk"], a["dvv"],
+        a["dg"], a["db"], a["ds0"], a["ws"], a["wsb"], None))
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(B=-1), "KDA_ERR_INVALID_ARG"), (dict(N=2), "KDA_ERR_INVALID_ARG"),
+    (dict(do=None), "KDA_ERR_INVALID_ARG"), (dict(dg=None), "KDA_ERR_INVALID_ARG"),
+    (dict(dtype=5), "KDA_ERR_INVALID_ARG"), (dict(state_in=8), "KDA_ERR_INVALID_ARG"),
+    (dict(dk=96, dv=96), "KDA_ERR_UNSUPPORTED"),
+    (dict(), "KDA_ERR_INVALID_ARG")])            # no workspace
+def test_backward_rejects(lib, bad, code):
+    assert raw_bwd(_bargs(**bad)) == getattr(binding, code)
+
+
+def test_backward_zero_sequences_is_a_no_op(lib):
+    assert raw_bwd(_bargs(B=0, N=0)) == binding.KDA_OK
+
+
 def _iargs(**kw):
     base = _dargs(slots=64, P=4)
     base.update(kw)

@@ -1,0 +1,61 @@
+"""GPU parity: kda_backward (through the C ABI) against the fp64 oracle's
+reverse-mode gradients (oracle.backward, pinned by central differences of the
+C recurrence in tests/test_oracle_pins.py).  The kernel works in fp32 from the
+exact input values, so the fp32 bar applies to every gradient."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _util import TOL_F32, rel_err, to_np
+from kda_delta_rule_chunkwise_b200 import binding
+from kda_delta_rule_chunkwise_b200 import inputs as kin
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dq", "dk", "dv", "dg", "dbeta", "dstate_in")
+
+
+def check(inp, seed, with_ds=True, rows=None):
+    gen = torch.Generator().manual_seed(seed)
+    N = inp.N
+    do = torch.randn(inp.v.shape, generator=gen, dtype=torch.float32)
+    ds = torch.randn((N, inp.H, inp.dk, inp.dv), generator=gen) if with_ds else None
+    d = inp.to("cuda")
+    got = binding.kda_backward(d.q, d.k, d.v, d.g, d.beta, d.state_in, d.cu_seqlens, do.cuda(),
+                               None if ds is None else ds.cuda())
+    torch.cuda.synchronize()
+    assert binding.kda_check_device_error() == binding.KDA_OK
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy().astype(np.int64)
+    ref = oracle.backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.state_in, do, ds, cu_seqlens=cu)
+    errs = {}
+    for name, x, y in zip(NAMES, got, ref):
+        gx = to_np(x)
+        if rows is not None and name != "dstate_in":
+            gx, y = gx[:, rows], y[:, rows]
+        errs[name] = rel_err(gx, y)
+    print({k_: f"{v_:.2e}" for k_, v_ in errs.items()})
+    for name, e in errs.items():
+        assert e <= TOL_F32, f"{name}: {e:.3e}"
+
+
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("f32", 128), ("bf16", 128), ("bf16", 64)])
+def test_backward_dense(dtype, d):
+    inp = kin.prefill_inputs(2, 150, 2, d, d, dtype, seed=61, state="normal")
+    check(inp, seed=1)
+
+
+def test_backward_varlen_with_empty_and_ragged_sequences_no_state():
+    inp = kin.prefill_inputs(1, 200, 2, 128, 128, "bf16", seed=62, decay="split",
+                             lengths=[65, 0, 64, 71])
+    check(inp, seed=2, with_ds=False)
+
+
+def test_backward_clamped_decay_passes_no_gradient():
+    inp = kin.prefill_inputs(1, 70, 1, 64, 64, "f32", seed=63, state="normal")
+    inp.g[0, 10:20, 0, :8] = -7.0          # below the bound
+    check(inp, seed=3)
+    d = inp.to("cuda")
+    grads = binding.kda_backward(d.q, d.k, d.v, d.g, d.beta, d.state_in, None,
+                                 torch.ones(inp.v.shape, device="cuda"))
+    assert not grads[3][0, 10:20, 0, :8].any()

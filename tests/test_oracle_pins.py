@@ -268,3 +268,58 @@ def test_preprocess_then_recurrence_equals_recurrence_on_preprocessed_inputs():
                              oracle.preprocess(3.0 * q, 0.5 * k, x, flags)[2], b)
     np.testing.assert_allclose(out1[0], out2[0], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(out1[1], out2[1], rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- backward
+
+def _loss(q, k, v, g, b, s0, do, ds, cu=None):
+    o, s = oracle.recurrence(q, k, v, g, b, state_in=s0, cu_seqlens=cu)
+    return float(np.sum(o * do) + np.sum(s * ds))
+
+
+def test_backward_matches_central_differences_of_the_c_oracle():
+    """Every gradient entry against (L(x+e) - L(x-e)) / 2e, L evaluated by the C
+    recurrence (independent of the autograd graph); includes g below -5."""
+    rng = np.random.default_rng(11)
+    B, T, H, d = 1, 6, 2, 3
+    q, k, v = (rng.normal(size=(B, T, H, d)) for _ in range(3))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    g = -5.0 / (1.0 + np.exp(-rng.normal(size=(B, T, H, d))))
+    g[0, 2, 1, 0] = -6.5                                      # clamped: no gradient
+    b = 1 / (1 + np.exp(-rng.normal(size=(B, T, H))))
+    s0 = rng.normal(size=(B, H, d, d)) * 0.3
+    do = rng.normal(size=(B, T, H, d))
+    ds = rng.normal(size=(B, H, d, d))
+    grads = oracle.backward(q, k, v, g, b, s0, do, ds)
+    eps = 1e-6
+    for arr, gr in zip((q, k, v, g, b, s0), grads):
+        num = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            old = arr[i]
+            arr[i] = old + eps
+            lp = _loss(q, k, v, g, b, s0, do, ds)
+            arr[i] = old - eps
+            lm = _loss(q, k, v, g, b, s0, do, ds)
+            arr[i] = old
+            num[i] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(gr, num, rtol=1e-6, atol=1e-7)
+    assert grads[3][0, 2, 1, 0] == 0.0
+
+
+def test_backward_packed_sequences_are_independent():
+    rng = np.random.default_rng(12)
+    T, H, d = 9, 1, 4
+    q, k, v, g, do = (rng.normal(size=(1, T, H, d)) for _ in range(5))
+    g = -np.abs(g)
+    b = rng.uniform(0.1, 0.9, size=(1, T, H))
+    cu = np.array([0, 4, 4, 9])
+    s0 = rng.normal(size=(3, H, d, d))
+    full = oracle.backward(q, k, v, g, b, s0, do, None, cu_seqlens=cu)
+    part = oracle.backward(q[:, 4:], k[:, 4:], v[:, 4:], g[:, 4:], b[:, 4:], s0[2:], do[:, 4:])
+    for x, y in zip(full[:5], part[:5]):
+        np.testing.assert_allclose(x[:, 4:], y, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(full[5][2], part[5][0], rtol=1e-12, atol=1e-14)
+    # the empty sequence's state passes through: its gradient is dL/dS_final = 0
+    assert not full[5][1].any()

@@ -88,7 +88,11 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     float *pv = dos + D, *dl = pv + D, *vp = dl + D, *ddv = vp + D, *dpv = ddv + D;
     float *aks = dpv + D;                // a * k (the column weights of p = (Diag(a) S)^T k)
     float *red_c = aks + D;              // [RG][D] column partials (sums over a thread's rows)
-    float *red_r = red_c + RG * D;       // [2][CG][D] row partials (sums over a thread's columns)
+    // [2][D][CG + 1] row partials (sums over a thread's columns), rows padded by one
+    // word so that both the writes (one row, consecutive column groups) and the
+    // reads (one row per thread) are free of bank conflicts
+    constexpr int RS = CG + 1;
+    float *red_r = red_c + RG * D;
     __shared__ float bsh;
 
     int64_t ra, rb;
@@ -111,17 +115,41 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
         for (int i = 0; i < RPT; ++i) reinterpret_cast<float4 *>(dst + (size_t)(rg + RG * i) * D)[cg] = x[i];
     };
     auto tok_off = [&](int64_t t, int d) { return ((size_t)(ra + t) * H + h) * d; };
-    // token t's k, v, g (-> a and the clamp mask), beta into shared memory
-    auto load_kvgb = [&](int64_t t) {
-        for (int c = tid; c < D; c += NT) {
-            ks[c] = to_f32(k[tok_off(t, D) + c]);
-            vs[c] = to_f32(v[tok_off(t, D) + c]);
-            const float gv = to_f32(g[tok_off(t, D) + c]);
-            as[c] = expf(fmaxf(gv, -5.f));
-            ms[c] = gv >= -5.f ? 1.f : 0.f;
-            aks[c] = as[c] * ks[c];
+    // Token inputs travel one token ahead: fetch() issues the global loads of a
+    // token into registers (thread c < D holds channel c), stage() moves the
+    // fetched values into shared memory (k, v, a = exp(max(g, -5)), the clamp
+    // mask, a k, beta; q and do when the backward needs them), so each step's
+    // loads land while the previous step computes.
+    struct Tok { float k, v, g, q, dout, b; };
+    auto fetch = [&](int64_t t, bool with_q) {
+        Tok x{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (t < 0 || t >= len) return x;
+        if (tid < D) {
+            x.k = to_f32(k[tok_off(t, D) + tid]);
+            x.v = to_f32(v[tok_off(t, D) + tid]);
+            x.g = to_f32(g[tok_off(t, D) + tid]);
+            if (with_q) {
+                x.q = to_f32(q[tok_off(t, D) + tid]);
+                x.dout = dout[tok_off(t, D) + tid];
+            }
         }
-        if (tid == 0) bsh = to_f32(beta[(size_t)(ra + t) * H + h]);
+        if (tid == 0) x.b = to_f32(beta[(size_t)(ra + t) * H + h]);
+        return x;
+    };
+    auto stage = [&](const Tok &x, bool with_q) {
+        if (tid < D) {
+            ks[tid] = x.k;
+            vs[tid] = x.v;
+            const float a = expf(fmaxf(x.g, -5.f));
+            as[tid] = a;
+            ms[tid] = x.g >= -5.f ? 1.f : 0.f;
+            aks[tid] = a * x.k;
+            if (with_q) {
+                qs[tid] = x.q;
+                dos[tid] = x.dout;
+            }
+        }
+        if (tid == 0) bsh = x.b;
     };
     // column sums over rows of x[r][j] * w[r], result into out[j]
     auto col_sum = [&](const float4 (&x)[RPT], const float *w, float *out) {
@@ -164,10 +192,12 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     // ---- pass 1: forward, storing the state at every chunk start
     float4 S[RPT];
     ld_block(state_in ? state_in + sbase : nullptr, S);
+    Tok nx = fetch(0, false);
     for (int64_t t = 0; t < len; ++t) {
         if ((t % C) == 0) st_block(chunks + (size_t)(t / C) * D * D, S);
         __syncthreads();
-        load_kvgb(t);
+        stage(nx, false);
+        nx = fetch(t + 1, false);
         __syncthreads();
         fwd_step(S);
     }
@@ -179,24 +209,24 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
         const int64_t t0 = (int64_t)ci * C;
         const int cl = (int)((len - t0) < C ? (len - t0) : C);
         ld_block(chunks + (size_t)ci * D * D, S);
+        Tok fx = fetch(t0, false);
         for (int u = 0; u < cl; ++u) {   // rerun the chunk, keeping S before each token
             st_block(toks + (size_t)u * D * D, S);
             __syncthreads();
-            load_kvgb(t0 + u);
+            stage(fx, false);
+            fx = fetch(t0 + u + 1 < t0 + cl ? t0 + u + 1 : -1, false);
             __syncthreads();
             fwd_step(S);
         }
+        Tok bx = fetch(t0 + cl - 1, true);
         for (int u = cl - 1; u >= 0; --u) {
             const int64_t t = t0 + u;
-            __syncthreads();
-            load_kvgb(t);
-            for (int c = tid; c < D; c += NT) {
-                qs[c] = to_f32(q[tok_off(t, D) + c]);
-                dos[c] = dout[tok_off(t, D) + c];
-            }
-            __syncthreads();
             float4 Sp[RPT];                       // S_{t-1}; S' = Diag(a) S_{t-1} is formed inline
             ld_block(toks + (size_t)u * D * D, Sp);
+            __syncthreads();
+            stage(bx, true);
+            bx = fetch(u > 0 ? t - 1 : -1, true);
+            __syncthreads();
             col_sum(Sp, aks, pv);                 // p = S'^T k
             if (tid < D) {
                 vp[tid] = vs[tid] - pv[tid];
@@ -215,7 +245,7 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                 dS[i].z = fmaf(qr, do4.z, dS[i].z); dS[i].w = fmaf(qr, do4.w, dS[i].w);
                 const float4 St = make_float4(fmaf(kr, d4.x, a * Sp[i].x), fmaf(kr, d4.y, a * Sp[i].y),
                                               fmaf(kr, d4.z, a * Sp[i].z), fmaf(kr, d4.w, a * Sp[i].w));
-                red_r[cg * D + r] = St.x * do4.x + St.y * do4.y + St.z * do4.z + St.w * do4.w;
+                red_r[r * RS + cg] = St.x * do4.x + St.y * do4.y + St.z * do4.z + St.w * do4.w;
                 cs.x = fmaf(dS[i].x, kr, cs.x); cs.y = fmaf(dS[i].y, kr, cs.y);
                 cs.z = fmaf(dS[i].z, kr, cs.z); cs.w = fmaf(dS[i].w, kr, cs.w);
             }
@@ -223,7 +253,7 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             __syncthreads();
             if (tid < D) {
                 float aq = 0.f, ad = 0.f;
-                for (int x = 0; x < CG; ++x) aq += red_r[x * D + tid];
+                for (int x = 0; x < CG; ++x) aq += red_r[tid * RS + x];
 #pragma unroll 8
                 for (int x = 0; x < RG; ++x) ad += red_c[x * D + tid];
                 dq[tok_off(t, D) + tid] = aq;
@@ -246,12 +276,12 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             for (int i = 0; i < RPT; ++i) {
                 const int r = rg + RG * i;
                 const float kr = ks[r], a = as[r];
-                red_r[cg * D + r] = dS[i].x * d4.x + dS[i].y * d4.y + dS[i].z * d4.z + dS[i].w * d4.w +
+                red_r[r * RS + cg] = dS[i].x * d4.x + dS[i].y * d4.y + dS[i].z * d4.z + dS[i].w * d4.w +
                                     a * (Sp[i].x * dp4.x + Sp[i].y * dp4.y + Sp[i].z * dp4.z +
                                          Sp[i].w * dp4.w);
                 dS[i].x = fmaf(kr, dp4.x, dS[i].x); dS[i].y = fmaf(kr, dp4.y, dS[i].y);
                 dS[i].z = fmaf(kr, dp4.z, dS[i].z); dS[i].w = fmaf(kr, dp4.w, dS[i].w);
-                red_r[CG * D + cg * D + r] = dS[i].x * Sp[i].x + dS[i].y * Sp[i].y +
+                red_r[RS * D + r * RS + cg] = dS[i].x * Sp[i].x + dS[i].y * Sp[i].y +
                                              dS[i].z * Sp[i].z + dS[i].w * Sp[i].w;
                 dS[i].x *= a; dS[i].y *= a; dS[i].z *= a; dS[i].w *= a;
             }
@@ -259,8 +289,8 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             if (tid < D) {
                 float akk = 0.f, aa = 0.f;
                 for (int x = 0; x < CG; ++x) {
-                    akk += red_r[x * D + tid];
-                    aa += red_r[CG * D + x * D + tid];
+                    akk += red_r[tid * RS + x];
+                    aa += red_r[RS * D + tid * RS + x];
                 }
                 dk[tok_off(t, D) + tid] = akk;
                 dg[tok_off(t, D) + tid] = aa * as[tid] * ms[tid];
@@ -282,7 +312,7 @@ size_t backward_workspace_bytes(int64_t rows, int N, int H, int d) {
 template <int D, typename Tin>
 static cudaError_t launch_bwd_t(const BackwardArgs &a, cudaStream_t st) {
     using L = bwd::Lay<D>;
-    const size_t smem = (size_t)(12 * D + L::RG * D + 2 * L::CG * D) * sizeof(float);
+    const size_t smem = (size_t)(12 * D + L::RG * D + 2 * (L::CG + 1) * D) * sizeof(float);
     auto kern = bwd::backward_kernel<D, Tin>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

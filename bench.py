@@ -276,12 +276,29 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
         hso = torch.empty(s_out.shape, dtype=s_out.dtype, pin_memory=True)
         dq, dk_, dv_, dg, db, ds = (None if x is None else torch.empty_like(x)
                                     for x in (d.q, d.k, d.v, d.g, d.beta, d.state_in))
+        hcu = None if d.cu_seqlens is None else d.cu_seqlens.cpu().pin_memory()
+        dcu = None if d.cu_seqlens is None else torch.empty_like(d.cu_seqlens)
+        hws = None
+        if d.cu_seqlens is None:
+            # one library call on host buffers: segmented copies overlapped with the kernels
+            hws = torch.empty(binding.kda_prefill_host_workspace_bytes(
+                d.B, d.T, d.H, d.dk, d.dv, d.q.dtype, args.host_segment),
+                dtype=torch.uint8, device=dev)
+            e2e_api = "kda_chunk_prefill_host"
+        else:
+            # packed sequences: copies in, kda_chunk_prefill, copies out
+            e2e_api = "copies + kda_chunk_prefill"
 
         def e2e_step():
-            for dst, src in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (ds, hs)):
+            if hws is not None:
+                binding.kda_chunk_prefill_host(hq, hk, hv, hg, hb, hs, o=ho, state_out=hso,
+                                               segment=args.host_segment, workspace=hws)
+                return
+            for dst, src in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (ds, hs),
+                             (dcu, hcu)):
                 if dst is not None:
                     dst.copy_(src, non_blocking=True)
-            binding.kda_chunk_prefill(dq, dk_, dv_, dg, db, ds, None, o=o, state_out=s_out,
+            binding.kda_chunk_prefill(dq, dk_, dv_, dg, db, ds, dcu, o=o, state_out=s_out,
                                       workspace=ws)
             ho.copy_(o, non_blocking=True)
             hso.copy_(s_out, non_blocking=True)
@@ -302,8 +319,9 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
                "h2d_bytes_per_step": in_bytes,
                "d2h_bytes_per_step": o.numel() * o.element_size()
                + s_out.numel() * s_out.element_size(),
-               "steps": args.e2e_steps}
-        del hq, hk, hv, hg, hb, hs, ho, hso, dq, dk_, dv_, dg, db, ds
+               "steps": args.e2e_steps, "api": e2e_api,
+               "segment": (args.host_segment or 4096) if hws is not None else None}
+        del hq, hk, hv, hg, hb, hs, ho, hso, dq, dk_, dv_, dg, db, ds, hws, hcu, dcu
 
     # ---------------- the same step with intermediate states every CKPT_INTERVAL tokens
     ckpt_res = None
@@ -598,6 +616,8 @@ def main():
                     help="prefill workload of a step (default: the headline T=65536 one)")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--host-segment", type=int, default=0,
+                    help="tokens per segment of the host-buffer prefill (0: library default)")
     ap.add_argument("--ref-seconds", type=float, default=15.0,
                     help="target CPU seconds of one oracle sample (reference arm, cpu_baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

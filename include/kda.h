@@ -23,6 +23,7 @@
  * --------------------------------
  *  - All tensor arguments are DEVICE pointers owned by the caller, dense and
  *    row-major in the shapes given; the library never frees or keeps them.
+ *    (kda_chunk_prefill_host alone takes host pointers for its tensors.)
  *  - q, k, g share the shape [rows, H, dk]; v and o are [rows, H, dv];
  *    beta is [rows, H].  Element type is `dtype` for q, k, v, g and beta.
  *  - o is always fp32, and so is the state [N, H, dk, dv]: row c = key
@@ -305,6 +306,44 @@ KDA_API kda_status kda_chunk_prefill_static_scratch(const void *q, const void *k
                                                     int N, int H, int dk, int dv,
                                                     kda_dtype dtype, void *o, float *state_out,
                                                     void *stream);
+
+/*
+ * Prefill from HOST buffers, for a caller whose inputs and outputs live in
+ * host memory: the same recurrence and results as kda_chunk_prefill over B
+ * sequences of T tokens (no cu_seqlens), with the host <-> device copies done
+ * by the library and overlapped with the computation.
+ *
+ * The T axis is cut into segments of `segment` tokens (a positive multiple of
+ * 64; 0 picks 4096).  Segment s's inputs are copied in on one stream while
+ * segment s - 1 is computed on `stream` and segment s - 2's o is copied out on
+ * a third, so PCIe traffic in both directions overlaps and the call runs at
+ * about the rate of the slower copy direction.  Segment s starts from segment
+ * s - 1's final fp32 state, so the result is that of one call over all T
+ * tokens (the recurrence is sequential; segments end on chunk boundaries).
+ *
+ *  q, k, g, v, beta, o   HOST pointers in the layouts of kda_chunk_prefill
+ *                        (o fp32).  Page-locked memory (cudaHostAlloc,
+ *                        cudaHostRegister) gives the overlap; pageable memory
+ *                        is correct but copies synchronously.
+ *  state_in, state_out   HOST fp32 [B, H, dk, dv], or NULL (zero / not written)
+ *  workspace             DEVICE scratch of at least
+ *                        kda_prefill_host_workspace_bytes() bytes, 256-byte
+ *                        aligned: two segments of inputs and outputs, two
+ *                        states and the prefill workspace of one segment.
+ * The call is asynchronous on `stream` like every other: the host buffers
+ * must stay valid, and o / state_out are complete, once `stream` has reached
+ * the point after the call.  Returns KDA_ERR_UNSUPPORTED for sizes
+ * kda_chunk_prefill does not support or a segment that is not a multiple of
+ * 64, KDA_ERR_INVALID_ARG for NULL inputs or a short workspace.
+ */
+KDA_API size_t kda_prefill_host_workspace_bytes(int B, int64_t T, int H, int dk, int dv,
+                                                kda_dtype dtype, int64_t segment);
+KDA_API kda_status kda_chunk_prefill_host(const void *q, const void *k, const void *v,
+                                          const void *g, const void *beta,
+                                          const float *state_in, int B, int64_t T, int H,
+                                          int dk, int dv, kda_dtype dtype, float *o,
+                                          float *state_out, int64_t segment, void *workspace,
+                                          size_t workspace_bytes, void *stream);
 
 /* Static, human-readable name of a status code. */
 KDA_API const char *kda_status_string(kda_status s);

@@ -38,6 +38,8 @@ EXPORTED = (
     "kda_profile_enable",
     "kda_profile_last",
     "kda_chunk_prefill_static_scratch",
+    "kda_prefill_host_workspace_bytes",
+    "kda_chunk_prefill_host",
     "kda_status_string",
 )
 
@@ -97,6 +99,11 @@ def load(path: str = LIB_PATH):
     lib.kda_chunk_prefill_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                      i32, i32, i32, i32, vp, vp, vp]
     lib.kda_chunk_prefill_static_scratch.restype = i32
+    lib.kda_prefill_host_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i64]
+    lib.kda_prefill_host_workspace_bytes.restype = sz
+    lib.kda_chunk_prefill_host.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                           vp, vp, i64, vp, sz, vp]
+    lib.kda_chunk_prefill_host.restype = i32
     lib.kda_status_string.argtypes = [i32]
     lib.kda_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -164,6 +171,48 @@ def kda_chunk_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=Non
         B, T, N, H, dk, dv, _DTYPE[q.dtype], _ptr(o), _ptr(state_out),
         _ptr(workspace) if need else None, ws_bytes if need else 0, _stream(stream))
     _check(code, "kda_chunk_prefill")
+    return o, state_out
+
+
+def kda_prefill_host_workspace_bytes(B: int, T: int, H: int, dk: int, dv: int,
+                                     dtype: torch.dtype, segment: int = 0) -> int:
+    return int(load().kda_prefill_host_workspace_bytes(B, T, H, dk, dv, _DTYPE[dtype], segment))
+
+
+def kda_chunk_prefill_host(q, k, v, g, beta, state_in=None, *, o=None, state_out=None,
+                           segment=0, workspace=None, want_state=True, device=None,
+                           stream=None):
+    """Prefill of B sequences from HOST tensors (pinned for overlap); returns (o, state_out).
+
+    Same shapes as kda_chunk_prefill without cu_seqlens; o and state_out are
+    host fp32 tensors (pinned ones are allocated if not given).  The library
+    copies segments of `segment` tokens in and out while it computes; the
+    outputs are complete once `stream` (default: the current stream of
+    `device`, default cuda:0's) has passed the call.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta),
+                    ("state_in", state_in), ("o", o), ("state_out", state_out)):
+        _contig(name, t)
+        if t is not None and t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else \
+        torch.device(device)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, pin_memory=True)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    need = kda_prefill_host_workspace_bytes(B, T, H, dk, dv, q.dtype, segment)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(device):
+        code = load().kda_chunk_prefill_host(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), B, T, H, dk, dv,
+            _DTYPE[q.dtype], _ptr(o), _ptr(state_out), segment,
+            _ptr(workspace) if need else None, ws_bytes if need else 0, _stream(stream))
+    _check(code, "kda_chunk_prefill_host")
     return o, state_out
 
 
@@ -345,6 +394,15 @@ def raw_prefill_checkpointed(args: dict) -> int:
         args.get("state_in"), args.get("cu_seqlens"), args["B"], args["T"], args["N"],
         args["H"], args["dk"], args["dv"], args["dtype"], args.get("o"), args.get("state_out"),
         args["interval"], args.get("ckpt"), args.get("ckpt_capacity", 0),
+        args.get("workspace"), args.get("workspace_bytes", 0), args.get("stream")))
+
+
+def raw_prefill_host(args: dict) -> int:
+    lib = load()
+    return int(lib.kda_chunk_prefill_host(
+        args.get("q"), args.get("k"), args.get("v"), args.get("g"), args.get("beta"),
+        args.get("state_in"), args["B"], args["T"], args["H"], args["dk"], args["dv"],
+        args["dtype"], args.get("o"), args.get("state_out"), args.get("segment", 0),
         args.get("workspace"), args.get("workspace_bytes", 0), args.get("stream")))
 
 

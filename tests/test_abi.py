@@ -230,3 +230,51 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(RuntimeError, match="libkda.so not found"):
         binding.load(str(tmp_path / "nope.so"))
+
+
+def test_host_prefill_workspace_bytes(lib):
+    al = lambda x: (x + 255) // 256 * 256
+    H, d = 2, 128
+    # T = 1000 < the default segment: one segment of 1024 rows (T rounded up to the chunk)
+    rows = 1024
+    pre = al(lib.kda_chunk_prefill_workspace_bytes(rows, 1, H, d, d, binding.KDA_BF16))
+    ins = 4 * al(rows * H * d * 2) + al(rows * H * 2)
+    want = 2 * ins + 2 * al(rows * H * d * 4) + 2 * al(H * d * d * 4) + pre
+    assert lib.kda_prefill_host_workspace_bytes(1, 1000, H, d, d, binding.KDA_BF16, 0) == want
+    # an explicit segment sizes the buffers, whatever T is
+    rows = 3 * 256
+    pre = al(lib.kda_chunk_prefill_workspace_bytes(rows, 3, H, 64, 64, binding.KDA_F32))
+    ins = 4 * al(rows * H * 64 * 4) + al(rows * H * 4)
+    want = 2 * ins + 2 * al(rows * H * 64 * 4) + 2 * al(3 * H * 64 * 64 * 4) + pre
+    assert lib.kda_prefill_host_workspace_bytes(3, 5000, H, 64, 64, binding.KDA_F32, 256) == want
+    for bad in ((1, 1000, H, d, d, binding.KDA_BF16, 100),    # segment not a multiple of 64
+                (1, 1000, H, 96, 96, binding.KDA_BF16, 0), (1, 1000, H, 128, 64, binding.KDA_F32, 0),
+                (0, 1000, H, d, d, binding.KDA_BF16, 0), (1, 1000, H, d, d, 7, 0)):
+        assert lib.kda_prefill_host_workspace_bytes(*bad) == 0
+
+
+def _hargs(**kw):
+    base = dict(q=16, k=32, v=48, g=64, beta=80, state_in=None, B=1, T=100, H=2, dk=64, dv=64,
+                dtype=binding.KDA_F32, o=96, state_out=None, segment=0, workspace=None,
+                workspace_bytes=0)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(B=-1), "KDA_ERR_INVALID_ARG"), (dict(T=-5), "KDA_ERR_INVALID_ARG"),
+    (dict(H=0), "KDA_ERR_INVALID_ARG"), (dict(dtype=4), "KDA_ERR_INVALID_ARG"),
+    (dict(segment=-64), "KDA_ERR_INVALID_ARG"), (dict(q=None), "KDA_ERR_INVALID_ARG"),
+    (dict(beta=None), "KDA_ERR_INVALID_ARG"), (dict(o=None), "KDA_ERR_INVALID_ARG"),
+    (dict(dk=96, dv=96), "KDA_ERR_UNSUPPORTED"), (dict(dk=128), "KDA_ERR_UNSUPPORTED"),
+    (dict(segment=96), "KDA_ERR_UNSUPPORTED"),
+    (dict(), "KDA_ERR_INVALID_ARG"),                                   # no workspace
+    (dict(workspace=256, workspace_bytes=1024), "KDA_ERR_INVALID_ARG"),    # short workspace
+    (dict(workspace=128, workspace_bytes=1 << 40), "KDA_ERR_INVALID_ARG")])  # misaligned
+def test_host_prefill_rejects(lib, bad, code):
+    assert binding.raw_prefill_host(_hargs(**bad)) == getattr(binding, code)
+
+
+def test_host_prefill_empty_is_a_no_op(lib):
+    assert binding.raw_prefill_host(_hargs(B=0)) == binding.KDA_OK
+    assert binding.raw_prefill_host(_hargs(T=0)) == binding.KDA_OK

@@ -96,9 +96,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
 }
 
 // As mbar_wait, and also gives up as soon as another thread of the CTA has
-// raised the shared abort flag (set here on a timeout), or any CTA has set the
-// device error word, so that one missing arrival ends every waiting role of
-// every CTA within microseconds instead of one time limit per CTA.
+// raised the shared abort flag (set here on a timeout), or any CTA has recorded
+// a timeout in the device error word, so that one missing arrival ends every
+// waiting role of every CTA within microseconds instead of one time limit per
+// CTA.  Other error bits (an out-of-range index) do not stop the work.
 __device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t parity,
                                                     uint32_t *err, volatile uint32_t *abort,
                                                     uint64_t limit_ns = kWaitLimitNs) {
@@ -108,7 +109,7 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t pari
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (gerr && *gerr) {   // some CTA already gave up: do not wait out the limit too
+        if (gerr && (*gerr & ERR_WAIT_TIMEOUT)) {   // some CTA already gave up: do not wait out the limit too
             *abort = 1u;
             return false;
         }

@@ -389,6 +389,37 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
     del d, o, s_out, ws
     torch.cuda.empty_cache()
 
+    # ---------------- backward on the T=8192 workload (dL/do random, dL/dS_T zero)
+    if args.backward:
+        bw = kin.workload_inputs("prefill_h32_t8192_d128", seed=args.seed + 4000 + rank, device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(args.seed + 5000 + rank)
+        dout = torch.randn(bw.v.shape, generator=gen, device=dev, dtype=torch.float32)
+        wsb = torch.empty(binding.load().kda_backward_workspace_bytes(bw.B * bw.T, bw.N, bw.H, 128, 128),
+                          dtype=torch.uint8, device=dev)
+        bstep = lambda: binding.kda_backward(bw.q, bw.k, bw.v, bw.g, bw.beta, bw.state_in, None, dout,
+                                             workspace=wsb)
+        bstep()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        st = torch.cuda.current_stream()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nb = 2
+        ev0.record(st)
+        for _ in range(nb):
+            bstep()
+        ev1.record(st)
+        torch.cuda.synchronize()
+        b_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        extra["backward"] = {"workload": "prefill_h32_t8192_d128", "steps": nb,
+                             "ms_per_step": round(b_ms / nb, 3),
+                             "value": aggregate_throughput(bw.B * bw.T, world, nb, b_ms),
+                             "unit": "tokens/s",
+                             "kernel": "backward_kernel (fp32, one CTA per (sequence, head, value-column slice)) + backward_reduce_kernel"}
+        del bw, dout, wsb
+        torch.cuda.empty_cache()
+
     # ---------------- decode workload
     decode = None
     if args.decode_steps <= 0:
@@ -467,37 +498,6 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
     }
     del dec, pool, slots, od
     torch.cuda.empty_cache()
-
-    # ---------------- backward on the T=8192 workload (dL/do random, dL/dS_T zero)
-    if args.backward:
-        bw = kin.workload_inputs("prefill_h32_t8192_d128", seed=args.seed + 4000 + rank, device=dev)
-        gen = torch.Generator(device=dev)
-        gen.manual_seed(args.seed + 5000 + rank)
-        dout = torch.randn(bw.v.shape, generator=gen, device=dev, dtype=torch.float32)
-        wsb = torch.empty(binding.load().kda_backward_workspace_bytes(bw.B * bw.T, bw.N, bw.H, 128, 128),
-                          dtype=torch.uint8, device=dev)
-        bstep = lambda: binding.kda_backward(bw.q, bw.k, bw.v, bw.g, bw.beta, bw.state_in, None, dout,
-                                             workspace=wsb)
-        bstep()
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        st = torch.cuda.current_stream()
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        nb = 2
-        ev0.record(st)
-        for _ in range(nb):
-            bstep()
-        ev1.record(st)
-        torch.cuda.synchronize()
-        b_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-        extra["backward"] = {"workload": "prefill_h32_t8192_d128", "steps": nb,
-                             "ms_per_step": round(b_ms / nb, 3),
-                             "value": aggregate_throughput(bw.B * bw.T, world, nb, b_ms),
-                             "unit": "tokens/s",
-                             "kernel": "backward_kernel (fp32, one CTA per (sequence, head))"}
-        del bw, dout, wsb
-        torch.cuda.empty_cache()
 
     return finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path,
                   decode, e2e, clk, extra)

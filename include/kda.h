@@ -228,9 +228,13 @@ KDA_API kda_status kda_decode_step_indexed(const void *q, const void *k, const v
  * The inputs are those of the forward call (q, k, v, g, beta in `dtype`,
  * state_in fp32 or NULL, the same cu_seqlens convention).  g's clamp at -5
  * passes no gradient below the bound.  The pages give no formulas for the
- * backward; it is the exact derivative of the recurrence (one CTA per
- * (sequence, head), fp32, recomputing states from stored chunk starts).
+ * backward; it is the exact derivative of the recurrence (fp32, recomputing
+ * states from stored chunk starts; with few (sequence, head) units the value
+ * columns are split over several CTAs whose partial sums are added in a fixed
+ * order, so results are the same on every run).
  *  workspace  at least kda_backward_workspace_bytes() bytes, 16-byte aligned
+ *             (chunk-start states, per-token states of one chunk per unit, and
+ *             the partial sums when the columns are split)
  * Supported sizes as for the prefill (dk == dv in {64, 128}).
  */
 KDA_API size_t kda_backward_workspace_bytes(int64_t rows, int N, int H, int dk, int dv);

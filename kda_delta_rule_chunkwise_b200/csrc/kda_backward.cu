@@ -14,9 +14,15 @@
 //     dS'  = dS + k dp^T;       da = rowsum(dS' * S_{t-1})
 //     dg   = da * a  (0 where g < -5);   dS_{t-1} = Diag(a) dS'
 //
-// One CTA of 256 threads per (sequence, head), fp32 throughout (bf16 inputs
-// are read exactly).  Each thread keeps a (D / RG) x 4 block of S and of dS in
-// registers; column sums over rows and row sums over columns go through
+// One CTA of 256 threads per (sequence, head, value-column slice), fp32
+// throughout (bf16 inputs are read exactly).  Every step above is local to a
+// set of value columns (the recurrence updates the columns of S
+// independently) except the sums over columns: dq, dk, da and dbeta.  So a
+// few units are cut into NSL column slices, one CTA each, and the slices
+// write those four as partial sums that a second kernel adds up in slice
+// order (deterministic); with many units NSL = 1 and the CTA writes them
+// directly.  Each thread keeps a (D / RG) x 4 block of its slice of S and of
+// dS in registers; column sums over rows and row sums over columns go through
 // shared memory.  Pass 1 runs the recurrence forward and stores the state at
 // every chunk start (C = 64 tokens) in the workspace.  Pass 2 walks the chunks
 // backwards: it reruns the chunk forward from its stored start state, storing
@@ -33,13 +39,20 @@ namespace bwd {
 constexpr int C = 64;     // tokens per stored chunk state
 constexpr int NT = 256;   // threads per CTA
 
-template <int D>
+template <int D, int DVS>
 struct Lay {
-    static constexpr int CG = D / 4;         // column groups of 4
+    static constexpr int CG = DVS / 4;       // column groups of 4
     static constexpr int RG = NT / CG;       // row groups
     static constexpr int RPT = D / RG;       // rows per thread
-    static_assert(D % RG == 0, "rows must split evenly");
+    static constexpr int PW = 3 * D + 4;     // partial sums per (token, head): dq, dk, da, dbeta
+    static_assert(D % RG == 0 && RPT >= 1, "rows must split evenly");
 };
+
+// column slices per (sequence, head): enough CTAs to cover the SMs when there
+// are few units
+__host__ __device__ inline int slices_for(int64_t units) {
+    return units <= 37 ? 4 : (units <= 74 ? 2 : 1);
+}
 
 // rows [a, b) of sequence n: equal-length batch, or the packed offsets clamped
 // to [0, T] and made non-decreasing (the prefill's rule)
@@ -67,32 +80,38 @@ __device__ __forceinline__ int64_t chunk_base(const int32_t *cu, int64_t T, int 
     return acc;
 }
 
-template <int D, typename Tin>
+template <int D, int DVS, typename Tin>
 __global__ void __launch_bounds__(NT, 1)
 backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                 const Tin *__restrict__ g, const Tin *__restrict__ beta, const float *state_in,
-                const int32_t *__restrict__ cu, int64_t T, int N, int H,
+                const int32_t *__restrict__ cu, int64_t T, int N, int H, int64_t rows,
                 const float *__restrict__ dout, const float *dstate_out,
                 float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv,
                 float *__restrict__ dg, float *__restrict__ dbeta, float *dstate_in,
-                float *__restrict__ ws_chunks, float *__restrict__ ws_tokens) {
-    using L = Lay<D>;
-    constexpr int CG = L::CG, RG = L::RG, RPT = L::RPT;
-    const int unit = blockIdx.x;
+                float *__restrict__ ws_chunks, float *__restrict__ ws_tokens,
+                float *__restrict__ part) {
+    using L = Lay<D, DVS>;
+    constexpr int CG = L::CG, RG = L::RG, RPT = L::RPT, PW = L::PW;
+    constexpr int NSL = D / DVS;
+    const int unit = blockIdx.x / NSL, slice = blockIdx.x % NSL;
     const int n = unit / H, h = unit % H;
     if (n >= N) return;
     const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+    const int j0 = slice * DVS;          // first value column of this slice
 
     extern __shared__ float shm[];
-    float *qs = shm, *ks = qs + D, *vs = ks + D, *as = vs + D, *ms = as + D, *dos = ms + D;
-    float *pv = dos + D, *dl = pv + D, *vp = dl + D, *ddv = vp + D, *dpv = ddv + D;
-    float *aks = dpv + D;                // a * k (the column weights of p = (Diag(a) S)^T k)
-    float *red_c = aks + D;              // [RG][D] column partials (sums over a thread's rows)
+    // per key channel (D): q, k, a, clamp mask, a k; per value column of the slice (DVS):
+    // v, do, p, delta, v - p, dd, dp
+    float *qs = shm, *ks = qs + D, *as = ks + D, *ms = as + D;
+    float *aks = ms + D;                 // a * k (the column weights of p = (Diag(a) S)^T k)
+    float *vs = aks + D, *dos = vs + DVS, *pv = dos + DVS, *dl = pv + DVS, *vp = dl + DVS;
+    float *ddv = vp + DVS, *dpv = ddv + DVS;
+    float *red_c = dpv + DVS;            // [RG][DVS] column partials (sums over a thread's rows)
     // [2][D][CG + 1] row partials (sums over a thread's columns), rows padded by one
     // word so that both the writes (one row, consecutive column groups) and the
     // reads (one row per thread) are free of bank conflicts
     constexpr int RS = CG + 1;
-    float *red_r = red_c + RG * D;
+    float *red_r = red_c + RG * DVS;
     __shared__ float bsh;
 
     int64_t ra, rb;
@@ -103,17 +122,20 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     float *toks = ws_tokens + (size_t)unit * C * D * D;
     const size_t sbase = ((size_t)n * H + h) * D * D;
 
-    // this thread's block: rows rg + RG i, columns 4 cg .. 4 cg + 3
+    // this thread's block of a D x D state: rows rg + RG i, columns j0 + 4 cg .. + 3
     auto ld_block = [&](const float *src, float4 (&x)[RPT]) {
 #pragma unroll
         for (int i = 0; i < RPT; ++i)
-            x[i] = src ? reinterpret_cast<const float4 *>(src + (size_t)(rg + RG * i) * D)[cg]
+            x[i] = src ? reinterpret_cast<const float4 *>(src + (size_t)(rg + RG * i) * D + j0)[cg]
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     };
     auto st_block = [&](float *dst, const float4 (&x)[RPT]) {
 #pragma unroll
-        for (int i = 0; i < RPT; ++i) reinterpret_cast<float4 *>(dst + (size_t)(rg + RG * i) * D)[cg] = x[i];
+        for (int i = 0; i < RPT; ++i)
+            reinterpret_cast<float4 *>(dst + (size_t)(rg + RG * i) * D + j0)[cg] = x[i];
     };
+    // partial sums of token t (slices > 1): [NSL][rows][H][PW]
+    auto part_of = [&](int64_t t) { return part + (((size_t)slice * rows + (ra + t)) * H + h) * PW; };
     auto tok_off = [&](int64_t t, int d) { return ((size_t)(ra + t) * H + h) * d; };
     // Token inputs travel one token ahead: fetch() issues the global loads of a
     // token into registers (thread c < D holds channel c), stage() moves the
@@ -126,12 +148,12 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
         if (t < 0 || t >= len) return x;
         if (tid < D) {
             x.k = to_f32(k[tok_off(t, D) + tid]);
-            x.v = to_f32(v[tok_off(t, D) + tid]);
             x.g = to_f32(g[tok_off(t, D) + tid]);
-            if (with_q) {
-                x.q = to_f32(q[tok_off(t, D) + tid]);
-                x.dout = dout[tok_off(t, D) + tid];
-            }
+            if (with_q) x.q = to_f32(q[tok_off(t, D) + tid]);
+        }
+        if (tid < DVS) {
+            x.v = to_f32(v[tok_off(t, D) + j0 + tid]);
+            if (with_q) x.dout = dout[tok_off(t, D) + j0 + tid];
         }
         if (tid == 0) x.b = to_f32(beta[(size_t)(ra + t) * H + h]);
         return x;
@@ -139,15 +161,15 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     auto stage = [&](const Tok &x, bool with_q) {
         if (tid < D) {
             ks[tid] = x.k;
-            vs[tid] = x.v;
             const float a = expf(fmaxf(x.g, -5.f));
             as[tid] = a;
             ms[tid] = x.g >= -5.f ? 1.f : 0.f;
             aks[tid] = a * x.k;
-            if (with_q) {
-                qs[tid] = x.q;
-                dos[tid] = x.dout;
-            }
+            if (with_q) qs[tid] = x.q;
+        }
+        if (tid < DVS) {
+            vs[tid] = x.v;
+            if (with_q) dos[tid] = x.dout;
         }
         if (tid == 0) bsh = x.b;
     };
@@ -160,12 +182,12 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             s.x = fmaf(x[i].x, wr, s.x); s.y = fmaf(x[i].y, wr, s.y);
             s.z = fmaf(x[i].z, wr, s.z); s.w = fmaf(x[i].w, wr, s.w);
         }
-        reinterpret_cast<float4 *>(red_c + rg * D)[cg] = s;
+        reinterpret_cast<float4 *>(red_c + rg * DVS)[cg] = s;
         __syncthreads();
-        if (tid < D) {
+        if (tid < DVS) {
             float acc = 0.f;
 #pragma unroll 8
-            for (int r = 0; r < RG; ++r) acc += red_c[r * D + tid];
+            for (int r = 0; r < RG; ++r) acc += red_c[r * DVS + tid];
             out[tid] = acc;
         }
         __syncthreads();
@@ -178,7 +200,7 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             S[i].x *= a; S[i].y *= a; S[i].z *= a; S[i].w *= a;
         }
         col_sum(S, ks, pv);                           // p = S'^T k
-        if (tid < D) dl[tid] = bsh * (vs[tid] - pv[tid]);
+        if (tid < DVS) dl[tid] = bsh * (vs[tid] - pv[tid]);
         __syncthreads();
         const float4 d4 = reinterpret_cast<const float4 *>(dl)[cg];
 #pragma unroll
@@ -228,7 +250,7 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             bx = fetch(u > 0 ? t - 1 : -1, true);
             __syncthreads();
             col_sum(Sp, aks, pv);                 // p = S'^T k
-            if (tid < D) {
+            if (tid < DVS) {
                 vp[tid] = vs[tid] - pv[tid];
                 dl[tid] = bsh * vp[tid];          // delta
             }
@@ -249,25 +271,32 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                 cs.x = fmaf(dS[i].x, kr, cs.x); cs.y = fmaf(dS[i].y, kr, cs.y);
                 cs.z = fmaf(dS[i].z, kr, cs.z); cs.w = fmaf(dS[i].w, kr, cs.w);
             }
-            reinterpret_cast<float4 *>(red_c + rg * D)[cg] = cs;
+            reinterpret_cast<float4 *>(red_c + rg * DVS)[cg] = cs;
             __syncthreads();
             if (tid < D) {
-                float aq = 0.f, ad = 0.f;
+                float aq = 0.f;
                 for (int x = 0; x < CG; ++x) aq += red_r[tid * RS + x];
+                if (NSL == 1) dq[tok_off(t, D) + tid] = aq;
+                else part_of(t)[tid] = aq;
+            }
+            if (tid < DVS) {
+                float ad = 0.f;
 #pragma unroll 8
-                for (int x = 0; x < RG; ++x) ad += red_c[x * D + tid];
-                dq[tok_off(t, D) + tid] = aq;
+                for (int x = 0; x < RG; ++x) ad += red_c[x * DVS + tid];
                 ddv[tid] = ad;                                   // dd
-                dv[tok_off(t, D) + tid] = bsh * ad;
+                dv[tok_off(t, D) + j0 + tid] = bsh * ad;
                 dpv[tid] = -bsh * ad;                            // dp
             }
             __syncthreads();
             if (tid < 32) {                                      // dbeta = dd . (v - p)
                 float s = 0.f;
-                for (int c = tid; c < D; c += 32) s = fmaf(ddv[c], vp[c], s);
+                for (int c = tid; c < DVS; c += 32) s = fmaf(ddv[c], vp[c], s);
 #pragma unroll
                 for (int m = 16; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
-                if (tid == 0) dbeta[(size_t)(ra + t) * H + h] = s;
+                if (tid == 0) {
+                    if (NSL == 1) dbeta[(size_t)(ra + t) * H + h] = s;
+                    else part_of(t)[3 * D] = s;
+                }
             }
             const float4 dp4 = reinterpret_cast<const float4 *>(dpv)[cg];
             // row partials of dk = dS delta + S' dp and of da = rowsum(dS' * S_{t-1}),
@@ -292,8 +321,13 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                     akk += red_r[tid * RS + x];
                     aa += red_r[RS * D + tid * RS + x];
                 }
-                dk[tok_off(t, D) + tid] = akk;
-                dg[tok_off(t, D) + tid] = aa * as[tid] * ms[tid];
+                if (NSL == 1) {
+                    dk[tok_off(t, D) + tid] = akk;
+                    dg[tok_off(t, D) + tid] = aa * as[tid] * ms[tid];
+                } else {
+                    part_of(t)[D + tid] = akk;
+                    part_of(t)[2 * D + tid] = aa;   // da; the reduction applies a and the mask
+                }
             }
         }
     }
@@ -301,37 +335,99 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     if (dstate_in) st_block(dstate_in + sbase, dS);
 }
 
+// Sums of the column slices' partials, in slice order: dq, dk, dbeta, and
+// dg = da a (0 where g < -5).  CTA (unit, i) takes rows i, i + G, ... of its
+// sequence, one key channel per thread.
+template <int D, int NSL, typename Tin>
+__global__ void __launch_bounds__(D)
+backward_reduce_kernel(const Tin *__restrict__ g, const int32_t *__restrict__ cu, int64_t T, int N,
+                       int H, int64_t rows, int G, const float *__restrict__ part,
+                       float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dg,
+                       float *__restrict__ dbeta) {
+    constexpr int PW = 3 * D + 4;
+    const int unit = blockIdx.x / G, gi = blockIdx.x % G;
+    const int n = unit / H, h = unit % H;
+    if (n >= N) return;
+    int64_t ra, rb;
+    rows_of(cu, T, n, ra, rb);
+    const int c = threadIdx.x;
+    for (int64_t t = ra + gi; t < rb; t += G) {
+        const size_t th = (size_t)t * H + h;
+        float sq = 0.f, sk = 0.f, sa = 0.f, sb = 0.f;
+#pragma unroll
+        for (int s = 0; s < NSL; ++s) {
+            const float *p = part + ((size_t)s * rows * H + th) * PW;
+            sq += p[c];
+            sk += p[D + c];
+            sa += p[2 * D + c];
+            if (c == 0) sb += p[3 * D];
+        }
+        const float gv = to_f32(g[th * D + c]);
+        dq[th * D + c] = sq;
+        dk[th * D + c] = sk;
+        dg[th * D + c] = sa * expf(fmaxf(gv, -5.f)) * (gv >= -5.f ? 1.f : 0.f);
+        if (c == 0) dbeta[th] = sb;
+    }
+}
+
 }  // namespace bwd
 
 size_t backward_workspace_bytes(int64_t rows, int N, int H, int d) {
     const int64_t chunk_states = ((rows + bwd::C - 1) / bwd::C + N) * (int64_t)H;
     const int64_t token_states = (int64_t)N * H * bwd::C;
-    return (size_t)(chunk_states + token_states) * d * d * sizeof(float);
+    const int nsl = bwd::slices_for((int64_t)N * H);
+    const int64_t partials = nsl > 1 ? (int64_t)nsl * rows * H * (3 * d + 4) : 0;
+    return (size_t)(chunk_states + token_states) * d * d * sizeof(float) +
+           (size_t)partials * sizeof(float);
+}
+
+template <int D, int NSL, typename Tin>
+static cudaError_t launch_bwd_t(const BackwardArgs &a, cudaStream_t st) {
+    constexpr int DVS = D / NSL;
+    using L = bwd::Lay<D, DVS>;
+    const size_t smem =
+        (size_t)(5 * D + 7 * DVS + L::RG * DVS + 2 * (L::CG + 1) * D) * sizeof(float);
+    auto kern = bwd::backward_kernel<D, DVS, Tin>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t units = (int64_t)a.N * a.H;
+    const int64_t chunk_states = ((a.rows + bwd::C - 1) / bwd::C + a.N) * (int64_t)a.H;
+    const int64_t token_states = units * bwd::C;
+    float *ws = (float *)a.workspace;
+    float *part = ws + (size_t)(chunk_states + token_states) * D * D;
+    kern<<<(unsigned)(units * NSL), bwd::NT, smem, st>>>(
+        (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, (const Tin *)a.g, (const Tin *)a.beta,
+        a.state_in, a.cu_seqlens, a.T, a.N, a.H, a.rows, a.dout, a.dstate_out, a.dq, a.dk, a.dv,
+        a.dg, a.dbeta, a.dstate_in, ws, ws + (size_t)chunk_states * D * D, part);
+    e = cudaGetLastError();
+    Profiler::mark(st);
+    if constexpr (NSL > 1) {
+        if (e != cudaSuccess) return e;
+        // about eight CTAs per SM for the reduction
+        const int G = (int)(units >= 1184 ? 1 : 1184 / units);
+        bwd::backward_reduce_kernel<D, NSL, Tin><<<(unsigned)(units * G), D, 0, st>>>(
+            (const Tin *)a.g, a.cu_seqlens, a.T, a.N, a.H, a.rows, G, part, a.dq, a.dk, a.dg,
+            a.dbeta);
+        e = cudaGetLastError();
+        Profiler::mark(st);
+    }
+    return e;
 }
 
 template <int D, typename Tin>
-static cudaError_t launch_bwd_t(const BackwardArgs &a, cudaStream_t st) {
-    using L = bwd::Lay<D>;
-    const size_t smem = (size_t)(12 * D + L::RG * D + 2 * (L::CG + 1) * D) * sizeof(float);
-    auto kern = bwd::backward_kernel<D, Tin>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int64_t chunk_states = ((a.rows + bwd::C - 1) / bwd::C + a.N) * (int64_t)a.H;
-    float *ws = (float *)a.workspace;
-    kern<<<a.N * a.H, bwd::NT, smem, st>>>(
-        (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, (const Tin *)a.g, (const Tin *)a.beta,
-        a.state_in, a.cu_seqlens, a.T, a.N, a.H, a.dout, a.dstate_out, a.dq, a.dk, a.dv, a.dg,
-        a.dbeta, a.dstate_in, ws, ws + (size_t)chunk_states * D * D);
-    e = cudaGetLastError();
-    Profiler::mark(st);
-    return e;
+static cudaError_t launch_bwd_d(const BackwardArgs &a, cudaStream_t st) {
+    switch (bwd::slices_for((int64_t)a.N * a.H)) {
+    case 4: return launch_bwd_t<D, 4, Tin>(a, st);
+    case 2: return launch_bwd_t<D, 2, Tin>(a, st);
+    default: return launch_bwd_t<D, 1, Tin>(a, st);
+    }
 }
 
 cudaError_t launch_backward(const BackwardArgs &a, bool bf16, cudaStream_t st) {
     if (a.N * (int64_t)a.H == 0) return cudaSuccess;
     if (a.d == 64)
-        return bf16 ? launch_bwd_t<64, __nv_bfloat16>(a, st) : launch_bwd_t<64, float>(a, st);
-    return bf16 ? launch_bwd_t<128, __nv_bfloat16>(a, st) : launch_bwd_t<128, float>(a, st);
+        return bf16 ? launch_bwd_d<64, __nv_bfloat16>(a, st) : launch_bwd_d<64, float>(a, st);
+    return bf16 ? launch_bwd_d<128, __nv_bfloat16>(a, st) : launch_bwd_d<128, float>(a, st);
 }
 
 }  // namespace kda

@@ -167,8 +167,15 @@ def test_prefill_ex_rejects(lib, bad, code):
 
 
 def test_backward_workspace_bytes(lib):
-    assert lib.kda_backward_workspace_bytes(1000, 1, 2, 128, 128) == \
-        ((1000 + 63) // 64 + 1) * 2 * 128 * 128 * 4 + 1 * 2 * 64 * 128 * 128 * 4
+    states = ((1000 + 63) // 64 + 1) * 2 * 128 * 128 * 4 + 1 * 2 * 64 * 128 * 128 * 4
+    # 2 units: four value-column slices, each with its partial sums of dq, dk, da, dbeta
+    partials = 4 * 1000 * 2 * (3 * 128 + 4) * 4
+    assert lib.kda_backward_workspace_bytes(1000, 1, 2, 128, 128) == states + partials
+    # 50 units: two slices; 100 units: one, no partials
+    assert lib.kda_backward_workspace_bytes(1000, 1, 50, 64, 64) == \
+        ((1000 + 63) // 64 + 1) * 50 * 64 * 64 * 4 + 50 * 64 * 64 * 64 * 4 + 2 * 1000 * 50 * (3 * 64 + 4) * 4
+    assert lib.kda_backward_workspace_bytes(1000, 1, 100, 64, 64) == \
+        ((1000 + 63) // 64 + 1) * 100 * 64 * 64 * 4 + 100 * 64 * 64 * 64 * 4
     assert lib.kda_backward_workspace_bytes(10, 1, 2, 96, 96) == 0
 
 

@@ -59,3 +59,21 @@ def test_backward_clamped_decay_passes_no_gradient():
     grads = binding.kda_backward(d.q, d.k, d.v, d.g, d.beta, d.state_in, None,
                                  torch.ones(inp.v.shape, device="cuda"))
     assert not grads[3][0, 10:20, 0, :8].any()
+
+
+@pytest.mark.parametrize("B,H", [(1, 40), (2, 40)])
+def test_backward_column_slices(B, H):
+    """40 units: the value columns go to two CTAs per (sequence, head) and the
+    cross-column sums through partials; 80 units: one CTA, direct writes."""
+    inp = kin.prefill_inputs(B, 70, H, 64, 64, "bf16", seed=64 + B, state="normal")
+    check(inp, seed=4)
+
+
+def test_backward_column_slices_are_deterministic():
+    inp = kin.prefill_inputs(1, 130, 3, 128, 128, "bf16", seed=65, state="normal").to("cuda")
+    do = torch.randn(inp.v.shape, generator=torch.Generator().manual_seed(5)).cuda()
+    a = binding.kda_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.state_in, None, do)
+    b = binding.kda_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.state_in, None, do)
+    torch.cuda.synchronize()
+    for name, x, y in zip(NAMES, a, b):
+        assert torch.equal(x, y), name

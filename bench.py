@@ -416,7 +416,7 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
                              "ms_per_step": round(b_ms / nb, 3),
                              "value": aggregate_throughput(bw.B * bw.T, world, nb, b_ms),
                              "unit": "tokens/s",
-                             "kernel": "backward_kernel (fp32, one CTA per (sequence, head, value-column slice)) + backward_reduce_kernel"}
+                             "kernel": "backward_sliced_kernel (fp32, one CTA per (sequence, head, 32-column slice)) + backward_reduce_kernel"}
         del bw, dout, wsb
         torch.cuda.empty_cache()
 

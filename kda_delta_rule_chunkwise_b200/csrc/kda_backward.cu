@@ -32,9 +32,14 @@
 // straightforward form of the backward, not a tensor-core chunked one.
 #include "kda_common.cuh"
 #include "kda_launch.h"
+#include "sm100.cuh"
 
 namespace kda {
 namespace bwd {
+
+using sm100::cp_async16;
+using sm100::cp_async_commit;
+using sm100::cp_async_wait_all;
 
 constexpr int C = 64;     // tokens per stored chunk state
 constexpr int NT = 256;   // threads per CTA
@@ -335,6 +340,315 @@ backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     if (dstate_in) st_block(dstate_in + sbase, dS);
 }
 
+// Sliced form (DVS <= 64 value columns per CTA): warp w owns the columns
+// j0 + 4 w .. + 3 of the slice, lane l the key rows l + 32 i.  Column sums
+// (p, dd) are warp shuffles.  Token inputs move in batches of TB tokens: the
+// raw rows of the next batch are copied into shared memory (cp.async, double
+// buffered) while the current batch is computed, so the loads' latency is
+// paid once per batch instead of once per token.  The sums over columns (dq,
+// dk, da, dbeta) of a batch's tokens are added up once per batch.
+template <int D, int DVS, typename Tin>
+struct BwdBatch {
+    static constexpr int NW = DVS / 4;              // warps: 4 value columns each
+    static constexpr int NTH = 32 * NW;
+    static constexpr int RPT = D / 32;              // key rows per lane
+    static constexpr int TB = NW <= 8 ? 8 : 4;      // tokens per batch
+    static constexpr int ES = (int)sizeof(Tin);
+    // one token's raw inputs in shared memory (bytes): k, g, q rows; v, do slices; beta
+    static constexpr int RK = 0, RG = D * ES, RQ = 2 * D * ES, RV = 3 * D * ES;
+    static constexpr int RDO = RV + DVS * ES, RB = RDO + DVS * 4;
+    static constexpr int TOKB = (RB + 4 + 15) / 16 * 16;
+    static constexpr int PK = D * ES / 16, PV = DVS * ES / 16, PD = DVS * 4 / 16;
+    static constexpr int STG = 2 * TB * TOKB;       // two batch buffers
+    static constexpr int RED = TB * (3 * NW * D + NW) * 4;   // a batch's row partials
+    static constexpr int SMEM = STG + RED;
+    static_assert(NTH >= D && RV % 16 == 0 && RDO % 16 == 0, "layout");
+};
+
+template <int D, int DVS, typename Tin>
+__global__ void __launch_bounds__(8 * DVS, 1)
+backward_sliced_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                       const Tin *__restrict__ g, const Tin *__restrict__ beta, const float *state_in,
+                       const int32_t *__restrict__ cu, int64_t T, int N, int H, int64_t rows,
+                       const float *__restrict__ dout, const float *dstate_out,
+                       float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv,
+                       float *__restrict__ dg, float *__restrict__ dbeta, float *dstate_in,
+                       float *__restrict__ ws_chunks, float *__restrict__ ws_tokens,
+                       float *__restrict__ part) {
+    using B = BwdBatch<D, DVS, Tin>;
+    constexpr int NW = B::NW, NTH = B::NTH, RPT = B::RPT, TB = B::TB, TOKB = B::TOKB;
+    constexpr int NSL = D / DVS;
+    constexpr int PW = 3 * D + 4;
+    const int unit = blockIdx.x / NSL, slice = blockIdx.x % NSL;
+    const int n = unit / H, h = unit % H;
+    if (n >= N) return;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int j0 = slice * DVS;                  // first value column of this slice
+    const int jc = j0 + 4 * w;                   // this warp's first value column
+
+    extern __shared__ __align__(16) uint8_t smb[];
+    uint8_t *stg = smb;                                              // [2][TB][TOKB]
+    float *red = reinterpret_cast<float *>(smb + B::STG);            // [TB][3 NW D + NW]
+
+    int64_t ra, rb;
+    rows_of(cu, T, n, ra, rb);
+    const int64_t len = rb - ra;
+    const int nch = (int)((len + C - 1) / C);
+    float *chunks = ws_chunks + (size_t)(chunk_base(cu, T, n) * H + (int64_t)h * nch) * D * D;
+    float *toks = ws_tokens + (size_t)unit * C * D * D;
+    const size_t sbase = ((size_t)n * H + h) * D * D;
+    auto tok_off = [&](int64_t t, int d) { return ((size_t)(ra + t) * H + h) * d; };
+
+    // this thread's block of a D x D state: rows lane + 32 i, columns jc .. jc + 3
+    auto ld_block = [&](const float *src, float4 (&x)[RPT]) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i)
+            x[i] = src ? *reinterpret_cast<const float4 *>(src + (size_t)(lane + 32 * i) * D + jc)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    auto st_block = [&](float *dst, const float4 (&x)[RPT]) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) *reinterpret_cast<float4 *>(dst + (size_t)(lane + 32 * i) * D + jc) = x[i];
+    };
+    // sum over the 32 lanes (the key rows) of four column partials
+    auto warp_sum4 = [&](float4 x) {
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+            x.x += __shfl_xor_sync(0xffffffffu, x.x, m);
+            x.y += __shfl_xor_sync(0xffffffffu, x.y, m);
+            x.z += __shfl_xor_sync(0xffffffffu, x.z, m);
+            x.w += __shfl_xor_sync(0xffffffffu, x.w, m);
+        }
+        return x;
+    };
+    // Copies of the raw inputs of tokens t_first + dir * tau (tau < cnt) into
+    // batch buffer buf, with beta into a register of thread tau.
+    float breg = 0.f;
+    auto issue = [&](int buf, int64_t t_first, int cnt, int dir, bool bwd) {
+        constexpr int PK = B::PK, PV = B::PV, PD = B::PD;
+        const int cpt = bwd ? 3 * PK + PV + PD : 2 * PK + PV;
+        for (int task = tid; task < cnt * cpt; task += NTH) {
+            const int tau = task / cpt;
+            int pc = task % cpt;
+            const int64_t t = t_first + (int64_t)dir * tau;
+            uint8_t *dst = stg + (size_t)(buf * TB + tau) * TOKB;
+            const uint8_t *src;
+            if (pc < PK) {
+                src = reinterpret_cast<const uint8_t *>(k + tok_off(t, D)) + 16 * pc;
+                dst += B::RK + 16 * pc;
+            } else if ((pc -= PK) < PK) {
+                src = reinterpret_cast<const uint8_t *>(g + tok_off(t, D)) + 16 * pc;
+                dst += B::RG + 16 * pc;
+            } else if ((pc -= PK) < PV) {
+                src = reinterpret_cast<const uint8_t *>(v + tok_off(t, D) + j0) + 16 * pc;
+                dst += B::RV + 16 * pc;
+            } else if ((pc -= PV) < PK) {
+                src = reinterpret_cast<const uint8_t *>(q + tok_off(t, D)) + 16 * pc;
+                dst += B::RQ + 16 * pc;
+            } else {
+                pc -= PK;
+                src = reinterpret_cast<const uint8_t *>(dout + tok_off(t, D) + j0) + 16 * pc;
+                dst += B::RDO + 16 * pc;
+            }
+            cp_async16(dst, src, 16u);
+        }
+        cp_async_commit();
+        if (tid < cnt) breg = to_f32(beta[(size_t)(ra + t_first + (int64_t)dir * tid) * H + h]);
+    };
+    // the landed batch becomes visible (beta from the registers of its threads)
+    auto land = [&](int buf, int cnt) {
+        cp_async_wait_all();
+        if (tid < cnt) *reinterpret_cast<float *>(stg + (size_t)(buf * TB + tid) * TOKB + B::RB) = breg;
+        __syncthreads();
+    };
+    auto kval = [&](const uint8_t *tb, int c) { return to_f32(reinterpret_cast<const Tin *>(tb + B::RK)[c]); };
+    auto qval = [&](const uint8_t *tb, int c) { return to_f32(reinterpret_cast<const Tin *>(tb + B::RQ)[c]); };
+    auto gval = [&](const uint8_t *tb, int c) { return to_f32(reinterpret_cast<const Tin *>(tb + B::RG)[c]); };
+    auto vval4 = [&](const uint8_t *tb) {
+        const Tin *p = reinterpret_cast<const Tin *>(tb + B::RV) + 4 * w;
+        return make_float4(to_f32(p[0]), to_f32(p[1]), to_f32(p[2]), to_f32(p[3]));
+    };
+    // forward token step on S from the token's raw inputs: S <- Diag(a) S + k delta^T
+    auto fwd_step = [&](float4 (&S)[RPT], const uint8_t *tb) {
+        float kr[RPT], ar[RPT];
+        float4 pp = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const int r = lane + 32 * i;
+            kr[i] = kval(tb, r);
+            ar[i] = expf(fmaxf(gval(tb, r), -5.f));
+            const float ak = ar[i] * kr[i];
+            pp.x = fmaf(ak, S[i].x, pp.x); pp.y = fmaf(ak, S[i].y, pp.y);
+            pp.z = fmaf(ak, S[i].z, pp.z); pp.w = fmaf(ak, S[i].w, pp.w);
+        }
+        pp = warp_sum4(pp);                                           // p = S'^T k
+        const float b = *reinterpret_cast<const float *>(tb + B::RB);
+        const float4 vv = vval4(tb);
+        const float4 dl = make_float4(b * (vv.x - pp.x), b * (vv.y - pp.y), b * (vv.z - pp.z),
+                                      b * (vv.w - pp.w));
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            S[i].x = fmaf(kr[i], dl.x, ar[i] * S[i].x); S[i].y = fmaf(kr[i], dl.y, ar[i] * S[i].y);
+            S[i].z = fmaf(kr[i], dl.z, ar[i] * S[i].z); S[i].w = fmaf(kr[i], dl.w, ar[i] * S[i].w);
+        }
+    };
+    // forward over tokens t_begin .. t_begin + count - 1, storing the state before
+    // token u to dst: at chunk starts (u % C == 0, slot u / C) or, with every_token, always
+    // (slot u)
+    auto forward = [&](int64_t t_begin, int64_t count, float4 (&S)[RPT], float *dst, bool every_token) {
+        __syncthreads();   // both batch buffers are free
+        const int64_t nb = (count + TB - 1) / TB;
+        if (nb > 0) issue(0, t_begin, (int)(count < TB ? count : TB), 1, false);
+        for (int64_t bi = 0; bi < nb; ++bi) {
+            const int buf = (int)(bi & 1);
+            const int64_t u0 = bi * TB;
+            const int cnt = (int)((count - u0) < TB ? (count - u0) : TB);
+            land(buf, cnt);
+            if (bi + 1 < nb) {
+                const int64_t u1 = u0 + TB;
+                issue(buf ^ 1, t_begin + u1, (int)((count - u1) < TB ? (count - u1) : TB), 1, false);
+            }
+            for (int tau = 0; tau < cnt; ++tau) {
+                const int64_t u = u0 + tau;
+                if (every_token) st_block(dst + (size_t)u * D * D, S);
+                else if ((u % C) == 0) st_block(dst + (size_t)(u / C) * D * D, S);
+                fwd_step(S, stg + (size_t)(buf * TB + tau) * TOKB);
+            }
+        }
+    };
+
+    // ---- pass 1: forward, storing the state at every chunk start
+    float4 S[RPT];
+    ld_block(state_in ? state_in + sbase : nullptr, S);
+    forward(0, len, S, chunks, false);
+
+    // ---- pass 2: chunks in reverse
+    float4 dS[RPT];
+    ld_block(dstate_out ? dstate_out + sbase : nullptr, dS);
+    for (int ci = nch - 1; ci >= 0; --ci) {
+        const int64_t t0 = (int64_t)ci * C;
+        const int cl = (int)((len - t0) < C ? (len - t0) : C);
+        // rerun the chunk, keeping the state before each token
+        ld_block(chunks + (size_t)ci * D * D, S);
+        forward(t0, cl, S, toks, true);
+        // the token steps in reverse, batch by batch (tokens t_hi, t_hi - 1, ...)
+        __syncthreads();
+        const int nb = (cl + TB - 1) / TB;
+        issue(0, t0 + cl - 1, cl < TB ? cl : TB, -1, true);
+        float4 Sp[RPT], Spn[RPT];                 // S_{t-1} of this step and of the next
+        ld_block(toks + (size_t)(cl - 1) * D * D, Sp);
+        for (int bi = 0; bi < nb; ++bi) {
+            const int buf = bi & 1;
+            const int hi = cl - 1 - bi * TB;                       // highest token (in chunk) of this batch
+            const int cnt = hi + 1 < TB ? hi + 1 : TB;
+            land(buf, cnt);
+            if (bi + 1 < nb) {
+                const int hi1 = hi - TB;
+                issue(buf ^ 1, t0 + hi1, hi1 + 1 < TB ? hi1 + 1 : TB, -1, true);
+            }
+            for (int tau = 0; tau < cnt; ++tau) {
+                const int u = hi - tau;
+                const int64_t t = t0 + u;
+                const uint8_t *tb = stg + (size_t)(buf * TB + tau) * TOKB;
+                float *rq = red + (size_t)tau * (3 * NW * D + NW);  // this token's row partials
+                if (u > 0) ld_block(toks + (size_t)(u - 1) * D * D, Spn);
+                float kr[RPT], ar[RPT], qr[RPT];
+                float4 pp = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    const int r = lane + 32 * i;
+                    kr[i] = kval(tb, r);
+                    qr[i] = qval(tb, r);
+                    ar[i] = expf(fmaxf(gval(tb, r), -5.f));
+                    const float ak = ar[i] * kr[i];
+                    pp.x = fmaf(ak, Sp[i].x, pp.x); pp.y = fmaf(ak, Sp[i].y, pp.y);
+                    pp.z = fmaf(ak, Sp[i].z, pp.z); pp.w = fmaf(ak, Sp[i].w, pp.w);
+                }
+                pp = warp_sum4(pp);                                 // p = S'^T k
+                const float b = *reinterpret_cast<const float *>(tb + B::RB);
+                const float4 vv = vval4(tb);
+                const float4 do4 = *reinterpret_cast<const float4 *>(tb + B::RDO + 16 * w);
+                const float4 vp = make_float4(vv.x - pp.x, vv.y - pp.y, vv.z - pp.z, vv.w - pp.w);
+                const float4 dl = make_float4(b * vp.x, b * vp.y, b * vp.z, b * vp.w);
+                // dS += q do^T; row partials of dq = S_t do; column partials of dd = dS^T k
+                float4 cs = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    const int r = lane + 32 * i;
+                    dS[i].x = fmaf(qr[i], do4.x, dS[i].x); dS[i].y = fmaf(qr[i], do4.y, dS[i].y);
+                    dS[i].z = fmaf(qr[i], do4.z, dS[i].z); dS[i].w = fmaf(qr[i], do4.w, dS[i].w);
+                    const float4 St = make_float4(fmaf(kr[i], dl.x, ar[i] * Sp[i].x),
+                                                  fmaf(kr[i], dl.y, ar[i] * Sp[i].y),
+                                                  fmaf(kr[i], dl.z, ar[i] * Sp[i].z),
+                                                  fmaf(kr[i], dl.w, ar[i] * Sp[i].w));
+                    rq[w * D + r] = St.x * do4.x + St.y * do4.y + St.z * do4.z + St.w * do4.w;
+                    cs.x = fmaf(dS[i].x, kr[i], cs.x); cs.y = fmaf(dS[i].y, kr[i], cs.y);
+                    cs.z = fmaf(dS[i].z, kr[i], cs.z); cs.w = fmaf(dS[i].w, kr[i], cs.w);
+                }
+                const float4 dd = warp_sum4(cs);
+                if (lane == 0) {
+                    *reinterpret_cast<float4 *>(dv + tok_off(t, D) + jc) =
+                        make_float4(b * dd.x, b * dd.y, b * dd.z, b * dd.w);
+                    rq[3 * NW * D + w] = dd.x * vp.x + dd.y * vp.y + dd.z * vp.z + dd.w * vp.w;
+                }
+                const float4 dp = make_float4(-b * dd.x, -b * dd.y, -b * dd.z, -b * dd.w);
+                // row partials of dk = dS delta + S' dp and of da = rowsum(dS' * S_{t-1}),
+                // with dS' = dS + k dp^T; then dS <- Diag(a) dS'
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    const int r = lane + 32 * i;
+                    rq[NW * D + w * D + r] =
+                        dS[i].x * dl.x + dS[i].y * dl.y + dS[i].z * dl.z + dS[i].w * dl.w +
+                        ar[i] * (Sp[i].x * dp.x + Sp[i].y * dp.y + Sp[i].z * dp.z + Sp[i].w * dp.w);
+                    dS[i].x = fmaf(kr[i], dp.x, dS[i].x); dS[i].y = fmaf(kr[i], dp.y, dS[i].y);
+                    dS[i].z = fmaf(kr[i], dp.z, dS[i].z); dS[i].w = fmaf(kr[i], dp.w, dS[i].w);
+                    rq[2 * NW * D + w * D + r] = dS[i].x * Sp[i].x + dS[i].y * Sp[i].y +
+                                                dS[i].z * Sp[i].z + dS[i].w * Sp[i].w;
+                    dS[i].x *= ar[i]; dS[i].y *= ar[i]; dS[i].z *= ar[i]; dS[i].w *= ar[i];
+                }
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) Sp[i] = Spn[i];
+            }
+            __syncthreads();
+            // sums over the warps' columns, token by token
+            if (tid < D) {
+                for (int tau = 0; tau < cnt; ++tau) {
+                    const int64_t t = t0 + hi - tau;
+                    const float *rq = red + (size_t)tau * (3 * NW * D + NW);
+                    float aq = 0.f, akk = 0.f, aa = 0.f;
+#pragma unroll
+                    for (int x = 0; x < NW; ++x) {
+                        aq += rq[x * D + tid];
+                        akk += rq[NW * D + x * D + tid];
+                        aa += rq[2 * NW * D + x * D + tid];
+                    }
+                    if (NSL == 1) {
+                        const float gv = gval(stg + (size_t)(buf * TB + tau) * TOKB, tid);
+                        dq[tok_off(t, D) + tid] = aq;
+                        dk[tok_off(t, D) + tid] = akk;
+                        dg[tok_off(t, D) + tid] = aa * expf(fmaxf(gv, -5.f)) * (gv >= -5.f ? 1.f : 0.f);
+                    } else {
+                        float *pt = part + (((size_t)slice * rows + (ra + t)) * H + h) * PW;
+                        pt[tid] = aq;
+                        pt[D + tid] = akk;
+                        pt[2 * D + tid] = aa;
+                    }
+                }
+            }
+            if (tid < cnt) {
+                const int64_t t = t0 + hi - tid;
+                const float *rq = red + (size_t)tid * (3 * NW * D + NW);
+                float sb = 0.f;
+#pragma unroll
+                for (int x = 0; x < NW; ++x) sb += rq[3 * NW * D + x];
+                if (NSL == 1) dbeta[(size_t)(ra + t) * H + h] = sb;
+                else part[(((size_t)slice * rows + (ra + t)) * H + h) * PW + 3 * D] = sb;
+            }
+        }
+    }
+    if (dstate_in) st_block(dstate_in + sbase, dS);
+}
+
 // Sums of the column slices' partials, in slice order: dq, dk, dbeta, and
 // dg = da a (0 where g < -5).  CTA (unit, i) takes rows i, i + G, ... of its
 // sequence, one key channel per thread.
@@ -384,21 +698,37 @@ size_t backward_workspace_bytes(int64_t rows, int N, int H, int d) {
 template <int D, int NSL, typename Tin>
 static cudaError_t launch_bwd_t(const BackwardArgs &a, cudaStream_t st) {
     constexpr int DVS = D / NSL;
-    using L = bwd::Lay<D, DVS>;
-    const size_t smem =
-        (size_t)(5 * D + 7 * DVS + L::RG * DVS + 2 * (L::CG + 1) * D) * sizeof(float);
-    auto kern = bwd::backward_kernel<D, DVS, Tin>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const int64_t units = (int64_t)a.N * a.H;
     const int64_t chunk_states = ((a.rows + bwd::C - 1) / bwd::C + a.N) * (int64_t)a.H;
     const int64_t token_states = units * bwd::C;
     float *ws = (float *)a.workspace;
     float *part = ws + (size_t)(chunk_states + token_states) * D * D;
-    kern<<<(unsigned)(units * NSL), bwd::NT, smem, st>>>(
-        (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, (const Tin *)a.g, (const Tin *)a.beta,
-        a.state_in, a.cu_seqlens, a.T, a.N, a.H, a.rows, a.dout, a.dstate_out, a.dq, a.dk, a.dv,
-        a.dg, a.dbeta, a.dstate_in, ws, ws + (size_t)chunk_states * D * D, part);
+    cudaError_t e;
+    if constexpr (DVS <= 64) {
+        // warp-per-column-group form with batched token inputs
+        using BB = bwd::BwdBatch<D, DVS, Tin>;
+        const size_t smem = BB::SMEM;
+        auto kern = bwd::backward_sliced_kernel<D, DVS, Tin>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)(units * NSL), BB::NTH, smem, st>>>(
+            (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, (const Tin *)a.g,
+            (const Tin *)a.beta, a.state_in, a.cu_seqlens, a.T, a.N, a.H, a.rows, a.dout,
+            a.dstate_out, a.dq, a.dk, a.dv, a.dg, a.dbeta, a.dstate_in, ws,
+            ws + (size_t)chunk_states * D * D, part);
+    } else {
+        using L = bwd::Lay<D, DVS>;
+        const size_t smem =
+            (size_t)(5 * D + 7 * DVS + L::RG * DVS + 2 * (L::CG + 1) * D) * sizeof(float);
+        auto kern = bwd::backward_kernel<D, DVS, Tin>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)(units * NSL), bwd::NT, smem, st>>>(
+            (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, (const Tin *)a.g,
+            (const Tin *)a.beta, a.state_in, a.cu_seqlens, a.T, a.N, a.H, a.rows, a.dout,
+            a.dstate_out, a.dq, a.dk, a.dv, a.dg, a.dbeta, a.dstate_in, ws,
+            ws + (size_t)chunk_states * D * D, part);
+    }
     e = cudaGetLastError();
     Profiler::mark(st);
     if constexpr (NSL > 1) {

@@ -77,3 +77,29 @@ def test_backward_column_slices_are_deterministic():
     torch.cuda.synchronize()
     for name, x, y in zip(NAMES, a, b):
         assert torch.equal(x, y), name
+
+
+def test_backward_full_size_sampled_heads():
+    """The configuration the benchmark times (one sequence, T = 8192, H = 32,
+    four column slices per head): all heads run on the GPU, heads 0 and 31 are
+    checked against the oracle (heads are independent, so this is exact)."""
+    inp = kin.workload_inputs("prefill_h32_t8192_d128", seed=7)
+    do = torch.randn(inp.v.shape, generator=torch.Generator().manual_seed(8), dtype=torch.float32)
+    d = inp.to("cuda")
+    got = binding.kda_backward(d.q, d.k, d.v, d.g, d.beta, d.state_in, None, do.cuda())
+    torch.cuda.synchronize()
+    assert binding.kda_check_device_error() == binding.KDA_OK
+    heads = [0, 31]
+    pick = lambda x: x[:, :, heads].contiguous()
+    s0 = None if inp.state_in is None else inp.state_in[:, heads].contiguous()
+    ref = oracle.backward(pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.g), pick(inp.beta), s0,
+                          pick(do), None)
+    errs = {}
+    for name, x, y in zip(NAMES, got, ref):
+        if x is None:
+            continue
+        gx = to_np(x[:, heads] if name == "dstate_in" else x[:, :, heads])
+        errs[name] = rel_err(gx, y)
+    print({k_: f"{v_:.2e}" for k_, v_ in errs.items()})
+    for name, e in errs.items():
+        assert e <= TOL_F32, f"{name}: {e:.3e}"

@@ -103,3 +103,18 @@ def test_backward_full_size_sampled_heads():
     print({k_: f"{v_:.2e}" for k_, v_ in errs.items()})
     for name, e in errs.items():
         assert e <= TOL_F32, f"{name}: {e:.3e}"
+
+
+def test_backward_many_units_d128():
+    """80 (sequence, head) units at d = 128: one CTA of 256 threads per unit over
+    all 128 value columns (the unsliced kernel)."""
+    inp = kin.prefill_inputs(2, 70, 40, 128, 128, "bf16", seed=66, state="normal")
+    check(inp, seed=6)
+
+
+def test_backward_many_short_sequences():
+    """300 packed sequences of 0..9 tokens (many empty ones), 2 heads."""
+    lengths = kin.varlen_lengths(300, 0, 9, seed=67)
+    inp = kin.prefill_inputs(1, sum(lengths), 2, 64, 64, "f32", seed=67, state="normal",
+                             lengths=lengths)
+    check(inp, seed=7)

@@ -89,6 +89,15 @@ def test_bf16_varlen_edge_lengths():
     check(inp, TOL_BF16, what="bf16 varlen")
 
 
+def test_bf16_many_short_sequences():
+    """1500 packed sequences of 0..9 tokens (more sequences than the chunk table's
+    1024 threads, many empty ones), 2 heads."""
+    lens = kin.varlen_lengths(1500, 0, 9, seed=12)
+    inp = kin.prefill_inputs(1, sum(lens), 2, 128, 128, "bf16", seed=12, state="normal",
+                             lengths=lens)
+    check(inp, TOL_BF16, what="bf16 1500 short sequences")
+
+
 @pytest.mark.parametrize("H", [1, 100, 150])
 def test_bf16_slice_layouts(H):
     """(sequence, head) counts that select each dv-slice width of the state pass."""

@@ -320,6 +320,33 @@ def kda_backward(q, k, v, g, beta, state_in, cu_seqlens, dout, dstate_out=None, 
     return dq, dk_, dv_, dg, db, ds0
 
 
+class KDAPrefill(torch.autograd.Function):
+    """The prefill as a differentiable op: forward is kda_chunk_prefill, backward
+    is kda_backward (the exact gradients of the recurrence, fp32, cast to each
+    input's dtype).  Returns (o, state_out); cu_seqlens gets no gradient."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, beta, state_in=None, cu_seqlens=None):
+        o, s = kda_chunk_prefill(q, k, v, g, beta, state_in, cu_seqlens)
+        ctx.save_for_backward(q, k, v, g, beta, state_in, cu_seqlens)
+        return o, s
+
+    @staticmethod
+    def backward(ctx, do, dstate):
+        q, k, v, g, beta, state_in, cu = ctx.saved_tensors
+        grads = kda_backward(q, k, v, g, beta, state_in, cu, do.contiguous().float(),
+                             None if dstate is None else dstate.contiguous().float(),
+                             want_dstate_in=state_in is not None)
+        dq, dk_, dv_, dg, db, ds0 = grads
+        return (dq.to(q.dtype), dk_.to(k.dtype), dv_.to(v.dtype), dg.to(g.dtype),
+                db.to(beta.dtype), ds0, None)
+
+
+def kda_prefill_autograd(q, k, v, g, beta, state_in=None, cu_seqlens=None):
+    """Differentiable prefill (see KDAPrefill): (o, state_out)."""
+    return KDAPrefill.apply(q, k, v, g, beta, state_in, cu_seqlens)
+
+
 def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
     """One decode step; `state` [N, H, dk, dv] fp32 is updated in place.  Returns o (fp32)."""
     N, H, dk = q.shape

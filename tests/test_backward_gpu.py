@@ -118,3 +118,24 @@ def test_backward_many_short_sequences():
     inp = kin.prefill_inputs(1, sum(lengths), 2, 64, 64, "f32", seed=67, state="normal",
                              lengths=lengths)
     check(inp, seed=7)
+
+
+def test_autograd_wrapper_matches_the_backward_call():
+    """KDAPrefill through torch.autograd gives kda_backward's gradients exactly, and
+    they match the oracle."""
+    inp = kin.prefill_inputs(2, 90, 2, 64, 64, "f32", seed=68, state="normal").to("cuda")
+    leaves = [x.clone().requires_grad_(True) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta,
+                                                       inp.state_in)]
+    o, s = binding.kda_prefill_autograd(*leaves)
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    wo = torch.randn(o.shape, generator=gen, device="cuda")
+    ws = torch.randn(s.shape, generator=gen, device="cuda")
+    ((o * wo).sum() + (s * ws).sum()).backward()
+    direct = binding.kda_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.state_in, None, wo, ws)
+    torch.cuda.synchronize()
+    for name, leaf, ref in zip(NAMES, leaves, direct):
+        assert torch.equal(leaf.grad, ref), name
+    c = inp.to("cpu")
+    want = oracle.backward(c.q, c.k, c.v, c.g, c.beta, c.state_in, wo.cpu(), ws.cpu())
+    for name, leaf, y in zip(NAMES, leaves, want):
+        assert rel_err(to_np(leaf.grad), y) <= TOL_F32, name

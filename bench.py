@@ -653,7 +653,7 @@ def main():
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
     if rank == 0:
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:   # the oracle baseline is an N = 1 figure
             threads = cpu_threads()
             v, dt, smp = sized_oracle_sample(args.seed, args.ref_seconds, threads)
             res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": oracle_cores(threads),

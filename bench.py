@@ -166,7 +166,7 @@ def aggregate_throughput(units_per_rank_step: float, world: int, steps: int, ms_
 
 def time_prefill(binding, d, o, s_out, ws, steps, warmup, profile=False):
     st = torch.cuda.current_stream()
-    call = lambda: binding.kda_chunk_prefill(d.q, d.k, d.v, d.g, d.beta, d.state_in, None,
+    call = lambda: binding.kda_chunk_prefill(d.q, d.k, d.v, d.g, d.beta, d.state_in, d.cu_seqlens,
                                              o=o, state_out=s_out, workspace=ws)
     for _ in range(warmup):
         call()
@@ -239,7 +239,11 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
     n_k = len(per[0])
     k_avg = [sum(p[i] for p in per) / len(per) for i in range(n_k)]
     names = ["chunk_table_kernel", "intra_chunk_kernel", "state_pass_kernel"][:n_k]
-    head_chunks = H * B * ((T + 63) // 64)
+    if d.cu_seqlens is None:
+        head_chunks = H * B * ((T + 63) // 64)
+    else:   # packed sequences: each one's chunks
+        cu_h = d.cu_seqlens.cpu().tolist()
+        head_chunks = H * sum((cu_h[i + 1] - cu_h[i] + 63) // 64 for i in range(len(cu_h) - 1))
     k_bytes = {
         "chunk_table_kernel": 8 * (d.N + 1),
         "intra_chunk_kernel": head_chunks * (64 * (3 * 128 * 2 + 2) + SLOT_BYTES),

@@ -48,8 +48,8 @@ FLOPS_PER_TOKEN_HEAD = 139264                                 # algorithmic MMA 
 # launch from one ncu capture (profiles/), valid only for the kernel source it was taken
 # on: the sha256 prefix of that .cu file.  A changed source reports null.
 NCU_TRAFFIC = {
-    "intra_chunk_kernel": ("kda_prefill_bf16.cu", "1698401d6e201f53", (202423040 + 216636672) / 4096),
-    "state_pass_kernel": ("kda_prefill_bf16.cu", "1698401d6e201f53", (339787264 + 110925824) / 4096),
+    "intra_chunk_kernel": ("kda_prefill_bf16.cu", "5816df7998ae0054", (202408704 + 216729088) / 4096),
+    "state_pass_kernel": ("kda_prefill_bf16.cu", "5816df7998ae0054", (339792384 + 109159424) / 4096),
     "decode_kernel": ("kda_decode.cu", "4f1c8c21d6ac8934", 545290752 + 482616576),
 }
 
@@ -238,7 +238,8 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
     per = time_prefill(binding, d, o, s_out, ws, max(2, args.steps), 1, profile=True)
     n_k = len(per[0])
     k_avg = [sum(p[i] for p in per) / len(per) for i in range(n_k)]
-    names = ["chunk_table_kernel", "intra_chunk_kernel", "state_pass_kernel"][:n_k]
+    # (the chunk table is built for packed sequences only)
+    names = (["chunk_table_kernel"] if n_k == 3 else []) + ["intra_chunk_kernel", "state_pass_kernel"]
     if d.cu_seqlens is None:
         head_chunks = H * B * ((T + 63) // 64)
     else:   # packed sequences: each one's chunks
@@ -509,7 +510,9 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
 
 def finish(args, world, w, B, T, H, in_bytes, value, ms_step, roofline, roofline_path, decode,
            e2e, clk, extra):
-    launches = args.steps * 3 + 2 * max(0, args.decode_steps)   # prefill, decode, indexed decode
+    # prefill (2 kernels, 3 with the chunk table of packed sequences), decode, indexed decode
+    per_step = 3 if w.get("kind") == "varlen" else 2
+    launches = args.steps * per_step + 2 * max(0, args.decode_steps)
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),

@@ -272,8 +272,9 @@ KDA_API kda_status kda_selftest_bounded_wait(int64_t timeout_us, void *stream);
  * replaces the previous record.  kda_profile_last() waits for the last
  * recorded event and writes the device time of each kernel of the most
  * recent call, in launch order, to ms[0 .. *count-1] (at most `capacity`).
- * Prefill (bf16) launches three kernels: chunk table, intra-chunk products,
- * state pass; prefill (fp32) and decode launch one.
+ * Prefill (bf16) launches the intra-chunk products and the state pass, after a
+ * chunk-table kernel when cu_seqlens is given; prefill (fp32) and decode
+ * launch one.
  */
 KDA_API kda_status kda_profile_enable(int enable);
 KDA_API kda_status kda_profile_last(float *ms, int capacity, int *count);

@@ -937,7 +937,12 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
     int64_t ra, rb;
     seq_rows(chunk_off, cu != nullptr, T, N, n, ra, rb);
     const int nch = (int)((rb - ra + C - 1) / C);
-    const int c0 = chunk_off[n];
+    // first chunk of the sequence: from the table for packed sequences, else n chunks
+    // of T each (no table is built for equal-length batches)
+    const int c0 = cu ? chunk_off[n] : n * (int)((T + C - 1) / C);
+    // first intermediate-state entry of the sequence, likewise
+    const int64_t ck0 = cu ? (int64_t)chunk_off[2 * (N + 1) + n]
+                           : (int64_t)n * ((T > 0 && ckpt_interval > 0) ? (T - 1) / ckpt_interval : 0);
     const uint8_t *slots = ws + header_bytes(N);
     const int j0 = slice * DVS;   // first value channel of this slice
 
@@ -1265,7 +1270,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 if (ckpt_interval > 0 && ok) {
                     const int64_t done = (int64_t)(j + 1) * C;
                     if (done % ckpt_interval == 0 && done < rb - ra) {
-                        const int64_t e = (int64_t)chunk_off[2 * (N + 1) + n] + done / ckpt_interval - 1;
+                        const int64_t e = ck0 + done / ckpt_interval - 1;
                         if (e < ckpt_capacity) {
                             float4 *dst = reinterpret_cast<float4 *>(
                                 ckpt + (((size_t)e * H + h) * D + c) * D + j0);
@@ -1329,12 +1334,16 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
     if (a.dk != tc::D || a.dv != tc::D) return cudaErrorInvalidValue;
     uint8_t *ws = (uint8_t *)a.workspace;
-    tc::chunk_table_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.T, a.N,
-                                               a.ckpt_interval,
-                                               reinterpret_cast<int32_t *>(ws));
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    Profiler::mark(st);
+    cudaError_t e = cudaSuccess;
+    if (a.cu_seqlens) {
+        // packed sequences: row bounds and first chunks per sequence (both kernels
+        // below compute them by arithmetic for an equal-length batch)
+        tc::chunk_table_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.T, a.N, a.ckpt_interval,
+                                                   reinterpret_cast<int32_t *>(ws));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        Profiler::mark(st);
+    }
     const int64_t rows = (int64_t)a.B * a.T;
     const int64_t max_chunks =
         a.cu_seqlens ? (rows + tc::C - 1) / tc::C + a.N : (int64_t)a.N * ((a.T + tc::C - 1) / tc::C);

@@ -80,7 +80,9 @@ def test_intra_chunk_products(L, decay):
     d = inp.to("cuda")
     need = binding.kda_chunk_prefill_workspace_bytes(64 + L, 1, H, 128, 128, torch.bfloat16)
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    binding.kda_chunk_prefill(d.q, d.k, d.v, d.g, d.beta, None, None, workspace=ws)
+    # one packed sequence, so that the chunk table is built (equal-length batches skip it)
+    cu = torch.tensor([0, 64 + L], dtype=torch.int32, device="cuda")
+    binding.kda_chunk_prefill(d.q, d.k, d.v, d.g, d.beta, None, cu, workspace=ws)
     torch.cuda.synchronize()
     wsh = ws.cpu().numpy()
     hb = header_bytes(1)

@@ -43,7 +43,19 @@
  *    it in a per-library error word and exits; kda_check_device_error()
  *    reports it as KDA_ERR_TIMEOUT.  Kernels never trap.
  *  - Thread safety: calls on different streams may run concurrently, except
- *    that the error word is shared by every call in the process.
+ *    that the error word is shared by every call in the process.  A wait that
+ *    gives up ends only the launch it belongs to: a timeout recorded by an
+ *    earlier or a concurrent launch never cuts short another launch's work.
+ *  - Debug input scan: with the environment variable KDA_DEBUG_CHECKS=1 (read
+ *    at every call), each prefill and decode call first scans g and records
+ *    any value outside [-5, 0] (or NaN) in the error word, which the next
+ *    kda_check_device_error() reports as KDA_ERR_INPUT_RANGE.  The contract
+ *    on g is a property of the model's gate (the lower bound of neurohive.io
+ *    "Kimi K3 ... overview", section "Sequence length: hybrid KDA and Gated
+ *    MLA attention"); the scan reports a caller's inputs leaving it and
+ *    changes no result.  It is skipped when g holds gate logits
+ *    (KDA_PREP_GATE_LOGIT); for packed sequences it covers the rows
+ *    [cu_seqlens[0], cu_seqlens[N]).
  */
 #ifndef KDA_H
 #define KDA_H
@@ -66,7 +78,8 @@ typedef enum {
     KDA_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, bad cu_seqlens shape, short workspace */
     KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. dk != dv, d not 64/128) */
     KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
-    KDA_ERR_TIMEOUT = 4        /* a device-side bounded wait gave up (see kda_check_device_error) */
+    KDA_ERR_TIMEOUT = 4,       /* a device-side bounded wait gave up (see kda_check_device_error) */
+    KDA_ERR_INPUT_RANGE = 5    /* debug scan only: a log-decay outside [-5, 0] or NaN (KDA_DEBUG_CHECKS) */
 } kda_status;
 
 typedef enum {
@@ -247,11 +260,16 @@ KDA_API kda_status kda_backward(const void *q, const void *k, const void *v, con
                                 size_t workspace_bytes, void *stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device error word.
- * Returns KDA_ERR_INVALID_ARG if a kernel since the last call skipped work
- * because of an out-of-range index read on the device (kda_decode_step_indexed
- * slots), else KDA_ERR_TIMEOUT if one gave up a bounded wait, KDA_ERR_CUDA if
- * the stream reported an error, KDA_OK otherwise.
+ * Synchronises `stream`, then reads the device error word and reports ONE
+ * recorded condition, clearing only that one, most severe first:
+ *   KDA_ERR_TIMEOUT      a kernel gave up a bounded wait since it was last reported
+ *   KDA_ERR_INVALID_ARG  a kernel skipped work because of an out-of-range index
+ *                        read on the device (kda_decode_step_indexed slots, a
+ *                        snapshot array too small for kda_chunk_prefill_checkpointed)
+ *   KDA_ERR_INPUT_RANGE  the debug input scan (KDA_DEBUG_CHECKS=1) saw a
+ *                        log-decay outside [-5, 0]
+ * so calling it until it returns KDA_OK drains every condition.  Returns
+ * KDA_ERR_CUDA if the stream reported an error, KDA_OK if nothing is recorded.
  */
 KDA_API kda_status kda_check_device_error(void *stream);
 

@@ -17,7 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkda.so")
 
-KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_INPUT_RANGE = range(6)
 KDA_F32, KDA_BF16 = 0, 1
 KDA_PREP_GATE_LOGIT, KDA_PREP_L2NORM_QK = 1, 2
 _DTYPE = {torch.float32: KDA_F32, torch.bfloat16: KDA_BF16}

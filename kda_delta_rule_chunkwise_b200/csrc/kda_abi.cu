@@ -5,13 +5,17 @@
 #include "kda_common.cuh"
 #include "kda_launch.h"
 
+#include <atomic>
 #include <mutex>
 
 namespace {
 
-// One error word per device context, in this library's own device memory.
-// Kernels receive its device address as an argument.
-__device__ uint32_t g_kda_error_word;
+// One error area per device context, in this library's own device memory:
+// word 0 = error bits, word 1 = epoch of the latest launch that timed out
+// (kda_common.cuh).  Kernels receive its device address as an argument.
+__device__ uint32_t g_kda_error_word[2];
+
+std::atomic<uint32_t> g_epoch{0};
 
 constexpr int kMaxDevices = 64;
 uint32_t *g_err_ptr[kMaxDevices];
@@ -47,6 +51,14 @@ std::mutex g_prof_mu;
 }  // namespace
 
 namespace kda {
+
+uint32_t next_launch_epoch() {
+    uint32_t e;
+    do {
+        e = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+    } while (e == 0);   // 0 is the word's initial value: never an epoch
+    return e;
+}
 
 void Profiler::begin(cudaStream_t st) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -91,6 +103,7 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        case KDA_ERR_INPUT_RANGE: return "KDA_ERR_INPUT_RANGE";
     }
     return "KDA_ERR_UNKNOWN";
 }
@@ -128,8 +141,14 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
     if (!err) return KDA_ERR_CUDA;
     kda::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, B, T, N, H, dk, dv,
                        o, state_out, workspace, workspace_bytes, err,
-                       ckpt_interval, ckpt, ckpt_capacity, flags};
+                       ckpt_interval, ckpt, ckpt_capacity, flags, kda::next_launch_epoch()};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // debug input scan (not with gate logits in g: every logit is a valid input)
+    if (kda::debug_checks_enabled() && !(flags & KDA_PREP_GATE_LOGIT)) {
+        const cudaError_t e = kda::launch_input_scan(g, rows, H, dk, dtype == KDA_BF16,
+                                                     cu_seqlens, N, err, st);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
     kda::Profiler::begin(st);
     // the tensor-core path is for bf16 at d = 128; fp32, and bf16 at d = 64, take the
     // fp32 SIMT kernel (which reads either input type)
@@ -215,6 +234,12 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     if (N == 0) return KDA_OK;
     if ((reinterpret_cast<uintptr_t>(state) & 15u) != 0) return KDA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kda::debug_checks_enabled()) {
+        uint32_t *err = error_word_ptr();
+        if (!err) return KDA_ERR_CUDA;
+        if (kda::launch_input_scan(g, N, H, dk, dtype == KDA_BF16, nullptr, N, err, st) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    }
     kda::Profiler::begin(st);
     return from_cuda(kda::launch_decode(q, k, v, g, beta, state, N, H, dk, dtype == KDA_BF16, o,
                                         nullptr, N, nullptr, st));
@@ -236,6 +261,9 @@ kda_status kda_decode_step_indexed(const void *q, const void *k, const void *v, 
     uint32_t *err = error_word_ptr();
     if (!err) return KDA_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kda::debug_checks_enabled() &&
+        kda::launch_input_scan(g, N, H, dk, dtype == KDA_BF16, nullptr, N, err, st) != cudaSuccess)
+        return KDA_ERR_CUDA;
     kda::Profiler::begin(st);
     return from_cuda(kda::launch_decode(q, k, v, g, beta, state_pool, N, H, dk,
                                         dtype == KDA_BF16, o, slots, P, err, st));
@@ -283,13 +311,28 @@ kda_status kda_check_device_error(void *stream) {
     uint32_t word = 0;
     if (cudaMemcpyFromSymbol(&word, g_kda_error_word, sizeof(word)) != cudaSuccess)
         return KDA_ERR_CUDA;
-    if (word != 0) {
-        const uint32_t zero = 0;
-        if (cudaMemcpyToSymbol(g_kda_error_word, &zero, sizeof(zero)) != cudaSuccess)
-            return KDA_ERR_CUDA;
-        return (word & kda::ERR_BAD_INDEX) ? KDA_ERR_INVALID_ARG : KDA_ERR_TIMEOUT;
+    if (word == 0) return KDA_OK;
+    // One condition per call, most severe first; only the reported bits are
+    // cleared, so a following call reports the next one.
+    uint32_t bits;
+    kda_status s;
+    if (word & (kda::ERR_WAIT_TIMEOUT | kda::ERR_SELFTEST)) {
+        bits = kda::ERR_WAIT_TIMEOUT | kda::ERR_SELFTEST;
+        s = KDA_ERR_TIMEOUT;
+    } else if (word & kda::ERR_BAD_INDEX) {
+        bits = kda::ERR_BAD_INDEX;
+        s = KDA_ERR_INVALID_ARG;
+    } else if (word & kda::ERR_INPUT_RANGE) {
+        bits = kda::ERR_INPUT_RANGE;
+        s = KDA_ERR_INPUT_RANGE;
+    } else {
+        bits = word;
+        s = KDA_ERR_TIMEOUT;
     }
-    return KDA_OK;
+    const uint32_t rest = word & ~bits;
+    if (cudaMemcpyToSymbol(g_kda_error_word, &rest, sizeof(rest)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return s;
 }
 
 kda_status kda_profile_enable(int enable) {

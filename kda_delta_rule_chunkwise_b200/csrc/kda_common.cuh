@@ -8,13 +8,27 @@
 
 namespace kda {
 
-// Bits recorded in the device error word (one 32-bit word per library
-// instance and device, cleared by kda_check_device_error).
+// The device error area, one per library instance and device, is two 32-bit
+// words.  err[0] holds the bits below, reported (and cleared one at a time) by
+// kda_check_device_error.  err[1] holds the epoch of the latest launch in which
+// a bounded wait gave up: every launch that can wait gets a fresh nonzero
+// epoch from the host, and its CTAs stop waiting early only when err[1] holds
+// their own epoch.  So a timeout left over from an earlier launch (or from the
+// bounded-wait self test), or one in a launch running concurrently on another
+// stream, never cuts short the waits of a healthy launch.
 enum : uint32_t {
     ERR_WAIT_TIMEOUT = 1u,     // a bounded mbarrier/flag wait gave up
     ERR_SELFTEST = 2u,         // set by the bounded-wait self test
     ERR_BAD_INDEX = 4u,        // an index argument read on the device was out of range
+    ERR_INPUT_RANGE = 8u,      // the debug input scan found a log-decay outside [-5, 0]
 };
+
+// Record a timeout of the launch with the given epoch.
+__device__ __forceinline__ void record_timeout(uint32_t *err, uint32_t epoch) {
+    if (!err) return;
+    atomicOr(err, ERR_WAIT_TIMEOUT);
+    atomicExch(err + 1, epoch);
+}
 
 // Upper bound on the wall time of one device-side wait.  Legitimate waits in
 // these kernels last microseconds; anything past this bound means a missing
@@ -96,26 +110,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
 }
 
 // As mbar_wait, and also gives up as soon as another thread of the CTA has
-// raised the shared abort flag (set here on a timeout), or any CTA has recorded
-// a timeout in the device error word, so that one missing arrival ends every
-// waiting role of every CTA within microseconds instead of one time limit per
-// CTA.  Other error bits (an out-of-range index) do not stop the work.
+// raised the shared abort flag (set here on a timeout), or another CTA of the
+// same launch (same epoch) has recorded a timeout, so that one missing arrival
+// ends every waiting role of every CTA of the launch within microseconds
+// instead of one time limit per CTA.  Timeouts of other launches and the other
+// error bits (an out-of-range index) do not stop the work.
 __device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t parity,
-                                                    uint32_t *err, volatile uint32_t *abort,
+                                                    uint32_t *err, uint32_t epoch,
+                                                    volatile uint32_t *abort,
                                                     uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    const volatile uint32_t *gerr = err;
+    const volatile uint32_t *gepoch = err ? err + 1 : nullptr;
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (gerr && (*gerr & ERR_WAIT_TIMEOUT)) {   // some CTA already gave up: do not wait out the limit too
+        if (gepoch && *gepoch == epoch) {   // a CTA of this launch gave up: do not wait out the limit too
             *abort = 1u;
             return false;
         }
         if (globaltimer_ns() - t0 > limit_ns) break;
     }
-    if (err) atomicOr(err, ERR_WAIT_TIMEOUT);
+    record_timeout(err, epoch);
     *abort = 1u;
     return false;
 }

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "kda.h"
 #include "kda_launch.h"
@@ -73,6 +74,43 @@ cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, 
     return cudaSuccess;
 }
 
+// The two side streams and nine events of the copy pipeline, created once per
+// device on first use and kept until the process exits (creating and
+// destroying them on every call is driver work on a path that runs at the PCIe
+// limit).  One call at a time enqueues on them: the mutex is held while a call
+// enqueues its copies and kernels.  Reusing an event across calls is safe:
+// every wait a call enqueues refers to the record made before it.
+struct CopyPipeline {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[9] = {};   // start, in_ready[2], in_free[2], out_ready[2], out_free[2]
+};
+constexpr int kMaxDevices = 64;
+CopyPipeline g_pipes[kMaxDevices];
+
+// The current device's pipeline with its mutex locked (in `lk`), or nullptr.
+CopyPipeline *pipeline_for_current_device(std::unique_lock<std::mutex> &lk) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    CopyPipeline &p = g_pipes[dev];
+    lk = std::unique_lock<std::mutex>(p.mu);
+    if (p.ready) return &p;
+    bool ok = cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking) == cudaSuccess;
+    for (auto &e : p.ev)
+        ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        for (auto &e : p.ev)
+            if (e) cudaEventDestroy(e), e = nullptr;
+        if (p.s_in) cudaStreamDestroy(p.s_in), p.s_in = nullptr;
+        if (p.s_out) cudaStreamDestroy(p.s_out), p.s_out = nullptr;
+        return nullptr;
+    }
+    p.ready = true;
+    return &p;
+}
+
 }  // namespace
 
 extern "C" {
@@ -101,21 +139,16 @@ kda_status kda_chunk_prefill_host(const void *q, const void *k, const void *v, c
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    cudaStream_t s_in = nullptr, s_out = nullptr;
-    cudaEvent_t ev[9] = {};   // start, in_ready[2], in_free[2], out_ready[2], out_free[2]
+    std::unique_lock<std::mutex> lk;
+    CopyPipeline *pipe = pipeline_for_current_device(lk);
+    if (!pipe) return KDA_ERR_CUDA;
+    cudaStream_t s_in = pipe->s_in, s_out = pipe->s_out;
+    cudaEvent_t *ev = pipe->ev;
     kda_status st = KDA_OK;
     auto ok = [&](cudaError_t e) {
         if (e != cudaSuccess && st == KDA_OK) st = KDA_ERR_CUDA;
         return st == KDA_OK;
     };
-    if (!ok(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking)) ||
-        !ok(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking))) {
-        if (s_in) cudaStreamDestroy(s_in);
-        if (s_out) cudaStreamDestroy(s_out);
-        return st;
-    }
-    for (auto &e : ev)
-        if (!ok(cudaEventCreateWithFlags(&e, cudaEventDisableTiming))) break;
     cudaEvent_t start = ev[0], *in_ready = ev + 1, *in_free = ev + 3, *out_ready = ev + 5,
                 *out_free = ev + 7;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -178,15 +211,11 @@ kda_status kda_chunk_prefill_host(const void *q, const void *k, const void *v, c
     // when it stopped early on an error, so that the caller may free its
     // buffers once its stream is done.
     for (cudaStream_t side : {s_in, s_out}) {
-        if (in_free[0] && cudaEventRecord(in_free[0], side) == cudaSuccess)
+        if (cudaEventRecord(in_free[0], side) == cudaSuccess)
             cudaStreamWaitEvent(cs, in_free[0], 0);
         else
             cudaStreamSynchronize(side);
     }
-    for (auto &e : ev)
-        if (e) cudaEventDestroy(e);
-    cudaStreamDestroy(s_in);
-    cudaStreamDestroy(s_out);
     return st;
 }
 

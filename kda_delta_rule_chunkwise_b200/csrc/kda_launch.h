@@ -28,7 +28,11 @@ struct PrefillArgs {
     float *ckpt = nullptr;
     int64_t ckpt_capacity = 0;
     uint32_t flags = 0;          // KDA_PREP_* input preprocessing (kda.h)
+    uint32_t epoch = 0;          // this launch's nonzero epoch (see kda_common.cuh)
 };
+
+// A fresh nonzero epoch for one launch of kernels that use bounded waits.
+uint32_t next_launch_epoch();
 
 // Optional per-kernel event recording (see kda_profile_enable).  Launchers
 // call mark() before their first kernel and after each kernel.
@@ -44,6 +48,12 @@ size_t prefill_tc_workspace_bytes(int64_t rows, int N, int H, int d);
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *g,
                           const void *beta, float *state, int N, int H, int d, bool bf16,
                           void *o, const int32_t *slots, int P, uint32_t *err, cudaStream_t st);
+// Debug input scan (kda_debug.cu): sets ERR_INPUT_RANGE when a log-decay of
+// rows [cu[0], cu[N]) (all rows when cu is null) lies outside [-5, 0] or is NaN.
+cudaError_t launch_input_scan(const void *g, int64_t rows, int H, int dk, bool bf16,
+                              const int32_t *cu, int N, uint32_t *err, cudaStream_t st);
+// True when the environment variable KDA_DEBUG_CHECKS is set to 1 (read per call).
+bool debug_checks_enabled();
 cudaError_t launch_selftest_wait(uint64_t timeout_us, uint32_t *err, cudaStream_t st);
 
 // Backward (kda_backward.cu).  Gradients are fp32; inputs fp32 or bf16.

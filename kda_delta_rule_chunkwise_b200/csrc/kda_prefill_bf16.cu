@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(256, 2)
 intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ g, const __nv_bfloat16 *__restrict__ beta,
                    const int32_t *__restrict__ cu, int64_t T, int N, int H, uint32_t flags,
-                   uint8_t *__restrict__ ws, uint32_t *err) {
+                   uint8_t *__restrict__ ws, uint32_t *err, uint32_t epoch) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -517,7 +517,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
     for (int rd = 0; rd < 4; ++rd) {
         const uint32_t buf = A_OPS + (rd & 1) * A_RBUF;
-        if (rd >= 2 && ok) ok = mbar_wait_abortable(&bars[rd - 2], ph, err, abort_flag);
+        if (rd >= 2 && ok) ok = mbar_wait_abortable(&bars[rd - 2], ph, err, epoch, abort_flag);
         if (ok) {
             const int c0 = 32 * rd + 4 * p_l;
 #pragma unroll
@@ -581,7 +581,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             mma_commit(&bars[rd]);
         }
     }
-    if (ok) ok = mbar_wait_abortable(&bars[3], ph, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[3], ph, err, epoch, abort_flag);
     tc_fence_after();
 
     // ---- A2: K*Gamma (the high halves of the packed pairs) into the MN-major B operand of
@@ -764,7 +764,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         mma_commit(&bars[4]);
     }
-    if (ok) ok = mbar_wait_abortable(&bars[4], ph, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[4], ph, err, epoch, abort_flag);
     tc_fence_after();
     if (ok && warp < 4) {
         const int r = 16 * warp + (lane & 15);
@@ -808,7 +808,7 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         bulk_s2g(slot + kSlotTR, sm + A_TR, 16384);
         bulk_commit();
     }
-    if (ok) ok = mbar_wait_abortable(&bars[5], ph, err, abort_flag);
+    if (ok) ok = mbar_wait_abortable(&bars[5], ph, err, epoch, abort_flag);
     tc_fence_after();
     // the operand tiles are free once D1 has completed and the bulk store has
     // read [T; R]: the next item's rows go out now
@@ -915,7 +915,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                   const int32_t *__restrict__ cu, int64_t T, int N, int H,
                   const uint8_t *__restrict__ ws, float *__restrict__ o,
                   float *state_out, int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity,
-                  uint32_t *err) {
+                  uint32_t *err, uint32_t epoch) {
     using Lay = BLayout<DVS>;
     constexpr int NSL = D / DVS;
     constexpr int CPR = DVS / 8;   // 16-byte pieces per V row
@@ -992,7 +992,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         int issued = 0;
         for (int j = 0; j < nch; ++j) {
             const int st = j % NST;
-            if (j >= NST && !mbar_wait_abortable(&bars[EMPTY0 + st], empty_par(j), err, abort_flag))
+            if (j >= NST && !mbar_wait_abortable(&bars[EMPTY0 + st], empty_par(j), err, epoch, abort_flag))
                 break;
             uint8_t *stg = sm + st * Lay::kStageR;
             const uint8_t *src = slots + ((size_t)(c0 + j) * H + h) * kSlotBytes;
@@ -1023,7 +1023,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         bool ok = true;
         for (int j = 0; j < nch; ++j) {
             const int st = j % NST;
-            if (ok) ok = mbar_wait_abortable(&bars[VRAW0 + st], full_par(j), err, abort_flag);
+            if (ok) ok = mbar_wait_abortable(&bars[VRAW0 + st], full_par(j), err, epoch, abort_flag);
             if (ok) {
                 uint8_t *vt = sm + st * Lay::kStageR + kSlotBytes;
 #pragma unroll
@@ -1050,7 +1050,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         for (int j = 0; j < nch; ++j) {
             const int b = j & 1, st = j % NST;
             const uint32_t tTD = b ? tTD1 : tTD0;
-            if (ok) ok = mbar_wait_abortable(&bars[TDFULL0 + b], (j >> 1) & 1, err, abort_flag);
+            if (ok) ok = mbar_wait_abortable(&bars[TDFULL0 + b], (j >> 1) & 1, err, epoch, abort_flag);
             tc_fence_after();
             const int64_t t0 = ra + (int64_t)j * C;
             const int L = chunk_len(j);
@@ -1091,7 +1091,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 named_bar(1, 64);   // both U warps (4 and 5) have written their rows
                 if (issuer && ok) {
                     // and the state is scaled by Gamma_j (normally long since)
-                    ok = mbar_wait_abortable(&bars[TSSCALED], j & 1, err, abort_flag);
+                    ok = mbar_wait_abortable(&bars[TSSCALED], j & 1, err, epoch, abort_flag);
                     if (ok) {
                         tc_fence_after();
                         // S += Khat^T U   (descriptors advance by their start-address field)
@@ -1184,11 +1184,11 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
                 bool okk = ok_in;
                 if (okk) mbar_arrive(&bars[TSSCALED]);
                 if (okk && v_issued < j) {
-                    okk = mbar_wait_abortable(&bars[FULL0 + st], full_par(j), err, abort_flag);
-                    if (okk) okk = mbar_wait_abortable(&bars[VREADY0 + st], full_par(j), err, abort_flag);
+                    okk = mbar_wait_abortable(&bars[FULL0 + st], full_par(j), err, epoch, abort_flag);
+                    if (okk) okk = mbar_wait_abortable(&bars[VREADY0 + st], full_par(j), err, epoch, abort_flag);
                     if (okk && j >= 2)
                         okk = mbar_wait_abortable(&bars[TDEMPTY0 + b], ((j >> 1) + 1) & 1, err,
-                                                  abort_flag);
+                                                  epoch, abort_flag);
                     if (okk) {
                         tc_fence_after();
                         issue_vterm(j);
@@ -1217,7 +1217,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             return *s_grp_ok != 0u;
         };
         auto gamma_of = [&](int j, bool &ok) {
-            if (ok) ok = mbar_wait_abortable(&bars[FULL0 + j % NST], full_par(j), err, abort_flag);
+            if (ok) ok = mbar_wait_abortable(&bars[FULL0 + j % NST], full_par(j), err, epoch, abort_flag);
             return ok ? reinterpret_cast<const float *>(sm + (j % NST) * Lay::kStageR + kSlotGam)[c]
                       : 0.f;
         };
@@ -1250,7 +1250,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             }
             for (int j = 0; j < nch; ++j) {
                 // S_{j+1} = TS after the state update of chunk j
-                if (ok) ok = mbar_wait_abortable(&bars[TSFULL], j & 1, err, abort_flag);
+                if (ok) ok = mbar_wait_abortable(&bars[TSFULL], j & 1, err, epoch, abort_flag);
                 tc_fence_after();
                 if (ok) {
 #pragma unroll
@@ -1325,7 +1325,7 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
     kern<<<grid, 384, Lay::kBytes, st>>>((const __nv_bfloat16 *)a.v, a.state_in, a.cu_seqlens,
                                          a.T, a.N, a.H, (const uint8_t *)a.workspace,
                                          (float *)a.o, a.state_out, a.ckpt_interval, a.ckpt,
-                                         a.ckpt_capacity, a.err);
+                                         a.ckpt_capacity, a.err, a.epoch);
     e = cudaGetLastError();
     Profiler::mark(st);
     return e;
@@ -1360,7 +1360,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
         const int64_t ctas = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
         kern<<<(unsigned)ctas, 256, tc::A_SMEM, st>>>(
             (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
-            (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, a.flags, ws, a.err);
+            (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, a.flags, ws, a.err, a.epoch);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -43,11 +43,13 @@ prefill_f32_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
     int64_t r0, r1;
     if (cu_seqlens) {
-        int64_t a = cu_seqlens[n], b = cu_seqlens[n + 1];
-        a = a < 0 ? 0 : (a > T ? T : a);
-        b = b < 0 ? 0 : (b > T ? T : b);
-        r0 = a;
-        r1 = b < a ? a : b;
+        // offsets clamped to [0, T] and raised to the running maximum of the
+        // previous ones, as on every other path: sequences never overlap
+        auto cl = [&](int64_t x) { return x < 0 ? (int64_t)0 : (x > T ? T : x); };
+        int64_t run = 0;
+        for (int i = 0; i <= n; ++i) run = max(run, cl(cu_seqlens[i]));
+        r0 = run;
+        r1 = max(run, cl(cu_seqlens[n + 1]));
     } else {
         r0 = (int64_t)n * T;
         r1 = r0 + T;

@@ -85,3 +85,61 @@ def compare_units(ref, got, tol, what=""):
     assert eo <= tol, f"{what}: output error {eo:.3e} > {tol}"
     assert es <= tol, f"{what}: final-state error {es:.3e} > {tol}"
     return eo, es
+
+
+def compare_all_units(inp, o_gpu, s_gpu, tol, what="", budget=1 << 21, n_threads=None):
+    """Every (sequence, head) unit of a call against the oracle, element by element.
+
+    The oracle runs on groups of units of at most `budget` token-heads (whole
+    sequences, all heads or a slice of them) so that host memory stays
+    bounded; the error metric max|delta| / rms(reference) is taken over the
+    whole output tensor and over all final states, as for a single comparison.
+    """
+    if inp.cu_seqlens is None:
+        cu = np.arange(inp.B + 1) * inp.T
+    else:
+        cu = inp.cu_seqlens.cpu().numpy().astype(np.int64)
+    N, H = len(cu) - 1, inp.H
+    o_rows = o_gpu.reshape((-1,) + tuple(o_gpu.shape[2:])).cpu()
+    s_all = s_gpu.cpu()
+    acc = {"o": [0.0, 0.0, 0], "s": [0.0, 0.0, 0]}   # max|delta|, sum ref^2, count
+
+    def add(key, got, ref):
+        a = acc[key]
+        got = np.asarray(got, np.float64)
+        assert np.all(np.isfinite(got)), f"{what}: non-finite {key}"
+        a[0] = max(a[0], float(np.max(np.abs(got - ref))) if ref.size else 0.0)
+        a[1] += float(np.sum(ref * ref))
+        a[2] += ref.size
+
+    def run(seqs, heads):
+        ref = oracle_prefill(inp, heads=heads, seqs=seqs, n_threads=n_threads)
+        for (n, h), (o_ref, s_ref) in ref.items():
+            a, e = int(cu[n]), int(cu[n + 1])
+            add("o", to_np(o_rows[a:e, h]), o_ref)
+            add("s", to_np(s_all[n, h]), s_ref)
+
+    group, tok = [], 0
+    for n in range(N):
+        ln = int(cu[n + 1] - cu[n])
+        if ln * H > budget:                 # one long sequence: slices of heads
+            hs = max(1, budget // max(ln, 1))
+            for h0 in range(0, H, hs):
+                run([n], list(range(h0, min(H, h0 + hs))))
+            continue
+        if group and (tok + ln) * H > budget:
+            run(group, list(range(H)))
+            group, tok = [], 0
+        group.append(n)
+        tok += ln
+    if group:
+        run(group, list(range(H)))
+    errs = {}
+    for key, (mx, ss, cnt) in acc.items():
+        rms = np.sqrt(ss / max(cnt, 1))
+        errs[key] = mx / rms if rms > 0 else mx
+    print(f"{what}: all {N} x {H} units: output error {errs['o']:.3e}, "
+          f"final-state error {errs['s']:.3e} (bar {tol})")
+    assert errs["o"] <= tol, f"{what}: output error {errs['o']:.3e} > {tol}"
+    assert errs["s"] <= tol, f"{what}: final-state error {errs['s']:.3e} > {tol}"
+    return errs["o"], errs["s"]

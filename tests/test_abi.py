@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings(lib):
     for code, name in enumerate(["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED",
-                                 "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]):
+                                 "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT", "KDA_ERR_INPUT_RANGE"]):
         assert binding.status_string(code) == name
 
 

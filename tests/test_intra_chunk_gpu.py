@@ -19,6 +19,7 @@ import numpy as np
 import pytest
 import torch
 
+from _precision_emulation import chunk_factors
 from _util import rel_err
 from kda_delta_rule_chunkwise_b200 import binding
 from kda_delta_rule_chunkwise_b200 import inputs as kin
@@ -99,13 +100,23 @@ def test_intra_chunk_products(L, decay):
             errs = {"T": rel_err(TR[:n, :n], T), "R": rel_err(TR[64:64 + n, :n], R),
                     "W": rel_err(-WP[:n], W), "P": rel_err(WP[64:64 + n], P),
                     "Khat": rel_err(Kh[:n], Khr)}
-            print(tag, {k_: f"{v_:.2e}" for k_, v_ in errs.items()})
-            # Intermediates: fp16 storage (2^-12 relative) of products built on tf32
-            # Akk/Aqk (2^-11 relative per operand, with cancellation in the sums);
-            # checked at 5e-2 of each matrix's rms.  The end-to-end outputs are held
-            # to the 2e-2 bar in test_prefill_gpu.py.
+            # Bar per matrix, derived from the precision scheme rather than fixed: the
+            # same factors evaluated in fp64 with every operand rounded as the kernel
+            # stores it (tf32 Akk/Aqk operands, fp32 accumulation, fp16 storage; see
+            # _precision_emulation) have an error e_emul against the definitions
+            # above.  The kernel differs from that emulation only in the order of its
+            # fp32 sums and in its exp / reciprocal, so it must stay within a small
+            # multiple of it: bar = 4 e_emul, at least 4e-3 (a few fp16 ulps of the
+            # largest element).  The end-to-end outputs are held to the 2e-2 bar in
+            # test_prefill_gpu.py.
+            em = chunk_factors(f(inp.q[0, t0:t0 + n, h]), f(inp.k[0, t0:t0 + n, h]),
+                               f(inp.g[0, t0:t0 + n, h]), f(inp.beta[0, t0:t0 + n, h]))
+            emul = {"T": rel_err(em["T"], T), "R": rel_err(em["R"], R), "W": rel_err(em["W"], W),
+                    "P": rel_err(em["P"], P), "Khat": rel_err(em["Khat"], Khr)}
+            print(tag, {k_: f"{v_:.2e} (emulated {emul[k_]:.2e})" for k_, v_ in errs.items()})
             for name, e in errs.items():
-                assert e < 5e-2, f"{tag} {name}: {e:.3e}"
+                bar = max(4 * emul[name], 4e-3)
+                assert e < bar, f"{tag} {name}: {e:.3e} > {bar:.3e}"
             # Gamma_L = exp(G_L) <= 1 in fp32: absolute error (values below the fp32
             # range, e.g. e^-160 after a fast-decaying chunk, are 0)
             assert np.max(np.abs(Gam - Gr)) < 1e-6, tag + " Gamma"

@@ -7,7 +7,8 @@ import numpy as np
 import pytest
 import torch
 
-from _util import TOL_BF16, TOL_F32, compare_units, gather_gpu, oracle_prefill, rel_err, to_np
+from _util import (TOL_BF16, TOL_F32, compare_all_units, compare_units, gather_gpu,
+                   oracle_prefill, rel_err, to_np)
 from kda_delta_rule_chunkwise_b200 import binding
 from kda_delta_rule_chunkwise_b200 import inputs as kin
 
@@ -152,25 +153,26 @@ def test_bf16_prefill_then_decode_matches_long_prefill():
 
 @pytest.mark.slow
 def test_bf16_full_h32_t8192():
-    """B=1, H=32, T=8192, d=128, zero state: oracle on a sample of heads."""
+    """B=1, H=32, T=8192, d=128, zero state: every head against the oracle."""
     inp = kin.workload_inputs("prefill_h32_t8192_d128", seed=0, device="cuda")
-    check(inp, TOL_BF16, heads=[0, 13, 31], what="H32 T8192")
+    o, s = run(inp)
+    compare_all_units(inp.to("cpu"), o, s, TOL_BF16, what="H32 T8192")
 
 
 @pytest.mark.slow
 def test_bf16_full_h32_t65536_split():
-    """B=1, H=32, T=65536, split fast/slow decay, nonzero state: sampled heads."""
+    """B=1, H=32, T=65536, split fast/slow decay, nonzero state: every head."""
     inp = kin.workload_inputs("prefill_h32_t65536_d128_split", seed=0, device="cuda")
-    check(inp, TOL_BF16, heads=[5, 30], what="H32 T65536")
+    o, s = run(inp)
+    compare_all_units(inp.to("cpu"), o, s, TOL_BF16, what="H32 T65536")
 
 
 @pytest.mark.slow
 def test_bf16_full_varlen_64_sequences():
-    """64 packed sequences of 128..16384 tokens, H=32: sampled (sequence, head) units."""
+    """64 packed sequences of 128..16384 tokens, H=32: all 64 x 32 (sequence, head) units."""
     inp = kin.workload_inputs("varlen_64seq_128to16384_h32_d128", seed=0, device="cuda")
-    lens = np.diff(inp.cu_seqlens.cpu().numpy())
-    seqs = [int(np.argmin(lens)), int(np.argmax(lens)), 17]
-    check(inp, TOL_BF16, heads=[3], seqs=seqs, what="varlen 64 seqs")
+    o, s = run(inp)
+    compare_all_units(inp.to("cpu"), o, s, TOL_BF16, what="varlen 64 seqs")
 
 
 def test_bf16_prefill_is_deterministic():

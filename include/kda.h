@@ -122,6 +122,9 @@ KDA_API size_t kda_chunk_prefill_workspace_bytes(int64_t rows, int N, int H, int
  *  state_out   [N, H, dk, dv] fp32, final state per sequence, or NULL (not
  *              written).  May alias state_in exactly (in-place update).
  *              A zero-length sequence gets state_out = state_in (or zeros).
+ *  With dtype KDA_BF16 and d = 128 (the tensor-core path) q, k, g and v are
+ *  read as TMA tiles: their base addresses must be 16-byte aligned (else
+ *  KDA_ERR_INVALID_ARG) and B*T must stay below 2^31 (else KDA_ERR_UNSUPPORTED).
  *  workspace   device scratch of at least kda_chunk_prefill_workspace_bytes()
  *              bytes, 256-byte aligned, or NULL when that size is 0.  Its
  *              contents on return are the per-chunk intermediates of the

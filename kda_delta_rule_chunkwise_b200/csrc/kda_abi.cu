@@ -135,6 +135,13 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
     if (need > 0 && (!workspace || workspace_bytes < need ||
                      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
         return KDA_ERR_INVALID_ARG;
+    // the tensor-core path reads q, k, g and v as TMA tiles: 16-byte aligned bases,
+    // row coordinates that fit in int32
+    if (dtype == KDA_BF16 && dk == 128 && rows > 0) {
+        for (const void *p : {q, k, g, v})
+            if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return KDA_ERR_INVALID_ARG;
+        if (rows > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    }
     if (N == 0) return KDA_OK;
 
     uint32_t *err = error_word_ptr();

@@ -48,8 +48,11 @@
 // |v| and |state| stay below 65504.
 #include <cuda_fp16.h>
 
+#include <cstring>
+
 #include "kda_common.cuh"
 #include "kda_launch.h"
+#include "kda_tma.h"
 #include "sm100.cuh"
 
 namespace kda {
@@ -242,10 +245,11 @@ constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64 
 constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64     16 KiB
 constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128          16 KiB
 constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 solve scratch (32 x 32)               4 KiB
-// next item's rows, prefetched once D1 has completed (all of the above is dead by then)
-constexpr uint32_t A_QST = A_OPS + 16384;     // bf16 q [64][128], pieces permuted per row   16 KiB
-constexpr uint32_t A_KST = A_OPS + 32768;     // bf16 k, same layout                         16 KiB
-constexpr uint32_t A_GST = A_OPS + 49152;     // bf16 g [64][128]                            16 KiB
+// next item's rows, loaded by TMA once D1 has completed (all of the above is dead by then);
+// each tile is the TMA box layout of stage_off(): two 64-channel blocks of 64 rows x 128 B
+constexpr uint32_t A_QST = A_OPS + 16384;     // bf16 q [64][128]                            16 KiB
+constexpr uint32_t A_KST = A_OPS + 32768;     // bf16 k                                      16 KiB
+constexpr uint32_t A_GST = A_OPS + 49152;     // bf16 g                                      16 KiB
 constexpr uint32_t A_SMEM = A_OPS + 2 * A_RBUF + 1024;   // + alignment slack (= 112640)
 static_assert(A_Y + 4096 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
 static_assert(A_QST >= A_AK + 16384 && A_GST + 16384 <= A_OPS + 2 * A_RBUF, "staging area");
@@ -257,6 +261,13 @@ static_assert(A_OPS % 1024 == 0 && A_RBUF % 1024 == 0 && A_AQ % 1024 == 0 && A_T
 // consecutive rows (one row per lane) then spread over all banks.
 __device__ __forceinline__ int e1_at(int row, int col4) {   // col4: multiple of 4
     return row * 128 + (((col4 >> 2) ^ (row & 31)) << 2);
+}
+// Byte offset of (row, channel) in a staged [64][128] bf16 input tile as the TMA
+// box loads land: channels [0, 64) and [64, 128) in two blocks 8 KiB apart, each
+// 64 lines of 128 B with the 128-byte swizzle (16-byte piece index XOR row % 8).
+__device__ __forceinline__ uint32_t stage_off(int row, int ch) {
+    return (uint32_t)((ch >> 6) * 8192 + row * 128 + ((((ch & 63) >> 3) ^ (row & 7)) << 4) +
+                      (ch & 7) * 2);
 }
 // first row-group of the packed K^(a) tile: 0, 2, 6, 12
 __device__ __forceinline__ int at_group(int a) { return a * (a + 1); }
@@ -294,10 +305,12 @@ __device__ __forceinline__ float4 rcp4(float4 a) {
 
 // PREP: the input-preprocessing variant (flags at run time); the plain variant
 // compiles without any of it.
+// q, k and g arrive as TMA tiles (tensor maps over [rows, H, 128] bf16, boxes of
+// 64 channels x 64 rows); beta is read per row.
 template <bool PREP>
 __global__ void __launch_bounds__(256, 2)
-intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                   const __nv_bfloat16 *__restrict__ g, const __nv_bfloat16 *__restrict__ beta,
+intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16 *__restrict__ beta,
                    const int32_t *__restrict__ cu, int64_t T, int N, int H, uint32_t flags,
                    uint8_t *__restrict__ ws, uint32_t *err, uint32_t epoch) {
     extern __shared__ uint8_t smem_raw[];
@@ -353,26 +366,28 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     const int p_l = lane & 7, rsub = lane >> 3;
     auto a1_row = [&](int it) { return it == 0 ? 4 * warp + rsub : 32 + 4 * (warp ^ 4) + rsub; };
 
-    // Next item's q, k, g rows go to the staging area with cp.async (rows past
-    // the chunk zero-filled) while the current item finishes; beta into a
-    // register.  q and k rows have their 16-byte piece p at p ^ 4 (r % 4) so the
-    // operand-round reads below are free of bank conflicts; g is row-major.
+    // Next item's q, k, g rows go to the staging area as six TMA boxes (one thread
+    // issues them; their bytes complete bars[6]) while the current item finishes;
+    // beta into a register.  Rows past the chunk's end are zeroed once the tiles
+    // have landed (the boxes read the next rows of the tensor there, or zeros past
+    // its end).
     float bnext = 0.f;
+    int loads_issued = 0, items_done = 0;   // tile loads issued / consumed by this CTA
     auto prefetch = [&](int64_t item) {
         int64_t t0n;
         int Ln;
         locate(item, t0n, Ln);
         const int hn = (int)(item % H);
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&bars[6], 3 * 16384);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int task = tid + 256 * i, r = task >> 4, pc = task & 15;
-            const size_t off = ((size_t)(t0n + (r < Ln ? r : 0)) * H + hn) * D + pc * 8;
-            const uint32_t src_bytes = r < Ln ? 16u : 0u;
-            const uint32_t sw = (uint32_t)(r * 256 + ((pc ^ ((r & 3) << 2)) << 4));
-            cp_async16(sm + A_QST + sw, q + off, src_bytes);
-            cp_async16(sm + A_KST + sw, k + off, src_bytes);
-            cp_async16(sm + A_GST + task * 16, g + off, src_bytes);
+            for (int blk = 0; blk < 2; ++blk) {
+                tma_load_3d(sm + A_QST + blk * 8192, &tm_q, 64 * blk, hn, (int)t0n, &bars[6]);
+                tma_load_3d(sm + A_KST + blk * 8192, &tm_k, 64 * blk, hn, (int)t0n, &bars[6]);
+                tma_load_3d(sm + A_GST + blk * 8192, &tm_g, 64 * blk, hn, (int)t0n, &bars[6]);
+            }
         }
+        ++loads_issued;
         bnext = (tid < Ln) ? __bfloat162float(beta[(size_t)(t0n + (tid < 64 ? tid : 0)) * H + hn]) : 0.f;
     };
 
@@ -380,12 +395,13 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         tmem_alloc(tmem_ptr, 256);
         tmem_relinquish();
     }
-    if (tid == 32) {
+    if (tid == 0) {
         for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 4);   // operand rounds: four issuers
         for (int i = 4; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
         *abort_flag = 0u;
     }
+    __syncthreads();
     if ((int64_t)blockIdx.x < n_items) prefetch(blockIdx.x);
     tc_fence_before();
     __syncthreads();
@@ -400,15 +416,25 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     locate(item, t0, L);
     uint8_t *slot = ws + header_bytes(N) + (size_t)item * kSlotBytes;
 
-    // ---- this item's rows have landed (each thread waits for its own copies)
-    cp_async_wait_all();
+    // ---- this item's rows have landed; rows past the chunk's end are zeroed
+    const bool landed = mbar_wait_abortable(&bars[6], ph, err, epoch, abort_flag);
+    if (landed) ++items_done;
+    if (landed && L < C) {
+        for (int task = tid; task < (C - L) * 3 * 2; task += 256) {
+            const int r = L + task / 6, which = task % 6;
+            uint4 *line = reinterpret_cast<uint4 *>(sm + A_QST + (which >> 1) * 16384 +
+                                                     (which & 1) * 8192 + r * 128);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) line[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
     if (__syncthreads_or(*abort_flag != 0u)) break;
-    const __nv_bfloat16 *gst = reinterpret_cast<const __nv_bfloat16 *>(sm + A_GST);
     const int c = tid & 127, half = tid >> 7;
     float p[32];   // clamped log-decay of rows 32*half + i, then its prefix sums
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-        const float x = __bfloat162float(gst[(half * 32 + i) * D + c]);
+        const float x = __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16 *>(sm + A_GST + stage_off(half * 32 + i, c)));
         // gate from a logit: g = -5 sigmoid(x), inside (-5, 0) by construction.  Rows
         // past the chunk's end decay by nothing (their staged x is 0, which the
         // gate would map to -2.5): the block factors and EL then stay <= 1.
@@ -426,12 +452,12 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     float *inv_norm = reinterpret_cast<float *>(sm + A_GST);   // [2][64]: q rows, then k rows
     if (PREP && (flags & KDA_PREP_L2NORM_QK)) {
         const int which = tid >> 7, row = (tid >> 1) & 63, hf = tid & 1;
-        const uint8_t *src = sm + (which ? A_KST : A_QST) + row * 256;
+        const uint8_t *src = sm + (which ? A_KST : A_QST);
         float ss = 0.f;
 #pragma unroll
         for (int pc = 8 * hf; pc < 8 * hf + 8; ++pc) {
             float x[8];
-            unpack8(*reinterpret_cast<const uint4 *>(src + ((pc ^ ((row & 3) << 2)) << 4)), x);
+            unpack8(*reinterpret_cast<const uint4 *>(src + stage_off(row, pc * 8)), x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
         }
@@ -499,9 +525,8 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
             const int r = a1_row(it);
-            const int c0 = 32 * rd + 4 * p_l;   // 16-byte piece c0 / 8, 8-byte half (c0 / 4) & 1
-            const uint32_t sw =
-                (uint32_t)(r * 256 + (((c0 >> 3) ^ ((r & 3) << 2)) << 4) + ((c0 >> 2) & 1) * 8);
+            const int c0 = 32 * rd + 4 * p_l;   // four channels: one 8-byte half of a 16-byte piece
+            const uint32_t sw = stage_off(r, c0);
             qv[rd][it] = *reinterpret_cast<const uint2 *>(sm + A_QST + sw);
             kv[rd][it] = *reinterpret_cast<const uint2 *>(sm + A_KST + sw);
         }
@@ -858,7 +883,10 @@ intra_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
     tc_fence_after();
     }   // item loop
-    cp_async_wait_all();
+    // a load issued for an item this CTA will not process (the loop left early on an
+    // abort) must land before the CTA's shared memory is released (bounded wait)
+    if (tid == 0 && loads_issued > items_done)
+        mbar_wait(&bars[6], (uint32_t)(items_done & 1), err, 1ull << 28);
     if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
@@ -885,6 +913,16 @@ struct BLayout {
     static constexpr uint32_t oBar = oUB + kUB;
     static constexpr uint32_t kBytes = oBar + 256 + 1024;      // + barriers + alignment slack
     static constexpr uint32_t kTmemCols = DVS == 32 ? 128 : (DVS == 64 ? 256 : 512);
+    // V slice as its TMA boxes land: 64 rows of DVS channels, MN-major (channel
+    // contiguous) with the swizzle that matches the line length: 64-byte lines and
+    // the 64-byte swizzle for DVS = 32; 128-byte lines and the 128-byte swizzle
+    // otherwise, in 64-channel blocks 8 KiB apart.  These are the canonical UMMA
+    // MN-major swizzled layouts of the [T; R] V operand.
+    static constexpr uint32_t kVLine = DVS == 32 ? 64 : 128;
+    static constexpr Swizzle kVSwz = DVS == 32 ? SW_64B : SW_128B;
+    static constexpr uint32_t kVSbo = 8 * kVLine;            // 8-row (k) groups
+    static constexpr uint32_t kVLbo = 64 * kVLine;           // 64-channel blocks
+    static constexpr uint32_t kVKstep = 16 * kVLine;         // 16 rows: one K step of an MMA
     static_assert(kBytes <= 227 * 1024, "state pass shared memory");
 };
 
@@ -911,7 +949,7 @@ __device__ __forceinline__ void named_bar(uint32_t id, uint32_t nthreads) {
 // wait only skips work), so a timeout can never leave a barrier half-joined.
 template <int DVS>
 __global__ void __launch_bounds__(384, 1)
-state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
+state_pass_kernel(const __grid_constant__ CUtensorMap tm_v, const float *state_in,
                   const int32_t *__restrict__ cu, int64_t T, int N, int H,
                   const uint8_t *__restrict__ ws, float *__restrict__ o,
                   float *state_out, int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity,
@@ -954,7 +992,7 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
         for (int i = 0; i < Lay::NST; ++i) {
             mbar_init(&bars[FULL0 + i], 1);
             mbar_init(&bars[EMPTY0 + i], 1);
-            mbar_init(&bars[VRAW0 + i], 32);
+            mbar_init(&bars[VRAW0 + i], 1);
             mbar_init(&bars[VREADY0 + i], 1);
         }
         mbar_init(&bars[TDFULL0], 1);
@@ -985,40 +1023,41 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
 
     if (warp == 0) {
         // ------------------------------------------------ producer
-        // Chunk j's slot image goes in with one bulk copy; its V slice with
-        // cp.async straight into the operand positions (rows past the end of
-        // the sequence zero-filled), whose landing the lanes report on VRAW.
-        // Nothing here waits for a copy, so loads run NST chunks ahead.
+        // Chunk j's slot image goes in with one bulk copy; its V slice as TMA boxes
+        // straight into the operand layout (rows past the chunk's end are zeroed by
+        // the converters).  Both complete on mbarriers by their bytes, so nothing
+        // here waits for a copy and loads run NST chunks ahead.
         int issued = 0;
         for (int j = 0; j < nch; ++j) {
             const int st = j % NST;
-            if (j >= NST && !mbar_wait_abortable(&bars[EMPTY0 + st], empty_par(j), err, epoch, abort_flag))
+            if (j >= NST &&
+                !mbar_wait_abortable(&bars[EMPTY0 + st], empty_par(j), err, epoch, abort_flag))
                 break;
             uint8_t *stg = sm + st * Lay::kStageR;
             const uint8_t *src = slots + ((size_t)(c0 + j) * H + h) * kSlotBytes;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[FULL0 + st], kSlotBytes);
                 bulk_g2s(stg, src, kSlotBytes, &bars[FULL0 + st]);
+                const int t0 = (int)(ra + (int64_t)j * C);
+                mbar_arrive_expect_tx(&bars[VRAW0 + st], Lay::kVBytes);
+#pragma unroll
+                for (int blk = 0; blk < (DVS + 63) / 64; ++blk)
+                    tma_load_3d(stg + kSlotBytes + blk * 8192, &tm_v, j0 + 64 * blk, h, t0,
+                                &bars[VRAW0 + st]);
             }
-            const int64_t t0 = ra + (int64_t)j * C;
-            const int L = chunk_len(j);
-            uint8_t *vt = stg + kSlotBytes;
-            for (int task = lane; task < 64 * CPR; task += 32) {
-                const int r = task / CPR, ch = task % CPR;
-                const int rr = r < L ? r : 0;
-                cp_async16(vt + interleave_mnmajor_off(ch * 8, r, Lay::kKGroup),
-                           v + ((size_t)(t0 + rr) * H + h) * D + j0 + ch * 8, r < L ? 16u : 0u);
-            }
-            cp_async_arrive(&bars[VRAW0 + st]);
             issued = j + 1;
         }
         // drain: never leave the CTA with copies still landing in its shared memory
-        cp_async_wait_all();
         for (int j = issued - NST; j < issued; ++j)
-            if (j >= 0) mbar_wait(&bars[FULL0 + j % NST], full_par(j), err, 1ull << 28);
+            if (j >= 0) {
+                mbar_wait(&bars[FULL0 + j % NST], full_par(j), err, 1ull << 28);
+                mbar_wait(&bars[VRAW0 + j % NST], full_par(j), err, 1ull << 28);
+            }
     } else if (warp == 2 || warp == 3) {
         // ------------------------------------------------ V converters (64 threads)
-        // bf16 -> fp16 in place; each 16-byte piece holds 8 values of one row.
+        // bf16 -> fp16 in place; each 16-byte piece holds 8 values of one row (the
+        // swizzle only permutes pieces within a line).  Rows past the chunk's end
+        // hold the next rows of the tensor (or zeros past its end): they become 0.
         const int ct = tid - 64;
         bool ok = true;
         for (int j = 0; j < nch; ++j) {
@@ -1026,12 +1065,19 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             if (ok) ok = mbar_wait_abortable(&bars[VRAW0 + st], full_par(j), err, epoch, abort_flag);
             if (ok) {
                 uint8_t *vt = sm + st * Lay::kStageR + kSlotBytes;
+                const int L = chunk_len(j);
 #pragma unroll
                 for (int i = 0; i < CPR; ++i) {
-                    uint4 *pc = reinterpret_cast<uint4 *>(vt) + ct + 64 * i;
-                    float x[8];
-                    unpack8(*pc, x);
-                    *pc = pack8(x);
+                    const int idx = ct + 64 * i;
+                    const int row = ((idx * 16) % 8192) / (int)Lay::kVLine;
+                    uint4 *pc = reinterpret_cast<uint4 *>(vt) + idx;
+                    if (row < L) {
+                        float x[8];
+                        unpack8(*pc, x);
+                        *pc = pack8(x);
+                    } else {
+                        *pc = make_uint4(0u, 0u, 0u, 0u);
+                    }
                 }
             }
             fence_async_smem();
@@ -1154,11 +1200,12 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ v, const float *state_in,
             const int st = j % NST;
             const uint32_t tTD = (j & 1) ? tTD1 : tTD0;
             const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotTR, 16, 1024, SW_128B);
-            const uint64_t bd0 = smem_desc(stage_addr(st) + kSlotBytes, Lay::kKGroup, 128, SW_NONE);
+            const uint64_t bd0 =
+                smem_desc(stage_addr(st) + kSlotBytes, Lay::kVLbo, Lay::kVSbo, Lay::kVSwz);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_f16(tTD, ad0 + (uint64_t)(kk * 32 / 16),
-                        bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, kk > 0);
+                        bd0 + (uint64_t)(kk * Lay::kVKstep / 16), id_nn, kk > 0);
             v_issued = j;
         };
         auto vterm_ready = [&](int j) {   // one poll: slot, V slice and accumulator free
@@ -1321,8 +1368,16 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lay::kBytes);
     if (e != cudaSuccess) return e;
+    // TMA boxes of the V slice: DVS (at most 64) channels x 64 rows of one head
+    CUtensorMap tv;
+    const int64_t rows = (int64_t)a.B * a.T;
+    if (rows > 0 && !make_rows_heads_tmap(&tv, a.v, rows, a.H, tc::D, DVS < 64 ? DVS : 64, tc::C,
+                                          DVS == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (rows == 0) memset(&tv, 0, sizeof(tv));   // no chunk: the map is never used
     const int grid = a.N * a.H * (tc::D / DVS);
-    kern<<<grid, 384, Lay::kBytes, st>>>((const __nv_bfloat16 *)a.v, a.state_in, a.cu_seqlens,
+    kern<<<grid, 384, Lay::kBytes, st>>>(tv, a.state_in, a.cu_seqlens,
                                          a.T, a.N, a.H, (const uint8_t *)a.workspace,
                                          (float *)a.o, a.state_out, a.ckpt_interval, a.ckpt,
                                          a.ckpt_capacity, a.err, a.epoch);
@@ -1358,9 +1413,16 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
         const int64_t items = max_chunks * a.H;
         if (items > INT32_MAX - 65536) return cudaErrorInvalidValue;
         const int64_t ctas = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
+        // TMA tiles of q, k, g: 64 channels x 64 rows of one head per box
+        CUtensorMap tq, tk, tg;
+        if (rows > INT32_MAX ||
+            !make_rows_heads_tmap(&tq, a.q, rows, a.H, tc::D, 64, tc::C, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_rows_heads_tmap(&tk, a.k, rows, a.H, tc::D, 64, tc::C, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_rows_heads_tmap(&tg, a.g, rows, a.H, tc::D, 64, tc::C, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
         kern<<<(unsigned)ctas, 256, tc::A_SMEM, st>>>(
-            (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
-            (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, a.flags, ws, a.err, a.epoch);
+            tq, tk, tg, (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, a.flags, ws,
+            a.err, a.epoch);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

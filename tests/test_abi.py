@@ -84,6 +84,17 @@ def test_prefill_bf16_requires_workspace(lib):
     assert binding.raw_prefill(a) == binding.KDA_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("which", ["q", "k", "v", "g"])
+def test_prefill_bf16_requires_16_byte_aligned_tiles(lib, which):
+    """The tensor-core path loads q, k, g and v as TMA tiles: a base that is not
+    16-byte aligned is refused before anything is launched."""
+    need = lib.kda_chunk_prefill_workspace_bytes(16, 1, 2, 128, 128, binding.KDA_BF16)
+    a = _args(dtype=binding.KDA_BF16, dk=128, dv=128, q=1 << 20, k=2 << 20, v=3 << 20,
+              g=4 << 20, beta=5 << 20, o=6 << 20, workspace=8 << 20, workspace_bytes=need)
+    a[which] += 8
+    assert binding.raw_prefill(a) == binding.KDA_ERR_INVALID_ARG
+
+
 def test_prefill_zero_sequences_is_a_no_op(lib):
     # N = B = 0: nothing to do, nothing launched
     assert binding.raw_prefill(_args(B=0, N=0, q=None, k=None, v=None, g=None, beta=None,

@@ -660,76 +660,63 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // over four blocks, so N^4 = 0 and
     //     X = (I + N)^-1 Xd = (I - N)(I + N^2) Xd:
     //     N = Xd E,  N2 = N N,  P1 = Xd + N2 Xd,  X = P1 - N P1,
-    // four dependent 64x64x64 tf32 products (M=64: accumulator row 16q + l in TMEM
-    // lane 32q + l, l < 16).  tf32 operands must be K-major on both sides (the MMA
-    // reads a tf32 B operand as K-major whatever the descriptor's major bit says),
-    // so D = Y Z takes Y in its "A form" (Y[i][k] at ut(i, k)) and Z in its "B form"
-    // (Z[k][n] at ut(n, k), i.e. Z transposed).  The diagonal blocks of P1 and X are
-    // Xd's exact fp32 values (N2 Xd and N P1 are strictly block-lower).
-    // Buffers (16 KiB each): U1 = A_TR (Xd A form, then N A form), U2 = A_Y (E B form,
-    // N B form, N2 A form, P1 B form), U3 = A_AK (Xd B form, once Akk is consumed;
-    // then P1 exact, row-major fp32).
+    // four dependent 64x64x64 tf32 products (M=64: accumulator rows 16q + l in TMEM
+    // lanes 32q + l, l < 16).  Every operand is a 64x64 tf32 tile in the K-major
+    // 128-byte-swizzled layout, which is also the MN-major layout of its transpose
+    // role, so each matrix is stored once and serves as A (K-major) or B (MN-major).
+    // The diagonal blocks of P1 and X are Xd's exact fp32 values (N2 Xd and N P1 are
+    // strictly block-lower).  Buffers: U1 = A_TR (Xd, then P1), U2 = A_Y (E, then N),
+    // U3 = A_AK (N2, once Akk has been consumed).
     {
         constexpr uint32_t U1 = A_TR, U2 = A_Y, U3 = A_AK;
         auto ut = [](int i, int j) { return sw128_kmajor_off32((uint32_t)i, (uint32_t)j, 8192u); };
-        auto blk_lower = [](int i, int j) { return (i >> 4) > (j >> 4); };
+        // zero Xd's off-diagonal blocks (U1) and copy E (U2), tf32, one row quarter per thread
         if (ok && tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = EL[tid - 128];
-        // E in B form (E[k][n] at ut(n, k)): thread n reads column n of Akk (lanes over n:
-        // conflict-free) for 16 values of k and writes them contiguous; Xd's A form: its
-        // off-diagonal blocks zeroed here, its diagonal blocks by the forward substitution
         if (ok) {
-            const int nn = tid & 63, k0 = 16 * (tid >> 6);
+            const int i = tid >> 2, j0 = 16 * (tid & 3);
+            const bool diag = (i >> 4) == (j0 >> 4);
 #pragma unroll
             for (int cq = 0; cq < 4; ++cq) {
-                float e[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int kk = k0 + 4 * cq + u;
-                    e[u] = blk_lower(kk, nn) ? AK[kk * 64 + nn] : 0.f;
-                }
-                *reinterpret_cast<float4 *>(sm + U2 + ut(nn, k0 + 4 * cq)) = tf4(make_float4(e[0], e[1], e[2], e[3]));
-            }
-            const int i = tid >> 2, j0 = 16 * (tid & 3);
-            if ((i >> 4) != (j0 >> 4)) {
-#pragma unroll
-                for (int cq = 0; cq < 4; ++cq)
-                    *reinterpret_cast<float4 *>(sm + U1 + ut(i, j0 + 4 * cq)) = make_float4(0.f, 0.f, 0.f, 0.f);
+                const int j = j0 + 4 * cq;
+                const float4 e = diag ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(AK + i * 64 + j);
+                *reinterpret_cast<float4 *>(sm + U2 + ut(i, j)) = tf4(e);
+                if (!diag) *reinterpret_cast<float4 *>(sm + U1 + ut(i, j)) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         // the diagonal blocks: column j of inv(I + Akk_aa) by forward substitution (exact fp32)
-        float x[16];
-        const int fa = tid >> 4, fj = tid & 15, fo = 16 * fa;
         if (ok && tid < 64) {
+            const int a = tid >> 4, j = tid & 15, o = 16 * a;
+            float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                float acc = (i == fj) ? 1.f : 0.f;
+                float acc = (i == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int m = 0; m < i; ++m) acc = fmaf(-AK[(fo + i) * 64 + fo + m], x[m], acc);
+                for (int m = 0; m < i; ++m) acc = fmaf(-AK[(o + i) * 64 + o + m], x[m], acc);
                 x[i] = acc;
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + U1 + ut(fo + i, fo + fj)) = x[i];
+            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + U1 + ut(o + i, o + j)) = x[i];
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        // one 64x64x64 tf32 product D = A B into TMEM columns dcol, then its rows
+        // (lane < 16 of each warp: row m, columns 32 uh .. 32 uh + 31) in registers
         const int uq = warp & 3, uh = warp >> 2, um = 16 * uq + (lane & 15);
         uint32_t ucommit = 0;
-        auto ut_issue = [&](uint32_t abuf, uint32_t bbuf, uint32_t dcol) {
+        auto ut_mma = [&](uint32_t abuf, uint32_t bbuf, uint32_t dcol, float (&d)[32]) {
             if (ok && tid == 0) {
-                const uint32_t id = idesc(FMT_TF32, 64, 64, 0, 0);
+                const uint32_t id = idesc(FMT_TF32, 64, 64, 0, 1);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_tf32(tmem + dcol, smem_desc(sbase + abuf + ko, 16, 1024, SW_128B),
-                             smem_desc(sbase + bbuf + ko, 16, 1024, SW_128B), id, kk > 0);
+                    const uint64_t ad = smem_desc(sbase + abuf + (kk >> 2) * 8192 + (kk & 3) * 32, 16,
+                                                  1024, SW_128B);
+                    const uint64_t bd = smem_desc(sbase + bbuf + kk * 1024, 8192, 1024, SW_128B);
+                    mma_tf32(tmem + dcol, ad, bd, id, kk > 0);
                 }
                 mma_commit(&bars[7]);
             }
-        };
-        // wait for the product, then row um, columns 32 uh .. 32 uh + 31 into d
-        auto ut_read = [&](uint32_t dcol, float (&d)[32]) {
             if (ok) ok = mbar_wait_abortable(&bars[7], ucommit & 1u, err, epoch, abort_flag);
             ++ucommit;
             tc_fence_after();
@@ -739,73 +726,42 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_wait_ld();
             }
         };
-        auto ut_sync = [&]() {
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-        };
-        // A form of row um (columns of this thread's half), contiguous
-        auto put_a = [&](uint32_t buf, const float (&v)[32]) {
+        // row um, columns 32 uh .. + 31, of a tf32 operand tile
+        auto ut_store = [&](uint32_t buf, const float (&v)[32]) {
             if (ok && lane < 16) {
 #pragma unroll
                 for (int c4 = 0; c4 < 8; ++c4)
                     *reinterpret_cast<float4 *>(sm + buf + ut(um, 32 * uh + 4 * c4)) =
                         tf4(make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]));
             }
-        };
-        // B form of row um (Y[um][n] at ut(n, um)), one value per row of the tile
-        auto put_b = [&](uint32_t buf, const float (&v)[32]) {
-            if (ok && lane < 16) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    *reinterpret_cast<float *>(sm + buf + ut(32 * uh + e, um)) = tf32r(v[e]);
-            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
         };
         float d[32];
-        ut_issue(U1, U2, 0);                  // N = Xd E
-        // meanwhile: Xd in B form into U3 (every read of Akk came before the barrier
-        // above): zero blocks, and the forward-substitution threads' columns as rows
-        if (ok) {
-            const int nn = tid >> 2, k0 = 16 * (tid & 3);
-            if ((nn >> 4) != (k0 >> 4)) {
+        ut_mma(U1, U2, 0, d);        // N = Xd E
+        ut_store(U2, d);
+        ut_mma(U2, U2, 64, d);       // N2 = N N
+        ut_store(U3, d);
+        ut_mma(U3, U1, 0, d);        // N2 Xd
+        // P1 = Xd + N2 Xd (Xd exact from U1): rounded into U1 as the next B operand,
+        // exact into AK (row-major fp32; N2 in U3 = AK is consumed by now)
+        if (ok && lane < 16) {
 #pragma unroll
-                for (int cq = 0; cq < 4; ++cq)
-                    *reinterpret_cast<float4 *>(sm + U3 + ut(nn, k0 + 4 * cq)) = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int c4 = 0; c4 < 8; ++c4) {
+                const int col = 32 * uh + 4 * c4;
+                const float4 xd = ld4(reinterpret_cast<const float *>(sm + U1 + ut(um, col)));
+                d[4 * c4] += xd.x;
+                d[4 * c4 + 1] += xd.y;
+                d[4 * c4 + 2] += xd.z;
+                d[4 * c4 + 3] += xd.w;
+                *reinterpret_cast<float4 *>(AK + um * 64 + col) =
+                    make_float4(d[4 * c4], d[4 * c4 + 1], d[4 * c4 + 2], d[4 * c4 + 3]);
             }
         }
-        if (ok && tid < 64) {
-#pragma unroll
-            for (int cq = 0; cq < 4; ++cq)
-                *reinterpret_cast<float4 *>(sm + U3 + ut(fo + fj, fo + 4 * cq)) =
-                    make_float4(x[4 * cq], x[4 * cq + 1], x[4 * cq + 2], x[4 * cq + 3]);
-        }
-        ut_read(0, d);
-        put_a(U1, d);                         // N, A form (Xd's A form is consumed)
-        put_b(U2, d);                         // N, B form (E is consumed)
-        ut_sync();
-        ut_issue(U1, U2, 64);                 // N2 = N N
-        ut_read(64, d);
-        put_a(U2, d);                         // N2, A form
-        ut_sync();
-        ut_issue(U2, U3, 0);                  // N2 Xd
-        ut_read(0, d);
-        // P1 = Xd + N2 Xd, with Xd exact from its B form in U3
-        if (ok && lane < 16) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) d[e] += *reinterpret_cast<const float *>(sm + U3 + ut(32 * uh + e, um));
-        }
-        __syncthreads();                      // U3 is read before P1 overwrites it
-        if (ok && lane < 16) {
-#pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4)
-                *reinterpret_cast<float4 *>(AK + um * 64 + 32 * uh + 4 * c4) =
-                    make_float4(d[4 * c4], d[4 * c4 + 1], d[4 * c4 + 2], d[4 * c4 + 3]);
-        }
-        put_b(U2, d);                         // P1, B form (N2 is consumed)
-        ut_sync();
-        ut_issue(U1, U2, 64);                 // N P1
-        ut_read(64, d);
+        ut_store(U1, d);
+        ut_mma(U2, U1, 64, d);       // N P1
         // X = P1 - N P1 (lower triangular), T = X Diag(beta) into rows 0..63 of [T; R]
         // (fp16, K-major SW128; U1 is free once N P1 has completed)
         if (ok && lane < 16) {
@@ -1397,482 +1353,6 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_v, const float *state_i
     }
 }
 
-// ======================================================================
-// Phase B with one hand-off per chunk (32-column value slices)
-// ======================================================================
-// With Ut_j = T_j V_j the state update S_{j+1} = Diag(Gamma_j) S_j + Khat_j^T U_j,
-// U_j = Ut_j - W_j S_j, regroups as
-//     S_{j+1} = Diag(Gamma_j) S_j + A'_j S_j + Khat_j^T Ut_j,    A'_j = -Khat_j^T W_j,
-// and the outputs as O_j = R_j V_j + P_j S_j.  A'_j (128 x 128) and Khat_j^T Ut_j
-// do not depend on the state, so they are formed off the chunk-to-chunk chain;
-// what remains on it is one TMEM -> register -> shared-memory hand-off (the fp16
-// copy of S_j and Gamma_j S_j back into TMEM, both fp32-exact in the diagonal
-// term) and one group of 8 MMAs, A'_j S_j.
-//
-// Roles (512 threads), each with its own mbarriers (all waits bounded):
-//   warp 0      producer: slot image (one bulk copy) and V slice (TMA) per chunk
-//   warp 1      TMEM owner; lane 0 issues TD_j = [T; R]_j V_j and TA_j = Khat_j^T (-W_j)
-//   warps 2-3   V converters (bf16 -> fp16 in place, rows past the chunk zeroed)
-//   warps 4-5   Ut rows of TD_j -> fp16 (UB); lane 0 of warp 4 issues TX_j = Khat_j^T Ut_j
-//   warps 6-7   O rows: R_j V_j (TD_j) + P_j S_j (TO_j) -> o
-//   warps 8-11  the chain: S_j = TS + TX_{j-1} -> fp16 SB_j and TS <- Gamma_j S_j;
-//               lane 0 of warp 8 issues TS += A'_j SB_j, then TO_j = [-W; P]_j SB_j
-//   warps 12-15 A' builders: TA_j -> fp16 K-major operand AB_j
-// Every accumulator is fed by one issuing thread in a fixed order, so results are
-// the same on every run.
-struct B1Layout {
-    static constexpr int DVS = 32, NST = 2;
-    static constexpr uint32_t kVBytes = 64 * DVS * 2;                 // V slice, 4 KiB
-    static constexpr uint32_t kStage = kSlotBytes + kVBytes;          // 70656, 1024-multiple
-    static constexpr uint32_t kAB = 32768;                            // fp16 A', 128 x 128
-    static constexpr uint32_t kSB = 128 * DVS * 2;                    // fp16 S (K=128 x N=32)
-    static constexpr uint32_t kUB = 64 * DVS * 2;                     // fp16 Ut (K=64 x N=32)
-    static constexpr uint32_t kKGroup = (DVS / 8) * 128;              // interleaved MN-major k-group stride
-    static constexpr uint32_t oAB = NST * kStage;
-    static constexpr uint32_t oSB = oAB + 2 * kAB;
-    static constexpr uint32_t oUB = oSB + 2 * kSB;
-    static constexpr uint32_t oBar = oUB + kUB;
-    static constexpr uint32_t kBytes = oBar + 512 + 1024;
-    // TMEM columns
-    static constexpr uint32_t cTD = 0, cTO = 64, cTX = 128, cTS = 192, cTA = 256;
-    static_assert(kStage % 1024 == 0 && oAB % 1024 == 0, "swizzled operands need 1024-byte alignment");
-    static_assert(kBytes <= 227 * 1024, "state pass shared memory");
-};
-
-enum B1Bar {
-    A_FULL0 = 0, A_EMPTY0 = 2, A_VRAW0 = 4, A_VREADY0 = 6, A_TDFULL0 = 8, A_TDEMPTY0 = 10,
-    A_TAFULL0 = 12, A_TAEMPTY0 = 14, A_AFULL0 = 16, A_AEMPTY0 = 18, A_TXFULL0 = 20,
-    A_TXEMPTY0 = 22, A_TOFULL0 = 24, A_TOEMPTY0 = 26, A_TSFULL = 28, A_DRAIN_AUX, A_DRAIN_U,
-    A_DRAIN_S, A_NBARS
-};
-static_assert(A_NBARS * 8 + 16 <= 512, "phase B barrier area");
-
-__global__ void __launch_bounds__(512, 1)
-state_pass_a_kernel(const __grid_constant__ CUtensorMap tm_v, const float *state_in,
-                    const int32_t *__restrict__ cu, int64_t T, int N, int H,
-                    const uint8_t *__restrict__ ws, float *__restrict__ o, float *state_out,
-                    int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity, uint32_t *err,
-                    uint32_t epoch) {
-    using Lay = B1Layout;
-    using VL = BLayout<32>;   // the V slice's TMA layout (64-byte lines, 64-byte swizzle)
-    constexpr int DVS = Lay::DVS, NSL = D / DVS, NST = Lay::NST, CPR = DVS / 8;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const uint32_t sbase = smem_u32(sm);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::oBar);
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + A_NBARS);
-    volatile uint32_t *abort_flag = tmem_ptr + 1;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int slice = blockIdx.x % NSL;
-    const int unit = blockIdx.x / NSL;
-    const int n = unit / H, h = unit % H;
-    if (n >= N) return;
-    const int32_t *chunk_off = reinterpret_cast<const int32_t *>(ws);
-    int64_t ra, rb;
-    seq_rows(chunk_off, cu != nullptr, T, N, n, ra, rb);
-    const int nch = (int)((rb - ra + C - 1) / C);
-    const int c0 = cu ? chunk_off[n] : n * (int)((T + C - 1) / C);
-    const int64_t ck0 = cu ? (int64_t)chunk_off[2 * (N + 1) + n]
-                           : (int64_t)n * ((T > 0 && ckpt_interval > 0) ? (T - 1) / ckpt_interval : 0);
-    const uint8_t *slots = ws + header_bytes(N);
-    const int j0 = slice * DVS;
-
-    if (warp == 1) {
-        tmem_alloc(tmem_ptr, 512);
-        tmem_relinquish();
-    }
-    if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[A_FULL0 + i], 1);
-            mbar_init(&bars[A_EMPTY0 + i], 2);      // the U issuer's and the state issuer's commits
-            mbar_init(&bars[A_VRAW0 + i], 1);
-            mbar_init(&bars[A_VREADY0 + i], 1);
-            mbar_init(&bars[A_TDFULL0 + i], 1);
-            mbar_init(&bars[A_TDEMPTY0 + i], 4);    // the four U/O warps
-            mbar_init(&bars[A_TAFULL0 + i], 1);
-            mbar_init(&bars[A_TAEMPTY0 + i], 4);    // the four builder warps
-            mbar_init(&bars[A_AFULL0 + i], 1);
-            mbar_init(&bars[A_AEMPTY0 + i], 1);
-            mbar_init(&bars[A_TXFULL0 + i], 1);
-            mbar_init(&bars[A_TXEMPTY0 + i], 4);    // the four state warps
-            mbar_init(&bars[A_TOFULL0 + i], 1);
-            mbar_init(&bars[A_TOEMPTY0 + i], 2);    // the two O warps
-        }
-        mbar_init(&bars[A_TSFULL], 1);
-        mbar_init(&bars[A_DRAIN_AUX], 1);
-        mbar_init(&bars[A_DRAIN_U], 1);
-        mbar_init(&bars[A_DRAIN_S], 1);
-        mbar_fence_init();
-        *abort_flag = 0u;
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_ptr;
-    auto stage_addr = [&](int st) { return sbase + st * Lay::kStage; };
-    // parity of chunk j's completion of a two-deep barrier, and of chunk j-2's (before reuse)
-    auto par = [](int j) { return (uint32_t)((j >> 1) & 1); };
-    auto par_prev = [](int j) { return (uint32_t)(((j >> 1) + 1) & 1); };
-    auto chunk_len = [&](int j) {
-        const int64_t t0 = ra + (int64_t)j * C;
-        return (int)((rb - t0) < C ? (rb - t0) : C);
-    };
-    auto wait = [&](int bar, uint32_t parity) {
-        return mbar_wait_abortable(&bars[bar], parity, err, epoch, abort_flag);
-    };
-    const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);    // A K-major, B MN-major
-    const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);    // A MN-major, B MN-major
-    const uint32_t id_a = idesc(FMT_F16, 128, 128, 1, 1);     // Khat^T (-W)
-
-    if (warp == 0) {
-        // ------------------------------------------------ producer
-        int issued = 0;
-        for (int j = 0; j < nch; ++j) {
-            const int st = j % NST;
-            if (j >= NST && !wait(A_EMPTY0 + st, par_prev(j))) break;
-            uint8_t *stg = sm + st * Lay::kStage;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[A_FULL0 + st], kSlotBytes);
-                bulk_g2s(stg, slots + ((size_t)(c0 + j) * H + h) * kSlotBytes, kSlotBytes,
-                         &bars[A_FULL0 + st]);
-                mbar_arrive_expect_tx(&bars[A_VRAW0 + st], Lay::kVBytes);
-                tma_load_3d(stg + kSlotBytes, &tm_v, j0, h, (int)(ra + (int64_t)j * C),
-                            &bars[A_VRAW0 + st]);
-            }
-            issued = j + 1;
-        }
-        for (int j = issued - NST; j < issued; ++j)
-            if (j >= 0) {
-                mbar_wait(&bars[A_FULL0 + j % NST], par(j), err, 1ull << 28);
-                mbar_wait(&bars[A_VRAW0 + j % NST], par(j), err, 1ull << 28);
-            }
-    } else if (warp == 1) {
-        // ------------------------------------------------ TMEM owner; lane 0: TD_j and TA_j
-        if (lane == 0) {
-            bool ok = true;
-            for (int j = 0; j < nch && ok; ++j) {
-                const int st = j % NST, b = j & 1;
-                ok = wait(A_FULL0 + st, par(j)) && wait(A_VREADY0 + st, par(j));
-                if (ok && j >= 2) ok = wait(A_TDEMPTY0 + b, par_prev(j)) && wait(A_TAEMPTY0 + b, par_prev(j));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t sa = stage_addr(st);
-                {   // TD_j = [T; R]_j V_j
-                    const uint64_t ad0 = smem_desc(sa + kSlotTR, 16, 1024, SW_128B);
-                    const uint64_t bd0 = smem_desc(sa + kSlotBytes, VL::kVLbo, VL::kVSbo, VL::kVSwz);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(tmem + Lay::cTD + 32 * b, ad0 + (uint64_t)(kk * 32 / 16),
-                                bd0 + (uint64_t)(kk * VL::kVKstep / 16), id_nn, kk > 0);
-                    mma_commit(&bars[A_TDFULL0 + b]);
-                }
-                {   // TA_j = Khat_j^T (-W_j): A = Khat (MN-major over channels), B = the -W
-                    // rows of [-W; P] read as an MN-major K=token x N=channel operand
-                    const uint64_t ad0 = smem_desc(sa + kSlotKh, kKhMNBlock, 1024, SW_128B);
-                    const uint64_t bd0 = smem_desc(sa + kSlotWP, kWPKBlock, 1024, SW_128B);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(tmem + Lay::cTA + 128 * b, ad0 + (uint64_t)(kk * 2048 / 16),
-                                bd0 + (uint64_t)(kk * 2048 / 16), id_a, kk > 0);
-                    mma_commit(&bars[A_TAFULL0 + b]);
-                }
-            }
-            mma_commit(&bars[A_DRAIN_AUX]);
-            mbar_wait(&bars[A_DRAIN_AUX], 0, err, 1ull << 28);
-        }
-        __syncwarp();
-    } else if (warp == 2 || warp == 3) {
-        // ------------------------------------------------ V converters (64 threads)
-        const int ct = tid - 64;
-        bool ok = true;
-        for (int j = 0; j < nch; ++j) {
-            const int st = j % NST;
-            if (ok) ok = wait(A_VRAW0 + st, par(j));
-            if (ok) {
-                uint8_t *vt = sm + st * Lay::kStage + kSlotBytes;
-                const int L = chunk_len(j);
-#pragma unroll
-                for (int i = 0; i < CPR; ++i) {
-                    const int idx = ct + 64 * i;
-                    const int row = (idx * 16) / (int)VL::kVLine;
-                    uint4 *pc = reinterpret_cast<uint4 *>(vt) + idx;
-                    if (row < L) {
-                        float x[8];
-                        unpack8(*pc, x);
-                        *pc = pack8(x);
-                    } else {
-                        *pc = make_uint4(0u, 0u, 0u, 0u);
-                    }
-                }
-            }
-            fence_async_smem();
-            named_bar(3, 64);
-            if (ct == 0 && ok) mbar_arrive(&bars[A_VREADY0 + st]);
-        }
-    } else if (warp == 4 || warp == 5) {
-        // ------------------------------------------------ Ut rows -> UB; TX_j = Khat_j^T Ut_j
-        const int quad = warp - 4, row = 32 * quad + lane;
-        const bool issuer = (warp == 4 && lane == 0);
-        bool ok = true;
-        for (int j = 0; j < nch; ++j) {
-            const int st = j % NST, b = j & 1;
-            if (ok) ok = wait(A_TDFULL0 + b, par(j));
-            // UB is free once the previous chunk's TX product has completed
-            if (ok && j >= 1) ok = wait(A_TXFULL0 + ((j - 1) & 1), par(j - 1));
-            tc_fence_after();
-            if (ok) {
-                float x[32];
-                tmem_ld16(taddr(tmem, 32 * quad, Lay::cTD + 32 * b), *reinterpret_cast<float(*)[16]>(x));
-                tmem_ld16(taddr(tmem, 32 * quad, Lay::cTD + 32 * b + 16),
-                          *reinterpret_cast<float(*)[16]>(x + 16));
-                tmem_wait_ld();
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) y[e] = x[8 * p + e];
-                    *reinterpret_cast<uint4 *>(sm + Lay::oUB +
-                                               interleave_mnmajor_off(8 * p, row, Lay::kKGroup)) = pack8(y);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&bars[A_TDEMPTY0 + b]);
-            fence_async_smem();
-            named_bar(1, 64);
-            if (issuer && ok) {
-                if (j >= 2) ok = wait(A_TXEMPTY0 + b, par_prev(j));
-                if (ok) {
-                    tc_fence_after();
-                    const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotKh, kKhMNBlock, 1024, SW_128B);
-                    const uint64_t bd0 = smem_desc(sbase + Lay::oUB, Lay::kKGroup, 128, SW_NONE);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(tmem + Lay::cTX + 32 * b, ad0 + (uint64_t)(kk * 2048 / 16),
-                                bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_mm, kk > 0);
-                    mma_commit(&bars[A_TXFULL0 + b]);
-                    mma_commit(&bars[A_EMPTY0 + st]);
-                }
-            }
-        }
-        if (issuer) {
-            mma_commit(&bars[A_DRAIN_U]);
-            mbar_wait(&bars[A_DRAIN_U], 0, err, 1ull << 28);
-        }
-    } else if (warp == 6 || warp == 7) {
-        // ------------------------------------------------ O rows: R V (TD) + P S (TO) -> o
-        const int quad = warp - 4, r = 32 * quad + lane - 64;
-        bool ok = true;
-        for (int j = 0; j < nch; ++j) {
-            const int b = j & 1;
-            const int64_t t0 = ra + (int64_t)j * C;
-            const int L = chunk_len(j);
-            float xr[32], xp[32];
-            if (ok) ok = wait(A_TDFULL0 + b, par(j));
-            tc_fence_after();
-            if (ok) {
-                tmem_ld16(taddr(tmem, 32 * quad, Lay::cTD + 32 * b), *reinterpret_cast<float(*)[16]>(xr));
-                tmem_ld16(taddr(tmem, 32 * quad, Lay::cTD + 32 * b + 16),
-                          *reinterpret_cast<float(*)[16]>(xr + 16));
-                tmem_wait_ld();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&bars[A_TDEMPTY0 + b]);
-            if (ok) ok = wait(A_TOFULL0 + b, par(j));
-            tc_fence_after();
-            if (ok) {
-                tmem_ld16(taddr(tmem, 32 * quad, Lay::cTO + 32 * b), *reinterpret_cast<float(*)[16]>(xp));
-                tmem_ld16(taddr(tmem, 32 * quad, Lay::cTO + 32 * b + 16),
-                          *reinterpret_cast<float(*)[16]>(xp + 16));
-                tmem_wait_ld();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&bars[A_TOEMPTY0 + b]);
-            if (ok && r < L) {
-                float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * D + j0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    dst[i] = make_float4(xr[4 * i] + xp[4 * i], xr[4 * i + 1] + xp[4 * i + 1],
-                                         xr[4 * i + 2] + xp[4 * i + 2], xr[4 * i + 3] + xp[4 * i + 3]);
-            }
-        }
-    } else if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------ the chain
-        const int quad = warp - 8;
-        const int c = 32 * quad + lane;   // key channel = TMEM lane
-        const bool issuer = (warp == 8 && lane == 0);
-        const uint32_t tS = taddr(tmem + Lay::cTS, 32 * quad, 0);
-        const size_t srow = (((size_t)n * H + h) * D + c) * D + j0;
-        float xa[32];
-        auto load_state = [&](int j, bool &ok) {   // S_j = TS + TX_{j-1} into xa
-            if (ok) ok = wait(A_TSFULL, (uint32_t)((j - 1) & 1)) && wait(A_TXFULL0 + ((j - 1) & 1), par(j - 1));
-            tc_fence_after();
-            if (ok) {
-                float tx[32];
-                tmem_ld16(tS, *reinterpret_cast<float(*)[16]>(xa));
-                tmem_ld16(tS + 16, *reinterpret_cast<float(*)[16]>(xa + 16));
-                const uint32_t tX = taddr(tmem + Lay::cTX + 32 * ((j - 1) & 1), 32 * quad, 0);
-                tmem_ld16(tX, *reinterpret_cast<float(*)[16]>(tx));
-                tmem_ld16(tX + 16, *reinterpret_cast<float(*)[16]>(tx + 16));
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) xa[e] += tx[e];
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&bars[A_TXEMPTY0 + ((j - 1) & 1)]);
-        };
-        if (nch == 0) {
-            if (state_out)
-                for (int i = 0; i < DVS / 4; ++i)
-                    reinterpret_cast<float4 *>(state_out + srow)[i] =
-                        state_in ? reinterpret_cast<const float4 *>(state_in + srow)[i]
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-            bool ok = true;
-#pragma unroll
-            for (int i = 0; i < DVS / 4; ++i) {
-                const float4 f = state_in ? reinterpret_cast<const float4 *>(state_in + srow)[i]
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                xa[4 * i] = f.x; xa[4 * i + 1] = f.y; xa[4 * i + 2] = f.z; xa[4 * i + 3] = f.w;
-            }
-            for (int j = 0; j < nch; ++j) {
-                const int st = j % NST, b = j & 1;
-                if (j >= 1) {
-                    load_state(j, ok);
-                    // intermediate state: S after j C tokens, when that is a multiple of the
-                    // interval strictly inside the sequence
-                    if (ckpt_interval > 0 && ok) {
-                        const int64_t done = (int64_t)j * C;
-                        if (done % ckpt_interval == 0 && done < rb - ra) {
-                            const int64_t e = ck0 + done / ckpt_interval - 1;
-                            if (e < ckpt_capacity) {
-                                float4 *dst = reinterpret_cast<float4 *>(ckpt + (((size_t)e * H + h) * D + c) * D + j0);
-#pragma unroll
-                                for (int i = 0; i < DVS / 4; ++i)
-                                    dst[i] = make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
-                            } else if (lane == 0) {
-                                atomicOr(err, ERR_BAD_INDEX);
-                            }
-                        }
-                    }
-                }
-                // Gamma_j of this channel, from the slot image
-                if (ok) ok = wait(A_FULL0 + st, par(j));
-                const float gam = ok ? reinterpret_cast<const float *>(sm + st * Lay::kStage + kSlotGam)[c] : 0.f;
-                if (ok) {
-                    uint8_t *sbp = sm + Lay::oSB + b * Lay::kSB;
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        const float *x = xa + 16 * p;
-                        float y0[8], y1[8], z[16];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            y0[e] = x[e];
-                            y1[e] = x[8 + e];
-                        }
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) z[e] = x[e] * gam;
-                        tmem_st16(tS + 16 * p, z);
-                        *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p, c, Lay::kKGroup)) = pack8(y0);
-                        *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p + 8, c, Lay::kKGroup)) = pack8(y1);
-                    }
-                    tmem_wait_st();
-                }
-                fence_async_smem();
-                tc_fence_before();
-                named_bar(2, 128);
-                if (issuer && ok) {
-                    ok = wait(A_AFULL0 + b, par(j));
-                    if (ok) {
-                        tc_fence_after();
-                        const uint64_t bs0 = smem_desc(sbase + Lay::oSB + b * Lay::kSB, Lay::kKGroup, 128, SW_NONE);
-                        {   // TS += A'_j S_j  (the chain)
-                            const uint64_t ad0 = smem_desc(sbase + Lay::oAB + b * Lay::kAB, 16, 1024, SW_128B);
-#pragma unroll
-                            for (int kk = 0; kk < 8; ++kk)
-                                mma_f16(tmem + Lay::cTS, ad0 + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) / 16),
-                                        bs0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, 1);
-                            mma_commit(&bars[A_TSFULL]);
-                            mma_commit(&bars[A_AEMPTY0 + b]);
-                        }
-                        if (j >= 2) ok = wait(A_TOEMPTY0 + b, par_prev(j));
-                        if (ok) {   // TO_j = [-W; P]_j S_j  (rows 64..127: P_j S_j)
-                            tc_fence_after();
-                            const uint64_t ad0 = smem_desc(stage_addr(st) + kSlotWP, 16, 1024, SW_128B);
-#pragma unroll
-                            for (int kk = 0; kk < 8; ++kk)
-                                mma_f16(tmem + Lay::cTO + 32 * b,
-                                        ad0 + (uint64_t)(((kk >> 2) * kWPKBlock + (kk & 3) * 32) / 16),
-                                        bs0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, kk > 0);
-                            mma_commit(&bars[A_TOFULL0 + b]);
-                            mma_commit(&bars[A_EMPTY0 + st]);
-                        }
-                    }
-                }
-            }
-            // the final state S_nch = TS + TX_{nch-1}
-            load_state(nch, ok);
-            if (ok && state_out && !*abort_flag) {
-#pragma unroll
-                for (int i = 0; i < DVS / 4; ++i)
-                    reinterpret_cast<float4 *>(state_out + srow)[i] =
-                        make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
-            }
-            if (issuer) {
-                mma_commit(&bars[A_DRAIN_S]);
-                mbar_wait(&bars[A_DRAIN_S], 0, err, 1ull << 28);
-            }
-        }
-    } else {
-        // ------------------------------------------------ A' builders: TA_j -> fp16 AB_j
-        const int quad = warp - 12;
-        const int c = 32 * quad + lane;   // row of A' = TMEM lane
-        bool ok = true;
-        for (int j = 0; j < nch; ++j) {
-            const int b = j & 1;
-            if (ok) ok = wait(A_TAFULL0 + b, par(j));
-            if (ok && j >= 2) ok = wait(A_AEMPTY0 + b, par_prev(j));
-            tc_fence_after();
-            if (ok) {
-                uint8_t *ab = sm + Lay::oAB + b * Lay::kAB;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float x[64];
-#pragma unroll
-                    for (int p = 0; p < 4; ++p)
-                        tmem_ld16(taddr(tmem, 32 * quad, Lay::cTA + 128 * b + 64 * hh + 16 * p),
-                                  *reinterpret_cast<float(*)[16]>(x + 16 * p));
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        float y[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = x[8 * p + e];
-                        *reinterpret_cast<uint4 *>(ab + sw128_kmajor_off(c, 64 * hh + 8 * p, 16384)) = pack8(y);
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&bars[A_TAEMPTY0 + b]);
-            fence_async_smem();
-            named_bar(4, 128);
-            if (warp == 12 && lane == 0 && ok) mbar_arrive(&bars[A_AFULL0 + b]);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-}
-
 }  // namespace tc
 
 // ======================================================================
@@ -1904,27 +1384,6 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
                                          a.T, a.N, a.H, (const uint8_t *)a.workspace,
                                          (float *)a.o, a.state_out, a.ckpt_interval, a.ckpt,
                                          a.ckpt_capacity, a.err, a.epoch);
-    e = cudaGetLastError();
-    Profiler::mark(st);
-    return e;
-}
-
-static cudaError_t launch_state_pass_a(const PrefillArgs &a, cudaStream_t st) {
-    using Lay = tc::B1Layout;
-    auto kern = tc::state_pass_a_kernel;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Lay::kBytes);
-    if (e != cudaSuccess) return e;
-    CUtensorMap tv;
-    const int64_t rows = (int64_t)a.B * a.T;
-    if (rows > 0 && !make_rows_heads_tmap(&tv, a.v, rows, a.H, tc::D, Lay::DVS, tc::C,
-                                          CU_TENSOR_MAP_SWIZZLE_64B))
-        return cudaErrorInvalidValue;
-    if (rows == 0) memset(&tv, 0, sizeof(tv));
-    const int grid = a.N * a.H * (tc::D / Lay::DVS);
-    kern<<<grid, 512, Lay::kBytes, st>>>(tv, a.state_in, a.cu_seqlens, a.T, a.N, a.H,
-                                         (const uint8_t *)a.workspace, (float *)a.o, a.state_out,
-                                         a.ckpt_interval, a.ckpt, a.ckpt_capacity, a.err, a.epoch);
     e = cudaGetLastError();
     Profiler::mark(st);
     return e;
@@ -1973,7 +1432,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
     Profiler::mark(st);
     // dv-slices: enough CTAs to cover the SMs when there are few (sequence, head) units
     const int64_t units = (int64_t)a.N * a.H;
-    if (units <= 74) return launch_state_pass_a(a, st);
+    if (units <= 74) return launch_state_pass<32>(a, st);
     if (units <= 148) return launch_state_pass<64>(a, st);
     return launch_state_pass<128>(a, st);
 }

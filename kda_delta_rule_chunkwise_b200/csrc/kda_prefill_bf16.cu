@@ -244,14 +244,14 @@ constexpr uint32_t A_AK = A_OPS;              // fp32 [64][64] Akk, then X in pl
 constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64         8 KiB
 constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64     16 KiB
 constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128          16 KiB
-constexpr uint32_t A_Y = A_OPS + 57344;       // tf32 64x64 operand of the UT solve          16 KiB
+constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 solve scratch (32 x 32)               4 KiB
 // next item's rows, loaded by TMA once D1 has completed (all of the above is dead by then);
 // each tile is the TMA box layout of stage_off(): two 64-channel blocks of 64 rows x 128 B
 constexpr uint32_t A_QST = A_OPS + 16384;     // bf16 q [64][128]                            16 KiB
 constexpr uint32_t A_KST = A_OPS + 32768;     // bf16 k                                      16 KiB
 constexpr uint32_t A_GST = A_OPS + 49152;     // bf16 g                                      16 KiB
 constexpr uint32_t A_SMEM = A_OPS + 2 * A_RBUF + 1024;   // + alignment slack (= 112640)
-static_assert(A_Y + 16384 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
+static_assert(A_Y + 4096 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
 static_assert(A_QST >= A_AK + 16384 && A_GST + 16384 <= A_OPS + 2 * A_RBUF, "staging area");
 static_assert(3 * 128 * 4 + 128 * 4 <= 16384, "A0 scratch (tot, G_L) must not reach the staging area");
 static_assert(A_OPS % 1024 == 0 && A_RBUF % 1024 == 0 && A_AQ % 1024 == 0 && A_TR % 1024 == 0 &&
@@ -329,6 +329,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float *tot = reinterpret_cast<float *>(sm + A_OPS);              // [3][128] half sums
     float *GLv = tot + 3 * 128;                                       // [128] G_L
     float *AK = reinterpret_cast<float *>(sm + A_AK);
+    float *Yb = reinterpret_cast<float *>(sm + A_Y);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int32_t *chunk_off = reinterpret_cast<const int32_t *>(ws);
@@ -653,40 +654,16 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
 
 
-    // ---- A3: X = (I + Akk)^-1 on the tensor cores, T = X Diag(beta).
-    // With Xd the inverse of the block diagonal of I + Akk (its four unit-lower 16x16
-    // diagonal blocks, by fp32 forward substitution) and E the strictly block-lower
-    // part of Akk, I + Akk = Xd^-1 (I + N) with N = Xd E.  N is strictly block-lower
-    // over four blocks, so N^4 = 0 and
-    //     X = (I + N)^-1 Xd = (I - N)(I + N^2) Xd:
-    //     N = Xd E,  N2 = N N,  P1 = Xd + N2 Xd,  X = P1 - N P1,
-    // four dependent 64x64x64 tf32 products (M=64: accumulator rows 16q + l in TMEM
-    // lanes 32q + l, l < 16).  Every operand is a 64x64 tf32 tile in the K-major
-    // 128-byte-swizzled layout, which is also the MN-major layout of its transpose
-    // role, so each matrix is stored once and serves as A (K-major) or B (MN-major).
-    // The diagonal blocks of P1 and X are Xd's exact fp32 values (N2 Xd and N P1 are
-    // strictly block-lower).  Buffers: U1 = A_TR (Xd, then P1), U2 = A_Y (E, then N),
-    // U3 = A_AK (N2, once Akk has been consumed).
+    // ---- A3: X = (I + Akk)^-1 in place over AK (fp32), by 2x2 block merges:
+    //   inv([[L11, 0], [L21, L22]]) = [[X11, 0], [-X22 (L21 X11), X22]]
+    // 16x16 diagonal blocks by forward substitution, then two merges 16 -> 32
+    // (in parallel), then one merge 32 -> 64.  The strictly upper part of AK is
+    // zero throughout.  (Every __syncthreads below is reached by all threads.)
     {
-        constexpr uint32_t U1 = A_TR, U2 = A_Y, U3 = A_AK;
-        auto ut = [](int i, int j) { return sw128_kmajor_off32((uint32_t)i, (uint32_t)j, 8192u); };
-        // zero Xd's off-diagonal blocks (U1) and copy E (U2), tf32, one row quarter per thread
+        float x[16];
+        const int a = tid >> 4, j = tid & 15, o = 16 * a;
         if (ok && tid >= 128) reinterpret_cast<float *>(slot + kSlotGam)[tid - 128] = EL[tid - 128];
-        if (ok) {
-            const int i = tid >> 2, j0 = 16 * (tid & 3);
-            const bool diag = (i >> 4) == (j0 >> 4);
-#pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {
-                const int j = j0 + 4 * cq;
-                const float4 e = diag ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(AK + i * 64 + j);
-                *reinterpret_cast<float4 *>(sm + U2 + ut(i, j)) = tf4(e);
-                if (!diag) *reinterpret_cast<float4 *>(sm + U1 + ut(i, j)) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-        // the diagonal blocks: column j of inv(I + Akk_aa) by forward substitution (exact fp32)
         if (ok && tid < 64) {
-            const int a = tid >> 4, j = tid & 15, o = 16 * a;
-            float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 float acc = (i == j) ? 1.f : 0.f;
@@ -694,88 +671,108 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int m = 0; m < i; ++m) acc = fmaf(-AK[(o + i) * 64 + o + m], x[m], acc);
                 x[i] = acc;
             }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + U1 + ut(o + i, o + j)) = x[i];
         }
-        fence_async_smem();
-        tc_fence_before();
         __syncthreads();
-        tc_fence_after();
-        // one 64x64x64 tf32 product D = A B into TMEM columns dcol, then its rows
-        // (lane < 16 of each warp: row m, columns 32 uh .. 32 uh + 31) in registers
-        const int uq = warp & 3, uh = warp >> 2, um = 16 * uq + (lane & 15);
-        uint32_t ucommit = 0;
-        auto ut_mma = [&](uint32_t abuf, uint32_t bbuf, uint32_t dcol, float (&d)[32]) {
-            if (ok && tid == 0) {
-                const uint32_t id = idesc(FMT_TF32, 64, 64, 0, 1);
+        if (ok && tid < 64) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = smem_desc(sbase + abuf + (kk >> 2) * 8192 + (kk & 3) * 32, 16,
-                                                  1024, SW_128B);
-                    const uint64_t bd = smem_desc(sbase + bbuf + kk * 1024, 8192, 1024, SW_128B);
-                    mma_tf32(tmem + dcol, ad, bd, id, kk > 0);
-                }
-                mma_commit(&bars[7]);
-            }
-            if (ok) ok = mbar_wait_abortable(&bars[7], ucommit & 1u, err, epoch, abort_flag);
-            ++ucommit;
-            tc_fence_after();
-            if (ok) {
-                tmem_ld16(taddr(tmem, 32 * uq, dcol + 32 * uh), *reinterpret_cast<float(*)[16]>(d));
-                tmem_ld16(taddr(tmem, 32 * uq, dcol + 32 * uh + 16), *reinterpret_cast<float(*)[16]>(d + 16));
-                tmem_wait_ld();
-            }
-        };
-        // row um, columns 32 uh .. + 31, of a tf32 operand tile
-        auto ut_store = [&](uint32_t buf, const float (&v)[32]) {
-            if (ok && lane < 16) {
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
-                    *reinterpret_cast<float4 *>(sm + buf + ut(um, 32 * uh + 4 * c4)) =
-                        tf4(make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]));
-            }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-        };
-        float d[32];
-        ut_mma(U1, U2, 0, d);        // N = Xd E
-        ut_store(U2, d);
-        ut_mma(U2, U2, 64, d);       // N2 = N N
-        ut_store(U3, d);
-        ut_mma(U3, U1, 0, d);        // N2 Xd
-        // P1 = Xd + N2 Xd (Xd exact from U1): rounded into U1 as the next B operand,
-        // exact into AK (row-major fp32; N2 in U3 = AK is consumed by now)
-        if (ok && lane < 16) {
-#pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4) {
-                const int col = 32 * uh + 4 * c4;
-                const float4 xd = ld4(reinterpret_cast<const float *>(sm + U1 + ut(um, col)));
-                d[4 * c4] += xd.x;
-                d[4 * c4 + 1] += xd.y;
-                d[4 * c4 + 2] += xd.z;
-                d[4 * c4 + 3] += xd.w;
-                *reinterpret_cast<float4 *>(AK + um * 64 + col) =
-                    make_float4(d[4 * c4], d[4 * c4 + 1], d[4 * c4 + 2], d[4 * c4 + 3]);
-            }
+            for (int i = 0; i < 16; ++i) AK[(o + i) * 64 + o + j] = x[i];
         }
-        ut_store(U1, d);
-        ut_mma(U2, U1, 64, d);       // N P1
-        // X = P1 - N P1 (lower triangular), T = X Diag(beta) into rows 0..63 of [T; R]
-        // (fp16, K-major SW128; U1 is free once N P1 has completed)
-        if (ok && lane < 16) {
+    }
+    __syncthreads();
+    // merge 16 -> 32 for diagonal pairs p = 0, 1 (rows/cols 32p .. 32p+31):
+    //   Y = A_{2p+1,2p} X_{2p,2p};  X_{2p+1,2p} = -X_{2p+1,2p+1} Y
+    // thread: pair pr, column j, rows i and i + 8 (row operands as float4, the
+    // column operand shared by both rows)
+    {
+        const int pr = tid >> 7, j = tid & 15, i = (tid >> 4) & 7;
+        const int o = 32 * pr;
+        const float *r0 = AK + (o + 16 + i) * 64 + o, *r1 = r0 + 8 * 64;
+        if (ok) {
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                const int c0 = 32 * uh + 8 * ch;
-                const float4 pa = ld4(AK + um * 64 + c0), pb = ld4(AK + um * 64 + c0 + 4);
-                const float pv[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-                float y[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    y[e] = c0 + e <= um ? (pv[e] - d[8 * ch + e]) * bs[c0 + e] : 0.f;
-                *reinterpret_cast<uint4 *>(sm + A_TR + sw128_kmajor_off(um, c0, 0)) = pack8(y);
+            for (int t4 = 0; t4 < 4; ++t4) {
+                const float4 a0 = ld4(r0 + 4 * t4), a1 = ld4(r1 + 4 * t4);
+                const float x0 = AK[(o + 4 * t4) * 64 + o + j], x1 = AK[(o + 4 * t4 + 1) * 64 + o + j];
+                const float x2 = AK[(o + 4 * t4 + 2) * 64 + o + j], x3 = AK[(o + 4 * t4 + 3) * 64 + o + j];
+                acc0 = fmaf(a0.x, x0, fmaf(a0.y, x1, fmaf(a0.z, x2, fmaf(a0.w, x3, acc0))));
+                acc1 = fmaf(a1.x, x0, fmaf(a1.y, x1, fmaf(a1.z, x2, fmaf(a1.w, x3, acc1))));
             }
+            Yb[pr * 256 + i * 16 + j] = acc0;
+            Yb[pr * 256 + (i + 8) * 16 + j] = acc1;
+        }
+        __syncthreads();
+        if (ok) {
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int t4 = 0; t4 < 4; ++t4) {
+                const float4 a0 = ld4(r0 + 16 + 4 * t4), a1 = ld4(r1 + 16 + 4 * t4);
+                const float *yc = Yb + pr * 256 + 64 * t4 + j;
+                const float y0 = yc[0], y1 = yc[16], y2 = yc[32], y3 = yc[48];
+                acc0 = fmaf(a0.x, y0, fmaf(a0.y, y1, fmaf(a0.z, y2, fmaf(a0.w, y3, acc0))));
+                acc1 = fmaf(a1.x, y0, fmaf(a1.y, y1, fmaf(a1.z, y2, fmaf(a1.w, y3, acc1))));
+            }
+            AK[(o + 16 + i) * 64 + o + j] = -acc0;
+            AK[(o + 24 + i) * 64 + o + j] = -acc1;
+        }
+        __syncthreads();
+    }
+    // merge 32 -> 64:  Z = A21 X11 (32x32);  X21 = -X22 Z
+    // thread (i0 = warp, j = lane) computes rows i0 + 8q, q = 0..3, of column j;
+    // the row operands are warp-uniform (broadcast float4 loads), the zero upper
+    // triangles make the fixed trip counts exact
+    {
+        const int j = lane, i0 = warp;
+        if (ok) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4) {
+                float xv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) xv[u] = AK[(4 * t4 + u) * 64 + j];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const float4 av = ld4(AK + (32 + i0 + 8 * qq) * 64 + 4 * t4);
+                    acc[qq] = fmaf(av.x, xv[0], fmaf(av.y, xv[1], fmaf(av.z, xv[2], fmaf(av.w, xv[3], acc[qq]))));
+                }
+            }
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) Yb[(i0 + 8 * qq) * 32 + j] = acc[qq];
+        }
+        __syncthreads();
+        if (ok) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4) {
+                float zv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) zv[u] = Yb[(4 * t4 + u) * 32 + j];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    // X22 is lower triangular: row i0 + 8 qq has no terms past column
+                    // i0 + 8 qq (a warp-uniform bound, so whole blocks are skipped)
+                    if (t4 <= (i0 >> 2) + 2 * qq) {
+                        const float4 av = ld4(AK + (32 + i0 + 8 * qq) * 64 + 32 + 4 * t4);
+                        acc[qq] = fmaf(av.x, zv[0], fmaf(av.y, zv[1], fmaf(av.z, zv[2], fmaf(av.w, zv[3], acc[qq]))));
+                    }
+                }
+            }
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) AK[(32 + i0 + 8 * qq) * 64 + j] = -acc[qq];
+        }
+        __syncthreads();
+    }
+    // T = X Diag(beta) into rows 0..63 of [T; R] (fp16, K-major SW128)
+    if (ok) {
+        for (int task = tid; task < 64 * 8; task += 256) {
+            const int r = task >> 3, ch = task & 7;
+            const float4 xa = ld4(AK + r * 64 + ch * 8), xb = ld4(AK + r * 64 + ch * 8 + 4);
+            const float4 ba = ld4(bs + ch * 8), bb = ld4(bs + ch * 8 + 4);
+            const float xv[8] = {xa.x * ba.x, xa.y * ba.y, xa.z * ba.z, xa.w * ba.w,
+                                 xb.x * bb.x, xb.y * bb.y, xb.z * bb.z, xb.w * bb.w};
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = (ch * 8 + e <= r) ? xv[e] : 0.f;
+            *reinterpret_cast<uint4 *>(sm + A_TR + sw128_kmajor_off(r, ch * 8, 0)) = pack8(x);
         }
     }
     fence_async_smem();

@@ -54,29 +54,37 @@ DECODE_BYTES_PER_UNIT = 2 * STATE_BYTES + 4 * 128 * 2 + 2 + O_BYTES_ALGO   # 132
 FLOPS_PER_TOKEN_HEAD = 139264                                 # algorithmic MMA flops (causal halves once)
 
 # Per-kernel figures from one ncu capture (profiles/), valid only for the kernel
-# source they were taken on (sha256 prefix of that .cu file; a changed source
-# reports null): DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per
-# (chunk, head) unit, or per launch for decode, and the tensor-pipe activity in
-# percent (sm__pipe_tensor_cycles_active over the kernel), or None.
+# source they were taken on: the sha256 prefix of the kernel's .cu file followed
+# by the headers it includes (a changed source reports null).  DRAM bytes
+# (dram__bytes_read.sum + dram__bytes_write.sum) per (chunk, head) unit, or per
+# launch for decode, and the tensor-pipe activity in percent
+# (sm__pipe_tensor_cycles_active over the kernel), or None.
+PREFILL_SOURCES = ("kda_prefill_bf16.cu", "kda_common.cuh", "sm100.cuh", "kda_tma.h", "kda_launch.h")
 NCU = {
-    "intra_chunk_kernel": ("kda_prefill_bf16.cu", "5816df7998ae0054", (202408704 + 216729088) / 4096, 8.2),
-    "state_pass_kernel": ("kda_prefill_bf16.cu", "5816df7998ae0054", (339792384 + 109159424) / 4096, 8.6),
-    "decode_kernel": ("kda_decode.cu", "4f1c8c21d6ac8934", 545290752 + 482616576, None),
+    "intra_chunk_kernel": (PREFILL_SOURCES, "pending", (202496000 + 216710912) / 4096, 8.2),
+    "state_pass_kernel": (PREFILL_SOURCES, "pending", (339790080 + 109562112) / 4096, 9.0),
+    "decode_kernel": (("kda_decode.cu",), "4f1c8c21d6ac8934", 545290752 + 482616576, None),
 }
 
 
-def _ncu_entry(kernel: str):
+def source_digest(files) -> str:
     import hashlib
+    h = hashlib.sha256()
+    for fname in files:
+        with open(os.path.join(ROOT, "kda_delta_rule_chunkwise_b200", "csrc", fname), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_entry(kernel: str):
     ent = NCU.get(kernel)
     if ent is None:
         return None
-    fname, digest = ent[0], ent[1]
-    path = os.path.join(ROOT, "kda_delta_rule_chunkwise_b200", "csrc", fname)
     try:
-        cur = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+        cur = source_digest(ent[0])
     except OSError:
         return None
-    return ent if cur == digest else None
+    return ent if cur == ent[1] else None
 
 
 def ncu_traffic(kernel: str, units: float):

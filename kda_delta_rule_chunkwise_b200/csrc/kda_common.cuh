@@ -34,6 +34,9 @@ __device__ __forceinline__ void record_timeout(uint32_t *err, uint32_t epoch) {
 // these kernels last microseconds; anything past this bound means a missing
 // arrival, and the waiting thread gives up instead of hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+// A wait longer than this is not a normal hand-off; only then do waiters look at
+// the other CTAs' abort word in device memory.
+constexpr uint64_t kSlowWaitNs = 50000ull;          // 50 us
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
@@ -125,11 +128,17 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t pari
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (gepoch && *gepoch == epoch) {   // a CTA of this launch gave up: do not wait out the limit too
-            *abort = 1u;
-            return false;
+        // The device-memory epoch word is read only once a wait has lasted longer
+        // than any wait of a healthy launch (tens of microseconds): a global load
+        // in every poll would delay noticing a completed phase by its latency.
+        const uint64_t dt = globaltimer_ns() - t0;
+        if (dt > kSlowWaitNs) {
+            if (gepoch && *gepoch == epoch) {   // a CTA of this launch gave up: do not wait out the limit too
+                *abort = 1u;
+                return false;
+            }
+            if (dt > limit_ns) break;
         }
-        if (globaltimer_ns() - t0 > limit_ns) break;
     }
     record_timeout(err, epoch);
     *abort = 1u;

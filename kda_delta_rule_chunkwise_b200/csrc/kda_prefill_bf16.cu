@@ -245,15 +245,21 @@ constexpr uint32_t A_AQ = A_OPS + 16384;      // fp16 Aqk, MN-major SW128 64x64 
 constexpr uint32_t A_TR = A_OPS + 24576;      // fp16 [T; R], K-major SW128 128x64     16 KiB
 constexpr uint32_t A_KT = A_OPS + 40960;      // fp16 K*Gamma, MN-major SW128          16 KiB
 constexpr uint32_t A_Y = A_OPS + 57344;       // fp32 solve scratch (32 x 32)               4 KiB
-// next item's rows, loaded by TMA once D1 has completed (all of the above is dead by then);
-// each tile is the TMA box layout of stage_off(): two 64-channel blocks of 64 rows x 128 B
-constexpr uint32_t A_QST = A_OPS + 16384;     // bf16 q [64][128]                            16 KiB
-constexpr uint32_t A_KST = A_OPS + 32768;     // bf16 k                                      16 KiB
-constexpr uint32_t A_GST = A_OPS + 49152;     // bf16 g                                      16 KiB
+// next item's rows, loaded by TMA as soon as D1 has completed: the regions of AK (dead
+// after the solve), K*Gamma (dead after D1) and the solve scratch with the tail; none
+// overlaps [T; R], which a bulk store may still be reading.  Each tile is the TMA box
+// layout of stage_off(): two 64-channel blocks of 64 rows x 128 B.
+constexpr uint32_t A_QST = A_AK;              // bf16 q [64][128]                            16 KiB
+constexpr uint32_t A_KST = A_KT;              // bf16 k                                      16 KiB
+constexpr uint32_t A_GST = A_Y;               // bf16 g                                      16 KiB
+// A0 scratch (block sums, G_L), in the Aqk region (free until A2)
+constexpr uint32_t A_A0S = A_AQ;
 constexpr uint32_t A_SMEM = A_OPS + 2 * A_RBUF + 1024;   // + alignment slack (= 112640)
 static_assert(A_Y + 4096 <= A_OPS + 2 * A_RBUF, "phase A post-MMA region overflows");
-static_assert(A_QST >= A_AK + 16384 && A_GST + 16384 <= A_OPS + 2 * A_RBUF, "staging area");
-static_assert(3 * 128 * 4 + 128 * 4 <= 16384, "A0 scratch (tot, G_L) must not reach the staging area");
+static_assert(A_GST + 16384 <= A_OPS + 2 * A_RBUF, "staging area");
+static_assert((A_QST >= A_TR + 16384 || A_QST + 16384 <= A_TR) && (A_KST >= A_TR + 16384 || A_KST + 16384 <= A_TR) &&
+              (A_GST >= A_TR + 16384 || A_GST + 16384 <= A_TR), "staging must not overlap [T; R]");
+static_assert(3 * 128 * 4 + 128 * 4 <= 8192, "A0 scratch (tot, G_L) fits the Aqk region");
 static_assert(A_OPS % 1024 == 0 && A_RBUF % 1024 == 0 && A_AQ % 1024 == 0 && A_TR % 1024 == 0 &&
               A_KT % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // E1 is stored [64][128] fp32 with its 16-byte pieces (4 channels) permuted per
@@ -326,7 +332,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + A_MISC + A_M_TMEM);
     volatile uint32_t *abort_flag = tmem_ptr + 1;
     // used only inside A0, before any operand round: parked in the operand region
-    float *tot = reinterpret_cast<float *>(sm + A_OPS);              // [3][128] half sums
+    float *tot = reinterpret_cast<float *>(sm + A_A0S);              // [3][128] half sums
     float *GLv = tot + 3 * 128;                                       // [128] G_L
     float *AK = reinterpret_cast<float *>(sm + A_AK);
     float *Yb = reinterpret_cast<float *>(sm + A_Y);
@@ -371,7 +377,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // beta into a register.  Rows past the chunk's end are zeroed once the tiles
     // have landed (the boxes read the next rows of the tensor there, or zeros past
     // its end).
-    float bnext = 0.f;
+    __nv_bfloat16 bnext = __float2bfloat16(0.f);   // raw: converted where it is used
     int loads_issued = 0, items_done = 0;   // tile loads issued / consumed by this CTA
     auto prefetch = [&](int64_t item) {
         int64_t t0n;
@@ -379,6 +385,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         locate(item, t0n, Ln);
         const int hn = (int)(item % H);
         if (tid == 0) {
+            fence_async_smem();   // earlier generic writes to the staging regions come first
             mbar_arrive_expect_tx(&bars[6], 3 * 16384);
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk) {
@@ -388,7 +395,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
         }
         ++loads_issued;
-        bnext = (tid < Ln) ? __bfloat162float(beta[(size_t)(t0n + (tid < 64 ? tid : 0)) * H + hn]) : 0.f;
+        bnext = (tid < Ln) ? beta[(size_t)(t0n + (tid < 64 ? tid : 0)) * H + hn] : __float2bfloat16(0.f);
     };
 
     if (warp == 0) {
@@ -422,8 +429,8 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (landed && L < C) {
         for (int task = tid; task < (C - L) * 3 * 2; task += 256) {
             const int r = L + task / 6, which = task % 6;
-            uint4 *line = reinterpret_cast<uint4 *>(sm + A_QST + (which >> 1) * 16384 +
-                                                     (which & 1) * 8192 + r * 128);
+            const uint32_t base = (which >> 1) == 0 ? A_QST : ((which >> 1) == 1 ? A_KST : A_GST);
+            uint4 *line = reinterpret_cast<uint4 *>(sm + base + (which & 1) * 8192 + r * 128);
 #pragma unroll
             for (int i = 0; i < 8; ++i) line[i] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -445,7 +452,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             p[i] = fmaxf(x, -5.f);   // rows past the end are staged as zero
         }
     }
-    if (tid < 64) bs[tid] = bnext;
+    if (tid < 64) bs[tid] = __bfloat162float(bnext);
     __syncthreads();
     // the g staging is free now: it holds 1 / |q_r| and 1 / |k_r| when q, k are to be
     // normalised here (two threads per row; a zero row stays zero)
@@ -530,6 +537,9 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             qv[rd][it] = *reinterpret_cast<const uint2 *>(sm + A_QST + sw);
             kv[rd][it] = *reinterpret_cast<const uint2 *>(sm + A_KST + sw);
         }
+    // the previous item's bulk store of [T; R] has read its source before the
+    // operand rounds below overwrite that region
+    if (tid == 0) bulk_wait_read();
     __syncthreads();
 
     // ---- A1: Akk / Aqk on tensor cores (tf32), four double-buffered rounds of 32 channels.
@@ -835,10 +845,9 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (ok) ok = mbar_wait_abortable(&bars[5], ph, err, epoch, abort_flag);
     tc_fence_after();
-    // the operand tiles are free once D1 has completed and the bulk store has
-    // read [T; R]: the next item's rows go out now
-    if (tid == 0) bulk_wait_read();
-    __syncthreads();
+    // the staging regions are free once D1 has completed: the next item's rows go
+    // out now (the bulk store of [T; R] is waited for before the next item's
+    // operand rounds overwrite it)
     if (ok && (int64_t)item + gridDim.x < n_items) prefetch(item + gridDim.x);
 
     // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = Q*Gamma - R (K*Gamma), in two

@@ -98,3 +98,87 @@ def backward(q, k, v, g, beta, S0, dout, dS_final, C=64):
         for acc, x in zip(grads, gr):
             acc[sl] = x
     return (*grads, dS)
+
+
+# ---------------------------------------------------------------- the WY-slot form
+# The same adjoint split the way a chunk-parallel implementation on top of the
+# forward's workspace would run it: the chunk-to-chunk chain needs only the
+# forward's per-chunk factors (T, R, W, P, Khat, Gamma_L), and the gradients of
+# those factors are then pulled back to q, k, g, beta without the state.
+
+def wy_factors(q, k, g, beta):
+    L = q.shape[0]
+    G = np.cumsum(np.maximum(g, -5.0), 0)
+    gam = np.exp(G)
+    E = np.exp(G[:, None, :] - G[None, :, :])
+    M = np.tril(np.einsum("rc,sc,rsc->rs", k, k, E), -1)
+    Aqk = np.tril(np.einsum("rc,sc,rsc->rs", q, k, E))
+    X = np.linalg.inv(np.eye(L) + beta[:, None] * M)
+    T = X * beta[None, :]
+    Kt, Qt = k * gam, q * gam
+    R = Aqk @ T
+    return dict(gam=gam, gam_l=np.exp(G[L - 1]), E=E, M=M, Aqk=Aqk, X=X, T=T, Kt=Kt, Qt=Qt,
+                Kh=k * np.exp(G[L - 1][None, :] - G), R=R, W=T @ Kt, P=Qt - R @ Kt)
+
+
+def wy_state_part(f, v, S, dO, dS_end):
+    """The chain step and the factor gradients: only f's T, R, W, P, Khat, Gamma_L,
+    the chunk's V, its start state S, dO and dS' are used."""
+    U = f["T"] @ v - f["W"] @ S
+    dU = f["Kh"] @ dS_end
+    dS = f["gam_l"][:, None] * dS_end + f["P"].T @ dO - f["W"].T @ dU
+    dV = f["T"].T @ dU + f["R"].T @ dO
+    grads = dict(dT=dU @ v.T, dR=dO @ v.T, dW=-dU @ S.T, dP=dO @ S.T, dKh=U @ dS_end.T,
+                 dGl=np.sum(dS_end * S, axis=1))
+    return dS, dV, grads
+
+
+def wy_input_part(q, k, g, beta, f, gr):
+    """Pull the factor gradients back to q, k, g, beta (no state involved)."""
+    L = q.shape[0]
+    E, gam, gam_l = f["E"], f["gam"], f["gam_l"]
+    dP = gr["dP"]
+    dR = gr["dR"] - dP @ f["Kt"].T
+    dKt = f["T"].T @ gr["dW"] - f["R"].T @ dP
+    dT = gr["dT"] + f["Aqk"].T @ dR + gr["dW"] @ f["Kt"].T
+    dAqk = np.tril(dR @ f["T"].T)
+    dbeta = np.sum(f["X"] * dT, axis=0)
+    dAkk = np.tril(-f["X"].T @ (dT * beta[None, :]) @ f["X"].T, -1)
+    dbeta = dbeta + np.sum(dAkk * f["M"], axis=1)
+    dM = beta[:, None] * dAkk
+
+    def decayed(a, b, dF):
+        return (np.einsum("rs,sc,rsc->rc", dF, b, E), np.einsum("rs,rc,rsc->sc", dF, a, E))
+
+    da_q, db_qk = decayed(q, k, dAqk)
+    da_k, db_kk = decayed(k, k, dM)
+    dKh = gr["dKh"]
+    dq = dP * gam + da_q
+    dk = dKt * gam + dKh * (gam_l[None, :] / gam) + db_qk + da_k + db_kk
+    dG = (f["Qt"] * dP + f["Kt"] * dKt - f["Kh"] * dKh + q * da_q - k * db_qk + k * da_k
+          - k * db_kk)
+    dG[L - 1] += np.sum(f["Kh"] * dKh, axis=0) + gam_l * gr["dGl"]
+    dg = np.cumsum(dG[::-1], axis=0)[::-1] * (g >= -5.0)
+    return dq, dk, dg, dbeta
+
+
+def wy_backward(q, k, v, g, beta, S0, dout, dS_final, C=64):
+    """As backward(), through the WY-slot split."""
+    T_len = q.shape[0]
+    starts = list(range(0, T_len, C))
+    states, facs = [np.array(S0, np.float64)], []
+    for t0 in starts:
+        sl = slice(t0, min(T_len, t0 + C))
+        f = wy_factors(q[sl], k[sl], g[sl], beta[sl])
+        facs.append(f)
+        U = f["T"] @ v[sl] - f["W"] @ states[-1]
+        states.append(f["gam_l"][:, None] * states[-1] + f["Kh"].T @ U)
+    dq, dk, dv, dg, db = (np.zeros_like(x, dtype=np.float64) for x in (q, k, v, g, beta))
+    dS = np.array(dS_final, np.float64)
+    for ci in reversed(range(len(starts))):
+        sl = slice(starts[ci], min(T_len, starts[ci] + C))
+        dS_prev, dv[sl], gr = wy_state_part(facs[ci], v[sl], states[ci], dout[sl], dS)
+        dq[sl], dk[sl], dg[sl], db[sl] = wy_input_part(q[sl], k[sl], g[sl], beta[sl], facs[ci], gr)
+        dS = dS_prev
+    return dq, dk, dv, dg, db, dS
+

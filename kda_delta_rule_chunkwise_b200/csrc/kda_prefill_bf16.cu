@@ -76,10 +76,13 @@ constexpr uint32_t kKhMNBlock = 8192;    // bytes between the two 64-channel MN-
 // in chunk_off[N]), int32 bound[N+1] (the row offsets actually used:
 // cu_seqlens clamped to [0, T] and made non-decreasing by a running maximum,
 // so that sequences never overlap and the chunk total never exceeds the
-// workspace bound) and int32 ckpt_off[N+1] (first intermediate-state entry of
-// each sequence, total in ckpt_off[N]).  Then the slots, 1024-aligned.
+// workspace bound), int32 ckpt_off[N+1] (first intermediate-state entry of
+// each sequence, total in ckpt_off[N]) and int32 order[N+1] (the sequences by
+// decreasing chunk count, so that the state pass starts the longest chains
+// first; identity order past kOrderMaxN sequences).  Then the slots, 1024-aligned.
+constexpr int kOrderMaxN = 8192;
 __host__ __device__ inline uint32_t header_bytes(int N) {
-    return (uint32_t)(((size_t)(N + 1) * 12 + 1023) & ~(size_t)1023);
+    return (uint32_t)(((size_t)(N + 1) * 16 + 1023) & ~(size_t)1023);
 }
 
 // ======================================================================
@@ -152,6 +155,22 @@ chunk_table_kernel(const int32_t *__restrict__ cu, int64_t T, int N, int64_t ckp
     };
     exclusive_sum(nchunks, chunk_off);
     exclusive_sum(nckpt, ckpt_off);
+    // longest first: the rank of sequence n among all by (chunk count descending,
+    // index ascending) is its position in the order (a strict total order)
+    int32_t *order = hdr + 3 * (N + 1);
+    for (int n = tid; n < N; n += nt) {
+        if (N > kOrderMaxN) {
+            order[n] = n;
+            continue;
+        }
+        const int32_t cn = chunk_off[n + 1] - chunk_off[n];
+        int rank = 0;
+        for (int m = 0; m < N; ++m) {
+            const int32_t cm = chunk_off[m + 1] - chunk_off[m];
+            rank += (cm > cn || (cm == cn && m < n)) ? 1 : 0;
+        }
+        order[rank] = n;
+    }
 }
 
 // Rows [a, b) of sequence n (bound[] from the header when packed).
@@ -978,9 +997,10 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_v, const float *state_i
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int slice = blockIdx.x % NSL;
     const int unit = blockIdx.x / NSL;
-    const int n = unit / H, h = unit % H;
-    if (n >= N) return;
     const int32_t *chunk_off = reinterpret_cast<const int32_t *>(ws);
+    if (unit / H >= N) return;
+    // packed sequences run longest first (order[] from the chunk table)
+    const int n = cu ? chunk_off[3 * (N + 1) + unit / H] : unit / H, h = unit % H;
     int64_t ra, rb;
     seq_rows(chunk_off, cu != nullptr, T, N, n, ra, rb);
     const int nch = (int)((rb - ra + C - 1) / C);

@@ -30,7 +30,7 @@ SLOT = 66560
 
 
 def header_bytes(N):
-    return ((N + 1) * 12 + 1023) & ~1023
+    return ((N + 1) * 16 + 1023) & ~1023
 
 
 def kmajor_off(row, col, kblock):

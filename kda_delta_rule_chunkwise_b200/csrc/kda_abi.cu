@@ -38,7 +38,7 @@ bool supported_dim(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128);
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
 // ---- kernel timing (kda_profile_enable / kda_profile_last)
-constexpr int kMaxMarks = 8;
+constexpr int kMaxMarks = 16;
 struct ProfState {
     bool enabled = false;
     int device = -1;
@@ -299,12 +299,21 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const void 
     for (const void *p : {(const void *)state_in, (const void *)dstate_out, (const void *)dstate_in})
         if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return KDA_ERR_INVALID_ARG;
     const size_t need = kda_backward_workspace_bytes(rows, N, H, dk, dv);
+    const bool chunked = dtype == KDA_BF16 && dk == 128;   // through the tensor-core forward
     if (N > 0 && (!workspace || workspace_bytes < need ||
-                  (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0))
+                  (reinterpret_cast<uintptr_t>(workspace) & (chunked ? 255u : 15u)) != 0))
         return KDA_ERR_INVALID_ARG;
+    if (chunked && rows > 0) {
+        for (const void *p : {q, k, g, v})
+            if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return KDA_ERR_INVALID_ARG;
+        if (rows > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    }
     if (N == 0) return KDA_OK;
+    uint32_t *err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
     kda::BackwardArgs a{q, k, v, g, beta, state_in, cu_seqlens, rows, T, N, H, dk, dout,
-                        dstate_out, dq, dk_out, dv_out, dg, dbeta, dstate_in, workspace};
+                        dstate_out, dq, dk_out, dv_out, dg, dbeta, dstate_in, workspace,
+                        err, kda::next_launch_epoch()};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     kda::Profiler::begin(st);
     return from_cuda(kda::launch_backward(a, dtype == KDA_BF16, st));

@@ -691,8 +691,12 @@ size_t backward_workspace_bytes(int64_t rows, int N, int H, int d) {
     const int64_t token_states = (int64_t)N * H * bwd::C;
     const int nsl = bwd::slices_for((int64_t)N * H);
     const int64_t partials = nsl > 1 ? (int64_t)nsl * rows * H * (3 * d + 4) : 0;
-    return (size_t)(chunk_states + token_states) * d * d * sizeof(float) +
-           (size_t)partials * sizeof(float);
+    const size_t simt = (size_t)(chunk_states + token_states) * d * d * sizeof(float) +
+                        (size_t)partials * sizeof(float);
+    // d = 128 may take the chunked path (bf16 inputs): room for either
+    if (d != 128) return simt;
+    const size_t chunked = backward_chunked_workspace_bytes(rows, N, H);
+    return simt > chunked ? simt : chunked;
 }
 
 template <int D, int NSL, typename Tin>
@@ -755,6 +759,8 @@ static cudaError_t launch_bwd_d(const BackwardArgs &a, cudaStream_t st) {
 
 cudaError_t launch_backward(const BackwardArgs &a, bool bf16, cudaStream_t st) {
     if (a.N * (int64_t)a.H == 0) return cudaSuccess;
+    // bf16 at d = 128: through the chunked form on top of the tensor-core forward
+    if (bf16 && a.d == 128) return launch_backward_chunked(a, st);
     if (a.d == 64)
         return bf16 ? launch_bwd_d<64, __nv_bfloat16>(a, st) : launch_bwd_d<64, float>(a, st);
     return bf16 ? launch_bwd_d<128, __nv_bfloat16>(a, st) : launch_bwd_d<128, float>(a, st);

@@ -1,0 +1,789 @@
+// KDA backward through the chunked (WY) form, bf16 inputs, d = 128.
+//
+// The forward runs in its chunked form (kda_prefill_bf16.cu) with a snapshot of
+// the state at every chunk start, which leaves the per-chunk factors
+// T = (I + Akk)^-1 Diag(beta), R = Aqk T, W = T (K*Gamma), P = Q*Gamma - R (K*Gamma),
+// Khat = K*exp(G_L - G) and Gamma_L in the workspace slots.  With dS' the
+// gradient of a chunk's end state and dO of its outputs, the adjoint splits
+// (the delta rule with per-channel retention of neurohive.io "Kimi K3 ...
+// overview", section "Sequence length: hybrid KDA and Gated MLA attention";
+// the pages give no formulas for its gradient):
+//
+//   chain, chunks in reverse (bwd_chain_kernel, per (sequence, head, dv-slice)):
+//       dU = Khat dS',   dS = Diag(Gamma_L) dS' + P^T dO - W^T dU
+//   per chunk, independently (bwd_factor_kernel):
+//       U = T V - W S,  dV = T^T dU + R^T dO,  dT = dU V^T,  dR = dO V^T,
+//       dW = -dU S^T,  dP = dO S^T,  dKhat = U dS'^T,  dGamma_L = rowsum(dS' * S)
+//   per chunk, independently and without the state (bwd_input_kernel):
+//       the factor gradients pulled back to q, k, g, beta through the chunk's
+//       construction (decay-rescaled Akk / Aqk, the UT solve, R, W, P, Khat).
+//
+// All three run fp32 SIMT products on shared-memory tiles; the factors come
+// from the forward's fp16 slots.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kda_common.cuh"
+#include "kda_launch.h"
+#include "sm100.cuh"
+
+namespace kda {
+namespace cbw {
+
+constexpr int C = 64, D = 128, NT = 256;
+
+// ---- the forward's slot layout (kda_prefill_bf16.cu), read here
+constexpr uint32_t kSlotWP = 0, kSlotTR = 32768, kSlotKh = 49152, kSlotGam = 65536;
+constexpr uint32_t kSlotBytes = 66560;
+
+__device__ __forceinline__ float h2f(const uint8_t *base, uint32_t off) {
+    return __half2float(*reinterpret_cast<const __half *>(base + off));
+}
+// [-W; P]: 128 rows (0..63 = -W, 64..127 = P) x 128 channels, K-major, 128-byte
+// swizzle, 64-channel blocks 16 KiB apart
+__device__ __forceinline__ uint32_t wp_off(int r, int c) {
+    return (uint32_t)((c >> 6) * 16384 + (r >> 3) * 1024 + (r & 7) * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) +
+                      (c & 7) * 2);
+}
+// [T; R]: 128 rows (0..63 = T, 64..127 = R) x 64 columns, K-major, 128-byte swizzle
+__device__ __forceinline__ uint32_t tr_off(int r, int s) {
+    return (uint32_t)(kSlotTR + (r >> 3) * 1024 + (r & 7) * 128 + (((s >> 3) ^ (r & 7)) << 4) + (s & 7) * 2);
+}
+// Khat (token t, channel c): channel contiguous, 128-byte swizzle, 64-channel blocks 8 KiB apart
+__device__ __forceinline__ uint32_t kh_off(int t, int c) {
+    return (uint32_t)(kSlotKh + (c >> 6) * 8192 + (t >> 3) * 1024 + (t & 7) * 128 +
+                      ((((c & 63) >> 3) ^ (t & 7)) << 4) + (c & 7) * 2);
+}
+
+// out(i, j, sum_k A(i, k) B(k, j)) for an M x N result, on 256 threads as a
+// 16 x 16 grid: thread (ty, tx) owns rows ty + 16 a and columns tx + 16 b.  A, B
+// and out are functors; the sums run over k in order (fp32 FMA), so a result
+// is the same on every run.
+template <int M, int N, int K, typename FA, typename FB, typename FO>
+__device__ __forceinline__ void smm(FA A, FB B, FO out) {
+    constexpr int TM = M / 16, TN = N / 16;
+    static_assert(M % 16 == 0 && N % 16 == 0, "tile");
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float r[TM][TN];
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < TN; ++b) r[a][b] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        float av[TM], bv[TN];
+#pragma unroll
+        for (int a = 0; a < TM; ++a) av[a] = A(ty + 16 * a, k);
+#pragma unroll
+        for (int b = 0; b < TN; ++b) bv[b] = B(k, tx + 16 * b);
+#pragma unroll
+        for (int a = 0; a < TM; ++a)
+#pragma unroll
+            for (int b = 0; b < TN; ++b) r[a][b] = fmaf(av[a], bv[b], r[a][b]);
+    }
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < TN; ++b) out(ty + 16 * a, tx + 16 * b, r[a][b]);
+}
+
+// rows [a, b) of sequence n: equal-length batch, or the chunk table's clamped offsets
+__device__ __forceinline__ void seq_rows(const int32_t *hdr, bool packed, int64_t T, int N, int n,
+                                         int64_t &a, int64_t &b) {
+    if (packed) {
+        a = hdr[(N + 1) + n];
+        b = hdr[(N + 1) + n + 1];
+    } else {
+        a = (int64_t)n * T;
+        b = a + T;
+    }
+}
+__device__ __forceinline__ int first_chunk(const int32_t *hdr, bool packed, int64_t T, int n) {
+    return packed ? hdr[n] : n * (int)((T + C - 1) / C);
+}
+// state at the start of chunk j of sequence n: state_in (j = 0, or zero), else the
+// forward's snapshot after j C tokens
+__device__ __forceinline__ const float *chunk_state(const int32_t *hdr, bool packed, int64_t T, int N,
+                                                    int H, int n, int h, int j, const float *state_in,
+                                                    const float *snaps) {
+    if (j == 0) return state_in ? state_in + ((size_t)n * H + h) * D * D : nullptr;
+    const int64_t e = packed ? (int64_t)hdr[2 * (N + 1) + n] + j - 1
+                             : (int64_t)n * ((T - 1) / C) + j - 1;
+    return snaps + ((size_t)e * H + h) * D * D;
+}
+
+// ======================================================================
+// chain: dU_j = Khat_j dS'_j, dS_j = Diag(Gamma_L) dS'_j + P_j^T dO_j - W_j^T dU_j
+// one CTA per (sequence, head, 32-column slice), chunks in reverse
+// ======================================================================
+constexpr int CH_DVS = 32;
+constexpr int CH_LD = CH_DVS + 4;
+constexpr uint32_t CH_SLOT = 0;                                   // slot image (66 560 B)
+constexpr uint32_t CH_DS = kSlotBytes;                            // dS' [128][CH_LD] fp32
+constexpr uint32_t CH_Y = CH_DS + 128 * CH_LD * 4;                // dU  [64][CH_LD]
+constexpr uint32_t CH_DO = CH_Y + 64 * CH_LD * 4;                 // dO  [64][CH_LD]
+constexpr uint32_t CH_SMEM = CH_DO + 64 * CH_LD * 4;
+
+__global__ void __launch_bounds__(NT, 1)
+bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T, int N,
+                 int H, const float *__restrict__ dout, const float *dstate_out,
+                 float *__restrict__ ws_dS, float *__restrict__ ws_dU, float *dstate_in,
+                 uint32_t hdr_bytes) {
+    constexpr int NSL = D / CH_DVS;
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int slice = blockIdx.x % NSL, unit = blockIdx.x / NSL;
+    const int n = unit / H, h = unit % H;
+    if (n >= N) return;
+    const int tid = threadIdx.x;
+    const int j0 = slice * CH_DVS;
+    const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
+    const bool packed = cu != nullptr;
+    int64_t ra, rb;
+    seq_rows(hdr, packed, T, N, n, ra, rb);
+    const int nch = (int)((rb - ra + C - 1) / C);
+    const int c0 = first_chunk(hdr, packed, T, n);
+    uint8_t *slot = sm + CH_SLOT;
+    float *dS = reinterpret_cast<float *>(sm + CH_DS);
+    float *Y = reinterpret_cast<float *>(sm + CH_Y);
+    float *dO = reinterpret_cast<float *>(sm + CH_DO);
+    const size_t sbase = ((size_t)n * H + h) * D * D;
+    // dS' of the last chunk = dL/dS_final
+    for (int i = tid; i < 128 * CH_DVS; i += NT) {
+        const int c = i / CH_DVS, jj = i % CH_DVS;
+        dS[c * CH_LD + jj] = dstate_out ? dstate_out[sbase + (size_t)c * D + j0 + jj] : 0.f;
+    }
+    for (int j = nch - 1; j >= 0; --j) {
+        const int64_t t0 = ra + (int64_t)j * C;
+        const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+        const size_t item = (size_t)(c0 + j) * H + h;
+        __syncthreads();   // the previous step's reads of slot, Y and dO are done
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(fws + hdr_bytes + item * kSlotBytes);
+            uint4 *dst = reinterpret_cast<uint4 *>(slot);
+            for (int i = tid; i < (int)(kSlotBytes / 16); i += NT) dst[i] = src[i];
+        }
+        for (int i = tid; i < 64 * CH_DVS; i += NT) {
+            const int t = i / CH_DVS, jj = i % CH_DVS;
+            dO[t * CH_LD + jj] = t < L ? dout[((size_t)(t0 + t) * H + h) * D + j0 + jj] : 0.f;
+        }
+        // dS' of this chunk, for the factor kernel
+        for (int i = tid; i < 128 * CH_DVS; i += NT) {
+            const int c = i / CH_DVS, jj = i % CH_DVS;
+            ws_dS[(item * D + c) * D + j0 + jj] = dS[c * CH_LD + jj];
+        }
+        __syncthreads();
+        // dU = Khat dS'
+        smm<64, CH_DVS, 128>([&](int t, int c) { return h2f(slot, kh_off(t, c)); },
+                             [&](int c, int jj) { return dS[c * CH_LD + jj]; },
+                             [&](int t, int jj, float x) { Y[t * CH_LD + jj] = x; });
+        __syncthreads();
+        for (int i = tid; i < 64 * CH_DVS; i += NT) {
+            const int t = i / CH_DVS, jj = i % CH_DVS;
+            ws_dU[(item * 64 + t) * D + j0 + jj] = Y[t * CH_LD + jj];
+        }
+        // dS = Diag(Gamma_L) dS' + P^T dO + (-W)^T dU   (the slot holds -W); each thread
+        // overwrites only the elements it alone reads
+        {
+            const float *gam = reinterpret_cast<const float *>(slot + kSlotGam);
+            const int tx = tid & 15, ty = tid >> 4;
+            float r[8][2];
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) r[a][b] = gam[ty + 16 * a] * dS[(ty + 16 * a) * CH_LD + tx + 16 * b];
+#pragma unroll 2
+            for (int t = 0; t < 64; ++t) {
+                float pw[8], wn[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    pw[a] = h2f(slot, wp_off(64 + t, ty + 16 * a));
+                    wn[a] = h2f(slot, wp_off(t, ty + 16 * a));
+                }
+                const float o0 = dO[t * CH_LD + tx], o1 = dO[t * CH_LD + tx + 16];
+                const float y0 = Y[t * CH_LD + tx], y1 = Y[t * CH_LD + tx + 16];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    r[a][0] = fmaf(pw[a], o0, fmaf(wn[a], y0, r[a][0]));
+                    r[a][1] = fmaf(pw[a], o1, fmaf(wn[a], y1, r[a][1]));
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) dS[(ty + 16 * a) * CH_LD + tx + 16 * b] = r[a][b];
+        }
+    }
+    __syncthreads();
+    if (dstate_in)
+        for (int i = tid; i < 128 * CH_DVS; i += NT) {
+            const int c = i / CH_DVS, jj = i % CH_DVS;
+            dstate_in[sbase + (size_t)c * D + j0 + jj] = dS[c * CH_LD + jj];
+        }
+}
+
+
+// ======================================================================
+// factor gradients, one CTA per (chunk, head):
+//   U = T V - W S,  dV = T^T dU + R^T dO (the final dv),  dT = dU V^T,  dR = dO V^T,
+//   dW = -dU S^T,  dP = dO S^T,  dKhat = U dS'^T,  dGamma_L = rowsum(dS' * S)
+// ======================================================================
+constexpr int LD = 132;                                  // fp32 row stride of 128-wide tiles
+constexpr uint32_t FG_FLOATS = 64 * 64 * 2 + 64 * 128 * 3 + 128;
+constexpr uint32_t FG_DT = 0, FG_DR = 4096, FG_DW = 8192, FG_DP = 16384, FG_DKH = 24576, FG_DGL = 32768;
+constexpr uint32_t F_R0 = 0;                             // V [64][LD] + [T; R] raw | S [128][LD]
+constexpr uint32_t F_TR = 64 * LD * 4;                   //   [T; R] raw (16 KiB) after V
+constexpr uint32_t F_R1 = 128 * LD * 4;                  // dU [64][LD] + dO [64][LD] | dS' [128][LD]
+constexpr uint32_t F_R2 = F_R1 + 128 * LD * 4;           // U [64][LD] (dV first)
+constexpr uint32_t F_WP = F_R2 + 64 * LD * 4;            // [-W; P] raw (32 KiB)
+constexpr uint32_t F_SMEM = F_WP + 32768;
+static_assert(F_TR + 16384 <= F_R1, "factor kernel layout");
+
+// (sequence, chunk within it) of a global chunk index: equal-length arithmetic,
+// or the last sequence whose first chunk is <= cidx (binary search)
+__device__ __forceinline__ void locate_chunk(const int32_t *hdr, bool packed, int64_t T, int N,
+                                             int cidx, int &n, int &j) {
+    if (!packed) {
+        const int cps = (int)((T + C - 1) / C);
+        n = cidx / cps;
+        j = cidx - n * cps;
+        return;
+    }
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (hdr[mid] <= cidx) lo = mid; else hi = mid - 1;
+    }
+    n = lo;
+    j = cidx - hdr[lo];
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(NT, 1)
+bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T, int N,
+                  int H, const Tin *__restrict__ v, const float *state_in,
+                  const float *__restrict__ snaps, const float *__restrict__ dout,
+                  const float *__restrict__ ws_dS, const float *__restrict__ ws_dU,
+                  float *__restrict__ fg, float *__restrict__ dv, uint32_t hdr_bytes) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int tid = threadIdx.x;
+    const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
+    const bool packed = cu != nullptr;
+    const int total = packed ? hdr[N] : N * (int)((T + C - 1) / C);
+    const int cidx = blockIdx.x / H, h = blockIdx.x % H;
+    if (cidx >= total) return;
+    int n, j;
+    locate_chunk(hdr, packed, T, N, cidx, n, j);
+    int64_t ra, rb;
+    seq_rows(hdr, packed, T, N, n, ra, rb);
+    const int64_t t0 = ra + (int64_t)j * C;
+    const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+    const size_t item = (size_t)cidx * H + h;
+    const uint8_t *slot = fws + hdr_bytes + item * kSlotBytes;
+    float *V = reinterpret_cast<float *>(sm + F_R0);
+    const uint8_t *trw = sm + F_TR;          // [T; R] raw (offsets tr_off - kSlotTR)
+    float *dU = reinterpret_cast<float *>(sm + F_R1);
+    float *dO = dU + 64 * LD;
+    float *U = reinterpret_cast<float *>(sm + F_R2);
+    const uint8_t *wpw = sm + F_WP;          // [-W; P] raw (offsets wp_off)
+    float *out = fg + item * FG_FLOATS;
+
+    // ---- phase 1: V, dU, dO, [T; R] and [-W; P] in shared memory
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int t = i >> 7, c = i & 127;
+        V[t * LD + c] = t < L ? to_f32(v[((size_t)(t0 + t) * H + h) * D + c]) : 0.f;
+        dU[t * LD + c] = ws_dU[(item * 64 + t) * D + c];
+        dO[t * LD + c] = t < L ? dout[((size_t)(t0 + t) * H + h) * D + c] : 0.f;
+    }
+    for (int i = tid; i < 16384 / 16; i += NT)
+        reinterpret_cast<uint4 *>(sm + F_TR)[i] = reinterpret_cast<const uint4 *>(slot + kSlotTR)[i];
+    for (int i = tid; i < 32768 / 16; i += NT)
+        reinterpret_cast<uint4 *>(sm + F_WP)[i] = reinterpret_cast<const uint4 *>(slot + kSlotWP)[i];
+    __syncthreads();
+    auto Tm = [&](int r, int s) { return h2f(trw, tr_off(r, s) - kSlotTR); };        // T[r][s]
+    auto Rm = [&](int r, int s) { return h2f(trw, tr_off(64 + r, s) - kSlotTR); };   // R[r][s]
+    // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out)
+    smm<64, 128, 64>([&](int s, int t) { return Tm(t, s); }, [&](int t, int c) { return dU[t * LD + c]; },
+                     [&](int s, int c, float x) { U[s * LD + c] = x; });
+    smm<64, 128, 64>([&](int s, int t) { return Rm(t, s); }, [&](int t, int c) { return dO[t * LD + c]; },
+                     [&](int s, int c, float x) { U[s * LD + c] += x; });
+    __syncthreads();
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int s = i >> 7, c = i & 127;
+        if (s < L) dv[((size_t)(t0 + s) * H + h) * D + c] = U[s * LD + c];
+    }
+    // dT = dU V^T, dR = dO V^T
+    smm<64, 64, 128>([&](int t, int c) { return dU[t * LD + c]; }, [&](int c, int s) { return V[s * LD + c]; },
+                     [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; });
+    smm<64, 64, 128>([&](int t, int c) { return dO[t * LD + c]; }, [&](int c, int s) { return V[s * LD + c]; },
+                     [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; });
+    __syncthreads();   // U's buffer (dV) is read out
+    // U = T V
+    smm<64, 128, 64>([&](int t, int s) { return Tm(t, s); }, [&](int s, int c) { return V[s * LD + c]; },
+                     [&](int t, int c, float x) { U[t * LD + c] = x; });
+    __syncthreads();   // V and [T; R] are consumed
+
+    // ---- phase 2: S
+    float *S = reinterpret_cast<float *>(sm + F_R0);
+    {
+        const float *Sg = chunk_state(hdr, packed, T, N, H, n, h, j, state_in, snaps);
+        for (int i = tid; i < 128 * 128; i += NT) {
+            const int c = i >> 7, jj = i & 127;
+            S[c * LD + jj] = Sg ? Sg[i] : 0.f;
+        }
+    }
+    __syncthreads();
+    // U += (-W) S   (the slot holds -W)
+    smm<64, 128, 128>([&](int t, int c) { return h2f(wpw, wp_off(t, c)); },
+                      [&](int c, int jj) { return S[c * LD + jj]; },
+                      [&](int t, int jj, float x) { U[t * LD + jj] += x; });
+    // dW = -dU S^T, dP = dO S^T
+    smm<64, 128, 128>([&](int t, int jj) { return dU[t * LD + jj]; }, [&](int jj, int c) { return S[c * LD + jj]; },
+                      [&](int t, int c, float x) { out[FG_DW + t * 128 + c] = -x; });
+    smm<64, 128, 128>([&](int t, int jj) { return dO[t * LD + jj]; }, [&](int jj, int c) { return S[c * LD + jj]; },
+                      [&](int t, int c, float x) { out[FG_DP + t * 128 + c] = x; });
+    __syncthreads();   // dU and dO are consumed
+
+    // ---- phase 3: dS'
+    float *dSp = reinterpret_cast<float *>(sm + F_R1);
+    for (int i = tid; i < 128 * 128; i += NT) {
+        const int c = i >> 7, jj = i & 127;
+        dSp[c * LD + jj] = ws_dS[item * D * D + i];
+    }
+    __syncthreads();
+    if (tid < 128) {
+        float a = 0.f;
+        for (int jj = 0; jj < 128; ++jj) a = fmaf(dSp[tid * LD + jj], S[tid * LD + jj], a);
+        out[FG_DGL + tid] = a;
+    }
+    // dKhat = U dS'^T
+    smm<64, 128, 128>([&](int t, int jj) { return U[t * LD + jj]; }, [&](int jj, int c) { return dSp[c * LD + jj]; },
+                      [&](int t, int c, float x) { out[FG_DKH + t * 128 + c] = x; });
+}
+
+
+// ======================================================================
+// input side, one CTA per (chunk, head), in three kernels with the chunk's
+// 64 x 64 intermediates in the workspace (IW_* offsets, floats per item):
+//   recompute   Aqk, M (decay-rescaled, the forward's 16-row references)
+//   pullback    X = (I + Diag(beta) M)^-1, T, R, K*Gamma;
+//               dR' = dR - dP (K*Gamma)^T,  dKt = T^T dW - R^T dP,
+//               dT' = dT + Aqk^T dR' + dW (K*Gamma)^T,  dAqk = tril(dR' T^T),
+//               dbeta = colsum(X * dT') + rowsum(dAkk * M),
+//               dAkk = strict_tril(-X^T (dT' Diag(beta)) X^T),  dM = Diag(beta) dAkk
+//   assemble    the decayed adjoints of Aqk (q, k) and M (k, k), then
+//               dq = dP Gamma + da_q,
+//               dk = dKt Gamma + dKhat Gamma_L / Gamma + db_qk + da_k + db_kk,
+//               dG = (Q*Gamma) dP + (K*Gamma) dKt - Khat dKhat + q da_q - k db_qk
+//                    + k da_k - k db_kk  (+ sum_r Khat dKhat + Gamma_L dGamma_L at row L-1),
+//               dg = reverse cumsum of dG over the rows, 0 where g < -5
+// A decayed form F[r,s] = sum_c a_r b_s exp(G_r - G_s) (s <= r) has
+//   da_r = E1_r sum_s dF[r,s] b_s exp(R_a - G_s)          (a = block of r)
+//   db_s = sum_a exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r
+// with E1_r = exp(G_r - R_a) in [e^-80, 1] and exp(R_a - G_s) <= e^80: the
+// factorisation the forward uses, in fp32.
+// ======================================================================
+constexpr uint32_t IW_AQK = 0, IW_M = 4096, IW_DAQK = 8192, IW_DM = 12288, IW_DKT = 16384,
+                   IW_DB = 16384 + 8192, IW_FLOATS = 16384 + 8192 + 64;
+
+// G = cumsum(max(g, -5)) over the chunk's rows (rows past L decay by nothing), and
+// the block references R_a = G at the end of block a - 1 (R_0 = 0), per channel
+template <typename Tin>
+__device__ __forceinline__ void chunk_cumsum(const Tin *g, int64_t t0, int H, int h, int L, float *G,
+                                             float *Rref) {
+    const int tid = threadIdx.x;
+    if (tid < 128) {
+        float acc = 0.f;
+        for (int r = 0; r < 64; ++r) {
+            const float x = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + tid]), -5.f) : 0.f;
+            acc += x;
+            G[r * LD + tid] = acc;
+            if ((r & 15) == 15 && r < 63) Rref[((r + 1) >> 4) * 128 + tid] = acc;
+        }
+        Rref[tid] = 0.f;
+    }
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(NT, 1)
+bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T,
+                     int N, int H, const Tin *__restrict__ q, const Tin *__restrict__ k,
+                     const Tin *__restrict__ g, float *__restrict__ iw) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int tid = threadIdx.x;
+    const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
+    const bool packed = cu != nullptr;
+    const int total = packed ? hdr[N] : N * (int)((T + C - 1) / C);
+    const int cidx = blockIdx.x / H, h = blockIdx.x % H;
+    if (cidx >= total) return;
+    int n, j;
+    locate_chunk(hdr, packed, T, N, cidx, n, j);
+    int64_t ra, rb;
+    seq_rows(hdr, packed, T, N, n, ra, rb);
+    const int64_t t0 = ra + (int64_t)j * C;
+    const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+    float *G = reinterpret_cast<float *>(sm);              // [64][LD]
+    float *QE = G + 64 * LD;                               // q_r E1_r
+    float *KE = QE + 64 * LD;                              // k_r E1_r
+    float *KF = KE + 64 * LD;                              // k_s exp(R_a - G_s), block a's
+    float *Rref = KF + 64 * LD;                            // [4][128]
+    float *out = iw + ((size_t)cidx * H + h) * IW_FLOATS;
+    chunk_cumsum(g, t0, H, h, L, G, Rref);
+    __syncthreads();
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int r = i >> 7, c = i & 127;
+        const float e1 = __expf(G[r * LD + c] - Rref[(r >> 4) * 128 + c]);
+        const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
+        QE[r * LD + c] = r < L ? to_f32(q[off]) * e1 : 0.f;
+        KE[r * LD + c] = r < L ? to_f32(k[off]) * e1 : 0.f;
+    }
+    for (int a = 0; a < 4; ++a) {
+        const int ns = 16 * (a + 1);   // rows s <= 16a + 15
+        __syncthreads();
+        for (int i = tid; i < ns * 128; i += NT) {
+            const int s = i >> 7, c = i & 127;
+            KF[s * LD + c] = s < L ? to_f32(k[((size_t)(t0 + s) * H + h) * D + c]) *
+                                         __expf(Rref[a * 128 + c] - G[s * LD + c])
+                                   : 0.f;
+        }
+        for (int i = tid + ns * 128; i < 64 * 128; i += NT) KF[(i >> 7) * LD + (i & 127)] = 0.f;
+        __syncthreads();
+        // rows 16a .. 16a + 15 of Aqk (s <= r) and M (s < r)
+        smm<16, 64, 128>([&](int r, int c) { return QE[(16 * a + r) * LD + c]; },
+                         [&](int c, int s) { return KF[s * LD + c]; },
+                         [&](int r, int s, float x) {
+                             out[IW_AQK + (16 * a + r) * 64 + s] = s <= 16 * a + r ? x : 0.f;
+                         });
+        smm<16, 64, 128>([&](int r, int c) { return KE[(16 * a + r) * LD + c]; },
+                         [&](int c, int s) { return KF[s * LD + c]; },
+                         [&](int r, int s, float x) {
+                             out[IW_M + (16 * a + r) * 64 + s] = s < 16 * a + r ? x : 0.f;
+                         });
+    }
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(NT, 1)
+bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T,
+                    int N, int H, const Tin *__restrict__ k, const Tin *__restrict__ g,
+                    const Tin *__restrict__ beta, const float *__restrict__ fg,
+                    float *__restrict__ iw) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    constexpr int L6 = 68;   // row stride of 64 x 64 tiles
+    const int tid = threadIdx.x;
+    const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
+    const bool packed = cu != nullptr;
+    const int total = packed ? hdr[N] : N * (int)((T + C - 1) / C);
+    const int cidx = blockIdx.x / H, h = blockIdx.x % H;
+    if (cidx >= total) return;
+    int n, j;
+    locate_chunk(hdr, packed, T, N, cidx, n, j);
+    int64_t ra, rb;
+    seq_rows(hdr, packed, T, N, n, ra, rb);
+    const int64_t t0 = ra + (int64_t)j * C;
+    const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+    const size_t item = (size_t)cidx * H + h;
+    float *io = iw + item * IW_FLOATS;
+    const float *fgi = fg + item * FG_FLOATS;
+    float *Aq = reinterpret_cast<float *>(sm);            // Aqk        [64][L6]
+    float *Mm = Aq + 64 * L6;                              // M
+    float *X = Mm + 64 * L6;                               // X = (I + Diag(beta) M)^-1
+    float *Rm = X + 64 * L6;                               // R = Aqk T
+    float *dTp = Rm + 64 * L6;                             // dT'
+    float *dRp = dTp + 64 * L6;                            // dR'
+    float *Wk = dRp + 64 * L6;                             // scratch [64][L6]
+    float *Kt = Wk + 64 * L6;                              // K * Gamma  [64][LD]
+    float *bs = Kt + 64 * LD;                              // beta [64]
+    for (int i = tid; i < 64 * 64; i += NT) {
+        const int r = i >> 6, s = i & 63;
+        Aq[r * L6 + s] = io[IW_AQK + i];
+        Mm[r * L6 + s] = io[IW_M + i];
+    }
+    if (tid < 64) bs[tid] = tid < L ? to_f32(beta[(size_t)(t0 + tid) * H + h]) : 0.f;
+    if (tid < 128) {   // K * Gamma, Gamma = exp(cumsum(max(g, -5)))
+        float acc = 0.f;
+        for (int r = 0; r < 64; ++r) {
+            const size_t off = ((size_t)(t0 + r) * H + h) * D + tid;
+            acc += r < L ? fmaxf(to_f32(g[off]), -5.f) : 0.f;
+            Kt[r * LD + tid] = r < L ? to_f32(k[off]) * __expf(acc) : 0.f;
+        }
+    }
+    __syncthreads();
+    // X: column i of (I + Diag(beta) M)^-1 by forward substitution, four partial sums
+    if (tid < 64) {
+        const int col = tid;
+        for (int r = 0; r < 64; ++r) {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            int m = col;
+            for (; m + 3 < r; m += 4) {
+                a0 = fmaf(Mm[r * L6 + m], X[m * L6 + col], a0);
+                a1 = fmaf(Mm[r * L6 + m + 1], X[(m + 1) * L6 + col], a1);
+                a2 = fmaf(Mm[r * L6 + m + 2], X[(m + 2) * L6 + col], a2);
+                a3 = fmaf(Mm[r * L6 + m + 3], X[(m + 3) * L6 + col], a3);
+            }
+            for (; m < r; ++m) a0 = fmaf(Mm[r * L6 + m], X[m * L6 + col], a0);
+            const float sum = (a0 + a1) + (a2 + a3);
+            X[r * L6 + col] = r < col ? 0.f : ((r == col ? 1.f : 0.f) - bs[r] * sum);
+        }
+    }
+    __syncthreads();
+    // R = Aqk T, T = X Diag(beta)
+    smm<64, 64, 64>([&](int r, int m) { return Aq[r * L6 + m]; }, [&](int m, int s) { return X[m * L6 + s] * bs[s]; },
+                    [&](int r, int s, float x) { Rm[r * L6 + s] = x; });
+    __syncthreads();
+    // dR' = dR - dP (K Gamma)^T
+    smm<64, 64, 128>([&](int t, int c) { return fgi[FG_DP + t * 128 + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
+                     [&](int t, int s, float x) { dRp[t * L6 + s] = fgi[FG_DR + t * 64 + s] - x; });
+    // dT'_0 = dT + dW (K Gamma)^T
+    smm<64, 64, 128>([&](int t, int c) { return fgi[FG_DW + t * 128 + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
+                     [&](int t, int s, float x) { dTp[t * L6 + s] = fgi[FG_DT + t * 64 + s] + x; });
+    // dKt = T^T dW - R^T dP  -> workspace
+    smm<64, 128, 64>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return fgi[FG_DW + t * 128 + c]; },
+                     [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] = x; });
+    __syncthreads();
+    smm<64, 128, 64>([&](int s, int t) { return Rm[t * L6 + s]; }, [&](int t, int c) { return fgi[FG_DP + t * 128 + c]; },
+                     [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] -= x; });
+    // dT' += Aqk^T dR'
+    smm<64, 64, 64>([&](int r, int m) { return Aq[m * L6 + r]; }, [&](int m, int s) { return dRp[m * L6 + s]; },
+                    [&](int r, int s, float x) { dTp[r * L6 + s] += x; });
+    // dAqk = tril(dR' T^T) -> workspace
+    smm<64, 64, 64>([&](int r, int m) { return dRp[r * L6 + m]; }, [&](int m, int s) { return X[s * L6 + m] * bs[m]; },
+                    [&](int r, int s, float x) { io[IW_DAQK + r * 64 + s] = s <= r ? x : 0.f; });
+    __syncthreads();
+    // Wk = X^T (dT' Diag(beta))
+    smm<64, 64, 64>([&](int r, int m) { return X[m * L6 + r]; }, [&](int m, int s) { return dTp[m * L6 + s] * bs[s]; },
+                    [&](int r, int s, float x) { Wk[r * L6 + s] = x; });
+    __syncthreads();
+    // dAkk = strict_tril(-Wk X^T), dM = Diag(beta) dAkk -> workspace; dAkk * M row sums
+    smm<64, 64, 64>([&](int r, int m) { return Wk[r * L6 + m]; }, [&](int m, int s) { return X[s * L6 + m]; },
+                    [&](int r, int s, float x) {
+                        const float dakk = s < r ? -x : 0.f;
+                        Rm[r * L6 + s] = dakk;                       // R is consumed: reuse for dAkk
+                        io[IW_DM + r * 64 + s] = bs[r] * dakk;
+                    });
+    __syncthreads();
+    // dbeta_s = sum_r X[r,s] dT'[r,s] + sum_t dAkk[s,t] M[s,t]
+    if (tid < 64) {
+        float a = 0.f, b = 0.f;
+        for (int r = 0; r < 64; ++r) {
+            a = fmaf(X[r * L6 + tid], dTp[r * L6 + tid], a);
+            b = fmaf(Rm[tid * L6 + r], Mm[tid * L6 + r], b);
+        }
+        io[IW_DB + tid] = a + b;
+    }
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(NT, 1)
+bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T,
+                    int N, int H, const Tin *__restrict__ q, const Tin *__restrict__ k,
+                    const Tin *__restrict__ g, const float *__restrict__ fg,
+                    const float *__restrict__ iw, float *__restrict__ dq, float *__restrict__ dk,
+                    float *__restrict__ dg, float *__restrict__ dbeta) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int tid = threadIdx.x;
+    const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
+    const bool packed = cu != nullptr;
+    const int total = packed ? hdr[N] : N * (int)((T + C - 1) / C);
+    const int cidx = blockIdx.x / H, h = blockIdx.x % H;
+    if (cidx >= total) return;
+    int n, j;
+    locate_chunk(hdr, packed, T, N, cidx, n, j);
+    int64_t ra, rb;
+    seq_rows(hdr, packed, T, N, n, ra, rb);
+    const int64_t t0 = ra + (int64_t)j * C;
+    const int L = (int)((rb - t0) < C ? (rb - t0) : C);
+    const size_t item = (size_t)cidx * H + h;
+    const float *io = iw + item * IW_FLOATS;
+    const float *fgi = fg + item * FG_FLOATS;
+    float *G = reinterpret_cast<float *>(sm);             // [64][LD]
+    float *AE = G + 64 * LD;                               // a_r E1_r (q or k)
+    float *KF = AE + 64 * LD;                              // k_s exp(R_a - G_s), block a's
+    float *dG = KF + 64 * LD;                              // dG accumulator
+    float *Dq = dG + 64 * LD;                              // dq accumulator
+    float *Dk = Dq + 64 * LD;                              // dk accumulator
+    float *Rref = Dk + 64 * LD;                            // [4][128]
+    chunk_cumsum(g, t0, H, h, L, G, Rref);
+    __syncthreads();
+    auto qv = [&](int r, int c) { return r < L ? to_f32(q[((size_t)(t0 + r) * H + h) * D + c]) : 0.f; };
+    auto kv = [&](int r, int c) { return r < L ? to_f32(k[((size_t)(t0 + r) * H + h) * D + c]) : 0.f; };
+    const float *gl = G + 63 * LD;   // G at the last row = G_L (rows past L add nothing)
+    // the elementwise terms
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int r = i >> 7, c = i & 127;
+        const float Gr = G[r * LD + c], gam = __expf(Gr), kh_f = __expf(gl[c] - Gr);
+        const float qq = qv(r, c), kk = kv(r, c);
+        const float dP = fgi[FG_DP + r * 128 + c], dKt = io[IW_DKT + r * 128 + c];
+        const float dKh = fgi[FG_DKH + r * 128 + c];
+        Dq[r * LD + c] = dP * gam;
+        Dk[r * LD + c] = dKt * gam + dKh * kh_f;
+        dG[r * LD + c] = qq * gam * dP + kk * gam * dKt - kk * kh_f * dKh;
+    }
+    // decayed adjoints: first Aqk with (a, b) = (q, k), then M with (k, k)
+    for (int form = 0; form < 2; ++form) {
+        const float *dF = io + (form == 0 ? IW_DAQK : IW_DM);
+        __syncthreads();
+        for (int i = tid; i < 64 * 128; i += NT) {
+            const int r = i >> 7, c = i & 127;
+            const float e1 = __expf(G[r * LD + c] - Rref[(r >> 4) * 128 + c]);
+            AE[r * LD + c] = (form == 0 ? qv(r, c) : kv(r, c)) * e1;
+        }
+        for (int a = 0; a < 4; ++a) {
+            const int ns = 16 * (a + 1);
+            __syncthreads();
+            for (int i = tid; i < 64 * 128; i += NT) {
+                const int s = i >> 7, c = i & 127;
+                KF[s * LD + c] = s < ns ? __expf(Rref[a * 128 + c] - G[s * LD + c]) : 0.f;   // exp(R_a - G_s)
+            }
+            __syncthreads();
+            // da_r (rows of block a) = E1_r sum_s dF[r,s] b_s exp(R_a - G_s), b = k
+            smm<16, 128, 64>([&](int r, int s) { return dF[(16 * a + r) * 64 + s]; },
+                             [&](int s, int c) { return kv(s, c) * KF[s * LD + c]; },
+                             [&](int r, int c, float x) {
+                                 const int rr = 16 * a + r;
+                                 const float da = x * __expf(G[rr * LD + c] - Rref[a * 128 + c]);
+                                 const float av = form == 0 ? qv(rr, c) : kv(rr, c);
+                                 if (form == 0) Dq[rr * LD + c] += da; else Dk[rr * LD + c] += da;
+                                 dG[rr * LD + c] += av * da;
+                             });
+            // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s <= 16a + 15
+            smm<64, 128, 16>([&](int s, int r) { return dF[(16 * a + r) * 64 + s]; },
+                             [&](int r, int c) { return AE[(16 * a + r) * LD + c]; },
+                             [&](int s, int c, float x) {
+                                 if (s >= ns) return;
+                                 const float db = x * KF[s * LD + c];
+                                 Dk[s * LD + c] += db;
+                                 dG[s * LD + c] -= kv(s, c) * db;
+                             });
+        }
+    }
+    __syncthreads();
+    // row L-1 also carries G_L's gradient: sum_r Khat dKhat + Gamma_L dGamma_L; then
+    // dg = reverse cumsum of dG, 0 where g < -5
+    if (tid < 128 && L > 0) {
+        const int c = tid;
+        float s_kh = 0.f;
+        for (int r = 0; r < L; ++r)
+            s_kh = fmaf(kv(r, c) * __expf(gl[c] - G[r * LD + c]), fgi[FG_DKH + r * 128 + c], s_kh);
+        dG[(L - 1) * LD + c] += s_kh + __expf(gl[c]) * fgi[FG_DGL + c];
+        float acc = 0.f;
+        for (int r = L - 1; r >= 0; --r) {
+            acc += dG[r * LD + c];
+            const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
+            dg[off] = to_f32(g[off]) >= -5.f ? acc : 0.f;
+        }
+    }
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int r = i >> 7, c = i & 127;
+        if (r < L) {
+            const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
+            dq[off] = Dq[r * LD + c];
+            dk[off] = Dk[r * LD + c];
+        }
+    }
+    if (tid < L) dbeta[(size_t)(t0 + tid) * H + h] = io[IW_DB + tid];
+}
+
+}  // namespace cbw
+
+// ======================================================================
+// host side
+// ======================================================================
+namespace {
+struct CwLayout {
+    int64_t max_chunks;
+    size_t fws, o, snaps, sout, dS, dU, fg, iw, total;
+};
+size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+CwLayout cw_layout(int64_t rows, int N, int H) {
+    CwLayout L;
+    L.max_chunks = (rows + cbw::C - 1) / cbw::C + N;
+    const size_t mch = (size_t)L.max_chunks * H, dd = (size_t)cbw::D * cbw::D;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t o = off; off += al256(bytes); return o; };
+    L.fws = take(prefill_tc_workspace_bytes(rows, N, H, cbw::D));
+    L.o = take((size_t)rows * H * cbw::D * 4);
+    L.snaps = take(mch * dd * 4);
+    L.sout = take((size_t)N * H * dd * 4);
+    L.dS = take(mch * dd * 4);
+    L.dU = take(mch * 64 * cbw::D * 4);
+    L.fg = take(mch * cbw::FG_FLOATS * 4);
+    L.iw = take(mch * cbw::IW_FLOATS * 4);
+    L.total = off;
+    return L;
+}
+template <typename K>
+cudaError_t set_smem(K kern, uint32_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+}  // namespace
+
+size_t backward_chunked_workspace_bytes(int64_t rows, int N, int H) {
+    return cw_layout(rows, N, H).total;
+}
+
+cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
+    using namespace cbw;
+    using bf = __nv_bfloat16;
+    const CwLayout L = cw_layout(a.rows, a.N, a.H);
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    uint8_t *fws = ws + L.fws;
+    float *snaps = reinterpret_cast<float *>(ws + L.snaps);
+    // 1. the forward in its chunked form, with a snapshot at every chunk start
+    PrefillArgs f{};
+    f.q = a.q; f.k = a.k; f.v = a.v; f.g = a.g; f.beta = a.beta;
+    f.state_in = a.state_in;
+    f.cu_seqlens = a.cu_seqlens;
+    f.B = a.cu_seqlens ? 1 : (a.T > 0 ? (int)(a.rows / a.T) : a.N);
+    f.T = a.T;
+    f.N = a.N; f.H = a.H; f.dk = D; f.dv = D;
+    f.o = ws + L.o;
+    f.state_out = reinterpret_cast<float *>(ws + L.sout);
+    f.workspace = fws;
+    f.workspace_bytes = prefill_tc_workspace_bytes(a.rows, a.N, a.H, D);
+    f.err = a.err;
+    f.ckpt_interval = C;
+    f.ckpt = snaps;
+    f.ckpt_capacity = L.max_chunks;
+    f.epoch = a.epoch;
+    cudaError_t e = launch_prefill_tc(f, st);
+    if (e != cudaSuccess) return e;
+    const uint32_t hb = (uint32_t)(((size_t)(a.N + 1) * 16 + 1023) & ~(size_t)1023);
+    float *dS = reinterpret_cast<float *>(ws + L.dS), *dU = reinterpret_cast<float *>(ws + L.dU);
+    float *fg = reinterpret_cast<float *>(ws + L.fg), *iw = reinterpret_cast<float *>(ws + L.iw);
+    // 2. the chain, chunks in reverse
+    if ((e = set_smem(bwd_chain_kernel, CH_SMEM)) != cudaSuccess) return e;
+    bwd_chain_kernel<<<(unsigned)(a.N * a.H * (D / CH_DVS)), NT, CH_SMEM, st>>>(
+        fws, a.cu_seqlens, a.T, a.N, a.H, a.dout, a.dstate_out, dS, dU, a.dstate_in, hb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    Profiler::mark(st);
+    // 3.-6. per chunk: factor gradients (and dv), recompute, pull-back, assembly
+    const unsigned items = (unsigned)(L.max_chunks * a.H);
+    if ((e = set_smem(bwd_factor_kernel<bf>, F_SMEM)) != cudaSuccess) return e;
+    bwd_factor_kernel<bf><<<items, NT, F_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.v,
+                                                     a.state_in, snaps, a.dout, dS, dU, fg, a.dv, hb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    Profiler::mark(st);
+    constexpr uint32_t RC_SMEM = 4 * 64 * LD * 4 + 4 * 128 * 4;
+    if ((e = set_smem(bwd_recompute_kernel<bf>, RC_SMEM)) != cudaSuccess) return e;
+    bwd_recompute_kernel<bf><<<items, NT, RC_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
+                                                         (const bf *)a.k, (const bf *)a.g, iw);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    Profiler::mark(st);
+    constexpr uint32_t PB_SMEM = 7 * 64 * 68 * 4 + 64 * LD * 4 + 64 * 4;
+    if ((e = set_smem(bwd_pullback_kernel<bf>, PB_SMEM)) != cudaSuccess) return e;
+    bwd_pullback_kernel<bf><<<items, NT, PB_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.k,
+                                                        (const bf *)a.g, (const bf *)a.beta, fg, iw);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    Profiler::mark(st);
+    constexpr uint32_t AS_SMEM = 6 * 64 * LD * 4 + 4 * 128 * 4;
+    if ((e = set_smem(bwd_assemble_kernel<bf>, AS_SMEM)) != cudaSuccess) return e;
+    bwd_assemble_kernel<bf><<<items, NT, AS_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
+                                                        (const bf *)a.k, (const bf *)a.g, fg, iw, a.dq,
+                                                        a.dk, a.dg, a.dbeta);
+    e = cudaGetLastError();
+    Profiler::mark(st);
+    return e;
+}
+
+}  // namespace kda

@@ -66,8 +66,13 @@ struct BackwardArgs {
     const float *dout, *dstate_out;
     float *dq, *dk, *dv, *dg, *dbeta, *dstate_in;
     void *workspace;
+    uint32_t *err = nullptr;     // device error word (the chunked path's forward waits)
+    uint32_t epoch = 0;
 };
 size_t backward_workspace_bytes(int64_t rows, int N, int H, int d);
 cudaError_t launch_backward(const BackwardArgs &a, bool bf16, cudaStream_t st);
+// Backward through the chunked form (kda_backward_chunked.cu): bf16 inputs, d = 128.
+size_t backward_chunked_workspace_bytes(int64_t rows, int N, int H);
+cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st);
 
 }  // namespace kda

@@ -515,11 +515,24 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
         ev1.record(st)
         torch.cuda.synchronize()
         b_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        # per-kernel device times of one call (events on the launching stream)
+        binding.kda_profile_enable(True)
+        bstep()
+        kms = binding.kda_profile_last(16)
+        binding.kda_profile_enable(False)
+        names = ["chunk_table_kernel"] if len(kms) == 8 else []
+        names += ["intra_chunk_kernel (forward)", "state_pass_kernel (forward, snapshots every chunk)",
+                  "bwd_chain_kernel", "bwd_factor_kernel", "bwd_recompute_kernel",
+                  "bwd_pullback_kernel", "bwd_assemble_kernel"]
         extra["backward"] = {"workload": "prefill_h32_t8192_d128", "steps": nb,
                              "ms_per_step": round(b_ms / nb, 3),
                              "value": aggregate_throughput(bw.B * bw.T, world, nb, b_ms),
                              "unit": "tokens/s",
-                             "kernel": "backward_sliced_kernel (fp32, one CTA per (sequence, head, 32-column slice)) + backward_reduce_kernel"}
+                             "path": "chunked form (bf16, d = 128): the tensor-core forward with a "
+                                     "snapshot per chunk, a reverse chain over chunks, then per-chunk "
+                                     "factor gradients and their pull-back (fp32 products)",
+                             "kernel_ms": ({n: round(x, 4) for n, x in zip(names, kms)}
+                                           if len(names) == len(kms) else [round(x, 4) for x in kms])}
         del bw, dout, wsb
         torch.cuda.empty_cache()
 

@@ -118,8 +118,12 @@ __device__ __forceinline__ const float *chunk_state(const int32_t *hdr, bool pac
 // ======================================================================
 constexpr int CH_DVS = 32;
 constexpr int CH_LD = CH_DVS + 4;
+constexpr int LDF = 132;                                          // fp32 row stride of 128-wide tiles
 constexpr uint32_t CH_SLOT = 0;                                   // slot image (66 560 B)
-constexpr uint32_t CH_DS = kSlotBytes;                            // dS' [128][CH_LD] fp32
+constexpr uint32_t CH_KH = kSlotBytes;                            // Khat [64][LDF] fp32
+constexpr uint32_t CH_WN = CH_KH + 64 * LDF * 4;                  // -W   [64][LDF]
+constexpr uint32_t CH_P = CH_WN + 64 * LDF * 4;                   // P    [64][LDF]
+constexpr uint32_t CH_DS = CH_P + 64 * LDF * 4;                   // dS' [128][CH_LD] fp32
 constexpr uint32_t CH_Y = CH_DS + 128 * CH_LD * 4;                // dU  [64][CH_LD]
 constexpr uint32_t CH_DO = CH_Y + 64 * CH_LD * 4;                 // dO  [64][CH_LD]
 constexpr uint32_t CH_SMEM = CH_DO + 64 * CH_LD * 4;
@@ -143,6 +147,9 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
     const int nch = (int)((rb - ra + C - 1) / C);
     const int c0 = first_chunk(hdr, packed, T, n);
     uint8_t *slot = sm + CH_SLOT;
+    float *Kh = reinterpret_cast<float *>(sm + CH_KH);
+    float *Wn = reinterpret_cast<float *>(sm + CH_WN);
+    float *Pm = reinterpret_cast<float *>(sm + CH_P);
     float *dS = reinterpret_cast<float *>(sm + CH_DS);
     float *Y = reinterpret_cast<float *>(sm + CH_Y);
     float *dO = reinterpret_cast<float *>(sm + CH_DO);
@@ -171,9 +178,16 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
             const int c = i / CH_DVS, jj = i % CH_DVS;
             ws_dS[(item * D + c) * D + j0 + jj] = dS[c * CH_LD + jj];
         }
+        __syncthreads();   // the slot image has landed
+        for (int i = tid; i < 64 * 128; i += NT) {
+            const int t = i >> 7, c = i & 127;
+            Kh[t * LDF + c] = h2f(slot, kh_off(t, c));
+            Wn[t * LDF + c] = h2f(slot, wp_off(t, c));
+            Pm[t * LDF + c] = h2f(slot, wp_off(64 + t, c));
+        }
         __syncthreads();
         // dU = Khat dS'
-        smm<64, CH_DVS, 128>([&](int t, int c) { return h2f(slot, kh_off(t, c)); },
+        smm<64, CH_DVS, 128>([&](int t, int c) { return Kh[t * LDF + c]; },
                              [&](int c, int jj) { return dS[c * CH_LD + jj]; },
                              [&](int t, int jj, float x) { Y[t * CH_LD + jj] = x; });
         __syncthreads();
@@ -196,8 +210,8 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
                 float pw[8], wn[8];
 #pragma unroll
                 for (int a = 0; a < 8; ++a) {
-                    pw[a] = h2f(slot, wp_off(64 + t, ty + 16 * a));
-                    wn[a] = h2f(slot, wp_off(t, ty + 16 * a));
+                    pw[a] = Pm[t * LDF + ty + 16 * a];
+                    wn[a] = Wn[t * LDF + ty + 16 * a];
                 }
                 const float o0 = dO[t * CH_LD + tx], o1 = dO[t * CH_LD + tx + 16];
                 const float y0 = Y[t * CH_LD + tx], y1 = Y[t * CH_LD + tx + 16];
@@ -231,13 +245,16 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
 constexpr int LD = 132;                                  // fp32 row stride of 128-wide tiles
 constexpr uint32_t FG_FLOATS = 64 * 64 * 2 + 64 * 128 * 3 + 128;
 constexpr uint32_t FG_DT = 0, FG_DR = 4096, FG_DW = 8192, FG_DP = 16384, FG_DKH = 24576, FG_DGL = 32768;
-constexpr uint32_t F_R0 = 0;                             // V [64][LD] + [T; R] raw | S [128][LD]
-constexpr uint32_t F_TR = 64 * LD * 4;                   //   [T; R] raw (16 KiB) after V
-constexpr uint32_t F_R1 = 128 * LD * 4;                  // dU [64][LD] + dO [64][LD] | dS' [128][LD]
+constexpr int L6 = 68;                                   // fp32 row stride of 64-wide tiles
+constexpr uint32_t F_R0 = 0;                             // V [64][LD] + T, R [64][L6] | S [128][LD]
+constexpr uint32_t F_T = 64 * LD * 4;                    //   T [64][L6] after V
+constexpr uint32_t F_RR = F_T + 64 * L6 * 4;             //   R [64][L6]
+constexpr uint32_t F_R1 = F_RR + 64 * L6 * 4;           // dU [64][LD] + dO [64][LD] | dS' [128][LD]
 constexpr uint32_t F_R2 = F_R1 + 128 * LD * 4;           // U [64][LD] (dV first)
-constexpr uint32_t F_WP = F_R2 + 64 * LD * 4;            // [-W; P] raw (32 KiB)
-constexpr uint32_t F_SMEM = F_WP + 32768;
-static_assert(F_TR + 16384 <= F_R1, "factor kernel layout");
+constexpr uint32_t F_WN = F_R2 + 64 * LD * 4;            // -W [64][LD]
+constexpr uint32_t F_SMEM = F_WN + 64 * LD * 4;
+static_assert(128 * LD * 4 <= F_R1, "factor kernel layout: S fits the first region");
+static_assert(F_SMEM <= 227 * 1024, "factor kernel shared memory");
 
 // (sequence, chunk within it) of a global chunk index: equal-length arithmetic,
 // or the last sequence whose first chunk is <= cidx (binary search)
@@ -281,11 +298,12 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     const size_t item = (size_t)cidx * H + h;
     const uint8_t *slot = fws + hdr_bytes + item * kSlotBytes;
     float *V = reinterpret_cast<float *>(sm + F_R0);
-    const uint8_t *trw = sm + F_TR;          // [T; R] raw (offsets tr_off - kSlotTR)
+    float *Tf = reinterpret_cast<float *>(sm + F_T);
+    float *Rf = reinterpret_cast<float *>(sm + F_RR);
     float *dU = reinterpret_cast<float *>(sm + F_R1);
     float *dO = dU + 64 * LD;
     float *U = reinterpret_cast<float *>(sm + F_R2);
-    const uint8_t *wpw = sm + F_WP;          // [-W; P] raw (offsets wp_off)
+    float *Wnf = reinterpret_cast<float *>(sm + F_WN);
     float *out = fg + item * FG_FLOATS;
 
     // ---- phase 1: V, dU, dO, [T; R] and [-W; P] in shared memory
@@ -295,13 +313,18 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
         dU[t * LD + c] = ws_dU[(item * 64 + t) * D + c];
         dO[t * LD + c] = t < L ? dout[((size_t)(t0 + t) * H + h) * D + c] : 0.f;
     }
-    for (int i = tid; i < 16384 / 16; i += NT)
-        reinterpret_cast<uint4 *>(sm + F_TR)[i] = reinterpret_cast<const uint4 *>(slot + kSlotTR)[i];
-    for (int i = tid; i < 32768 / 16; i += NT)
-        reinterpret_cast<uint4 *>(sm + F_WP)[i] = reinterpret_cast<const uint4 *>(slot + kSlotWP)[i];
+    for (int i = tid; i < 64 * 64; i += NT) {
+        const int r = i >> 6, s2 = i & 63;
+        Tf[r * L6 + s2] = h2f(slot, tr_off(r, s2));
+        Rf[r * L6 + s2] = h2f(slot, tr_off(64 + r, s2));
+    }
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int t = i >> 7, c = i & 127;
+        Wnf[t * LD + c] = h2f(slot, wp_off(t, c));
+    }
     __syncthreads();
-    auto Tm = [&](int r, int s) { return h2f(trw, tr_off(r, s) - kSlotTR); };        // T[r][s]
-    auto Rm = [&](int r, int s) { return h2f(trw, tr_off(64 + r, s) - kSlotTR); };   // R[r][s]
+    auto Tm = [&](int r, int s2) { return Tf[r * L6 + s2]; };   // T[r][s]
+    auto Rm = [&](int r, int s2) { return Rf[r * L6 + s2]; };   // R[r][s]
     // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out)
     smm<64, 128, 64>([&](int s, int t) { return Tm(t, s); }, [&](int t, int c) { return dU[t * LD + c]; },
                      [&](int s, int c, float x) { U[s * LD + c] = x; });
@@ -334,7 +357,7 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     }
     __syncthreads();
     // U += (-W) S   (the slot holds -W)
-    smm<64, 128, 128>([&](int t, int c) { return h2f(wpw, wp_off(t, c)); },
+    smm<64, 128, 128>([&](int t, int c) { return Wnf[t * LD + c]; },
                       [&](int c, int jj) { return S[c * LD + jj]; },
                       [&](int t, int jj, float x) { U[t * LD + jj] += x; });
     // dW = -dU S^T, dP = dO S^T
@@ -469,7 +492,6 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                     const Tin *__restrict__ beta, const float *__restrict__ fg,
                     float *__restrict__ iw) {
     extern __shared__ __align__(16) uint8_t sm[];
-    constexpr int L6 = 68;   // row stride of 64 x 64 tiles
     const int tid = threadIdx.x;
     const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
     const bool packed = cu != nullptr;
@@ -493,13 +515,20 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     float *dRp = dTp + 64 * L6;                            // dR'
     float *Wk = dRp + 64 * L6;                             // scratch [64][L6]
     float *Kt = Wk + 64 * L6;                              // K * Gamma  [64][LD]
-    float *bs = Kt + 64 * LD;                              // beta [64]
+    float *dPs = Kt + 64 * LD;                             // dP [64][LD]
+    float *dWs = dPs + 64 * LD;                            // dW [64][LD]
+    float *bs = dWs + 64 * LD;                             // beta [64]
     for (int i = tid; i < 64 * 64; i += NT) {
         const int r = i >> 6, s = i & 63;
         Aq[r * L6 + s] = io[IW_AQK + i];
         Mm[r * L6 + s] = io[IW_M + i];
     }
     if (tid < 64) bs[tid] = tid < L ? to_f32(beta[(size_t)(t0 + tid) * H + h]) : 0.f;
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int t = i >> 7, c = i & 127;
+        dPs[t * LD + c] = fgi[FG_DP + i];
+        dWs[t * LD + c] = fgi[FG_DW + i];
+    }
     if (tid < 128) {   // K * Gamma, Gamma = exp(cumsum(max(g, -5)))
         float acc = 0.f;
         for (int r = 0; r < 64; ++r) {
@@ -532,16 +561,16 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                     [&](int r, int s, float x) { Rm[r * L6 + s] = x; });
     __syncthreads();
     // dR' = dR - dP (K Gamma)^T
-    smm<64, 64, 128>([&](int t, int c) { return fgi[FG_DP + t * 128 + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
+    smm<64, 64, 128>([&](int t, int c) { return dPs[t * LD + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
                      [&](int t, int s, float x) { dRp[t * L6 + s] = fgi[FG_DR + t * 64 + s] - x; });
     // dT'_0 = dT + dW (K Gamma)^T
-    smm<64, 64, 128>([&](int t, int c) { return fgi[FG_DW + t * 128 + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
+    smm<64, 64, 128>([&](int t, int c) { return dWs[t * LD + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
                      [&](int t, int s, float x) { dTp[t * L6 + s] = fgi[FG_DT + t * 64 + s] + x; });
     // dKt = T^T dW - R^T dP  -> workspace
-    smm<64, 128, 64>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return fgi[FG_DW + t * 128 + c]; },
+    smm<64, 128, 64>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return dWs[t * LD + c]; },
                      [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] = x; });
     __syncthreads();
-    smm<64, 128, 64>([&](int s, int t) { return Rm[t * L6 + s]; }, [&](int t, int c) { return fgi[FG_DP + t * 128 + c]; },
+    smm<64, 128, 64>([&](int s, int t) { return Rm[t * L6 + s]; }, [&](int t, int c) { return dPs[t * LD + c]; },
                      [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] -= x; });
     // dT' += Aqk^T dR'
     smm<64, 64, 64>([&](int r, int m) { return Aq[m * L6 + r]; }, [&](int m, int s) { return dRp[m * L6 + s]; },
@@ -597,12 +626,13 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     const float *io = iw + item * IW_FLOATS;
     const float *fgi = fg + item * FG_FLOATS;
     float *G = reinterpret_cast<float *>(sm);             // [64][LD]
-    float *AE = G + 64 * LD;                               // a_r E1_r (q or k)
-    float *KF = AE + 64 * LD;                              // k_s exp(R_a - G_s), block a's
+    float *KF = G + 64 * LD;                               // exp(R_a - G_s), block a's
     float *dG = KF + 64 * LD;                              // dG accumulator
     float *Dq = dG + 64 * LD;                              // dq accumulator
     float *Dk = Dq + 64 * LD;                              // dk accumulator
-    float *Rref = Dk + 64 * LD;                            // [4][128]
+    float *KK = Dk + 64 * LD;                              // k_s exp(R_a - G_s)
+    float *AE = KK + 64 * LD;                              // a_r E1_r for the 16 rows of block a
+    float *Rref = AE + 16 * LD;                            // [4][128]
     chunk_cumsum(g, t0, H, h, L, G, Rref);
     __syncthreads();
     auto qv = [&](int r, int c) { return r < L ? to_f32(q[((size_t)(t0 + r) * H + h) * D + c]) : 0.f; };
@@ -622,23 +652,22 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     // decayed adjoints: first Aqk with (a, b) = (q, k), then M with (k, k)
     for (int form = 0; form < 2; ++form) {
         const float *dF = io + (form == 0 ? IW_DAQK : IW_DM);
-        __syncthreads();
-        for (int i = tid; i < 64 * 128; i += NT) {
-            const int r = i >> 7, c = i & 127;
-            const float e1 = __expf(G[r * LD + c] - Rref[(r >> 4) * 128 + c]);
-            AE[r * LD + c] = (form == 0 ? qv(r, c) : kv(r, c)) * e1;
-        }
         for (int a = 0; a < 4; ++a) {
             const int ns = 16 * (a + 1);
             __syncthreads();
             for (int i = tid; i < 64 * 128; i += NT) {
                 const int s = i >> 7, c = i & 127;
                 KF[s * LD + c] = s < ns ? __expf(Rref[a * 128 + c] - G[s * LD + c]) : 0.f;   // exp(R_a - G_s)
+                KK[s * LD + c] = kv(s, c) * KF[s * LD + c];                                     // k_s exp(R_a - G_s)
+            }
+            for (int i = tid; i < 16 * 128; i += NT) {
+                const int r = i >> 7, c = i & 127, rr = 16 * a + r;
+                AE[r * LD + c] = (form == 0 ? qv(rr, c) : kv(rr, c)) * __expf(G[rr * LD + c] - Rref[a * 128 + c]);
             }
             __syncthreads();
             // da_r (rows of block a) = E1_r sum_s dF[r,s] b_s exp(R_a - G_s), b = k
             smm<16, 128, 64>([&](int r, int s) { return dF[(16 * a + r) * 64 + s]; },
-                             [&](int s, int c) { return kv(s, c) * KF[s * LD + c]; },
+                             [&](int s, int c) { return KK[s * LD + c]; },
                              [&](int r, int c, float x) {
                                  const int rr = 16 * a + r;
                                  const float da = x * __expf(G[rr * LD + c] - Rref[a * 128 + c]);
@@ -648,7 +677,7 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                              });
             // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s <= 16a + 15
             smm<64, 128, 16>([&](int s, int r) { return dF[(16 * a + r) * 64 + s]; },
-                             [&](int r, int c) { return AE[(16 * a + r) * LD + c]; },
+                             [&](int r, int c) { return AE[r * LD + c]; },
                              [&](int s, int c, float x) {
                                  if (s >= ns) return;
                                  const float db = x * KF[s * LD + c];
@@ -770,13 +799,15 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
                                                          (const bf *)a.k, (const bf *)a.g, iw);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t PB_SMEM = 7 * 64 * 68 * 4 + 64 * LD * 4 + 64 * 4;
+    constexpr uint32_t PB_SMEM = 7 * 64 * L6 * 4 + 3 * 64 * LD * 4 + 64 * 4;
+    static_assert(PB_SMEM <= 227 * 1024, "pull-back shared memory");
     if ((e = set_smem(bwd_pullback_kernel<bf>, PB_SMEM)) != cudaSuccess) return e;
     bwd_pullback_kernel<bf><<<items, NT, PB_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.k,
                                                         (const bf *)a.g, (const bf *)a.beta, fg, iw);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t AS_SMEM = 6 * 64 * LD * 4 + 4 * 128 * 4;
+    constexpr uint32_t AS_SMEM = 6 * 64 * LD * 4 + 16 * LD * 4 + 4 * 128 * 4;
+    static_assert(AS_SMEM <= 227 * 1024, "assembly shared memory");
     if ((e = set_smem(bwd_assemble_kernel<bf>, AS_SMEM)) != cudaSuccess) return e;
     bwd_assemble_kernel<bf><<<items, NT, AS_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
                                                         (const bf *)a.k, (const bf *)a.g, fg, iw, a.dq,

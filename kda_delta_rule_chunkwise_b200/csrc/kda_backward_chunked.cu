@@ -23,6 +23,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "sm100.cuh"
@@ -538,24 +540,40 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
         }
     }
     __syncthreads();
-    // X: column i of (I + Diag(beta) M)^-1 by forward substitution, four partial sums
+    // X = (I + A)^-1, A = Diag(beta) M (strictly lower), by 16 x 16 blocks: the
+    // diagonal blocks by forward substitution (thread = block a, column j), then
+    // block row i from the rows above: X[i, 0:i] = -X_ii (A[i, 0:i] X[0:i, 0:i])
+    for (int i = tid; i < 64 * 64; i += NT) X[(i >> 6) * L6 + (i & 63)] = 0.f;
+    __syncthreads();
     if (tid < 64) {
-        const int col = tid;
-        for (int r = 0; r < 64; ++r) {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            int m = col;
-            for (; m + 3 < r; m += 4) {
-                a0 = fmaf(Mm[r * L6 + m], X[m * L6 + col], a0);
-                a1 = fmaf(Mm[r * L6 + m + 1], X[(m + 1) * L6 + col], a1);
-                a2 = fmaf(Mm[r * L6 + m + 2], X[(m + 2) * L6 + col], a2);
-                a3 = fmaf(Mm[r * L6 + m + 3], X[(m + 3) * L6 + col], a3);
-            }
-            for (; m < r; ++m) a0 = fmaf(Mm[r * L6 + m], X[m * L6 + col], a0);
-            const float sum = (a0 + a1) + (a2 + a3);
-            X[r * L6 + col] = r < col ? 0.f : ((r == col ? 1.f : 0.f) - bs[r] * sum);
+        const int a = tid >> 4, jc = tid & 15, o = 16 * a;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = r == jc ? 1.f : 0.f;
+#pragma unroll
+            for (int m = 0; m < r; ++m) acc = fmaf(-bs[o + r] * Mm[(o + r) * L6 + o + m], x[m], acc);
+            x[r] = acc;
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) X[(o + r) * L6 + o + jc] = x[r];
     }
     __syncthreads();
+    auto block_row = [&](auto ic) {
+        constexpr int I = decltype(ic)::value, W = 16 * I;
+        // Wk[r][m] = sum_{p < W} A[16I + r][p] X[p][m]
+        smm<16, W, W>([&](int r, int p) { return bs[16 * I + r] * Mm[(16 * I + r) * L6 + p]; },
+                      [&](int p, int m) { return X[p * L6 + m]; },
+                      [&](int r, int m, float v) { Wk[r * L6 + m] = v; });
+        __syncthreads();
+        smm<16, W, 16>([&](int r, int p) { return X[(16 * I + r) * L6 + 16 * I + p]; },
+                       [&](int p, int m) { return Wk[p * L6 + m]; },
+                       [&](int r, int m, float v) { X[(16 * I + r) * L6 + m] = -v; });
+        __syncthreads();
+    };
+    block_row(std::integral_constant<int, 1>{});
+    block_row(std::integral_constant<int, 2>{});
+    block_row(std::integral_constant<int, 3>{});
     // R = Aqk T, T = X Diag(beta)
     smm<64, 64, 64>([&](int r, int m) { return Aq[r * L6 + m]; }, [&](int m, int s) { return X[m * L6 + s] * bs[s]; },
                     [&](int r, int s, float x) { Rm[r * L6 + s] = x; });
@@ -632,7 +650,8 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     float *Dk = Dq + 64 * LD;                              // dk accumulator
     float *KK = Dk + 64 * LD;                              // k_s exp(R_a - G_s)
     float *AE = KK + 64 * LD;                              // a_r E1_r for the 16 rows of block a
-    float *Rref = AE + 16 * LD;                            // [4][128]
+    float *dFs = AE + 16 * LD;                             // dAqk, then dM  [64][L6]
+    float *Rref = dFs + 64 * L6;                           // [4][128]
     chunk_cumsum(g, t0, H, h, L, G, Rref);
     __syncthreads();
     auto qv = [&](int r, int c) { return r < L ? to_f32(q[((size_t)(t0 + r) * H + h) * D + c]) : 0.f; };
@@ -651,7 +670,10 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     }
     // decayed adjoints: first Aqk with (a, b) = (q, k), then M with (k, k)
     for (int form = 0; form < 2; ++form) {
-        const float *dF = io + (form == 0 ? IW_DAQK : IW_DM);
+        const float *dF = dFs;
+        __syncthreads();   // the previous form's products are done with dFs
+        for (int i = tid; i < 64 * 64; i += NT)
+            dFs[(i >> 6) * L6 + (i & 63)] = io[(form == 0 ? IW_DAQK : IW_DM) + i];
         for (int a = 0; a < 4; ++a) {
             const int ns = 16 * (a + 1);
             __syncthreads();
@@ -666,7 +688,7 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
             }
             __syncthreads();
             // da_r (rows of block a) = E1_r sum_s dF[r,s] b_s exp(R_a - G_s), b = k
-            smm<16, 128, 64>([&](int r, int s) { return dF[(16 * a + r) * 64 + s]; },
+            smm<16, 128, 64>([&](int r, int s) { return dF[(16 * a + r) * L6 + s]; },
                              [&](int s, int c) { return KK[s * LD + c]; },
                              [&](int r, int c, float x) {
                                  const int rr = 16 * a + r;
@@ -676,7 +698,7 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                                  dG[rr * LD + c] += av * da;
                              });
             // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s <= 16a + 15
-            smm<64, 128, 16>([&](int s, int r) { return dF[(16 * a + r) * 64 + s]; },
+            smm<64, 128, 16>([&](int s, int r) { return dF[(16 * a + r) * L6 + s]; },
                              [&](int r, int c) { return AE[r * LD + c]; },
                              [&](int s, int c, float x) {
                                  if (s >= ns) return;
@@ -806,7 +828,7 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
                                                         (const bf *)a.g, (const bf *)a.beta, fg, iw);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t AS_SMEM = 6 * 64 * LD * 4 + 16 * LD * 4 + 4 * 128 * 4;
+    constexpr uint32_t AS_SMEM = 6 * 64 * LD * 4 + 16 * LD * 4 + 64 * L6 * 4 + 4 * 128 * 4;
     static_assert(AS_SMEM <= 227 * 1024, "assembly shared memory");
     if ((e = set_smem(bwd_assemble_kernel<bf>, AS_SMEM)) != cudaSuccess) return e;
     bwd_assemble_kernel<bf><<<items, NT, AS_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,

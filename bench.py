@@ -255,14 +255,18 @@ def run_ours(args, rank, world, dev):
         clk.__exit__(None, None, None)
 
 
-def prefill_kernel_names(d):
-    """The kernels one prefill call launches for these inputs, in launch order: the
-    tensor-core path (bf16, d = 128) runs the chunk table (packed sequences only),
-    the intra-chunk products and the state pass; fp32 and d = 64 run one SIMT kernel."""
+def prefill_kernel_names(d, n_timed):
+    """The kernels one prefill call launches for these inputs, in launch order, given
+    how many the profiler timed: the tensor-core path (bf16, d = 128) runs the chunk
+    table (packed sequences only), then either one kernel for both phases (few
+    (sequence, head) units) or the intra-chunk products and the state pass; fp32 and
+    d = 64 run one SIMT kernel."""
     if d.q.dtype != torch.bfloat16 or d.dk != 128:
         return ["prefill_f32_kernel"]
-    return (["chunk_table_kernel"] if d.cu_seqlens is not None else []) + \
-        ["intra_chunk_kernel", "state_pass_kernel"]
+    table = ["chunk_table_kernel"] if d.cu_seqlens is not None else []
+    if n_timed == len(table) + 1:
+        return table + ["prefill_fused_kernel"]
+    return table + ["intra_chunk_kernel", "state_pass_kernel"]
 
 
 def prefill_units(d):
@@ -286,6 +290,7 @@ def algorithmic_bytes(d, tokens):
         "state_pass_kernel": th * (V_BYTES + O_BYTES_ALGO) + states,
     }
     path = th * PREFILL_BYTES_PER_TOKEN_HEAD + states
+    per["prefill_fused_kernel"] = path
     per["prefill_f32_kernel"] = path
     return path, per, path + th * (O_BYTES_WRITTEN - O_BYTES_ALGO)
 
@@ -300,7 +305,7 @@ def measure_prefill(binding, d, steps, warmup, peaks, world, dev, o, s_out, ws):
     # per-kernel device time: a second, profiled pass on the same inputs (events on
     # the launching stream around each kernel)
     per = time_prefill(binding, d, o, s_out, ws, max(2, steps), 1, profile=True)
-    names = prefill_kernel_names(d)
+    names = prefill_kernel_names(d, len(per[0]))
     assert all(len(p) == len(names) for p in per), (names, per[0])
     k_avg = [sum(p[i] for p in per) / len(per) for i in range(len(names))]
     path_bytes, k_bytes, path_bytes_o32 = algorithmic_bytes(d, tokens)
@@ -520,9 +525,14 @@ def _run_ours_timed(args, rank, world, dev, binding, kin, peaks, w, d, B, T, H, 
         bstep()
         kms = binding.kda_profile_last(16)
         binding.kda_profile_enable(False)
-        names = ["chunk_table_kernel"] if len(kms) == 8 else []
-        names += ["intra_chunk_kernel (forward)", "state_pass_kernel (forward, snapshots every chunk)",
-                  "bwd_chain_kernel", "bwd_factor_kernel", "bwd_recompute_kernel",
+        # the forward is one kernel (both phases) or two; packed sequences add the table
+        table = ["chunk_table_kernel"] if bw.cu_seqlens is not None else []
+        fwd = (["prefill_fused_kernel (forward, snapshots every chunk)"]
+               if len(kms) - len(table) == 6
+               else ["intra_chunk_kernel (forward)",
+                     "state_pass_kernel (forward, snapshots every chunk)"])
+        names = table + fwd
+        names += ["bwd_chain_kernel", "bwd_factor_kernel", "bwd_recompute_kernel",
                   "bwd_pullback_kernel", "bwd_assemble_kernel"]
         extra["backward"] = {"workload": "prefill_h32_t8192_d128", "steps": nb,
                              "ms_per_step": round(b_ms / nb, 3),

@@ -89,6 +89,44 @@ __device__ __forceinline__ void smm(FA A, FB B, FO out) {
         for (int b = 0; b < TN; ++b) out(ty + 16 * a, tx + 16 * b, r[a][b]);
 }
 
+// The same product when both operands are row-major fp32 with K contiguous:
+// out(i, j, sum_k A[i][k] B[j][k]) (A times B transposed), four k at a time as
+// 16-byte loads (lda, ldb multiples of 4, K a multiple of 4).  Same thread
+// mapping and summation order as smm.
+template <int M, int N, int K, typename FO>
+__device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, int ldb, FO out) {
+    constexpr int TM = M / 16, TN = N / 16;
+    static_assert(M % 16 == 0 && N % 16 == 0 && K % 4 == 0, "tile");
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float r[TM][TN];
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < TN; ++b) r[a][b] = 0.f;
+#pragma unroll 2
+    for (int k = 0; k < K; k += 4) {
+        float4 av[TM], bv[TN];
+#pragma unroll
+        for (int a = 0; a < TM; ++a) av[a] = *reinterpret_cast<const float4 *>(A + (ty + 16 * a) * lda + k);
+#pragma unroll
+        for (int b = 0; b < TN; ++b) bv[b] = *reinterpret_cast<const float4 *>(B + (tx + 16 * b) * ldb + k);
+#pragma unroll
+        for (int a = 0; a < TM; ++a)
+#pragma unroll
+            for (int b = 0; b < TN; ++b) {
+                float x = r[a][b];
+                x = fmaf(av[a].x, bv[b].x, x);
+                x = fmaf(av[a].y, bv[b].y, x);
+                x = fmaf(av[a].z, bv[b].z, x);
+                r[a][b] = fmaf(av[a].w, bv[b].w, x);
+            }
+    }
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < TN; ++b) out(ty + 16 * a, tx + 16 * b, r[a][b]);
+}
+
 // rows [a, b) of sequence n: equal-length batch, or the chunk table's clamped offsets
 __device__ __forceinline__ void seq_rows(const int32_t *hdr, bool packed, int64_t T, int N, int n,
                                          int64_t &a, int64_t &b) {
@@ -338,10 +376,8 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
         if (s < L) dv[((size_t)(t0 + s) * H + h) * D + c] = U[s * LD + c];
     }
     // dT = dU V^T, dR = dO V^T
-    smm<64, 64, 128>([&](int t, int c) { return dU[t * LD + c]; }, [&](int c, int s) { return V[s * LD + c]; },
-                     [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; });
-    smm<64, 64, 128>([&](int t, int c) { return dO[t * LD + c]; }, [&](int c, int s) { return V[s * LD + c]; },
-                     [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; });
+    smm_nt<64, 64, 128>(dU, LD, V, LD, [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; });
+    smm_nt<64, 64, 128>(dO, LD, V, LD, [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; });
     __syncthreads();   // U's buffer (dV) is read out
     // U = T V
     smm<64, 128, 64>([&](int t, int s) { return Tm(t, s); }, [&](int s, int c) { return V[s * LD + c]; },
@@ -363,10 +399,8 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
                       [&](int c, int jj) { return S[c * LD + jj]; },
                       [&](int t, int jj, float x) { U[t * LD + jj] += x; });
     // dW = -dU S^T, dP = dO S^T
-    smm<64, 128, 128>([&](int t, int jj) { return dU[t * LD + jj]; }, [&](int jj, int c) { return S[c * LD + jj]; },
-                      [&](int t, int c, float x) { out[FG_DW + t * 128 + c] = -x; });
-    smm<64, 128, 128>([&](int t, int jj) { return dO[t * LD + jj]; }, [&](int jj, int c) { return S[c * LD + jj]; },
-                      [&](int t, int c, float x) { out[FG_DP + t * 128 + c] = x; });
+    smm_nt<64, 128, 128>(dU, LD, S, LD, [&](int t, int c, float x) { out[FG_DW + t * 128 + c] = -x; });
+    smm_nt<64, 128, 128>(dO, LD, S, LD, [&](int t, int c, float x) { out[FG_DP + t * 128 + c] = x; });
     __syncthreads();   // dU and dO are consumed
 
     // ---- phase 3: dS'
@@ -382,8 +416,7 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
         out[FG_DGL + tid] = a;
     }
     // dKhat = U dS'^T
-    smm<64, 128, 128>([&](int t, int jj) { return U[t * LD + jj]; }, [&](int jj, int c) { return dSp[c * LD + jj]; },
-                      [&](int t, int c, float x) { out[FG_DKH + t * 128 + c] = x; });
+    smm_nt<64, 128, 128>(U, LD, dSp, LD, [&](int t, int c, float x) { out[FG_DKH + t * 128 + c] = x; });
 }
 
 
@@ -579,11 +612,9 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                     [&](int r, int s, float x) { Rm[r * L6 + s] = x; });
     __syncthreads();
     // dR' = dR - dP (K Gamma)^T
-    smm<64, 64, 128>([&](int t, int c) { return dPs[t * LD + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
-                     [&](int t, int s, float x) { dRp[t * L6 + s] = fgi[FG_DR + t * 64 + s] - x; });
+    smm_nt<64, 64, 128>(dPs, LD, Kt, LD, [&](int t, int s, float x) { dRp[t * L6 + s] = fgi[FG_DR + t * 64 + s] - x; });
     // dT'_0 = dT + dW (K Gamma)^T
-    smm<64, 64, 128>([&](int t, int c) { return dWs[t * LD + c]; }, [&](int c, int s) { return Kt[s * LD + c]; },
-                     [&](int t, int s, float x) { dTp[t * L6 + s] = fgi[FG_DT + t * 64 + s] + x; });
+    smm_nt<64, 64, 128>(dWs, LD, Kt, LD, [&](int t, int s, float x) { dTp[t * L6 + s] = fgi[FG_DT + t * 64 + s] + x; });
     // dKt = T^T dW - R^T dP  -> workspace
     smm<64, 128, 64>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return dWs[t * LD + c]; },
                      [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] = x; });
@@ -602,7 +633,7 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                     [&](int r, int s, float x) { Wk[r * L6 + s] = x; });
     __syncthreads();
     // dAkk = strict_tril(-Wk X^T), dM = Diag(beta) dAkk -> workspace; dAkk * M row sums
-    smm<64, 64, 64>([&](int r, int m) { return Wk[r * L6 + m]; }, [&](int m, int s) { return X[s * L6 + m]; },
+    smm_nt<64, 64, 64>(Wk, L6, X, L6,
                     [&](int r, int s, float x) {
                         const float dakk = s < r ? -x : 0.f;
                         Rm[r * L6 + s] = dakk;                       // R is consumed: reuse for dAkk

@@ -145,4 +145,60 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t pari
     return false;
 }
 
+// ---------------------------------------------------------------- ready words
+// A 32-bit word in device memory that one CTA sets (release) and another waits
+// for (acquire), within one launch.
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Eight consecutive words (32-byte aligned) by one acquire load.
+__device__ __forceinline__ void ld_acquire_gpu_v8(const uint32_t *p, uint32_t (&w)[8]) {
+    asm volatile("ld.acquire.gpu.global.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
+                   "=r"(w[6]), "=r"(w[7])
+                 : "l"(p)
+                 : "memory");
+}
+
+// Orders this thread's generic-proxy accesses to global memory with its later
+// (or, on the writing side, earlier) async-proxy accesses: bulk and TMA copies.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *word == value, with the abort rules of mbar_wait_abortable.
+// Polls back off with a short sleep (the word lives in L2).
+__device__ __forceinline__ bool word_wait_abortable(const uint32_t *word, uint32_t value,
+                                                    uint32_t *err, uint32_t epoch,
+                                                    volatile uint32_t *abort,
+                                                    uint64_t limit_ns = kWaitLimitNs) {
+    if (ld_acquire_gpu(word) == value) return true;
+    const uint64_t t0 = globaltimer_ns();
+    const volatile uint32_t *gepoch = err ? err + 1 : nullptr;
+    for (;;) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(word) == value) return true;
+        if (*abort) return false;
+        const uint64_t dt = globaltimer_ns() - t0;
+        if (dt > kSlowWaitNs) {
+            if (gepoch && *gepoch == epoch) {
+                *abort = 1u;
+                return false;
+            }
+            if (dt > limit_ns) break;
+        }
+    }
+    record_timeout(err, epoch);
+    *abort = 1u;
+    return false;
+}
+
 }  // namespace kda

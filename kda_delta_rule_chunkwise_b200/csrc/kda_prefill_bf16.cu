@@ -81,6 +81,10 @@ constexpr uint32_t kKhMNBlock = 8192;    // bytes between the two 64-channel MN-
 // decreasing chunk count, so that the state pass starts the longest chains
 // first; identity order past kOrderMaxN sequences).  Then the slots, 1024-aligned.
 constexpr int kOrderMaxN = 8192;
+// Ready words of the one-launch form: one per (chunk, head) item, head-major with
+// each head's row padded to a multiple of 8 words (32 bytes), so that eight
+// consecutive chunks of a head are read by two aligned 16-byte loads.
+__host__ __device__ inline int ready_stride(int chunks) { return (chunks + 7) & ~7; }
 __host__ __device__ inline uint32_t header_bytes(int N) {
     return (uint32_t)(((size_t)(N + 1) * 16 + 1023) & ~(size_t)1023);
 }
@@ -249,7 +253,8 @@ constexpr uint32_t A_M_EL = 1792;     //   fp32 [4][128]
 constexpr uint32_t A_M_PF = 3840;     //   fp32 [2][128]: F_0 F_1 and F_0 F_1 F_2
 constexpr uint32_t A_M_BARS = 4864;   //   8 mbarriers
 constexpr uint32_t A_M_TMEM = 4928;   //   TMEM base address + abort flag
-constexpr uint32_t A_M_END = 4936;
+constexpr uint32_t A_M_NEXT = 4936;   //   next item (from the device counter)
+constexpr uint32_t A_M_END = 4940;
 constexpr uint32_t A_OPS = 37888;     // operand region (two uses, below)
 static_assert(A_MISC + A_M_END <= A_OPS, "phase A misc region overflows into the operands");
 static_assert(A_M_BARS % 8 == 0 && A_M_F % 16 == 0 && A_M_EL % 16 == 0 && A_M_PF % 16 == 0,
@@ -332,15 +337,20 @@ __device__ __forceinline__ float4 rcp4(float4 a) {
 // compiles without any of it.
 // q, k and g arrive as TMA tiles (tensor maps over [rows, H, 128] bf16, boxes of
 // 64 channels x 64 rows); beta is read per row.
+//
+// The body runs in two kernels.  cta and ncta are this CTA's index among the
+// CTAs that run phase A and their number.  sched == nullptr: the CTA takes
+// items cta, cta + ncta, ...; otherwise each item comes from the device counter
+// *sched (zero before the launch), so items go out in increasing order, chunk
+// by chunk, to whichever CTA is free.  ready != nullptr: once an item's slot is
+// complete in device memory it is published by a release store of the launch's
+// epoch into ready[item].
 template <bool PREP>
-__global__ void __launch_bounds__(256, 2)
-intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16 *__restrict__ beta,
-                   const int32_t *__restrict__ cu, int64_t T, int N, int H, uint32_t flags,
-                   uint8_t *__restrict__ ws, uint32_t *err, uint32_t epoch) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+__device__ __forceinline__ void intra_chunk_body(
+    const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_g,
+    const __nv_bfloat16 *__restrict__ beta, const int32_t *__restrict__ cu, int64_t T, int N, int H,
+    uint32_t flags, uint8_t *__restrict__ ws, uint32_t *err, uint32_t epoch, uint8_t *sm, int cta,
+    int ncta, uint32_t *sched, uint32_t *ready) {
     const uint32_t sbase = smem_u32(sm);
     float *E1 = reinterpret_cast<float *>(sm + A_E1);
     float *bs = reinterpret_cast<float *>(sm + A_MISC + A_M_BETA);    // [64]
@@ -350,6 +360,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + A_MISC + A_M_BARS);   // [8]
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + A_MISC + A_M_TMEM);
     volatile uint32_t *abort_flag = tmem_ptr + 1;
+    volatile int *s_next = reinterpret_cast<volatile int *>(sm + A_MISC + A_M_NEXT);
     // used only inside A0, before any operand round: parked in the operand region
     float *tot = reinterpret_cast<float *>(sm + A_A0S);              // [3][128] half sums
     float *GLv = tot + 3 * 128;                                       // [128] G_L
@@ -408,9 +419,9 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_arrive_expect_tx(&bars[6], 3 * 16384);
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk) {
-                tma_load_3d(sm + A_QST + blk * 8192, &tm_q, 64 * blk, hn, (int)t0n, &bars[6]);
-                tma_load_3d(sm + A_KST + blk * 8192, &tm_k, 64 * blk, hn, (int)t0n, &bars[6]);
-                tma_load_3d(sm + A_GST + blk * 8192, &tm_g, 64 * blk, hn, (int)t0n, &bars[6]);
+                tma_load_3d(sm + A_QST + blk * 8192, tm_q, 64 * blk, hn, (int)t0n, &bars[6]);
+                tma_load_3d(sm + A_KST + blk * 8192, tm_k, 64 * blk, hn, (int)t0n, &bars[6]);
+                tma_load_3d(sm + A_GST + blk * 8192, tm_g, 64 * blk, hn, (int)t0n, &bars[6]);
             }
         }
         ++loads_issued;
@@ -426,21 +437,34 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int i = 4; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
         *abort_flag = 0u;
+        *s_next = sched ? (int)atomicAdd(sched, 1u) : cta;
     }
     __syncthreads();
-    if ((int64_t)blockIdx.x < n_items) prefetch(blockIdx.x);
+    const int first_item = *s_next;
+    if ((int64_t)first_item < n_items) prefetch(first_item);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
 
+    // publish a finished item: the slot's generic stores (all threads, ordered by
+    // the CTA barrier before this call) and this thread's bulk store of [T; R]
+    // are complete before the release store of the epoch
+    auto publish = [&](int it) {
+        bulk_wait_all();
+        fence_proxy_async_global();
+        st_release_gpu(ready + (size_t)(it % H) * ready_stride((int)(n_items / H)) + it / H, epoch);
+    };
     uint32_t ph = 0;   // mbarrier phase parity: each barrier completes once per item
+    int prev_item = -1, next_item = 0;
     // (items fit in int32: the host checks max_chunks * H against INT32_MAX)
-    for (int item = blockIdx.x; item < (int)n_items; item += gridDim.x, ph ^= 1u) {
+    for (int item = first_item; item < (int)n_items; item = next_item, ph ^= 1u) {
     int64_t t0;
     int L;
     locate(item, t0, L);
     uint8_t *slot = ws + header_bytes(N) + (size_t)item * kSlotBytes;
+    // the next item from the counter (its value is needed only after a barrier)
+    const int claimed = (sched && tid == 0) ? (int)atomicAdd(sched, 1u) : 0;
 
     // ---- this item's rows have landed; rows past the chunk's end are zeroed
     const bool landed = mbar_wait_abortable(&bars[6], ph, err, epoch, abort_flag);
@@ -455,6 +479,8 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
     }
     if (__syncthreads_or(*abort_flag != 0u)) break;
+    if (ready && tid == 0 && prev_item >= 0) publish(prev_item);
+    prev_item = item;
     const int c = tid & 127, half = tid >> 7;
     float p[32];   // clamped log-decay of rows 32*half + i, then its prefix sums
 #pragma unroll
@@ -472,6 +498,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
     }
     if (tid < 64) bs[tid] = __bfloat162float(bnext);
+    if (tid == 0) *s_next = sched ? claimed : item + ncta;
     __syncthreads();
     // the g staging is free now: it holds 1 / |q_r| and 1 / |k_r| when q, k are to be
     // normalised here (two threads per row; a zero row stays zero)
@@ -867,7 +894,8 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // the staging regions are free once D1 has completed: the next item's rows go
     // out now (the bulk store of [T; R] is waited for before the next item's
     // operand rounds overwrite it)
-    if (ok && (int64_t)item + gridDim.x < n_items) prefetch(item + gridDim.x);
+    next_item = *s_next;
+    if (ok && (int64_t)next_item < n_items) prefetch(next_item);
 
     // ---- A6: rows 0..63 -> -W, rows 64..127 -> P = Q*Gamma - R (K*Gamma), in two
     // halves of 32 columns (fewer live registers)
@@ -918,10 +946,24 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
+    if (ready && tid == 0 && prev_item >= 0 && !*abort_flag) publish(prev_item);
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
+}
+
+template <bool PREP>
+__global__ void __launch_bounds__(256, 2)
+intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16 *__restrict__ beta,
+                   const int32_t *__restrict__ cu, int64_t T, int N, int H, uint32_t flags,
+                   uint8_t *__restrict__ ws, uint32_t *err, uint32_t epoch) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    intra_chunk_body<PREP>(&tm_q, &tm_k, &tm_g, beta, cu, T, N, H, flags, ws, err, epoch, sm,
+                           (int)blockIdx.x, (int)gridDim.x, nullptr, nullptr);
 }
 
 // ======================================================================
@@ -1379,15 +1421,530 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_v, const float *state_i
     }
 }
 
+
+// ======================================================================
+// One launch for both phases
+// ======================================================================
+// With few (sequence, head) units the state pass needs few CTAs, and run after
+// phase A it holds the GPU alone, latency-bound, for 40 % of the step.  In
+// prefill_fused_kernel the first CTAs run the state pass while the others run
+// phase A, taking items from a device counter in chunk order; phase A publishes
+// each finished slot (release store of the launch's epoch into its ready word)
+// and the state pass copies a slot in only after an acquire load has seen that
+// word.  Phase A never waits on the state pass, so the launch finishes whether
+// or not all of its CTAs are resident at once; every wait is bounded.
+//
+// The state pass here fits the launch's 256 threads and phase A's shared
+// memory: one copy of each slot part, in regions that free at different times
+// so that each is refilled while the chain works on something else:
+//   [T; R]: free once the V term [T; R] V has run (VDONE; the V term is issued
+//     as soon as its operands are in, ahead of the state), refilled during the
+//     rest of the chunk;
+//   the V slice (an input, read from device memory): two copies, loaded two
+//     chunks ahead;
+//   Gamma_L: two copies (the state copy of chunk j reads its own while chunk
+//     j + 1's lands);
+//   [-W; P]: free once the chunk products have completed (TDFULL), refilled
+//     during the U copy-out, the state update and the next state copy;
+//   Khat: free once the state update has completed (TSFULL), refilled during
+//     the state copy, the chunk products and the U copy-out.
+template <int DVS>
+struct FLayout {
+    static constexpr uint32_t oWP = 0;                   // slot bytes [0, 32768)
+    static constexpr uint32_t oTR = kSlotTR;             // slot bytes [32768, 49152)
+    static constexpr uint32_t oV = 49152;                // V slices, 2 x 64 rows x DVS
+    static constexpr uint32_t kVBytes = 64 * DVS * 2;
+    static constexpr uint32_t oGam = oV + 2 * kVBytes;   // Gamma_L, 2 x 128 fp32
+    static constexpr uint32_t kTTx = 16384 + 512;        // tx of one [T; R] + Gamma_L fill
+    static constexpr uint32_t oKh = (oGam + 1024 + 1023) & ~1023u;
+    static constexpr uint32_t oSB = oKh + 16384;         // fp16 S  (K=128 x N=DVS)
+    static constexpr uint32_t oUB = oSB + 128 * DVS * 2; // fp16 U  (K=64 x N=DVS)
+    static constexpr uint32_t oBar = oUB + 64 * DVS * 2;
+    static constexpr uint32_t kBytes = oBar + 256;
+    static constexpr uint32_t kKGroup = (DVS / 8) * 128;
+    static constexpr uint32_t kVLine = DVS == 32 ? 64 : 128;
+    static constexpr Swizzle kVSwz = DVS == 32 ? SW_64B : SW_128B;
+    static constexpr uint32_t kVSbo = 8 * kVLine;
+    static constexpr uint32_t kVLbo = 64 * kVLine;
+    static constexpr uint32_t kVKstep = 16 * kVLine;
+    static constexpr uint32_t kTmemCols = DVS == 32 ? 128 : 256;   // TD0, TD1, TS
+    static_assert(DVS == 32 || DVS == 64, "one-launch state pass slice");
+    static_assert(kBytes + 1024 <= A_SMEM, "state pass must fit phase A's shared memory");
+    static_assert(oV % 1024 == 0 && kVBytes % 512 == 0 && oKh % 1024 == 0 && oSB % 128 == 0 &&
+                  oUB % 128 == 0, "operand alignment");
+};
+
+enum FBar { F_WFULL = 0, F_TFULL, F_VFULL0, F_VFULL1, F_VREADY, F_VDONE, F_YFULL, F_TD0, F_TD1,
+            F_TSFULL, F_TSSCALED, F_DRAIN_S, F_DRAIN_U, F_NBARS };
+
+// Roles (256 threads): warps 0-3 state group (TMEM lane = key channel; fp16
+// copy of S, Gamma scaling; thread 0 issues the chunk products and every
+// copy); warps 4-7 U group (TMEM lane = row of [U; O]; U copy-out, O to
+// device memory, V conversion; thread 128 issues the state update).
+// Each barrier completes once per chunk, and no copy into a region is issued
+// before every waiter has passed the region's previous phase, so a parity wait
+// never meets a barrier two phases ahead.
+template <int DVS>
+__device__ __forceinline__ void state_pass_role(
+    const CUtensorMap *tm_v, const float *state_in, const int32_t *__restrict__ cu, int64_t T,
+    int N, int H, const uint8_t *__restrict__ ws, const uint32_t *ready, float *__restrict__ o,
+    float *state_out, int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity, uint32_t *err,
+    uint32_t epoch, uint8_t *sm, int cta) {
+    using Lay = FLayout<DVS>;
+    constexpr int NSL = D / DVS;
+    constexpr int CPR = DVS / 8;   // 16-byte pieces per V row
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::oBar);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + F_NBARS);
+    volatile uint32_t *abort_flag = tmem_ptr + 1;
+    volatile uint32_t *s_grp_ok = tmem_ptr + 2;   // state-group leader -> group
+    volatile uint32_t *s_u_ok = tmem_ptr + 3;     // U-group leader -> group
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int slice = cta % NSL, unit = cta / NSL;
+    const int32_t *chunk_off = reinterpret_cast<const int32_t *>(ws);
+    if (unit / H >= N) return;
+    const int n = cu ? chunk_off[3 * (N + 1) + unit / H] : unit / H, h = unit % H;
+    int64_t ra, rb;
+    seq_rows(chunk_off, cu != nullptr, T, N, n, ra, rb);
+    const int nch = (int)((rb - ra + C - 1) / C);
+    const int c0 = cu ? chunk_off[n] : n * (int)((T + C - 1) / C);
+    const int64_t ck0 = cu ? (int64_t)chunk_off[2 * (N + 1) + n]
+                           : (int64_t)n * ((T > 0 && ckpt_interval > 0) ? (T - 1) / ckpt_interval : 0);
+    const uint8_t *slots = ws + header_bytes(N);
+    const int j0 = slice * DVS;
+    const int nct_total = cu ? chunk_off[N] : N * (int)((T + C - 1) / C);   // chunks of the launch
+
+    if (warp == 0) {
+        tmem_alloc(tmem_ptr, Lay::kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < F_NBARS; ++i) mbar_init(&bars[i], 1);
+        mbar_fence_init();
+        *abort_flag = 0u;
+        *s_grp_ok = 1u;
+        *s_u_ok = 1u;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    const uint32_t tTD0 = tmem, tTD1 = tmem + DVS, tTS = tmem + 2 * DVS;
+    auto chunk_len = [&](int j) {
+        const int64_t t0 = ra + (int64_t)j * C;
+        return (int)((rb - t0) < C ? (rb - t0) : C);
+    };
+    auto slot_of = [&](int j) { return slots + ((size_t)(c0 + j) * H + h) * kSlotBytes; };
+    auto gam_buf = [&](int j) { return reinterpret_cast<float *>(sm + Lay::oGam + (j & 1) * 512); };
+    auto v_off = [&](int j) { return Lay::oV + (uint32_t)(j & 1) * Lay::kVBytes; };   // V slice of chunk j
+
+    if (warp < 4) {
+        // ------------------------------------------------ state group
+        // Only thread 0 (the leader) polls barriers and ready words; the group
+        // waits for it at named barriers, which take no issue slots from the
+        // phase A CTA that shares the SM.
+        const int c = tid;   // key channel = TMEM lane
+        const bool issuer = tid == 0;
+        const uint32_t tS = taddr(tTS, 32 * warp, 0);
+        const size_t srow = (((size_t)n * H + h) * D + c) * D + j0;
+        const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
+        uint8_t *sbp = sm + Lay::oSB;
+        // issuer bookkeeping: copies issued per region, V terms issued, ready words seen
+        int t_loads = 0, v_loads = 0, w_loads = 0, y_loads = 0, v_issued = -1, seen = c0 - 1;
+        const uint32_t *rrow = ready + (size_t)h * ready_stride(nct_total);
+        // chunk j's ready word observed (acquire) before any copy of its slot: eight
+        // words (consecutive chunks of this head) per 32-byte acquire load, one
+        // acquire load of the word itself when they are not all set
+        auto ensure_ready = [&](int j) {
+            const int cc = c0 + j;
+            if (cc <= seen) return true;
+            const int g = cc & ~7;
+            uint32_t w[8];
+            ld_acquire_gpu_v8(rrow + g, w);
+            int m = cc - 1;
+            bool run = true;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int ci = g + i;
+                if (run && ci >= cc && ci < c0 + nch) {
+                    if (w[i] == epoch) m = ci; else run = false;
+                }
+            }
+            if (m >= cc) {
+                seen = m;
+                return true;
+            }
+            if (!word_wait_abortable(rrow + cc, epoch, err, epoch, abort_flag)) return false;
+            seen = cc;
+            return true;
+        };
+        // [T; R] and Gamma_L of chunk j by bulk copy, after its ready word
+        auto load_t = [&](int j) {
+            if (!ensure_ready(j)) return false;
+            fence_proxy_async_global();
+            const uint8_t *src = slot_of(j);
+            mbar_arrive_expect_tx(&bars[F_TFULL], Lay::kTTx);
+            bulk_g2s(sm + Lay::oTR, src + kSlotTR, 16384, &bars[F_TFULL]);
+            bulk_g2s(gam_buf(j), src + kSlotGam, 512, &bars[F_TFULL]);
+            ++t_loads;
+            return true;
+        };
+        // the V slice of chunk j (an input: no ready word) into its copy by TMA
+        auto load_vs = [&](int j) {
+            uint64_t *bar = &bars[(j & 1) ? F_VFULL1 : F_VFULL0];
+            mbar_arrive_expect_tx(bar, Lay::kVBytes);
+            tma_load_3d(sm + v_off(j), tm_v, j0, h, (int)(ra + (int64_t)j * C), bar);
+            ++v_loads;
+        };
+        // [-W; P] and Khat of chunk j (its ready word was seen by load_t(j))
+        auto load_w = [&](int j) {
+            mbar_arrive_expect_tx(&bars[F_WFULL], 32768);
+            bulk_g2s(sm + Lay::oWP, slot_of(j), 32768, &bars[F_WFULL]);
+            ++w_loads;
+        };
+        auto load_y = [&](int j) {
+            mbar_arrive_expect_tx(&bars[F_YFULL], 16384);
+            bulk_g2s(sm + Lay::oKh, slot_of(j) + kSlotKh, 16384, &bars[F_YFULL]);
+            ++y_loads;
+        };
+        auto issue_vterm = [&](int j) {
+            const uint32_t tTD = (j & 1) ? tTD1 : tTD0;
+            const uint64_t ad0 = smem_desc(sbase + Lay::oTR, 16, 1024, SW_128B);
+            const uint64_t bd0 = smem_desc(sbase + v_off(j), Lay::kVLbo, Lay::kVSbo, Lay::kVSwz);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(tTD, ad0 + (uint64_t)(kk * 32 / 16), bd0 + (uint64_t)(kk * Lay::kVKstep / 16),
+                        id_nn, kk > 0);
+            mma_commit(&bars[F_VDONE]);
+            v_issued = j;
+        };
+        // fp16 copy of S (B operand of the state term) and TS <- Gamma * S
+        auto put_state = [&](const float *xa, float gam) {
+#pragma unroll
+            for (int p = 0; p < DVS / 16; ++p) {
+                const float *x = xa + 16 * p;
+                float y0[8], y1[8], z[16];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    y0[e] = x[e];
+                    y1[e] = x[8 + e];
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) z[e] = x[e] * gam;
+                tmem_st16(tS + 16 * p, z);
+                *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p, c, Lay::kKGroup)) =
+                    pack8(y0);
+                *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p + 8, c, Lay::kKGroup)) =
+                    pack8(y1);
+            }
+            tmem_wait_st();
+        };
+        // leader, after the group's state copy: release the state update of chunk j
+        // (TSSCALED) and issue [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j
+        auto issue_products = [&](int j) {
+            mbar_arrive(&bars[F_TSSCALED]);
+            if (v_issued < j) {
+                if (!mbar_wait_abortable(&bars[F_VREADY], j & 1, err, epoch, abort_flag)) return false;
+                tc_fence_after();
+                issue_vterm(j);
+            }
+            if (!mbar_wait_abortable(&bars[F_WFULL], j & 1, err, epoch, abort_flag)) return false;
+            tc_fence_after();
+            const uint32_t tTD = (j & 1) ? tTD1 : tTD0;
+            const uint64_t ad0 = smem_desc(sbase + Lay::oWP, 16, 1024, SW_128B);
+            const uint64_t bd0 = smem_desc(sbase + Lay::oSB, Lay::kKGroup, 128, SW_NONE);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_f16(tTD, ad0 + (uint64_t)(((kk >> 2) * kWPKBlock + (kk & 3) * 32) / 16),
+                        bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_nn, 1);
+            mma_commit(&bars[(j & 1) ? F_TD1 : F_TD0]);
+            return true;
+        };
+        if (nch == 0) {
+            if (state_out)
+                for (int i = 0; i < DVS / 4; ++i)
+                    reinterpret_cast<float4 *>(state_out + srow)[i] =
+                        state_in ? reinterpret_cast<const float4 *>(state_in + srow)[i]
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            bool ok = true;
+            float xa[DVS];
+#pragma unroll
+            for (int i = 0; i < DVS / 4; ++i) {
+                const float4 f = state_in ? reinterpret_cast<const float4 *>(state_in + srow)[i]
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                xa[4 * i] = f.x; xa[4 * i + 1] = f.y; xa[4 * i + 2] = f.z; xa[4 * i + 3] = f.w;
+            }
+            if (issuer) {
+                load_vs(0);
+                if (nch > 1) load_vs(1);
+                ok = load_t(0);
+                if (ok) {
+                    load_w(0);
+                    load_y(0);
+                    ok = mbar_wait_abortable(&bars[F_TFULL], 0, err, epoch, abort_flag);
+                }
+                *s_grp_ok = ok ? 1u : 0u;
+            }
+            named_bar(2, 128);
+            ok = *s_grp_ok != 0u;
+            if (ok) put_state(xa, gam_buf(0)[c]);
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(2, 128);
+            if (issuer && ok) ok = issue_products(0);
+            for (int j = 0; j < nch; ++j) {
+                const bool more = j + 1 < nch;
+                if (issuer) {
+                    if (ok && more) {
+                        // once the V term of chunk j has run (the whole group has read
+                        // Gamma_j and every U thread has converted V_j by then): [T; R] of
+                        // chunk j + 1, and the V slice of chunk j + 2 into V_j's copy
+                        ok = mbar_wait_abortable(&bars[F_VDONE], j & 1, err, epoch, abort_flag);
+                        if (ok && j + 2 < nch) load_vs(j + 2);
+                        if (ok) ok = load_t(j + 1);
+                        // until the state update of chunk j lands: [-W; P] of chunk j + 1
+                        // once the chunk products of j have completed, and the V term of
+                        // j + 1 once its V slice is converted (bounded; the waits below
+                        // complete whatever is left)
+                        bool w_done = false;
+                        if (ok) {
+                            const uint64_t tw = globaltimer_ns();
+                            while (!mbar_try_wait(&bars[F_TSFULL], j & 1) && !*abort_flag) {
+                                if (!w_done &&
+                                    mbar_try_wait(&bars[(j & 1) ? F_TD1 : F_TD0], (j >> 1) & 1)) {
+                                    load_w(j + 1);
+                                    w_done = true;
+                                }
+                                if (v_issued < j + 1 && mbar_try_wait(&bars[F_VREADY], (j + 1) & 1) &&
+                                    mbar_try_wait(&bars[F_TFULL], (j + 1) & 1)) {
+                                    tc_fence_after();
+                                    issue_vterm(j + 1);
+                                }
+                                if (globaltimer_ns() - tw > kSlowWaitNs) break;
+                            }
+                            if (!w_done) {
+                                ok = mbar_wait_abortable(&bars[(j & 1) ? F_TD1 : F_TD0], (j >> 1) & 1,
+                                                         err, epoch, abort_flag);
+                                if (ok) load_w(j + 1);
+                            }
+                        }
+                    }
+                    // S_{j+1} = TS after the state update of chunk j; then Khat is free
+                    if (ok) ok = mbar_wait_abortable(&bars[F_TSFULL], j & 1, err, epoch, abort_flag);
+                    if (ok && more) {
+                        load_y(j + 1);
+                        ok = mbar_wait_abortable(&bars[F_TFULL], (j + 1) & 1, err, epoch, abort_flag);
+                    }
+                    *s_grp_ok = ok ? 1u : 0u;
+                }
+                named_bar(2, 128);
+                ok = *s_grp_ok != 0u;
+                tc_fence_after();
+                if (ok) {
+#pragma unroll
+                    for (int p = 0; p < DVS / 16; ++p)
+                        tmem_ld16(tS + 16 * p, *reinterpret_cast<float(*)[16]>(xa + 16 * p));
+                    tmem_wait_ld();
+                }
+                if (!more) break;
+                if (ok) put_state(xa, gam_buf(j + 1)[c]);
+                fence_async_smem();
+                tc_fence_before();
+                named_bar(2, 128);
+                if (issuer && ok) ok = issue_products(j + 1);
+                // intermediate state: S after (j + 1) C tokens, when that is a multiple of
+                // the interval strictly inside the sequence (the stores overlap the
+                // chunk products)
+                if (ckpt_interval > 0 && ok) {
+                    const int64_t done = (int64_t)(j + 1) * C;
+                    if (done % ckpt_interval == 0 && done < rb - ra) {
+                        const int64_t e = ck0 + done / ckpt_interval - 1;
+                        if (e < ckpt_capacity) {
+                            float4 *dst = reinterpret_cast<float4 *>(
+                                ckpt + (((size_t)e * H + h) * D + c) * D + j0);
+#pragma unroll
+                            for (int i = 0; i < DVS / 4; ++i)
+                                dst[i] = make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
+                        } else if (lane == 0) {
+                            atomicOr(err, ERR_BAD_INDEX);
+                        }
+                    }
+                }
+            }
+            if (ok && state_out && !*abort_flag) {
+#pragma unroll
+                for (int i = 0; i < DVS / 4; ++i)
+                    reinterpret_cast<float4 *>(state_out + srow)[i] =
+                        make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
+            }
+            if (issuer) {
+                mma_commit(&bars[F_DRAIN_S]);
+                mbar_wait(&bars[F_DRAIN_S], 0, err, 1ull << 28);
+                // copies issued and never consumed (after an abort) land before exit
+                if (t_loads > 0) mbar_wait(&bars[F_TFULL], (t_loads - 1) & 1, err, 1ull << 28);
+                for (int jl = v_loads - 2; jl < v_loads; ++jl)
+                    if (jl >= 0)
+                        mbar_wait(&bars[(jl & 1) ? F_VFULL1 : F_VFULL0], (jl >> 1) & 1, err, 1ull << 28);
+                if (w_loads > 0) mbar_wait(&bars[F_WFULL], (w_loads - 1) & 1, err, 1ull << 28);
+                if (y_loads > 0) mbar_wait(&bars[F_YFULL], (y_loads - 1) & 1, err, 1ull << 28);
+            }
+        }
+    } else {
+        // ------------------------------------------------ U group (leader: thread 128)
+        const int quad = warp - 4;
+        const int row = 32 * quad + lane;   // TMEM lane: U rows 0..63, O rows 64..127
+        const int ct = tid - 128;
+        const bool issuer = tid == 128;
+        const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
+        bool ok = true;
+        for (int j = 0; j < nch; ++j) {
+            // V slice of chunk j: bf16 -> fp16 in place, rows past the chunk's end -> 0
+            if (issuer) {
+                if (ok)
+                    ok = mbar_wait_abortable(&bars[(j & 1) ? F_VFULL1 : F_VFULL0], (j >> 1) & 1, err, epoch,
+                                             abort_flag);
+                *s_u_ok = ok ? 1u : 0u;
+            }
+            named_bar(1, 128);
+            ok = *s_u_ok != 0u;
+            if (ok) {
+                uint8_t *vt = sm + v_off(j);
+                const int L = chunk_len(j);
+#pragma unroll
+                for (int i = 0; i < CPR / 2; ++i) {
+                    const int idx = ct + 128 * i;
+                    const int vrow = ((idx * 16) % 8192) / (int)Lay::kVLine;
+                    uint4 *pc = reinterpret_cast<uint4 *>(vt) + idx;
+                    if (vrow < L) {
+                        float x[8];
+                        unpack8(*pc, x);
+                        *pc = pack8(x);
+                    } else {
+                        *pc = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+            }
+            fence_async_smem();
+            named_bar(1, 128);
+            // [U; O]_j out of TMEM once the chunk products have completed
+            const int b = j & 1;
+            const uint32_t tTD = b ? tTD1 : tTD0;
+            if (issuer) {
+                if (ok) {
+                    mbar_arrive(&bars[F_VREADY]);
+                    ok = mbar_wait_abortable(&bars[b ? F_TD1 : F_TD0], (j >> 1) & 1, err, epoch, abort_flag);
+                }
+                *s_u_ok = ok ? 1u : 0u;
+            }
+            named_bar(1, 128);
+            ok = *s_u_ok != 0u;
+            tc_fence_after();
+            const int64_t t0 = ra + (int64_t)j * C;
+            const int L = chunk_len(j);
+            float xa[DVS];
+            if (ok) {
+#pragma unroll
+                for (int p = 0; p < DVS / 16; ++p)
+                    tmem_ld16(taddr(tTD, 32 * quad, 16 * p), *reinterpret_cast<float(*)[16]>(xa + 16 * p));
+                tmem_wait_ld();
+                if (quad < 2) {
+#pragma unroll
+                    for (int p = 0; p < DVS / 16; ++p) {
+                        float y0[8], y1[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            y0[e] = xa[16 * p + e];
+                            y1[e] = xa[16 * p + 8 + e];
+                        }
+                        *reinterpret_cast<uint4 *>(
+                            sm + Lay::oUB + interleave_mnmajor_off(16 * p, row, Lay::kKGroup)) = pack8(y0);
+                        *reinterpret_cast<uint4 *>(
+                            sm + Lay::oUB + interleave_mnmajor_off(16 * p + 8, row, Lay::kKGroup)) =
+                            pack8(y1);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(1, 128);
+            if (issuer && ok) {
+                // S_{j+1} = Gamma_j S_j + Khat_j^T U_j
+                ok = mbar_wait_abortable(&bars[F_YFULL], j & 1, err, epoch, abort_flag);
+                if (ok) ok = mbar_wait_abortable(&bars[F_TSSCALED], j & 1, err, epoch, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    const uint64_t ad0 = smem_desc(sbase + Lay::oKh, kKhMNBlock, 1024, SW_128B);
+                    const uint64_t bd0 = smem_desc(sbase + Lay::oUB, Lay::kKGroup, 128, SW_NONE);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16(tTS, ad0 + (uint64_t)(kk * 2048 / 16),
+                                bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_mm, 1);
+                    mma_commit(&bars[F_TSFULL]);
+                }
+            }
+            // O rows to device memory (fp32), after the state update is on its way
+            const int r = row - 64;
+            if (ok && quad >= 2 && r < L) {
+                float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * D + j0);
+#pragma unroll
+                for (int i = 0; i < DVS / 4; ++i)
+                    dst[i] = make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
+            }
+        }
+        if (issuer) {
+            mma_commit(&bars[F_DRAIN_U]);
+            mbar_wait(&bars[F_DRAIN_U], 0, err, 1ull << 28);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Lay::kTmemCols);
+    }
+}
+
+// The first n_state CTAs run the state pass (DVS value columns each), the rest
+// phase A.
+template <bool PREP, int DVS>
+__global__ void __launch_bounds__(256, 2)
+prefill_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+                     const __nv_bfloat16 *__restrict__ beta, const int32_t *__restrict__ cu,
+                     int64_t T, int N, int H, uint32_t flags, uint8_t *__restrict__ ws,
+                     const float *state_in, float *__restrict__ o, float *state_out,
+                     int64_t ckpt_interval, float *ckpt, int64_t ckpt_capacity, uint32_t *sched,
+                     uint32_t *ready, int n_state, uint32_t *err, uint32_t epoch) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    if ((int)blockIdx.x < n_state)
+        state_pass_role<DVS>(&tm_v, state_in, cu, T, N, H, ws, ready, o, state_out, ckpt_interval,
+                             ckpt, ckpt_capacity, err, epoch, sm, (int)blockIdx.x);
+    else
+        intra_chunk_body<PREP>(&tm_q, &tm_k, &tm_g, beta, cu, T, N, H, flags, ws, err, epoch, sm,
+                               (int)blockIdx.x - n_state, (int)gridDim.x - n_state, sched, ready);
+}
+
 }  // namespace tc
 
 // ======================================================================
 // host side
 // ======================================================================
+// Workspace: header, slots, then (for the one-launch form) a 256-byte area
+// holding phase A's item counter and one ready word per (chunk, head) item.
+static size_t sched_offset(int64_t rows, int N, int H) {
+    const int64_t max_chunks = (rows + tc::C - 1) / tc::C + N;
+    return (size_t)tc::header_bytes(N) + (size_t)max_chunks * H * tc::kSlotBytes;
+}
+
 size_t prefill_tc_workspace_bytes(int64_t rows, int N, int H, int d) {
     if (d != tc::D) return 0;
     const int64_t max_chunks = (rows + tc::C - 1) / tc::C + N;
-    return (size_t)tc::header_bytes(N) + (size_t)max_chunks * H * tc::kSlotBytes;
+    return sched_offset(rows, N, H) + 256 +
+           (((size_t)tc::ready_stride((int)max_chunks) * H * 4 + 255) & ~(size_t)255);
 }
 
 template <int DVS>
@@ -1415,6 +1972,54 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
     return e;
 }
 
+// One launch for both phases (tc::prefill_fused_kernel) when the state pass
+// needs at most kFusedMaxStateCtas CTAs of kFusedDVS value columns; otherwise
+// the two-kernel form.  The grid assumes two CTAs per SM (phase A's shared
+// memory and 128 registers per thread); correctness does not depend on it.
+constexpr int kFusedDVS = 64;
+constexpr int64_t kFusedMaxStateCtas = 74;
+
+static cudaError_t launch_fused(const PrefillArgs &a, int64_t rows, int64_t max_chunks,
+                                cudaStream_t st) {
+    auto kern = a.flags ? tc::prefill_fused_kernel<true, kFusedDVS>
+                        : tc::prefill_fused_kernel<false, kFusedDVS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc::A_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t n_state = (int64_t)a.N * a.H * (tc::D / kFusedDVS);
+    const int64_t items = max_chunks * a.H;
+    if (items > INT32_MAX - 65536 || rows > INT32_MAX) return cudaErrorInvalidValue;
+    int64_t n_a = 2 * (int64_t)sms - n_state;
+    if (n_a > items) n_a = items;
+    if (n_a < 1) n_a = 1;
+    CUtensorMap tq, tk, tg, tv;
+    if (!make_rows_heads_tmap(&tq, a.q, rows, a.H, tc::D, 64, tc::C, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_rows_heads_tmap(&tk, a.k, rows, a.H, tc::D, 64, tc::C, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_rows_heads_tmap(&tg, a.g, rows, a.H, tc::D, 64, tc::C, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_rows_heads_tmap(&tv, a.v, rows, a.H, tc::D, kFusedDVS, tc::C,
+                              CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    uint8_t *ws = (uint8_t *)a.workspace;
+    uint32_t *sched = reinterpret_cast<uint32_t *>(ws + sched_offset(rows, a.N, a.H));
+    uint32_t *ready = sched + 64;
+    // the counter and every ready word start at zero (epochs are nonzero)
+    e = cudaMemsetAsync(sched, 0, 256 + (size_t)tc::ready_stride((int)max_chunks) * a.H * 4, st);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(n_state + n_a), 256, tc::A_SMEM, st>>>(
+        tq, tk, tg, tv, (const __nv_bfloat16 *)a.beta, a.cu_seqlens, a.T, a.N, a.H, a.flags, ws,
+        a.state_in, (float *)a.o, a.state_out, a.ckpt_interval, a.ckpt, a.ckpt_capacity, sched,
+        ready, (int)n_state, a.err, a.epoch);
+    e = cudaGetLastError();
+    Profiler::mark(st);
+    return e;
+}
+
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
     if (a.dk != tc::D || a.dv != tc::D) return cudaErrorInvalidValue;
     uint8_t *ws = (uint8_t *)a.workspace;
@@ -1431,6 +2036,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
     const int64_t rows = (int64_t)a.B * a.T;
     const int64_t max_chunks =
         a.cu_seqlens ? (rows + tc::C - 1) / tc::C + a.N : (int64_t)a.N * ((a.T + tc::C - 1) / tc::C);
+    const int64_t units = (int64_t)a.N * a.H;
+    if (max_chunks > 0 && units * (tc::D / kFusedDVS) <= kFusedMaxStateCtas) {
+        return launch_fused(a, rows, max_chunks, st);
+    }
     if (max_chunks > 0) {
         auto kern = a.flags ? tc::intra_chunk_kernel<true> : tc::intra_chunk_kernel<false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::A_SMEM);
@@ -1457,7 +2066,6 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st) {
     }
     Profiler::mark(st);
     // dv-slices: enough CTAs to cover the SMs when there are few (sequence, head) units
-    const int64_t units = (int64_t)a.N * a.H;
     if (units <= 74) return launch_state_pass<32>(a, st);
     if (units <= 148) return launch_state_pass<64>(a, st);
     return launch_state_pass<128>(a, st);

@@ -159,6 +159,21 @@ __device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// A word in shared memory handed from one thread of the CTA to another.
+__device__ __forceinline__ uint32_t ld_acquire_cta_shared(const volatile uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];"
+                 : "=r"(v)
+                 : "r"(smem_u32(const_cast<const uint32_t *>(p)))
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta_shared(volatile uint32_t *p, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(const_cast<uint32_t *>(p))),
+                 "r"(v)
+                 : "memory");
+}
+
 // Eight consecutive words (32-byte aligned) by one acquire load.
 __device__ __forceinline__ void ld_acquire_gpu_v8(const uint32_t *p, uint32_t (&w)[8]) {
     asm volatile("ld.acquire.gpu.global.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"

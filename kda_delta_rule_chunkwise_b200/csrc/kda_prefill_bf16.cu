@@ -1475,7 +1475,8 @@ struct FLayout {
 };
 
 enum FBar { F_WFULL = 0, F_TFULL, F_VFULL0, F_VFULL1, F_VREADY, F_VDONE, F_YFULL, F_TD0, F_TD1,
-            F_TSFULL, F_TSSCALED, F_DRAIN_S, F_DRAIN_U, F_NBARS };
+            F_TSFULL, F_DRAIN_S, F_DRAIN_U, F_NBARS };
+static_assert(F_NBARS * 8 + 5 * 4 <= 256, "one-launch state pass barrier area");
 
 // Roles (256 threads): warps 0-3 state group (TMEM lane = key channel; fp16
 // copy of S, Gamma scaling; thread 0 issues the chunk products and every
@@ -1499,6 +1500,8 @@ __device__ __forceinline__ void state_pass_role(
     volatile uint32_t *abort_flag = tmem_ptr + 1;
     volatile uint32_t *s_grp_ok = tmem_ptr + 2;   // state-group leader -> group
     volatile uint32_t *s_u_ok = tmem_ptr + 3;     // U-group leader -> group
+    // highest chunk (launch index) whose ready word the U-group leader has seen
+    volatile uint32_t *s_seen = tmem_ptr + 4;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int slice = cta % NSL, unit = cta / NSL;
@@ -1525,6 +1528,7 @@ __device__ __forceinline__ void state_pass_role(
         *abort_flag = 0u;
         *s_grp_ok = 1u;
         *s_u_ok = 1u;
+        *s_seen = (uint32_t)(c0 - 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -1553,12 +1557,18 @@ __device__ __forceinline__ void state_pass_role(
         // issuer bookkeeping: copies issued per region, V terms issued, ready words seen
         int t_loads = 0, v_loads = 0, w_loads = 0, y_loads = 0, v_issued = -1, seen = c0 - 1;
         const uint32_t *rrow = ready + (size_t)h * ready_stride(nct_total);
-        // chunk j's ready word observed (acquire) before any copy of its slot: eight
-        // words (consecutive chunks of this head) per 32-byte acquire load, one
+        // chunk j's ready word observed (acquire) before any copy of its slot: as a
+        // rule by the U-group leader ahead of time (handed over in s_seen); else here,
+        // eight words (consecutive chunks of this head) per 32-byte acquire load, one
         // acquire load of the word itself when they are not all set
         auto ensure_ready = [&](int j) {
             const int cc = c0 + j;
             if (cc <= seen) return true;
+            const int sv = (int)ld_acquire_cta_shared(s_seen);
+            if (cc <= sv) {
+                seen = sv;
+                return true;
+            }
             const int g = cc & ~7;
             uint32_t w[8];
             ld_acquire_gpu_v8(rrow + g, w);
@@ -1619,31 +1629,39 @@ __device__ __forceinline__ void state_pass_role(
             mma_commit(&bars[F_VDONE]);
             v_issued = j;
         };
-        // fp16 copy of S (B operand of the state term) and TS <- Gamma * S
-        auto put_state = [&](const float *xa, float gam) {
+        // fp16 copy of S (B operand of the state term)
+        auto put_state = [&](const float *xa) {
 #pragma unroll
             for (int p = 0; p < DVS / 16; ++p) {
                 const float *x = xa + 16 * p;
-                float y0[8], y1[8], z[16];
+                float y0[8], y1[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     y0[e] = x[e];
                     y1[e] = x[8 + e];
                 }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) z[e] = x[e] * gam;
-                tmem_st16(tS + 16 * p, z);
                 *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p, c, Lay::kKGroup)) =
                     pack8(y0);
                 *reinterpret_cast<uint4 *>(sbp + interleave_mnmajor_off(16 * p + 8, c, Lay::kKGroup)) =
                     pack8(y1);
             }
-            tmem_wait_st();
         };
-        // leader, after the group's state copy: release the state update of chunk j
-        // (TSSCALED) and issue [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j
+        // S_{j+1} = Gamma_j S_j + D_j in registers, D_j = Khat_j^T U_j from TS (the
+        // state update accumulates into a fresh tile: no scaled state goes back to TMEM)
+        auto advance_state = [&](float *xa, float gam) {
+#pragma unroll
+            for (int hp = 0; hp < DVS / 32; ++hp) {
+                float d[32];
+                tmem_ld16(tS + 32 * hp, *reinterpret_cast<float(*)[16]>(d));
+                tmem_ld16(tS + 32 * hp + 16, *reinterpret_cast<float(*)[16]>(d + 16));
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) xa[32 * hp + e] = fmaf(gam, xa[32 * hp + e], d[e]);
+            }
+        };
+        // leader, after the group's state copy: issue
+        // [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j
         auto issue_products = [&](int j) {
-            mbar_arrive(&bars[F_TSSCALED]);
             if (v_issued < j) {
                 if (!mbar_wait_abortable(&bars[F_VREADY], j & 1, err, epoch, abort_flag)) return false;
                 tc_fence_after();
@@ -1689,7 +1707,7 @@ __device__ __forceinline__ void state_pass_role(
             }
             named_bar(2, 128);
             ok = *s_grp_ok != 0u;
-            if (ok) put_state(xa, gam_buf(0)[c]);
+            if (ok) put_state(xa);
             fence_async_smem();
             tc_fence_before();
             named_bar(2, 128);
@@ -1731,7 +1749,7 @@ __device__ __forceinline__ void state_pass_role(
                             }
                         }
                     }
-                    // S_{j+1} = TS after the state update of chunk j; then Khat is free
+                    // the state update of chunk j has landed in TS; then Khat is free
                     if (ok) ok = mbar_wait_abortable(&bars[F_TSFULL], j & 1, err, epoch, abort_flag);
                     if (ok && more) {
                         load_y(j + 1);
@@ -1742,14 +1760,9 @@ __device__ __forceinline__ void state_pass_role(
                 named_bar(2, 128);
                 ok = *s_grp_ok != 0u;
                 tc_fence_after();
-                if (ok) {
-#pragma unroll
-                    for (int p = 0; p < DVS / 16; ++p)
-                        tmem_ld16(tS + 16 * p, *reinterpret_cast<float(*)[16]>(xa + 16 * p));
-                    tmem_wait_ld();
-                }
+                if (ok) advance_state(xa, gam_buf(j)[c]);
                 if (!more) break;
-                if (ok) put_state(xa, gam_buf(j + 1)[c]);
+                if (ok) put_state(xa);
                 fence_async_smem();
                 tc_fence_before();
                 named_bar(2, 128);
@@ -1798,6 +1811,8 @@ __device__ __forceinline__ void state_pass_role(
         const int ct = tid - 128;
         const bool issuer = tid == 128;
         const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
+        const uint32_t *urow = ready + (size_t)h * ready_stride(nct_total);
+        int useen = c0 - 1;   // leader: highest chunk whose ready word it has seen
         bool ok = true;
         for (int j = 0; j < nch; ++j) {
             // V slice of chunk j: bf16 -> fp16 in place, rows past the chunk's end -> 0
@@ -1834,6 +1849,27 @@ __device__ __forceinline__ void state_pass_role(
             if (issuer) {
                 if (ok) {
                     mbar_arrive(&bars[F_VREADY]);
+                    // while the chunk products run: the next ready words (eight chunks
+                    // of this head per 32-byte acquire load, never waiting), handed
+                    // to the state-group leader
+                    if (useen < c0 + nch - 1 && useen < c0 + j + 16) {
+                        const int g = (useen + 1) & ~7;
+                        uint32_t w[8];
+                        ld_acquire_gpu_v8(urow + g, w);
+                        int m = useen;
+                        bool run = true;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int ci = g + i;
+                            if (run && ci > useen && ci < c0 + nch) {
+                                if (w[i] == epoch) m = ci; else run = false;
+                            }
+                        }
+                        if (m > useen) {
+                            useen = m;
+                            st_release_cta_shared(s_seen, (uint32_t)m);
+                        }
+                    }
                     ok = mbar_wait_abortable(&bars[b ? F_TD1 : F_TD0], (j >> 1) & 1, err, epoch, abort_flag);
                 }
                 *s_u_ok = ok ? 1u : 0u;
@@ -1870,9 +1906,9 @@ __device__ __forceinline__ void state_pass_role(
             tc_fence_before();
             named_bar(1, 128);
             if (issuer && ok) {
-                // S_{j+1} = Gamma_j S_j + Khat_j^T U_j
+                // D_j = Khat_j^T U_j into TS (the state group has read D_{j-1}: the
+                // chunk products of j were issued after it)
                 ok = mbar_wait_abortable(&bars[F_YFULL], j & 1, err, epoch, abort_flag);
-                if (ok) ok = mbar_wait_abortable(&bars[F_TSSCALED], j & 1, err, epoch, abort_flag);
                 if (ok) {
                     tc_fence_after();
                     const uint64_t ad0 = smem_desc(sbase + Lay::oKh, kKhMNBlock, 1024, SW_128B);
@@ -1880,7 +1916,7 @@ __device__ __forceinline__ void state_pass_role(
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16(tTS, ad0 + (uint64_t)(kk * 2048 / 16),
-                                bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_mm, 1);
+                                bd0 + (uint64_t)(kk * 2 * Lay::kKGroup / 16), id_mm, kk > 0);
                     mma_commit(&bars[F_TSFULL]);
                 }
             }

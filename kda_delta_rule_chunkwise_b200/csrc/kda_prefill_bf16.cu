@@ -1663,6 +1663,7 @@ __device__ __forceinline__ void state_pass_role(
         // [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j
         auto issue_products = [&](int j) {
             if (v_issued < j) {
+                if (!mbar_wait_abortable(&bars[F_TFULL], j & 1, err, epoch, abort_flag)) return false;
                 if (!mbar_wait_abortable(&bars[F_VREADY], j & 1, err, epoch, abort_flag)) return false;
                 tc_fence_after();
                 issue_vterm(j);
@@ -1749,12 +1750,11 @@ __device__ __forceinline__ void state_pass_role(
                             }
                         }
                     }
-                    // the state update of chunk j has landed in TS; then Khat is free
+                    // the state update of chunk j has landed in TS; then Khat is free.
+                    // ([T; R] and Gamma_L of chunk j + 1 are waited for only before the
+                    // V term: the state copy-out below needs Gamma_j, which is in.)
                     if (ok) ok = mbar_wait_abortable(&bars[F_TSFULL], j & 1, err, epoch, abort_flag);
-                    if (ok && more) {
-                        load_y(j + 1);
-                        ok = mbar_wait_abortable(&bars[F_TFULL], (j + 1) & 1, err, epoch, abort_flag);
-                    }
+                    if (ok && more) load_y(j + 1);
                     *s_grp_ok = ok ? 1u : 0u;
                 }
                 named_bar(2, 128);

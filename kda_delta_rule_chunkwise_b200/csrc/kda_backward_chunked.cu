@@ -44,8 +44,8 @@ __device__ __forceinline__ float h2f(const uint8_t *base, uint32_t off) {
 // [-W; P]: 128 rows (0..63 = -W, 64..127 = P) x 128 channels, K-major, 128-byte
 // swizzle, 64-channel blocks 16 KiB apart
 __device__ __forceinline__ uint32_t wp_off(int r, int c) {
-    return (uint32_t)((c >> 6) * 16384 + (r >> 3) * 1024 + (r & 7) * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) +
-                      (c & 7) * 2);
+    return (uint32_t)(kSlotWP + (c >> 6) * 16384 + (r >> 3) * 1024 + (r & 7) * 128 +
+                      ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2);
 }
 // [T; R]: 128 rows (0..63 = T, 64..127 = R) x 64 columns, K-major, 128-byte swizzle
 __device__ __forceinline__ uint32_t tr_off(int r, int s) {

@@ -165,12 +165,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32
         : "memory");
 }
 
-// Bring `bytes` of global memory into L2 ahead of a later copy (a hint: no
-// completion to wait for).  16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // 1-D bulk copy shared -> global in this thread's bulk group (commit with
 // bulk_commit).  Both addresses 16-byte aligned, bytes a multiple of 16; the
 // shared source must have been made visible to the async proxy.

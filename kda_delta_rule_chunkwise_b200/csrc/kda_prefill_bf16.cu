@@ -2010,7 +2010,9 @@ static cudaError_t launch_state_pass(const PrefillArgs &a, cudaStream_t st) {
 
 // One launch for both phases (tc::prefill_fused_kernel) when the state pass
 // needs at most kFusedMaxStateCtas CTAs of kFusedDVS value columns; otherwise
-// the two-kernel form.  The grid assumes two CTAs per SM (phase A's shared
+// the two-kernel form.  The choice depends on the shapes only, so a call with
+// intermediate states runs the same kernels as one without (its o and final
+// state are the same bit for bit).  The grid assumes two CTAs per SM (phase A's shared
 // memory and 128 registers per thread); correctness does not depend on it.
 constexpr int kFusedDVS = 64;
 constexpr int64_t kFusedMaxStateCtas = 74;

@@ -1474,14 +1474,15 @@ struct FLayout {
                   oUB % 128 == 0, "operand alignment");
 };
 
-enum FBar { F_WFULL = 0, F_TFULL, F_VFULL0, F_VFULL1, F_VREADY, F_VDONE, F_YFULL, F_TD0, F_TD1,
-            F_TSFULL, F_DRAIN_S, F_DRAIN_U, F_NBARS };
+enum FBar { F_WFULL = 0, F_TFULL, F_VFULL0, F_VFULL1, F_VDONE, F_YFULL, F_TD0, F_TD1, F_TSFULL,
+            F_DRAIN_S, F_DRAIN_U, F_NBARS };
 static_assert(F_NBARS * 8 + 5 * 4 <= 256, "one-launch state pass barrier area");
 
 // Roles (256 threads): warps 0-3 state group (TMEM lane = key channel; fp16
-// copy of S, Gamma scaling; thread 0 issues the chunk products and every
-// copy); warps 4-7 U group (TMEM lane = row of [U; O]; U copy-out, O to
-// device memory, V conversion; thread 128 issues the state update).
+// copy of S, Gamma scaling; thread 0 issues the state term [-W; P] S and every
+// copy); warps 4-7 U group (TMEM lane = row of [U; O]; V conversion, U
+// copy-out, O to device memory; thread 128 issues the V term [T; R] V as soon
+// as its operands are in, and the state update).
 // Each barrier completes once per chunk, and no copy into a region is issued
 // before every waiter has passed the region's previous phase, so a parity wait
 // never meets a barrier two phases ahead.
@@ -1555,7 +1556,7 @@ __device__ __forceinline__ void state_pass_role(
         const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
         uint8_t *sbp = sm + Lay::oSB;
         // issuer bookkeeping: copies issued per region, V terms issued, ready words seen
-        int t_loads = 0, v_loads = 0, w_loads = 0, y_loads = 0, v_issued = -1, seen = c0 - 1;
+        int t_loads = 0, v_loads = 0, w_loads = 0, y_loads = 0, seen = c0 - 1;
         const uint32_t *rrow = ready + (size_t)h * ready_stride(nct_total);
         // chunk j's ready word observed (acquire) before any copy of its slot: as a
         // rule by the U-group leader ahead of time (handed over in s_seen); else here,
@@ -1618,17 +1619,6 @@ __device__ __forceinline__ void state_pass_role(
             bulk_g2s(sm + Lay::oKh, slot_of(j) + kSlotKh, 16384, &bars[F_YFULL]);
             ++y_loads;
         };
-        auto issue_vterm = [&](int j) {
-            const uint32_t tTD = (j & 1) ? tTD1 : tTD0;
-            const uint64_t ad0 = smem_desc(sbase + Lay::oTR, 16, 1024, SW_128B);
-            const uint64_t bd0 = smem_desc(sbase + v_off(j), Lay::kVLbo, Lay::kVSbo, Lay::kVSwz);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tTD, ad0 + (uint64_t)(kk * 32 / 16), bd0 + (uint64_t)(kk * Lay::kVKstep / 16),
-                        id_nn, kk > 0);
-            mma_commit(&bars[F_VDONE]);
-            v_issued = j;
-        };
         // fp16 copy of S (B operand of the state term)
         auto put_state = [&](const float *xa) {
 #pragma unroll
@@ -1659,15 +1649,11 @@ __device__ __forceinline__ void state_pass_role(
                 for (int e = 0; e < 32; ++e) xa[32 * hp + e] = fmaf(gam, xa[32 * hp + e], d[e]);
             }
         };
-        // leader, after the group's state copy: issue
-        // [U; O]_j = [T; R]_j V_j + [-W; P]_j S_j
+        // leader, after the group's state copy: [U; O]_j += [-W; P]_j S_j onto the V term
+        // [T; R]_j V_j, which the U-group leader issued (its completion orders the two)
         auto issue_products = [&](int j) {
-            if (v_issued < j) {
-                if (!mbar_wait_abortable(&bars[F_TFULL], j & 1, err, epoch, abort_flag)) return false;
-                if (!mbar_wait_abortable(&bars[F_VREADY], j & 1, err, epoch, abort_flag)) return false;
-                tc_fence_after();
-                issue_vterm(j);
-            }
+            if (!mbar_wait_abortable(&bars[F_TFULL], j & 1, err, epoch, abort_flag)) return false;
+            if (!mbar_wait_abortable(&bars[F_VDONE], j & 1, err, epoch, abort_flag)) return false;
             if (!mbar_wait_abortable(&bars[F_WFULL], j & 1, err, epoch, abort_flag)) return false;
             tc_fence_after();
             const uint32_t tTD = (j & 1) ? tTD1 : tTD0;
@@ -1718,37 +1704,16 @@ __device__ __forceinline__ void state_pass_role(
                 if (issuer) {
                     if (ok && more) {
                         // once the V term of chunk j has run (the whole group has read
-                        // Gamma_j and every U thread has converted V_j by then): [T; R] of
+                        // Gamma_j: the state term of j was issued after it): [T; R] of
                         // chunk j + 1, and the V slice of chunk j + 2 into V_j's copy
                         ok = mbar_wait_abortable(&bars[F_VDONE], j & 1, err, epoch, abort_flag);
                         if (ok && j + 2 < nch) load_vs(j + 2);
                         if (ok) ok = load_t(j + 1);
-                        // until the state update of chunk j lands: [-W; P] of chunk j + 1
-                        // once the chunk products of j have completed, and the V term of
-                        // j + 1 once its V slice is converted (bounded; the waits below
-                        // complete whatever is left)
-                        bool w_done = false;
-                        if (ok) {
-                            const uint64_t tw = globaltimer_ns();
-                            while (!mbar_try_wait(&bars[F_TSFULL], j & 1) && !*abort_flag) {
-                                if (!w_done &&
-                                    mbar_try_wait(&bars[(j & 1) ? F_TD1 : F_TD0], (j >> 1) & 1)) {
-                                    load_w(j + 1);
-                                    w_done = true;
-                                }
-                                if (v_issued < j + 1 && mbar_try_wait(&bars[F_VREADY], (j + 1) & 1) &&
-                                    mbar_try_wait(&bars[F_TFULL], (j + 1) & 1)) {
-                                    tc_fence_after();
-                                    issue_vterm(j + 1);
-                                }
-                                if (globaltimer_ns() - tw > kSlowWaitNs) break;
-                            }
-                            if (!w_done) {
-                                ok = mbar_wait_abortable(&bars[(j & 1) ? F_TD1 : F_TD0], (j >> 1) & 1,
-                                                         err, epoch, abort_flag);
-                                if (ok) load_w(j + 1);
-                            }
-                        }
+                        // [-W; P] of chunk j + 1 once the chunk products of j have completed
+                        if (ok)
+                            ok = mbar_wait_abortable(&bars[(j & 1) ? F_TD1 : F_TD0], (j >> 1) & 1, err,
+                                                     epoch, abort_flag);
+                        if (ok) load_w(j + 1);
                     }
                     // the state update of chunk j has landed in TS; then Khat is free.
                     // ([T; R] and Gamma_L of chunk j + 1 are waited for only before the
@@ -1811,6 +1776,7 @@ __device__ __forceinline__ void state_pass_role(
         const int ct = tid - 128;
         const bool issuer = tid == 128;
         const uint32_t id_mm = idesc(FMT_F16, 128, DVS, 1, 1);   // A MN-major, B MN-major
+        const uint32_t id_nn = idesc(FMT_F16, 128, DVS, 0, 1);   // A K-major, B MN-major
         const uint32_t *urow = ready + (size_t)h * ready_stride(nct_total);
         int useen = c0 - 1;   // leader: highest chunk whose ready word it has seen
         bool ok = true;
@@ -1847,8 +1813,18 @@ __device__ __forceinline__ void state_pass_role(
             const int b = j & 1;
             const uint32_t tTD = b ? tTD1 : tTD0;
             if (issuer) {
+                // the V term [T; R]_j V_j into TD[j % 2] (free: the U copy-out of chunk
+                // j - 2 read it before the state update of j - 2 was issued)
+                if (ok) ok = mbar_wait_abortable(&bars[F_TFULL], j & 1, err, epoch, abort_flag);
                 if (ok) {
-                    mbar_arrive(&bars[F_VREADY]);
+                    tc_fence_after();
+                    const uint64_t ad0 = smem_desc(sbase + Lay::oTR, 16, 1024, SW_128B);
+                    const uint64_t bd0 = smem_desc(sbase + v_off(j), Lay::kVLbo, Lay::kVSbo, Lay::kVSwz);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16(tTD, ad0 + (uint64_t)(kk * 32 / 16),
+                                bd0 + (uint64_t)(kk * Lay::kVKstep / 16), id_nn, kk > 0);
+                    mma_commit(&bars[F_VDONE]);
                     // while the chunk products run: the next ready words (eight chunks
                     // of this head per 32-byte acquire load, never waiting), handed
                     // to the state-group leader

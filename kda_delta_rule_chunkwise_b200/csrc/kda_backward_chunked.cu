@@ -651,20 +651,31 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     }
 }
 
+// One CTA per (chunk, head, 32-channel slice): every step below is independent
+// per key channel except the 64 x 64 adjoint tiles dAqk and dM, which each slice
+// reads whole.  Slices keep the shared memory at 75 KB, so that three CTAs share
+// an SM.
+constexpr int AS_CW = 32;                 // channels per CTA
+constexpr int AS_LS = AS_CW + 4;          // fp32 row stride
+constexpr uint32_t AS_SMEM = (6 * 64 * AS_LS + 16 * AS_LS + 64 * L6 + 4 * AS_CW) * 4;
+
 template <typename Tin>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 3)
 bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T,
                     int N, int H, const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ g, const float *__restrict__ fg,
                     const float *__restrict__ iw, float *__restrict__ dq, float *__restrict__ dk,
                     float *__restrict__ dg, float *__restrict__ dbeta) {
     extern __shared__ __align__(16) uint8_t sm[];
+    constexpr int CW = AS_CW, LS = AS_LS, NSL = D / CW;
     const int tid = threadIdx.x;
     const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
     const bool packed = cu != nullptr;
     const int total = packed ? hdr[N] : N * (int)((T + C - 1) / C);
-    const int cidx = blockIdx.x / H, h = blockIdx.x % H;
+    const int slice = blockIdx.x % NSL, itm = blockIdx.x / NSL;
+    const int cidx = itm / H, h = itm % H;
     if (cidx >= total) return;
+    const int cb = slice * CW;   // first channel of the slice
     int n, j;
     locate_chunk(hdr, packed, T, N, cidx, n, j);
     int64_t ra, rb;
@@ -674,30 +685,44 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     const size_t item = (size_t)cidx * H + h;
     const float *io = iw + item * IW_FLOATS;
     const float *fgi = fg + item * FG_FLOATS;
-    float *G = reinterpret_cast<float *>(sm);             // [64][LD]
-    float *KF = G + 64 * LD;                               // exp(R_a - G_s), block a's
-    float *dG = KF + 64 * LD;                              // dG accumulator
-    float *Dq = dG + 64 * LD;                              // dq accumulator
-    float *Dk = Dq + 64 * LD;                              // dk accumulator
-    float *KK = Dk + 64 * LD;                              // k_s exp(R_a - G_s)
-    float *AE = KK + 64 * LD;                              // a_r E1_r for the 16 rows of block a
-    float *dFs = AE + 16 * LD;                             // dAqk, then dM  [64][L6]
-    float *Rref = dFs + 64 * L6;                           // [4][128]
-    chunk_cumsum(g, t0, H, h, L, G, Rref);
+    float *G = reinterpret_cast<float *>(sm);             // [64][LS] chunk-local cumsum
+    float *KF = G + 64 * LS;                               // exp(R_a - G_s), block a's
+    float *dG = KF + 64 * LS;                              // dG accumulator
+    float *Dq = dG + 64 * LS;                              // dq accumulator
+    float *Dk = Dq + 64 * LS;                              // dk accumulator
+    float *KK = Dk + 64 * LS;                              // k_s exp(R_a - G_s)
+    float *AE = KK + 64 * LS;                              // a_r E1_r for the 16 rows of block a
+    float *dFs = AE + 16 * LS;                             // dAqk, then dM  [64][L6]
+    float *Rref = dFs + 64 * L6;                           // [4][CW]
+    // chunk-local cumsum of this slice's channels and the 16-row references
+    if (tid < CW) {
+        float acc = 0.f;
+        for (int r = 0; r < 64; ++r) {
+            const float x = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + cb + tid]), -5.f) : 0.f;
+            acc += x;
+            G[r * LS + tid] = acc;
+            if ((r & 15) == 15 && r < 63) Rref[((r + 1) >> 4) * CW + tid] = acc;
+        }
+        Rref[tid] = 0.f;
+    }
     __syncthreads();
-    auto qv = [&](int r, int c) { return r < L ? to_f32(q[((size_t)(t0 + r) * H + h) * D + c]) : 0.f; };
-    auto kv = [&](int r, int c) { return r < L ? to_f32(k[((size_t)(t0 + r) * H + h) * D + c]) : 0.f; };
-    const float *gl = G + 63 * LD;   // G at the last row = G_L (rows past L add nothing)
+    auto qv = [&](int r, int cc) {
+        return r < L ? to_f32(q[((size_t)(t0 + r) * H + h) * D + cb + cc]) : 0.f;
+    };
+    auto kv = [&](int r, int cc) {
+        return r < L ? to_f32(k[((size_t)(t0 + r) * H + h) * D + cb + cc]) : 0.f;
+    };
+    const float *gl = G + 63 * LS;   // G at the last row = G_L (rows past L add nothing)
     // the elementwise terms
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int r = i >> 7, c = i & 127;
-        const float Gr = G[r * LD + c], gam = __expf(Gr), kh_f = __expf(gl[c] - Gr);
-        const float qq = qv(r, c), kk = kv(r, c);
+    for (int i = tid; i < 64 * CW; i += NT) {
+        const int r = i / CW, cc = i % CW, c = cb + cc;
+        const float Gr = G[r * LS + cc], gam = __expf(Gr), kh_f = __expf(gl[cc] - Gr);
+        const float qq = qv(r, cc), kk = kv(r, cc);
         const float dP = fgi[FG_DP + r * 128 + c], dKt = io[IW_DKT + r * 128 + c];
         const float dKh = fgi[FG_DKH + r * 128 + c];
-        Dq[r * LD + c] = dP * gam;
-        Dk[r * LD + c] = dKt * gam + dKh * kh_f;
-        dG[r * LD + c] = qq * gam * dP + kk * gam * dKt - kk * kh_f * dKh;
+        Dq[r * LS + cc] = dP * gam;
+        Dk[r * LS + cc] = dKt * gam + dKh * kh_f;
+        dG[r * LS + cc] = qq * gam * dP + kk * gam * dKt - kk * kh_f * dKh;
     }
     // decayed adjoints: first Aqk with (a, b) = (q, k), then M with (k, k)
     for (int form = 0; form < 2; ++form) {
@@ -708,62 +733,62 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
         for (int a = 0; a < 4; ++a) {
             const int ns = 16 * (a + 1);
             __syncthreads();
-            for (int i = tid; i < 64 * 128; i += NT) {
-                const int s = i >> 7, c = i & 127;
-                KF[s * LD + c] = s < ns ? __expf(Rref[a * 128 + c] - G[s * LD + c]) : 0.f;   // exp(R_a - G_s)
-                KK[s * LD + c] = kv(s, c) * KF[s * LD + c];                                     // k_s exp(R_a - G_s)
+            for (int i = tid; i < 64 * CW; i += NT) {
+                const int s = i / CW, cc = i % CW;
+                KF[s * LS + cc] = s < ns ? __expf(Rref[a * CW + cc] - G[s * LS + cc]) : 0.f;   // exp(R_a - G_s)
+                KK[s * LS + cc] = kv(s, cc) * KF[s * LS + cc];                                   // k_s exp(R_a - G_s)
             }
-            for (int i = tid; i < 16 * 128; i += NT) {
-                const int r = i >> 7, c = i & 127, rr = 16 * a + r;
-                AE[r * LD + c] = (form == 0 ? qv(rr, c) : kv(rr, c)) * __expf(G[rr * LD + c] - Rref[a * 128 + c]);
+            for (int i = tid; i < 16 * CW; i += NT) {
+                const int r = i / CW, cc = i % CW, rr = 16 * a + r;
+                AE[r * LS + cc] = (form == 0 ? qv(rr, cc) : kv(rr, cc)) * __expf(G[rr * LS + cc] - Rref[a * CW + cc]);
             }
             __syncthreads();
             // da_r (rows of block a) = E1_r sum_s dF[r,s] b_s exp(R_a - G_s), b = k
-            smm<16, 128, 64>([&](int r, int s) { return dF[(16 * a + r) * L6 + s]; },
-                             [&](int s, int c) { return KK[s * LD + c]; },
-                             [&](int r, int c, float x) {
-                                 const int rr = 16 * a + r;
-                                 const float da = x * __expf(G[rr * LD + c] - Rref[a * 128 + c]);
-                                 const float av = form == 0 ? qv(rr, c) : kv(rr, c);
-                                 if (form == 0) Dq[rr * LD + c] += da; else Dk[rr * LD + c] += da;
-                                 dG[rr * LD + c] += av * da;
-                             });
+            smm<16, CW, 64>([&](int r, int s) { return dF[(16 * a + r) * L6 + s]; },
+                            [&](int s, int cc) { return KK[s * LS + cc]; },
+                            [&](int r, int cc, float x) {
+                                const int rr = 16 * a + r;
+                                const float da = x * __expf(G[rr * LS + cc] - Rref[a * CW + cc]);
+                                const float av = form == 0 ? qv(rr, cc) : kv(rr, cc);
+                                if (form == 0) Dq[rr * LS + cc] += da; else Dk[rr * LS + cc] += da;
+                                dG[rr * LS + cc] += av * da;
+                            });
             // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s <= 16a + 15
-            smm<64, 128, 16>([&](int s, int r) { return dF[(16 * a + r) * L6 + s]; },
-                             [&](int r, int c) { return AE[r * LD + c]; },
-                             [&](int s, int c, float x) {
-                                 if (s >= ns) return;
-                                 const float db = x * KF[s * LD + c];
-                                 Dk[s * LD + c] += db;
-                                 dG[s * LD + c] -= kv(s, c) * db;
-                             });
+            smm<64, CW, 16>([&](int s, int r) { return dF[(16 * a + r) * L6 + s]; },
+                            [&](int r, int cc) { return AE[r * LS + cc]; },
+                            [&](int s, int cc, float x) {
+                                if (s >= ns) return;
+                                const float db = x * KF[s * LS + cc];
+                                Dk[s * LS + cc] += db;
+                                dG[s * LS + cc] -= kv(s, cc) * db;
+                            });
         }
     }
     __syncthreads();
     // row L-1 also carries G_L's gradient: sum_r Khat dKhat + Gamma_L dGamma_L; then
     // dg = reverse cumsum of dG, 0 where g < -5
-    if (tid < 128 && L > 0) {
-        const int c = tid;
+    if (tid < CW && L > 0) {
+        const int cc = tid, c = cb + tid;
         float s_kh = 0.f;
         for (int r = 0; r < L; ++r)
-            s_kh = fmaf(kv(r, c) * __expf(gl[c] - G[r * LD + c]), fgi[FG_DKH + r * 128 + c], s_kh);
-        dG[(L - 1) * LD + c] += s_kh + __expf(gl[c]) * fgi[FG_DGL + c];
+            s_kh = fmaf(kv(r, cc) * __expf(gl[cc] - G[r * LS + cc]), fgi[FG_DKH + r * 128 + c], s_kh);
+        dG[(L - 1) * LS + cc] += s_kh + __expf(gl[cc]) * fgi[FG_DGL + c];
         float acc = 0.f;
         for (int r = L - 1; r >= 0; --r) {
-            acc += dG[r * LD + c];
+            acc += dG[r * LS + cc];
             const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
             dg[off] = to_f32(g[off]) >= -5.f ? acc : 0.f;
         }
     }
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int r = i >> 7, c = i & 127;
+    for (int i = tid; i < 64 * CW; i += NT) {
+        const int r = i / CW, cc = i % CW;
         if (r < L) {
-            const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
-            dq[off] = Dq[r * LD + c];
-            dk[off] = Dk[r * LD + c];
+            const size_t off = ((size_t)(t0 + r) * H + h) * D + cb + cc;
+            dq[off] = Dq[r * LS + cc];
+            dk[off] = Dk[r * LS + cc];
         }
     }
-    if (tid < L) dbeta[(size_t)(t0 + tid) * H + h] = io[IW_DB + tid];
+    if (slice == 0 && tid < L) dbeta[(size_t)(t0 + tid) * H + h] = io[IW_DB + tid];
 }
 
 }  // namespace cbw
@@ -859,10 +884,9 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
                                                         (const bf *)a.g, (const bf *)a.beta, fg, iw);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t AS_SMEM = 6 * 64 * LD * 4 + 16 * LD * 4 + 64 * L6 * 4 + 4 * 128 * 4;
-    static_assert(AS_SMEM <= 227 * 1024, "assembly shared memory");
-    if ((e = set_smem(bwd_assemble_kernel<bf>, AS_SMEM)) != cudaSuccess) return e;
-    bwd_assemble_kernel<bf><<<items, NT, AS_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
+    static_assert(3 * (cbw::AS_SMEM + 1024) <= 228 * 1024, "assembly: three CTAs per SM");
+    if ((e = set_smem(bwd_assemble_kernel<bf>, cbw::AS_SMEM)) != cudaSuccess) return e;
+    bwd_assemble_kernel<bf><<<items * (cbw::D / cbw::AS_CW), NT, cbw::AS_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
                                                         (const bf *)a.k, (const bf *)a.g, fg, iw, a.dq,
                                                         a.dk, a.dg, a.dbeta);
     e = cudaGetLastError();

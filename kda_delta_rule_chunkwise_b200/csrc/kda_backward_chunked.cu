@@ -32,6 +32,8 @@
 namespace kda {
 namespace cbw {
 
+using namespace sm100;
+
 constexpr int C = 64, D = 128, NT = 256;
 
 // ---- the forward's slot layout (kda_prefill_bf16.cu), read here
@@ -165,14 +167,17 @@ constexpr uint32_t CH_WN = CH_KH + 64 * LDF * 4;                  // -W   [64][L
 constexpr uint32_t CH_P = CH_WN + 64 * LDF * 4;                   // P    [64][LDF]
 constexpr uint32_t CH_DS = CH_P + 64 * LDF * 4;                   // dS' [128][CH_LD] fp32
 constexpr uint32_t CH_Y = CH_DS + 128 * CH_LD * 4;                // dU  [64][CH_LD]
-constexpr uint32_t CH_DO = CH_Y + 64 * CH_LD * 4;                 // dO  [64][CH_LD]
-constexpr uint32_t CH_SMEM = CH_DO + 64 * CH_LD * 4;
+constexpr uint32_t CH_DO = CH_Y + 64 * CH_LD * 4;                 // dO  2 x [64][CH_LD]
+constexpr uint32_t CH_GAM = CH_DO + 2 * 64 * CH_LD * 4;           // Gamma_L [128]
+constexpr uint32_t CH_BAR = CH_GAM + 128 * 4;                     // slot-copy mbarrier
+constexpr uint32_t CH_SMEM = CH_BAR + 16;
+static_assert(CH_SMEM <= 227 * 1024, "chain kernel shared memory");
 
 __global__ void __launch_bounds__(NT, 1)
 bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T, int N,
                  int H, const float *__restrict__ dout, const float *dstate_out,
                  float *__restrict__ ws_dS, float *__restrict__ ws_dU, float *dstate_in,
-                 uint32_t hdr_bytes) {
+                 uint32_t hdr_bytes, uint32_t *err) {
     constexpr int NSL = D / CH_DVS;
     extern __shared__ __align__(16) uint8_t sm[];
     const int slice = blockIdx.x % NSL, unit = blockIdx.x / NSL;
@@ -192,40 +197,72 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
     float *Pm = reinterpret_cast<float *>(sm + CH_P);
     float *dS = reinterpret_cast<float *>(sm + CH_DS);
     float *Y = reinterpret_cast<float *>(sm + CH_Y);
-    float *dO = reinterpret_cast<float *>(sm + CH_DO);
+    float *gam = reinterpret_cast<float *>(sm + CH_GAM);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + CH_BAR);
     const size_t sbase = ((size_t)n * H + h) * D * D;
+    // The next chunk's slot image goes in by one bulk copy (completing on `bar`) as
+    // soon as this chunk's has been decoded, and its dO rows by cp.async into the
+    // other dO buffer, so that neither load waits on device memory in the chain.
+    auto issue_slot = [&](int jn) {
+        if (tid == 0) {
+            fence_async_smem();   // the decode's reads of the previous image come first
+            mbar_arrive_expect_tx(bar, kSlotBytes);
+            bulk_g2s(slot, fws + hdr_bytes + ((size_t)(c0 + jn) * H + h) * kSlotBytes, kSlotBytes, bar);
+        }
+    };
+    auto issue_dO = [&](int jn, float *buf) {
+        const int64_t tn = ra + (int64_t)jn * C;
+        const int Ln = (int)((rb - tn) < C ? (rb - tn) : C);
+        for (int i = tid; i < 64 * (CH_DVS / 4); i += NT) {   // 16-byte pieces
+            const int t = i / (CH_DVS / 4), p4 = i % (CH_DVS / 4);
+            const float *src = dout + ((size_t)(tn + (t < Ln ? t : 0)) * H + h) * D + j0 + 4 * p4;
+            cp_async16(buf + t * CH_LD + 4 * p4, src, t < Ln ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_fence_init();
+    }
     // dS' of the last chunk = dL/dS_final
     for (int i = tid; i < 128 * CH_DVS; i += NT) {
         const int c = i / CH_DVS, jj = i % CH_DVS;
         dS[c * CH_LD + jj] = dstate_out ? dstate_out[sbase + (size_t)c * D + j0 + jj] : 0.f;
     }
+    __syncthreads();
+    if (nch > 0) {
+        issue_slot(nch - 1);
+        issue_dO(nch - 1, reinterpret_cast<float *>(sm + CH_DO));
+    }
+    bool ok = true;
+    int stuck = -1;   // the step whose slot copy was given up on (bounded wait)
     for (int j = nch - 1; j >= 0; --j) {
-        const int64_t t0 = ra + (int64_t)j * C;
-        const int L = (int)((rb - t0) < C ? (rb - t0) : C);
         const size_t item = (size_t)(c0 + j) * H + h;
-        __syncthreads();   // the previous step's reads of slot, Y and dO are done
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(fws + hdr_bytes + item * kSlotBytes);
-            uint4 *dst = reinterpret_cast<uint4 *>(slot);
-            for (int i = tid; i < (int)(kSlotBytes / 16); i += NT) dst[i] = src[i];
-        }
-        for (int i = tid; i < 64 * CH_DVS; i += NT) {
-            const int t = i / CH_DVS, jj = i % CH_DVS;
-            dO[t * CH_LD + jj] = t < L ? dout[((size_t)(t0 + t) * H + h) * D + j0 + jj] : 0.f;
-        }
+        const int step = nch - 1 - j;
+        float *dO = reinterpret_cast<float *>(sm + CH_DO) + (step & 1) * 64 * CH_LD;
         // dS' of this chunk, for the factor kernel
         for (int i = tid; i < 128 * CH_DVS; i += NT) {
             const int c = i / CH_DVS, jj = i % CH_DVS;
             ws_dS[(item * D + c) * D + j0 + jj] = dS[c * CH_LD + jj];
         }
-        __syncthreads();   // the slot image has landed
+        if (ok) {
+            ok = mbar_wait(bar, step & 1, err);   // the slot image has landed
+            if (!ok) stuck = step;
+        }
+        cp_async_wait_all();                            // this thread's dO pieces have
+        __syncthreads();
         for (int i = tid; i < 64 * 128; i += NT) {
             const int t = i >> 7, c = i & 127;
             Kh[t * LDF + c] = h2f(slot, kh_off(t, c));
             Wn[t * LDF + c] = h2f(slot, wp_off(t, c));
             Pm[t * LDF + c] = h2f(slot, wp_off(64 + t, c));
         }
-        __syncthreads();
+        if (tid < 128) gam[tid] = reinterpret_cast<const float *>(slot + kSlotGam)[tid];
+        __syncthreads();   // the image is decoded: the next one may land over it
+        if (j > 0 && ok) {
+            issue_slot(j - 1);
+            issue_dO(j - 1, reinterpret_cast<float *>(sm + CH_DO) + ((step + 1) & 1) * 64 * CH_LD);
+        }
         // dU = Khat dS'
         smm<64, CH_DVS, 128>([&](int t, int c) { return Kh[t * LDF + c]; },
                              [&](int c, int jj) { return dS[c * CH_LD + jj]; },
@@ -238,7 +275,6 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
         // dS = Diag(Gamma_L) dS' + P^T dO + (-W)^T dU   (the slot holds -W); each thread
         // overwrites only the elements it alone reads
         {
-            const float *gam = reinterpret_cast<const float *>(slot + kSlotGam);
             const int tx = tid & 15, ty = tid >> 4;
             float r[8][2];
 #pragma unroll
@@ -267,7 +303,11 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
 #pragma unroll
                 for (int b = 0; b < 2; ++b) dS[(ty + 16 * a) * CH_LD + tx + 16 * b] = r[a][b];
         }
+        __syncthreads();   // dS, Y and this dO buffer are consumed
     }
+    // a copy given up on (after a timeout) lands before exit
+    if (tid == 0 && stuck >= 0) mbar_wait(bar, stuck & 1, err, 1ull << 28);
+    cp_async_wait_all();
     __syncthreads();
     if (dstate_in)
         for (int i = tid; i < 128 * CH_DVS; i += NT) {
@@ -861,7 +901,7 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
     // 2. the chain, chunks in reverse
     if ((e = set_smem(bwd_chain_kernel, CH_SMEM)) != cudaSuccess) return e;
     bwd_chain_kernel<<<(unsigned)(a.N * a.H * (D / CH_DVS)), NT, CH_SMEM, st>>>(
-        fws, a.cu_seqlens, a.T, a.N, a.H, a.dout, a.dstate_out, dS, dU, a.dstate_in, hb);
+        fws, a.cu_seqlens, a.T, a.N, a.H, a.dout, a.dstate_out, dS, dU, a.dstate_in, hb, a.err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
     // 3.-6. per chunk: factor gradients (and dv), recompute, pull-back, assembly

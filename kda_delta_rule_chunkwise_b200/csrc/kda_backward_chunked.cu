@@ -523,8 +523,9 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
     float *G = reinterpret_cast<float *>(sm);              // [64][LD]
     float *QE = G + 64 * LD;                               // q_r E1_r
     float *KE = QE + 64 * LD;                              // k_r E1_r
-    float *KF = KE + 64 * LD;                              // k_s exp(R_a - G_s), block a's
-    float *Rref = KF + 64 * LD;                            // [4][128]
+    float *KFt = KE + 64 * LD;                             // [128][L6]: k_s exp(R_a - G_s), block a's
+    float *Rref = KFt + 128 * L6;                          // [4][128]
+    float *Kr = Rref + 4 * 128;                            // [64][LD]: k (0 past the chunk's end)
     float *out = iw + ((size_t)cidx * H + h) * IW_FLOATS;
     chunk_cumsum(g, t0, H, h, L, G, Rref);
     __syncthreads();
@@ -532,31 +533,45 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
         const int r = i >> 7, c = i & 127;
         const float e1 = __expf(G[r * LD + c] - Rref[(r >> 4) * 128 + c]);
         const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
+        const float kk = r < L ? to_f32(k[off]) : 0.f;
         QE[r * LD + c] = r < L ? to_f32(q[off]) * e1 : 0.f;
-        KE[r * LD + c] = r < L ? to_f32(k[off]) * e1 : 0.f;
+        KE[r * LD + c] = kk * e1;
+        Kr[r * LD + c] = kk;
     }
+    const int tx = tid & 15, ty = tid >> 4;   // output (row 16a + ty, columns tx + 16 b)
     for (int a = 0; a < 4; ++a) {
         const int ns = 16 * (a + 1);   // rows s <= 16a + 15
         __syncthreads();
-        for (int i = tid; i < ns * 128; i += NT) {
-            const int s = i >> 7, c = i & 127;
-            KF[s * LD + c] = s < L ? to_f32(k[((size_t)(t0 + s) * H + h) * D + c]) *
-                                         __expf(Rref[a * 128 + c] - G[s * LD + c])
-                                   : 0.f;
+        // k_s exp(R_a - G_s) stored channel-major, so that the product below reads
+        // consecutive s across a half-warp (conflict-free)
+        for (int i = tid; i < 64 * 128; i += NT) {
+            const int s = i & 63, c = i >> 6;
+            KFt[c * L6 + s] = s < ns ? Kr[s * LD + c] * __expf(Rref[a * 128 + c] - G[s * LD + c]) : 0.f;
         }
-        for (int i = tid + ns * 128; i < 64 * 128; i += NT) KF[(i >> 7) * LD + (i & 127)] = 0.f;
         __syncthreads();
-        // rows 16a .. 16a + 15 of Aqk (s <= r) and M (s < r)
-        smm<16, 64, 128>([&](int r, int c) { return QE[(16 * a + r) * LD + c]; },
-                         [&](int c, int s) { return KF[s * LD + c]; },
-                         [&](int r, int s, float x) {
-                             out[IW_AQK + (16 * a + r) * 64 + s] = s <= 16 * a + r ? x : 0.f;
-                         });
-        smm<16, 64, 128>([&](int r, int c) { return KE[(16 * a + r) * LD + c]; },
-                         [&](int c, int s) { return KF[s * LD + c]; },
-                         [&](int r, int s, float x) {
-                             out[IW_M + (16 * a + r) * 64 + s] = s < 16 * a + r ? x : 0.f;
-                         });
+        // rows 16a .. 16a + 15 of Aqk (s <= r) and of M (s < r) in one pass over the
+        // channels (the two share the decayed k operand); sums over c in order
+        float ra_[4], rm_[4];
+#pragma unroll
+        for (int b2 = 0; b2 < 4; ++b2) ra_[b2] = rm_[b2] = 0.f;
+        const float *qe = QE + (16 * a + ty) * LD, *ke = KE + (16 * a + ty) * LD;
+#pragma unroll 4
+        for (int c = 0; c < 128; ++c) {
+            const float x = qe[c], y = ke[c];
+#pragma unroll
+            for (int b2 = 0; b2 < 4; ++b2) {
+                const float kf = KFt[c * L6 + tx + 16 * b2];
+                ra_[b2] = fmaf(x, kf, ra_[b2]);
+                rm_[b2] = fmaf(y, kf, rm_[b2]);
+            }
+        }
+        const int r = 16 * a + ty;
+#pragma unroll
+        for (int b2 = 0; b2 < 4; ++b2) {
+            const int s2 = tx + 16 * b2;
+            out[IW_AQK + r * 64 + s2] = s2 <= r ? ra_[b2] : 0.f;
+            out[IW_M + r * 64 + s2] = s2 < r ? rm_[b2] : 0.f;
+        }
     }
 }
 
@@ -911,7 +926,7 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
                                                      a.state_in, snaps, a.dout, dS, dU, fg, a.dv, hb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t RC_SMEM = 4 * 64 * LD * 4 + 4 * 128 * 4;
+    constexpr uint32_t RC_SMEM = 4 * 64 * LD * 4 + 128 * L6 * 4 + 4 * 128 * 4;
     if ((e = set_smem(bwd_recompute_kernel<bf>, RC_SMEM)) != cudaSuccess) return e;
     bwd_recompute_kernel<bf><<<items, NT, RC_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
                                                          (const bf *)a.k, (const bf *)a.g, iw);

@@ -99,9 +99,12 @@ def test_bf16_many_short_sequences():
     check(inp, TOL_BF16, what="bf16 1500 short sequences")
 
 
-@pytest.mark.parametrize("H", [1, 100, 150])
+@pytest.mark.parametrize("H", [1, 37, 38, 48, 100, 150])
 def test_bf16_slice_layouts(H):
-    """(sequence, head) counts that select each dv-slice width of the state pass."""
+    """(sequence, head) counts that select each form of the bf16 prefill: one launch
+    for both phases (up to 37 units: H = 1, 37), and the two-kernel form with its
+    three state-pass slice widths (32 columns up to 74 units: H = 38, 48; 64 up to
+    148: H = 100; 128 beyond: H = 150)."""
     inp = kin.prefill_inputs(1, 130, H, 128, 128, "bf16", seed=9, state="normal")
     check(inp, TOL_BF16, heads=sorted({0, H // 2, H - 1}), what=f"bf16 H{H}")
 

@@ -486,15 +486,21 @@ constexpr uint32_t IW_AQK = 0, IW_M = 4096, IW_DAQK = 8192, IW_DM = 12288, IW_DK
 
 // G = cumsum(max(g, -5)) over the chunk's rows (rows past L decay by nothing), and
 // the block references R_a = G at the end of block a - 1 (R_0 = 0), per channel
+// (all threads: the rows load in parallel, then one thread per channel scans them
+// in shared memory; G is complete after the caller's next barrier)
 template <typename Tin>
 __device__ __forceinline__ void chunk_cumsum(const Tin *g, int64_t t0, int H, int h, int L, float *G,
                                              float *Rref) {
     const int tid = threadIdx.x;
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int r = i >> 7, c = i & 127;
+        G[r * LD + c] = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + c]), -5.f) : 0.f;
+    }
+    __syncthreads();
     if (tid < 128) {
         float acc = 0.f;
         for (int r = 0; r < 64; ++r) {
-            const float x = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + tid]), -5.f) : 0.f;
-            acc += x;
+            acc += G[r * LD + tid];
             G[r * LD + tid] = acc;
             if ((r & 15) == 15 && r < 63) Rref[((r + 1) >> 4) * 128 + tid] = acc;
         }
@@ -619,13 +625,24 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
         dPs[t * LD + c] = fgi[FG_DP + i];
         dWs[t * LD + c] = fgi[FG_DW + i];
     }
-    if (tid < 128) {   // K * Gamma, Gamma = exp(cumsum(max(g, -5)))
+    // K * Gamma, Gamma = exp(cumsum(max(g, -5))): the rows of g load in parallel,
+    // one thread per channel scans them in place, then the rows of k scale them
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int r = i >> 7, c = i & 127;
+        Kt[r * LD + c] = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + c]), -5.f) : 0.f;
+    }
+    __syncthreads();
+    if (tid < 128) {
         float acc = 0.f;
         for (int r = 0; r < 64; ++r) {
-            const size_t off = ((size_t)(t0 + r) * H + h) * D + tid;
-            acc += r < L ? fmaxf(to_f32(g[off]), -5.f) : 0.f;
-            Kt[r * LD + tid] = r < L ? to_f32(k[off]) * __expf(acc) : 0.f;
+            acc += Kt[r * LD + tid];
+            Kt[r * LD + tid] = __expf(acc);
         }
+    }
+    __syncthreads();
+    for (int i = tid; i < 64 * 128; i += NT) {
+        const int r = i >> 7, c = i & 127;
+        Kt[r * LD + c] = r < L ? to_f32(k[((size_t)(t0 + r) * H + h) * D + c]) * Kt[r * LD + c] : 0.f;
     }
     __syncthreads();
     // X = (I + A)^-1, A = Diag(beta) M (strictly lower), by 16 x 16 blocks: the
@@ -712,7 +729,7 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
 // an SM.
 constexpr int AS_CW = 32;                 // channels per CTA
 constexpr int AS_LS = AS_CW + 4;          // fp32 row stride
-constexpr uint32_t AS_SMEM = (6 * 64 * AS_LS + 16 * AS_LS + 64 * L6 + 4 * AS_CW) * 4;
+constexpr uint32_t AS_SMEM = (6 * 64 * AS_LS + 16 * AS_LS + 64 * L6 + 4 * AS_CW + 64) * 4;
 
 template <typename Tin>
 __global__ void __launch_bounds__(NT, 3)
@@ -749,12 +766,23 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     float *AE = KK + 64 * LS;                              // a_r E1_r for the 16 rows of block a
     float *dFs = AE + 16 * LS;                             // dAqk, then dM  [64][L6]
     float *Rref = dFs + 64 * L6;                           // [4][CW]
-    // chunk-local cumsum of this slice's channels and the 16-row references
+    uint32_t *below = reinterpret_cast<uint32_t *>(Rref + 4 * CW);   // [64]: bit cc set where g < -5
+    // chunk-local cumsum of this slice's channels and the 16-row references: the
+    // rows load in parallel (clamped, with the rows below the clamp flagged for
+    // dg), then one thread per channel scans them in shared memory
+    if (tid < 64) below[tid] = 0u;
+    __syncthreads();
+    for (int i = tid; i < 64 * CW; i += NT) {
+        const int r = i / CW, cc = i % CW;
+        const float x = r < L ? to_f32(g[((size_t)(t0 + r) * H + h) * D + cb + cc]) : 0.f;
+        G[r * LS + cc] = fmaxf(x, -5.f) * (r < L ? 1.f : 0.f);
+        if (r < L && !(x >= -5.f)) atomicOr(&below[r], 1u << cc);
+    }
+    __syncthreads();
     if (tid < CW) {
         float acc = 0.f;
         for (int r = 0; r < 64; ++r) {
-            const float x = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + cb + tid]), -5.f) : 0.f;
-            acc += x;
+            acc += G[r * LS + tid];
             G[r * LS + tid] = acc;
             if ((r & 15) == 15 && r < 63) Rref[((r + 1) >> 4) * CW + tid] = acc;
         }
@@ -820,19 +848,28 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
         }
     }
     __syncthreads();
-    // row L-1 also carries G_L's gradient: sum_r Khat dKhat + Gamma_L dGamma_L; then
-    // dg = reverse cumsum of dG, 0 where g < -5
+    // row L-1 also carries G_L's gradient: sum_r Khat dKhat + Gamma_L dGamma_L (the
+    // sum by 8-row groups over all threads, into KF, which is free now); then dg =
+    // reverse cumsum of dG, 0 where g < -5
+    {
+        const int cc = tid % CW, rg = tid / CW;   // NT / CW = 8 groups of 8 rows
+        float part = 0.f;
+#pragma unroll
+        for (int r = 8 * rg; r < 8 * rg + 8; ++r)
+            if (r < L)
+                part = fmaf(kv(r, cc) * __expf(gl[cc] - G[r * LS + cc]), fgi[FG_DKH + r * 128 + cb + cc], part);
+        KF[rg * LS + cc] = part;
+    }
+    __syncthreads();
     if (tid < CW && L > 0) {
         const int cc = tid, c = cb + tid;
         float s_kh = 0.f;
-        for (int r = 0; r < L; ++r)
-            s_kh = fmaf(kv(r, cc) * __expf(gl[cc] - G[r * LS + cc]), fgi[FG_DKH + r * 128 + c], s_kh);
+        for (int rg = 0; rg < NT / CW; ++rg) s_kh += KF[rg * LS + cc];
         dG[(L - 1) * LS + cc] += s_kh + __expf(gl[cc]) * fgi[FG_DGL + c];
         float acc = 0.f;
         for (int r = L - 1; r >= 0; --r) {
             acc += dG[r * LS + cc];
-            const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
-            dg[off] = to_f32(g[off]) >= -5.f ? acc : 0.f;
+            dg[((size_t)(t0 + r) * H + h) * D + c] = (below[r] >> cc) & 1u ? 0.f : acc;
         }
     }
     for (int i = tid; i < 64 * CW; i += NT) {

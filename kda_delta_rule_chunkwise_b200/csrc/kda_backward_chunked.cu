@@ -129,6 +129,48 @@ __device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, 
         for (int b = 0; b < TN; ++b) out(ty + 16 * a, tx + 16 * b, r[a][b]);
 }
 
+// The product with a row-major fp32 right operand B (ldb a multiple of 4):
+// out(i, j, sum_k A(i, k) B[k][j]).  Thread (ty, tx) owns rows ty + 16 a and the
+// four consecutive columns 4 tx + 64 b + e, read as one 16-byte load per k and b.
+// The sums run over k in order, as in smm.
+template <int M, int N, int K, typename FA, typename FO>
+__device__ __forceinline__ void smm_pb(FA A, const float *B, int ldb, FO out) {
+    constexpr int TM = M / 16, NB = N / 64;
+    static_assert(M % 16 == 0 && N % 64 == 0, "tile");
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float r[TM][NB][4];
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) r[a][b][e] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        float av[TM];
+        float4 bv[NB];
+#pragma unroll
+        for (int a = 0; a < TM; ++a) av[a] = A(ty + 16 * a, k);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) bv[b] = *reinterpret_cast<const float4 *>(B + k * ldb + 64 * b + 4 * tx);
+#pragma unroll
+        for (int a = 0; a < TM; ++a)
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                r[a][b][0] = fmaf(av[a], bv[b].x, r[a][b][0]);
+                r[a][b][1] = fmaf(av[a], bv[b].y, r[a][b][1]);
+                r[a][b][2] = fmaf(av[a], bv[b].z, r[a][b][2]);
+                r[a][b][3] = fmaf(av[a], bv[b].w, r[a][b][3]);
+            }
+    }
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) out(ty + 16 * a, 64 * b + 4 * tx + e, r[a][b][e]);
+}
+
 // rows [a, b) of sequence n: equal-length batch, or the chunk table's clamped offsets
 __device__ __forceinline__ void seq_rows(const int32_t *hdr, bool packed, int64_t T, int N, int n,
                                          int64_t &a, int64_t &b) {
@@ -406,10 +448,10 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     auto Tm = [&](int r, int s2) { return Tf[r * L6 + s2]; };   // T[r][s]
     auto Rm = [&](int r, int s2) { return Rf[r * L6 + s2]; };   // R[r][s]
     // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out)
-    smm<64, 128, 64>([&](int s, int t) { return Tm(t, s); }, [&](int t, int c) { return dU[t * LD + c]; },
-                     [&](int s, int c, float x) { U[s * LD + c] = x; });
-    smm<64, 128, 64>([&](int s, int t) { return Rm(t, s); }, [&](int t, int c) { return dO[t * LD + c]; },
-                     [&](int s, int c, float x) { U[s * LD + c] += x; });
+    smm_pb<64, 128, 64>([&](int s, int t) { return Tm(t, s); }, dU, LD,
+                        [&](int s, int c, float x) { U[s * LD + c] = x; });
+    smm_pb<64, 128, 64>([&](int s, int t) { return Rm(t, s); }, dO, LD,
+                        [&](int s, int c, float x) { U[s * LD + c] += x; });
     __syncthreads();
     for (int i = tid; i < 64 * 128; i += NT) {
         const int s = i >> 7, c = i & 127;
@@ -420,8 +462,8 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     smm_nt<64, 64, 128>(dO, LD, V, LD, [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; });
     __syncthreads();   // U's buffer (dV) is read out
     // U = T V
-    smm<64, 128, 64>([&](int t, int s) { return Tm(t, s); }, [&](int s, int c) { return V[s * LD + c]; },
-                     [&](int t, int c, float x) { U[t * LD + c] = x; });
+    smm_pb<64, 128, 64>([&](int t, int s) { return Tm(t, s); }, V, LD,
+                        [&](int t, int c, float x) { U[t * LD + c] = x; });
     __syncthreads();   // V and [T; R] are consumed
 
     // ---- phase 2: S
@@ -435,9 +477,8 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     }
     __syncthreads();
     // U += (-W) S   (the slot holds -W)
-    smm<64, 128, 128>([&](int t, int c) { return Wnf[t * LD + c]; },
-                      [&](int c, int jj) { return S[c * LD + jj]; },
-                      [&](int t, int jj, float x) { U[t * LD + jj] += x; });
+    smm_pb<64, 128, 128>([&](int t, int c) { return Wnf[t * LD + c]; }, S, LD,
+                         [&](int t, int jj, float x) { U[t * LD + jj] += x; });
     // dW = -dU S^T, dP = dO S^T
     smm_nt<64, 128, 128>(dU, LD, S, LD, [&](int t, int c, float x) { out[FG_DW + t * 128 + c] = -x; });
     smm_nt<64, 128, 128>(dO, LD, S, LD, [&](int t, int c, float x) { out[FG_DP + t * 128 + c] = x; });

@@ -129,6 +129,12 @@ KDA_API size_t kda_chunk_prefill_workspace_bytes(int64_t rows, int N, int H, int
  *              bytes, 256-byte aligned, or NULL when that size is 0.  Its
  *              contents on return are the per-chunk intermediates of the
  *              bf16 path (laid out for the state pass); callers may ignore them.
+ *
+ * bf16 at d = 128 with at most 37 (sequence, head) units runs both phases in
+ * one launch (the state pass beside the intra-chunk work, handed each chunk's
+ * intermediates through ready words in the workspace, every wait bounded);
+ * more units run the intra-chunk kernel, then the state pass.  The choice
+ * depends on the shapes only.
  */
 KDA_API kda_status kda_chunk_prefill(const void *q, const void *k, const void *v,
                              const void *g, const void *beta,

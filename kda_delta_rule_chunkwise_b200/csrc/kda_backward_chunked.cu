@@ -435,14 +435,27 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
         dU[t * LD + c] = ws_dU[(item * 64 + t) * D + c];
         dO[t * LD + c] = t < L ? dout[((size_t)(t0 + t) * H + h) * D + c] : 0.f;
     }
-    for (int i = tid; i < 64 * 64; i += NT) {
-        const int r = i >> 6, s2 = i & 63;
-        Tf[r * L6 + s2] = h2f(slot, tr_off(r, s2));
-        Rf[r * L6 + s2] = h2f(slot, tr_off(64 + r, s2));
+    // [T; R] and -W out of the slot by 16-byte pieces (8 fp16 of one row; the
+    // swizzle permutes whole pieces within a row)
+    auto unpack_h8 = [](uint4 u, float *dst) {
+        const __half2 *hp = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(hp[e]);
+            dst[2 * e] = f.x;
+            dst[2 * e + 1] = f.y;
+        }
+    };
+    for (int i = tid; i < 128 * 8; i += NT) {   // [T; R]: 128 rows x 8 pieces
+        const int r = i >> 3, pc = i & 7, lc = pc ^ (r & 7);
+        const uint4 u = *reinterpret_cast<const uint4 *>(slot + kSlotTR + (r >> 3) * 1024 + (r & 7) * 128 + pc * 16);
+        unpack_h8(u, r < 64 ? Tf + r * L6 + 8 * lc : Rf + (r - 64) * L6 + 8 * lc);
     }
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int t = i >> 7, c = i & 127;
-        Wnf[t * LD + c] = h2f(slot, wp_off(t, c));
+    for (int i = tid; i < 64 * 16; i += NT) {   // -W: rows 0..63 of [-W; P], 2 x 8 pieces per row
+        const int r = i >> 4, kb = (i >> 3) & 1, pc = i & 7, lc = pc ^ (r & 7);
+        const uint4 u = *reinterpret_cast<const uint4 *>(slot + kSlotWP + kb * 16384 + (r >> 3) * 1024 +
+                                                         (r & 7) * 128 + pc * 16);
+        unpack_h8(u, Wnf + r * LD + 64 * kb + 8 * lc);
     }
     __syncthreads();
     auto Tm = [&](int r, int s2) { return Tf[r * L6 + s2]; };   // T[r][s]

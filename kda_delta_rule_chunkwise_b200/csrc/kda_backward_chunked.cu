@@ -428,12 +428,23 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     float *Wnf = reinterpret_cast<float *>(sm + F_WN);
     float *out = fg + item * FG_FLOATS;
 
-    // ---- phase 1: V, dU, dO, [T; R] and [-W; P] in shared memory
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int t = i >> 7, c = i & 127;
-        V[t * LD + c] = t < L ? to_f32(v[((size_t)(t0 + t) * H + h) * D + c]) : 0.f;
-        dU[t * LD + c] = ws_dU[(item * 64 + t) * D + c];
-        dO[t * LD + c] = t < L ? dout[((size_t)(t0 + t) * H + h) * D + c] : 0.f;
+    const float *Sg = chunk_state(hdr, packed, T, N, H, n, h, j, state_in, snaps);
+    const float *dSg = ws_dS + item * D * D;
+    if (tid == 0) {   // S and dS' (64 KB each) are read in phases 2 and 3: start them toward L2
+        if (Sg) prefetch_l2(Sg, D * D * 4);
+        prefetch_l2(dSg, D * D * 4);
+    }
+    // ---- phase 1: V, dU, dO, [T; R] and [-W; P] in shared memory, 16 bytes
+    // per load (rows of 128 channels; every base is 16-byte aligned)
+    for (int i = tid; i < 64 * 32; i += NT) {
+        const int t = i >> 5, c = (i & 31) * 4;
+        const size_t off = ((size_t)(t0 + t) * H + h) * D + c;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(V + t * LD + c) = t < L ? load4_f32(v + off) : z;
+        *reinterpret_cast<float4 *>(dU + t * LD + c) =
+            *reinterpret_cast<const float4 *>(ws_dU + (item * 64 + t) * D + c);
+        *reinterpret_cast<float4 *>(dO + t * LD + c) =
+            t < L ? *reinterpret_cast<const float4 *>(dout + off) : z;
     }
     // [T; R] and -W out of the slot by 16-byte pieces (8 fp16 of one row; the
     // swizzle permutes whole pieces within a row)
@@ -481,12 +492,10 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
 
     // ---- phase 2: S
     float *S = reinterpret_cast<float *>(sm + F_R0);
-    {
-        const float *Sg = chunk_state(hdr, packed, T, N, H, n, h, j, state_in, snaps);
-        for (int i = tid; i < 128 * 128; i += NT) {
-            const int c = i >> 7, jj = i & 127;
-            S[c * LD + jj] = Sg ? Sg[i] : 0.f;
-        }
+    for (int i = tid; i < 128 * 32; i += NT) {
+        const int c = i >> 5, jj = (i & 31) * 4;
+        *reinterpret_cast<float4 *>(S + c * LD + jj) =
+            Sg ? *reinterpret_cast<const float4 *>(Sg + c * 128 + jj) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
     // U += (-W) S   (the slot holds -W)
@@ -499,9 +508,9 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
 
     // ---- phase 3: dS'
     float *dSp = reinterpret_cast<float *>(sm + F_R1);
-    for (int i = tid; i < 128 * 128; i += NT) {
-        const int c = i >> 7, jj = i & 127;
-        dSp[c * LD + jj] = ws_dS[item * D * D + i];
+    for (int i = tid; i < 128 * 32; i += NT) {
+        const int c = i >> 5, jj = (i & 31) * 4;
+        *reinterpret_cast<float4 *>(dSp + c * LD + jj) = *reinterpret_cast<const float4 *>(dSg + c * 128 + jj);
     }
     __syncthreads();
     if (tid < 128) {

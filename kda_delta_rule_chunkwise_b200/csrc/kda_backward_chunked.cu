@@ -555,9 +555,14 @@ template <typename Tin>
 __device__ __forceinline__ void chunk_cumsum(const Tin *g, int64_t t0, int H, int h, int L, float *G,
                                              float *Rref) {
     const int tid = threadIdx.x;
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int r = i >> 7, c = i & 127;
-        G[r * LD + c] = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + c]), -5.f) : 0.f;
+    for (int i = tid; i < 64 * 32; i += NT) {   // 4 channels per load
+        const int r = i >> 5, c = (i & 31) * 4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < L) {
+            x = load4_f32(g + ((size_t)(t0 + r) * H + h) * D + c);
+            x = make_float4(fmaxf(x.x, -5.f), fmaxf(x.y, -5.f), fmaxf(x.z, -5.f), fmaxf(x.w, -5.f));
+        }
+        *reinterpret_cast<float4 *>(G + r * LD + c) = x;
     }
     __syncthreads();
     if (tid < 128) {
@@ -598,14 +603,20 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
     float *out = iw + ((size_t)cidx * H + h) * IW_FLOATS;
     chunk_cumsum(g, t0, H, h, L, G, Rref);
     __syncthreads();
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int r = i >> 7, c = i & 127;
-        const float e1 = __expf(G[r * LD + c] - Rref[(r >> 4) * 128 + c]);
-        const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
-        const float kk = r < L ? to_f32(k[off]) : 0.f;
-        QE[r * LD + c] = r < L ? to_f32(q[off]) * e1 : 0.f;
-        KE[r * LD + c] = kk * e1;
-        Kr[r * LD + c] = kk;
+    for (int i = tid; i < 64 * 32; i += NT) {   // 4 channels per load
+        const int r = i >> 5, c0 = (i & 31) * 4;
+        const size_t off = ((size_t)(t0 + r) * H + h) * D + c0;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 k4 = r < L ? load4_f32(k + off) : z, q4 = r < L ? load4_f32(q + off) : z;
+        const float ka[4] = {k4.x, k4.y, k4.z, k4.w}, qa[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int c = c0 + e;
+            const float e1 = __expf(G[r * LD + c] - Rref[(r >> 4) * 128 + c]);
+            QE[r * LD + c] = qa[e] * e1;
+            KE[r * LD + c] = ka[e] * e1;
+            Kr[r * LD + c] = ka[e];
+        }
     }
     const int tx = tid & 15, ty = tid >> 4;   // output (row 16a + ty, columns tx + 16 b)
     for (int a = 0; a < 4; ++a) {
@@ -677,35 +688,42 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     float *dPs = Kt + 64 * LD;                             // dP [64][LD]
     float *dWs = dPs + 64 * LD;                            // dW [64][LD]
     float *bs = dWs + 64 * LD;                             // beta [64]
-    for (int i = tid; i < 64 * 64; i += NT) {
-        const int r = i >> 6, s = i & 63;
-        Aq[r * L6 + s] = io[IW_AQK + i];
-        Mm[r * L6 + s] = io[IW_M + i];
+    // all loads in 16-byte pieces of rows (io, fgi: 16-byte aligned workspace
+    // records; q, k, g rows of 128 channels)
+    for (int i = tid; i < 64 * 16; i += NT) {
+        const int r = i >> 4, s = (i & 15) * 4;
+        *reinterpret_cast<float4 *>(Aq + r * L6 + s) = *reinterpret_cast<const float4 *>(io + IW_AQK + r * 64 + s);
+        *reinterpret_cast<float4 *>(Mm + r * L6 + s) = *reinterpret_cast<const float4 *>(io + IW_M + r * 64 + s);
     }
     if (tid < 64) bs[tid] = tid < L ? to_f32(beta[(size_t)(t0 + tid) * H + h]) : 0.f;
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int t = i >> 7, c = i & 127;
-        dPs[t * LD + c] = fgi[FG_DP + i];
-        dWs[t * LD + c] = fgi[FG_DW + i];
+    for (int i = tid; i < 64 * 32; i += NT) {
+        const int t = i >> 5, c = (i & 31) * 4;
+        *reinterpret_cast<float4 *>(dPs + t * LD + c) = *reinterpret_cast<const float4 *>(fgi + FG_DP + t * 128 + c);
+        *reinterpret_cast<float4 *>(dWs + t * LD + c) = *reinterpret_cast<const float4 *>(fgi + FG_DW + t * 128 + c);
     }
     // K * Gamma, Gamma = exp(cumsum(max(g, -5))): the rows of g load in parallel,
     // one thread per channel scans them in place, then the rows of k scale them
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int r = i >> 7, c = i & 127;
-        Kt[r * LD + c] = r < L ? fmaxf(to_f32(g[((size_t)(t0 + r) * H + h) * D + c]), -5.f) : 0.f;
+    // (k waits in dTp..Wk, which are free until the products below)
+    float *Kr = dTp;   // [64][LD] over dTp, dRp and Wk (3 * 64 * L6 >= 64 * LD floats)
+    for (int i = tid; i < 64 * 32; i += NT) {
+        const int r = i >> 5, c = (i & 31) * 4;
+        const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+        if (r < L) {
+            x = load4_f32(g + off);
+            x = make_float4(fmaxf(x.x, -5.f), fmaxf(x.y, -5.f), fmaxf(x.z, -5.f), fmaxf(x.w, -5.f));
+            y = load4_f32(k + off);
+        }
+        *reinterpret_cast<float4 *>(Kt + r * LD + c) = x;
+        *reinterpret_cast<float4 *>(Kr + r * LD + c) = y;
     }
     __syncthreads();
     if (tid < 128) {
         float acc = 0.f;
         for (int r = 0; r < 64; ++r) {
             acc += Kt[r * LD + tid];
-            Kt[r * LD + tid] = __expf(acc);
+            Kt[r * LD + tid] = Kr[r * LD + tid] * __expf(acc);
         }
-    }
-    __syncthreads();
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int r = i >> 7, c = i & 127;
-        Kt[r * LD + c] = r < L ? to_f32(k[((size_t)(t0 + r) * H + h) * D + c]) * Kt[r * LD + c] : 0.f;
     }
     __syncthreads();
     // X = (I + A)^-1, A = Diag(beta) M (strictly lower), by 16 x 16 blocks: the
@@ -821,12 +839,12 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     const float *io = iw + item * IW_FLOATS;
     const float *fgi = fg + item * FG_FLOATS;
     float *G = reinterpret_cast<float *>(sm);             // [64][LS] chunk-local cumsum
-    float *KF = G + 64 * LS;                               // exp(R_a - G_s), block a's
-    float *dG = KF + 64 * LS;                              // dG accumulator
+    float *KK = G + 64 * LS;                               // k_s exp(R_a - G_s), block a's
+    float *dG = KK + 64 * LS;                              // dG accumulator
     float *Dq = dG + 64 * LS;                              // dq accumulator
     float *Dk = Dq + 64 * LS;                              // dk accumulator
-    float *KK = Dk + 64 * LS;                              // k_s exp(R_a - G_s)
-    float *AE = KK + 64 * LS;                              // a_r E1_r for the 16 rows of block a
+    float *Ks = Dk + 64 * LS;                              // k (0 past the chunk's end)
+    float *AE = Ks + 64 * LS;                              // a_r E1_r for the 16 rows of block a
     float *dFs = AE + 16 * LS;                             // dAqk, then dM  [64][L6]
     float *Rref = dFs + 64 * L6;                           // [4][CW]
     uint32_t *below = reinterpret_cast<uint32_t *>(Rref + 4 * CW);   // [64]: bit cc set where g < -5
@@ -835,11 +853,20 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     // dg), then one thread per channel scans them in shared memory
     if (tid < 64) below[tid] = 0u;
     __syncthreads();
-    for (int i = tid; i < 64 * CW; i += NT) {
-        const int r = i / CW, cc = i % CW;
-        const float x = r < L ? to_f32(g[((size_t)(t0 + r) * H + h) * D + cb + cc]) : 0.f;
-        G[r * LS + cc] = fmaxf(x, -5.f) * (r < L ? 1.f : 0.f);
-        if (r < L && !(x >= -5.f)) atomicOr(&below[r], 1u << cc);
+    for (int i = tid; i < 64 * (CW / 4); i += NT) {   // 4 channels per load
+        const int r = i / (CW / 4), cc = (i % (CW / 4)) * 4;
+        const size_t off = ((size_t)(t0 + r) * H + h) * D + cb + cc;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+        if (r < L) {
+            x = load4_f32(g + off);
+            y = load4_f32(k + off);
+            const uint32_t m = (!(x.x >= -5.f) ? 1u : 0u) | (!(x.y >= -5.f) ? 2u : 0u) |
+                               (!(x.z >= -5.f) ? 4u : 0u) | (!(x.w >= -5.f) ? 8u : 0u);
+            if (m) atomicOr(&below[r], m << cc);
+            x = make_float4(fmaxf(x.x, -5.f), fmaxf(x.y, -5.f), fmaxf(x.z, -5.f), fmaxf(x.w, -5.f));
+        }
+        *reinterpret_cast<float4 *>(G + r * LS + cc) = x;
+        *reinterpret_cast<float4 *>(Ks + r * LS + cc) = y;
     }
     __syncthreads();
     if (tid < CW) {
@@ -855,64 +882,107 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     auto qv = [&](int r, int cc) {
         return r < L ? to_f32(q[((size_t)(t0 + r) * H + h) * D + cb + cc]) : 0.f;
     };
-    auto kv = [&](int r, int cc) {
-        return r < L ? to_f32(k[((size_t)(t0 + r) * H + h) * D + cb + cc]) : 0.f;
-    };
+    auto kv = [&](int r, int cc) { return Ks[r * LS + cc]; };
     const float *gl = G + 63 * LS;   // G at the last row = G_L (rows past L add nothing)
     // the elementwise terms
-    for (int i = tid; i < 64 * CW; i += NT) {
-        const int r = i / CW, cc = i % CW, c = cb + cc;
-        const float Gr = G[r * LS + cc], gam = __expf(Gr), kh_f = __expf(gl[cc] - Gr);
-        const float qq = qv(r, cc), kk = kv(r, cc);
-        const float dP = fgi[FG_DP + r * 128 + c], dKt = io[IW_DKT + r * 128 + c];
-        const float dKh = fgi[FG_DKH + r * 128 + c];
-        Dq[r * LS + cc] = dP * gam;
-        Dk[r * LS + cc] = dKt * gam + dKh * kh_f;
-        dG[r * LS + cc] = qq * gam * dP + kk * gam * dKt - kk * kh_f * dKh;
-    }
-    // decayed adjoints: first Aqk with (a, b) = (q, k), then M with (k, k)
-    for (int form = 0; form < 2; ++form) {
-        const float *dF = dFs;
-        __syncthreads();   // the previous form's products are done with dFs
-        for (int i = tid; i < 64 * 64; i += NT)
-            dFs[(i >> 6) * L6 + (i & 63)] = io[(form == 0 ? IW_DAQK : IW_DM) + i];
-        for (int a = 0; a < 4; ++a) {
-            const int ns = 16 * (a + 1);
-            __syncthreads();
-            for (int i = tid; i < 64 * CW; i += NT) {
-                const int s = i / CW, cc = i % CW;
-                KF[s * LS + cc] = s < ns ? __expf(Rref[a * CW + cc] - G[s * LS + cc]) : 0.f;   // exp(R_a - G_s)
-                KK[s * LS + cc] = kv(s, cc) * KF[s * LS + cc];                                   // k_s exp(R_a - G_s)
-            }
-            for (int i = tid; i < 16 * CW; i += NT) {
-                const int r = i / CW, cc = i % CW, rr = 16 * a + r;
-                AE[r * LS + cc] = (form == 0 ? qv(rr, cc) : kv(rr, cc)) * __expf(G[rr * LS + cc] - Rref[a * CW + cc]);
-            }
-            __syncthreads();
-            // da_r (rows of block a) = E1_r sum_s dF[r,s] b_s exp(R_a - G_s), b = k
-            smm<16, CW, 64>([&](int r, int s) { return dF[(16 * a + r) * L6 + s]; },
-                            [&](int s, int cc) { return KK[s * LS + cc]; },
-                            [&](int r, int cc, float x) {
-                                const int rr = 16 * a + r;
-                                const float da = x * __expf(G[rr * LS + cc] - Rref[a * CW + cc]);
-                                const float av = form == 0 ? qv(rr, cc) : kv(rr, cc);
-                                if (form == 0) Dq[rr * LS + cc] += da; else Dk[rr * LS + cc] += da;
-                                dG[rr * LS + cc] += av * da;
-                            });
-            // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s <= 16a + 15
-            smm<64, CW, 16>([&](int s, int r) { return dF[(16 * a + r) * L6 + s]; },
-                            [&](int r, int cc) { return AE[r * LS + cc]; },
-                            [&](int s, int cc, float x) {
-                                if (s >= ns) return;
-                                const float db = x * KF[s * LS + cc];
-                                Dk[s * LS + cc] += db;
-                                dG[s * LS + cc] -= kv(s, cc) * db;
-                            });
+    for (int i = tid; i < 64 * (CW / 4); i += NT) {   // 4 channels per load
+        const int r = i / (CW / 4), cc0 = (i % (CW / 4)) * 4, c0 = cb + cc0;
+        const float4 q4 = r < L ? load4_f32(q + ((size_t)(t0 + r) * H + h) * D + c0)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 dP4 = *reinterpret_cast<const float4 *>(fgi + FG_DP + r * 128 + c0);
+        const float4 dKt4 = *reinterpret_cast<const float4 *>(io + IW_DKT + r * 128 + c0);
+        const float4 dKh4 = *reinterpret_cast<const float4 *>(fgi + FG_DKH + r * 128 + c0);
+        const float qa[4] = {q4.x, q4.y, q4.z, q4.w}, dPa[4] = {dP4.x, dP4.y, dP4.z, dP4.w};
+        const float dKta[4] = {dKt4.x, dKt4.y, dKt4.z, dKt4.w}, dKha[4] = {dKh4.x, dKh4.y, dKh4.z, dKh4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int cc = cc0 + e;
+            const float Gr = G[r * LS + cc], gam = __expf(Gr), kh_f = __expf(gl[cc] - Gr);
+            const float kk = kv(r, cc);
+            Dq[r * LS + cc] = dPa[e] * gam;
+            Dk[r * LS + cc] = dKta[e] * gam + dKha[e] * kh_f;
+            dG[r * LS + cc] = qa[e] * gam * dPa[e] + kk * gam * dKta[e] - kk * kh_f * dKha[e];
         }
+    }
+    // decayed adjoints: first Aqk with (a, b) = (q, k), then M with (k, k).  dF is
+    // lower triangular, so block a's sums run over s <= 16a + 15 only.
+    const int warp = tid >> 5, lane = tid & 31;
+    auto block = [&](auto ac, int form) {
+        constexpr int A = decltype(ac)::value, NS = 16 * (A + 1), KQ = NS / 4;
+        const float *dF = dFs;
+        __syncthreads();   // the previous block's products are done with KK and AE
+        for (int i = tid; i < NS * CW; i += NT) {
+            const int s = i / CW, cc = i % CW;
+            KK[s * LS + cc] = Ks[s * LS + cc] * __expf(Rref[A * CW + cc] - G[s * LS + cc]);
+        }
+        for (int i = tid; i < 16 * CW; i += NT) {
+            const int r = i / CW, cc = i % CW, rr = 16 * A + r;
+            AE[r * LS + cc] = (form == 0 ? qv(rr, cc) : kv(rr, cc)) * __expf(G[rr * LS + cc] - Rref[A * CW + cc]);
+        }
+        __syncthreads();
+        // da_r (rows of block a) = E1_r sum_s dF[r,s] k_s exp(R_a - G_s): warp w takes
+        // rows 16a + 2w, 16a + 2w + 1; lane = 8 kq + cq sums s in the kq-th quarter of
+        // [0, NS) for columns 4 cq .. 4 cq + 3, then the quarters are added across lanes
+        {
+            float acc[2][4];
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+            const int kq = lane >> 3, cq = lane & 7;
+            const float *d0 = dF + (16 * A + 2 * warp) * L6;
+#pragma unroll 4
+            for (int s2 = kq * KQ; s2 < kq * KQ + KQ; ++s2) {
+                const float x0 = d0[s2], x1 = d0[L6 + s2];
+                const float4 b = *reinterpret_cast<const float4 *>(KK + s2 * LS + 4 * cq);
+                acc[0][0] = fmaf(x0, b.x, acc[0][0]); acc[0][1] = fmaf(x0, b.y, acc[0][1]);
+                acc[0][2] = fmaf(x0, b.z, acc[0][2]); acc[0][3] = fmaf(x0, b.w, acc[0][3]);
+                acc[1][0] = fmaf(x1, b.x, acc[1][0]); acc[1][1] = fmaf(x1, b.y, acc[1][1]);
+                acc[1][2] = fmaf(x1, b.z, acc[1][2]); acc[1][3] = fmaf(x1, b.w, acc[1][3]);
+            }
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    acc[x][y] += __shfl_xor_sync(0xffffffffu, acc[x][y], 8);
+                    acc[x][y] += __shfl_xor_sync(0xffffffffu, acc[x][y], 16);
+                }
+            // every lane of a quarter group holds the sums; lane kq finishes row
+            // 2w + (kq >> 1), columns 4 cq + 2 (kq & 1) + e
+            const int rsel = kq >> 1, csel = kq & 1, rr = 16 * A + 2 * warp + rsel;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float x = rsel ? (csel ? acc[1][2 + e] : acc[1][e]) : (csel ? acc[0][2 + e] : acc[0][e]);
+                const int cc = 4 * cq + 2 * csel + e;
+                const float da = x * __expf(G[rr * LS + cc] - Rref[A * CW + cc]);
+                const float av = form == 0 ? qv(rr, cc) : kv(rr, cc);
+                if (form == 0) Dq[rr * LS + cc] += da; else Dk[rr * LS + cc] += da;
+                dG[rr * LS + cc] += av * da;
+            }
+        }
+        __syncthreads();   // block a's rows of Dk and dG take db next
+        // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s < NS
+        smm<NS, CW, 16>([&](int s2, int r) { return dF[(16 * A + r) * L6 + s2]; },
+                        [&](int r, int cc) { return AE[r * LS + cc]; },
+                        [&](int s2, int cc, float x) {
+                            const float db = x * __expf(Rref[A * CW + cc] - G[s2 * LS + cc]);
+                            Dk[s2 * LS + cc] += db;
+                            dG[s2 * LS + cc] -= kv(s2, cc) * db;
+                        });
+    };
+    for (int form = 0; form < 2; ++form) {
+        __syncthreads();   // the previous form's products are done with dFs
+        for (int i = tid; i < 64 * 16; i += NT)
+            *reinterpret_cast<float4 *>(dFs + (i >> 4) * L6 + (i & 15) * 4) =
+                *reinterpret_cast<const float4 *>(io + (form == 0 ? IW_DAQK : IW_DM) + i * 4);
+        block(std::integral_constant<int, 0>{}, form);
+        block(std::integral_constant<int, 1>{}, form);
+        block(std::integral_constant<int, 2>{}, form);
+        block(std::integral_constant<int, 3>{}, form);
     }
     __syncthreads();
     // row L-1 also carries G_L's gradient: sum_r Khat dKhat + Gamma_L dGamma_L (the
-    // sum by 8-row groups over all threads, into KF, which is free now); then dg =
+    // sum by 8-row groups over all threads, into KK, which is free now); then dg =
     // reverse cumsum of dG, 0 where g < -5
     {
         const int cc = tid % CW, rg = tid / CW;   // NT / CW = 8 groups of 8 rows
@@ -921,13 +991,13 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
         for (int r = 8 * rg; r < 8 * rg + 8; ++r)
             if (r < L)
                 part = fmaf(kv(r, cc) * __expf(gl[cc] - G[r * LS + cc]), fgi[FG_DKH + r * 128 + cb + cc], part);
-        KF[rg * LS + cc] = part;
+        KK[rg * LS + cc] = part;
     }
     __syncthreads();
     if (tid < CW && L > 0) {
         const int cc = tid, c = cb + tid;
         float s_kh = 0.f;
-        for (int rg = 0; rg < NT / CW; ++rg) s_kh += KF[rg * LS + cc];
+        for (int rg = 0; rg < NT / CW; ++rg) s_kh += KK[rg * LS + cc];
         dG[(L - 1) * LS + cc] += s_kh + __expf(gl[cc]) * fgi[FG_DGL + c];
         float acc = 0.f;
         for (int r = L - 1; r >= 0; --r) {

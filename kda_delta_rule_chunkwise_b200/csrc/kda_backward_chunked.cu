@@ -214,6 +214,7 @@ constexpr uint32_t CH_GAM = CH_DO + 2 * 64 * CH_LD * 4;           // Gamma_L [12
 constexpr uint32_t CH_BAR = CH_GAM + 128 * 4;                     // slot-copy mbarrier
 constexpr uint32_t CH_SMEM = CH_BAR + 16;
 static_assert(CH_SMEM <= 227 * 1024, "chain kernel shared memory");
+static_assert(CH_DVS == 32 && NT == 256, "chain kernel thread map: 32 x 8 threads, four columns each");
 
 __global__ void __launch_bounds__(NT, 1)
 bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T, int N,
@@ -283,9 +284,10 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
         const int step = nch - 1 - j;
         float *dO = reinterpret_cast<float *>(sm + CH_DO) + (step & 1) * 64 * CH_LD;
         // dS' of this chunk, for the factor kernel
-        for (int i = tid; i < 128 * CH_DVS; i += NT) {
-            const int c = i / CH_DVS, jj = i % CH_DVS;
-            ws_dS[(item * D + c) * D + j0 + jj] = dS[c * CH_LD + jj];
+        for (int i = tid; i < 128 * (CH_DVS / 4); i += NT) {
+            const int c = i / (CH_DVS / 4), jj = (i % (CH_DVS / 4)) * 4;
+            *reinterpret_cast<float4 *>(ws_dS + (item * D + c) * D + j0 + jj) =
+                *reinterpret_cast<const float4 *>(dS + c * CH_LD + jj);
         }
         if (ok) {
             ok = mbar_wait(bar, step & 1, err);   // the slot image has landed
@@ -293,11 +295,18 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
         }
         cp_async_wait_all();                            // this thread's dO pieces have
         __syncthreads();
-        for (int i = tid; i < 64 * 128; i += NT) {
-            const int t = i >> 7, c = i & 127;
-            Kh[t * LDF + c] = h2f(slot, kh_off(t, c));
-            Wn[t * LDF + c] = h2f(slot, wp_off(t, c));
-            Pm[t * LDF + c] = h2f(slot, wp_off(64 + t, c));
+        // Khat, -W and P by 16-byte pieces (8 channels of one row; the swizzle
+        // permutes whole pieces within a row, see kh_off and wp_off)
+        for (int i = tid; i < 3 * 64 * 16; i += NT) {
+            const int part = i >> 10, t = (i >> 4) & 63, kb = (i >> 3) & 1, pc = i & 7, lc = pc ^ (t & 7);
+            const uint32_t off = part == 0 ? kSlotKh + kb * 8192 : kSlotWP + kb * 16384 + (part == 2 ? 8192 : 0);
+            const uint4 u = *reinterpret_cast<const uint4 *>(slot + off + (t >> 3) * 1024 + (t & 7) * 128 + pc * 16);
+            float *dst = (part == 0 ? Kh : part == 1 ? Wn : Pm) + t * LDF + 64 * kb + 8 * lc;
+            const __half2 *hp = reinterpret_cast<const __half2 *>(&u);
+            const float2 f0 = __half22float2(hp[0]), f1 = __half22float2(hp[1]);
+            const float2 f2 = __half22float2(hp[2]), f3 = __half22float2(hp[3]);
+            *reinterpret_cast<float4 *>(dst) = make_float4(f0.x, f0.y, f1.x, f1.y);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
         }
         if (tid < 128) gam[tid] = reinterpret_cast<const float *>(slot + kSlotGam)[tid];
         __syncthreads();   // the image is decoded: the next one may land over it
@@ -305,45 +314,66 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
             issue_slot(j - 1);
             issue_dO(j - 1, reinterpret_cast<float *>(sm + CH_DO) + ((step + 1) & 1) * 64 * CH_LD);
         }
-        // dU = Khat dS'
-        smm<64, CH_DVS, 128>([&](int t, int c) { return Kh[t * LDF + c]; },
-                             [&](int c, int jj) { return dS[c * CH_LD + jj]; },
-                             [&](int t, int jj, float x) { Y[t * CH_LD + jj] = x; });
-        __syncthreads();
-        for (int i = tid; i < 64 * CH_DVS; i += NT) {
-            const int t = i / CH_DVS, jj = i % CH_DVS;
-            ws_dU[(item * 64 + t) * D + j0 + jj] = Y[t * CH_LD + jj];
-        }
-        // dS = Diag(Gamma_L) dS' + P^T dO + (-W)^T dU   (the slot holds -W); each thread
-        // overwrites only the elements it alone reads
+        // thread (q, cq), q = 4 warp + lane / 8, cq = lane % 8, owns columns
+        // 4 cq .. 4 cq + 3 of the slice; operands are read as 16-byte pieces
+        const int cq = tid & 7, q = tid >> 3;
+        // dU = Khat dS': rows 2q, 2q + 1, four channels at a time
         {
-            const int tx = tid & 15, ty = tid >> 4;
-            float r[8][2];
+            float r[2][4];
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
+            for (int x = 0; x < 2; ++x)
 #pragma unroll
-                for (int b = 0; b < 2; ++b) r[a][b] = gam[ty + 16 * a] * dS[(ty + 16 * a) * CH_LD + tx + 16 * b];
+                for (int e = 0; e < 4; ++e) r[x][e] = 0.f;
+            const float *k0 = Kh + 2 * q * LDF;
 #pragma unroll 2
-            for (int t = 0; t < 64; ++t) {
-                float pw[8], wn[8];
+            for (int c = 0; c < 128; c += 4) {
+                const float4 a0 = *reinterpret_cast<const float4 *>(k0 + c);
+                const float4 a1 = *reinterpret_cast<const float4 *>(k0 + LDF + c);
+                const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-                for (int a = 0; a < 8; ++a) {
-                    pw[a] = Pm[t * LDF + ty + 16 * a];
-                    wn[a] = Wn[t * LDF + ty + 16 * a];
-                }
-                const float o0 = dO[t * CH_LD + tx], o1 = dO[t * CH_LD + tx + 16];
-                const float y0 = Y[t * CH_LD + tx], y1 = Y[t * CH_LD + tx + 16];
-#pragma unroll
-                for (int a = 0; a < 8; ++a) {
-                    r[a][0] = fmaf(pw[a], o0, fmaf(wn[a], y0, r[a][0]));
-                    r[a][1] = fmaf(pw[a], o1, fmaf(wn[a], y1, r[a][1]));
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float4 b = *reinterpret_cast<const float4 *>(dS + (c + kk) * CH_LD + 4 * cq);
+                    r[0][0] = fmaf(av0[kk], b.x, r[0][0]); r[0][1] = fmaf(av0[kk], b.y, r[0][1]);
+                    r[0][2] = fmaf(av0[kk], b.z, r[0][2]); r[0][3] = fmaf(av0[kk], b.w, r[0][3]);
+                    r[1][0] = fmaf(av1[kk], b.x, r[1][0]); r[1][1] = fmaf(av1[kk], b.y, r[1][1]);
+                    r[1][2] = fmaf(av1[kk], b.z, r[1][2]); r[1][3] = fmaf(av1[kk], b.w, r[1][3]);
                 }
             }
-            __syncthreads();
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
+            for (int x = 0; x < 2; ++x) {
+                const float4 o = make_float4(r[x][0], r[x][1], r[x][2], r[x][3]);
+                *reinterpret_cast<float4 *>(Y + (2 * q + x) * CH_LD + 4 * cq) = o;
+                *reinterpret_cast<float4 *>(ws_dU + (item * 64 + 2 * q + x) * D + j0 + 4 * cq) = o;
+            }
+        }
+        __syncthreads();
+        // dS = Diag(Gamma_L) dS' + P^T dO + (-W)^T dU   (the slot holds -W): channels
+        // 4q .. 4q + 3; each thread overwrites only the elements it alone reads
+        {
+            float r[4][4];
 #pragma unroll
-                for (int b = 0; b < 2; ++b) dS[(ty + 16 * a) * CH_LD + tx + 16 * b] = r[a][b];
+            for (int x = 0; x < 4; ++x) {
+                const float4 d = *reinterpret_cast<const float4 *>(dS + (4 * q + x) * CH_LD + 4 * cq);
+                const float gm = gam[4 * q + x];
+                r[x][0] = gm * d.x; r[x][1] = gm * d.y; r[x][2] = gm * d.z; r[x][3] = gm * d.w;
+            }
+#pragma unroll 4
+            for (int t = 0; t < 64; ++t) {
+                const float4 pw = *reinterpret_cast<const float4 *>(Pm + t * LDF + 4 * q);
+                const float4 wn = *reinterpret_cast<const float4 *>(Wn + t * LDF + 4 * q);
+                const float4 o = *reinterpret_cast<const float4 *>(dO + t * CH_LD + 4 * cq);
+                const float4 y = *reinterpret_cast<const float4 *>(Y + t * CH_LD + 4 * cq);
+                const float pv[4] = {pw.x, pw.y, pw.z, pw.w}, wv[4] = {wn.x, wn.y, wn.z, wn.w};
+                const float ov[4] = {o.x, o.y, o.z, o.w}, yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) r[x][e] = fmaf(pv[x], ov[e], fmaf(wv[x], yv[e], r[x][e]));
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                *reinterpret_cast<float4 *>(dS + (4 * q + x) * CH_LD + 4 * cq) =
+                    make_float4(r[x][0], r[x][1], r[x][2], r[x][3]);
         }
         __syncthreads();   // dS, Y and this dO buffer are consumed
     }

@@ -254,9 +254,9 @@ KDA_API kda_status kda_decode_step_indexed(const void *q, const void *k, const v
  * states from stored chunk starts; with few (sequence, head) units the value
  * columns are split over several CTAs whose partial sums are added in a fixed
  * order, so results are the same on every run).
- *  For bf16 with dk = 128 (the chunked form) q, k, v, g and do must be 16-byte
- *  aligned, else KDA_ERR_INVALID_ARG; state_in, dstate_out and dstate_in
- *  always must.
+ *  For bf16 with dk = 128 (the chunked form) q, k, v, g, do and dv must be
+ *  16-byte aligned, else KDA_ERR_INVALID_ARG; state_in, dstate_out and
+ *  dstate_in always must.
  *  workspace  at least kda_backward_workspace_bytes() bytes, 16-byte aligned
  *             (chunk-start states, per-token states of one chunk per unit, and
  *             the partial sums when the columns are split)

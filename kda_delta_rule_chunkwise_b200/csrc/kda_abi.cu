@@ -304,7 +304,7 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const void 
                   (reinterpret_cast<uintptr_t>(workspace) & (chunked ? 255u : 15u)) != 0))
         return KDA_ERR_INVALID_ARG;
     if (chunked && rows > 0) {
-        for (const void *p : {q, k, g, v, (const void *)dout})
+        for (const void *p : {q, k, g, v, (const void *)dout, (const void *)dv_out})
             if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return KDA_ERR_INVALID_ARG;
         if (rows > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
     }

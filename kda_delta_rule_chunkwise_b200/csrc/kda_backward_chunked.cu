@@ -404,7 +404,8 @@ constexpr uint32_t F_RR = F_T + 64 * L6 * 4;             //   R [64][L6]
 constexpr uint32_t F_R1 = F_RR + 64 * L6 * 4;           // dU [64][LD] + dO [64][LD] | dS' [128][LD]
 constexpr uint32_t F_R2 = F_R1 + 128 * LD * 4;           // U [64][LD] (dV first)
 constexpr uint32_t F_WN = F_R2 + 64 * LD * 4;            // -W [64][LD]
-constexpr uint32_t F_SMEM = F_WN + 64 * LD * 4;
+constexpr uint32_t F_BAR = F_WN + 64 * LD * 4;             // 3 mbarriers: dU + dO, S, dS'
+constexpr uint32_t F_SMEM = F_BAR + 32;
 static_assert(128 * LD * 4 <= F_R1, "factor kernel layout: S fits the first region");
 static_assert(F_SMEM <= 227 * 1024, "factor kernel shared memory");
 
@@ -433,7 +434,7 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
                   int H, const Tin *__restrict__ v, const float *state_in,
                   const float *__restrict__ snaps, const float *__restrict__ dout,
                   const float *__restrict__ ws_dS, const float *__restrict__ ws_dU,
-                  float *__restrict__ fg, float *__restrict__ dv, uint32_t hdr_bytes) {
+                  float *__restrict__ fg, float *__restrict__ dv, uint32_t hdr_bytes, uint32_t *err) {
     extern __shared__ __align__(16) uint8_t sm[];
     const int tid = threadIdx.x;
     const int32_t *hdr = reinterpret_cast<const int32_t *>(fws);
@@ -460,21 +461,37 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
 
     const float *Sg = chunk_state(hdr, packed, T, N, H, n, h, j, state_in, snaps);
     const float *dSg = ws_dS + item * D * D;
-    if (tid == 0) {   // S and dS' (64 KB each) are read in phases 2 and 3: start them toward L2
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + F_BAR);
+    if (tid == 0) {
+        // S and dS' (64 KB each) are read in phases 2 and 3: start them toward L2
         if (Sg) prefetch_l2(Sg, D * D * 4);
         prefetch_l2(dSg, D * D * 4);
+        for (int b = 0; b < 3; ++b) mbar_init(&bars[b], 1);
+        mbar_fence_init();
     }
-    // ---- phase 1: V, dU, dO, [T; R] and [-W; P] in shared memory, 16 bytes
-    // per load (rows of 128 channels; every base is 16-byte aligned)
+    __syncthreads();
+    // The fp32 operands dU, dO, S and dS' come in by bulk copies, one per 512-byte
+    // row, each group completing on its own barrier; the issuing threads fence
+    // against the generic accesses the region saw before (barrier first).
+    auto copy_rows = [&](float *dst, const float *src, size_t src_stride, int rows, int t_lo, uint64_t *bar) {
+        const int t = tid - t_lo;
+        if (t >= 0 && t < rows) {
+            fence_async_smem();
+            bulk_g2s(dst + t * LD, src + (size_t)t * src_stride, 512, bar);
+        }
+    };
+    // ---- phase 1: dU, dO (rows past the chunk's end are zero) by bulk copies;
+    // V, [T; R] and -W by 16-byte loads (rows of 128 channels; every base is
+    // 16-byte aligned)
+    if (tid == 0) mbar_arrive_expect_tx(&bars[0], (uint32_t)(64 + L) * 512u);
+    copy_rows(dU, ws_dU + item * 64 * D, D, 64, 0, &bars[0]);
+    copy_rows(dO, dout + ((size_t)t0 * H + h) * D, (size_t)H * D, L, 64, &bars[0]);
     for (int i = tid; i < 64 * 32; i += NT) {
         const int t = i >> 5, c = (i & 31) * 4;
         const size_t off = ((size_t)(t0 + t) * H + h) * D + c;
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<float4 *>(V + t * LD + c) = t < L ? load4_f32(v + off) : z;
-        *reinterpret_cast<float4 *>(dU + t * LD + c) =
-            *reinterpret_cast<const float4 *>(ws_dU + (item * 64 + t) * D + c);
-        *reinterpret_cast<float4 *>(dO + t * LD + c) =
-            t < L ? *reinterpret_cast<const float4 *>(dout + off) : z;
+        if (t >= L) *reinterpret_cast<float4 *>(dO + t * LD + c) = z;
     }
     // [T; R] and -W out of the slot by 16-byte pieces (8 fp16 of one row; the
     // swizzle permutes whole pieces within a row)
@@ -498,7 +515,18 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
                                                          (r & 7) * 128 + pc * 16);
         unpack_h8(u, Wnf + r * LD + 64 * kb + 8 * lc);
     }
-    __syncthreads();
+    // a copy given up on (after a timeout) lands before the CTA exits; the item's
+    // results are then not written (the error word says why)
+    auto drain = [&](int nb) {
+        if (tid == 0)
+            for (int b = 0; b < nb; ++b)
+                if (b != 1 || Sg) mbar_wait(&bars[b], 0, err, 1ull << 28);
+        __syncthreads();
+    };
+    if (!__syncthreads_and(mbar_wait(&bars[0], 0, err))) {
+        drain(1);
+        return;
+    }
     auto Tm = [&](int r, int s2) { return Tf[r * L6 + s2]; };   // T[r][s]
     auto Rm = [&](int r, int s2) { return Rf[r * L6 + s2]; };   // R[r][s]
     // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out)
@@ -507,9 +535,11 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     smm_pb<64, 128, 64>([&](int s, int t) { return Rm(t, s); }, dO, LD,
                         [&](int s, int c, float x) { U[s * LD + c] += x; });
     __syncthreads();
-    for (int i = tid; i < 64 * 128; i += NT) {
-        const int s = i >> 7, c = i & 127;
-        if (s < L) dv[((size_t)(t0 + s) * H + h) * D + c] = U[s * LD + c];
+    for (int i = tid; i < 64 * 32; i += NT) {
+        const int s = i >> 5, c = (i & 31) * 4;
+        if (s < L)
+            *reinterpret_cast<float4 *>(dv + ((size_t)(t0 + s) * H + h) * D + c) =
+                *reinterpret_cast<const float4 *>(U + s * LD + c);
     }
     // dT = dU V^T, dR = dO V^T
     smm_nt<64, 64, 128>(dU, LD, V, LD, [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; });
@@ -520,14 +550,19 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
                         [&](int t, int c, float x) { U[t * LD + c] = x; });
     __syncthreads();   // V and [T; R] are consumed
 
-    // ---- phase 2: S
+    // ---- phase 2: S (zero without an initial state)
     float *S = reinterpret_cast<float *>(sm + F_R0);
-    for (int i = tid; i < 128 * 32; i += NT) {
-        const int c = i >> 5, jj = (i & 31) * 4;
-        *reinterpret_cast<float4 *>(S + c * LD + jj) =
-            Sg ? *reinterpret_cast<const float4 *>(Sg + c * 128 + jj) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (Sg) {
+        if (tid == 0) mbar_arrive_expect_tx(&bars[1], 128u * 512u);
+        copy_rows(S, Sg, D, 128, 0, &bars[1]);
+    } else {
+        for (int i = tid; i < 128 * 32; i += NT)
+            *reinterpret_cast<float4 *>(S + (i >> 5) * LD + (i & 31) * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
+    if (!__syncthreads_and(Sg ? mbar_wait(&bars[1], 0, err) : true)) {
+        drain(2);
+        return;
+    }
     // U += (-W) S   (the slot holds -W)
     smm_pb<64, 128, 128>([&](int t, int c) { return Wnf[t * LD + c]; }, S, LD,
                          [&](int t, int jj, float x) { U[t * LD + jj] += x; });
@@ -538,11 +573,12 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
 
     // ---- phase 3: dS'
     float *dSp = reinterpret_cast<float *>(sm + F_R1);
-    for (int i = tid; i < 128 * 32; i += NT) {
-        const int c = i >> 5, jj = (i & 31) * 4;
-        *reinterpret_cast<float4 *>(dSp + c * LD + jj) = *reinterpret_cast<const float4 *>(dSg + c * 128 + jj);
+    if (tid == 0) mbar_arrive_expect_tx(&bars[2], 128u * 512u);
+    copy_rows(dSp, dSg, D, 128, 0, &bars[2]);
+    if (!__syncthreads_and(mbar_wait(&bars[2], 0, err))) {
+        drain(3);
+        return;
     }
-    __syncthreads();
     if (tid < 128) {
         float a = 0.f;
         for (int jj = 0; jj < 128; ++jj) a = fmaf(dSp[tid * LD + jj], S[tid * LD + jj], a);
@@ -627,8 +663,8 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
     float *G = reinterpret_cast<float *>(sm);              // [64][LD]
     float *QE = G + 64 * LD;                               // q_r E1_r
     float *KE = QE + 64 * LD;                              // k_r E1_r
-    float *KFt = KE + 64 * LD;                             // [128][L6]: k_s exp(R_a - G_s), block a's
-    float *Rref = KFt + 128 * L6;                          // [4][128]
+    float *KF = KE + 64 * LD;                              // [64][LD]: k_s exp(R_a - G_s), block a's
+    float *Rref = KF + 64 * LD;                            // [4][128]
     float *Kr = Rref + 4 * 128;                            // [64][LD]: k (0 past the chunk's end)
     float *out = iw + ((size_t)cidx * H + h) * IW_FLOATS;
     chunk_cumsum(g, t0, H, h, L, G, Rref);
@@ -649,40 +685,51 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
         }
     }
     const int tx = tid & 15, ty = tid >> 4;   // output (row 16a + ty, columns tx + 16 b)
-    for (int a = 0; a < 4; ++a) {
-        const int ns = 16 * (a + 1);   // rows s <= 16a + 15
+    // block a of rows needs columns s <= 16a + 15 only (both forms are lower triangular)
+    auto block = [&](auto ac) {
+        constexpr int A = decltype(ac)::value, NS = 16 * (A + 1), NB = A + 1;
         __syncthreads();
-        // k_s exp(R_a - G_s) stored channel-major, so that the product below reads
-        // consecutive s across a half-warp (conflict-free)
-        for (int i = tid; i < 64 * 128; i += NT) {
-            const int s = i & 63, c = i >> 6;
-            KFt[c * L6 + s] = s < ns ? Kr[s * LD + c] * __expf(Rref[a * 128 + c] - G[s * LD + c]) : 0.f;
+        // k_s exp(R_a - G_s) for s < NS, row-major like k
+        for (int i = tid; i < NS * 32; i += NT) {
+            const int s2 = i >> 5, c = (i & 31) * 4;
+            const float4 kr = *reinterpret_cast<const float4 *>(Kr + s2 * LD + c);
+            const float4 g4 = *reinterpret_cast<const float4 *>(G + s2 * LD + c);
+            const float4 rf = *reinterpret_cast<const float4 *>(Rref + A * 128 + c);
+            *reinterpret_cast<float4 *>(KF + s2 * LD + c) =
+                make_float4(kr.x * __expf(rf.x - g4.x), kr.y * __expf(rf.y - g4.y),
+                            kr.z * __expf(rf.z - g4.z), kr.w * __expf(rf.w - g4.w));
         }
         __syncthreads();
         // rows 16a .. 16a + 15 of Aqk (s <= r) and of M (s < r) in one pass over the
         // channels (the two share the decayed k operand); sums over c in order
-        float ra_[4], rm_[4];
+        float ra_[NB], rm_[NB];
 #pragma unroll
-        for (int b2 = 0; b2 < 4; ++b2) ra_[b2] = rm_[b2] = 0.f;
-        const float *qe = QE + (16 * a + ty) * LD, *ke = KE + (16 * a + ty) * LD;
-#pragma unroll 4
-        for (int c = 0; c < 128; ++c) {
-            const float x = qe[c], y = ke[c];
+        for (int b2 = 0; b2 < NB; ++b2) ra_[b2] = rm_[b2] = 0.f;
+        const float *qe = QE + (16 * A + ty) * LD, *ke = KE + (16 * A + ty) * LD;
+#pragma unroll 2
+        for (int c = 0; c < 128; c += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(qe + c);
+            const float4 y = *reinterpret_cast<const float4 *>(ke + c);
 #pragma unroll
-            for (int b2 = 0; b2 < 4; ++b2) {
-                const float kf = KFt[c * L6 + tx + 16 * b2];
-                ra_[b2] = fmaf(x, kf, ra_[b2]);
-                rm_[b2] = fmaf(y, kf, rm_[b2]);
+            for (int b2 = 0; b2 < NB; ++b2) {
+                const float4 kf = *reinterpret_cast<const float4 *>(KF + (tx + 16 * b2) * LD + c);
+                ra_[b2] = fmaf(x.w, kf.w, fmaf(x.z, kf.z, fmaf(x.y, kf.y, fmaf(x.x, kf.x, ra_[b2]))));
+                rm_[b2] = fmaf(y.w, kf.w, fmaf(y.z, kf.z, fmaf(y.y, kf.y, fmaf(y.x, kf.x, rm_[b2]))));
             }
         }
-        const int r = 16 * a + ty;
+        const int r = 16 * A + ty;
 #pragma unroll
         for (int b2 = 0; b2 < 4; ++b2) {
             const int s2 = tx + 16 * b2;
-            out[IW_AQK + r * 64 + s2] = s2 <= r ? ra_[b2] : 0.f;
-            out[IW_M + r * 64 + s2] = s2 < r ? rm_[b2] : 0.f;
+            const float va = b2 < NB ? ra_[b2 < NB ? b2 : 0] : 0.f, vm = b2 < NB ? rm_[b2 < NB ? b2 : 0] : 0.f;
+            out[IW_AQK + r * 64 + s2] = s2 <= r ? va : 0.f;
+            out[IW_M + r * 64 + s2] = s2 < r ? vm : 0.f;
         }
-    }
+    };
+    block(std::integral_constant<int, 0>{});
+    block(std::integral_constant<int, 1>{});
+    block(std::integral_constant<int, 2>{});
+    block(std::integral_constant<int, 3>{});
 }
 
 template <typename Tin>
@@ -1123,10 +1170,10 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
     const unsigned items = (unsigned)(L.max_chunks * a.H);
     if ((e = set_smem(bwd_factor_kernel<bf>, F_SMEM)) != cudaSuccess) return e;
     bwd_factor_kernel<bf><<<items, NT, F_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.v,
-                                                     a.state_in, snaps, a.dout, dS, dU, fg, a.dv, hb);
+                                                     a.state_in, snaps, a.dout, dS, dU, fg, a.dv, hb, a.err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t RC_SMEM = 4 * 64 * LD * 4 + 128 * L6 * 4 + 4 * 128 * 4;
+    constexpr uint32_t RC_SMEM = 5 * 64 * LD * 4 + 4 * 128 * 4;   // G, QE, KE, KF, Rref, k
     if ((e = set_smem(bwd_recompute_kernel<bf>, RC_SMEM)) != cudaSuccess) return e;
     bwd_recompute_kernel<bf><<<items, NT, RC_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
                                                          (const bf *)a.k, (const bf *)a.g, iw);

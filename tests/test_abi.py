@@ -211,8 +211,10 @@ def raw_bwd(a):
     (dict(dtype=5), "KDA_ERR_INVALID_ARG"), (dict(state_in=8), "KDA_ERR_INVALID_ARG"),
     (dict(dk=96, dv=96), "KDA_ERR_UNSUPPORTED"),
     (dict(), "KDA_ERR_INVALID_ARG"),             # no workspace
-    # the chunked form (bf16, d = 128) reads do in 16-byte pieces
+    # the chunked form (bf16, d = 128) reads do and writes dv in 16-byte pieces
     (dict(dtype=binding.KDA_BF16, dk=128, dv=128, ws=256, wsb=1 << 40, do=104),
+     "KDA_ERR_INVALID_ARG"),
+    (dict(dtype=binding.KDA_BF16, dk=128, dv=128, ws=256, wsb=1 << 40, dvv=136),
      "KDA_ERR_INVALID_ARG")])
 def test_backward_rejects(lib, bad, code):
     assert raw_bwd(_bargs(**bad)) == getattr(binding, code)

@@ -91,6 +91,55 @@ __device__ __forceinline__ void smm(FA A, FB B, FO out) {
         for (int b = 0; b < TN; ++b) out(ty + 16 * a, tx + 16 * b, r[a][b]);
 }
 
+// 64-row products whose terms vanish outside a band of k that depends on the
+// row: thread (ty, tx) owns the four consecutive rows 4 ty .. 4 ty + 3 (so warp w
+// owns rows 8w .. 8w + 7) and columns tx + 16 b, and sums
+//   out(i, j, sum_{k in [lo1, hi1)} A1(i, k) B1(k, j) + sum_{k in [lo2, hi2)} A2(i, k) B2(k, j))
+// with the ranges taken per warp (range(w, lo1, hi1, lo2, hi2)), in order of k.
+template <int N, typename FA1, typename FB1, typename FA2, typename FB2, typename FR, typename FO>
+__device__ __forceinline__ void smm_rows2(FA1 A1, FB1 B1, FA2 A2, FB2 B2, FR range, FO out) {
+    constexpr int TM = 4, TN = N / 16;
+    static_assert(N % 16 == 0, "tile");
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    int lo1, hi1, lo2, hi2;
+    range(threadIdx.x >> 5, lo1, hi1, lo2, hi2);
+    float r[TM][TN];
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < TN; ++b) r[a][b] = 0.f;
+    auto run = [&](auto A, auto B, int lo, int hi) {
+#pragma unroll 4
+        for (int k = lo; k < hi; ++k) {
+            float av[TM], bv[TN];
+#pragma unroll
+            for (int a = 0; a < TM; ++a) av[a] = A(TM * ty + a, k);
+#pragma unroll
+            for (int b = 0; b < TN; ++b) bv[b] = B(k, tx + 16 * b);
+#pragma unroll
+            for (int a = 0; a < TM; ++a)
+#pragma unroll
+                for (int b = 0; b < TN; ++b) r[a][b] = fmaf(av[a], bv[b], r[a][b]);
+        }
+    };
+    run(A1, B1, lo1, hi1);
+    run(A2, B2, lo2, hi2);
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < TN; ++b) out(TM * ty + a, tx + 16 * b, r[a][b]);
+}
+// one product: the second pair is empty
+template <int N, typename FA, typename FB, typename FR, typename FO>
+__device__ __forceinline__ void smm_rows(FA A, FB B, FR range, FO out) {
+    smm_rows2<N>(A, B, A, B,
+                 [&](int w, int &lo1, int &hi1, int &lo2, int &hi2) {
+                     range(w, lo1, hi1);
+                     lo2 = hi2 = 0;
+                 },
+                 out);
+}
+
 // The same product when both operands are row-major fp32 with K contiguous:
 // out(i, j, sum_k A[i][k] B[j][k]) (A times B transposed), four k at a time as
 // 16-byte loads (lda, ldb multiples of 4, K a multiple of 4).  Same thread
@@ -837,38 +886,45 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     block_row(std::integral_constant<int, 1>{});
     block_row(std::integral_constant<int, 2>{});
     block_row(std::integral_constant<int, 3>{});
-    // R = Aqk T, T = X Diag(beta)
-    smm<64, 64, 64>([&](int r, int m) { return Aq[r * L6 + m]; }, [&](int m, int s) { return X[m * L6 + s] * bs[s]; },
-                    [&](int r, int s, float x) { Rm[r * L6 + s] = x; });
+    // The lower-triangular factors (Aqk, X, T, R) make most of the sums below
+    // run over a band of k: a warp's rows 8w .. 8w + 7 need k <= 8w + 7 or k >= 8w.
+    auto k_upto = [](int w, int &lo, int &hi) { lo = 0; hi = 8 * w + 8; };
+    auto k_from = [](int w, int &lo, int &hi) { lo = 8 * w; hi = 64; };
+    // R = Aqk T, T = X Diag(beta): R[r][s] sums m in [s, r]
+    smm_rows<64>([&](int r, int m) { return Aq[r * L6 + m]; }, [&](int m, int s) { return X[m * L6 + s] * bs[s]; },
+                 k_upto, [&](int r, int s, float x) { Rm[r * L6 + s] = x; });
     __syncthreads();
     // dR' = dR - dP (K Gamma)^T
     smm_nt<64, 64, 128>(dPs, LD, Kt, LD, [&](int t, int s, float x) { dRp[t * L6 + s] = fgi[FG_DR + t * 64 + s] - x; });
     // dT'_0 = dT + dW (K Gamma)^T
     smm_nt<64, 64, 128>(dWs, LD, Kt, LD, [&](int t, int s, float x) { dTp[t * L6 + s] = fgi[FG_DT + t * 64 + s] + x; });
-    // dKt = T^T dW - R^T dP  -> workspace
-    smm<64, 128, 64>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return dWs[t * LD + c]; },
-                     [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] = x; });
+    // dKt = T^T dW - R^T dP -> workspace (both sum t >= s)
+    smm_rows2<128>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return dWs[t * LD + c]; },
+                   [&](int s, int t) { return -Rm[t * L6 + s]; }, [&](int t, int c) { return dPs[t * LD + c]; },
+                   [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = lo2 = 8 * w; hi1 = hi2 = 64; },
+                   [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] = x; });
     __syncthreads();
-    smm<64, 128, 64>([&](int s, int t) { return Rm[t * L6 + s]; }, [&](int t, int c) { return dPs[t * LD + c]; },
-                     [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] -= x; });
-    // dT' += Aqk^T dR'
-    smm<64, 64, 64>([&](int r, int m) { return Aq[m * L6 + r]; }, [&](int m, int s) { return dRp[m * L6 + s]; },
-                    [&](int r, int s, float x) { dTp[r * L6 + s] += x; });
-    // dAqk = tril(dR' T^T) -> workspace
-    smm<64, 64, 64>([&](int r, int m) { return dRp[r * L6 + m]; }, [&](int m, int s) { return X[s * L6 + m] * bs[m]; },
-                    [&](int r, int s, float x) { io[IW_DAQK + r * 64 + s] = s <= r ? x : 0.f; });
+    // dT' += Aqk^T dR' (sums m >= r)
+    smm_rows<64>([&](int r, int m) { return Aq[m * L6 + r]; }, [&](int m, int s) { return dRp[m * L6 + s]; },
+                 k_from, [&](int r, int s, float x) { dTp[r * L6 + s] += x; });
+    // dAqk = tril(dR' T^T) -> workspace, as its transpose: dAqk[r][s] = sum_{m <= s}
+    // T[s][m] dR'[r][m], rows s
+    smm_rows<64>([&](int s2, int m) { return X[s2 * L6 + m] * bs[m]; }, [&](int m, int r) { return dRp[r * L6 + m]; },
+                 k_upto, [&](int s2, int r, float x) { io[IW_DAQK + r * 64 + s2] = s2 <= r ? x : 0.f; });
     __syncthreads();
-    // Wk = X^T (dT' Diag(beta))
-    smm<64, 64, 64>([&](int r, int m) { return X[m * L6 + r]; }, [&](int m, int s) { return dTp[m * L6 + s] * bs[s]; },
-                    [&](int r, int s, float x) { Wk[r * L6 + s] = x; });
+    // Wk = X^T (dT' Diag(beta)) (sums m >= r)
+    smm_rows<64>([&](int r, int m) { return X[m * L6 + r]; }, [&](int m, int s) { return dTp[m * L6 + s] * bs[s]; },
+                 k_from, [&](int r, int s, float x) { Wk[r * L6 + s] = x; });
     __syncthreads();
-    // dAkk = strict_tril(-Wk X^T), dM = Diag(beta) dAkk -> workspace; dAkk * M row sums
-    smm_nt<64, 64, 64>(Wk, L6, X, L6,
-                    [&](int r, int s, float x) {
-                        const float dakk = s < r ? -x : 0.f;
-                        Rm[r * L6 + s] = dakk;                       // R is consumed: reuse for dAkk
-                        io[IW_DM + r * 64 + s] = bs[r] * dakk;
-                    });
+    // dAkk = strict_tril(-Wk X^T), dM = Diag(beta) dAkk -> workspace, as the
+    // transpose: dAkk[r][s] = -sum_{m <= s} X[s][m] Wk[r][m], rows s
+    smm_rows<64>([&](int s2, int m) { return X[s2 * L6 + m]; }, [&](int m, int r) { return Wk[r * L6 + m]; },
+                 k_upto,
+                 [&](int s2, int r, float x) {
+                     const float dakk = s2 < r ? -x : 0.f;
+                     Rm[r * L6 + s2] = dakk;                       // R is consumed: reuse for dAkk
+                     io[IW_DM + r * 64 + s2] = bs[r] * dakk;
+                 });
     __syncthreads();
     // dbeta_s = sum_r X[r,s] dT'[r,s] + sum_t dAkk[s,t] M[s,t]
     if (tid < 64) {

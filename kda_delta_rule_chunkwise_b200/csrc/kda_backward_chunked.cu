@@ -129,6 +129,54 @@ __device__ __forceinline__ void smm_rows2(FA1 A1, FB1 B1, FA2 A2, FB2 B2, FR ran
 #pragma unroll
         for (int b = 0; b < TN; ++b) out(TM * ty + a, tx + 16 * b, r[a][b]);
 }
+// The same banded sums with row-major fp32 right operands (ldb a multiple of 4):
+// thread (ty, tx) owns rows 4 ty .. 4 ty + 3 and the four consecutive columns
+// 4 tx + 64 b + e, read as one 16-byte load per k and b (as smm_pb).
+template <int N, typename FA1, typename FA2, typename FR, typename FO>
+__device__ __forceinline__ void smm_rows2_pb(FA1 A1, const float *B1, int ldb1, FA2 A2, const float *B2,
+                                             int ldb2, FR range, FO out) {
+    constexpr int TM = 4, NB = N / 64;
+    static_assert(N % 64 == 0, "tile");
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    int lo1, hi1, lo2, hi2;
+    range(threadIdx.x >> 5, lo1, hi1, lo2, hi2);
+    float r[TM][NB][4];
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) r[a][b][e] = 0.f;
+    auto run = [&](auto A, const float *B, int ldb, int lo, int hi) {
+#pragma unroll 4
+        for (int k = lo; k < hi; ++k) {
+            float av[TM];
+            float4 bv[NB];
+#pragma unroll
+            for (int a = 0; a < TM; ++a) av[a] = A(TM * ty + a, k);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) bv[b] = *reinterpret_cast<const float4 *>(B + k * ldb + 64 * b + 4 * tx);
+#pragma unroll
+            for (int a = 0; a < TM; ++a)
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    r[a][b][0] = fmaf(av[a], bv[b].x, r[a][b][0]);
+                    r[a][b][1] = fmaf(av[a], bv[b].y, r[a][b][1]);
+                    r[a][b][2] = fmaf(av[a], bv[b].z, r[a][b][2]);
+                    r[a][b][3] = fmaf(av[a], bv[b].w, r[a][b][3]);
+                }
+        }
+    };
+    run(A1, B1, ldb1, lo1, hi1);
+    run(A2, B2, ldb2, lo2, hi2);
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) out(TM * ty + a, 64 * b + 4 * tx + e, r[a][b][e]);
+}
+
 // one product: the second pair is empty
 template <int N, typename FA, typename FB, typename FR, typename FO>
 __device__ __forceinline__ void smm_rows(FA A, FB B, FR range, FO out) {
@@ -578,11 +626,11 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     }
     auto Tm = [&](int r, int s2) { return Tf[r * L6 + s2]; };   // T[r][s]
     auto Rm = [&](int r, int s2) { return Rf[r * L6 + s2]; };   // R[r][s]
-    // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out)
-    smm_pb<64, 128, 64>([&](int s, int t) { return Tm(t, s); }, dU, LD,
-                        [&](int s, int c, float x) { U[s * LD + c] = x; });
-    smm_pb<64, 128, 64>([&](int s, int t) { return Rm(t, s); }, dO, LD,
-                        [&](int s, int c, float x) { U[s * LD + c] += x; });
+    // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out); T and
+    // R are lower triangular, so row s sums t >= s only
+    smm_rows2_pb<128>([&](int s, int t) { return Tm(t, s); }, dU, LD, [&](int s, int t) { return Rm(t, s); }, dO,
+                      LD, [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = lo2 = 8 * w; hi1 = hi2 = 64; },
+                      [&](int s, int c, float x) { U[s * LD + c] = x; });
     __syncthreads();
     for (int i = tid; i < 64 * 32; i += NT) {
         const int s = i >> 5, c = (i & 31) * 4;
@@ -594,9 +642,10 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     smm_nt<64, 64, 128>(dU, LD, V, LD, [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; });
     smm_nt<64, 64, 128>(dO, LD, V, LD, [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; });
     __syncthreads();   // U's buffer (dV) is read out
-    // U = T V
-    smm_pb<64, 128, 64>([&](int t, int s) { return Tm(t, s); }, V, LD,
-                        [&](int t, int c, float x) { U[t * LD + c] = x; });
+    // U = T V (row t sums s <= t)
+    smm_rows2_pb<128>([&](int t, int s) { return Tm(t, s); }, V, LD, [&](int t, int s) { return Tm(t, s); }, V, LD,
+                      [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = 0; hi1 = 8 * w + 8; lo2 = hi2 = 0; },
+                      [&](int t, int c, float x) { U[t * LD + c] = x; });
     __syncthreads();   // V and [T; R] are consumed
 
     // ---- phase 2: S (zero without an initial state)

@@ -740,8 +740,9 @@ __device__ __forceinline__ void chunk_cumsum(const Tin *g, int64_t t0, int H, in
     }
 }
 
+constexpr int RC_LDK = 136;   // row stride (elements) of the staged k rows: 16-byte aligned rows
 template <typename Tin>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 2)
 bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T,
                      int N, int H, const Tin *__restrict__ q, const Tin *__restrict__ k,
                      const Tin *__restrict__ g, float *__restrict__ iw) {
@@ -759,27 +760,21 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
     const int64_t t0 = ra + (int64_t)j * C;
     const int L = (int)((rb - t0) < C ? (rb - t0) : C);
     float *G = reinterpret_cast<float *>(sm);              // [64][LD]
-    float *QE = G + 64 * LD;                               // q_r E1_r
-    float *KE = QE + 64 * LD;                              // k_r E1_r
-    float *KF = KE + 64 * LD;                              // [64][LD]: k_s exp(R_a - G_s), block a's
-    float *Rref = KF + 64 * LD;                            // [4][128]
-    float *Kr = Rref + 4 * 128;                            // [64][LD]: k (0 past the chunk's end)
+    float *KF = G + 64 * LD;                               // [64][LD]: k_s exp(R_a - G_s), block a's
+    float *QE = KF + 64 * LD;                              // [16][LD]: q_r E1_r, rows of block a
+    float *KE = QE + 16 * LD;                              // [16][LD]: k_r E1_r
+    float *Rref = KE + 16 * LD;                            // [4][128]
+    static_assert(sizeof(Tin) == 2, "the recompute kernel's shared memory is sized for 16-bit k");
+    Tin *Kb = reinterpret_cast<Tin *>(Rref + 4 * 128);     // [64][RC_LDK]: k as given (0 past the end)
     float *out = iw + ((size_t)cidx * H + h) * IW_FLOATS;
     chunk_cumsum(g, t0, H, h, L, G, Rref);
-    __syncthreads();
-    for (int i = tid; i < 64 * 32; i += NT) {   // 4 channels per load
-        const int r = i >> 5, c0 = (i & 31) * 4;
-        const size_t off = ((size_t)(t0 + r) * H + h) * D + c0;
-        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 k4 = r < L ? load4_f32(k + off) : z, q4 = r < L ? load4_f32(q + off) : z;
-        const float ka[4] = {k4.x, k4.y, k4.z, k4.w}, qa[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int c = c0 + e;
-            const float e1 = __expf(G[r * LD + c] - Rref[(r >> 4) * 128 + c]);
-            QE[r * LD + c] = qa[e] * e1;
-            KE[r * LD + c] = ka[e] * e1;
-            Kr[r * LD + c] = ka[e];
+    {
+        constexpr int PR = 128 * (int)sizeof(Tin) / 16;   // 16-byte pieces per row
+        for (int i = tid; i < 64 * PR; i += NT) {
+            const int r = i / PR, pc = i % PR;
+            const uint4 u = r < L ? *reinterpret_cast<const uint4 *>(k + ((size_t)(t0 + r) * H + h) * D + pc * (16 / sizeof(Tin)))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(Kb + r * RC_LDK + pc * (16 / sizeof(Tin))) = u;
         }
     }
     const int tx = tid & 15, ty = tid >> 4;   // output (row 16a + ty, columns tx + 16 b)
@@ -790,12 +785,25 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
         // k_s exp(R_a - G_s) for s < NS, row-major like k
         for (int i = tid; i < NS * 32; i += NT) {
             const int s2 = i >> 5, c = (i & 31) * 4;
-            const float4 kr = *reinterpret_cast<const float4 *>(Kr + s2 * LD + c);
+            const float4 kr = load4_f32(Kb + s2 * RC_LDK + c);
             const float4 g4 = *reinterpret_cast<const float4 *>(G + s2 * LD + c);
             const float4 rf = *reinterpret_cast<const float4 *>(Rref + A * 128 + c);
             *reinterpret_cast<float4 *>(KF + s2 * LD + c) =
                 make_float4(kr.x * __expf(rf.x - g4.x), kr.y * __expf(rf.y - g4.y),
                             kr.z * __expf(rf.z - g4.z), kr.w * __expf(rf.w - g4.w));
+        }
+        // q_r E1_r and k_r E1_r, E1_r = exp(G_r - R_a), for the 16 rows of block a
+        for (int i = tid; i < 16 * 32; i += NT) {
+            const int r = i >> 5, c = (i & 31) * 4, rr = 16 * A + r;
+            const float4 g4 = *reinterpret_cast<const float4 *>(G + rr * LD + c);
+            const float4 rf = *reinterpret_cast<const float4 *>(Rref + A * 128 + c);
+            const float4 e = make_float4(__expf(g4.x - rf.x), __expf(g4.y - rf.y), __expf(g4.z - rf.z),
+                                         __expf(g4.w - rf.w));
+            const float4 q4 = rr < L ? load4_f32(q + ((size_t)(t0 + rr) * H + h) * D + c)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 k4 = load4_f32(Kb + rr * RC_LDK + c);
+            *reinterpret_cast<float4 *>(QE + r * LD + c) = make_float4(q4.x * e.x, q4.y * e.y, q4.z * e.z, q4.w * e.w);
+            *reinterpret_cast<float4 *>(KE + r * LD + c) = make_float4(k4.x * e.x, k4.y * e.y, k4.z * e.z, k4.w * e.w);
         }
         __syncthreads();
         // rows 16a .. 16a + 15 of Aqk (s <= r) and of M (s < r) in one pass over the
@@ -803,7 +811,7 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
         float ra_[NB], rm_[NB];
 #pragma unroll
         for (int b2 = 0; b2 < NB; ++b2) ra_[b2] = rm_[b2] = 0.f;
-        const float *qe = QE + (16 * A + ty) * LD, *ke = KE + (16 * A + ty) * LD;
+        const float *qe = QE + ty * LD, *ke = KE + ty * LD;
 #pragma unroll 2
         for (int c = 0; c < 128; c += 4) {
             const float4 x = *reinterpret_cast<const float4 *>(qe + c);
@@ -1278,7 +1286,9 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
                                                      a.state_in, snaps, a.dout, dS, dU, fg, a.dv, hb, a.err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t RC_SMEM = 5 * 64 * LD * 4 + 4 * 128 * 4;   // G, QE, KE, KF, Rref, k
+    // G, KF, QE and KE of one row block, Rref, k (bf16): two CTAs per SM
+    constexpr uint32_t RC_SMEM = (2 * 64 + 2 * 16) * LD * 4 + 4 * 128 * 4 + 64 * RC_LDK * 2;
+    static_assert(2 * (RC_SMEM + 1024) <= 228 * 1024, "recompute: two CTAs per SM");
     if ((e = set_smem(bwd_recompute_kernel<bf>, RC_SMEM)) != cudaSuccess) return e;
     bwd_recompute_kernel<bf><<<items, NT, RC_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.q,
                                                          (const bf *)a.k, (const bf *)a.g, iw);

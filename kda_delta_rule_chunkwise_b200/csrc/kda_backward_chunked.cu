@@ -838,8 +838,13 @@ bwd_recompute_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict_
     block(std::integral_constant<int, 3>{});
 }
 
+// Shared memory of the pull-back: five 64 x 64 regions (reused as the phases
+// free them) and two 64 x 32 channel-quarter tiles, 104 KB: two CTAs per SM.
+constexpr int PB_LQ = 36;                                   // fp32 row stride of 32-wide tiles
+constexpr uint32_t PB_SMEM = 5 * 64 * L6 * 4 + 2 * 64 * PB_LQ * 4 + 8 * 32 * 4 + 64 * 4;
+
 template <typename Tin>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 2)
 bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T,
                     int N, int H, const Tin *__restrict__ k, const Tin *__restrict__ g,
                     const Tin *__restrict__ beta, const float *__restrict__ fg,
@@ -860,60 +865,27 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     const size_t item = (size_t)cidx * H + h;
     float *io = iw + item * IW_FLOATS;
     const float *fgi = fg + item * FG_FLOATS;
-    float *Aq = reinterpret_cast<float *>(sm);            // Aqk        [64][L6]
-    float *Mm = Aq + 64 * L6;                              // M
-    float *X = Mm + 64 * L6;                               // X = (I + Diag(beta) M)^-1
-    float *Rm = X + 64 * L6;                               // R = Aqk T
-    float *dTp = Rm + 64 * L6;                             // dT'
-    float *dRp = dTp + 64 * L6;                            // dR'
-    float *Wk = dRp + 64 * L6;                             // scratch [64][L6]
-    float *Kt = Wk + 64 * L6;                              // K * Gamma  [64][LD]
-    float *dPs = Kt + 64 * LD;                             // dP [64][LD]
-    float *dWs = dPs + 64 * LD;                            // dW [64][LD]
-    float *bs = dWs + 64 * LD;                             // beta [64]
-    // all loads in 16-byte pieces of rows (io, fgi: 16-byte aligned workspace
-    // records; q, k, g rows of 128 channels)
+    // regions [64][L6]: 0 Aqk, then dR'; 1 M, then dT'; 2 X; 3 R, then Aqk again;
+    // 4 the X scratch, then K*Gamma of a channel quarter, then Wk
+    float *Rg0 = reinterpret_cast<float *>(sm);
+    float *Rg1 = Rg0 + 64 * L6, *Rg2 = Rg1 + 64 * L6, *Rg3 = Rg2 + 64 * L6, *Rg4 = Rg3 + 64 * L6;
+    float *dPq = Rg4 + 64 * L6;                            // dP, dW of a channel quarter [64][PB_LQ]
+    float *dWq = dPq + 64 * PB_LQ;
+    float *gsum = dWq + 64 * PB_LQ;                        // [8][32] row-group sums of the quarter's g
+    float *bs = gsum + 8 * 32;                             // beta [64]
+    float *Aq = Rg0, *Mm = Rg1, *X = Rg2, *Rm = Rg3, *Wk = Rg4;
+    // ---- phase 1: X = (I + Diag(beta) M)^-1, R = Aqk T
     for (int i = tid; i < 64 * 16; i += NT) {
         const int r = i >> 4, s = (i & 15) * 4;
         *reinterpret_cast<float4 *>(Aq + r * L6 + s) = *reinterpret_cast<const float4 *>(io + IW_AQK + r * 64 + s);
         *reinterpret_cast<float4 *>(Mm + r * L6 + s) = *reinterpret_cast<const float4 *>(io + IW_M + r * 64 + s);
+        *reinterpret_cast<float4 *>(X + r * L6 + s) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (tid < 64) bs[tid] = tid < L ? to_f32(beta[(size_t)(t0 + tid) * H + h]) : 0.f;
-    for (int i = tid; i < 64 * 32; i += NT) {
-        const int t = i >> 5, c = (i & 31) * 4;
-        *reinterpret_cast<float4 *>(dPs + t * LD + c) = *reinterpret_cast<const float4 *>(fgi + FG_DP + t * 128 + c);
-        *reinterpret_cast<float4 *>(dWs + t * LD + c) = *reinterpret_cast<const float4 *>(fgi + FG_DW + t * 128 + c);
-    }
-    // K * Gamma, Gamma = exp(cumsum(max(g, -5))): the rows of g load in parallel,
-    // one thread per channel scans them in place, then the rows of k scale them
-    // (k waits in dTp..Wk, which are free until the products below)
-    float *Kr = dTp;   // [64][LD] over dTp, dRp and Wk (3 * 64 * L6 >= 64 * LD floats)
-    for (int i = tid; i < 64 * 32; i += NT) {
-        const int r = i >> 5, c = (i & 31) * 4;
-        const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
-        if (r < L) {
-            x = load4_f32(g + off);
-            x = make_float4(fmaxf(x.x, -5.f), fmaxf(x.y, -5.f), fmaxf(x.z, -5.f), fmaxf(x.w, -5.f));
-            y = load4_f32(k + off);
-        }
-        *reinterpret_cast<float4 *>(Kt + r * LD + c) = x;
-        *reinterpret_cast<float4 *>(Kr + r * LD + c) = y;
-    }
-    __syncthreads();
-    if (tid < 128) {
-        float acc = 0.f;
-        for (int r = 0; r < 64; ++r) {
-            acc += Kt[r * LD + tid];
-            Kt[r * LD + tid] = Kr[r * LD + tid] * __expf(acc);
-        }
-    }
     __syncthreads();
     // X = (I + A)^-1, A = Diag(beta) M (strictly lower), by 16 x 16 blocks: the
     // diagonal blocks by forward substitution (thread = block a, column j), then
     // block row i from the rows above: X[i, 0:i] = -X_ii (A[i, 0:i] X[0:i, 0:i])
-    for (int i = tid; i < 64 * 64; i += NT) X[(i >> 6) * L6 + (i & 63)] = 0.f;
-    __syncthreads();
     if (tid < 64) {
         const int a = tid >> 4, jc = tid & 15, o = 16 * a;
         float x[16];
@@ -950,16 +922,77 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
     // R = Aqk T, T = X Diag(beta): R[r][s] sums m in [s, r]
     smm_rows<64>([&](int r, int m) { return Aq[r * L6 + m]; }, [&](int m, int s) { return X[m * L6 + s] * bs[s]; },
                  k_upto, [&](int r, int s, float x) { Rm[r * L6 + s] = x; });
-    __syncthreads();
-    // dR' = dR - dP (K Gamma)^T
-    smm_nt<64, 64, 128>(dPs, LD, Kt, LD, [&](int t, int s, float x) { dRp[t * L6 + s] = fgi[FG_DR + t * 64 + s] - x; });
-    // dT'_0 = dT + dW (K Gamma)^T
-    smm_nt<64, 64, 128>(dWs, LD, Kt, LD, [&](int t, int s, float x) { dTp[t * L6 + s] = fgi[FG_DT + t * 64 + s] + x; });
-    // dKt = T^T dW - R^T dP -> workspace (both sum t >= s)
-    smm_rows2<128>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return dWs[t * LD + c]; },
-                   [&](int s, int t) { return -Rm[t * L6 + s]; }, [&](int t, int c) { return dPs[t * LD + c]; },
-                   [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = lo2 = 8 * w; hi1 = hi2 = 64; },
-                   [&](int s, int c, float x) { io[IW_DKT + s * 128 + c] = x; });
+    __syncthreads();   // Aqk and M are consumed (Aqk comes back in phase 3, M from the workspace)
+
+    // ---- phase 2, by quarters of 32 channels: K*Gamma, dR' = dR - dP (K Gamma)^T,
+    // dT'_0 = dT + dW (K Gamma)^T (both summed over the quarters in order), and
+    // dKt = T^T dW - R^T dP -> workspace (sums t >= s)
+    float *dRp = Rg0, *dTp = Rg1, *Ktq = Rg4;   // Ktq: [64][PB_LQ]
+    for (int i = tid; i < 64 * 16; i += NT) {
+        const int r = i >> 4, s = (i & 15) * 4;
+        *reinterpret_cast<float4 *>(dRp + r * L6 + s) = *reinterpret_cast<const float4 *>(fgi + FG_DR + r * 64 + s);
+        *reinterpret_cast<float4 *>(dTp + r * L6 + s) = *reinterpret_cast<const float4 *>(fgi + FG_DT + r * 64 + s);
+    }
+    for (int qd = 0; qd < 4; ++qd) {
+        const int cb = 32 * qd;
+        __syncthreads();   // the previous quarter's products are done with its tiles
+        // the quarter's dP, dW, g (clamped; 0 past the chunk's end) and k
+        float4 kq[2];
+        for (int i = tid, it = 0; i < 64 * 8; i += NT, ++it) {
+            const int r = i >> 3, c = (i & 7) * 4;
+            *reinterpret_cast<float4 *>(dPq + r * PB_LQ + c) = *reinterpret_cast<const float4 *>(fgi + FG_DP + r * 128 + cb + c);
+            *reinterpret_cast<float4 *>(dWq + r * PB_LQ + c) = *reinterpret_cast<const float4 *>(fgi + FG_DW + r * 128 + cb + c);
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+            if (r < L) {
+                const size_t off = ((size_t)(t0 + r) * H + h) * D + cb + c;
+                x = load4_f32(g + off);
+                x = make_float4(fmaxf(x.x, -5.f), fmaxf(x.y, -5.f), fmaxf(x.z, -5.f), fmaxf(x.w, -5.f));
+                y = load4_f32(k + off);
+            }
+            *reinterpret_cast<float4 *>(Ktq + r * PB_LQ + c) = x;
+            kq[it] = y;
+        }
+        __syncthreads();
+        // Gamma = exp(cumsum over rows): thread (group gr of 8 rows, channel cc) sums
+        // its rows, the group offsets come from the groups above
+        {
+            const int cc = tid & 31, gr = tid >> 5;
+            float run = 0.f, loc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                run += Ktq[(8 * gr + e) * PB_LQ + cc];
+                loc[e] = run;
+            }
+            gsum[gr * 32 + cc] = run;
+            __syncthreads();
+            float off = 0.f;
+            for (int g2 = 0; g2 < gr; ++g2) off += gsum[g2 * 32 + cc];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) Ktq[(8 * gr + e) * PB_LQ + cc] = __expf(off + loc[e]);
+        }
+        __syncthreads();
+        for (int i = tid, it = 0; i < 64 * 8; i += NT, ++it) {   // K * Gamma (the same rows as the load)
+            const int r = i >> 3, c = (i & 7) * 4;
+            float4 *p4 = reinterpret_cast<float4 *>(Ktq + r * PB_LQ + c);
+            const float4 e = *p4;
+            *p4 = make_float4(kq[it].x * e.x, kq[it].y * e.y, kq[it].z * e.z, kq[it].w * e.w);
+        }
+        __syncthreads();
+        smm_nt<64, 64, 32>(dPq, PB_LQ, Ktq, PB_LQ, [&](int t, int s, float x) { dRp[t * L6 + s] -= x; });
+        smm_nt<64, 64, 32>(dWq, PB_LQ, Ktq, PB_LQ, [&](int t, int s, float x) { dTp[t * L6 + s] += x; });
+        smm_rows2<32>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return dWq[t * PB_LQ + c]; },
+                      [&](int s, int t) { return -Rm[t * L6 + s]; }, [&](int t, int c) { return dPq[t * PB_LQ + c]; },
+                      [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = lo2 = 8 * w; hi1 = hi2 = 64; },
+                      [&](int s, int c, float x) { io[IW_DKT + s * 128 + cb + c] = x; });
+    }
+    __syncthreads();   // R is consumed: its region takes Aqk again
+
+    // ---- phase 3
+    Aq = Rg3;
+    for (int i = tid; i < 64 * 16; i += NT) {
+        const int r = i >> 4, s = (i & 15) * 4;
+        *reinterpret_cast<float4 *>(Aq + r * L6 + s) = *reinterpret_cast<const float4 *>(io + IW_AQK + r * 64 + s);
+    }
     __syncthreads();
     // dT' += Aqk^T dR' (sums m >= r)
     smm_rows<64>([&](int r, int m) { return Aq[m * L6 + r]; }, [&](int m, int s) { return dRp[m * L6 + s]; },
@@ -974,13 +1007,14 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                  k_from, [&](int r, int s, float x) { Wk[r * L6 + s] = x; });
     __syncthreads();
     // dAkk = strict_tril(-Wk X^T), dM = Diag(beta) dAkk -> workspace, as the
-    // transpose: dAkk[r][s] = -sum_{m <= s} X[s][m] Wk[r][m], rows s
+    // transpose: dAkk[r][s] = -sum_{m <= s} X[s][m] Wk[r][m], rows s (into dR''s region)
+    float *dAkk = Rg0;
     smm_rows<64>([&](int s2, int m) { return X[s2 * L6 + m]; }, [&](int m, int r) { return Wk[r * L6 + m]; },
                  k_upto,
                  [&](int s2, int r, float x) {
-                     const float dakk = s2 < r ? -x : 0.f;
-                     Rm[r * L6 + s2] = dakk;                       // R is consumed: reuse for dAkk
-                     io[IW_DM + r * 64 + s2] = bs[r] * dakk;
+                     const float d = s2 < r ? -x : 0.f;
+                     dAkk[r * L6 + s2] = d;
+                     io[IW_DM + r * 64 + s2] = bs[r] * d;
                  });
     __syncthreads();
     // dbeta_s = sum_r X[r,s] dT'[r,s] + sum_t dAkk[s,t] M[s,t]
@@ -988,7 +1022,7 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
         float a = 0.f, b = 0.f;
         for (int r = 0; r < 64; ++r) {
             a = fmaf(X[r * L6 + tid], dTp[r * L6 + tid], a);
-            b = fmaf(Rm[tid * L6 + r], Mm[tid * L6 + r], b);
+            b = fmaf(dAkk[tid * L6 + r], io[IW_M + tid * 64 + r], b);
         }
         io[IW_DB + tid] = a + b;
     }
@@ -1294,8 +1328,7 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
                                                          (const bf *)a.k, (const bf *)a.g, iw);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);
-    constexpr uint32_t PB_SMEM = 7 * 64 * L6 * 4 + 3 * 64 * LD * 4 + 64 * 4;
-    static_assert(PB_SMEM <= 227 * 1024, "pull-back shared memory");
+    static_assert(2 * (PB_SMEM + 1024) <= 228 * 1024, "pull-back: two CTAs per SM");
     if ((e = set_smem(bwd_pullback_kernel<bf>, PB_SMEM)) != cudaSuccess) return e;
     bwd_pullback_kernel<bf><<<items, NT, PB_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.k,
                                                         (const bf *)a.g, (const bf *)a.beta, fg, iw);

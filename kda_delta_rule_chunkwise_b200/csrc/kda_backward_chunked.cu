@@ -1118,15 +1118,23 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
         const float4 dKh4 = *reinterpret_cast<const float4 *>(fgi + FG_DKH + r * 128 + c0);
         const float qa[4] = {q4.x, q4.y, q4.z, q4.w}, dPa[4] = {dP4.x, dP4.y, dP4.z, dP4.w};
         const float dKta[4] = {dKt4.x, dKt4.y, dKt4.z, dKt4.w}, dKha[4] = {dKh4.x, dKh4.y, dKh4.z, dKh4.w};
+        // shared-memory rows by 16-byte pieces (a quarter-warp covers one row)
+        const float4 G4 = *reinterpret_cast<const float4 *>(G + r * LS + cc0);
+        const float4 gl4 = *reinterpret_cast<const float4 *>(gl + cc0);
+        const float4 k4 = *reinterpret_cast<const float4 *>(Ks + r * LS + cc0);
+        const float Ga[4] = {G4.x, G4.y, G4.z, G4.w}, gla[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
+        const float ka[4] = {k4.x, k4.y, k4.z, k4.w};
+        float dq4[4], dk4[4], dg4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const int cc = cc0 + e;
-            const float Gr = G[r * LS + cc], gam = __expf(Gr), kh_f = __expf(gl[cc] - Gr);
-            const float kk = kv(r, cc);
-            Dq[r * LS + cc] = dPa[e] * gam;
-            Dk[r * LS + cc] = dKta[e] * gam + dKha[e] * kh_f;
-            dG[r * LS + cc] = qa[e] * gam * dPa[e] + kk * gam * dKta[e] - kk * kh_f * dKha[e];
+            const float gam = __expf(Ga[e]), kh_f = __expf(gla[e] - Ga[e]);
+            dq4[e] = dPa[e] * gam;
+            dk4[e] = dKta[e] * gam + dKha[e] * kh_f;
+            dg4[e] = qa[e] * gam * dPa[e] + ka[e] * gam * dKta[e] - ka[e] * kh_f * dKha[e];
         }
+        *reinterpret_cast<float4 *>(Dq + r * LS + cc0) = make_float4(dq4[0], dq4[1], dq4[2], dq4[3]);
+        *reinterpret_cast<float4 *>(Dk + r * LS + cc0) = make_float4(dk4[0], dk4[1], dk4[2], dk4[3]);
+        *reinterpret_cast<float4 *>(dG + r * LS + cc0) = make_float4(dg4[0], dg4[1], dg4[2], dg4[3]);
     }
     // decayed adjoints: first Aqk with (a, b) = (q, k), then M with (k, k).  dF is
     // lower triangular, so block a's sums run over s <= 16a + 15 only.
@@ -1172,11 +1180,14 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                     acc[x][y] += __shfl_xor_sync(0xffffffffu, acc[x][y], 16);
                 }
             // every lane of a quarter group holds the sums; lane kq finishes row
-            // 2w + (kq >> 1), columns 4 cq + 2 (kq & 1) + e
+            // 2w + (kq >> 1), columns 4 cq + 2 (kq & 1) + e (the second row takes its
+            // two columns in the other order, so that the rows fall on different banks)
             const int rsel = kq >> 1, csel = kq & 1, rr = 16 * A + 2 * warp + rsel;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float x = rsel ? (csel ? acc[1][2 + e] : acc[1][e]) : (csel ? acc[0][2 + e] : acc[0][e]);
+            for (int e0 = 0; e0 < 2; ++e0) {
+                const int e = rsel ? 1 - e0 : e0;
+                const float x = rsel ? (csel ? (e ? acc[1][3] : acc[1][2]) : (e ? acc[1][1] : acc[1][0]))
+                                     : (csel ? (e ? acc[0][3] : acc[0][2]) : (e ? acc[0][1] : acc[0][0]));
                 const int cc = 4 * cq + 2 * csel + e;
                 const float da = x * __expf(G[rr * LS + cc] - Rref[A * CW + cc]);
                 const float av = form == 0 ? qv(rr, cc) : kv(rr, cc);

@@ -314,19 +314,23 @@ __device__ __forceinline__ const float *chunk_state(const int32_t *hdr, bool pac
 // ======================================================================
 constexpr int CH_DVS = 32;
 constexpr int CH_LD = CH_DVS + 4;
-constexpr int LDF = 132;                                          // fp32 row stride of 128-wide tiles
-constexpr uint32_t CH_SLOT = 0;                                   // slot image (66 560 B)
-constexpr uint32_t CH_KH = kSlotBytes;                            // Khat [64][LDF] fp32
-constexpr uint32_t CH_WN = CH_KH + 64 * LDF * 4;                  // -W   [64][LDF]
-constexpr uint32_t CH_P = CH_WN + 64 * LDF * 4;                   // P    [64][LDF]
-constexpr uint32_t CH_DS = CH_P + 64 * LDF * 4;                   // dS' [128][CH_LD] fp32
+constexpr uint32_t CH_SLOT = 0;                                   // 2 slot images (66 560 B each)
+constexpr uint32_t CH_DS = 2 * kSlotBytes;                        // dS' [128][CH_LD] fp32
 constexpr uint32_t CH_Y = CH_DS + 128 * CH_LD * 4;                // dU  [64][CH_LD]
 constexpr uint32_t CH_DO = CH_Y + 64 * CH_LD * 4;                 // dO  2 x [64][CH_LD]
-constexpr uint32_t CH_GAM = CH_DO + 2 * 64 * CH_LD * 4;           // Gamma_L [128]
-constexpr uint32_t CH_BAR = CH_GAM + 128 * 4;                     // slot-copy mbarrier
+constexpr uint32_t CH_BAR = CH_DO + 2 * 64 * CH_LD * 4;           // one slot-copy mbarrier per image
 constexpr uint32_t CH_SMEM = CH_BAR + 16;
 static_assert(CH_SMEM <= 227 * 1024, "chain kernel shared memory");
+static_assert(kSlotBytes % 16 == 0, "slot images start on 16-byte boundaries");
 static_assert(CH_DVS == 32 && NT == 256, "chain kernel thread map: 32 x 8 threads, four columns each");
+
+// four consecutive fp16 channels of a slot image (8 bytes at byte offset off)
+__device__ __forceinline__ float4 h4(const uint8_t *img, uint32_t off) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(img + off);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
 
 __global__ void __launch_bounds__(NT, 1)
 bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T, int N,
@@ -346,26 +350,26 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
     seq_rows(hdr, packed, T, N, n, ra, rb);
     const int nch = (int)((rb - ra + C - 1) / C);
     const int c0 = first_chunk(hdr, packed, T, n);
-    uint8_t *slot = sm + CH_SLOT;
-    float *Kh = reinterpret_cast<float *>(sm + CH_KH);
-    float *Wn = reinterpret_cast<float *>(sm + CH_WN);
-    float *Pm = reinterpret_cast<float *>(sm + CH_P);
     float *dS = reinterpret_cast<float *>(sm + CH_DS);
     float *Y = reinterpret_cast<float *>(sm + CH_Y);
-    float *gam = reinterpret_cast<float *>(sm + CH_GAM);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + CH_BAR);
     const size_t sbase = ((size_t)n * H + h) * D * D;
-    // The next chunk's slot image goes in by one bulk copy (completing on `bar`) as
-    // soon as this chunk's has been decoded, and its dO rows by cp.async into the
-    // other dO buffer, so that neither load waits on device memory in the chain.
-    auto issue_slot = [&](int jn) {
+    // The products read Khat, -W, P and Gamma_L straight from the fp16 slot image
+    // (8 bytes = 4 channels of one row per load; the 128-byte swizzle keeps a
+    // piece's 8 channels together). Two images: the next chunk's comes in by one
+    // bulk copy (completing on its own barrier) and its dO rows by cp.async into
+    // the other dO buffer while this chunk runs.
+    auto img_of = [&](int step) { return sm + CH_SLOT + (uint32_t)(step & 1) * kSlotBytes; };
+    auto issue_slot = [&](int jn, int step) {
         if (tid == 0) {
-            fence_async_smem();   // the decode's reads of the previous image come first
-            mbar_arrive_expect_tx(bar, kSlotBytes);
-            bulk_g2s(slot, fws + hdr_bytes + ((size_t)(c0 + jn) * H + h) * kSlotBytes, kSlotBytes, bar);
+            fence_async_smem();   // the previous readers of this image come first
+            mbar_arrive_expect_tx(&bar[step & 1], kSlotBytes);
+            bulk_g2s(img_of(step), fws + hdr_bytes + ((size_t)(c0 + jn) * H + h) * kSlotBytes, kSlotBytes,
+                     &bar[step & 1]);
         }
     };
-    auto issue_dO = [&](int jn, float *buf) {
+    auto issue_dO = [&](int jn, int step) {
+        float *buf = reinterpret_cast<float *>(sm + CH_DO) + (step & 1) * 64 * CH_LD;
         const int64_t tn = ra + (int64_t)jn * C;
         const int Ln = (int)((rb - tn) < C ? (rb - tn) : C);
         for (int i = tid; i < 64 * (CH_DVS / 4); i += NT) {   // 16-byte pieces
@@ -376,59 +380,54 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
         cp_async_commit();
     };
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         mbar_fence_init();
     }
     // dS' of the last chunk = dL/dS_final
-    for (int i = tid; i < 128 * CH_DVS; i += NT) {
-        const int c = i / CH_DVS, jj = i % CH_DVS;
-        dS[c * CH_LD + jj] = dstate_out ? dstate_out[sbase + (size_t)c * D + j0 + jj] : 0.f;
+    for (int i = tid; i < 128 * (CH_DVS / 4); i += NT) {
+        const int c = i / (CH_DVS / 4), jj = (i % (CH_DVS / 4)) * 4;
+        *reinterpret_cast<float4 *>(dS + c * CH_LD + jj) =
+            dstate_out ? *reinterpret_cast<const float4 *>(dstate_out + sbase + (size_t)c * D + j0 + jj)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
     if (nch > 0) {
-        issue_slot(nch - 1);
-        issue_dO(nch - 1, reinterpret_cast<float *>(sm + CH_DO));
+        issue_slot(nch - 1, 0);
+        issue_dO(nch - 1, 0);
     }
     bool ok = true;
-    int stuck = -1;   // the step whose slot copy was given up on (bounded wait)
-    for (int j = nch - 1; j >= 0; --j) {
+    int iss0 = nch > 0 ? 1 : 0, iss1 = 0, wt0 = 0, wt1 = 0;   // slot copies issued / waited for, per image
+    // thread (q, cq), q = 4 warp + lane / 8, cq = lane % 8, owns columns
+    // 4 cq .. 4 cq + 3 of the slice
+    const int cq = tid & 7, q = tid >> 3;
+    for (int step = 0; step < nch; ++step) {
+        const int j = nch - 1 - step;
         const size_t item = (size_t)(c0 + j) * H + h;
-        const int step = nch - 1 - j;
-        float *dO = reinterpret_cast<float *>(sm + CH_DO) + (step & 1) * 64 * CH_LD;
+        const uint8_t *img = img_of(step);
+        const float *dO = reinterpret_cast<const float *>(sm + CH_DO) + (step & 1) * 64 * CH_LD;
+        // the next chunk's image and dO, into the buffers the previous step released
+        if (j > 0 && ok) {
+            issue_slot(j - 1, step + 1);
+            issue_dO(j - 1, step + 1);
+            if ((step + 1) & 1) ++iss1; else ++iss0;
+        }
         // dS' of this chunk, for the factor kernel
         for (int i = tid; i < 128 * (CH_DVS / 4); i += NT) {
             const int c = i / (CH_DVS / 4), jj = (i % (CH_DVS / 4)) * 4;
             *reinterpret_cast<float4 *>(ws_dS + (item * D + c) * D + j0 + jj) =
                 *reinterpret_cast<const float4 *>(dS + c * CH_LD + jj);
         }
+        bool got = false;   // this chunk's image has landed
         if (ok) {
-            ok = mbar_wait(bar, step & 1, err);   // the slot image has landed
-            if (!ok) stuck = step;
+            got = mbar_wait(&bar[step & 1], (step >> 1) & 1, err);
+            if (got) {
+                if (step & 1) ++wt1; else ++wt0;
+            }
         }
-        cp_async_wait_all();                            // this thread's dO pieces have
-        __syncthreads();
-        // Khat, -W and P by 16-byte pieces (8 channels of one row; the swizzle
-        // permutes whole pieces within a row, see kh_off and wp_off)
-        for (int i = tid; i < 3 * 64 * 16; i += NT) {
-            const int part = i >> 10, t = (i >> 4) & 63, kb = (i >> 3) & 1, pc = i & 7, lc = pc ^ (t & 7);
-            const uint32_t off = part == 0 ? kSlotKh + kb * 8192 : kSlotWP + kb * 16384 + (part == 2 ? 8192 : 0);
-            const uint4 u = *reinterpret_cast<const uint4 *>(slot + off + (t >> 3) * 1024 + (t & 7) * 128 + pc * 16);
-            float *dst = (part == 0 ? Kh : part == 1 ? Wn : Pm) + t * LDF + 64 * kb + 8 * lc;
-            const __half2 *hp = reinterpret_cast<const __half2 *>(&u);
-            const float2 f0 = __half22float2(hp[0]), f1 = __half22float2(hp[1]);
-            const float2 f2 = __half22float2(hp[2]), f3 = __half22float2(hp[3]);
-            *reinterpret_cast<float4 *>(dst) = make_float4(f0.x, f0.y, f1.x, f1.y);
-            *reinterpret_cast<float4 *>(dst + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
-        }
-        if (tid < 128) gam[tid] = reinterpret_cast<const float *>(slot + kSlotGam)[tid];
-        __syncthreads();   // the image is decoded: the next one may land over it
-        if (j > 0 && ok) {
-            issue_slot(j - 1);
-            issue_dO(j - 1, reinterpret_cast<float *>(sm + CH_DO) + ((step + 1) & 1) * 64 * CH_LD);
-        }
-        // thread (q, cq), q = 4 warp + lane / 8, cq = lane % 8, owns columns
-        // 4 cq .. 4 cq + 3 of the slice; operands are read as 16-byte pieces
-        const int cq = tid & 7, q = tid >> 3;
+        if (j > 0 && ok) cp_async_wait_group1(); else cp_async_wait_all();   // this thread's dO pieces
+        ok = __syncthreads_and(got) != 0;
+        if (!ok) break;
         // dU = Khat dS': rows 2q, 2q + 1, four channels at a time
         {
             float r[2][4];
@@ -436,11 +435,9 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
             for (int x = 0; x < 2; ++x)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) r[x][e] = 0.f;
-            const float *k0 = Kh + 2 * q * LDF;
 #pragma unroll 2
             for (int c = 0; c < 128; c += 4) {
-                const float4 a0 = *reinterpret_cast<const float4 *>(k0 + c);
-                const float4 a1 = *reinterpret_cast<const float4 *>(k0 + LDF + c);
+                const float4 a0 = h4(img, kh_off(2 * q, c)), a1 = h4(img, kh_off(2 * q + 1, c));
                 const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
@@ -463,16 +460,17 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
         // 4q .. 4q + 3; each thread overwrites only the elements it alone reads
         {
             float r[4][4];
+            const float4 gm4 = *reinterpret_cast<const float4 *>(img + kSlotGam + 16 * q);
+            const float gmv[4] = {gm4.x, gm4.y, gm4.z, gm4.w};
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 const float4 d = *reinterpret_cast<const float4 *>(dS + (4 * q + x) * CH_LD + 4 * cq);
-                const float gm = gam[4 * q + x];
-                r[x][0] = gm * d.x; r[x][1] = gm * d.y; r[x][2] = gm * d.z; r[x][3] = gm * d.w;
+                r[x][0] = gmv[x] * d.x; r[x][1] = gmv[x] * d.y; r[x][2] = gmv[x] * d.z; r[x][3] = gmv[x] * d.w;
             }
 #pragma unroll 4
             for (int t = 0; t < 64; ++t) {
-                const float4 pw = *reinterpret_cast<const float4 *>(Pm + t * LDF + 4 * q);
-                const float4 wn = *reinterpret_cast<const float4 *>(Wn + t * LDF + 4 * q);
+                const float4 pw = h4(img, wp_off(64 + t, 4 * q));
+                const float4 wn = h4(img, wp_off(t, 4 * q));
                 const float4 o = *reinterpret_cast<const float4 *>(dO + t * CH_LD + 4 * cq);
                 const float4 y = *reinterpret_cast<const float4 *>(Y + t * CH_LD + 4 * cq);
                 const float pv[4] = {pw.x, pw.y, pw.z, pw.w}, wv[4] = {wn.x, wn.y, wn.z, wn.w};
@@ -487,16 +485,20 @@ bwd_chain_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu
                 *reinterpret_cast<float4 *>(dS + (4 * q + x) * CH_LD + 4 * cq) =
                     make_float4(r[x][0], r[x][1], r[x][2], r[x][3]);
         }
-        __syncthreads();   // dS, Y and this dO buffer are consumed
+        __syncthreads();   // dS, Y, this image and this dO buffer are consumed
     }
-    // a copy given up on (after a timeout) lands before exit
-    if (tid == 0 && stuck >= 0) mbar_wait(bar, stuck & 1, err, 1ull << 28);
+    // copies given up on (after a timeout) land before exit
+    if (tid == 0) {
+        for (; wt0 < iss0; ++wt0) mbar_wait(&bar[0], wt0 & 1, err, 1ull << 28);
+        for (; wt1 < iss1; ++wt1) mbar_wait(&bar[1], wt1 & 1, err, 1ull << 28);
+    }
     cp_async_wait_all();
     __syncthreads();
-    if (dstate_in)
-        for (int i = tid; i < 128 * CH_DVS; i += NT) {
-            const int c = i / CH_DVS, jj = i % CH_DVS;
-            dstate_in[sbase + (size_t)c * D + j0 + jj] = dS[c * CH_LD + jj];
+    if (dstate_in && ok)
+        for (int i = tid; i < 128 * (CH_DVS / 4); i += NT) {
+            const int c = i / (CH_DVS / 4), jj = (i % (CH_DVS / 4)) * 4;
+            *reinterpret_cast<float4 *>(dstate_in + sbase + (size_t)c * D + j0 + jj) =
+                *reinterpret_cast<const float4 *>(dS + c * CH_LD + jj);
         }
 }
 

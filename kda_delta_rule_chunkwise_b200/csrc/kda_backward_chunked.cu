@@ -149,12 +149,12 @@ __device__ __forceinline__ void smm_rows2(FA1 A1, FB1 B1, FA2 A2, FB2 B2, FR ran
 // 4 tx + 64 b + e, read as one 16-byte load per k and b (as smm_pb).
 template <int N, typename FA1, typename FA2, typename FR, typename FO>
 __device__ __forceinline__ void smm_rows2_pb(FA1 A1, const float *B1, int ldb1, FA2 A2, const float *B2,
-                                             int ldb2, FR range, FO out) {
+                                             int ldb2, FR range, FO out, const int lt = (int)threadIdx.x) {
     constexpr int TM = 4, NB = N / 64;
     static_assert(N % 64 == 0, "tile");
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int tx = lt & 15, ty = lt >> 4;
     int lo1, hi1, lo2, hi2;
-    range(threadIdx.x >> 5, lo1, hi1, lo2, hi2);
+    range(lt >> 5, lo1, hi1, lo2, hi2);
     float r[TM][NB][4];
 #pragma unroll
     for (int a = 0; a < TM; ++a)
@@ -208,10 +208,11 @@ __device__ __forceinline__ void smm_rows(FA A, FB B, FR range, FO out) {
 // 16-byte loads (lda, ldb multiples of 4, K a multiple of 4).  Same thread
 // mapping and summation order as smm.
 template <int M, int N, int K, typename FO>
-__device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, int ldb, FO out) {
+__device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, int ldb, FO out,
+                                       const int lt = (int)threadIdx.x) {
     constexpr int TM = M / 16, TN = N / 16;
     static_assert(M % 16 == 0 && N % 16 == 0 && K % 4 == 0, "tile");
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int tx = lt & 15, ty = lt >> 4;
     float r[TM][TN];
 #pragma unroll
     for (int a = 0; a < TM; ++a)
@@ -246,10 +247,10 @@ __device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, 
 // four consecutive columns 4 tx + 64 b + e, read as one 16-byte load per k and b.
 // The sums run over k in order, as in smm.
 template <int M, int N, int K, typename FA, typename FO>
-__device__ __forceinline__ void smm_pb(FA A, const float *B, int ldb, FO out) {
+__device__ __forceinline__ void smm_pb(FA A, const float *B, int ldb, FO out, const int lt = (int)threadIdx.x) {
     constexpr int TM = M / 16, NB = N / 64;
     static_assert(M % 16 == 0 && N % 64 == 0, "tile");
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int tx = lt & 15, ty = lt >> 4;
     float r[TM][NB][4];
 #pragma unroll
     for (int a = 0; a < TM; ++a)
@@ -542,8 +543,14 @@ __device__ __forceinline__ void locate_chunk(const int32_t *hdr, bool packed, in
     j = cidx - hdr[lo];
 }
 
+// 512 threads: two groups of 256 run independent products side by side (the
+// products' 16 x 16 thread grids are per group), so that each SM has 16 warps
+// to hide shared-memory and load latency with the same per-thread tiles.
+constexpr int FNT = 2 * NT;
+__device__ __forceinline__ void group_bar(int id) { asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory"); }
+
 template <typename Tin>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(FNT, 1)
 bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ cu, int64_t T, int N,
                   int H, const Tin *__restrict__ v, const float *state_in,
                   const float *__restrict__ snaps, const float *__restrict__ dout,
@@ -597,10 +604,11 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     // ---- phase 1: dU, dO (rows past the chunk's end are zero) by bulk copies;
     // V, [T; R] and -W by 16-byte loads (rows of 128 channels; every base is
     // 16-byte aligned)
+    const int grp = tid >> 8, lt = tid & 255;   // product group, thread within it
     if (tid == 0) mbar_arrive_expect_tx(&bars[0], (uint32_t)(64 + L) * 512u);
     copy_rows(dU, ws_dU + item * 64 * D, D, 64, 0, &bars[0]);
     copy_rows(dO, dout + ((size_t)t0 * H + h) * D, (size_t)H * D, L, 64, &bars[0]);
-    for (int i = tid; i < 64 * 32; i += NT) {
+    for (int i = tid; i < 64 * 32; i += FNT) {
         const int t = i >> 5, c = (i & 31) * 4;
         const size_t off = ((size_t)(t0 + t) * H + h) * D + c;
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -618,12 +626,12 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
             dst[2 * e + 1] = f.y;
         }
     };
-    for (int i = tid; i < 128 * 8; i += NT) {   // [T; R]: 128 rows x 8 pieces
+    for (int i = tid; i < 128 * 8; i += FNT) {   // [T; R]: 128 rows x 8 pieces
         const int r = i >> 3, pc = i & 7, lc = pc ^ (r & 7);
         const uint4 u = *reinterpret_cast<const uint4 *>(slot + kSlotTR + (r >> 3) * 1024 + (r & 7) * 128 + pc * 16);
         unpack_h8(u, r < 64 ? Tf + r * L6 + 8 * lc : Rf + (r - 64) * L6 + 8 * lc);
     }
-    for (int i = tid; i < 64 * 16; i += NT) {   // -W: rows 0..63 of [-W; P], 2 x 8 pieces per row
+    for (int i = tid; i < 64 * 16; i += FNT) {   // -W: rows 0..63 of [-W; P], 2 x 8 pieces per row
         const int r = i >> 4, kb = (i >> 3) & 1, pc = i & 7, lc = pc ^ (r & 7);
         const uint4 u = *reinterpret_cast<const uint4 *>(slot + kSlotWP + kb * 16384 + (r >> 3) * 1024 +
                                                          (r & 7) * 128 + pc * 16);
@@ -643,26 +651,31 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
     }
     auto Tm = [&](int r, int s2) { return Tf[r * L6 + s2]; };   // T[r][s]
     auto Rm = [&](int r, int s2) { return Rf[r * L6 + s2]; };   // R[r][s]
-    // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out); T and
-    // R are lower triangular, so row s sums t >= s only
-    smm_rows2_pb<128>([&](int s, int t) { return Tm(t, s); }, dU, LD, [&](int s, int t) { return Rm(t, s); }, dO,
-                      LD, [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = lo2 = 8 * w; hi1 = hi2 = 64; },
-                      [&](int s, int c, float x) { U[s * LD + c] = x; });
-    __syncthreads();
-    for (int i = tid; i < 64 * 32; i += NT) {
-        const int s = i >> 5, c = (i & 31) * 4;
-        if (s < L)
-            *reinterpret_cast<float4 *>(dv + ((size_t)(t0 + s) * H + h) * D + c) =
-                *reinterpret_cast<const float4 *>(U + s * LD + c);
+    if (grp == 0) {
+        // dV = T^T dU + R^T dO (into U's buffer, then the rows of the chunk out); T
+        // and R are lower triangular, so row s sums t >= s only
+        smm_rows2_pb<128>([&](int s, int t) { return Tm(t, s); }, dU, LD, [&](int s, int t) { return Rm(t, s); },
+                          dO, LD,
+                          [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = lo2 = 8 * w; hi1 = hi2 = 64; },
+                          [&](int s, int c, float x) { U[s * LD + c] = x; }, lt);
+        group_bar(1);
+        for (int i = lt; i < 64 * 32; i += NT) {
+            const int s = i >> 5, c = (i & 31) * 4;
+            if (s < L)
+                *reinterpret_cast<float4 *>(dv + ((size_t)(t0 + s) * H + h) * D + c) =
+                    *reinterpret_cast<const float4 *>(U + s * LD + c);
+        }
+        group_bar(1);   // U's buffer (dV) is read out
+        // U = T V (row t sums s <= t)
+        smm_rows2_pb<128>([&](int t, int s) { return Tm(t, s); }, V, LD, [&](int t, int s) { return Tm(t, s); }, V,
+                          LD,
+                          [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = 0; hi1 = 8 * w + 8; lo2 = hi2 = 0; },
+                          [&](int t, int c, float x) { U[t * LD + c] = x; }, lt);
+    } else {
+        // dT = dU V^T, dR = dO V^T
+        smm_nt<64, 64, 128>(dU, LD, V, LD, [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; }, lt);
+        smm_nt<64, 64, 128>(dO, LD, V, LD, [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; }, lt);
     }
-    // dT = dU V^T, dR = dO V^T
-    smm_nt<64, 64, 128>(dU, LD, V, LD, [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; });
-    smm_nt<64, 64, 128>(dO, LD, V, LD, [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; });
-    __syncthreads();   // U's buffer (dV) is read out
-    // U = T V (row t sums s <= t)
-    smm_rows2_pb<128>([&](int t, int s) { return Tm(t, s); }, V, LD, [&](int t, int s) { return Tm(t, s); }, V, LD,
-                      [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = 0; hi1 = 8 * w + 8; lo2 = hi2 = 0; },
-                      [&](int t, int c, float x) { U[t * LD + c] = x; });
     __syncthreads();   // V and [T; R] are consumed
 
     // ---- phase 2: S (zero without an initial state)
@@ -671,19 +684,22 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
         if (tid == 0) mbar_arrive_expect_tx(&bars[1], 128u * 512u);
         copy_rows(S, Sg, D, 128, 0, &bars[1]);
     } else {
-        for (int i = tid; i < 128 * 32; i += NT)
+        for (int i = tid; i < 128 * 32; i += FNT)
             *reinterpret_cast<float4 *>(S + (i >> 5) * LD + (i & 31) * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (!__syncthreads_and(Sg ? mbar_wait(&bars[1], 0, err) : true)) {
         drain(2);
         return;
     }
-    // U += (-W) S   (the slot holds -W)
-    smm_pb<64, 128, 128>([&](int t, int c) { return Wnf[t * LD + c]; }, S, LD,
-                         [&](int t, int jj, float x) { U[t * LD + jj] += x; });
-    // dW = -dU S^T, dP = dO S^T
-    smm_nt<64, 128, 128>(dU, LD, S, LD, [&](int t, int c, float x) { out[FG_DW + t * 128 + c] = -x; });
-    smm_nt<64, 128, 128>(dO, LD, S, LD, [&](int t, int c, float x) { out[FG_DP + t * 128 + c] = x; });
+    // group 0: U += (-W) S (the slot holds -W); group 1: dW = -dU S^T; each group
+    // then half of dP = dO S^T (key channels 64 g .. 64 g + 63)
+    if (grp == 0)
+        smm_pb<64, 128, 128>([&](int t, int c) { return Wnf[t * LD + c]; }, S, LD,
+                             [&](int t, int jj, float x) { U[t * LD + jj] += x; }, lt);
+    else
+        smm_nt<64, 128, 128>(dU, LD, S, LD, [&](int t, int c, float x) { out[FG_DW + t * 128 + c] = -x; }, lt);
+    smm_nt<64, 64, 128>(dO, LD, S + 64 * grp * LD, LD,
+                        [&](int t, int c, float x) { out[FG_DP + t * 128 + 64 * grp + c] = x; }, lt);
     __syncthreads();   // dU and dO are consumed
 
     // ---- phase 3: dS'
@@ -699,8 +715,9 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
         for (int jj = 0; jj < 128; ++jj) a = fmaf(dSp[tid * LD + jj], S[tid * LD + jj], a);
         out[FG_DGL + tid] = a;
     }
-    // dKhat = U dS'^T
-    smm_nt<64, 128, 128>(U, LD, dSp, LD, [&](int t, int c, float x) { out[FG_DKH + t * 128 + c] = x; });
+    // dKhat = U dS'^T (key channels 64 g .. 64 g + 63 per group)
+    smm_nt<64, 64, 128>(U, LD, dSp + 64 * grp * LD, LD,
+                        [&](int t, int c, float x) { out[FG_DKH + t * 128 + 64 * grp + c] = x; }, lt);
 }
 
 
@@ -1344,7 +1361,7 @@ cudaError_t launch_backward_chunked(const BackwardArgs &a, cudaStream_t st) {
     // 3.-6. per chunk: factor gradients (and dv), recompute, pull-back, assembly
     const unsigned items = (unsigned)(L.max_chunks * a.H);
     if ((e = set_smem(bwd_factor_kernel<bf>, F_SMEM)) != cudaSuccess) return e;
-    bwd_factor_kernel<bf><<<items, NT, F_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.v,
+    bwd_factor_kernel<bf><<<items, FNT, F_SMEM, st>>>(fws, a.cu_seqlens, a.T, a.N, a.H, (const bf *)a.v,
                                                      a.state_in, snaps, a.dout, dS, dU, fg, a.dv, hb, a.err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     Profiler::mark(st);

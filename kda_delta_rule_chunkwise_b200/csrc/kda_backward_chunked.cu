@@ -1224,9 +1224,8 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
                                      : (csel ? (e ? acc[0][3] : acc[0][2]) : (e ? acc[0][1] : acc[0][0]));
                 const int cc = 4 * cq + 2 * csel + e;
                 const float da = x * __expf(G[rr * LS + cc] - Rref[A * CW + cc]);
-                const float av = form == 0 ? qv(rr, cc) : kv(rr, cc);
                 if (form == 0) Dq[rr * LS + cc] += da; else Dk[rr * LS + cc] += da;
-                dG[rr * LS + cc] += av * da;
+                dG[rr * LS + cc] += x * AE[(rr - 16 * A) * LS + cc];   // a_r da_r = x a_r E1_r
             }
         }
         __syncthreads();   // block a's rows of Dk and dG take db next

@@ -207,7 +207,9 @@ __device__ __forceinline__ void smm_rows(FA A, FB B, FR range, FO out) {
 // out(i, j, sum_k A[i][k] B[j][k]) (A times B transposed), four k at a time as
 // 16-byte loads (lda, ldb multiples of 4, K a multiple of 4).  Same thread
 // mapping and summation order as smm.
-template <int M, int N, int K, typename FO>
+// LOWER: only the 16 x 16 blocks on and below the diagonal are summed; the
+// blocks above it come out as 0.
+template <int M, int N, int K, bool LOWER = false, typename FO>
 __device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, int ldb, FO out,
                                        const int lt = (int)threadIdx.x) {
     constexpr int TM = M / 16, TN = N / 16;
@@ -229,6 +231,7 @@ __device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, 
         for (int a = 0; a < TM; ++a)
 #pragma unroll
             for (int b = 0; b < TN; ++b) {
+                if (LOWER && b > a) continue;
                 float x = r[a][b];
                 x = fmaf(av[a].x, bv[b].x, x);
                 x = fmaf(av[a].y, bv[b].y, x);
@@ -239,7 +242,7 @@ __device__ __forceinline__ void smm_nt(const float *A, int lda, const float *B, 
 #pragma unroll
     for (int a = 0; a < TM; ++a)
 #pragma unroll
-        for (int b = 0; b < TN; ++b) out(ty + 16 * a, tx + 16 * b, r[a][b]);
+        for (int b = 0; b < TN; ++b) out(ty + 16 * a, tx + 16 * b, (LOWER && b > a) ? 0.f : r[a][b]);
 }
 
 // The product with a row-major fp32 right operand B (ldb a multiple of 4):
@@ -673,8 +676,10 @@ bwd_factor_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__ c
                           [&](int t, int c, float x) { U[t * LD + c] = x; }, lt);
     } else {
         // dT = dU V^T, dR = dO V^T
-        smm_nt<64, 64, 128>(dU, LD, V, LD, [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; }, lt);
-        smm_nt<64, 64, 128>(dO, LD, V, LD, [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; }, lt);
+        // (only the blocks on and below the diagonal matter: T and R are lower
+        // triangular, and the pull-back reads no entry of dT or dR above it)
+        smm_nt<64, 64, 128, true>(dU, LD, V, LD, [&](int t, int s, float x) { out[FG_DT + t * 64 + s] = x; }, lt);
+        smm_nt<64, 64, 128, true>(dO, LD, V, LD, [&](int t, int s, float x) { out[FG_DR + t * 64 + s] = x; }, lt);
     }
     __syncthreads();   // V and [T; R] are consumed
 
@@ -1012,8 +1017,9 @@ bwd_pullback_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
             *p4 = make_float4(kq[it].x * e.x, kq[it].y * e.y, kq[it].z * e.z, kq[it].w * e.w);
         }
         __syncthreads();
-        smm_nt<64, 64, 32>(dPq, PB_LQ, Ktq, PB_LQ, [&](int t, int s, float x) { dRp[t * L6 + s] -= x; });
-        smm_nt<64, 64, 32>(dWq, PB_LQ, Ktq, PB_LQ, [&](int t, int s, float x) { dTp[t * L6 + s] += x; });
+        // (the blocks above the diagonal of dR' and dT' reach no output: they stay 0)
+        smm_nt<64, 64, 32, true>(dPq, PB_LQ, Ktq, PB_LQ, [&](int t, int s, float x) { dRp[t * L6 + s] -= x; });
+        smm_nt<64, 64, 32, true>(dWq, PB_LQ, Ktq, PB_LQ, [&](int t, int s, float x) { dTp[t * L6 + s] += x; });
         smm_rows2<32>([&](int s, int t) { return X[t * L6 + s] * bs[s]; }, [&](int t, int c) { return dWq[t * PB_LQ + c]; },
                       [&](int s, int t) { return -Rm[t * L6 + s]; }, [&](int t, int c) { return dPq[t * PB_LQ + c]; },
                       [](int w, int &lo1, int &hi1, int &lo2, int &hi2) { lo1 = lo2 = 8 * w; hi1 = hi2 = 64; },

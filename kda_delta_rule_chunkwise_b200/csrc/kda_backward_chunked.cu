@@ -14,11 +14,12 @@
 //   per chunk, independently (bwd_factor_kernel):
 //       U = T V - W S,  dV = T^T dU + R^T dO,  dT = dU V^T,  dR = dO V^T,
 //       dW = -dU S^T,  dP = dO S^T,  dKhat = U dS'^T,  dGamma_L = rowsum(dS' * S)
-//   per chunk, independently and without the state (bwd_input_kernel):
-//       the factor gradients pulled back to q, k, g, beta through the chunk's
-//       construction (decay-rescaled Akk / Aqk, the UT solve, R, W, P, Khat).
+//   per chunk, independently and without the state (bwd_recompute_kernel,
+//   bwd_pullback_kernel, bwd_assemble_kernel): the factor gradients pulled back
+//   to q, k, g, beta through the chunk's construction (decay-rescaled Akk / Aqk,
+//   the UT solve, R, W, P, Khat).
 //
-// All three run fp32 SIMT products on shared-memory tiles; the factors come
+// All of them run fp32 SIMT products on shared-memory tiles; the factors come
 // from the forward's fp16 slots.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

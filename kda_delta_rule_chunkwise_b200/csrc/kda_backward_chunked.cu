@@ -1236,14 +1236,47 @@ bwd_assemble_kernel(const uint8_t *__restrict__ fws, const int32_t *__restrict__
             }
         }
         __syncthreads();   // block a's rows of Dk and dG take db next
-        // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s < NS
-        smm<NS, CW, 16>([&](int s2, int r) { return dF[(16 * A + r) * L6 + s2]; },
-                        [&](int r, int cc) { return AE[r * LS + cc]; },
-                        [&](int s2, int cc, float x) {
-                            const float db = x * __expf(Rref[A * CW + cc] - G[s2 * LS + cc]);
-                            Dk[s2 * LS + cc] += db;
-                            dG[s2 * LS + cc] -= kv(s2, cc) * db;
-                        });
+        // db_s += exp(R_a - G_s) sum_{r in a} dF[r,s] a_r E1_r, for s < NS: thread
+        // (rg = tid / 8, cq = tid % 8) takes rows rg and rg + 32 (those below NS) and
+        // columns 4 cq .. 4 cq + 3, read as 16-byte pieces
+        {
+            constexpr int NR = NS > 32 ? 2 : 1;
+            const int rg = tid >> 3, cq = tid & 7;
+            if (rg < NS) {
+                const bool two = NR == 2 && rg + 32 < NS;
+                float acc[NR][4];
+#pragma unroll
+                for (int x = 0; x < NR; ++x)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[x][e] = 0.f;
+#pragma unroll 4
+                for (int r = 0; r < 16; ++r) {
+                    const float4 b4 = *reinterpret_cast<const float4 *>(AE + r * LS + 4 * cq);
+#pragma unroll
+                    for (int x = 0; x < NR; ++x) {
+                        const float av = (x == 0 || two) ? dF[(16 * A + r) * L6 + rg + 32 * x] : 0.f;
+                        acc[x][0] = fmaf(av, b4.x, acc[x][0]); acc[x][1] = fmaf(av, b4.y, acc[x][1]);
+                        acc[x][2] = fmaf(av, b4.z, acc[x][2]); acc[x][3] = fmaf(av, b4.w, acc[x][3]);
+                    }
+                }
+#pragma unroll
+                for (int x = 0; x < NR; ++x) {
+                    if (x == 1 && !two) break;
+                    const int s2 = rg + 32 * x, o = s2 * LS + 4 * cq;
+                    const float4 g4 = *reinterpret_cast<const float4 *>(G + o);
+                    const float4 rf = *reinterpret_cast<const float4 *>(Rref + A * CW + 4 * cq);
+                    const float4 k4 = *reinterpret_cast<const float4 *>(Ks + o);
+                    float4 dk4 = *reinterpret_cast<const float4 *>(Dk + o);
+                    float4 dg4 = *reinterpret_cast<const float4 *>(dG + o);
+                    const float d0 = acc[x][0] * __expf(rf.x - g4.x), d1 = acc[x][1] * __expf(rf.y - g4.y);
+                    const float d2 = acc[x][2] * __expf(rf.z - g4.z), d3 = acc[x][3] * __expf(rf.w - g4.w);
+                    dk4.x += d0; dk4.y += d1; dk4.z += d2; dk4.w += d3;
+                    dg4.x -= k4.x * d0; dg4.y -= k4.y * d1; dg4.z -= k4.z * d2; dg4.w -= k4.w * d3;
+                    *reinterpret_cast<float4 *>(Dk + o) = dk4;
+                    *reinterpret_cast<float4 *>(dG + o) = dg4;
+                }
+            }
+        }
     };
     for (int form = 0; form < 2; ++form) {
         __syncthreads();   // the previous form's products are done with dFs

@@ -61,7 +61,7 @@ FLOPS_PER_TOKEN_HEAD = 139264                                 # algorithmic MMA 
 # (sm__pipe_tensor_cycles_active over the kernel), or None.
 PREFILL_SOURCES = ("kda_prefill_bf16.cu", "kda_common.cuh", "sm100.cuh", "kda_tma.h", "kda_launch.h")
 NCU = {
-    "prefill_fused_kernel": (PREFILL_SOURCES, "5d610f5cdf0a3c9e", (348278528 + 362011648) / 4096, 8.9),
+    "prefill_fused_kernel": (PREFILL_SOURCES, "8cdfe7b6f92d16e6", (299425536 + 355247616) / 4096, 8.9),
     "intra_chunk_kernel": (PREFILL_SOURCES, "96b42b1b1ffcc8c0", (202737408 + 217004544) / 4096, 8.2),
     "state_pass_kernel": (PREFILL_SOURCES, "96b42b1b1ffcc8c0", (339793920 + 109534720) / 4096, 9.0),
     "decode_kernel": (("kda_decode.cu",), "4f1c8c21d6ac8934", 545290752 + 482616576, None),

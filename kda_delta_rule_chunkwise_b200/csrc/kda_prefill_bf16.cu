@@ -58,6 +58,14 @@
 namespace kda {
 namespace tc {
 
+// Pause of a phase A CTA between items when its SM also runs a state-pass chain
+// in the one-launch form. The chain bounds that launch, and a phase A CTA next
+// to it slows it by sharing issue slots, shared memory and TMEM. Measured at
+// T=65536, H=32: 3.04 ms without a pause, 2.93 ms for 5-8 us (one item takes
+// about 18 us), 3.00 ms at 10 us. With the gate and norms computed inside, the
+// pause made the step slower (3.24 -> 3.42 ms), so that form does not pause.
+constexpr unsigned kChainYieldNs = 6000;
+
 using namespace sm100;
 
 constexpr int C = 64;      // chunk length
@@ -480,6 +488,18 @@ __device__ __forceinline__ void intra_chunk_body(
     }
     if (__syncthreads_or(*abort_flag != 0u)) break;
     if (ready && tid == 0 && prev_item >= 0) publish(prev_item);
+    // one launch: a phase A CTA on an SM that also runs a state-pass chain pauses
+    // between items (its other threads wait at the barrier below), leaving the
+    // SM's issue slots, shared memory and TMEM to the chain, which bounds the
+    // launch (the SMs that run chains are marked in the scheduler area).  Not
+    // with preprocessing inside: its longer items make phase A the bound.
+    if (!PREP && sched && tid == 0) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        if ((smid >> 5) < 8u &&
+            ((*reinterpret_cast<volatile const uint32_t *>(sched + 8 + (smid >> 5)) >> (smid & 31)) & 1u))
+            __nanosleep(kChainYieldNs);
+    }
     prev_item = item;
     const int c = tid & 127, half = tid >> 7;
     float p[32];   // clamped log-decay of rows 32*half + i, then its prefix sums
@@ -1932,12 +1952,18 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    if ((int)blockIdx.x < n_state)
+    if ((int)blockIdx.x < n_state) {
+        if (threadIdx.x == 0) {   // mark this SM as running a chain (words 8 .. 15 of the scheduler area)
+            uint32_t smid;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+            if ((smid >> 5) < 8u) atomicOr(sched + 8 + (smid >> 5), 1u << (smid & 31));
+        }
         state_pass_role<DVS>(&tm_v, state_in, cu, T, N, H, ws, ready, o, state_out, ckpt_interval,
                              ckpt, ckpt_capacity, err, epoch, sm, (int)blockIdx.x);
-    else
+    } else {
         intra_chunk_body<PREP>(&tm_q, &tm_k, &tm_g, beta, cu, T, N, H, flags, ws, err, epoch, sm,
                                (int)blockIdx.x - n_state, (int)gridDim.x - n_state, sched, ready);
+    }
 }
 
 }  // namespace tc

@@ -133,14 +133,20 @@ def wy_state_part(f, v, S, dO, dS_end):
     return dS, dV, grads
 
 
-def wy_input_part(q, k, g, beta, f, gr):
-    """Pull the factor gradients back to q, k, g, beta (no state involved)."""
+def wy_input_part(q, k, g, beta, f, gr, upper=None):
+    """Pull the factor gradients back to q, k, g, beta (no state involved).
+    upper(shape), when given, is added to the strictly upper triangles of dR' and
+    dT' as they are formed: no output may depend on those entries."""
     L = q.shape[0]
     E, gam, gam_l = f["E"], f["gam"], f["gam_l"]
     dP = gr["dP"]
     dR = gr["dR"] - dP @ f["Kt"].T
+    if upper is not None:
+        dR = dR + np.triu(upper(dR.shape), 1)
     dKt = f["T"].T @ gr["dW"] - f["R"].T @ dP
     dT = gr["dT"] + f["Aqk"].T @ dR + gr["dW"] @ f["Kt"].T
+    if upper is not None:
+        dT = dT + np.triu(upper(dT.shape), 1)
     dAqk = np.tril(dR @ f["T"].T)
     dbeta = np.sum(f["X"] * dT, axis=0)
     dAkk = np.tril(-f["X"].T @ (dT * beta[None, :]) @ f["X"].T, -1)
@@ -162,8 +168,8 @@ def wy_input_part(q, k, g, beta, f, gr):
     return dq, dk, dg, dbeta
 
 
-def wy_backward(q, k, v, g, beta, S0, dout, dS_final, C=64):
-    """As backward(), through the WY-slot split."""
+def wy_backward(q, k, v, g, beta, S0, dout, dS_final, C=64, upper=None):
+    """As backward(), through the WY-slot split (upper: see wy_input_part)."""
     T_len = q.shape[0]
     starts = list(range(0, T_len, C))
     states, facs = [np.array(S0, np.float64)], []
@@ -178,7 +184,7 @@ def wy_backward(q, k, v, g, beta, S0, dout, dS_final, C=64):
     for ci in reversed(range(len(starts))):
         sl = slice(starts[ci], min(T_len, starts[ci] + C))
         dS_prev, dv[sl], gr = wy_state_part(facs[ci], v[sl], states[ci], dout[sl], dS)
-        dq[sl], dk[sl], dg[sl], db[sl] = wy_input_part(q[sl], k[sl], g[sl], beta[sl], facs[ci], gr)
+        dq[sl], dk[sl], dg[sl], db[sl] = wy_input_part(q[sl], k[sl], g[sl], beta[sl], facs[ci], gr, upper)
         dS = dS_prev
     return dq, dk, dv, dg, db, dS
 

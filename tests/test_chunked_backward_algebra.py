@@ -34,3 +34,22 @@ def test_chunked_backward_equals_the_oracle(T, d, C, form):
                            b[None, :, None], S0[None, None], dout[None, :, None], dS_final[None, None])
     for name, x, w in zip(["dq", "dk", "dv", "dg", "dbeta", "dS0"], got, want):
         assert rel_err(x, np.reshape(w, x.shape)) < 1e-10, name
+
+
+def test_upper_triangles_of_dR_and_dT_reach_no_output():
+    """T, R, X and Aqk are lower triangular, so only the lower parts (diagonal
+    included) of dR' = dR - dP (K Gamma)^T and dT' reach dAkk, dAqk and dbeta.
+    The chunked backward leaves the 16 x 16 blocks above the diagonal of dT, dR
+    and of those two products at 0; here large noise in every strictly upper
+    entry must leave all gradients unchanged."""
+    inp = kin.prefill_inputs(1, 150, 1, 16, 16, "f32", seed=5, state="normal")
+    f64 = lambda x: x.double().numpy()
+    q, k, v, g, b = (f64(x[0, :, 0]) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta))
+    S0 = f64(inp.state_in[0, 0])
+    rng = np.random.default_rng(11)
+    dout, dS_final = rng.normal(size=(150, 16)), rng.normal(size=(16, 16))
+    want = wy_backward(q, k, v, g, b, S0, dout, dS_final, C=64)
+    noise = np.random.default_rng(12)
+    got = wy_backward(q, k, v, g, b, S0, dout, dS_final, C=64, upper=lambda shp: 1e3 * noise.normal(size=shp))
+    for name, x, w in zip(["dq", "dk", "dv", "dg", "dbeta", "dS0"], got, want):
+        assert rel_err(x, w) < 1e-10, name
